@@ -1,0 +1,474 @@
+"""Benchmark of one Lighthouse Attention layer (forward + backward) on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload pretrain|long|extreme] [--attn tc|mma] [--no-cpu] [--no-dense]
+
+A step is one pass of the whole hot path over one batch of synthetic input:
+pyramid + scores, joint top-S, gather, causal sub-sequence attention,
+scatter-back, then the backward through scatter-back, attention and gather.
+The default workload is the pretraining shape (B=1, H=16, N=98,304, d=64,
+p=4, L=4, S=8192, bf16, 1% high-norm outlier tokens).  Inputs (3 x 201 MB plus
+dO) are larger than the 126 MB L2, so no flush is needed between steps.
+
+Rank 0 prints one JSON line.  With torchrun (N > 1) every rank runs its own
+independent copy of the workload (heads are independent: weak scaling, no
+collective on the data path); the step time is the max over ranks.
+`--impl reference` times the CPU oracle on this host instead (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+from long_context_lh_b200.synth import WORKLOADS, make_inputs  # noqa: E402
+
+METRIC = "Lighthouse layer tokens/s fwd & fwd+bwd at N=98K/512K; % of HBM/TC roofline"
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        d = json.load(open(p))
+        return {k: float(d[k]) for k in ("hbm_gbs", "bf16_tflops", "bf16_tflops_sustained")}, "measured"
+    except Exception:
+        return PEAKS_FALLBACK, "fallback"
+
+
+# ------------------------------------------------------------ algorithmic work
+def algorithmic(w):
+    """Algorithmic bytes / FLOPs per stage for one step (whole job on one GPU).
+
+    Bytes count each tensor the stage must read or write once (inputs in the
+    workload dtype, pyramid fp32, gathered rows bf16, sub-sequence gradients
+    fp32); FLOPs count the causal attention products only."""
+    U, N, d, S, M = w.B * w.H, w.N, w.d, w.S, w.M
+    es = 2 if w.dtype == "bf16" else 4
+    E = N * d
+    R = (M - N) / N
+    return {
+        "pyramid_score": U * (3 * E * es + 12 * E * R + 4 * M),
+        "topk": U * (4 * M + 4 * M + 8 * S),
+        "gather": U * (S * 4 + S * 3 * d * (4 + 2)),
+        "attn_fwd_flop": U * 2.0 * S * S * d,
+        "scatter": U * (4 * M + S * d * 2 + E * es + 4 * N),
+        "scatter_bwd": U * (E * es + 4 * N + 4 * M + S * d * 2),
+        "attn_bwd_flop": U * 5.0 * S * S * d,
+        "gather_bwd": U * (4 * M + 3 * S * d * 4 + 3 * E * es),
+    }
+
+
+# --------------------------------------------------------------------- clocks
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "50"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except Exception:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *a):
+        if self.proc:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ------------------------------------------------------------------ our arm
+def run_ours(args, rank, world, local_rank):
+    import numpy as np  # noqa: F401
+    from long_context_lh_b200 import lighthouse as lh
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    w = WORKLOADS[args.workload]
+    if args.attn == "mma":
+        lh.lh_set_attention_impl(1)
+    elif args.attn == "tc":
+        lh.lh_set_attention_impl(0)
+    peaks, peaks_src = load_peaks()
+    shp = lh.make_shape(w.B, w.H, w.N, w.d, w.p, w.L, w.S)
+    dt = lh.dtype_code(w.torch_dtype)
+    x = make_inputs(w, dev)
+    q, k, v, dO = x["q"], x["k"], x["v"], x["dO"]
+    o = torch.empty_like(q)
+    dq, dk, dv = (torch.empty_like(q) for _ in range(3))
+    saved = torch.empty(lh.lh_saved_bytes(shp), dtype=torch.uint8, device=dev)
+    wsb = lh.lh_workspace_bytes(shp, dt, True)
+    ws = torch.empty(wsb, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.Stream(device=dev)
+    sp = stream.cuda_stream
+
+    def step():
+        lh.lh_forward(shp, dt, q, k, v, 0.0, o, saved, ws, wsb, sp)
+        lh.lh_backward(shp, dt, saved, dO, 0.0, dq, dk, dv, ws, wsb, sp)
+
+    def fwd_only():
+        lh.lh_forward(shp, dt, q, k, v, 0.0, o, saved, ws, wsb, sp)
+
+    # stage-by-stage replica of the same launches, for per-kernel durations
+    M = w.M
+    U = w.B * w.H
+    base = saved
+
+    def view(which, dtype, n):
+        off = lh.lh_saved_offset(shp, which)
+        return base[off:off + n * torch.tensor([], dtype=dtype).element_size()].view(dtype)
+
+    idx = view(lh.SAVED_IDX, torch.int32, U * w.S)
+    pos = view(lh.SAVED_POS, torch.int32, U * w.S)
+    slot = view(lh.SAVED_SLOT, torch.int32, U * M)
+    qs, ks, vs, os_ = (view(i, torch.float16, U * w.S * w.d)
+                       for i in (lh.SAVED_QS, lh.SAVED_KS, lh.SAVED_VS, lh.SAVED_OS))
+    lse = view(lh.SAVED_LSE, torch.float32, U * w.S)
+    ic = view(lh.SAVED_INV_COUNT, torch.float32, U * w.N)
+    npyr = max(U * (M - w.N) * w.d, 1)
+    pq, pk, pv = (torch.empty(npyr, dtype=torch.float32, device=dev) for _ in range(3))
+    score = torch.empty(U * M, dtype=torch.float32, device=dev)
+    dos = torch.empty(U * w.S * w.d, dtype=torch.float16, device=dev)
+    dqs, dks, dvs = (torch.empty(U * w.S * w.d, dtype=torch.float32, device=dev) for _ in range(3))
+    abw = lh.lh_attn_bwd_workspace_bytes(shp)
+    aws = torch.empty(abw, dtype=torch.uint8, device=dev)
+    stages = ["pyramid_score", "topk", "gather", "attn_fwd", "scatter", "scatter_bwd",
+              "attn_bwd", "gather_bwd"]
+    def staged(evs):
+        # identical launches to lh_forward + lh_backward, with events between stages
+        evs[0].record(stream)
+        lh.lh_build_pyramid_score(shp, dt, q, k, v, pq, pk, pv, score, sp)
+        evs[1].record(stream)
+        lh.lh_topk_select(shp, score, idx, pos, slot, None, 0, sp)
+        evs[2].record(stream)
+        lh.lh_gather(shp, dt, q, k, v, pq, pk, pv, idx, qs, ks, vs, sp)
+        evs[3].record(stream)
+        lh.lh_subseq_attn_fwd(shp, qs, ks, vs, 0.0, os_, lse, sp)
+        evs[4].record(stream)
+        lh.lh_scatter_back(shp, dt, os_, slot, o, ic, sp)
+        evs[5].record(stream)
+        lh.lh_scatter_back_bwd(shp, dt, dO, slot, ic, dos, sp)
+        evs[6].record(stream)
+        lh.lh_subseq_attn_bwd(shp, qs, ks, vs, os_, lse, dos, 0.0, dqs, dks, dvs, aws, abw, sp)
+        evs[7].record(stream)
+        lh.lh_gather_bwd(shp, dt, dqs, dks, dvs, slot, dq, dk, dv, sp)
+        evs[8].record(stream)
+
+    dist = world > 1
+
+    def barrier():
+        if dist:
+            torch.distributed.barrier()
+
+    def timed(fn, K):
+        barrier()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(K):
+            fn()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        ms = e0.elapsed_time(e1)
+        barrier()
+        if dist:
+            t = torch.tensor([ms], device=dev)
+            torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+            ms = float(t.item())
+        return ms
+
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            step()
+        torch.cuda.synchronize()
+        status = lh.lh_read_device_status(stream)
+        with ClockSampler(local_rank) as clk:
+            ms_total = timed(step, args.steps)
+        ms_step = ms_total / args.steps
+        ms_fwd = timed(fwd_only, args.steps) / args.steps
+        # per-stage durations over the same number of steps
+        evs_all = []
+        torch.cuda.synchronize()
+        for _ in range(args.steps):
+            evs = [torch.cuda.Event(enable_timing=True) for _ in range(9)]
+            staged(evs)
+            evs_all.append(evs)
+        torch.cuda.synchronize()
+        stage_ms = {s: statistics.mean(e[i].elapsed_time(e[i + 1]) for e in evs_all)
+                    for i, s in enumerate(stages)}
+        status |= lh.lh_read_device_status(stream)
+
+    tokens = w.B * w.N
+    value = world * tokens / (ms_step / 1e3)
+    alg = algorithmic(w)
+    hbm = peaks["hbm_gbs"]
+    tc = peaks["bf16_tflops"]
+    stage_report = {}
+    for s in stages:
+        t = stage_ms[s] / 1e3
+        if s.startswith("attn"):
+            fl = alg[s + "_flop"]
+            stage_report[s] = {"ms": stage_ms[s], "tflops": fl / t / 1e12, "frac_tc": fl / t / 1e12 / tc}
+        else:
+            b = alg[s]
+            stage_report[s] = {"ms": stage_ms[s], "gbs": b / t / 1e9, "frac_hbm": b / t / 1e9 / hbm}
+    dominant = max(stages, key=lambda s: stage_ms[s])
+    if dominant.startswith("attn"):
+        ach = stage_report[dominant]["tflops"]
+        roof = {"kernel": dominant, "bound": "tensor", "achieved": ach, "peak": tc,
+                "unit": "TFLOP/s", "frac": ach / tc, "traffic": None,
+                "peak_source": f"{peaks_src} bf16_tflops (burst)"}
+    else:
+        ach = stage_report[dominant]["gbs"]
+        roof = {"kernel": dominant, "bound": "hbm", "achieved": ach, "peak": hbm, "unit": "GB/s",
+                "frac": ach / hbm, "traffic": None, "peak_source": f"{peaks_src} hbm_gbs"}
+
+    # dense causal attention (torch SDPA, flash/cuDNN backend) on the same shapes
+    dense = None
+    if not args.no_dense and rank == 0:
+        dense = dense_sdpa(w, q, k, v, dO, stream, args)
+
+    # end to end through the public API with pinned host buffers
+    e2e = e2e_run(lh, w, shp, dt, x, dev, stream, args, dist)
+    launches = launches_per_step(lh, w)
+    out = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded N(0,1) Q/K/V/dO, 1% tokens x4; no corpus or weights)",
+        "config": {"workload": f"{w.name}: B={w.B} H={w.H} N={w.N} d={w.d} p={w.p} L={w.L} S={w.S} {w.dtype}",
+                   "B": w.B, "H": w.H, "N": w.N, "d": w.d, "p": w.p, "L": w.L, "S": w.S,
+                   "l2": "inputs larger than L2 (3 x %.0f MB + dO), no flush" % (w.B * w.H * w.N * w.d * 2 / 1e6),
+                   "attention": "tcgen05" if lh.lh_attention_impl_in_use() == 0 else "mma_sync",
+                   "parallelism": f"replicas x{world} (heads independent)"},
+        "fwd_tokens_per_s": world * tokens / (ms_fwd / 1e3), "ms_fwd": ms_fwd,
+        "roofline": roof, "stages": stage_report, "dense_sdpa": dense, "e2e": e2e,
+        "gpu_launches": launches * args.steps, "gpu_launches_per_step": launches,
+        "device_status": status, "peaks": peaks, "peaks_source": peaks_src,
+    }
+    if rank == 0:
+        out["clocks"] = clk.summary()
+        if not args.no_cpu:
+            out["cpu_baseline"] = cpu_baseline(w, budget_s=args.cpu_budget)
+        print(json.dumps(out), flush=True)
+
+
+def launches_per_step(lh, w):
+    """Kernels of this library launched per step (lh_forward + lh_backward)."""
+    shp = lh.make_shape(w.B, w.H, w.N, w.d, w.p, w.L, w.S)
+    return lh.lh_kernel_launches(shp, False) + lh.lh_kernel_launches(shp, True)
+
+
+def dense_sdpa(w, q, k, v, dO, stream, args):
+    import torch.nn.functional as F
+    try:
+        qd = q.detach().requires_grad_(True)
+        kd = k.detach().requires_grad_(True)
+        vd = v.detach().requires_grad_(True)
+        with torch.cuda.stream(stream):
+            def f():
+                return F.scaled_dot_product_attention(qd, kd, vd, is_causal=True)
+
+            def fb():
+                out = F.scaled_dot_product_attention(qd, kd, vd, is_causal=True)
+                out.backward(dO)
+
+            for _ in range(2):
+                with torch.no_grad():
+                    f()
+                fb()
+            torch.cuda.synchronize()
+            n = max(1, min(args.steps, 5))
+            e0, e1, e2 = (torch.cuda.Event(enable_timing=True) for _ in range(3))
+            e0.record(stream)
+            for _ in range(n):
+                with torch.no_grad():
+                    f()
+            e1.record(stream)
+            for _ in range(n):
+                fb()
+            e2.record(stream)
+            torch.cuda.synchronize()
+        return {"fwd_ms": e0.elapsed_time(e1) / n, "fwd_bwd_ms": e1.elapsed_time(e2) / n,
+                "backend": "torch.nn.functional.scaled_dot_product_attention(is_causal=True)"}
+    except Exception as ex:  # pragma: no cover
+        return {"error": str(ex)[:200]}
+
+
+def e2e_run(lh, w, shp, dt, x, dev, stream, args, dist):
+    """Same step through lh_forward/lh_backward with host<->device copies inside."""
+    host = {n: t.cpu().pin_memory() for n, t in x.items()}
+    dev_in = {n: torch.empty_like(t) for n, t in x.items()}
+    o = torch.empty_like(x["q"])
+    grads = [torch.empty_like(x["q"]) for _ in range(3)]
+    out_host = [torch.empty(o.shape, dtype=o.dtype).pin_memory() for _ in range(4)]
+    saved = torch.empty(lh.lh_saved_bytes(shp), dtype=torch.uint8, device=dev)
+    wsb = lh.lh_workspace_bytes(shp, dt, True)
+    ws = torch.empty(wsb, dtype=torch.uint8, device=dev)
+    sp = stream.cuda_stream
+    h2d = sum(t.numel() * t.element_size() for t in host.values())
+    d2h = sum(t.numel() * t.element_size() for t in out_host)
+
+    def step():
+        for n in host:
+            dev_in[n].copy_(host[n], non_blocking=True)
+        lh.lh_forward(shp, dt, dev_in["q"], dev_in["k"], dev_in["v"], 0.0, o, saved, ws, wsb, sp)
+        lh.lh_backward(shp, dt, saved, dev_in["dO"], 0.0, *grads, ws, wsb, sp)
+        for src, dst in zip([o, *grads], out_host):
+            dst.copy_(src, non_blocking=True)
+
+    K = max(1, min(args.steps, 10))
+    with torch.cuda.stream(stream):
+        step()
+        torch.cuda.synchronize()
+        if dist:
+            torch.distributed.barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(K):
+            step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / K
+    if dist:
+        t = torch.tensor([ms], device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms = float(t.item())
+    world = torch.distributed.get_world_size() if dist else 1
+    return {"value": world * w.B * w.N / (ms / 1e3), "unit": "tokens/s", "ms_per_step": ms,
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+
+
+# ------------------------------------------------------------- CPU oracle
+def oracle_step(w, h, x_np):
+    """Oracle forward + backward of head h (all of its tokens)."""
+    import oracle
+    s1 = oracle.Shape(1, 1, w.N, w.d, w.p, w.L, w.S)
+    q, k, v, dO = (x_np[n][:, h:h + 1] for n in ("q", "k", "v", "dO"))
+    f = oracle.forward(s1, q, k, v)
+    oracle.backward(s1, f, dO)
+
+
+def cpu_baseline(w, budget_s=20.0, steps=None, warmup=0):
+    """Time the oracle on this host's cores: whole heads, until the budget is spent."""
+    import numpy as np  # noqa: F401
+    xc = make_inputs(w, "cpu")
+    x_np = {n: t.float().numpy() for n, t in xc.items()}
+    cores = os.cpu_count() or 1
+    for h in range(warmup):
+        oracle_step(w, h % w.H, x_np)
+    t0 = time.perf_counter()
+    heads = 0
+    times = []
+    while heads < w.H:
+        t1 = time.perf_counter()
+        oracle_step(w, heads % w.H, x_np)
+        times.append(time.perf_counter() - t1)
+        heads += 1
+        if steps is not None and heads >= steps:
+            break
+        if steps is None and time.perf_counter() - t0 >= budget_s:
+            break
+    el = time.perf_counter() - t0
+    value = w.B * w.N * (heads / w.H) / el
+    return {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+            "sample": f"{heads} of {w.H} heads of the {w.name} workload, forward+backward, "
+                      f"{el:.1f} s; tokens/s = B*N*(heads/H)/time",
+            "per_head_s": times}
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return
+    w = WORKLOADS[args.workload]
+    cb = cpu_baseline(w, steps=args.steps, warmup=args.warmup)
+    out = {"impl": "reference", "metric": METRIC, "value": cb["value"], "unit": "tokens/s",
+           "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+           "ms_per_step": 1e3 * sum(cb["per_head_s"]) / max(len(cb["per_head_s"]), 1),
+           "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+           "data": "synthetic", "config": {"workload": f"{w.name} (one head per step)"},
+           "cpu_baseline": {k: cb[k] for k in ("value", "unit", "cores", "kind", "sample")},
+           "e2e": {"value": cb["value"], "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                   "d2h_bytes_per_step": 0}}
+    print(json.dumps(out), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="pretrain", choices=["pretrain", "long", "extreme"])
+    ap.add_argument("--attn", default="auto", choices=["auto", "tc", "mma"])
+    ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--no-dense", action="store_true")
+    ap.add_argument("--cpu-budget", type=float, default=20.0)
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3) if args.impl == "ours" else args.warmup
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local_rank)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                             device_id=torch.device("cuda", local_rank))
+    try:
+        run_ours(args, rank, world, local_rank)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,221 @@
+/*
+ * lighthouse.h -- C ABI of a B200 (sm_100a) library for the data-parallel hot
+ * path of one Lighthouse Attention layer, forward and backward.
+ *
+ * The method, as two pages describe it:
+ *   [ES] gist.science/es, "Resumen Técnico: Pre-entrenamiento con Contexto Largo
+ *        mediante Atención Lighthouse", §2 Metodología (mirrored on gist.science/ja §2);
+ *   [PT] bitsgeniais.com.br, "Adeus Custo Quadrático! Como a Lighthouse Attention
+ *        Vai TURBINAR o Treinamento de LLMs!", section "A Grande Sacada: Lighthouse
+ *        Attention em Quatro Fases!" (phases 1-4):
+ *   (a) an L-level average-pooling pyramid over Q, K and V with pool factor p;
+ *   (b) a parameter-free score per entry from the l2 norms of Q and K, coarse
+ *       levels inheriting the max of their children;
+ *   (c) one top-S selection across all levels;
+ *   (d) a gather of the selected (Q, K, V) triplets into a dense,
+ *       position-sorted sub-sequence of length S;
+ *   (e) causal attention on that sub-sequence;
+ *   (f) a deterministic scatter-back of its outputs to the original positions;
+ *   and the backward through (f), (e) and (d) (no gradient through (c)).
+ *
+ * Notation, per unit u = (b, h): n_l = N / p^l, off_l = sum_{m<l} n_m,
+ * M = off_L entries; entry (l, j) has gid = off_l + j, covers tokens
+ * [j p^l, (j+1) p^l - 1] and is placed at pos = (j+1) p^l - 1.
+ *
+ * Readings of the pages fixed by this library (the pages leave them open):
+ *   score      = ||Q[t]|| + ||K[t]|| at level 0 (fp32, one fixed summation
+ *                order), coarse score = max over the p children;
+ *   ranking    = score descending, ties to the lower level then lower index
+ *                (lower gid), so the selected set is unique;
+ *   order      = (pos ascending, level ascending): children before the parent
+ *                that ends on the same token;
+ *   attention  = causal on the slot index, scale 1/sqrt(d) unless given;
+ *   scatter    = each token t gets the mean of the outputs of the selected
+ *                entries covering it (its "contributors"), summed in ascending
+ *                level; 0 when there is none.
+ *
+ * Conventions for every call:
+ *   - Pointers are DEVICE pointers unless a parameter says otherwise, to
+ *     contiguous row-major arrays with d innermost, 16-byte aligned.
+ *   - Q, K, V, O, dO, dQ, dK, dV are [B, H, N, d] in the call's lh_dtype.
+ *     The gathered sub-sequence (qs, ks, vs, os, dos) is fp16 (IEEE binary16)
+ *     [B, H, S, d]: the tensor-core operands of the attention, 3 more mantissa
+ *     bits than bf16; values beyond +-65504 saturate.  Pyramid levels are fp32;
+ *     gradients of the sub-sequence are fp32.
+ *   - The caller allocates and frees every buffer; the library allocates no
+ *     device memory and never synchronises the stream (except
+ *     lh_read_device_status).  All work is enqueued on `stream` (NULL = the
+ *     legacy default stream).
+ *   - Arguments are checked on the host before any launch; a call that
+ *     returns an error has enqueued nothing.  A launch failure returns
+ *     LH_ERR_CUDA.  No call traps, asserts or exits.
+ *   - Results are bitwise deterministic for identical inputs, shape and device.
+ *   - Non-finite inputs give unspecified values, never a crash or a hang.
+ *   - Shape limits: B, H >= 1; d in {64, 128}; 2 <= p; 1 <= L <= 8;
+ *     N % p^(L-1) == 0; 1 <= S <= M; M < 2^31 and B*H*M < 2^40.
+ */
+#ifndef LIGHTHOUSE_H
+#define LIGHTHOUSE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t. */
+typedef struct CUstream_st* lh_stream_t;
+
+typedef enum {
+  LH_OK = 0,
+  LH_ERR_INVALID_ARG = 1,   /* null or misaligned pointer, bad enum */
+  LH_ERR_SHAPE = 2,         /* shape outside the limits above */
+  LH_ERR_UNSUPPORTED = 3,   /* no kernel for this device or configuration */
+  LH_ERR_WORKSPACE = 4,     /* workspace smaller than the *_bytes query */
+  LH_ERR_CUDA = 5,          /* a CUDA runtime call or launch failed */
+  LH_ERR_DEVICE_STATUS = 6  /* a kernel reported a bounded wait that timed out */
+} lh_status;
+
+typedef enum { LH_F32 = 0, LH_BF16 = 1 } lh_dtype; /* dtype of Q,K,V,O,dO,dQ,dK,dV */
+
+typedef struct {
+  int64_t B, H, N;
+  int32_t d, p, L, S;
+} lh_shape;
+
+/* Human-readable name of a status code (static string). */
+const char* lh_status_string(lh_status s);
+
+/* Host-only check of a shape and dtype against the limits above; no CUDA call. */
+lh_status lh_validate(const lh_shape* shape, lh_dtype dtype);
+
+/* Number of pyramid entries M per unit, or -1 for an invalid shape. */
+int64_t lh_num_entries(const lh_shape* shape);
+
+/* Bytes of caller workspace that lh_forward (with_backward = 0) or both
+ * lh_forward and lh_backward (with_backward = 1) need; 0 for an invalid shape. */
+size_t lh_workspace_bytes(const lh_shape* shape, lh_dtype dtype, int with_backward);
+
+/* Bytes of the forward-to-backward state that lh_forward writes and
+ * lh_backward reads: selection (idx, pos, slot), gathered qs/ks/vs, os, lse. */
+size_t lh_saved_bytes(const lh_shape* shape);
+
+/* Byte offsets inside the saved buffer, for callers that want to look at it:
+ * which = 0 idx, 1 pos, 2 slot, 3 qs, 4 ks, 5 vs, 6 os, 7 lse, 8 inverse
+ * contributor count (fp32 [B,H,N], 1/c_t or 0).  -1 for a bad argument. */
+int64_t lh_saved_offset(const lh_shape* shape, int which);
+
+/* ---------------------------------------------------------------- stages */
+
+/* (a) Pyramid, [ES] §2.A / [PT] phase 1: for l = 1..L-1,
+ *   X^(l)[j] = (sum_{i<p} X^(l-1)[p j + i]) / p  (fp32, children in order),
+ * for X in {Q, K, V}.  q, k, v: [B,H,N,d] dtype.  pq, pk, pv: fp32
+ * [B,H,M-N,d], levels 1..L-1 concatenated (level 0 is the input itself).    */
+lh_status lh_build_pyramid(const lh_shape* shape, lh_dtype dtype, const void* q, const void* k,
+                           const void* v, float* pq, float* pk, float* pv, lh_stream_t stream);
+
+/* (a)+(b) in one pass over Q, K and V: the pyramid levels and all M scores,
+ * exactly as the two calls above compute them (this is what lh_forward runs).
+ * pq, pk, pv may be NULL when L == 1.                                        */
+lh_status lh_build_pyramid_score(const lh_shape* shape, lh_dtype dtype, const void* q,
+                                 const void* k, const void* v, float* pq, float* pk, float* pv,
+                                 float* score, lh_stream_t stream);
+
+/* (b) Score, [ES] §2.B / [PT] phase 2: score[t] = ||Q[t]||_2 + ||K[t]||_2 for
+ * level 0 (fp32: eight-element fmaf chains, then a pairwise tree, IEEE sqrt),
+ * and score^(l)[j] = max_{i<p} score^(l-1)[p j + i].  score: fp32 [B,H,M]. */
+lh_status lh_score(const lh_shape* shape, lh_dtype dtype, const void* q, const void* k,
+                   float* score, lh_stream_t stream);
+
+/* (c) Joint top-S over all levels, [ES] §2.B: the S entries with the largest
+ * (score, -gid), then ordered by (pos, level), [ES] §2.C.
+ * idx, pos: int32 [B,H,S] (gid and position of slot k); slot: int32 [B,H,M]
+ * (slot of each entry, -1 if not selected).  Scores must be >= 0 (they are
+ * sums of norms).  ws may be NULL when lh_topk_workspace_bytes() is 0.       */
+size_t lh_topk_workspace_bytes(const lh_shape* shape);
+lh_status lh_topk_select(const lh_shape* shape, const float* score, int32_t* idx, int32_t* pos,
+                         int32_t* slot, void* ws, size_t ws_bytes, lh_stream_t stream);
+
+/* (d) Gather, [ES] §2.C: xs[k] = fp16_rne(X^(l_k)[j_k]) (saturating), level 0
+ * read from the input, coarser levels from the pyramid.  qs, ks, vs: fp16
+ * [B,H,S,d].                                                                 */
+lh_status lh_gather(const lh_shape* shape, lh_dtype dtype, const void* q, const void* k,
+                    const void* v, const float* pq, const float* pk, const float* pv,
+                    const int32_t* idx, void* qs, void* ks, void* vs, lh_stream_t stream);
+
+/* (e) Causal attention on the sub-sequence, [ES] §2.C (stock SDPA on a dense
+ * sequence): os[k] = sum_{k'<=k} softmax_k'(scale <qs[k], ks[k']>) vs[k'],
+ * lse[k] = natural log of the softmax denominator (with the max folded in).
+ * scale <= 0 selects 1/sqrt(d).  qs, ks, vs, os: fp16 [B,H,S,d]; lse: fp32
+ * [B,H,S].  Products run on the tensor cores in fp16 with fp32 accumulation;
+ * the softmax weights P are rounded to fp16 before the product with vs.     */
+lh_status lh_subseq_attn_fwd(const lh_shape* shape, const void* qs, const void* ks,
+                             const void* vs, float scale, void* os, float* lse,
+                             lh_stream_t stream);
+
+/* (e') Backward of (e): textbook softmax adjoint, D = rowsum(dos * os),
+ * dS = P * (dos vs^T - D); dqs = scale dS ks, dks = scale dS^T qs,
+ * dvs = P^T dos.  dqs, dks, dvs: fp32 [B,H,S,d].  ws: lh_attn_bwd_workspace_bytes. */
+size_t lh_attn_bwd_workspace_bytes(const lh_shape* shape);
+lh_status lh_subseq_attn_bwd(const lh_shape* shape, const void* qs, const void* ks,
+                             const void* vs, const void* os, const float* lse, const void* dos,
+                             float scale, float* dqs, float* dks, float* dvs, void* ws,
+                             size_t ws_bytes, lh_stream_t stream);
+
+/* (f) Scatter-back, [ES] §2.C / [PT] phase 4: c_t = number of selected
+ * entries covering t; O[t] = (sum over them, ascending level, of os[slot]) / c_t,
+ * 0 when c_t = 0.  o: [B,H,N,d] dtype.  inv_count (optional, may be NULL):
+ * fp32 [B,H,N] receives 1/c_t (0 when c_t = 0).                              */
+lh_status lh_scatter_back(const lh_shape* shape, lh_dtype dtype, const void* os,
+                          const int32_t* slot, void* o, float* inv_count, lh_stream_t stream);
+
+/* (f') Adjoint of (f): dos[k] = sum_{t in span(k)} dO[t] / c_t.  dos: fp16
+ * [B,H,S,d].  inv_count may be NULL (then c_t is recounted from slot).     */
+lh_status lh_scatter_back_bwd(const lh_shape* shape, lh_dtype dtype, const void* dO,
+                              const int32_t* slot, const float* inv_count, void* dos,
+                              lh_stream_t stream);
+
+/* (d') Adjoint of (a)+(d): dX[t] = sum_{l ascending, selected} dxs[slot_l(t)] / p^l
+ * with slot_l(t) = slot[off_l + t / p^l], for X in {Q, K, V}.  dqs, dks, dvs:
+ * fp32 [B,H,S,d]; dq, dk, dv: [B,H,N,d] dtype.                               */
+lh_status lh_gather_bwd(const lh_shape* shape, lh_dtype dtype, const float* dqs,
+                        const float* dks, const float* dvs, const int32_t* slot, void* dq,
+                        void* dk, void* dv, lh_stream_t stream);
+
+/* ------------------------------------------------------- fused entry points */
+
+/* Whole forward: (a)-(f).  o: [B,H,N,d] dtype.  saved: lh_saved_bytes, kept by
+ * the caller for lh_backward.  ws: lh_workspace_bytes(shape, dtype, 0 or 1). */
+lh_status lh_forward(const lh_shape* shape, lh_dtype dtype, const void* q, const void* k,
+                     const void* v, float scale, void* o, void* saved, void* ws,
+                     size_t ws_bytes, lh_stream_t stream);
+
+/* Whole backward with the saved selection: (f'), (e'), (d').  dO: [B,H,N,d]
+ * dtype; dq, dk, dv: [B,H,N,d] dtype.  ws: lh_workspace_bytes(shape, dtype, 1). */
+lh_status lh_backward(const lh_shape* shape, lh_dtype dtype, const void* saved, const void* dO,
+                      float scale, void* dq, void* dk, void* dv, void* ws, size_t ws_bytes,
+                      lh_stream_t stream);
+
+/* Reads and clears the device status word that bounded waits in the kernels
+ * set when they give up (synchronises `stream`).  LH_OK or LH_ERR_DEVICE_STATUS;
+ * *code (may be NULL) receives the raw word (0 = none). */
+lh_status lh_read_device_status(lh_stream_t stream, uint32_t* code);
+
+/* Selects the attention implementation for subsequent calls on this process:
+ * 0 = tcgen05/TMEM (default on sm_100), 1 = warp-level mma.sync kernels (kept
+ * as the comparison baseline).  Returns the previous value. */
+int lh_set_attention_impl(int impl);
+
+/* The attention implementation the next call would use: 0 tcgen05, 1 mma.sync. */
+int lh_attention_impl_in_use(void);
+
+/* Number of kernel launches lh_forward (backward = 0) or lh_backward
+ * (backward = 1) enqueues for this shape with the current implementation;
+ * -1 for an invalid shape. */
+int lh_kernel_launches(const lh_shape* shape, int backward);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* LIGHTHOUSE_H */

@@ -1,0 +1,369 @@
+// k_gather_scatter.cu -- gather into the dense sub-sequence, scatter-back, and
+// the adjoints of both.
+//
+// Method: [ES] gist.science/es "Resumen Técnico: Pre-entrenamiento con Contexto
+// Largo mediante Atención Lighthouse" §2.C: the selected triplets form one dense
+// sequence (gather) and a deterministic kernel returns the attention outputs to
+// their original positions (scatter-back); §2.B: gradients flow back through
+// scatter-back, the attention and the gather only.  "Contributors" per original
+// position: phase 1 of bitsgeniais.com.br "Adeus Custo Quadrático! ...".
+//
+// Every kernel gives a group of G = d/8 consecutive lanes one row (or one
+// coarsest span) and lane c columns [8c, 8c+8): all HBM traffic is 128-bit and
+// coalesced, and every output element is written by exactly one thread in a
+// fixed order of additions (no atomics), so results are bitwise reproducible.
+#include "lh_internal.cuh"
+
+namespace lh {
+namespace {
+
+struct Lv {
+  int64_t N, M, S;
+  int L, p;
+  int64_t off[kMaxLevels + 1];
+  int64_t pw[kMaxLevels + 1];
+};
+
+Lv make_lv(const Geom& g) {
+  Lv v;
+  v.N = g.N;
+  v.M = g.M;
+  v.S = g.S;
+  v.L = g.L;
+  v.p = g.p;
+  for (int l = 0; l <= kMaxLevels; ++l) {
+    v.off[l] = g.off[l];
+    v.pw[l] = g.pw[l];
+  }
+  return v;
+}
+
+inline unsigned blocks_for(int64_t threads, int block) {
+  return (unsigned)((threads + block - 1) / block);
+}
+
+// ------------------------------------------------------------------ gather
+// xs[u,k] = fp16_rne(level row of gid idx[u,k]), saturating; level 0 from the input.
+template <typename Tin, int D>
+__global__ void __launch_bounds__(256) k_gather(
+    const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin* __restrict__ v,
+    const float* __restrict__ pq, const float* __restrict__ pk, const float* __restrict__ pv,
+    const int32_t* __restrict__ idx, __half* __restrict__ qs, __half* __restrict__ ks,
+    __half* __restrict__ vs, const Lv lv, int64_t rows) {
+  constexpr int G = D / 8;
+  const int64_t gt = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  const int64_t row = gt / G;  // u * S + slot
+  if (row >= rows) return;
+  const int c = (int)(gt % G);
+  const int64_t u = row / lv.S;
+  const int64_t gid = __ldg(idx + row);
+  float xq[8], xk[8], xv[8];
+  if (gid < lv.N) {
+    const int64_t o = (u * lv.N + gid) * D + 8 * c;
+    load8(q + o, xq);
+    load8(k + o, xk);
+    load8(v + o, xv);
+  } else {
+    const int64_t o = (u * (lv.M - lv.N) + (gid - lv.N)) * D + 8 * c;
+    load8(pq + o, xq);
+    load8(pk + o, xk);
+    load8(pv + o, xv);
+  }
+  const int64_t d = row * D + 8 * c;
+  store8(qs + d, xq);
+  store8(ks + d, xk);
+  store8(vs + d, xv);
+}
+
+// ------------------------------------------------------------- scatter-back
+// O[t] = (sum over selected entries covering t, ascending level, of os[slot]) / c_t.
+template <typename Tout, int D>
+__global__ void __launch_bounds__(256) k_scatter(const __half* __restrict__ os,
+                                                 const int32_t* __restrict__ slot,
+                                                 Tout* __restrict__ o, float* __restrict__ inv_count,
+                                                 const Lv lv, int64_t rows) {
+  constexpr int G = D / 8;
+  const int64_t gt = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  const int64_t row = gt / G;  // u * N + t
+  if (row >= rows) return;
+  const int c = (int)(gt % G);
+  const int64_t u = row / lv.N, t = row % lv.N;
+  const int32_t* sl = slot + u * lv.M;
+  float acc[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) acc[i] = 0.0f;
+  int cnt = 0;
+  for (int l = 0; l < lv.L; ++l) {
+    const int32_t s = __ldg(sl + lv.off[l] + t / lv.pw[l]);
+    if (s >= 0) {
+      float x[8];
+      load8(os + (u * lv.S + s) * D + 8 * c, x);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) acc[i] = __fadd_rn(acc[i], x[i]);
+      ++cnt;
+    }
+  }
+  if (cnt > 0) {
+    const float fc = (float)cnt;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) acc[i] = __fdiv_rn(acc[i], fc);
+  }
+  store8_stream(o + row * D + 8 * c, acc);
+  if (inv_count && c == 0) inv_count[row] = cnt > 0 ? __frcp_rn((float)cnt) : 0.0f;
+}
+
+// ---------------------------------------------------------- scatter-back bwd
+// dos[k] = sum_{t in span(k)} dO[t] / c_t, as a sum-pyramid of w[t] = dO[t]/c_t
+// over each coarsest span: dO is read once, each selected row written once.
+template <typename Tin, int D, int L>
+__global__ void __launch_bounds__(256) k_scatter_bwd(const Tin* __restrict__ dO,
+                                                     const int32_t* __restrict__ slot,
+                                                     const float* __restrict__ inv_count,
+                                                     __half* __restrict__ dos, const Lv lv,
+                                                     int64_t spans, int64_t groups) {
+  constexpr int G = D / 8;
+  constexpr int NL = (L > 1) ? (L - 1) : 1;
+  const int64_t gt = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  const int64_t group = gt / G;
+  if (group >= groups) return;
+  const int c = (int)(gt % G);
+  const int64_t Ptop = lv.pw[L - 1];
+  const int64_t u = group / spans;
+  const int64_t t0 = (group % spans) * Ptop;
+  const int32_t* sl = slot + u * lv.M;
+  const Tin* src = dO + (u * lv.N + t0) * D + 8 * c;
+  __half* dst = dos + u * lv.S * D + 8 * c;
+
+  float acc[NL][8];
+  int cnt[NL];
+#pragma unroll
+  for (int l = 0; l < NL; ++l) {
+    cnt[l] = 0;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) acc[l][i] = 0.0f;
+  }
+  for (int64_t r = 0; r < Ptop; ++r) {
+    const int64_t t = t0 + r;
+    float w[8];
+    load8_stream(src + r * D, w);
+    float ic;
+    if (inv_count) {
+      ic = __ldg(inv_count + u * lv.N + t);
+    } else {
+      int n = 0;
+#pragma unroll
+      for (int l = 0; l < L; ++l) n += (__ldg(sl + lv.off[l] + t / lv.pw[l]) >= 0) ? 1 : 0;
+      ic = n > 0 ? __frcp_rn((float)n) : 0.0f;
+    }
+#pragma unroll
+    for (int i = 0; i < 8; ++i) w[i] = __fmul_rn(w[i], ic);
+    const int32_t s0 = __ldg(sl + t);
+    if (s0 >= 0) store8(dst + (int64_t)s0 * D, w);
+    if constexpr (L == 1) continue;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) acc[0][i] = __fadd_rn(acc[0][i], w[i]);
+    cnt[0] += 1;
+#pragma unroll
+    for (int l = 0; l < NL; ++l) {
+      if (cnt[l] == lv.p) {
+        const int lev = l + 1;
+        const int64_t j = (t + 1) / lv.pw[lev] - 1;
+        const int32_t s = __ldg(sl + lv.off[lev] + j);
+        if (s >= 0) store8(dst + (int64_t)s * D, acc[l]);
+        if (l + 1 < NL) {
+#pragma unroll
+          for (int i = 0; i < 8; ++i) acc[l + 1][i] = __fadd_rn(acc[l + 1][i], acc[l][i]);
+          cnt[l + 1] += 1;
+        }
+#pragma unroll
+        for (int i = 0; i < 8; ++i) acc[l][i] = 0.0f;
+        cnt[l] = 0;
+      }
+    }
+  }
+}
+
+// --------------------------------------------------------------- gather bwd
+// dX[t] = sum_{l ascending, selected} dxs[slot_l(t)] / p^l, X in {Q, K, V}.
+template <typename Tout, int D>
+__global__ void __launch_bounds__(256) k_gather_bwd(
+    const float* __restrict__ dqs, const float* __restrict__ dks, const float* __restrict__ dvs,
+    const int32_t* __restrict__ slot, Tout* __restrict__ dq, Tout* __restrict__ dk,
+    Tout* __restrict__ dv, const Lv lv, int64_t rows) {
+  constexpr int G = D / 8;
+  const int64_t gt = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  const int64_t row = gt / G;  // u * N + t
+  if (row >= rows) return;
+  const int c = (int)(gt % G);
+  const int64_t u = row / lv.N, t = row % lv.N;
+  const int32_t* sl = slot + u * lv.M;
+  float aq[8], ak[8], av[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) aq[i] = ak[i] = av[i] = 0.0f;
+  for (int l = 0; l < lv.L; ++l) {
+    const int32_t s = __ldg(sl + lv.off[l] + t / lv.pw[l]);
+    if (s >= 0) {
+      const float inv = __frcp_rn((float)lv.pw[l]);
+      const int64_t o = (u * lv.S + s) * D + 8 * c;
+      float x[8];
+      load8(dqs + o, x);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) aq[i] = __fmaf_rn(x[i], inv, aq[i]);
+      load8(dks + o, x);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) ak[i] = __fmaf_rn(x[i], inv, ak[i]);
+      load8(dvs + o, x);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) av[i] = __fmaf_rn(x[i], inv, av[i]);
+    }
+  }
+  const int64_t o = row * D + 8 * c;
+  store8_stream(dq + o, aq);
+  store8_stream(dk + o, ak);
+  store8_stream(dv + o, av);
+}
+
+// ---------------------------------------------------------- D = rowsum(dO*O)
+template <int D>
+__global__ void __launch_bounds__(256) k_rowdot(const __half* __restrict__ os,
+                                                const __half* __restrict__ dos,
+                                                float* __restrict__ Dout, int64_t rows) {
+  constexpr int G = D / 8;
+  const int64_t gt = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  const int64_t row = gt / G;
+  if (row >= rows) return;
+  const int c = (int)(gt % G);
+  const int lane = threadIdx.x & 31;
+  const unsigned gmask = ((G == 32) ? 0xffffffffu : ((1u << G) - 1u)) << (lane & ~(G - 1));
+  float a[8], b[8];
+  load8(os + row * D + 8 * c, a);
+  load8(dos + row * D + 8 * c, b);
+  float s = 0.0f;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) s = __fmaf_rn(a[i], b[i], s);
+#pragma unroll
+  for (int off = 1; off < G; off <<= 1) s = __fadd_rn(s, __shfl_xor_sync(gmask, s, off));
+  if (c == 0) Dout[row] = s;
+}
+
+}  // namespace
+
+cudaError_t launch_gather(const Geom& g, lh_dtype dt, const void* q, const void* k, const void* v,
+                          const float* pq, const float* pk, const float* pv, const int32_t* idx,
+                          __half* qs, __half* ks, __half* vs, cudaStream_t st) {
+  const Lv lv = make_lv(g);
+  const int64_t rows = g.U * g.S;
+  const unsigned nb = blocks_for(rows * (g.d / 8), 256);
+  if (dt == LH_BF16) {
+    auto* a = static_cast<const __nv_bfloat16*>(q);
+    auto* b = static_cast<const __nv_bfloat16*>(k);
+    auto* c = static_cast<const __nv_bfloat16*>(v);
+    if (g.d == 64)
+      k_gather<__nv_bfloat16, 64><<<nb, 256, 0, st>>>(a, b, c, pq, pk, pv, idx, qs, ks, vs, lv, rows);
+    else
+      k_gather<__nv_bfloat16, 128><<<nb, 256, 0, st>>>(a, b, c, pq, pk, pv, idx, qs, ks, vs, lv, rows);
+  } else {
+    auto* a = static_cast<const float*>(q);
+    auto* b = static_cast<const float*>(k);
+    auto* c = static_cast<const float*>(v);
+    if (g.d == 64)
+      k_gather<float, 64><<<nb, 256, 0, st>>>(a, b, c, pq, pk, pv, idx, qs, ks, vs, lv, rows);
+    else
+      k_gather<float, 128><<<nb, 256, 0, st>>>(a, b, c, pq, pk, pv, idx, qs, ks, vs, lv, rows);
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_scatter(const Geom& g, lh_dtype dt, const __half* os,
+                           const int32_t* slot, void* o, float* inv_count, cudaStream_t st) {
+  const Lv lv = make_lv(g);
+  const int64_t rows = g.U * g.N;
+  const unsigned nb = blocks_for(rows * (g.d / 8), 256);
+  if (dt == LH_BF16) {
+    auto* out = static_cast<__nv_bfloat16*>(o);
+    if (g.d == 64)
+      k_scatter<__nv_bfloat16, 64><<<nb, 256, 0, st>>>(os, slot, out, inv_count, lv, rows);
+    else
+      k_scatter<__nv_bfloat16, 128><<<nb, 256, 0, st>>>(os, slot, out, inv_count, lv, rows);
+  } else {
+    auto* out = static_cast<float*>(o);
+    if (g.d == 64)
+      k_scatter<float, 64><<<nb, 256, 0, st>>>(os, slot, out, inv_count, lv, rows);
+    else
+      k_scatter<float, 128><<<nb, 256, 0, st>>>(os, slot, out, inv_count, lv, rows);
+  }
+  return cudaGetLastError();
+}
+
+namespace {
+template <typename Tin, int D>
+cudaError_t scatter_bwd_d(const Geom& g, const Tin* dO, const int32_t* slot, const float* ic,
+                          __half* dos, cudaStream_t st) {
+  const Lv lv = make_lv(g);
+  const int64_t spans = g.N / g.pw[g.L - 1];
+  const int64_t groups = g.U * spans;
+  const unsigned nb = blocks_for(groups * (D / 8), 256);
+  switch (g.L) {
+#define LH_CASE(LL)                                                                      \
+  case LL:                                                                               \
+    k_scatter_bwd<Tin, D, LL><<<nb, 256, 0, st>>>(dO, slot, ic, dos, lv, spans, groups); \
+    break;
+    LH_CASE(1) LH_CASE(2) LH_CASE(3) LH_CASE(4) LH_CASE(5) LH_CASE(6) LH_CASE(7) LH_CASE(8)
+#undef LH_CASE
+    default:
+      return cudaErrorInvalidValue;
+  }
+  return cudaGetLastError();
+}
+}  // namespace
+
+cudaError_t launch_scatter_bwd(const Geom& g, lh_dtype dt, const void* dO, const int32_t* slot,
+                               const float* inv_count, __half* dos, cudaStream_t st) {
+  if (dt == LH_BF16) {
+    auto* a = static_cast<const __nv_bfloat16*>(dO);
+    return g.d == 64 ? scatter_bwd_d<__nv_bfloat16, 64>(g, a, slot, inv_count, dos, st)
+                     : scatter_bwd_d<__nv_bfloat16, 128>(g, a, slot, inv_count, dos, st);
+  }
+  auto* a = static_cast<const float*>(dO);
+  return g.d == 64 ? scatter_bwd_d<float, 64>(g, a, slot, inv_count, dos, st)
+                   : scatter_bwd_d<float, 128>(g, a, slot, inv_count, dos, st);
+}
+
+cudaError_t launch_gather_bwd(const Geom& g, lh_dtype dt, const float* dqs, const float* dks,
+                              const float* dvs, const int32_t* slot, void* dq, void* dk, void* dv,
+                              cudaStream_t st) {
+  const Lv lv = make_lv(g);
+  const int64_t rows = g.U * g.N;
+  const unsigned nb = blocks_for(rows * (g.d / 8), 256);
+  if (dt == LH_BF16) {
+    auto* a = static_cast<__nv_bfloat16*>(dq);
+    auto* b = static_cast<__nv_bfloat16*>(dk);
+    auto* c = static_cast<__nv_bfloat16*>(dv);
+    if (g.d == 64)
+      k_gather_bwd<__nv_bfloat16, 64><<<nb, 256, 0, st>>>(dqs, dks, dvs, slot, a, b, c, lv, rows);
+    else
+      k_gather_bwd<__nv_bfloat16, 128><<<nb, 256, 0, st>>>(dqs, dks, dvs, slot, a, b, c, lv, rows);
+  } else {
+    auto* a = static_cast<float*>(dq);
+    auto* b = static_cast<float*>(dk);
+    auto* c = static_cast<float*>(dv);
+    if (g.d == 64)
+      k_gather_bwd<float, 64><<<nb, 256, 0, st>>>(dqs, dks, dvs, slot, a, b, c, lv, rows);
+    else
+      k_gather_bwd<float, 128><<<nb, 256, 0, st>>>(dqs, dks, dvs, slot, a, b, c, lv, rows);
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_attn_rowdot(const Geom& g, const __half* os, const __half* dos,
+                               float* D, cudaStream_t st) {
+  const int64_t rows = g.U * g.S;
+  const unsigned nb = blocks_for(rows * (g.d / 8), 256);
+  if (g.d == 64)
+    k_rowdot<64><<<nb, 256, 0, st>>>(os, dos, D, rows);
+  else
+    k_rowdot<128><<<nb, 256, 0, st>>>(os, dos, D, rows);
+  return cudaGetLastError();
+}
+
+}  // namespace lh

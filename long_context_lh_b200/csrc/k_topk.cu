@@ -1,0 +1,339 @@
+// k_topk.cu -- joint top-S over all pyramid levels and the gather order.
+//
+// Method: [ES] gist.science/es "Resumen Técnico: Pre-entrenamiento con Contexto
+// Largo mediante Atención Lighthouse" §2.B (one top-K across all levels) and
+// §2.C (the selected triplets are sorted topologically into one dense,
+// hole-free sequence; phase 3 of bitsgeniais.com.br "Adeus Custo Quadrático!").
+//
+// Selection rule: the S entries with the largest (score, -gid); the ranking is
+// a strict total order, so the set is unique.  Because it is a threshold rule,
+// no sort of the keys is needed, only the S-th largest key:
+//   1. radix select on the 32 score bits (scores are >= 0, so their bits order
+//      like their values) in digits of 11/11/10 bits, giving the threshold score
+//      T and how many entries scoring exactly T are still needed;
+//   2. if only some of the entries at T fit, radix select (ascending) on their
+//      gids gives the largest gid that still fits.
+//   Entry g is selected iff score > T, or score == T and gid <= that gid.
+// Gather order (pos ascending, then level ascending) is a fixed enumeration of
+// all entries: token t = 0..N-1, and at each t the levels l whose span ends at
+// t ((t+1) % p^l == 0).  One ordered stream compaction over that enumeration
+// gives slots directly, with no sort.
+//
+// B200 mapping: one thread-block cluster of CL CTAs per unit.  Each CTA
+// histograms its share of the unit's scores in shared memory; the cluster sums
+// the histograms through distributed shared memory, and every CTA picks the
+// digit redundantly (same integers, same result), so a pass costs one cluster
+// barrier.  The compaction uses per-warp ballots/scans, per-CTA totals through
+// DSMEM, and writes idx/pos/slot once.  Integer work only: bit-exact.
+#include <cooperative_groups.h>
+
+#include <atomic>
+
+#include "lh_internal.cuh"
+
+namespace cg = cooperative_groups;
+
+namespace lh {
+namespace {
+
+constexpr int kThreads = 1024;
+constexpr int kWarps = kThreads / 32;
+constexpr int kBins = 2048;
+
+struct TopkParams {
+  int64_t N, M;
+  int p, L, S;
+  int64_t unit0;
+  int64_t off[kMaxLevels + 1];
+  int64_t pw[kMaxLevels + 1];
+};
+
+__device__ __forceinline__ uint32_t warp_incl_scan(uint32_t v) {
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    uint32_t n = __shfl_up_sync(0xffffffffu, v, o);
+    if (lane >= o) v += n;
+  }
+  return v;
+}
+
+// Block-wide exclusive scan of one value per thread; returns the exclusive
+// prefix and writes the block total to *total (all threads see it).
+__device__ uint32_t block_excl_scan(uint32_t v, uint32_t* warp_buf, uint32_t* total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  uint32_t incl = warp_incl_scan(v);
+  if (lane == 31) warp_buf[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    uint32_t w = warp_buf[lane];
+    uint32_t wi = warp_incl_scan(w);
+    warp_buf[lane] = wi - w;  // exclusive
+    if (lane == 31) *total = wi;
+  }
+  __syncthreads();
+  uint32_t res = warp_buf[warp] + incl - v;
+  __syncthreads();  // warp_buf may be reused right after
+  return res;
+}
+
+struct Pick {
+  uint32_t bin;    // selected digit value
+  uint32_t before; // count of candidates ranked before that digit
+  uint32_t inbin;  // candidates with that digit
+};
+
+// Cluster-summed histogram -> digit where the need-th candidate falls.
+// descending: rank digits from the largest value down (scores), else up (gids).
+__device__ Pick pick_digit(cg::cluster_group& cluster, uint32_t* hist, int nbins, bool descending,
+                           uint32_t need, uint32_t* warp_buf, uint32_t* sh) {
+  const int CL = (int)cluster.num_blocks();
+  const int per = nbins / kThreads;  // 2 or 1 ordinals per thread
+  uint32_t tot[2] = {0, 0};
+  uint32_t local = 0;
+  for (int i = 0; i < per; ++i) {
+    const int ord = threadIdx.x * per + i;
+    const int bin = descending ? (nbins - 1 - ord) : ord;
+    uint32_t s = 0;
+    for (int r = 0; r < CL; ++r) s += cluster.map_shared_rank(hist, r)[bin];
+    tot[i] = s;
+    local += s;
+  }
+  uint32_t all;
+  uint32_t before = block_excl_scan(local, warp_buf, &all);
+  for (int i = 0; i < per; ++i) {
+    const int ord = threadIdx.x * per + i;
+    if (before < need && need <= before + tot[i]) {
+      sh[0] = descending ? (uint32_t)(nbins - 1 - ord) : (uint32_t)ord;
+      sh[1] = before;
+      sh[2] = tot[i];
+    }
+    before += tot[i];
+  }
+  __syncthreads();
+  Pick pk{sh[0], sh[1], sh[2]};
+  __syncthreads();
+  return pk;
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+    k_topk(const float* __restrict__ score, int32_t* __restrict__ idx, int32_t* __restrict__ pos,
+           int32_t* __restrict__ slot, const TopkParams prm) {
+  cg::cluster_group cluster = cg::this_cluster();
+  const int CL = (int)cluster.num_blocks();
+  const int rank = (int)cluster.block_rank();
+  const int64_t u = prm.unit0 + blockIdx.y;
+
+  __shared__ uint32_t hist[2][kBins];
+  __shared__ uint32_t warp_buf[32];
+  __shared__ uint32_t sh[4];
+  __shared__ uint32_t warp_tot[kWarps];
+  __shared__ uint32_t cta_total;
+
+  const uint32_t* key = reinterpret_cast<const uint32_t*>(score + u * prm.M);
+  const int64_t M = prm.M;
+  const int64_t per = (M + CL - 1) / CL;
+  const int64_t g_begin = imin64(M, (int64_t)rank * per);
+  const int64_t g_end = imin64(M, g_begin + per);
+
+  cluster.sync();  // every CTA of the cluster is running before DSMEM use
+
+  // ---- 1. threshold score by radix select on the key bits (descending)
+  uint32_t prefix = 0, pmask = 0, need = (uint32_t)prm.S, ties = 0;
+  int buf = 0;
+  // digits of the 32 key bits, high to low: [21,32), [10,21), [0,10)
+  for (int pass = 0; pass < 3; ++pass) {
+    const int shift = pass == 0 ? 21 : (pass == 1 ? 10 : 0);
+    const int nb = pass == 2 ? 1024 : 2048;
+    const uint32_t dmask = (uint32_t)nb - 1u;
+    for (int i = threadIdx.x; i < kBins; i += kThreads) hist[buf][i] = 0;
+    __syncthreads();
+    for (int64_t g = g_begin + threadIdx.x; g < g_end; g += kThreads) {
+      const uint32_t kv = __ldg(key + g);
+      if ((kv & pmask) == prefix) atomicAdd(&hist[buf][(kv >> shift) & dmask], 1u);
+    }
+    cluster.sync();
+    Pick pk = pick_digit(cluster, hist[buf], nb, true, need, warp_buf, sh);
+    prefix |= pk.bin << shift;
+    pmask |= dmask << shift;
+    need -= pk.before;
+    ties = pk.inbin;
+    buf ^= 1;
+  }
+  const uint32_t T = prefix;
+
+  // ---- 2. among entries scoring exactly T, the need smallest gids
+  int64_t gid_thr = INT64_MAX;
+  if (need < ties) {
+    int nbits = 1;
+    while (nbits < 31 && ((int64_t)1 << nbits) < M) ++nbits;
+    uint32_t gprefix = 0, gmask = 0;
+    for (int hi = nbits; hi > 0;) {
+      const int w = hi >= 11 ? 11 : hi;
+      const int shift = hi - w;
+      const int nb = 1 << w;
+      const uint32_t dmask = (uint32_t)nb - 1u;
+      for (int i = threadIdx.x; i < kBins; i += kThreads) hist[buf][i] = 0;
+      __syncthreads();
+      for (int64_t g = g_begin + threadIdx.x; g < g_end; g += kThreads) {
+        if (__ldg(key + g) == T && (((uint32_t)g) & gmask) == gprefix)
+          atomicAdd(&hist[buf][((uint32_t)g >> shift) & dmask], 1u);
+      }
+      cluster.sync();
+      // pick_digit needs nbins to be a multiple of the thread count or equal to
+      // 1024/2048; smaller digit widths are padded with empty bins.
+      const int nbp = nb < kThreads ? kThreads : nb;
+      Pick pk = pick_digit(cluster, hist[buf], nbp, false, need, warp_buf, sh);
+      gprefix |= pk.bin << shift;
+      gmask |= dmask << shift;
+      need -= pk.before;
+      buf ^= 1;
+      hi = shift;
+    }
+    gid_thr = (int64_t)gprefix;
+  }
+
+  // ---- 3. ordered compaction over (token, level)
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int64_t tper = (prm.N + CL - 1) / CL;
+  const int64_t t_begin = imin64(prm.N, (int64_t)rank * tper);
+  const int64_t t_end = imin64(prm.N, t_begin + tper);
+  const int64_t wper = ((t_end - t_begin + kWarps - 1) / kWarps + 31) / 32 * 32;
+  const int64_t w_begin = imin64(t_end, t_begin + warp * wper);
+  const int64_t w_end = imin64(t_end, w_begin + wper);
+
+  auto selected = [&](int64_t g) -> bool {
+    const uint32_t kv = __ldg(key + g);
+    return kv > T || (kv == T && g <= gid_thr);
+  };
+  // pass A: count per warp
+  uint32_t wcount = 0;
+  for (int64_t tb = w_begin; tb < w_end; tb += 32) {
+    const int64_t t = tb + lane;
+    uint32_t c = 0;
+    if (t < w_end) {
+      for (int l = 0; l < prm.L; ++l) {
+        if ((t + 1) % prm.pw[l] != 0) break;  // spans end at t only up to some level
+        c += selected(prm.off[l] + (t + 1) / prm.pw[l] - 1) ? 1u : 0u;
+      }
+    }
+    wcount += __reduce_add_sync(0xffffffffu, c);
+  }
+  if (lane == 0) warp_tot[warp] = wcount;
+  __syncthreads();
+  if (warp == 0) {
+    uint32_t w = warp_tot[lane];
+    uint32_t wi = warp_incl_scan(w);
+    warp_tot[lane] = wi - w;
+    if (lane == 31) cta_total = wi;
+  }
+  cluster.sync();
+  uint32_t base = 0;
+  for (int r = 0; r < rank; ++r) base += *cluster.map_shared_rank(&cta_total, r);
+  base += warp_tot[warp];
+  // pass B: write
+  int32_t* idx_u = idx + u * prm.S;
+  int32_t* pos_u = pos + u * prm.S;
+  int32_t* slot_u = slot + u * prm.M;
+  for (int64_t tb = w_begin; tb < w_end; tb += 32) {
+    const int64_t t = tb + lane;
+    uint32_t c = 0;
+    uint32_t selmask = 0;
+    if (t < w_end) {
+      for (int l = 0; l < prm.L; ++l) {
+        if ((t + 1) % prm.pw[l] != 0) break;
+        if (selected(prm.off[l] + (t + 1) / prm.pw[l] - 1)) {
+          selmask |= 1u << l;
+          ++c;
+        }
+      }
+    }
+    const uint32_t incl = warp_incl_scan(c);
+    uint32_t k = base + incl - c;
+    if (t < w_end) {
+      for (int l = 0; l < prm.L; ++l) {
+        if ((t + 1) % prm.pw[l] != 0) break;
+        const int64_t g = prm.off[l] + (t + 1) / prm.pw[l] - 1;
+        if (selmask & (1u << l)) {
+          idx_u[k] = (int32_t)g;
+          pos_u[k] = (int32_t)t;
+          slot_u[g] = (int32_t)k;
+          ++k;
+        } else {
+          slot_u[g] = -1;
+        }
+      }
+    }
+    base += __shfl_sync(0xffffffffu, incl, 31);
+  }
+  cluster.sync();  // keep shared memory alive until every remote read is done
+}
+
+}  // namespace
+
+cudaError_t launch_topk(const Geom& g, const float* score, int32_t* idx, int32_t* pos,
+                        int32_t* slot, cudaStream_t st) {
+  TopkParams prm;
+  prm.N = g.N;
+  prm.M = g.M;
+  prm.p = g.p;
+  prm.L = g.L;
+  prm.S = g.S;
+  for (int l = 0; l <= kMaxLevels; ++l) {
+    prm.off[l] = g.off[l];
+    prm.pw[l] = g.pw[l];
+  }
+  // Larger clusters for larger units: more SMs per unit, same barrier count.
+  // A 16-CTA cluster is a non-portable size; it is used only when this device
+  // can hold one (checked once per device).
+  int CL = 8;
+  if (g.M > ((int64_t)1 << 19)) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return cudaGetLastError();
+    static std::atomic<int> ok16[64];  // 0 unknown, 1 yes, 2 no
+    int state = dev < 64 ? ok16[dev].load() : 2;
+    if (state == 0) {
+      state = 2;
+      if (cudaFuncSetAttribute(k_topk, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) ==
+          cudaSuccess) {
+        cudaLaunchConfig_t q = {};
+        q.gridDim = dim3(16, 1, 1);
+        q.blockDim = dim3(kThreads, 1, 1);
+        cudaLaunchAttribute a[1];
+        a[0].id = cudaLaunchAttributeClusterDimension;
+        a[0].val.clusterDim.x = 16;
+        a[0].val.clusterDim.y = 1;
+        a[0].val.clusterDim.z = 1;
+        q.attrs = a;
+        q.numAttrs = 1;
+        int nclusters = 0;
+        if (cudaOccupancyMaxActiveClusters(&nclusters, k_topk, &q) == cudaSuccess && nclusters > 0)
+          state = 1;
+      }
+      (void)cudaGetLastError();
+      ok16[dev].store(state);
+    }
+    if (state == 1) CL = 16;
+  }
+  for (int64_t u0 = 0; u0 < g.U; u0 += 65535) {
+    prm.unit0 = u0;
+    const int64_t nu = g.U - u0 < 65535 ? g.U - u0 : 65535;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)CL, (unsigned)nu, 1);
+    cfg.blockDim = dim3(kThreads, 1, 1);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = (unsigned)CL;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, k_topk, score, idx, pos, slot, prm);
+    if (e != cudaSuccess) return e;
+  }
+  return cudaSuccess;
+}
+
+}  // namespace lh

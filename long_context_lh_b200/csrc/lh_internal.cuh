@@ -1,0 +1,176 @@
+// lh_internal.cuh -- shared definitions of the CUDA library (not part of the ABI).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/lighthouse.h"
+
+namespace lh {
+
+constexpr int kMaxLevels = 8;
+
+// Per-unit geometry derived from an lh_shape (host and device).
+struct Geom {
+  int64_t U;      // B * H independent units
+  int64_t N;      // tokens
+  int64_t M;      // pyramid entries per unit
+  int d, p, L, S;
+  int64_t pw[kMaxLevels + 1];   // p^l
+  int64_t off[kMaxLevels + 1];  // first gid of level l; off[L] = M
+};
+
+Geom make_geom(const lh_shape& s);
+
+// ---------------------------------------------------------------- device status
+// One word per device, set by kernels whose bounded waits give up and read and
+// cleared by lh_read_device_status.  It lives in the translation unit of the
+// kernels that wait (k_attn_tc.cu); this reads and clears it (synchronous).
+cudaError_t device_status_read_clear(uint32_t* value);
+
+enum : uint32_t {
+  kStatusAttnFwdTimeout = 0x100,
+  kStatusAttnBwdTimeout = 0x200,
+};
+
+__device__ __forceinline__ int64_t imin64(int64_t a, int64_t b) { return a < b ? a : b; }
+
+// ---------------------------------------------------------------- small helpers
+__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
+
+// Largest finite fp16; the sub-sequence saturates there instead of overflowing.
+constexpr float kHalfMax = 65504.0f;
+
+__device__ __forceinline__ float h_lo(uint32_t w) {
+  return __half2float(__ushort_as_half((unsigned short)(w & 0xffffu)));
+}
+__device__ __forceinline__ float h_hi(uint32_t w) {
+  return __half2float(__ushort_as_half((unsigned short)(w >> 16)));
+}
+__device__ __forceinline__ uint32_t pack_h2(float lo, float hi) {
+  __half2 h = __floats2half2_rn(lo, hi);  // .x = lo (low half)
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+__device__ __forceinline__ uint32_t pack_h2_sat(float lo, float hi) {
+  return pack_h2(fminf(fmaxf(lo, -kHalfMax), kHalfMax), fminf(fmaxf(hi, -kHalfMax), kHalfMax));
+}
+
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
+  __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);  // .x = lo (low half), .y = hi
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+
+// Load 8 consecutive elements of a row as fp32 (bf16 widening is exact).
+__device__ __forceinline__ void load8(const __nv_bfloat16* p, float (&x)[8]) {
+  uint4 w = __ldg(reinterpret_cast<const uint4*>(p));
+  x[0] = bf16_lo(w.x); x[1] = bf16_hi(w.x);
+  x[2] = bf16_lo(w.y); x[3] = bf16_hi(w.y);
+  x[4] = bf16_lo(w.z); x[5] = bf16_hi(w.z);
+  x[6] = bf16_lo(w.w); x[7] = bf16_hi(w.w);
+}
+__device__ __forceinline__ void load8(const float* p, float (&x)[8]) {
+  float4 a = __ldg(reinterpret_cast<const float4*>(p));
+  float4 b = __ldg(reinterpret_cast<const float4*>(p) + 1);
+  x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w;
+  x[4] = b.x; x[5] = b.y; x[6] = b.z; x[7] = b.w;
+}
+// Streaming variant for data read exactly once (keeps L2 for reused data).
+__device__ __forceinline__ void load8_stream(const __nv_bfloat16* p, float (&x)[8]) {
+  uint4 w = __ldcs(reinterpret_cast<const uint4*>(p));
+  x[0] = bf16_lo(w.x); x[1] = bf16_hi(w.x);
+  x[2] = bf16_lo(w.y); x[3] = bf16_hi(w.y);
+  x[4] = bf16_lo(w.z); x[5] = bf16_hi(w.z);
+  x[6] = bf16_lo(w.w); x[7] = bf16_hi(w.w);
+}
+__device__ __forceinline__ void load8_stream(const float* p, float (&x)[8]) {
+  float4 a = __ldcs(reinterpret_cast<const float4*>(p));
+  float4 b = __ldcs(reinterpret_cast<const float4*>(p) + 1);
+  x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w;
+  x[4] = b.x; x[5] = b.y; x[6] = b.z; x[7] = b.w;
+}
+
+__device__ __forceinline__ void load8(const __half* p, float (&x)[8]) {
+  uint4 w = __ldg(reinterpret_cast<const uint4*>(p));
+  x[0] = h_lo(w.x); x[1] = h_hi(w.x);
+  x[2] = h_lo(w.y); x[3] = h_hi(w.y);
+  x[4] = h_lo(w.z); x[5] = h_hi(w.z);
+  x[6] = h_lo(w.w); x[7] = h_hi(w.w);
+}
+// fp16 store that saturates at +-65504 (never writes inf)
+__device__ __forceinline__ void store8(__half* p, const float (&x)[8]) {
+  uint4 w;
+  w.x = pack_h2_sat(x[0], x[1]);
+  w.y = pack_h2_sat(x[2], x[3]);
+  w.z = pack_h2_sat(x[4], x[5]);
+  w.w = pack_h2_sat(x[6], x[7]);
+  *reinterpret_cast<uint4*>(p) = w;
+}
+
+__device__ __forceinline__ void store8(__nv_bfloat16* p, const float (&x)[8]) {
+  uint4 w;
+  w.x = pack_bf16(x[0], x[1]);
+  w.y = pack_bf16(x[2], x[3]);
+  w.z = pack_bf16(x[4], x[5]);
+  w.w = pack_bf16(x[6], x[7]);
+  *reinterpret_cast<uint4*>(p) = w;
+}
+__device__ __forceinline__ void store8(float* p, const float (&x)[8]) {
+  reinterpret_cast<float4*>(p)[0] = make_float4(x[0], x[1], x[2], x[3]);
+  reinterpret_cast<float4*>(p)[1] = make_float4(x[4], x[5], x[6], x[7]);
+}
+__device__ __forceinline__ void store8_stream(__nv_bfloat16* p, const float (&x)[8]) {
+  uint4 w;
+  w.x = pack_bf16(x[0], x[1]);
+  w.y = pack_bf16(x[2], x[3]);
+  w.z = pack_bf16(x[4], x[5]);
+  w.w = pack_bf16(x[6], x[7]);
+  __stcs(reinterpret_cast<uint4*>(p), w);
+}
+__device__ __forceinline__ void store8_stream(float* p, const float (&x)[8]) {
+  __stcs(reinterpret_cast<float4*>(p), make_float4(x[0], x[1], x[2], x[3]));
+  __stcs(reinterpret_cast<float4*>(p) + 1, make_float4(x[4], x[5], x[6], x[7]));
+}
+
+// ---------------------------------------------------------------- launchers
+// Each returns cudaSuccess or the launch error; arguments are already checked.
+cudaError_t launch_pyramid_score(const Geom& g, lh_dtype dt, const void* q, const void* k,
+                                 const void* v, float* pq, float* pk, float* pv, float* score,
+                                 cudaStream_t st);
+cudaError_t launch_topk(const Geom& g, const float* score, int32_t* idx, int32_t* pos,
+                        int32_t* slot, cudaStream_t st);
+cudaError_t launch_gather(const Geom& g, lh_dtype dt, const void* q, const void* k, const void* v,
+                          const float* pq, const float* pk, const float* pv, const int32_t* idx,
+                          __half* qs, __half* ks, __half* vs, cudaStream_t st);
+cudaError_t launch_scatter(const Geom& g, lh_dtype dt, const __half* os,
+                           const int32_t* slot, void* o, float* inv_count, cudaStream_t st);
+cudaError_t launch_scatter_bwd(const Geom& g, lh_dtype dt, const void* dO, const int32_t* slot,
+                               const float* inv_count, __half* dos, cudaStream_t st);
+cudaError_t launch_gather_bwd(const Geom& g, lh_dtype dt, const float* dqs, const float* dks,
+                              const float* dvs, const int32_t* slot, void* dq, void* dk, void* dv,
+                              cudaStream_t st);
+cudaError_t launch_attn_rowdot(const Geom& g, const __half* os, const __half* dos,
+                               float* D, cudaStream_t st);
+
+// Attention: two implementations with the same contract.
+cudaError_t launch_attn_fwd_mma(const Geom& g, const __half* qs, const __half* ks,
+                                const __half* vs, float scale, __half* os,
+                                float* lse, cudaStream_t st);
+cudaError_t launch_attn_bwd_mma(const Geom& g, const __half* qs, const __half* ks,
+                                const __half* vs, const __half* dos,
+                                const float* lse, const float* D, float scale, float* dqs,
+                                float* dks, float* dvs, cudaStream_t st);
+cudaError_t launch_attn_fwd_tc(const Geom& g, const __half* qs, const __half* ks,
+                               const __half* vs, float scale, __half* os,
+                               float* lse, cudaStream_t st);
+cudaError_t launch_attn_bwd_tc(const Geom& g, const __half* qs, const __half* ks,
+                               const __half* vs, const __half* dos,
+                               const float* lse, const float* D, float scale, float* dqs,
+                               float* dks, float* dvs, cudaStream_t st);
+bool attn_tc_available();
+int attn_tc_fwd_launches(const Geom& g);
+int attn_tc_bwd_launches(const Geom& g);
+
+}  // namespace lh

@@ -1,0 +1,105 @@
+"""Host-side checks of the C-ABI library (no GPU needed).
+
+The library must load on a machine without a GPU, export every entry point the
+header declares, and reject bad shapes/arguments on the host before any launch.
+"""
+import ctypes
+import os
+import re
+
+import pytest
+
+from long_context_lh_b200 import lighthouse as lh
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "lighthouse.h")
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(lh_[a-z0-9_]+)\s*\(", src)))
+
+
+def test_library_loads_and_exports_every_declared_symbol():
+    lib = lh._lib()
+    names = declared_functions()
+    assert len(names) >= 20
+    for n in names:
+        assert hasattr(lib, n), f"{n} declared in lighthouse.h but not exported"
+    assert sorted(lh.EXPORTED) == names
+
+
+def S(B=1, H=2, N=4096, d=64, p=4, L=3, S_=512):
+    return lh.make_shape(B, H, N, d, p, L, S_)
+
+
+def test_validate_accepts_the_workloads():
+    for shp in (S(), S(1, 16, 98304, 64, 4, 4, 8192), S(1, 16, 524288, 64, 4, 5, 16384),
+                S(1, 8, 1048576, 128, 4, 6, 16384), S(1, 1, 100, 64, 2, 1, 100)):
+        assert lh.lh_validate(shp, lh.LH_BF16) == lh.LH_OK
+        assert lh.lh_validate(shp, lh.LH_F32) == lh.LH_OK
+
+
+@pytest.mark.parametrize("bad", [
+    dict(d=96), dict(d=32), dict(p=1), dict(L=0), dict(L=9), dict(N=4095),
+    dict(S_=0), dict(S_=4096 + 1024 + 256 + 1), dict(B=0), dict(H=0), dict(N=0),
+    dict(N=16, p=4, L=4),  # p^(L-1) = 64 > N
+])
+def test_validate_rejects_bad_shapes(bad):
+    assert lh.lh_validate(S(**bad), lh.LH_BF16) == lh.LH_ERR_SHAPE
+
+
+def test_validate_rejects_bad_dtype_and_null_shape():
+    assert lh.lh_validate(S(), 7) == lh.LH_ERR_INVALID_ARG
+    f = lh._lib().lh_validate
+    assert f(None, lh.LH_BF16) == lh.LH_ERR_INVALID_ARG
+
+
+def test_num_entries_and_sizes():
+    shp = S(1, 16, 98304, 64, 4, 4, 8192)
+    M = 98304 + 24576 + 6144 + 1536
+    assert lh.lh_num_entries(shp) == M
+    assert lh.lh_num_entries(S(d=96)) == -1
+    saved = lh.lh_saved_bytes(shp)
+    U = 16
+    assert saved >= U * (8192 * 4 * 2 + M * 4 + 4 * 8192 * 64 * 2 + 8192 * 4 + 98304 * 4)
+    offs = [lh.lh_saved_offset(shp, i) for i in range(9)]
+    assert all(o % 256 == 0 for o in offs) and offs == sorted(offs)
+    assert lh.lh_saved_offset(shp, 9) == -1
+    ws_f = lh.lh_workspace_bytes(shp, lh.LH_BF16, False)
+    ws_b = lh.lh_workspace_bytes(shp, lh.LH_BF16, True)
+    assert ws_f >= U * (3 * (M - 98304) * 64 * 4 + M * 4)
+    assert ws_b >= ws_f and ws_b >= U * 8192 * (64 * 2 + 4 + 3 * 64 * 4)
+    assert lh.lh_workspace_bytes(S(d=96), lh.LH_BF16, True) == 0
+    assert lh.lh_topk_workspace_bytes(shp) == 0
+    assert lh.lh_attn_bwd_workspace_bytes(shp) >= U * 8192 * 4
+
+
+def test_bad_arguments_fail_before_any_launch():
+    """Null/misaligned pointers and short workspaces return errors without a GPU."""
+    lib = lh._lib()
+    shp = S()
+    r = lib.lh_forward(ctypes.byref(shp), lh.LH_BF16, None, None, None, 0.0, None, None, None,
+                       0, None)
+    assert r == lh.LH_ERR_INVALID_ARG
+    p = 1 << 20  # a fake, aligned address: never dereferenced because the check fails first
+    r = lib.lh_forward(ctypes.byref(shp), lh.LH_BF16, p, p, p, 0.0, p, p, p, 16, None)
+    assert r == lh.LH_ERR_WORKSPACE
+    r = lib.lh_score(ctypes.byref(shp), lh.LH_BF16, p + 4, p, p, None)
+    assert r == lh.LH_ERR_INVALID_ARG
+    r = lib.lh_subseq_attn_bwd(ctypes.byref(shp), p, p, p, p, p, p, 0.0, p, p, p, p, 0, None)
+    assert r == lh.LH_ERR_WORKSPACE
+    bad = S(d=96)
+    r = lib.lh_gather(ctypes.byref(bad), lh.LH_BF16, p, p, p, p, p, p, p, p, p, p, None)
+    assert r == lh.LH_ERR_SHAPE
+
+
+def test_status_strings():
+    for c in range(7):
+        assert lh.lh_status_string(c).startswith("LH_")
+
+
+def test_attention_impl_switch_roundtrip():
+    prev = lh.lh_set_attention_impl(1)
+    assert lh.lh_set_attention_impl(prev) == 1

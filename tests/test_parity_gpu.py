@@ -1,0 +1,326 @@
+"""CUDA path vs the CPU oracle, stage by stage and fused, through the C ABI.
+
+Tolerances (written here, used everywhere below):
+  * scores, selected index sets, positions, slot map: bit-exact (integer
+    results; both sides compute the scores in fp32 in the same fixed order);
+  * pyramid levels (fp32 on the GPU, fp64 in the oracle): |err| <= 1e-5 |ref|
+    + 1e-6 * rms(level);
+  * gathered rows (fp16): within half an fp16 ulp of the fp64 value;
+  * attention outputs and gradients: |err| <= 2e-2 + 2^-8 |ref| elementwise
+    (2e-2 absolute plus half a bf16 ulp for tensors stored in bf16), and
+    mean|err| / mean|ref| <= 1e-2.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from long_context_lh_b200 import lighthouse as lh
+from long_context_lh_b200.synth import WORKLOADS, make_inputs
+
+pytestmark = pytest.mark.gpu
+DEV = torch.device("cuda:0")
+
+
+def check_attn(got, ref, name):
+    got = np.asarray(got, np.float64)
+    ref = np.asarray(ref, np.float64)
+    err = np.abs(got - ref)
+    bound = 2e-2 + 2.0 ** -8 * np.abs(ref)
+    worst = np.unravel_index(np.argmax(err - bound), err.shape)
+    assert np.all(err <= bound), f"{name}: max err {err.max():.4g} at {worst} ref {ref[worst]:.4g}"
+    scale = np.abs(ref).mean()
+    if scale > 1e-6:  # a reference that is zero in exact arithmetic has no relative error
+        rel = err.mean() / scale
+        assert rel <= 1e-2, f"{name}: mean relative error {rel:.4g}"
+
+
+def check_pyramid(got, ref, name):
+    got = np.asarray(got, np.float64)
+    ref = np.asarray(ref, np.float64)
+    rms = np.sqrt(np.mean(ref ** 2)) if ref.size else 0.0
+    err = np.abs(got - ref)
+    assert np.all(err <= 1e-5 * np.abs(ref) + 1e-6 * rms), f"{name}: max err {err.max():.3g}"
+
+
+def check_gathered(got, ref):
+    """fp16 rounding (half an ulp, <= 2^-11 relative; subnormals below 2^-14 have
+    an absolute half-ulp of 2^-25) of an fp32 value within fp32 rounding of the
+    fp64 pyramid value."""
+    rms = np.sqrt(np.mean(ref ** 2))
+    err = np.abs(got - ref)
+    bound = 2.0 ** -11 * np.abs(ref) + 2.0 ** -25 + 1e-6 * rms
+    assert np.all(err <= bound), f"gather: max err {err.max():.3g}"
+
+
+def f64(t):
+    return t.detach().float().cpu().numpy().astype(np.float64)
+
+
+def to_dev(x):
+    return {k: v.to(DEV) for k, v in x.items()}
+
+
+def workload(name="tiny", **kw):
+    return WORKLOADS[name].with_(**kw)
+
+
+def oshape(w):
+    return oracle.Shape(w.B, w.H, w.N, w.d, w.p, w.L, w.S)
+
+
+def lshape(w):
+    return lh.make_shape(w.B, w.H, w.N, w.d, w.p, w.L, w.S)
+
+
+STAGE_CASES = [
+    dict(),                                                   # tiny: fp32, p=4, L=3, S=512
+    dict(dtype="bf16", dist="outliers"),
+    dict(dtype="bf16", d=128, p=2, L=5, N=2048, S=640),
+    dict(dtype="bf16", p=3, L=3, N=1152, S=200),              # non-power-of-two p, ragged S
+    dict(dtype="bf16", L=1, N=1000, S=333),
+    dict(dtype="bf16", p=2, L=2, N=256, S=384),               # S = M: everything selected
+    dict(dtype="bf16", N=512, S=1),
+]
+
+
+def run_front(w, x):
+    """GPU pyramid, score and selection for inputs x (device tensors)."""
+    shp, dt = lshape(w), lh.dtype_code(x["q"].dtype)
+    M = lh.lh_num_entries(shp)
+    U = w.B * w.H
+    pyr = [torch.zeros((w.B, w.H, max(M - w.N, 1), w.d), dtype=torch.float32, device=DEV)
+           for _ in range(3)]
+    score = torch.zeros((w.B, w.H, M), dtype=torch.float32, device=DEV)
+    lh.lh_build_pyramid(shp, dt, x["q"], x["k"], x["v"], *pyr)
+    lh.lh_score(shp, dt, x["q"], x["k"], score)
+    idx = torch.full((w.B, w.H, w.S), -7, dtype=torch.int32, device=DEV)
+    pos = torch.full_like(idx, -7)
+    slot = torch.full((w.B, w.H, M), -7, dtype=torch.int32, device=DEV)
+    lh.lh_topk_select(shp, score, idx, pos, slot)
+    torch.cuda.synchronize()
+    del U
+    return pyr, score, idx, pos, slot
+
+
+@pytest.mark.parametrize("case", STAGE_CASES, ids=lambda c: ",".join(f"{k}={v}" for k, v in c.items()) or "tiny")
+def test_front_stages_match_oracle(case):
+    w = workload(**case)
+    xc = make_inputs(w, "cpu", with_dO=False)
+    x = to_dev(xc)
+    pyr, score, idx, pos, slot = run_front(w, x)
+    s = oshape(w)
+    qf, kf, vf = (xc[n].float().numpy() for n in ("q", "k", "v"))
+    sc_ref = oracle.score(s, qf, kf)
+    assert np.array_equal(score.cpu().numpy(), sc_ref), "scores differ in some bit"
+    i_ref, p_ref, s_ref = oracle.select(s, sc_ref)
+    assert np.array_equal(idx.cpu().numpy(), i_ref)
+    assert np.array_equal(pos.cpu().numpy(), p_ref)
+    assert np.array_equal(slot.cpu().numpy(), s_ref)
+    if w.L > 1:
+        for t, ref in zip(pyr, (oracle.pyramid(s, a) for a in (qf, kf, vf))):
+            check_pyramid(t.cpu().numpy(), ref, "pyramid")
+
+
+def test_ties_beyond_inheritance_are_broken_by_gid():
+    """Quantised inputs make many equal scores; the radix select on gids must agree."""
+    w = workload(dtype="bf16", N=2048, S=300, H=3)
+    xc = make_inputs(w, "cpu", with_dO=False)
+    for n in ("q", "k"):
+        xc[n] = (xc[n].float() * 0).to(torch.bfloat16)
+        xc[n][..., 0] = torch.randint(0, 3, xc[n].shape[:-1]).to(torch.bfloat16)
+    x = to_dev(xc)
+    _, score, idx, pos, slot = run_front(w, x)
+    s = oshape(w)
+    sc_ref = oracle.score(s, xc["q"].float().numpy(), xc["k"].float().numpy())
+    assert np.array_equal(score.cpu().numpy(), sc_ref)
+    i_ref, p_ref, s_ref = oracle.select(s, sc_ref)
+    assert np.array_equal(idx.cpu().numpy(), i_ref)
+    assert np.array_equal(slot.cpu().numpy(), s_ref)
+
+
+def gpu_gather(w, x, pyr, idx):
+    shp, dt = lshape(w), lh.dtype_code(x["q"].dtype)
+    out = [torch.empty((w.B, w.H, w.S, w.d), dtype=torch.float16, device=DEV) for _ in range(3)]
+    lh.lh_gather(shp, dt, x["q"], x["k"], x["v"], *pyr, idx, *out)
+    return out
+
+
+@pytest.mark.parametrize("case", STAGE_CASES[:4], ids=str)
+def test_gather_and_scatter_match_oracle(case):
+    w = workload(**case)
+    xc = make_inputs(w, "cpu")
+    x = to_dev(xc)
+    pyr, score, idx, pos, slot = run_front(w, x)
+    qs, ks, vs = gpu_gather(w, x, pyr, idx)
+    s = oshape(w)
+    i_ref = idx.cpu().numpy()
+    for t, n in zip((qs, ks, vs), ("q", "k", "v")):
+        a = xc[n].float().numpy()
+        ref = oracle.gather(s, a, oracle.pyramid(s, a), i_ref)
+        check_gathered(f64(t), ref)
+    # scatter-back of arbitrary bf16 rows
+    os_ = torch.randn((w.B, w.H, w.S, w.d), device=DEV).to(torch.float16)
+    o = torch.empty((w.B, w.H, w.N, w.d), dtype=x["q"].dtype, device=DEV)
+    ic = torch.empty((w.B, w.H, w.N), dtype=torch.float32, device=DEV)
+    shp, dt = lshape(w), lh.dtype_code(x["q"].dtype)
+    lh.lh_scatter_back(shp, dt, os_, slot, o, ic)
+    ref = oracle.scatter(s, f64(os_), slot.cpu().numpy())
+    tol = 2.0 ** -8 if w.dtype == "bf16" else 1e-6
+    assert np.all(np.abs(f64(o) - ref) <= tol * np.abs(ref) + 1e-6)  # output-dtype rounding
+    # scatter-back adjoint, with and without the saved counts
+    dO = x["dO"]
+    for use_ic in (True, False):
+        dos = torch.empty((w.B, w.H, w.S, w.d), dtype=torch.float16, device=DEV)
+        lh.lh_scatter_back_bwd(shp, dt, dO, slot, ic if use_ic else None, dos)
+        ref = oracle.scatter_bwd(s, f64(dO), idx.cpu().numpy(), slot.cpu().numpy())
+        got = f64(dos)
+        assert np.all(np.abs(got - ref) <= 2.0 ** -11 * np.abs(ref) + 1e-5 * (1 + np.abs(ref).max()))
+    # gather adjoint
+    d3 = [torch.randn((w.B, w.H, w.S, w.d), device=DEV) for _ in range(3)]
+    dx = [torch.empty((w.B, w.H, w.N, w.d), dtype=x["q"].dtype, device=DEV) for _ in range(3)]
+    lh.lh_gather_bwd(shp, dt, *d3, slot, *dx)
+    for a, b in zip(d3, dx):
+        ref = oracle.gather_bwd(s, f64(a), slot.cpu().numpy())
+        assert np.all(np.abs(f64(b) - ref) <= tol * np.abs(ref) + 1e-6)
+
+
+ATTN_CASES = [(2, 512, 64), (1, 1000, 64), (1, 1, 64), (2, 384, 128), (1, 200, 128)]
+
+
+@pytest.mark.parametrize("impl", [0, 1], ids=["tcgen05", "mma_sync"])
+@pytest.mark.parametrize("U,S,d", ATTN_CASES)
+def test_attention_matches_oracle(U, S, d, impl):
+    prev = lh.lh_set_attention_impl(impl)
+    try:
+        g = torch.Generator().manual_seed(100 + S + d)
+        qs, ks, vs, dos = (torch.randn((1, U, S, d), generator=g).mul(1.5).to(torch.float16)
+                           for _ in range(4))
+        shp = lh.make_shape(1, U, max(S, 1), d, 2, 1, S)
+        qd, kd, vd, dod = (t.to(DEV) for t in (qs, ks, vs, dos))
+        os_ = torch.empty_like(qd)
+        lse = torch.empty((1, U, S), dtype=torch.float32, device=DEV)
+        lh.lh_subseq_attn_fwd(shp, qd, kd, vd, 0.0, os_, lse)
+        s = oracle.Shape(1, U, max(S, 1), d, 2, 1, S)
+        sc = 1.0 / np.sqrt(d)
+        o_ref, lse_ref = oracle.attn_fwd(s, f64(qs), f64(ks), f64(vs), sc)
+        check_attn(f64(os_), o_ref, "os")
+        assert np.abs(f64(lse) - lse_ref).max() < 2e-2
+        dq, dk, dv = (torch.empty((1, U, S, d), dtype=torch.float32, device=DEV) for _ in range(3))
+        wsb = lh.lh_attn_bwd_workspace_bytes(shp)
+        ws = torch.empty(wsb, dtype=torch.uint8, device=DEV)
+        lh.lh_subseq_attn_bwd(shp, qd, kd, vd, os_, lse, dod, 0.0, dq, dk, dv, ws, wsb)
+        refs = oracle.attn_bwd(s, f64(qs), f64(ks), f64(vs), f64(dos), sc)
+        for name, got, ref in zip(("dqs", "dks", "dvs"), (dq, dk, dv), refs):
+            check_attn(f64(got), ref, name)
+        assert lh.lh_read_device_status() == 0
+    finally:
+        lh.lh_set_attention_impl(prev)
+
+
+@pytest.mark.parametrize("case", [dict(), dict(dtype="bf16", dist="outliers", N=8192, S=1024, L=4),
+                                  dict(dtype="bf16", d=128, p=2, L=4, N=2048, S=500)], ids=str)
+def test_fused_forward_backward_match_oracle(case):
+    w = workload(**case)
+    xc = make_inputs(w, "cpu")
+    x = to_dev(xc)
+    o, saved = lh.forward(x["q"], x["k"], x["v"], w.p, w.L, w.S)
+    dq, dk, dv = lh.backward(saved, x["dO"])
+    torch.cuda.synchronize()
+    s = oshape(w)
+    f = [xc[n].float().numpy() for n in ("q", "k", "v", "dO")]
+    ref = oracle.forward(s, *f[:3])
+    sv = lambda which: lh.saved_view(saved.shape, saved.buf, which).cpu().numpy()
+    assert np.array_equal(sv(lh.SAVED_IDX), ref["idx"])
+    assert np.array_equal(sv(lh.SAVED_POS), ref["pos"])
+    assert np.array_equal(sv(lh.SAVED_SLOT), ref["slot"])
+    check_attn(f64(o), ref["o"], "o")
+    bref = oracle.backward(s, ref, f[3])
+    for name, t in (("dq", dq), ("dk", dk), ("dv", dv)):
+        check_attn(f64(t), bref[name], name)
+
+
+def test_degenerate_L1_full_selection_equals_causal_sdpa():
+    w = workload(dtype="bf16", L=1, N=512, S=512, H=2)
+    xc = make_inputs(w, "cpu")
+    x = to_dev(xc)
+    o, saved = lh.forward(x["q"], x["k"], x["v"], w.p, w.L, w.S)
+    assert torch.equal(lh.saved_view(saved.shape, saved.buf, lh.SAVED_IDX)[0, 0].cpu(),
+                       torch.arange(512, dtype=torch.int32))
+    ref = torch.nn.functional.scaled_dot_product_attention(
+        *(xc[n].double() for n in ("q", "k", "v")), is_causal=True)
+    check_attn(f64(o), ref.numpy(), "o")
+
+
+def test_bitwise_deterministic():
+    w = workload(dtype="bf16", dist="outliers", N=8192, S=1024, L=4, H=4)
+    x = to_dev(make_inputs(w, "cpu"))
+    outs = []
+    for _ in range(2):
+        o, saved = lh.forward(x["q"], x["k"], x["v"], w.p, w.L, w.S)
+        grads = lh.backward(saved, x["dO"])
+        outs.append([o.clone(), saved.buf.clone(), *[g.clone() for g in grads]])
+    for a, b in zip(*outs):
+        assert torch.equal(a, b)
+
+
+def test_pretraining_shape_full_size():
+    """The benchmark's workload (H=16, N=98,304, S=8192) in the launch the bench times.
+
+    Every head: scores and the selection bit-exact.  Heads 0 and H-1: pyramid,
+    gathered rows, 64 sampled attention rows and the tokens they scatter to;
+    head 0: the full attention backward."""
+    w = WORKLOADS["pretrain"]
+    xc = make_inputs(w, "cpu")
+    x = to_dev(xc)
+    o, saved = lh.forward(x["q"], x["k"], x["v"], w.p, w.L, w.S)
+    dq, dk, dv = lh.backward(saved, x["dO"])
+    torch.cuda.synchronize()
+    s = oshape(w)
+    qf, kf = xc["q"].float().numpy(), xc["k"].float().numpy()
+    sc_ref = oracle.score(s, qf, kf)
+    i_ref, p_ref, s_ref = oracle.select(s, sc_ref)
+    sv = lambda which: lh.saved_view(saved.shape, saved.buf, which)
+    assert np.array_equal(sv(lh.SAVED_IDX).cpu().numpy(), i_ref)
+    assert np.array_equal(sv(lh.SAVED_SLOT).cpu().numpy(), s_ref)
+    rng = np.random.default_rng(7)
+    for h in (0, w.H - 1):
+        s1 = s.unit()
+        xs = []
+        for n in ("q", "k", "v"):
+            a = xc[n][:, h:h + 1].float().numpy()
+            xs.append(oracle.gather(s1, a, oracle.pyramid(s1, a), i_ref[:, h:h + 1]))
+        for ref, which in zip(xs, (lh.SAVED_QS, lh.SAVED_KS, lh.SAVED_VS)):
+            check_gathered(f64(sv(which)[:, h:h + 1]), ref)
+        rows = np.sort(rng.choice(w.S, 64, replace=False)).astype(np.int32)
+        os_ref, lse_ref = oracle.attn_fwd(s1, *xs, 1.0 / np.sqrt(w.d), rows=rows)
+        check_attn(f64(sv(lh.SAVED_OS)[:, h:h + 1, rows]), os_ref, f"os head {h}")
+        # tokens whose contributors are all among the sampled rows
+        slot_h = s_ref[0, h]
+        os_full = np.full((w.S, w.d), np.nan)
+        os_full[rows] = os_ref[0, 0]
+        toks = rng.choice(w.N, 4096, replace=False)
+        got_o = f64(o[0, h])
+        checked = 0
+        for t in toks:
+            sl = [slot_h[s.level_off(l) + t // w.p ** l] for l in range(w.L)]
+            sl = [z for z in sl if z >= 0]
+            if not sl or not all(z in set(rows.tolist()) for z in sl):
+                continue
+            ref_t = np.mean([os_full[z] for z in sl], axis=0)
+            check_attn(got_o[t][None], ref_t[None], f"o token {t}")
+            checked += 1
+        assert checked > 0
+    # full attention backward of head 0 on the GPU's own bf16 operands
+    s1 = s.unit()
+    dos_gpu = torch.empty((1, 1, w.S, w.d), dtype=torch.float16, device=DEV)
+    lh.lh_scatter_back_bwd(lh.make_shape(1, 1, w.N, w.d, w.p, w.L, w.S), lh.LH_BF16,
+                           x["dO"][:, :1].contiguous(), sv(lh.SAVED_SLOT)[:, :1].contiguous(),
+                           sv(lh.SAVED_INV_COUNT)[:, :1].contiguous(), dos_gpu)
+    ops = [f64(sv(which)[:, :1]) for which in (lh.SAVED_QS, lh.SAVED_KS, lh.SAVED_VS)]
+    dos_ref = oracle.scatter_bwd(s1, xc["dO"][:, :1].float().numpy(), i_ref[:, :1], s_ref[:, :1])
+    check_attn(f64(dos_gpu), dos_ref, "dos head 0")
+    refs = oracle.attn_bwd(s1, *ops, f64(dos_gpu), 1.0 / np.sqrt(w.d))
+    dref = [oracle.gather_bwd(s1, r, s_ref[:, :1]) for r in refs]
+    for name, t, r in zip(("dq", "dk", "dv"), (dq, dk, dv), dref):
+        check_attn(f64(t[:, :1]), r, f"{name} head 0")
