@@ -163,6 +163,26 @@ lh_status lh_subseq_attn_bwd(const lh_shape* shape, const void* qs, const void* 
                              float scale, float* dqs, float* dks, float* dvs, void* ws,
                              size_t ws_bytes, lh_stream_t stream);
 
+/* (e'') The same backward as lh_subseq_attn_bwd, for callers that cannot
+ * allocate device memory or hand over a workspace -- for example code that runs
+ * under a memory planner which has already reserved every byte of the GPU, or
+ * a runtime where calling cudaMalloc mid-step is not allowed because it can
+ * synchronise the device.  The paper has no counterpart: this is a library
+ * convenience, not part of the method.  It allocates nothing: its scratch (one
+ * fp32 per row, the D vector) is a fixed 4 MiB array inside the library that
+ * every GPU loading the library holds until the process exits.
+ *   - At most 1,048,576 rows (B * H * S); larger shapes return
+ *     LH_ERR_WORKSPACE before anything is enqueued.
+ *   - All calls on one device share that array: calls whose kernels overlap on
+ *     the GPU (unordered streams) race; calls ordered on one stream are safe.
+ *   - The first call on each device looks up the array's device address and
+ *     caches it; make that first call before any stream capture.
+ * Arguments and results as for lh_subseq_attn_bwd, without ws / ws_bytes.  */
+lh_status lh_subseq_attn_bwd_noalloc(const lh_shape* shape, const void* qs, const void* ks,
+                                     const void* vs, const void* os, const float* lse,
+                                     const void* dos, float scale, float* dqs, float* dks,
+                                     float* dvs, lh_stream_t stream);
+
 /* (f) Scatter-back, [ES] §2.C / [PT] phase 4: c_t = number of selected
  * entries covering t; O[t] = (sum over them, ascending level, of os[slot]) / c_t,
  * 0 when c_t = 0.  o: [B,H,N,d] dtype.  inv_count (optional, may be NULL):

@@ -68,6 +68,8 @@ _SIGS = {
     "lh_attn_bwd_workspace_bytes": ([_SP], _SZ),
     "lh_subseq_attn_bwd": ([_SP, _VP, _VP, _VP, _VP, _VP, _VP, _F, _VP, _VP, _VP, _VP, _SZ,
                             _VP], _I),
+    "lh_subseq_attn_bwd_noalloc": ([_SP, _VP, _VP, _VP, _VP, _VP, _VP, _F, _VP, _VP, _VP,
+                                    _VP], _I),
     "lh_scatter_back": ([_SP, _I, _VP, _VP, _VP, _VP, _VP], _I),
     "lh_scatter_back_bwd": ([_SP, _I, _VP, _VP, _VP, _VP, _VP], _I),
     "lh_gather_bwd": ([_SP, _I, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP], _I),
@@ -223,6 +225,13 @@ def lh_subseq_attn_bwd(shape, qs, ks, vs, os_, lse, dos, scale, dqs, dks, dvs, w
     _check("lh_subseq_attn_bwd", _lib().lh_subseq_attn_bwd(
         ctypes.byref(shape), _p(qs), _p(ks), _p(vs), _p(os_), _p(lse), _p(dos), float(scale),
         _p(dqs), _p(dks), _p(dvs), _p(ws), ws_bytes, _st(stream)))
+
+
+def lh_subseq_attn_bwd_noalloc(shape, qs, ks, vs, os_, lse, dos, scale, dqs, dks, dvs,
+                               stream=None):
+    _check("lh_subseq_attn_bwd_noalloc", _lib().lh_subseq_attn_bwd_noalloc(
+        ctypes.byref(shape), _p(qs), _p(ks), _p(vs), _p(os_), _p(lse), _p(dos), float(scale),
+        _p(dqs), _p(dks), _p(dvs), _st(stream)))
 
 
 def lh_scatter_back(shape, dtype, os_, slot, o, inv_count=None, stream=None):

@@ -1,0 +1,57 @@
+"""lh_subseq_attn_bwd_noalloc: the attention backward without caller memory.
+
+Some callers cannot allocate device memory or pass a workspace (a memory
+planner owns every byte, or cudaMalloc is off limits mid-step because it can
+synchronise the device).  This entry point keeps its scratch in a fixed array
+inside the library instead.  The GPU test calls it through the C ABI twice in
+a row and checks both results against lh_subseq_attn_bwd, with the tolerance
+the other parity tests use.  This file is collected last on purpose.
+"""
+import ctypes
+
+import numpy as np
+import pytest
+import torch
+
+from long_context_lh_b200 import lighthouse as lh
+
+
+def check_close(got, ref, name):
+    got = got.double().cpu().numpy()
+    ref = ref.double().cpu().numpy()
+    err = np.abs(got - ref)
+    assert np.all(err <= 2e-2 + 2.0 ** -8 * np.abs(ref)), f"{name}: max err {err.max():.3g}"
+    scale = np.abs(ref).mean()
+    if scale > 1e-6:
+        assert err.mean() / scale <= 1e-2, name
+
+
+def test_noalloc_rejects_shapes_beyond_its_scratch():
+    lib = lh._lib()
+    shp = lh.make_shape(1, 256, 8192, 64, 2, 1, 8192)  # 2,097,152 rows > 1,048,576
+    p = 1 << 20  # aligned fake address, never dereferenced: the size check comes first
+    r = lib.lh_subseq_attn_bwd_noalloc(ctypes.byref(shp), p, p, p, p, p, p, 0.0, p, p, p, None)
+    assert r == lh.LH_ERR_WORKSPACE
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("U,S,d", [(16, 1024, 64), (3, 777, 128)])
+def test_noalloc_matches_workspace_entry_point_twice(U, S, d):
+    dev = torch.device("cuda:0")
+    g = torch.Generator(device=dev).manual_seed(4242 + S)
+    qs, ks, vs, dos = (torch.randn((1, U, S, d), generator=g, device=dev).to(torch.float16)
+                       for _ in range(4))
+    shp = lh.make_shape(1, U, S, d, 2, 1, S)
+    os_ = torch.empty_like(qs)
+    lse = torch.empty((1, U, S), dtype=torch.float32, device=dev)
+    lh.lh_subseq_attn_fwd(shp, qs, ks, vs, 0.0, os_, lse)
+    ref = [torch.empty((1, U, S, d), dtype=torch.float32, device=dev) for _ in range(3)]
+    wsb = lh.lh_attn_bwd_workspace_bytes(shp)
+    ws = torch.empty(wsb, dtype=torch.uint8, device=dev)
+    lh.lh_subseq_attn_bwd(shp, qs, ks, vs, os_, lse, dos, 0.0, *ref, ws, wsb)
+    for call in range(2):
+        got = [torch.full((1, U, S, d), float("nan"), device=dev) for _ in range(3)]
+        lh.lh_subseq_attn_bwd_noalloc(shp, qs, ks, vs, os_, lse, dos, 0.0, *got)
+        torch.cuda.synchronize()
+        for name, a, b in zip(("dqs", "dks", "dvs"), got, ref):
+            check_close(a, b, f"call {call} {name}")
