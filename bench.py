@@ -131,6 +131,8 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
     w = WORKLOADS[args.workload]
+    if args.heads:
+        w = w.with_(H=args.heads)
     if args.attn == "mma":
         lh.lh_set_attention_impl(1)
     elif args.attn == "tc":
@@ -275,7 +277,7 @@ def run_ours(args, rank, world, local_rank):
         dense = dense_sdpa(w, q, k, v, dO, stream, args)
 
     # end to end through the public API with pinned host buffers
-    e2e = e2e_run(lh, w, shp, dt, x, dev, stream, args, dist)
+    e2e = None if args.no_e2e else e2e_run(lh, w, shp, dt, x, dev, stream, args, dist)
     launches = launches_per_step(lh, w)
     out = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
@@ -285,7 +287,7 @@ def run_ours(args, rank, world, local_rank):
         "config": {"workload": f"{w.name}: B={w.B} H={w.H} N={w.N} d={w.d} p={w.p} L={w.L} S={w.S} {w.dtype}",
                    "B": w.B, "H": w.H, "N": w.N, "d": w.d, "p": w.p, "L": w.L, "S": w.S,
                    "l2": "inputs larger than L2 (3 x %.0f MB + dO), no flush" % (w.B * w.H * w.N * w.d * 2 / 1e6),
-                   "attention": "tcgen05" if lh.lh_attention_impl_in_use() == 0 else "mma_sync",
+                   "attention": {0: "tcgen05", 1: "mma_sync", 2: "tcgen05 fwd, mma_sync bwd"}[lh.lh_attention_impl_in_use()],
                    "parallelism": f"replicas x{world} (heads independent)"},
         "fwd_tokens_per_s": world * tokens / (ms_fwd / 1e3), "ms_fwd": ms_fwd,
         "roofline": roof, "stages": stage_report, "dense_sdpa": dense, "e2e": e2e,
@@ -450,6 +452,9 @@ def main():
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--no-dense", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=20.0)
+    ap.add_argument("--heads", type=int, default=0,
+                    help="override H (smaller cases for profiler captures; not a bench line)")
+    ap.add_argument("--no-e2e", action="store_true")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3) if args.impl == "ours" else args.warmup
     world = int(os.environ.get("WORLD_SIZE", "1"))

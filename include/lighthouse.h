@@ -227,7 +227,9 @@ lh_status lh_read_device_status(lh_stream_t stream, uint32_t* code);
  * as the comparison baseline).  Returns the previous value. */
 int lh_set_attention_impl(int impl);
 
-/* The attention implementation the next call would use: 0 tcgen05, 1 mma.sync. */
+/* The attention implementations the next calls would use: 0 tcgen05 for the
+ * forward and the backward, 1 mma.sync for both, 2 tcgen05 forward with the
+ * mma.sync backward. */
 int lh_attention_impl_in_use(void);
 
 /* Number of kernel launches lh_forward (backward = 0) or lh_backward

@@ -112,6 +112,13 @@ bool use_tc() {
   return attn_tc_available();
 }
 
+}  // namespace
+
+bool attn_fwd_uses_tc() { return use_tc(); }
+bool attn_bwd_uses_tc() { return use_tc() && attn_tc_bwd_available(); }
+
+namespace {
+
 inline lh_status cuda_status(cudaError_t e) { return e == cudaSuccess ? LH_OK : LH_ERR_CUDA; }
 
 #define LH_TRY(expr)                           \
@@ -127,7 +134,7 @@ float resolve_scale(const Geom& g, float scale) {
 lh_status attn_fwd(const Geom& g, const __half* qs, const __half* ks,
                    const __half* vs, float scale, __half* os, float* lse,
                    cudaStream_t st) {
-  if (use_tc()) return cuda_status(launch_attn_fwd_tc(g, qs, ks, vs, scale, os, lse, st));
+  if (attn_fwd_uses_tc()) return cuda_status(launch_attn_fwd_tc(g, qs, ks, vs, scale, os, lse, st));
   return cuda_status(launch_attn_fwd_mma(g, qs, ks, vs, scale, os, lse, st));
 }
 
@@ -136,7 +143,7 @@ lh_status attn_bwd(const Geom& g, const __half* qs, const __half* ks,
                    const __half* dos, float scale, float* dqs, float* dks, float* dvs,
                    float* Dvec, cudaStream_t st) {
   LH_TRY(launch_attn_rowdot(g, os, dos, Dvec, st));
-  if (use_tc())
+  if (attn_bwd_uses_tc())
     return cuda_status(launch_attn_bwd_tc(g, qs, ks, vs, dos, lse, Dvec, scale, dqs, dks, dvs, st));
   return cuda_status(launch_attn_bwd_mma(g, qs, ks, vs, dos, lse, Dvec, scale, dqs, dks, dvs, st));
 }
@@ -410,19 +417,21 @@ int lh_set_attention_impl(int impl) {
   return g_attn_impl.exchange(impl);
 }
 
-int lh_attention_impl_in_use(void) { return use_tc() ? 0 : 1; }
+int lh_attention_impl_in_use(void) {
+  const bool f = attn_fwd_uses_tc(), b = attn_bwd_uses_tc();
+  return f && b ? 0 : (!f && !b ? 1 : 2);
+}
 
 int lh_kernel_launches(const lh_shape* shape, int backward) {
   if (check_shape(shape) != LH_OK) return -1;
   const Geom g = make_geom(*shape);
   const int chunks = (int)((g.U + 65534) / 65535);  // grid.y limit per launch
-  const bool tc = use_tc();
   if (!backward) {
     // pyramid+score, top-k (per chunk), gather, attention (per chunk), scatter
-    return 1 + chunks + 1 + (tc ? attn_tc_fwd_launches(g) : chunks) + 1;
+    return 1 + chunks + 1 + (attn_fwd_uses_tc() ? attn_tc_fwd_launches(g) : chunks) + 1;
   }
   // scatter-back bwd, row dot, attention bwd, gather bwd
-  return 1 + 1 + (tc ? attn_tc_bwd_launches(g) : 2 * chunks) + 1;
+  return 1 + 1 + (attn_bwd_uses_tc() ? attn_tc_bwd_launches(g) : 2 * chunks) + 1;
 }
 
 }  // extern "C"

@@ -169,7 +169,10 @@ cudaError_t launch_attn_bwd_tc(const Geom& g, const __half* qs, const __half* ks
                                const __half* vs, const __half* dos,
                                const float* lse, const float* D, float scale, float* dqs,
                                float* dks, float* dvs, cudaStream_t st);
-bool attn_tc_available();
+bool attn_tc_available();      // tcgen05 forward can run on this device
+bool attn_tc_bwd_available();  // tcgen05 backward can run on this device
+bool attn_fwd_uses_tc();       // dispatch decisions (lh_set_attention_impl + availability)
+bool attn_bwd_uses_tc();
 int attn_tc_fwd_launches(const Geom& g);
 int attn_tc_bwd_launches(const Geom& g);
 

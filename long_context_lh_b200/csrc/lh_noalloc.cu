@@ -75,7 +75,7 @@ extern "C" lh_status lh_subseq_attn_bwd_noalloc(const lh_shape* shape, const voi
   auto* o = static_cast<const __half*>(os);
   auto* go = static_cast<const __half*>(dos);
   if (launch_attn_rowdot(g, o, go, Dvec, stream) != cudaSuccess) return LH_ERR_CUDA;
-  cudaError_t e = lh_attention_impl_in_use() == 0
+  cudaError_t e = attn_bwd_uses_tc()
                       ? launch_attn_bwd_tc(g, q, k, v, go, lse, Dvec, sc, dqs, dks, dvs, stream)
                       : launch_attn_bwd_mma(g, q, k, v, go, lse, Dvec, sc, dqs, dks, dvs, stream);
   return e == cudaSuccess ? LH_OK : LH_ERR_CUDA;
