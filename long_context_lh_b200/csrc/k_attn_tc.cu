@@ -184,7 +184,7 @@ __global__ void __launch_bounds__(kFwdThreads, (D == 64) ? 2 : 1)
     float m = -INFINITY, l = 0.0f, alpha_prev = 0.0f;
     bool ok = true;
     for (int j = 0; j < nkv; ++j) {
-      ok = mbar_wait(&bars->s_full, j & 1, abort, kStatus);
+      ok = warp_wait(&bars->s_full, j & 1, abort, kStatus);
       if (!ok) break;
       tc_fence_after();
       const bool diag = (j == qt);
@@ -205,7 +205,7 @@ __global__ void __launch_bounds__(kFwdThreads, (D == 64) ? 2 : 1)
       const float alpha = ex2(m - m_new);
       // fold P V of the previous tile into O (also frees the P buffer)
       if (j > 0) {
-        ok = mbar_wait(&bars->pv_done, (j - 1) & 1, abort, kStatus);
+        ok = warp_wait(&bars->pv_done, (j - 1) & 1, abort, kStatus);
         if (!ok) break;
         tc_fence_after();
 #pragma unroll
@@ -252,8 +252,8 @@ __global__ void __launch_bounds__(kFwdThreads, (D == 64) ? 2 : 1)
       m = m_new;
       alpha_prev = alpha;
     }
-    if (ok) ok = mbar_wait(&bars->pv_done, (nkv - 1) & 1, abort, kStatus);
-    if (ok) {
+    if (ok) ok = warp_wait(&bars->pv_done, (nkv - 1) & 1, abort, kStatus);
+    if (ok) {  // whole warps: the TMEM loads below are warp-collective
       tc_fence_after();
 #pragma unroll
       for (int h = 0; h < D / 32; ++h) {
@@ -285,6 +285,501 @@ __global__ void __launch_bounds__(kFwdThreads, (D == 64) ? 2 : 1)
   if (warp == 5) {
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+// ========================================================= backward: dK, dV
+// One CTA per (unit, 128-key tile kt); it walks the query tiles i >= kt.
+//   warp 4: TMA for K, V once and a ring of (Q_i, dO_i) tiles; its 32 lanes also
+//           stage lse_i * log2(e) and D_i of the 128 queries in shared memory;
+//   warp 5: MMA issuer: S^T = K Q_i^T and dP^T = V dO_i^T (TMEM, 128 columns
+//           each), then dV += P^T dO_i and dK += dS^T Q_i (TMEM, d columns each);
+//   warps 0-3: one key row each: P^T = 2^(S^T c - lse2) (zero where the query
+//           precedes the key), dS^T = P^T (dP^T - D), both to fp16 in swizzled
+//           shared memory as the A operands of the two accumulating products.
+// dK and dV never leave TMEM until the last tile: no atomics, fixed order.
+struct DkvBars {
+  uint64_t kv_full;
+  uint64_t q_full[2], q_empty[2];
+  uint64_t s_full, st_free, p_full, pdone, mma_done;
+  uint32_t tmem;
+  int abort;
+};
+
+template <int D>
+struct DkvLayout {
+  static constexpr int kStages = (D == 64) ? 2 : 1;
+  static constexpr int kTile = 128 * D * 2;
+  static constexpr int kK = 0;
+  static constexpr int kV = kK + kTile;
+  static constexpr int kQ = kV + kTile;                 // kStages
+  static constexpr int kDO = kQ + kStages * kTile;      // kStages
+  static constexpr int kPT = kDO + kStages * kTile;     // 128 x 128 fp16
+  static constexpr int kDST = kPT + 32768;              // 128 x 128 fp16
+  static constexpr int kLse = kDST + 32768;             // kStages x 128 fp32
+  static constexpr int kDv = kLse + kStages * 512;      // kStages x 128 fp32
+  static constexpr int kBar = kDv + kStages * 512;
+  static constexpr int kBytes = kBar + (int)sizeof(DkvBars);
+};
+
+template <int D>
+__global__ void __launch_bounds__(kFwdThreads, 1)
+    k_attn_bwd_dkdv_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
+                       const __grid_constant__ CUtensorMap tv, const __grid_constant__ CUtensorMap tdo,
+                       const float* __restrict__ lse, const float* __restrict__ Dv,
+                       float* __restrict__ dks, float* __restrict__ dvs, int S, int unit0,
+                       float scale, float scale_log2, int ntiles) {
+  using Lt = DkvLayout<D>;
+  constexpr int STG = Lt::kStages;
+  extern __shared__ __align__(1024) uint8_t smem[];
+  if (smem_u32(smem) & 1023u) {
+    if (threadIdx.x == 0) report_status(kStatusAttnBwdTimeout | 1u);
+    return;
+  }
+  DkvBars* bars = reinterpret_cast<DkvBars*>(smem + Lt::kBar);
+  uint8_t* sK = smem + Lt::kK;
+  uint8_t* sV = smem + Lt::kV;
+  uint8_t* sQ = smem + Lt::kQ;
+  uint8_t* sDO = smem + Lt::kDO;
+  uint8_t* sPT = smem + Lt::kPT;
+  uint8_t* sDST = smem + Lt::kDST;
+  float* sLse = reinterpret_cast<float*>(smem + Lt::kLse);
+  float* sDv = reinterpret_cast<float*>(smem + Lt::kDv);
+  volatile int* abort = &bars->abort;
+  constexpr uint32_t kStatus = kStatusAttnBwdTimeout;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int kt = (int)blockIdx.x;  // kt = 0 has the most query tiles: it starts first
+  const int u = unit0 + (int)blockIdx.y;
+  const int n = ntiles - kt;       // query tiles kt .. ntiles-1
+
+  if (threadIdx.x == 0) {
+    mbar_init(&bars->kv_full, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&bars->q_full[i], 33);
+      mbar_init(&bars->q_empty[i], 1);
+    }
+    mbar_init(&bars->s_full, 1);
+    mbar_init(&bars->st_free, 4);
+    mbar_init(&bars->p_full, 4);
+    mbar_init(&bars->pdone, 1);
+    mbar_init(&bars->mma_done, 1);
+    bars->abort = 0;
+    mbar_init_fence();
+  }
+  if (warp == 5) tmem_alloc(&bars->tmem, 512);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = bars->tmem;
+  const uint32_t tST = tmem, tDPT = tmem + 128, tDV = tmem + 256, tDK = tmem + 256 + D;
+
+  if (warp == 4) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      mbar_expect_tx(&bars->kv_full, 2 * Lt::kTile);
+      for (int h = 0; h < D / 64; ++h) {
+        tma_load_3d(sK + h * 16384, &tk, &bars->kv_full, h * 64, kt * 128, u);
+        tma_load_3d(sV + h * 16384, &tv, &bars->kv_full, h * 64, kt * 128, u);
+      }
+    }
+    int issued = 0;
+    for (int t = 0; t < n; ++t) {
+      const int st = t % STG, i = kt + t;
+      if (t >= STG && !warp_wait(&bars->q_empty[st], ((t - STG) / STG) & 1, abort, kStatus)) break;
+      if (lane == 0) {
+        mbar_expect_tx(&bars->q_full[st], 2 * Lt::kTile);
+        for (int h = 0; h < D / 64; ++h) {
+          tma_load_3d(sQ + st * Lt::kTile + h * 16384, &tq, &bars->q_full[st], h * 64, i * 128, u);
+          tma_load_3d(sDO + st * Lt::kTile + h * 16384, &tdo, &bars->q_full[st], h * 64, i * 128, u);
+        }
+      }
+      for (int c = lane; c < 128; c += 32) {
+        const int q = i * 128 + c;
+        const bool in = q < S;
+        // padded queries: lse2 = +inf makes their P^T (and dS^T) exactly zero
+        sLse[st * 128 + c] = in ? __ldg(lse + (int64_t)u * S + q) * kLog2e : INFINITY;
+        sDv[st * 128 + c] = in ? __ldg(Dv + (int64_t)u * S + q) : 0.0f;
+      }
+      mbar_arrive(&bars->q_full[st]);
+      issued = t + 1;
+    }
+    if (lane == 0) {
+      mbar_wait(&bars->kv_full, 0, abort, kStatus, false);
+      for (int t = (issued > STG ? issued - STG : 0); t < issued; ++t)
+        mbar_wait(&bars->q_full[t % STG], (t / STG) & 1, abort, kStatus, false);
+    }
+  } else if (warp == 5) {
+    // -------------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idS = idesc_f16(128, 128, false);
+      constexpr uint32_t idAcc = idesc_f16(128, D, true);
+      const uint32_t aK = smem_u32(sK), aV = smem_u32(sV), aQ = smem_u32(sQ), aDO = smem_u32(sDO);
+      const uint32_t aPT = smem_u32(sPT), aDST = smem_u32(sDST);
+      auto issue_grads = [&](int t) {  // dV += P^T dO_t, dK += dS^T Q_t
+        const int st = t % STG;
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t a = (kk >> 2) * 16384 + (kk & 3) * 32;
+          const uint32_t b = st * Lt::kTile + kk * 2048;
+          umma_f16(tDV, desc_kmajor(aPT + a), desc_mnmajor(aDO + b, 16384), idAcc, (t > 0 || kk > 0));
+          umma_f16(tDK, desc_kmajor(aDST + a), desc_mnmajor(aQ + b, 16384), idAcc, (t > 0 || kk > 0));
+        }
+        umma_commit(&bars->pdone);
+        umma_commit(&bars->q_empty[st]);
+      };
+      bool ok = mbar_wait(&bars->kv_full, 0, abort, kStatus);
+      for (int t = 0; ok && t < n; ++t) {
+        const int st = t % STG;
+        // with one (Q, dO) stage the previous tile's products must finish before
+        // the producer can bring the next tile into it
+        if (STG == 1 && t > 0) {
+          ok = mbar_wait(&bars->p_full, (t - 1) & 1, abort, kStatus);
+          if (!ok) break;
+          tc_fence_after();
+          issue_grads(t - 1);
+        }
+        ok = mbar_wait(&bars->q_full[st], (t / STG) & 1, abort, kStatus) &&
+             (t == 0 || mbar_wait(&bars->st_free, (t - 1) & 1, abort, kStatus));
+        if (!ok) break;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+          umma_f16(tST, desc_kmajor(aK + off), desc_kmajor(aQ + st * Lt::kTile + off), idS, kk > 0);
+          umma_f16(tDPT, desc_kmajor(aV + off), desc_kmajor(aDO + st * Lt::kTile + off), idS, kk > 0);
+        }
+        umma_commit(&bars->s_full);
+        if (STG > 1 && t > 0) {
+          ok = mbar_wait(&bars->p_full, (t - 1) & 1, abort, kStatus);
+          if (!ok) break;
+          tc_fence_after();
+          issue_grads(t - 1);
+        }
+      }
+      if (ok && mbar_wait(&bars->p_full, (n - 1) & 1, abort, kStatus)) {
+        tc_fence_after();
+        issue_grads(n - 1);
+      }
+      umma_commit(&bars->mma_done);
+      mbar_wait(&bars->mma_done, 0, abort, kStatus, false);
+    }
+  } else {
+    // ------------------------------------------------------- one key row per thread
+    const int r = threadIdx.x;
+    const uint32_t lane_addr = (uint32_t)(warp * 32) << 16;
+    bool ok = true;
+    for (int t = 0; t < n; ++t) {
+      const int st = t % STG;
+      ok = warp_wait(&bars->q_full[st], (t / STG) & 1, abort, kStatus) &&
+           warp_wait(&bars->s_full, t & 1, abort, kStatus);
+      if (!ok) break;
+      tc_fence_after();
+      const bool diag = (t == 0);
+      const float* cl = sLse + st * 128;
+      const float* cd = sDv + st * 128;
+#pragma unroll
+      for (int ch = 0; ch < 4; ++ch) {
+        uint32_t a[32], b[32];
+        tmem_ld32(tST + lane_addr + ch * 32, a);
+        tmem_ld32(tDPT + lane_addr + ch * 32, b);
+        tmem_ld_wait();
+        if (ch == 3) {  // S^T and dP^T of this tile are in registers: TMEM may be overwritten
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&bars->st_free);
+        }
+        uint32_t pp[16], pd[16];
+#pragma unroll
+        for (int e = 0; e < 32; e += 2) {
+          const int q = ch * 32 + e;
+          const float2 l2 = *reinterpret_cast<const float2*>(cl + q);
+          const float2 dd = *reinterpret_cast<const float2*>(cd + q);
+          float p0 = ex2(fmaf(__uint_as_float(a[e]), scale_log2, -l2.x));
+          float p1 = ex2(fmaf(__uint_as_float(a[e + 1]), scale_log2, -l2.y));
+          if (diag && q < r) p0 = 0.0f;
+          if (diag && q + 1 < r) p1 = 0.0f;
+          const float d0 = p0 * (__uint_as_float(b[e]) - dd.x);
+          const float d1 = p1 * (__uint_as_float(b[e + 1]) - dd.y);
+          pp[e >> 1] = pack_h2(p0, p1);
+          pd[e >> 1] = pack_h2_sat(d0, d1);
+        }
+        // the previous tile's products must be done reading the P^T / dS^T buffers
+        if (ch == 0 && t > 0 && !(ok = warp_wait(&bars->pdone, (t - 1) & 1, abort, kStatus))) break;
+#pragma unroll
+        for (int qd = 0; qd < 4; ++qd) {
+          const int c = ch * 4 + qd;  // 16-byte chunk of the 128-column row
+          const uint32_t off = (c >> 3) * 16384 + swz(r, c & 7);
+          *reinterpret_cast<uint4*>(sPT + off) =
+              make_uint4(pp[4 * qd], pp[4 * qd + 1], pp[4 * qd + 2], pp[4 * qd + 3]);
+          *reinterpret_cast<uint4*>(sDST + off) =
+              make_uint4(pd[4 * qd], pd[4 * qd + 1], pd[4 * qd + 2], pd[4 * qd + 3]);
+        }
+      }
+      if (!ok) break;
+      fence_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars->p_full);
+    }
+    if (ok) ok = warp_wait(&bars->pdone, (n - 1) & 1, abort, kStatus);
+    const int row = kt * 128 + r;
+    if (ok) {  // whole warps load TMEM; only rows inside the sequence are stored
+      tc_fence_after();
+      float* gv = dvs + ((int64_t)u * S + row) * D;
+      float* gk = dks + ((int64_t)u * S + row) * D;
+      const bool in = row < S;
+#pragma unroll
+      for (int h = 0; h < D / 32; ++h) {
+        uint32_t v[32];
+        tmem_ld32(tDV + lane_addr + h * 32, v);
+        tmem_ld_wait();
+        if (in) {
+#pragma unroll
+          for (int c = 0; c < 8; ++c)
+            *reinterpret_cast<float4*>(gv + h * 32 + 4 * c) =
+                make_float4(__uint_as_float(v[4 * c]), __uint_as_float(v[4 * c + 1]),
+                            __uint_as_float(v[4 * c + 2]), __uint_as_float(v[4 * c + 3]));
+        }
+        tmem_ld32(tDK + lane_addr + h * 32, v);
+        tmem_ld_wait();
+        if (in) {
+#pragma unroll
+          for (int c = 0; c < 8; ++c)
+            *reinterpret_cast<float4*>(gk + h * 32 + 4 * c) =
+                make_float4(__uint_as_float(v[4 * c]) * scale, __uint_as_float(v[4 * c + 1]) * scale,
+                            __uint_as_float(v[4 * c + 2]) * scale, __uint_as_float(v[4 * c + 3]) * scale);
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 5) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// ============================================================= backward: dQ
+// One CTA per (unit, 128-query tile qt); it walks the key tiles j <= qt.
+//   S = Q K_j^T, dP = dO V_j^T in TMEM; one query row per softmax thread:
+//   dS = P (dP - D) to fp16 in shared memory; dQ += dS K_j accumulates in TMEM.
+struct DqBars {
+  uint64_t q_full;
+  uint64_t kv_full[2], kv_empty[2];
+  uint64_t s_full, s_free, ds_full, dsdone, mma_done;
+  uint32_t tmem;
+  int abort;
+};
+
+template <int D>
+struct DqLayout {
+  static constexpr int kStages = (D == 64) ? 2 : 1;
+  static constexpr int kTile = 128 * D * 2;
+  static constexpr int kQ = 0;
+  static constexpr int kDO = kQ + kTile;
+  static constexpr int kK = kDO + kTile;             // kStages
+  static constexpr int kV = kK + kStages * kTile;    // kStages
+  static constexpr int kDS = kV + kStages * kTile;   // 128 x 128 fp16
+  static constexpr int kBar = kDS + 32768;
+  static constexpr int kBytes = kBar + (int)sizeof(DqBars);
+};
+
+template <int D>
+__global__ void __launch_bounds__(kFwdThreads, 1)
+    k_attn_bwd_dq_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
+                     const __grid_constant__ CUtensorMap tv, const __grid_constant__ CUtensorMap tdo,
+                     const float* __restrict__ lse, const float* __restrict__ Dv,
+                     float* __restrict__ dqs, int S, int unit0, float scale, float scale_log2,
+                     int ntiles) {
+  using Lt = DqLayout<D>;
+  constexpr int STG = Lt::kStages;
+  extern __shared__ __align__(1024) uint8_t smem[];
+  if (smem_u32(smem) & 1023u) {
+    if (threadIdx.x == 0) report_status(kStatusAttnBwdTimeout | 2u);
+    return;
+  }
+  DqBars* bars = reinterpret_cast<DqBars*>(smem + Lt::kBar);
+  uint8_t* sQ = smem + Lt::kQ;
+  uint8_t* sDO = smem + Lt::kDO;
+  uint8_t* sK = smem + Lt::kK;
+  uint8_t* sV = smem + Lt::kV;
+  uint8_t* sDS = smem + Lt::kDS;
+  volatile int* abort = &bars->abort;
+  constexpr uint32_t kStatus = kStatusAttnBwdTimeout;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int qt = ntiles - 1 - (int)blockIdx.x;  // most key tiles first
+  const int u = unit0 + (int)blockIdx.y;
+  const int n = qt + 1;
+
+  if (threadIdx.x == 0) {
+    mbar_init(&bars->q_full, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&bars->kv_full[i], 1);
+      mbar_init(&bars->kv_empty[i], 1);
+    }
+    mbar_init(&bars->s_full, 1);
+    mbar_init(&bars->s_free, 4);
+    mbar_init(&bars->ds_full, 4);
+    mbar_init(&bars->dsdone, 1);
+    mbar_init(&bars->mma_done, 1);
+    bars->abort = 0;
+    mbar_init_fence();
+  }
+  if (warp == 5) tmem_alloc(&bars->tmem, 512);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = bars->tmem;
+  const uint32_t tS = tmem, tDP = tmem + 128, tDQ = tmem + 256;
+
+  if (warp == 4) {
+    if (lane == 0) {
+      mbar_expect_tx(&bars->q_full, 2 * Lt::kTile);
+      for (int h = 0; h < D / 64; ++h) {
+        tma_load_3d(sQ + h * 16384, &tq, &bars->q_full, h * 64, qt * 128, u);
+        tma_load_3d(sDO + h * 16384, &tdo, &bars->q_full, h * 64, qt * 128, u);
+      }
+      int issued = 0;
+      for (int j = 0; j < n; ++j) {
+        const int st = j % STG;
+        if (j >= STG && !mbar_wait(&bars->kv_empty[st], ((j - STG) / STG) & 1, abort, kStatus)) break;
+        mbar_expect_tx(&bars->kv_full[st], 2 * Lt::kTile);
+        for (int h = 0; h < D / 64; ++h) {
+          tma_load_3d(sK + st * Lt::kTile + h * 16384, &tk, &bars->kv_full[st], h * 64, j * 128, u);
+          tma_load_3d(sV + st * Lt::kTile + h * 16384, &tv, &bars->kv_full[st], h * 64, j * 128, u);
+        }
+        issued = j + 1;
+      }
+      mbar_wait(&bars->q_full, 0, abort, kStatus, false);
+      for (int j = (issued > STG ? issued - STG : 0); j < issued; ++j)
+        mbar_wait(&bars->kv_full[j % STG], (j / STG) & 1, abort, kStatus, false);
+    }
+  } else if (warp == 5) {
+    if (lane == 0) {
+      constexpr uint32_t idS = idesc_f16(128, 128, false);
+      constexpr uint32_t idAcc = idesc_f16(128, D, true);
+      const uint32_t aQ = smem_u32(sQ), aDO = smem_u32(sDO), aK = smem_u32(sK), aV = smem_u32(sV);
+      const uint32_t aDS = smem_u32(sDS);
+      auto issue_dq = [&](int j) {  // dQ += dS_j K_j
+        const int st = j % STG;
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t a = aDS + (kk >> 2) * 16384 + (kk & 3) * 32;
+          const uint32_t b = aK + st * Lt::kTile + kk * 2048;
+          umma_f16(tDQ, desc_kmajor(a), desc_mnmajor(b, 16384), idAcc, (j > 0 || kk > 0));
+        }
+        umma_commit(&bars->dsdone);
+        umma_commit(&bars->kv_empty[st]);
+      };
+      bool ok = mbar_wait(&bars->q_full, 0, abort, kStatus);
+      for (int j = 0; ok && j < n; ++j) {
+        const int st = j % STG;
+        if (STG == 1 && j > 0) {  // one K/V stage: free it before the next tile loads
+          ok = mbar_wait(&bars->ds_full, (j - 1) & 1, abort, kStatus);
+          if (!ok) break;
+          tc_fence_after();
+          issue_dq(j - 1);
+        }
+        ok = mbar_wait(&bars->kv_full[st], (j / STG) & 1, abort, kStatus) &&
+             (j == 0 || mbar_wait(&bars->s_free, (j - 1) & 1, abort, kStatus));
+        if (!ok) break;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+          umma_f16(tS, desc_kmajor(aQ + off), desc_kmajor(aK + st * Lt::kTile + off), idS, kk > 0);
+          umma_f16(tDP, desc_kmajor(aDO + off), desc_kmajor(aV + st * Lt::kTile + off), idS, kk > 0);
+        }
+        umma_commit(&bars->s_full);
+        if (STG > 1 && j > 0) {
+          ok = mbar_wait(&bars->ds_full, (j - 1) & 1, abort, kStatus);
+          if (!ok) break;
+          tc_fence_after();
+          issue_dq(j - 1);
+        }
+      }
+      if (ok && mbar_wait(&bars->ds_full, (n - 1) & 1, abort, kStatus)) {
+        tc_fence_after();
+        issue_dq(n - 1);
+      }
+      umma_commit(&bars->mma_done);
+      mbar_wait(&bars->mma_done, 0, abort, kStatus, false);
+    }
+  } else {
+    const int r = threadIdx.x;
+    const uint32_t lane_addr = (uint32_t)(warp * 32) << 16;
+    const int row = qt * 128 + r;
+    const bool in = row < S;
+    const float lse2 = in ? __ldg(lse + (int64_t)u * S + row) * kLog2e : 0.0f;
+    const float Dr = in ? __ldg(Dv + (int64_t)u * S + row) : 0.0f;
+    bool ok = true;
+    for (int j = 0; j < n; ++j) {
+      ok = warp_wait(&bars->s_full, j & 1, abort, kStatus);
+      if (!ok) break;
+      tc_fence_after();
+      const bool diag = (j == qt);
+#pragma unroll
+      for (int ch = 0; ch < 4; ++ch) {
+        uint32_t a[32], b[32];
+        tmem_ld32(tS + lane_addr + ch * 32, a);
+        tmem_ld32(tDP + lane_addr + ch * 32, b);
+        tmem_ld_wait();
+        if (ch == 3) {
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&bars->s_free);
+        }
+        uint32_t pd[16];
+#pragma unroll
+        for (int e = 0; e < 32; e += 2) {
+          const int k = ch * 32 + e;
+          float p0 = ex2(fmaf(__uint_as_float(a[e]), scale_log2, -lse2));
+          float p1 = ex2(fmaf(__uint_as_float(a[e + 1]), scale_log2, -lse2));
+          if (diag && k > r) p0 = 0.0f;
+          if (diag && k + 1 > r) p1 = 0.0f;
+          pd[e >> 1] = pack_h2_sat(p0 * (__uint_as_float(b[e]) - Dr),
+                                   p1 * (__uint_as_float(b[e + 1]) - Dr));
+        }
+        if (ch == 0 && j > 0 && !(ok = warp_wait(&bars->dsdone, (j - 1) & 1, abort, kStatus))) break;
+#pragma unroll
+        for (int qd = 0; qd < 4; ++qd) {
+          const int c = ch * 4 + qd;
+          const uint32_t off = (c >> 3) * 16384 + swz(r, c & 7);
+          *reinterpret_cast<uint4*>(sDS + off) =
+              make_uint4(pd[4 * qd], pd[4 * qd + 1], pd[4 * qd + 2], pd[4 * qd + 3]);
+        }
+      }
+      if (!ok) break;
+      fence_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars->ds_full);
+    }
+    if (ok) ok = warp_wait(&bars->dsdone, (n - 1) & 1, abort, kStatus);
+    if (ok) {  // whole warps load TMEM; only rows inside the sequence are stored
+      tc_fence_after();
+      float* gq = dqs + ((int64_t)u * S + row) * D;
+#pragma unroll
+      for (int h = 0; h < D / 32; ++h) {
+        uint32_t v[32];
+        tmem_ld32(tDQ + lane_addr + h * 32, v);
+        tmem_ld_wait();
+        if (in) {
+#pragma unroll
+          for (int c = 0; c < 8; ++c)
+            *reinterpret_cast<float4*>(gq + h * 32 + 4 * c) =
+                make_float4(__uint_as_float(v[4 * c]) * scale, __uint_as_float(v[4 * c + 1]) * scale,
+                            __uint_as_float(v[4 * c + 2]) * scale, __uint_as_float(v[4 * c + 3]) * scale);
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 5) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
   }
 }
 
@@ -341,6 +836,31 @@ cudaError_t fwd_d(const Geom& g, const __half* qs, const __half* ks, const __hal
   return cudaGetLastError();
 }
 
+template <int D>
+cudaError_t bwd_d(const Geom& g, const __half* qs, const __half* ks, const __half* vs,
+                  const __half* dos, const float* lse, const float* Dv, float scale, float* dqs,
+                  float* dks, float* dvs, cudaStream_t st) {
+  CUtensorMap mq, mk, mv, mdo;
+  if (!make_map(&mq, qs, D, g.S, g.U) || !make_map(&mk, ks, D, g.S, g.U) ||
+      !make_map(&mv, vs, D, g.S, g.U) || !make_map(&mdo, dos, D, g.S, g.U))
+    return cudaErrorNotSupported;
+  constexpr int smem_a = DkvLayout<D>::kBytes, smem_b = DqLayout<D>::kBytes;
+  cudaError_t e = cudaFuncSetAttribute(k_attn_bwd_dkdv_tc<D>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, smem_a);
+  if (e != cudaSuccess) return e;
+  e = cudaFuncSetAttribute(k_attn_bwd_dq_tc<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_b);
+  if (e != cudaSuccess) return e;
+  const int ntiles = (int)((g.S + 127) / 128);
+  for (int64_t u0 = 0; u0 < g.U; u0 += 65535) {
+    const int64_t nu = g.U - u0 < 65535 ? g.U - u0 : 65535;
+    k_attn_bwd_dkdv_tc<D><<<dim3(ntiles, (unsigned)nu), kFwdThreads, smem_a, st>>>(
+        mq, mk, mv, mdo, lse, Dv, dks, dvs, (int)g.S, (int)u0, scale, scale * kLog2e, ntiles);
+    k_attn_bwd_dq_tc<D><<<dim3(ntiles, (unsigned)nu), kFwdThreads, smem_b, st>>>(
+        mq, mk, mv, mdo, lse, Dv, dqs, (int)g.S, (int)u0, scale, scale * kLog2e, ntiles);
+  }
+  return cudaGetLastError();
+}
+
 }  // namespace
 }  // namespace tc
 
@@ -352,9 +872,9 @@ bool attn_tc_available() {
     return false;
   return major == 10 && minor == 0 && tc::encode_fn() != nullptr;
 }
-bool attn_tc_bwd_available() { return false; }
+bool attn_tc_bwd_available() { return attn_tc_available(); }
 int attn_tc_fwd_launches(const Geom& g) { return (int)((g.U + 65534) / 65535); }
-int attn_tc_bwd_launches(const Geom&) { return 0; }
+int attn_tc_bwd_launches(const Geom& g) { return 2 * (int)((g.U + 65534) / 65535); }
 
 cudaError_t launch_attn_fwd_tc(const Geom& g, const __half* qs, const __half* ks,
                                const __half* vs, float scale, __half* os, float* lse,
@@ -364,10 +884,13 @@ cudaError_t launch_attn_fwd_tc(const Geom& g, const __half* qs, const __half* ks
                    : tc::fwd_d<128>(g, qs, ks, vs, scale, os, lse, st);
 }
 
-cudaError_t launch_attn_bwd_tc(const Geom&, const __half*, const __half*, const __half*,
-                               const __half*, const float*, const float*, float, float*, float*,
-                               float*, cudaStream_t) {
-  return cudaErrorNotSupported;
+cudaError_t launch_attn_bwd_tc(const Geom& g, const __half* qs, const __half* ks,
+                               const __half* vs, const __half* dos, const float* lse,
+                               const float* Dv, float scale, float* dqs, float* dks, float* dvs,
+                               cudaStream_t st) {
+  if (g.S > 0x7fffffff || g.U > 0x7fffffff) return cudaErrorInvalidValue;
+  return g.d == 64 ? tc::bwd_d<64>(g, qs, ks, vs, dos, lse, Dv, scale, dqs, dks, dvs, st)
+                   : tc::bwd_d<128>(g, qs, ks, vs, dos, lse, Dv, scale, dqs, dks, dvs, st);
 }
 
 }  // namespace lh

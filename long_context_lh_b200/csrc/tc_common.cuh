@@ -86,6 +86,13 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
   }
 }
 
+// mbar_wait for a whole warp: every lane gets the same answer, so a warp never
+// splits around the warp-collective (.sync.aligned) tcgen05 instructions.
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
+                                          uint32_t code) {
+  return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort, code));
+}
+
 // --------------------------------------------------------------------- TMA
 // 3-D tiled load (x = column, y = row within a unit, z = unit) into shared
 // memory, completing on `bar` with the bytes it delivers.  x * 2 bytes must be
