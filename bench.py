@@ -4,8 +4,9 @@
                     [--workload pretrain|long|extreme] [--attn tc|mma] [--no-cpu] [--no-dense]
 
 A step is one pass of the whole hot path over one batch of synthetic input:
-pyramid + scores, joint top-S, gather, causal sub-sequence attention,
-scatter-back, then the backward through scatter-back, attention and gather.
+pyramid + scores (one pass over Q, K, V), joint top-S, gather, causal
+sub-sequence attention, scatter-back, then the backward through scatter-back,
+attention and gather.
 The default workload is the pretraining shape (B=1, H=16, N=98,304, d=64,
 p=4, L=4, S=8192, bf16, 1% high-norm outlier tokens).  Inputs (3 x 201 MB plus
 dO) are larger than the 126 MB L2, so no flush is needed between steps.
@@ -47,20 +48,25 @@ def load_peaks():
 
 
 # ------------------------------------------------------------ algorithmic work
-def algorithmic(w):
+def algorithmic(w, span_rows=None):
     """Algorithmic bytes / FLOPs per stage for one step (whole job on one GPU).
 
     Bytes count each tensor the stage must read or write once (inputs in the
-    workload dtype, pyramid fp32, gathered rows bf16, sub-sequence gradients
-    fp32); FLOPs count the causal attention products only."""
+    workload dtype, gathered rows fp16, sub-sequence gradients fp32); FLOPs
+    count the causal attention products only.  The pooled gather must read, for
+    every selected entry, the p^l level-0 rows its pooled value is the mean of
+    (`span_rows`, summed over units, from the actual selection)."""
     U, N, d, S, M = w.B * w.H, w.N, w.d, w.S, w.M
     es = 2 if w.dtype == "bf16" else 4
     E = N * d
+    span_rows = U * S if span_rows is None else span_rows
     R = (M - N) / N
     return {
         "pyramid_score": U * (3 * E * es + 12 * E * R + 4 * M),
+        "score": U * (2 * E * es + 4 * M),
         "topk": U * (4 * M + 4 * M + 8 * S),
-        "gather": U * (S * 4 + S * 3 * d * (4 + 2)),
+        "gather": U * (4 * S + S * 3 * d * (4 + 2)),
+        "gather_pooled": U * 4 * S + span_rows * 3 * d * es + U * S * 3 * d * 2,
         "attn_fwd_flop": U * 2.0 * S * S * d,
         "scatter": U * (4 * M + S * d * 2 + E * es + 4 * N),
         "scatter_bwd": U * (E * es + 4 * N + 4 * M + S * d * 2),
@@ -180,8 +186,8 @@ def run_ours(args, rank, world, local_rank):
     dqs, dks, dvs = (torch.empty(U * w.S * w.d, dtype=torch.float32, device=dev) for _ in range(3))
     abw = lh.lh_attn_bwd_workspace_bytes(shp)
     aws = torch.empty(abw, dtype=torch.uint8, device=dev)
-    stages = ["pyramid_score", "topk", "gather", "attn_fwd", "scatter", "scatter_bwd",
-              "attn_bwd", "gather_bwd"]
+    stages = ["pyramid_score", "topk", "gather", "attn_fwd", "scatter", "scatter_bwd", "attn_bwd",
+              "gather_bwd"]
     def staged(evs):
         # identical launches to lh_forward + lh_backward, with events between stages
         evs[0].record(stream)
@@ -248,7 +254,12 @@ def run_ours(args, rank, world, local_rank):
 
     tokens = w.B * w.N
     value = world * tokens / (ms_step / 1e3)
-    alg = algorithmic(w)
+    # rows the pooled gather must read: p^level for every selected entry
+    gids = idx.view(U, w.S).long()
+    offs = torch.tensor([sum(w.level_len(m) for m in range(l)) for l in range(w.L + 1)], device=dev)
+    lev = torch.bucketize(gids, offs[1:], right=True)
+    span_rows = int((torch.tensor(w.p, device=dev, dtype=torch.float64) ** lev).sum().item())
+    alg = algorithmic(w, span_rows)
     hbm = peaks["hbm_gbs"]
     tc = peaks["bf16_tflops"]
     stage_report = {}

@@ -144,6 +144,16 @@ lh_status lh_gather(const lh_shape* shape, lh_dtype dtype, const void* q, const 
                     const void* v, const float* pq, const float* pk, const float* pv,
                     const int32_t* idx, void* qs, void* ks, void* vs, lh_stream_t stream);
 
+/* (a)+(d) for the selected entries only: the same rows as lh_gather on a
+ * pyramid from lh_build_pyramid (bit for bit: a coarse row is pooled from its
+ * span of level-0 rows with the pyramid's own order of fp32 additions and
+ * divisions), but no pyramid level is written; only the rows of selected spans
+ * are read: cheaper than the pyramid when the selected spans are few, dearer
+ * when they cover most of the sequence.                                     */
+lh_status lh_gather_pooled(const lh_shape* shape, lh_dtype dtype, const void* q, const void* k,
+                           const void* v, const int32_t* idx, void* qs, void* ks, void* vs,
+                           lh_stream_t stream);
+
 /* (e) Causal attention on the sub-sequence, [ES] §2.C (stock SDPA on a dense
  * sequence): os[k] = sum_{k'<=k} softmax_k'(scale <qs[k], ks[k']>) vs[k'],
  * lse[k] = natural log of the softmax denominator (with the max folded in).
@@ -205,8 +215,9 @@ lh_status lh_gather_bwd(const lh_shape* shape, lh_dtype dtype, const float* dqs,
 
 /* ------------------------------------------------------- fused entry points */
 
-/* Whole forward: (a)-(f).  o: [B,H,N,d] dtype.  saved: lh_saved_bytes, kept by
- * the caller for lh_backward.  ws: lh_workspace_bytes(shape, dtype, 0 or 1). */
+/* Whole forward: (a)+(b) in one pass, (c), (d), (e), (f).  o: [B,H,N,d] dtype.
+ * saved: lh_saved_bytes, kept by the caller for lh_backward.
+ * ws: lh_workspace_bytes(shape, dtype, 0 or 1). */
 lh_status lh_forward(const lh_shape* shape, lh_dtype dtype, const void* q, const void* k,
                      const void* v, float scale, void* o, void* saved, void* ws,
                      size_t ws_bytes, lh_stream_t stream);

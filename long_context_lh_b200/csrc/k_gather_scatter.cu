@@ -17,25 +17,34 @@
 namespace lh {
 namespace {
 
+// Per-unit geometry with 32-bit indices (M < 2^31 is a checked limit); unit
+// offsets stay 64-bit.  log2p >= 0 when p is a power of two: then the level-l
+// index of token t is a shift instead of a division.
 struct Lv {
-  int64_t N, M, S;
-  int L, p;
-  int64_t off[kMaxLevels + 1];
-  int64_t pw[kMaxLevels + 1];
+  int32_t N, M, S;
+  int32_t L, p, log2p;
+  int32_t off[kMaxLevels + 1];
+  int32_t pw[kMaxLevels + 1];
 };
 
 Lv make_lv(const Geom& g) {
   Lv v;
-  v.N = g.N;
-  v.M = g.M;
+  v.N = (int32_t)g.N;
+  v.M = (int32_t)g.M;
   v.S = g.S;
   v.L = g.L;
   v.p = g.p;
+  v.log2p = ((g.p & (g.p - 1)) == 0) ? __builtin_ctz((unsigned)g.p) : -1;
   for (int l = 0; l <= kMaxLevels; ++l) {
-    v.off[l] = g.off[l];
-    v.pw[l] = g.pw[l];
+    v.off[l] = (int32_t)g.off[l];
+    v.pw[l] = (int32_t)(g.pw[l] > 0x7fffffff ? 0x7fffffff : g.pw[l]);
   }
   return v;
+}
+
+// index at level l of the entry covering token t: floor(t / p^l)
+__device__ __forceinline__ int32_t lvl_index(const Lv& lv, int32_t t, int l) {
+  return lv.log2p >= 0 ? (t >> (l * lv.log2p)) : (int32_t)((uint32_t)t / (uint32_t)lv.pw[l]);
 }
 
 inline unsigned blocks_for(int64_t threads, int block) {
@@ -56,7 +65,7 @@ __global__ void __launch_bounds__(256) k_gather(
   if (row >= rows) return;
   const int c = (int)(gt % G);
   const int64_t u = row / lv.S;
-  const int64_t gid = __ldg(idx + row);
+  const int32_t gid = __ldg(idx + row);
   float xq[8], xk[8], xv[8];
   if (gid < lv.N) {
     const int64_t o = (u * lv.N + gid) * D + 8 * c;
@@ -64,7 +73,7 @@ __global__ void __launch_bounds__(256) k_gather(
     load8(k + o, xk);
     load8(v + o, xv);
   } else {
-    const int64_t o = (u * (lv.M - lv.N) + (gid - lv.N)) * D + 8 * c;
+    const int64_t o = (u * (int64_t)(lv.M - lv.N) + (gid - lv.N)) * D + 8 * c;
     load8(pq + o, xq);
     load8(pk + o, xk);
     load8(pv + o, xv);
@@ -73,6 +82,94 @@ __global__ void __launch_bounds__(256) k_gather(
   store8(qs + d, xq);
   store8(ks + d, xk);
   store8(vs + d, xv);
+}
+
+// ------------------------------------------------------------ pooled gather
+// Same result as k_gather on a pyramid, without the pyramid: a selected entry of
+// level l >= 1 is pooled from its span of level-0 rows with exactly the pyramid
+// kernel's arithmetic (children summed in order from 0.0f with fp32 adds, the
+// sum divided by p, level by level), so every value has the same bits.  Only
+// the rows of selected spans are read; no pooled level is written to HBM.
+constexpr int kPoolBatch = 4;  // level-0 rows whose loads are in flight together
+
+template <typename Tin, int D, int L>
+__device__ __forceinline__ void pool_span(const Tin* __restrict__ src, int lev, const Lv& lv,
+                                          float (&out)[8]) {
+  // src: first row of the span (this lane's 8 columns); p^lev rows at stride D;
+  // acc[l] is the running sum of the children of the current level-(l+1) entry
+  constexpr int NL = (L > 1) ? (L - 1) : 1;
+  float acc[NL][8];
+  int cnt[NL];
+#pragma unroll
+  for (int l = 0; l < NL; ++l) {
+    cnt[l] = 0;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) acc[l][i] = 0.0f;
+  }
+  const int rows = lv.pw[lev];
+  const float fp = (float)lv.p;
+  for (int r0 = 0; r0 < rows; r0 += kPoolBatch) {
+    float x[kPoolBatch][8];
+#pragma unroll
+    for (int b = 0; b < kPoolBatch; ++b)
+      if (r0 + b < rows) load8(src + (int64_t)(r0 + b) * D, x[b]);
+#pragma unroll
+    for (int b = 0; b < kPoolBatch; ++b) {
+      if (r0 + b >= rows) break;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) acc[0][i] = __fadd_rn(acc[0][i], x[b][i]);
+      cnt[0] += 1;
+#pragma unroll
+      for (int l = 0; l < NL; ++l) {
+        if (l + 1 > lev || cnt[l] != lv.p) break;
+        // level l+1 complete: its mean feeds level l+2 (or is the answer)
+        float m[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) m[i] = __fdiv_rn(acc[l][i], fp);
+        if (l + 1 == lev) {
+#pragma unroll
+          for (int i = 0; i < 8; ++i) out[i] = m[i];
+        } else if (l + 1 < NL) {
+#pragma unroll
+          for (int i = 0; i < 8; ++i) acc[l + 1][i] = __fadd_rn(acc[l + 1][i], m[i]);
+          cnt[l + 1] += 1;
+        }
+#pragma unroll
+        for (int i = 0; i < 8; ++i) acc[l][i] = 0.0f;
+        cnt[l] = 0;
+      }
+    }
+  }
+}
+
+template <typename Tin, int D, int L>
+__global__ void __launch_bounds__(256) k_gather_pooled(
+    const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin* __restrict__ v,
+    const int32_t* __restrict__ idx, __half* __restrict__ qs, __half* __restrict__ ks,
+    __half* __restrict__ vs, const Lv lv, int64_t rows) {
+  constexpr int G = D / 8;
+  const int64_t gt = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  const int64_t row = gt / G;  // u * S + slot
+  if (row >= rows) return;
+  const int c = (int)(gt % G);
+  const int64_t u = row / lv.S;
+  const int32_t gid = __ldg(idx + row);
+  int lev = 0;
+  while (lev + 1 < lv.L && gid >= lv.off[lev + 1]) ++lev;
+  const int32_t j = gid - lv.off[lev];
+  const int64_t first = (u * lv.N + (int64_t)j * lv.pw[lev]) * D + 8 * c;  // span start
+  const int64_t d = row * D + 8 * c;
+  const Tin* srcs[3] = {q + first, k + first, v + first};
+  __half* dsts[3] = {qs + d, ks + d, vs + d};
+#pragma unroll
+  for (int x = 0; x < 3; ++x) {
+    float val[8];
+    if (lev == 0)
+      load8(srcs[x], val);
+    else
+      pool_span<Tin, D, L>(srcs[x], lev, lv, val);
+    store8(dsts[x], val);
+  }
 }
 
 // ------------------------------------------------------------- scatter-back
@@ -87,14 +184,15 @@ __global__ void __launch_bounds__(256) k_scatter(const __half* __restrict__ os,
   const int64_t row = gt / G;  // u * N + t
   if (row >= rows) return;
   const int c = (int)(gt % G);
-  const int64_t u = row / lv.N, t = row % lv.N;
+  const int64_t u = row / lv.N;
+  const int32_t t = (int32_t)(row - u * lv.N);
   const int32_t* sl = slot + u * lv.M;
   float acc[8];
 #pragma unroll
   for (int i = 0; i < 8; ++i) acc[i] = 0.0f;
   int cnt = 0;
   for (int l = 0; l < lv.L; ++l) {
-    const int32_t s = __ldg(sl + lv.off[l] + t / lv.pw[l]);
+    const int32_t s = __ldg(sl + lv.off[l] + lvl_index(lv, t, l));
     if (s >= 0) {
       float x[8];
       load8(os + (u * lv.S + s) * D + 8 * c, x);
@@ -123,13 +221,14 @@ __global__ void __launch_bounds__(256) k_scatter_bwd(const Tin* __restrict__ dO,
                                                      int64_t spans, int64_t groups) {
   constexpr int G = D / 8;
   constexpr int NL = (L > 1) ? (L - 1) : 1;
+  constexpr int RB = 4;  // rows of dO whose loads are in flight together
   const int64_t gt = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   const int64_t group = gt / G;
   if (group >= groups) return;
   const int c = (int)(gt % G);
-  const int64_t Ptop = lv.pw[L - 1];
+  const int32_t Ptop = lv.pw[L - 1];
   const int64_t u = group / spans;
-  const int64_t t0 = (group % spans) * Ptop;
+  const int32_t t0 = (int32_t)(group - u * spans) * Ptop;
   const int32_t* sl = slot + u * lv.M;
   const Tin* src = dO + (u * lv.N + t0) * D + 8 * c;
   __half* dst = dos + u * lv.S * D + 8 * c;
@@ -142,42 +241,53 @@ __global__ void __launch_bounds__(256) k_scatter_bwd(const Tin* __restrict__ dO,
 #pragma unroll
     for (int i = 0; i < 8; ++i) acc[l][i] = 0.0f;
   }
-  for (int64_t r = 0; r < Ptop; ++r) {
-    const int64_t t = t0 + r;
-    float w[8];
-    load8_stream(src + r * D, w);
-    float ic;
-    if (inv_count) {
-      ic = __ldg(inv_count + u * lv.N + t);
-    } else {
-      int n = 0;
+  for (int32_t r0 = 0; r0 < Ptop; r0 += RB) {
+    float w[RB][8];
+    float ic[RB];
+    int32_t s0[RB];
 #pragma unroll
-      for (int l = 0; l < L; ++l) n += (__ldg(sl + lv.off[l] + t / lv.pw[l]) >= 0) ? 1 : 0;
-      ic = n > 0 ? __frcp_rn((float)n) : 0.0f;
+    for (int b = 0; b < RB; ++b) {
+      if (r0 + b < Ptop) {
+        const int32_t t = t0 + r0 + b;
+        load8_stream(src + (int64_t)(r0 + b) * D, w[b]);
+        s0[b] = __ldg(sl + t);
+        if (inv_count) {
+          ic[b] = __ldg(inv_count + u * lv.N + t);
+        } else {
+          int n = 0;
+#pragma unroll
+          for (int l = 0; l < L; ++l) n += (__ldg(sl + lv.off[l] + lvl_index(lv, t, l)) >= 0) ? 1 : 0;
+          ic[b] = n > 0 ? __frcp_rn((float)n) : 0.0f;
+        }
+      }
     }
 #pragma unroll
-    for (int i = 0; i < 8; ++i) w[i] = __fmul_rn(w[i], ic);
-    const int32_t s0 = __ldg(sl + t);
-    if (s0 >= 0) store8(dst + (int64_t)s0 * D, w);
-    if constexpr (L == 1) continue;
+    for (int b = 0; b < RB; ++b) {
+      if (r0 + b >= Ptop) break;
+      const int32_t t = t0 + r0 + b;
 #pragma unroll
-    for (int i = 0; i < 8; ++i) acc[0][i] = __fadd_rn(acc[0][i], w[i]);
-    cnt[0] += 1;
+      for (int i = 0; i < 8; ++i) w[b][i] = __fmul_rn(w[b][i], ic[b]);
+      if (s0[b] >= 0) store8(dst + (int64_t)s0[b] * D, w[b]);
+      if constexpr (L == 1) continue;
 #pragma unroll
-    for (int l = 0; l < NL; ++l) {
-      if (cnt[l] == lv.p) {
-        const int lev = l + 1;
-        const int64_t j = (t + 1) / lv.pw[lev] - 1;
-        const int32_t s = __ldg(sl + lv.off[lev] + j);
-        if (s >= 0) store8(dst + (int64_t)s * D, acc[l]);
-        if (l + 1 < NL) {
+      for (int i = 0; i < 8; ++i) acc[0][i] = __fadd_rn(acc[0][i], w[b][i]);
+      cnt[0] += 1;
 #pragma unroll
-          for (int i = 0; i < 8; ++i) acc[l + 1][i] = __fadd_rn(acc[l + 1][i], acc[l][i]);
-          cnt[l + 1] += 1;
+      for (int l = 0; l < NL; ++l) {
+        if (cnt[l] == lv.p) {
+          const int lev = l + 1;
+          const int32_t j = lvl_index(lv, t, lev);
+          const int32_t s = __ldg(sl + lv.off[lev] + j);
+          if (s >= 0) store8(dst + (int64_t)s * D, acc[l]);
+          if (l + 1 < NL) {
+#pragma unroll
+            for (int i = 0; i < 8; ++i) acc[l + 1][i] = __fadd_rn(acc[l + 1][i], acc[l][i]);
+            cnt[l + 1] += 1;
+          }
+#pragma unroll
+          for (int i = 0; i < 8; ++i) acc[l][i] = 0.0f;
+          cnt[l] = 0;
         }
-#pragma unroll
-        for (int i = 0; i < 8; ++i) acc[l][i] = 0.0f;
-        cnt[l] = 0;
       }
     }
   }
@@ -188,20 +298,24 @@ __global__ void __launch_bounds__(256) k_scatter_bwd(const Tin* __restrict__ dO,
 template <typename Tout, int D>
 __global__ void __launch_bounds__(256) k_gather_bwd(
     const float* __restrict__ dqs, const float* __restrict__ dks, const float* __restrict__ dvs,
-    const int32_t* __restrict__ slot, Tout* __restrict__ dq, Tout* __restrict__ dk,
-    Tout* __restrict__ dv, const Lv lv, int64_t rows) {
+    const int32_t* __restrict__ slot, const float* __restrict__ inv_count, Tout* __restrict__ dq,
+    Tout* __restrict__ dk, Tout* __restrict__ dv, const Lv lv, int64_t rows) {
   constexpr int G = D / 8;
   const int64_t gt = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   const int64_t row = gt / G;  // u * N + t
   if (row >= rows) return;
   const int c = (int)(gt % G);
-  const int64_t u = row / lv.N, t = row % lv.N;
+  const int64_t u = row / lv.N;
+  const int32_t t = (int32_t)(row - u * lv.N);
   const int32_t* sl = slot + u * lv.M;
   float aq[8], ak[8], av[8];
 #pragma unroll
   for (int i = 0; i < 8; ++i) aq[i] = ak[i] = av[i] = 0.0f;
-  for (int l = 0; l < lv.L; ++l) {
-    const int32_t s = __ldg(sl + lv.off[l] + t / lv.pw[l]);
+  // a token with no selected entry covering it (known from the forward's counts)
+  // gets zero gradients without any slot lookups
+  const int nl = (inv_count && __ldg(inv_count + row) == 0.0f) ? 0 : lv.L;
+  for (int l = 0; l < nl; ++l) {
+    const int32_t s = __ldg(sl + lv.off[l] + lvl_index(lv, t, l));
     if (s >= 0) {
       const float inv = __frcp_rn((float)lv.pw[l]);
       const int64_t o = (u * lv.S + s) * D + 8 * c;
@@ -274,6 +388,45 @@ cudaError_t launch_gather(const Geom& g, lh_dtype dt, const void* q, const void*
   return cudaGetLastError();
 }
 
+namespace {
+template <typename Tin, int D>
+cudaError_t gather_pooled_d(const Geom& g, const Tin* q, const Tin* k, const Tin* v,
+                            const int32_t* idx, __half* qs, __half* ks, __half* vs,
+                            cudaStream_t st) {
+  const Lv lv = make_lv(g);
+  const int64_t rows = g.U * g.S;
+  const unsigned nb = blocks_for(rows * (D / 8), 256);
+  switch (g.L) {
+#define LH_CASE(LL)                                                                              \
+  case LL:                                                                                       \
+    k_gather_pooled<Tin, D, LL><<<nb, 256, 0, st>>>(q, k, v, idx, qs, ks, vs, lv, rows);        \
+    break;
+    LH_CASE(1) LH_CASE(2) LH_CASE(3) LH_CASE(4) LH_CASE(5) LH_CASE(6) LH_CASE(7) LH_CASE(8)
+#undef LH_CASE
+    default:
+      return cudaErrorInvalidValue;
+  }
+  return cudaGetLastError();
+}
+}  // namespace
+
+cudaError_t launch_gather_pooled(const Geom& g, lh_dtype dt, const void* q, const void* k,
+                                 const void* v, const int32_t* idx, __half* qs, __half* ks,
+                                 __half* vs, cudaStream_t st) {
+  if (dt == LH_BF16) {
+    auto* a = static_cast<const __nv_bfloat16*>(q);
+    auto* b = static_cast<const __nv_bfloat16*>(k);
+    auto* c = static_cast<const __nv_bfloat16*>(v);
+    return g.d == 64 ? gather_pooled_d<__nv_bfloat16, 64>(g, a, b, c, idx, qs, ks, vs, st)
+                     : gather_pooled_d<__nv_bfloat16, 128>(g, a, b, c, idx, qs, ks, vs, st);
+  }
+  auto* a = static_cast<const float*>(q);
+  auto* b = static_cast<const float*>(k);
+  auto* c = static_cast<const float*>(v);
+  return g.d == 64 ? gather_pooled_d<float, 64>(g, a, b, c, idx, qs, ks, vs, st)
+                   : gather_pooled_d<float, 128>(g, a, b, c, idx, qs, ks, vs, st);
+}
+
 cudaError_t launch_scatter(const Geom& g, lh_dtype dt, const __half* os,
                            const int32_t* slot, void* o, float* inv_count, cudaStream_t st) {
   const Lv lv = make_lv(g);
@@ -330,8 +483,8 @@ cudaError_t launch_scatter_bwd(const Geom& g, lh_dtype dt, const void* dO, const
 }
 
 cudaError_t launch_gather_bwd(const Geom& g, lh_dtype dt, const float* dqs, const float* dks,
-                              const float* dvs, const int32_t* slot, void* dq, void* dk, void* dv,
-                              cudaStream_t st) {
+                              const float* dvs, const int32_t* slot, const float* inv_count,
+                              void* dq, void* dk, void* dv, cudaStream_t st) {
   const Lv lv = make_lv(g);
   const int64_t rows = g.U * g.N;
   const unsigned nb = blocks_for(rows * (g.d / 8), 256);
@@ -340,17 +493,17 @@ cudaError_t launch_gather_bwd(const Geom& g, lh_dtype dt, const float* dqs, cons
     auto* b = static_cast<__nv_bfloat16*>(dk);
     auto* c = static_cast<__nv_bfloat16*>(dv);
     if (g.d == 64)
-      k_gather_bwd<__nv_bfloat16, 64><<<nb, 256, 0, st>>>(dqs, dks, dvs, slot, a, b, c, lv, rows);
+      k_gather_bwd<__nv_bfloat16, 64><<<nb, 256, 0, st>>>(dqs, dks, dvs, slot, inv_count, a, b, c, lv, rows);
     else
-      k_gather_bwd<__nv_bfloat16, 128><<<nb, 256, 0, st>>>(dqs, dks, dvs, slot, a, b, c, lv, rows);
+      k_gather_bwd<__nv_bfloat16, 128><<<nb, 256, 0, st>>>(dqs, dks, dvs, slot, inv_count, a, b, c, lv, rows);
   } else {
     auto* a = static_cast<float*>(dq);
     auto* b = static_cast<float*>(dk);
     auto* c = static_cast<float*>(dv);
     if (g.d == 64)
-      k_gather_bwd<float, 64><<<nb, 256, 0, st>>>(dqs, dks, dvs, slot, a, b, c, lv, rows);
+      k_gather_bwd<float, 64><<<nb, 256, 0, st>>>(dqs, dks, dvs, slot, inv_count, a, b, c, lv, rows);
     else
-      k_gather_bwd<float, 128><<<nb, 256, 0, st>>>(dqs, dks, dvs, slot, a, b, c, lv, rows);
+      k_gather_bwd<float, 128><<<nb, 256, 0, st>>>(dqs, dks, dvs, slot, inv_count, a, b, c, lv, rows);
   }
   return cudaGetLastError();
 }

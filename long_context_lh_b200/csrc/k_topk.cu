@@ -41,12 +41,30 @@ constexpr int kWarps = kThreads / 32;
 constexpr int kBins = 2048;
 
 struct TopkParams {
-  int64_t N, M;
-  int p, L, S;
+  int32_t N, M;  // within-unit sizes fit 32 bits (M < 2^31 is a checked limit)
+  int p, L, S, log2p;
   int64_t unit0;
-  int64_t off[kMaxLevels + 1];
-  int64_t pw[kMaxLevels + 1];
+  int32_t off[kMaxLevels + 1];
+  int32_t pw[kMaxLevels + 1];
 };
+
+// Does the span of a level-l entry end at token t, i.e. p^l divides t + 1?
+__device__ __forceinline__ bool ends_at(const TopkParams& prm, uint32_t t1, int l) {
+  return prm.log2p >= 0 ? (t1 & ((uint32_t)prm.pw[l] - 1u)) == 0u : (t1 % (uint32_t)prm.pw[l]) == 0u;
+}
+// gid of the level-l entry whose span ends at token t (requires ends_at)
+__device__ __forceinline__ int32_t gid_at(const TopkParams& prm, uint32_t t1, int l) {
+  const uint32_t j1 = prm.log2p >= 0 ? (t1 >> (l * prm.log2p)) : t1 / (uint32_t)prm.pw[l];
+  return prm.off[l] + (int32_t)j1 - 1;
+}
+
+// Histogram increment with warp aggregation: lanes with the same bin add once.
+__device__ __forceinline__ void hist_add(uint32_t* hist, bool active, uint32_t bin) {
+  const unsigned act = __ballot_sync(0xffffffffu, active);
+  if (!active) return;
+  const unsigned same = __match_any_sync(act, bin);
+  if ((threadIdx.x & 31) == (unsigned)(__ffs(same) - 1)) atomicAdd(&hist[bin], (uint32_t)__popc(same));
+}
 
 __device__ __forceinline__ uint32_t warp_incl_scan(uint32_t v) {
   const int lane = threadIdx.x & 31;
@@ -148,9 +166,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t dmask = (uint32_t)nb - 1u;
     for (int i = threadIdx.x; i < kBins; i += kThreads) hist[buf][i] = 0;
     __syncthreads();
-    for (int64_t g = g_begin + threadIdx.x; g < g_end; g += kThreads) {
-      const uint32_t kv = __ldg(key + g);
-      if ((kv & pmask) == prefix) atomicAdd(&hist[buf][(kv >> shift) & dmask], 1u);
+    for (int64_t g0 = g_begin + (threadIdx.x & ~31); g0 < g_end; g0 += kThreads) {
+      const int64_t g = g0 + (threadIdx.x & 31);
+      const uint32_t kv = g < g_end ? __ldg(key + g) : 0u;
+      hist_add(hist[buf], g < g_end && (kv & pmask) == prefix, (kv >> shift) & dmask);
     }
     cluster.sync();
     Pick pk = pick_digit(cluster, hist[buf], nb, true, need, warp_buf, sh);
@@ -175,9 +194,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t dmask = (uint32_t)nb - 1u;
       for (int i = threadIdx.x; i < kBins; i += kThreads) hist[buf][i] = 0;
       __syncthreads();
-      for (int64_t g = g_begin + threadIdx.x; g < g_end; g += kThreads) {
-        if (__ldg(key + g) == T && (((uint32_t)g) & gmask) == gprefix)
-          atomicAdd(&hist[buf][((uint32_t)g >> shift) & dmask], 1u);
+      for (int64_t g0 = g_begin + (threadIdx.x & ~31); g0 < g_end; g0 += kThreads) {
+        const int64_t g = g0 + (threadIdx.x & 31);
+        const bool in = g < g_end && __ldg(key + (g < g_end ? g : g0)) == T &&
+                        (((uint32_t)g) & gmask) == gprefix;
+        hist_add(hist[buf], in, ((uint32_t)g >> shift) & dmask);
       }
       cluster.sync();
       // pick_digit needs nbins to be a multiple of the thread count or equal to
@@ -212,9 +233,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int64_t t = tb + lane;
     uint32_t c = 0;
     if (t < w_end) {
+      const uint32_t t1 = (uint32_t)t + 1u;
       for (int l = 0; l < prm.L; ++l) {
-        if ((t + 1) % prm.pw[l] != 0) break;  // spans end at t only up to some level
-        c += selected(prm.off[l] + (t + 1) / prm.pw[l] - 1) ? 1u : 0u;
+        if (!ends_at(prm, t1, l)) break;  // spans end at t only up to some level
+        c += selected(gid_at(prm, t1, l)) ? 1u : 0u;
       }
     }
     wcount += __reduce_add_sync(0xffffffffu, c);
@@ -240,9 +262,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint32_t c = 0;
     uint32_t selmask = 0;
     if (t < w_end) {
+      const uint32_t t1 = (uint32_t)t + 1u;
       for (int l = 0; l < prm.L; ++l) {
-        if ((t + 1) % prm.pw[l] != 0) break;
-        if (selected(prm.off[l] + (t + 1) / prm.pw[l] - 1)) {
+        if (!ends_at(prm, t1, l)) break;
+        if (selected(gid_at(prm, t1, l))) {
           selmask |= 1u << l;
           ++c;
         }
@@ -251,9 +274,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t incl = warp_incl_scan(c);
     uint32_t k = base + incl - c;
     if (t < w_end) {
+      const uint32_t t1 = (uint32_t)t + 1u;
       for (int l = 0; l < prm.L; ++l) {
-        if ((t + 1) % prm.pw[l] != 0) break;
-        const int64_t g = prm.off[l] + (t + 1) / prm.pw[l] - 1;
+        if (!ends_at(prm, t1, l)) break;
+        const int32_t g = gid_at(prm, t1, l);
         if (selmask & (1u << l)) {
           idx_u[k] = (int32_t)g;
           pos_u[k] = (int32_t)t;
@@ -274,14 +298,15 @@ __global__ void __launch_bounds__(kThreads, 1)
 cudaError_t launch_topk(const Geom& g, const float* score, int32_t* idx, int32_t* pos,
                         int32_t* slot, cudaStream_t st) {
   TopkParams prm;
-  prm.N = g.N;
-  prm.M = g.M;
+  prm.N = (int32_t)g.N;
+  prm.M = (int32_t)g.M;
   prm.p = g.p;
   prm.L = g.L;
   prm.S = g.S;
+  prm.log2p = ((g.p & (g.p - 1)) == 0) ? __builtin_ctz((unsigned)g.p) : -1;
   for (int l = 0; l <= kMaxLevels; ++l) {
-    prm.off[l] = g.off[l];
-    prm.pw[l] = g.pw[l];
+    prm.off[l] = (int32_t)g.off[l];
+    prm.pw[l] = (int32_t)(g.pw[l] > 0x7fffffff ? 0x7fffffff : g.pw[l]);
   }
   // Larger clusters for larger units: more SMs per unit, same barrier count.
   // A 16-CTA cluster is a non-portable size; it is used only when this device

@@ -270,6 +270,19 @@ lh_status lh_gather(const lh_shape* shape, lh_dtype dtype, const void* q, const 
                                    static_cast<__half*>(vs), stream));
 }
 
+lh_status lh_gather_pooled(const lh_shape* shape, lh_dtype dtype, const void* q, const void* k,
+                           const void* v, const int32_t* idx, void* qs, void* ks, void* vs,
+                           lh_stream_t stream) {
+  lh_status s = lh_validate(shape, dtype);
+  if (s != LH_OK) return s;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(idx) || !aligned16(qs) ||
+      !aligned16(ks) || !aligned16(vs))
+    return LH_ERR_INVALID_ARG;
+  return cuda_status(launch_gather_pooled(make_geom(*shape), dtype, q, k, v, idx,
+                                          static_cast<__half*>(qs), static_cast<__half*>(ks),
+                                          static_cast<__half*>(vs), stream));
+}
+
 lh_status lh_subseq_attn_fwd(const lh_shape* shape, const void* qs, const void* ks,
                              const void* vs, float scale, void* os, float* lse,
                              lh_stream_t stream) {
@@ -332,7 +345,7 @@ lh_status lh_gather_bwd(const lh_shape* shape, lh_dtype dtype, const float* dqs,
       !aligned16(dq) || !aligned16(dk) || !aligned16(dv))
     return LH_ERR_INVALID_ARG;
   return cuda_status(
-      launch_gather_bwd(make_geom(*shape), dtype, dqs, dks, dvs, slot, dq, dk, dv, stream));
+      launch_gather_bwd(make_geom(*shape), dtype, dqs, dks, dvs, slot, nullptr, dq, dk, dv, stream));
 }
 
 lh_status lh_forward(const lh_shape* shape, lh_dtype dtype, const void* q, const void* k,
@@ -400,7 +413,7 @@ lh_status lh_backward(const lh_shape* shape, lh_dtype dtype, const void* saved, 
   LH_TRY(launch_scatter_bwd(g, dtype, dO, slot, ic, dos, stream));
   s = attn_bwd(g, qs, ks, vs, os, lse, dos, resolve_scale(g, scale), dqs, dks, dvs, Dvec, stream);
   if (s != LH_OK) return s;
-  LH_TRY(launch_gather_bwd(g, dtype, dqs, dks, dvs, slot, dq, dk, dv, stream));
+  LH_TRY(launch_gather_bwd(g, dtype, dqs, dks, dvs, slot, ic, dq, dk, dv, stream));
   return LH_OK;
 }
 

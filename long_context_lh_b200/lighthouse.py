@@ -64,6 +64,7 @@ _SIGS = {
     "lh_topk_workspace_bytes": ([_SP], _SZ),
     "lh_topk_select": ([_SP, _VP, _VP, _VP, _VP, _VP, _SZ, _VP], _I),
     "lh_gather": ([_SP, _I, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP], _I),
+    "lh_gather_pooled": ([_SP, _I, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP], _I),
     "lh_subseq_attn_fwd": ([_SP, _VP, _VP, _VP, _F, _VP, _VP, _VP], _I),
     "lh_attn_bwd_workspace_bytes": ([_SP], _SZ),
     "lh_subseq_attn_bwd": ([_SP, _VP, _VP, _VP, _VP, _VP, _VP, _F, _VP, _VP, _VP, _VP, _SZ,
@@ -212,6 +213,12 @@ def lh_gather(shape, dtype, q, k, v, pq, pk, pv, idx, qs, ks, vs, stream=None):
     _check("lh_gather", _lib().lh_gather(
         ctypes.byref(shape), dtype, _p(q), _p(k), _p(v), _p(pq), _p(pk), _p(pv), _p(idx),
         _p(qs), _p(ks), _p(vs), _st(stream)))
+
+
+def lh_gather_pooled(shape, dtype, q, k, v, idx, qs, ks, vs, stream=None):
+    _check("lh_gather_pooled", _lib().lh_gather_pooled(
+        ctypes.byref(shape), dtype, _p(q), _p(k), _p(v), _p(idx), _p(qs), _p(ks), _p(vs),
+        _st(stream)))
 
 
 def lh_subseq_attn_fwd(shape, qs, ks, vs, scale, os_, lse, stream=None):

@@ -185,6 +185,21 @@ def test_gather_and_scatter_match_oracle(case):
         assert np.all(np.abs(f64(b) - ref) <= tol * np.abs(ref) + 1e-6)
 
 
+@pytest.mark.parametrize("case", STAGE_CASES, ids=str)
+def test_pooled_gather_equals_pyramid_gather_bitwise(case):
+    """lh_gather_pooled (no pyramid in HBM) == lh_gather on lh_build_pyramid, bit for bit."""
+    w = workload(**case)
+    x = to_dev(make_inputs(w, "cpu", with_dO=False))
+    pyr, score, idx, pos, slot = run_front(w, x)
+    a = gpu_gather(w, x, pyr, idx)
+    shp, dt = lshape(w), lh.dtype_code(x["q"].dtype)
+    b = [torch.empty_like(t) for t in a]
+    lh.lh_gather_pooled(shp, dt, x["q"], x["k"], x["v"], idx, *b)
+    torch.cuda.synchronize()
+    for ta, tb in zip(a, b):
+        assert torch.equal(ta, tb)
+
+
 ATTN_CASES = [(2, 512, 64), (1, 1000, 64), (1, 1, 64), (2, 384, 128), (1, 200, 128)]
 
 
