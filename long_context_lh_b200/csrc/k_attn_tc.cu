@@ -7,20 +7,19 @@
 // sub-sequence (row k sees k' <= k), scale 1/sqrt(d); §2.B: its backward is the
 // only path from the layer output back to the selected Q, K and V.
 //
-// Forward, one CTA per (unit, 128-query tile), 6 warps:
-//   warp 4 (one lane)  TMA producer: Q once, then K/V tiles of 128 keys into a
-//                      2-stage ring;
-//   warp 5 (one lane)  MMA issuer: S = Q K^T into TMEM (128 columns), then
-//                      PV = P V into TMEM (d columns) once P is in shared memory;
-//                      warp 5 also owns the TMEM allocation;
-//   warps 0-3          one thread per query row (= TMEM lane): row max over S,
-//                      P = 2^(s*scale*log2e - m) rounded to fp16 into swizzled
-//                      shared memory, running sum, and O kept in registers:
-//                      O <- alpha * O + PV each tile (online softmax).
-// S for tile j+1 is computed while the softmax threads finish tile j, and P V
-// for tile j while they find the max of tile j+1.  Every wait is bounded
-// (two seconds); on expiry the kernel records a status code, lets the other
-// roles drain, waits for its own TMA loads and MMAs, frees TMEM and returns.
+// All three kernels use one CTA per SM (512 TMEM columns) and 10 warps:
+//   warps 0-7  the row work: two threads per row of the 128-row tile (TMEM lane
+//              = row; warp w reads lanes 32*(w%4).. and one half of the columns,
+//              w/4), so 8 warps share the exponentials and the fp16 packing;
+//   warp 8     TMA producer (one lane issues; in the dK/dV kernel all 32 lanes
+//              also stage the per-query softmax statistics);
+//   warp 9     MMA issuer (one lane) and owner of the TMEM allocation.
+// Score tiles are read from TMEM into registers in one go and the buffer is
+// released at once, so the next tile's products run while the row work goes on.
+// Every mbarrier wait is bounded (two seconds); on expiry a status bit is set,
+// the roles drain, loads and MMAs in flight are waited for, TMEM is freed.
+// Rows past S are zero-filled by TMA (3-D tensor maps) and never stored; the
+// TMEM loads, being warp-collective, are always executed by whole warps.
 #include "tc_common.cuh"
 
 namespace lh {
@@ -37,37 +36,62 @@ namespace {
 
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kLog2e = 1.4426950408889634f;
-constexpr int kFwdThreads = 192;
-constexpr uint32_t kTmemCols = 256;
+constexpr int kThreads = 320;
+constexpr uint32_t kTmemCols = 512;
 
+__device__ __forceinline__ void rows_bar() {  // the 8 row-work warps only
+  asm volatile("bar.sync 1, 256;\n" ::: "memory");
+}
+
+// Two tcgen05.ld of 32 columns each, then one wait.
+__device__ __forceinline__ void tmem_ld64(uint32_t taddr, uint32_t (&a)[32], uint32_t (&b)[32]) {
+  tmem_ld32(taddr, a);
+  tmem_ld32(taddr + 32, b);
+  tmem_ld_wait();
+}
+
+__device__ __forceinline__ void store_row_half(uint8_t* tile_half, int r, const uint32_t (&pk)[32]) {
+  // one 64-column half of a row of a 128-byte-swizzled fp16 tile: 8 chunks of 16 B
+#pragma unroll
+  for (int c = 0; c < 8; ++c)
+    *reinterpret_cast<uint4*>(tile_half + swz(r, c)) =
+        make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+}
+
+// ================================================================= forward
 struct FwdBars {
   uint64_t q_full;
-  uint64_t kv_full[2];
-  uint64_t kv_empty[2];
-  uint64_t s_full, s_free, p_full, pv_done, mma_done;
+  uint64_t kv_full[3], kv_empty[3];
+  uint64_t s_full[2], s_free[2];
+  uint64_t p_full, pv_done, mma_done;
   uint32_t tmem;
   int abort;
+  float xmax[2][2][128];  // [tile parity][half][row]
+  float xsum[2][128];
 };
 
 template <int D>
 struct FwdLayout {
-  static constexpr int kTile = 128 * D * 2;  // one 128-row fp16 tile
+  static constexpr int kKS = (D == 64) ? 3 : 2;  // K/V stages
+  static constexpr int kTile = 128 * D * 2;
   static constexpr int kQ = 0;
-  static constexpr int kK = kQ + kTile;      // 2 stages
-  static constexpr int kV = kK + 2 * kTile;  // 2 stages
-  static constexpr int kP = kV + 2 * kTile;  // 128 x 128 fp16, two 64-column halves
-  static constexpr int kBar = kP + 128 * 128 * 2;
+  static constexpr int kK = kQ + kTile;
+  static constexpr int kV = kK + kKS * kTile;
+  static constexpr int kP = kV + kKS * kTile;  // 128 x 128 fp16
+  static constexpr int kBar = kP + 32768;
   static constexpr int kBytes = kBar + (int)sizeof(FwdBars);
 };
 
 template <int D>
-__global__ void __launch_bounds__(kFwdThreads, (D == 64) ? 2 : 1)
+__global__ void __launch_bounds__(kThreads, 1)
     k_attn_fwd_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
                   const __grid_constant__ CUtensorMap tv, __half* __restrict__ os,
-                  float* __restrict__ lse, int S, int unit0, float scale_log2, int ntiles) {
+                  float* __restrict__ lse, int S, int unit0, int nunits, float scale_log2,
+                  int ntiles) {
   using Lt = FwdLayout<D>;
+  constexpr int KS = Lt::kKS;
   extern __shared__ __align__(1024) uint8_t smem[];
-  if (smem_u32(smem) & 1023u) {  // swizzled tiles need 1024-byte alignment
+  if (smem_u32(smem) & 1023u) {
     if (threadIdx.x == 0) report_status(kStatusAttnFwdTimeout | 1u);
     return;
   }
@@ -77,44 +101,47 @@ __global__ void __launch_bounds__(kFwdThreads, (D == 64) ? 2 : 1)
   uint8_t* sV = smem + Lt::kV;
   uint8_t* sP = smem + Lt::kP;
   volatile int* abort = &bars->abort;
+  constexpr uint32_t kStatus = kStatusAttnFwdTimeout;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int qt = ntiles - 1 - (int)blockIdx.x;  // longest rows first
-  const int u = unit0 + (int)blockIdx.y;
-  const int nkv = qt + 1;
-  constexpr uint32_t kStatus = kStatusAttnFwdTimeout;
+  // 1-D grid ordered by work: all units' last (longest) query tiles first
+  const int qt = ntiles - 1 - (int)(blockIdx.x / nunits);
+  const int u = unit0 + (int)(blockIdx.x % nunits);
+  const int n = qt + 1;
 
   if (threadIdx.x == 0) {
     mbar_init(&bars->q_full, 1);
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < KS; ++i) {
       mbar_init(&bars->kv_full[i], 1);
       mbar_init(&bars->kv_empty[i], 1);
     }
-    mbar_init(&bars->s_full, 1);
-    mbar_init(&bars->s_free, 4);
-    mbar_init(&bars->p_full, 4);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&bars->s_full[b], 1);
+      mbar_init(&bars->s_free[b], 8);
+    }
+    mbar_init(&bars->p_full, 8);
     mbar_init(&bars->pv_done, 1);
     mbar_init(&bars->mma_done, 1);
     bars->abort = 0;
     mbar_init_fence();
   }
-  if (warp == 5) tmem_alloc(&bars->tmem, kTmemCols);
+  if (warp == 9) tmem_alloc(&bars->tmem, kTmemCols);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = bars->tmem;
-  const uint32_t tS = tmem, tPV = tmem + 128;
+  const uint32_t tO = tmem + 256;  // O accumulates here over all key tiles
 
-  if (warp == 4) {
+  if (warp == 8) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
       mbar_expect_tx(&bars->q_full, Lt::kTile);
       for (int h = 0; h < D / 64; ++h)
         tma_load_3d(sQ + h * 16384, &tq, &bars->q_full, h * 64, qt * 128, u);
       int issued = 0;
-      for (int j = 0; j < nkv; ++j) {
-        const int st = j & 1;
-        if (j >= 2 && !mbar_wait(&bars->kv_empty[st], ((j - 2) >> 1) & 1, abort, kStatus)) break;
+      for (int j = 0; j < n; ++j) {
+        const int st = j % KS;
+        if (j >= KS && !mbar_wait(&bars->kv_empty[st], ((j - KS) / KS) & 1, abort, kStatus)) break;
         mbar_expect_tx(&bars->kv_full[st], 2 * Lt::kTile);
         for (int h = 0; h < D / 64; ++h) {
           tma_load_3d(sK + st * Lt::kTile + h * 16384, &tk, &bars->kv_full[st], h * 64, j * 128, u);
@@ -122,182 +149,195 @@ __global__ void __launch_bounds__(kFwdThreads, (D == 64) ? 2 : 1)
         }
         issued = j + 1;
       }
-      // every load this thread issued lands before the CTA may exit
       mbar_wait(&bars->q_full, 0, abort, kStatus, false);
-      for (int j = (issued > 2 ? issued - 2 : 0); j < issued; ++j)
-        mbar_wait(&bars->kv_full[j & 1], (j >> 1) & 1, abort, kStatus, false);
+      for (int j = (issued > KS ? issued - KS : 0); j < issued; ++j)
+        mbar_wait(&bars->kv_full[j % KS], (j / KS) & 1, abort, kStatus, false);
     }
-  } else if (warp == 5) {
+  } else if (warp == 9) {
     // -------------------------------------------------------------- MMA issuer
     if (lane == 0) {
       constexpr uint32_t idS = idesc_f16(128, 128, false);
       constexpr uint32_t idPV = idesc_f16(128, D, true);
       const uint32_t aQ = smem_u32(sQ), aK = smem_u32(sK), aV = smem_u32(sV), aP = smem_u32(sP);
-      auto issue_s = [&](int st) {
+      auto issue_pv = [&](int i) {
+        const int st = i % KS;
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          umma_f16(tO, desc_kmajor(aP + (kk >> 2) * 16384 + (kk & 3) * 32),
+                   desc_mnmajor(aV + st * Lt::kTile + kk * 2048, 16384), idPV, (i > 0 || kk > 0));
+        umma_commit(&bars->pv_done);
+        umma_commit(&bars->kv_empty[st]);
+      };
+      bool ok = mbar_wait(&bars->q_full, 0, abort, kStatus);
+      for (int j = 0; ok && j < n; ++j) {
+        const int st = j % KS, b = j & 1;
+        ok = mbar_wait(&bars->kv_full[st], (j / KS) & 1, abort, kStatus) &&
+             (j < 2 || mbar_wait(&bars->s_free[b], ((j - 2) >> 1) & 1, abort, kStatus));
+        if (!ok) break;
+        tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-          umma_f16(tS, desc_kmajor(aQ + off), desc_kmajor(aK + st * Lt::kTile + off), idS,
-                   kk > 0);
+          umma_f16(tmem + b * 128, desc_kmajor(aQ + off), desc_kmajor(aK + st * Lt::kTile + off),
+                   idS, kk > 0);
         }
-        umma_commit(&bars->s_full);
-      };
-      bool ok = mbar_wait(&bars->q_full, 0, abort, kStatus) &&
-                mbar_wait(&bars->kv_full[0], 0, abort, kStatus);
-      if (ok) {
-        tc_fence_after();
-        issue_s(0);
-      }
-      for (int j = 0; ok && j < nkv; ++j) {
-        if (j + 1 < nkv) {
-          const int st1 = (j + 1) & 1;
-          ok = mbar_wait(&bars->kv_full[st1], ((j + 1) >> 1) & 1, abort, kStatus) &&
-               mbar_wait(&bars->s_free, j & 1, abort, kStatus);
+        umma_commit(&bars->s_full[b]);
+        if (j >= 1) {
+          ok = mbar_wait(&bars->p_full, (j - 1) & 1, abort, kStatus);
           if (!ok) break;
           tc_fence_after();
-          issue_s(st1);
+          issue_pv(j - 1);
         }
-        ok = mbar_wait(&bars->p_full, j & 1, abort, kStatus);
-        if (!ok) break;
-        tc_fence_after();
-        const int st = j & 1;
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint32_t a = aP + (kk >> 2) * 16384 + (kk & 3) * 32;
-          const uint32_t b = aV + st * Lt::kTile + kk * 2048;
-          umma_f16(tPV, desc_kmajor(a), desc_mnmajor(b, 16384), idPV, kk > 0);
-        }
-        umma_commit(&bars->pv_done);
-        umma_commit(&bars->kv_empty[st]);
       }
-      // all MMAs issued by this thread complete before TMEM is released
+      if (ok && mbar_wait(&bars->p_full, (n - 1) & 1, abort, kStatus)) {
+        tc_fence_after();
+        issue_pv(n - 1);
+      }
       umma_commit(&bars->mma_done);
       mbar_wait(&bars->mma_done, 0, abort, kStatus, false);
     }
   } else {
-    // ------------------------------------------------------- softmax, 1 row/thread
-    const int r = threadIdx.x;  // query row in the tile = TMEM lane
-    const uint32_t lane_addr = (uint32_t)(warp * 32) << 16;
-    float o[D];
-#pragma unroll
-    for (int i = 0; i < D; ++i) o[i] = 0.0f;
-    float m = -INFINITY, l = 0.0f, alpha_prev = 0.0f;
+    // ------------------------------------------- row work: two threads per row
+    // O accumulates in TMEM.  P is formed against a running reference max
+    // m_ref and O is rescaled (in TMEM) only when a tile's max exceeds m_ref
+    // by more than kRescale in the exp2 domain, so P <= 2^kRescale fits fp16;
+    // softmax is invariant to the reference, so the result is the same.
+    constexpr float kRescale = 8.0f;
+    const int qd = warp & 3, h = warp >> 2;
+    const int r = qd * 32 + lane;
+    const uint32_t lane_addr = (uint32_t)(qd * 32) << 16;
+    constexpr int DH = D / 2;  // O columns of this thread
+    float m_ref = -INFINITY, l = 0.0f;
     bool ok = true;
-    for (int j = 0; j < nkv; ++j) {
-      ok = warp_wait(&bars->s_full, j & 1, abort, kStatus);
-      if (!ok) break;
-      tc_fence_after();
-      const bool diag = (j == qt);
-      // pass 1: row max of the raw scores
+    for (int j = 0; j < n; ++j) {
+      const int b = j & 1;
+      uint32_t v0[32], v1[32];
       float mx = -INFINITY;
-#pragma unroll
-      for (int ch = 0; ch < 4; ++ch) {
-        uint32_t v[32];
-        tmem_ld32(tS + lane_addr + ch * 32, v);
-        tmem_ld_wait();
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const float x = __uint_as_float(v[i]);
-          if (!diag || ch * 32 + i <= r) mx = fmaxf(mx, x);
-        }
-      }
-      const float m_new = fmaxf(m, mx * scale_log2);
-      const float alpha = ex2(m - m_new);
-      // fold P V of the previous tile into O (also frees the P buffer)
-      if (j > 0) {
-        ok = warp_wait(&bars->pv_done, (j - 1) & 1, abort, kStatus);
-        if (!ok) break;
+      if (ok) ok = warp_wait(&bars->s_full[b], (j >> 1) & 1, abort, kStatus);
+      if (ok) {
         tc_fence_after();
+        tmem_ld64(tmem + b * 128 + lane_addr + h * 64, v0, v1);
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars->s_free[b]);  // S is in registers now
+        if (j == qt) {  // diagonal tile: keys past the query are masked
 #pragma unroll
-        for (int h = 0; h < D / 32; ++h) {
-          uint32_t v[32];
-          tmem_ld32(tPV + lane_addr + h * 32, v);
-          tmem_ld_wait();
+          for (int i = 0; i < 32; ++i)
+            mx = max3(mx, h * 64 + i <= r ? __uint_as_float(v0[i]) : -INFINITY,
+                      h * 64 + 32 + i <= r ? __uint_as_float(v1[i]) : -INFINITY);
+        } else {
 #pragma unroll
-          for (int i = 0; i < 32; ++i) o[h * 32 + i] = fmaf(o[h * 32 + i], alpha_prev, __uint_as_float(v[i]));
+          for (int i = 0; i < 32; ++i) mx = max3(mx, __uint_as_float(v0[i]), __uint_as_float(v1[i]));
         }
       }
-      // pass 2: P = 2^(s * scale_log2 - m_new) -> fp16 -> swizzled shared memory
-      float rs = 0.0f;
+      bars->xmax[b][h][r] = mx;
+      rows_bar();  // every row-work warp passes here once per tile, aborted or not
+      mx = fmaxf(mx, bars->xmax[b][h ^ 1][r]) * scale_log2;
+      // both threads of a row see the same mx and m_ref: same decision
+      const bool grow = mx > m_ref + kRescale;
+      const float m_new = grow ? mx : m_ref;
+      if (ok && j > 0) {
+        // P of the previous tile must be consumed before this tile's P is stored,
+        // and O must be complete before it is rescaled
+        ok = warp_wait(&bars->pv_done, (j - 1) & 1, abort, kStatus);
+        if (ok && __any_sync(0xffffffffu, grow)) {
+          tc_fence_after();
+          const float alpha = ex2(m_ref - m_new);  // 1 for rows that do not grow
 #pragma unroll
-      for (int ch = 0; ch < 4; ++ch) {
-        uint32_t v[32];
-        tmem_ld32(tS + lane_addr + ch * 32, v);
-        tmem_ld_wait();
-        uint32_t pk[16];
+          for (int c = 0; c < DH / 32; ++c) {
+            uint32_t ov[32];
+            tmem_ld32(tO + lane_addr + h * DH + c * 32, ov);
+            tmem_ld_wait();
 #pragma unroll
-        for (int i = 0; i < 32; i += 2) {
-          float p0 = ex2(fmaf(__uint_as_float(v[i]), scale_log2, -m_new));
-          float p1 = ex2(fmaf(__uint_as_float(v[i + 1]), scale_log2, -m_new));
-          if (diag && ch * 32 + i > r) p0 = 0.0f;
-          if (diag && ch * 32 + i + 1 > r) p1 = 0.0f;
-          rs += p0 + p1;
-          pk[i >> 1] = pack_h2(p0, p1);
-        }
-        uint8_t* base = sP + (ch >> 1) * 16384;
-#pragma unroll
-        for (int qd = 0; qd < 4; ++qd) {
-          const uint32_t c = (ch & 1) * 4 + qd;
-          *reinterpret_cast<uint4*>(base + swz(r, c)) =
-              make_uint4(pk[qd * 4], pk[qd * 4 + 1], pk[qd * 4 + 2], pk[qd * 4 + 3]);
+            for (int i = 0; i < 32; ++i) ov[i] = __float_as_uint(__uint_as_float(ov[i]) * alpha);
+            tmem_st32(tO + lane_addr + h * DH + c * 32, ov);
+          }
+          tmem_st_wait();
+          l *= alpha;
         }
       }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bars->s_free);
-      fence_async_smem();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bars->p_full);
-      l = fmaf(l, alpha, rs);
-      m = m_new;
-      alpha_prev = alpha;
+      m_ref = m_new;
+      if (ok) {
+        uint32_t pk[32];
+        const float2 cc = make_float2(scale_log2, scale_log2), nm = make_float2(-m_ref, -m_ref);
+        float2 sa = make_float2(0.0f, 0.0f), sb = make_float2(0.0f, 0.0f);
+        if (j == qt) {  // diagonal tile
+#pragma unroll
+          for (int i = 0; i < 32; i += 2) {
+            const float2 x = ffma2(make_float2(__uint_as_float(v0[i]), __uint_as_float(v0[i + 1])), cc, nm);
+            const float2 y = ffma2(make_float2(__uint_as_float(v1[i]), __uint_as_float(v1[i + 1])), cc, nm);
+            const float2 p = make_float2(h * 64 + i <= r ? ex2(x.x) : 0.0f, h * 64 + i + 1 <= r ? ex2(x.y) : 0.0f);
+            const float2 q = make_float2(h * 64 + 32 + i <= r ? ex2(y.x) : 0.0f,
+                                         h * 64 + 33 + i <= r ? ex2(y.y) : 0.0f);
+            sa = fadd2(sa, p);
+            sb = fadd2(sb, q);
+            pk[i >> 1] = h2(p.x, p.y);
+            pk[16 + (i >> 1)] = h2(q.x, q.y);
+          }
+        } else {
+#pragma unroll
+          for (int i = 0; i < 32; i += 2) {
+            const float2 x = ffma2(make_float2(__uint_as_float(v0[i]), __uint_as_float(v0[i + 1])), cc, nm);
+            const float2 y = ffma2(make_float2(__uint_as_float(v1[i]), __uint_as_float(v1[i + 1])), cc, nm);
+            const float2 p = make_float2(ex2(x.x), ex2(x.y));
+            const float2 q = make_float2(ex2(y.x), ex2(y.y));
+            sa = fadd2(sa, p);
+            sb = fadd2(sb, q);
+            pk[i >> 1] = h2(p.x, p.y);
+            pk[16 + (i >> 1)] = h2(q.x, q.y);
+          }
+        }
+        store_row_half(sP + h * 16384, r, pk);
+        tc_fence_before();  // orders the O rescale (TMEM stores) before the next product
+        fence_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars->p_full);
+        l += (sa.x + sa.y) + (sb.x + sb.y);
+      }
     }
-    if (ok) ok = warp_wait(&bars->pv_done, (nkv - 1) & 1, abort, kStatus);
-    if (ok) {  // whole warps: the TMEM loads below are warp-collective
+    if (ok) ok = warp_wait(&bars->pv_done, (n - 1) & 1, abort, kStatus);
+    bars->xsum[h][r] = l;
+    rows_bar();
+    const float lt = l + bars->xsum[h ^ 1][r];
+    const int row = qt * 128 + r;
+    if (ok) {  // whole warps load TMEM; only rows inside the sequence are stored
       tc_fence_after();
+      const float inv = 1.0f / lt;
+      __half* dst = os + ((int64_t)u * S + row) * D + h * DH;
 #pragma unroll
-      for (int h = 0; h < D / 32; ++h) {
-        uint32_t v[32];
-        tmem_ld32(tPV + lane_addr + h * 32, v);
+      for (int c = 0; c < DH / 32; ++c) {
+        uint32_t ov[32];
+        tmem_ld32(tO + lane_addr + h * DH + c * 32, ov);
         tmem_ld_wait();
+        if (row < S) {
 #pragma unroll
-        for (int i = 0; i < 32; ++i) o[h * 32 + i] = fmaf(o[h * 32 + i], alpha_prev, __uint_as_float(v[i]));
-      }
-      const int row = qt * 128 + r;
-      if (row < S) {
-        const float inv = 1.0f / l;
-        __half* dst = os + ((int64_t)u * S + row) * D;
-#pragma unroll
-        for (int c = 0; c < D / 8; ++c) {
-          uint4 w;
-          w.x = pack_h2(o[8 * c + 0] * inv, o[8 * c + 1] * inv);
-          w.y = pack_h2(o[8 * c + 2] * inv, o[8 * c + 3] * inv);
-          w.z = pack_h2(o[8 * c + 4] * inv, o[8 * c + 5] * inv);
-          w.w = pack_h2(o[8 * c + 6] * inv, o[8 * c + 7] * inv);
-          *reinterpret_cast<uint4*>(dst + 8 * c) = w;
+          for (int x = 0; x < 4; ++x) {
+            uint4 w;
+            w.x = h2_sat(__uint_as_float(ov[8 * x + 0]) * inv, __uint_as_float(ov[8 * x + 1]) * inv);
+            w.y = h2_sat(__uint_as_float(ov[8 * x + 2]) * inv, __uint_as_float(ov[8 * x + 3]) * inv);
+            w.z = h2_sat(__uint_as_float(ov[8 * x + 4]) * inv, __uint_as_float(ov[8 * x + 5]) * inv);
+            w.w = h2_sat(__uint_as_float(ov[8 * x + 6]) * inv, __uint_as_float(ov[8 * x + 7]) * inv);
+            *reinterpret_cast<uint4*>(dst + c * 32 + 8 * x) = w;
+          }
         }
-        lse[(int64_t)u * S + row] = (m + __log2f(l)) * kLn2;
       }
+      if (h == 0 && row < S) lse[(int64_t)u * S + row] = (m_ref + __log2f(lt)) * kLn2;
     }
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 5) {
+  if (warp == 9) {
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);
   }
 }
 
 // ========================================================= backward: dK, dV
-// One CTA per (unit, 128-key tile kt); it walks the query tiles i >= kt.
-//   warp 4: TMA for K, V once and a ring of (Q_i, dO_i) tiles; its 32 lanes also
-//           stage lse_i * log2(e) and D_i of the 128 queries in shared memory;
-//   warp 5: MMA issuer: S^T = K Q_i^T and dP^T = V dO_i^T (TMEM, 128 columns
-//           each), then dV += P^T dO_i and dK += dS^T Q_i (TMEM, d columns each);
-//   warps 0-3: one key row each: P^T = 2^(S^T c - lse2) (zero where the query
-//           precedes the key), dS^T = P^T (dP^T - D), both to fp16 in swizzled
-//           shared memory as the A operands of the two accumulating products.
-// dK and dV never leave TMEM until the last tile: no atomics, fixed order.
+// One CTA per (unit, 128-key tile kt), walking the query tiles i >= kt:
+// S^T = K Q_i^T and dP^T = V dO_i^T in TMEM; two threads per key row form
+// P^T = 2^(S^T c - lse2) (zero where the query precedes the key) and
+// dS^T = P^T (dP^T - D) in fp16 shared memory; dV += P^T dO_i and dK += dS^T Q_i
+// accumulate in TMEM over all query tiles (fixed order, no atomics).
 struct DkvBars {
   uint64_t kv_full;
   uint64_t q_full[2], q_empty[2];
@@ -312,23 +352,23 @@ struct DkvLayout {
   static constexpr int kTile = 128 * D * 2;
   static constexpr int kK = 0;
   static constexpr int kV = kK + kTile;
-  static constexpr int kQ = kV + kTile;                 // kStages
-  static constexpr int kDO = kQ + kStages * kTile;      // kStages
-  static constexpr int kPT = kDO + kStages * kTile;     // 128 x 128 fp16
-  static constexpr int kDST = kPT + 32768;              // 128 x 128 fp16
-  static constexpr int kLse = kDST + 32768;             // kStages x 128 fp32
-  static constexpr int kDv = kLse + kStages * 512;      // kStages x 128 fp32
+  static constexpr int kQ = kV + kTile;
+  static constexpr int kDO = kQ + kStages * kTile;
+  static constexpr int kPT = kDO + kStages * kTile;
+  static constexpr int kDST = kPT + 32768;
+  static constexpr int kLse = kDST + 32768;
+  static constexpr int kDv = kLse + kStages * 512;
   static constexpr int kBar = kDv + kStages * 512;
   static constexpr int kBytes = kBar + (int)sizeof(DkvBars);
 };
 
 template <int D>
-__global__ void __launch_bounds__(kFwdThreads, 1)
+__global__ void __launch_bounds__(kThreads, 1)
     k_attn_bwd_dkdv_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
                        const __grid_constant__ CUtensorMap tv, const __grid_constant__ CUtensorMap tdo,
                        const float* __restrict__ lse, const float* __restrict__ Dv,
                        float* __restrict__ dks, float* __restrict__ dvs, int S, int unit0,
-                       float scale, float scale_log2, int ntiles) {
+                       int nunits, float scale, float scale_log2, int ntiles) {
   using Lt = DkvLayout<D>;
   constexpr int STG = Lt::kStages;
   extern __shared__ __align__(1024) uint8_t smem[];
@@ -349,9 +389,10 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   constexpr uint32_t kStatus = kStatusAttnBwdTimeout;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int kt = (int)blockIdx.x;  // kt = 0 has the most query tiles: it starts first
-  const int u = unit0 + (int)blockIdx.y;
-  const int n = ntiles - kt;       // query tiles kt .. ntiles-1
+  // 1-D grid ordered by work: key tile 0 (the most query tiles) of every unit first
+  const int kt = (int)(blockIdx.x / nunits);
+  const int u = unit0 + (int)(blockIdx.x % nunits);
+  const int n = ntiles - kt;
 
   if (threadIdx.x == 0) {
     mbar_init(&bars->kv_full, 1);
@@ -360,22 +401,21 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       mbar_init(&bars->q_empty[i], 1);
     }
     mbar_init(&bars->s_full, 1);
-    mbar_init(&bars->st_free, 4);
-    mbar_init(&bars->p_full, 4);
+    mbar_init(&bars->st_free, 8);
+    mbar_init(&bars->p_full, 8);
     mbar_init(&bars->pdone, 1);
     mbar_init(&bars->mma_done, 1);
     bars->abort = 0;
     mbar_init_fence();
   }
-  if (warp == 5) tmem_alloc(&bars->tmem, 512);
+  if (warp == 9) tmem_alloc(&bars->tmem, kTmemCols);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = bars->tmem;
   const uint32_t tST = tmem, tDPT = tmem + 128, tDV = tmem + 256, tDK = tmem + 256 + D;
 
-  if (warp == 4) {
-    // ------------------------------------------------------------ producer
+  if (warp == 8) {
     if (lane == 0) {
       mbar_expect_tx(&bars->kv_full, 2 * Lt::kTile);
       for (int h = 0; h < D / 64; ++h) {
@@ -397,9 +437,10 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       for (int c = lane; c < 128; c += 32) {
         const int q = i * 128 + c;
         const bool in = q < S;
-        // padded queries: lse2 = +inf makes their P^T (and dS^T) exactly zero
-        sLse[st * 128 + c] = in ? __ldg(lse + (int64_t)u * S + q) * kLog2e : INFINITY;
-        sDv[st * 128 + c] = in ? __ldg(Dv + (int64_t)u * S + q) : 0.0f;
+        // stored negated: -lse*log2(e) and -D; padded queries get -inf, which
+        // makes their P^T (and dS^T) exactly zero
+        sLse[st * 128 + c] = in ? -__ldg(lse + (int64_t)u * S + q) * kLog2e : -INFINITY;
+        sDv[st * 128 + c] = in ? -__ldg(Dv + (int64_t)u * S + q) : 0.0f;
       }
       mbar_arrive(&bars->q_full[st]);
       issued = t + 1;
@@ -409,8 +450,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       for (int t = (issued > STG ? issued - STG : 0); t < issued; ++t)
         mbar_wait(&bars->q_full[t % STG], (t / STG) & 1, abort, kStatus, false);
     }
-  } else if (warp == 5) {
-    // -------------------------------------------------------------- MMA issuer
+  } else if (warp == 9) {
     if (lane == 0) {
       constexpr uint32_t idS = idesc_f16(128, 128, false);
       constexpr uint32_t idAcc = idesc_f16(128, D, true);
@@ -431,9 +471,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       bool ok = mbar_wait(&bars->kv_full, 0, abort, kStatus);
       for (int t = 0; ok && t < n; ++t) {
         const int st = t % STG;
-        // with one (Q, dO) stage the previous tile's products must finish before
-        // the producer can bring the next tile into it
-        if (STG == 1 && t > 0) {
+        if (STG == 1 && t > 0) {  // one stage: free it before the next tile is loaded
           ok = mbar_wait(&bars->p_full, (t - 1) & 1, abort, kStatus);
           if (!ok) break;
           tc_fence_after();
@@ -465,109 +503,112 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       mbar_wait(&bars->mma_done, 0, abort, kStatus, false);
     }
   } else {
-    // ------------------------------------------------------- one key row per thread
-    const int r = threadIdx.x;
-    const uint32_t lane_addr = (uint32_t)(warp * 32) << 16;
+    // --------------------------------------- row work: two threads per key row
+    const int qd = warp & 3, h = warp >> 2;
+    const int r = qd * 32 + lane;
+    const uint32_t lane_addr = (uint32_t)(qd * 32) << 16;
     bool ok = true;
-    for (int t = 0; t < n; ++t) {
+    for (int t = 0; t < n && ok; ++t) {
       const int st = t % STG;
       ok = warp_wait(&bars->q_full[st], (t / STG) & 1, abort, kStatus) &&
            warp_wait(&bars->s_full, t & 1, abort, kStatus);
       if (!ok) break;
       tc_fence_after();
-      const bool diag = (t == 0);
-      const float* cl = sLse + st * 128;
-      const float* cd = sDv + st * 128;
-#pragma unroll
-      for (int ch = 0; ch < 4; ++ch) {
-        uint32_t a[32], b[32];
-        tmem_ld32(tST + lane_addr + ch * 32, a);
-        tmem_ld32(tDPT + lane_addr + ch * 32, b);
-        tmem_ld_wait();
-        if (ch == 3) {  // S^T and dP^T of this tile are in registers: TMEM may be overwritten
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&bars->st_free);
+      uint32_t a0[32], a1[32], b0[32], b1[32];
+      tmem_ld32(tST + lane_addr + h * 64, a0);
+      tmem_ld32(tST + lane_addr + h * 64 + 32, a1);
+      tmem_ld32(tDPT + lane_addr + h * 64, b0);
+      tmem_ld32(tDPT + lane_addr + h * 64 + 32, b1);
+      tmem_ld_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars->st_free);  // S^T, dP^T are in registers now
+      const float* cl = sLse + st * 128 + h * 64;  // -lse2 of the 64 query columns
+      const float* cd = sDv + st * 128 + h * 64;   // -D
+      const float2 cc = make_float2(scale_log2, scale_log2);
+      uint32_t pp[32], pd[32];
+      auto pair = [&](int e, uint32_t s0, uint32_t s1, uint32_t g0, uint32_t g1, bool diag) {
+        const float2 nl = *reinterpret_cast<const float2*>(cl + e);
+        const float2 nd = *reinterpret_cast<const float2*>(cd + e);
+        const float2 x = ffma2(make_float2(__uint_as_float(s0), __uint_as_float(s1)), cc, nl);
+        float2 p = make_float2(ex2(x.x), ex2(x.y));
+        if (diag) {  // the query (column) precedes the key (row): masked
+          if (h * 64 + e < r) p.x = 0.0f;
+          if (h * 64 + e + 1 < r) p.y = 0.0f;
         }
-        uint32_t pp[16], pd[16];
+        const float2 ds = fmul2(p, fadd2(make_float2(__uint_as_float(g0), __uint_as_float(g1)), nd));
+        pp[e >> 1] = h2(p.x, p.y);
+        pd[e >> 1] = h2_sat(ds.x, ds.y);
+      };
+      if (t == 0) {
 #pragma unroll
         for (int e = 0; e < 32; e += 2) {
-          const int q = ch * 32 + e;
-          const float2 l2 = *reinterpret_cast<const float2*>(cl + q);
-          const float2 dd = *reinterpret_cast<const float2*>(cd + q);
-          float p0 = ex2(fmaf(__uint_as_float(a[e]), scale_log2, -l2.x));
-          float p1 = ex2(fmaf(__uint_as_float(a[e + 1]), scale_log2, -l2.y));
-          if (diag && q < r) p0 = 0.0f;
-          if (diag && q + 1 < r) p1 = 0.0f;
-          const float d0 = p0 * (__uint_as_float(b[e]) - dd.x);
-          const float d1 = p1 * (__uint_as_float(b[e + 1]) - dd.y);
-          pp[e >> 1] = pack_h2(p0, p1);
-          pd[e >> 1] = pack_h2_sat(d0, d1);
+          pair(e, a0[e], a0[e + 1], b0[e], b0[e + 1], true);
+          pair(e + 32, a1[e], a1[e + 1], b1[e], b1[e + 1], true);
         }
-        // the previous tile's products must be done reading the P^T / dS^T buffers
-        if (ch == 0 && t > 0 && !(ok = warp_wait(&bars->pdone, (t - 1) & 1, abort, kStatus))) break;
+      } else {
 #pragma unroll
-        for (int qd = 0; qd < 4; ++qd) {
-          const int c = ch * 4 + qd;  // 16-byte chunk of the 128-column row
-          const uint32_t off = (c >> 3) * 16384 + swz(r, c & 7);
-          *reinterpret_cast<uint4*>(sPT + off) =
-              make_uint4(pp[4 * qd], pp[4 * qd + 1], pp[4 * qd + 2], pp[4 * qd + 3]);
-          *reinterpret_cast<uint4*>(sDST + off) =
-              make_uint4(pd[4 * qd], pd[4 * qd + 1], pd[4 * qd + 2], pd[4 * qd + 3]);
+        for (int e = 0; e < 32; e += 2) {
+          pair(e, a0[e], a0[e + 1], b0[e], b0[e + 1], false);
+          pair(e + 32, a1[e], a1[e + 1], b1[e], b1[e + 1], false);
         }
       }
-      if (!ok) break;
+      if (t > 0 && !(ok = warp_wait(&bars->pdone, (t - 1) & 1, abort, kStatus))) break;
+      store_row_half(sPT + h * 16384, r, pp);
+      store_row_half(sDST + h * 16384, r, pd);
       fence_async_smem();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars->p_full);
     }
     if (ok) ok = warp_wait(&bars->pdone, (n - 1) & 1, abort, kStatus);
     const int row = kt * 128 + r;
-    if (ok) {  // whole warps load TMEM; only rows inside the sequence are stored
+    if (ok) {
       tc_fence_after();
-      float* gv = dvs + ((int64_t)u * S + row) * D;
-      float* gk = dks + ((int64_t)u * S + row) * D;
       const bool in = row < S;
+      constexpr int DH = D / 2;
+      float* gv = dvs + ((int64_t)u * S + row) * D + h * DH;
+      float* gk = dks + ((int64_t)u * S + row) * D + h * DH;
 #pragma unroll
-      for (int h = 0; h < D / 32; ++h) {
+      for (int c = 0; c < DH / 32; ++c) {
         uint32_t v[32];
-        tmem_ld32(tDV + lane_addr + h * 32, v);
+        tmem_ld32(tDV + lane_addr + h * DH + c * 32, v);
         tmem_ld_wait();
         if (in) {
 #pragma unroll
-          for (int c = 0; c < 8; ++c)
-            *reinterpret_cast<float4*>(gv + h * 32 + 4 * c) =
-                make_float4(__uint_as_float(v[4 * c]), __uint_as_float(v[4 * c + 1]),
-                            __uint_as_float(v[4 * c + 2]), __uint_as_float(v[4 * c + 3]));
+          for (int x = 0; x < 8; ++x)
+            *reinterpret_cast<float4*>(gv + c * 32 + 4 * x) =
+                make_float4(__uint_as_float(v[4 * x]), __uint_as_float(v[4 * x + 1]),
+                            __uint_as_float(v[4 * x + 2]), __uint_as_float(v[4 * x + 3]));
         }
-        tmem_ld32(tDK + lane_addr + h * 32, v);
+        tmem_ld32(tDK + lane_addr + h * DH + c * 32, v);
         tmem_ld_wait();
         if (in) {
 #pragma unroll
-          for (int c = 0; c < 8; ++c)
-            *reinterpret_cast<float4*>(gk + h * 32 + 4 * c) =
-                make_float4(__uint_as_float(v[4 * c]) * scale, __uint_as_float(v[4 * c + 1]) * scale,
-                            __uint_as_float(v[4 * c + 2]) * scale, __uint_as_float(v[4 * c + 3]) * scale);
+          for (int x = 0; x < 8; ++x)
+            *reinterpret_cast<float4*>(gk + c * 32 + 4 * x) =
+                make_float4(__uint_as_float(v[4 * x]) * scale, __uint_as_float(v[4 * x + 1]) * scale,
+                            __uint_as_float(v[4 * x + 2]) * scale, __uint_as_float(v[4 * x + 3]) * scale);
         }
       }
     }
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 5) {
+  if (warp == 9) {
     tc_fence_after();
-    tmem_dealloc(tmem, 512);
+    tmem_dealloc(tmem, kTmemCols);
   }
 }
 
 // ============================================================= backward: dQ
-// One CTA per (unit, 128-query tile qt); it walks the key tiles j <= qt.
-//   S = Q K_j^T, dP = dO V_j^T in TMEM; one query row per softmax thread:
-//   dS = P (dP - D) to fp16 in shared memory; dQ += dS K_j accumulates in TMEM.
+// One CTA per (unit, 128-query tile qt), walking the key tiles j <= qt:
+// S = Q K_j^T, dP = dO V_j^T in TMEM; two threads per query row form
+// dS = P (dP - D) in fp16 shared memory (double-buffered); dQ += dS K_j in TMEM.
 struct DqBars {
   uint64_t q_full;
   uint64_t kv_full[2], kv_empty[2];
-  uint64_t s_full, s_free, ds_full, dsdone, mma_done;
+  uint64_t s_full, s_free, mma_done;
+  uint64_t ds_full[2], dsdone[2];
   uint32_t tmem;
   int abort;
 };
@@ -578,20 +619,20 @@ struct DqLayout {
   static constexpr int kTile = 128 * D * 2;
   static constexpr int kQ = 0;
   static constexpr int kDO = kQ + kTile;
-  static constexpr int kK = kDO + kTile;             // kStages
-  static constexpr int kV = kK + kStages * kTile;    // kStages
-  static constexpr int kDS = kV + kStages * kTile;   // 128 x 128 fp16
-  static constexpr int kBar = kDS + 32768;
+  static constexpr int kK = kDO + kTile;
+  static constexpr int kV = kK + kStages * kTile;
+  static constexpr int kDS = kV + kStages * kTile;  // 2 buffers of 128 x 128 fp16
+  static constexpr int kBar = kDS + 2 * 32768;
   static constexpr int kBytes = kBar + (int)sizeof(DqBars);
 };
 
 template <int D>
-__global__ void __launch_bounds__(kFwdThreads, 1)
+__global__ void __launch_bounds__(kThreads, 1)
     k_attn_bwd_dq_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
                      const __grid_constant__ CUtensorMap tv, const __grid_constant__ CUtensorMap tdo,
                      const float* __restrict__ lse, const float* __restrict__ Dv,
-                     float* __restrict__ dqs, int S, int unit0, float scale, float scale_log2,
-                     int ntiles) {
+                     float* __restrict__ dqs, int S, int unit0, int nunits, float scale,
+                     float scale_log2, int ntiles) {
   using Lt = DqLayout<D>;
   constexpr int STG = Lt::kStages;
   extern __shared__ __align__(1024) uint8_t smem[];
@@ -609,8 +650,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   constexpr uint32_t kStatus = kStatusAttnBwdTimeout;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int qt = ntiles - 1 - (int)blockIdx.x;  // most key tiles first
-  const int u = unit0 + (int)blockIdx.y;
+  const int qt = ntiles - 1 - (int)(blockIdx.x / nunits);  // most key tiles first
+  const int u = unit0 + (int)(blockIdx.x % nunits);
   const int n = qt + 1;
 
   if (threadIdx.x == 0) {
@@ -618,23 +659,23 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     for (int i = 0; i < 2; ++i) {
       mbar_init(&bars->kv_full[i], 1);
       mbar_init(&bars->kv_empty[i], 1);
+      mbar_init(&bars->ds_full[i], 8);
+      mbar_init(&bars->dsdone[i], 1);
     }
     mbar_init(&bars->s_full, 1);
-    mbar_init(&bars->s_free, 4);
-    mbar_init(&bars->ds_full, 4);
-    mbar_init(&bars->dsdone, 1);
+    mbar_init(&bars->s_free, 8);
     mbar_init(&bars->mma_done, 1);
     bars->abort = 0;
     mbar_init_fence();
   }
-  if (warp == 5) tmem_alloc(&bars->tmem, 512);
+  if (warp == 9) tmem_alloc(&bars->tmem, kTmemCols);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = bars->tmem;
   const uint32_t tS = tmem, tDP = tmem + 128, tDQ = tmem + 256;
 
-  if (warp == 4) {
+  if (warp == 8) {
     if (lane == 0) {
       mbar_expect_tx(&bars->q_full, 2 * Lt::kTile);
       for (int h = 0; h < D / 64; ++h) {
@@ -656,32 +697,30 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       for (int j = (issued > STG ? issued - STG : 0); j < issued; ++j)
         mbar_wait(&bars->kv_full[j % STG], (j / STG) & 1, abort, kStatus, false);
     }
-  } else if (warp == 5) {
+  } else if (warp == 9) {
     if (lane == 0) {
       constexpr uint32_t idS = idesc_f16(128, 128, false);
       constexpr uint32_t idAcc = idesc_f16(128, D, true);
       const uint32_t aQ = smem_u32(sQ), aDO = smem_u32(sDO), aK = smem_u32(sK), aV = smem_u32(sV);
       const uint32_t aDS = smem_u32(sDS);
       auto issue_dq = [&](int j) {  // dQ += dS_j K_j
-        const int st = j % STG;
+        const int st = j % STG, b = j & 1;
+        if (!mbar_wait(&bars->ds_full[b], (j >> 1) & 1, abort, kStatus)) return false;
+        tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
-          const uint32_t a = aDS + (kk >> 2) * 16384 + (kk & 3) * 32;
-          const uint32_t b = aK + st * Lt::kTile + kk * 2048;
-          umma_f16(tDQ, desc_kmajor(a), desc_mnmajor(b, 16384), idAcc, (j > 0 || kk > 0));
+          const uint32_t a = aDS + b * 32768 + (kk >> 2) * 16384 + (kk & 3) * 32;
+          umma_f16(tDQ, desc_kmajor(a), desc_mnmajor(aK + st * Lt::kTile + kk * 2048, 16384), idAcc,
+                   (j > 0 || kk > 0));
         }
-        umma_commit(&bars->dsdone);
+        umma_commit(&bars->dsdone[b]);
         umma_commit(&bars->kv_empty[st]);
+        return true;
       };
       bool ok = mbar_wait(&bars->q_full, 0, abort, kStatus);
       for (int j = 0; ok && j < n; ++j) {
         const int st = j % STG;
-        if (STG == 1 && j > 0) {  // one K/V stage: free it before the next tile loads
-          ok = mbar_wait(&bars->ds_full, (j - 1) & 1, abort, kStatus);
-          if (!ok) break;
-          tc_fence_after();
-          issue_dq(j - 1);
-        }
+        if (STG == 1 && j > 0 && !(ok = issue_dq(j - 1))) break;
         ok = mbar_wait(&bars->kv_full[st], (j / STG) & 1, abort, kStatus) &&
              (j == 0 || mbar_wait(&bars->s_free, (j - 1) & 1, abort, kStatus));
         if (!ok) break;
@@ -693,93 +732,93 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
           umma_f16(tDP, desc_kmajor(aDO + off), desc_kmajor(aV + st * Lt::kTile + off), idS, kk > 0);
         }
         umma_commit(&bars->s_full);
-        if (STG > 1 && j > 0) {
-          ok = mbar_wait(&bars->ds_full, (j - 1) & 1, abort, kStatus);
-          if (!ok) break;
-          tc_fence_after();
-          issue_dq(j - 1);
-        }
+        if (STG > 1 && j > 0 && !(ok = issue_dq(j - 1))) break;
       }
-      if (ok && mbar_wait(&bars->ds_full, (n - 1) & 1, abort, kStatus)) {
-        tc_fence_after();
-        issue_dq(n - 1);
-      }
+      if (ok) issue_dq(n - 1);
       umma_commit(&bars->mma_done);
       mbar_wait(&bars->mma_done, 0, abort, kStatus, false);
     }
   } else {
-    const int r = threadIdx.x;
-    const uint32_t lane_addr = (uint32_t)(warp * 32) << 16;
+    // ------------------------------------- row work: two threads per query row
+    const int qd = warp & 3, h = warp >> 2;
+    const int r = qd * 32 + lane;
+    const uint32_t lane_addr = (uint32_t)(qd * 32) << 16;
     const int row = qt * 128 + r;
     const bool in = row < S;
     const float lse2 = in ? __ldg(lse + (int64_t)u * S + row) * kLog2e : 0.0f;
     const float Dr = in ? __ldg(Dv + (int64_t)u * S + row) : 0.0f;
     bool ok = true;
-    for (int j = 0; j < n; ++j) {
+    for (int j = 0; j < n && ok; ++j) {
       ok = warp_wait(&bars->s_full, j & 1, abort, kStatus);
       if (!ok) break;
       tc_fence_after();
-      const bool diag = (j == qt);
-#pragma unroll
-      for (int ch = 0; ch < 4; ++ch) {
-        uint32_t a[32], b[32];
-        tmem_ld32(tS + lane_addr + ch * 32, a);
-        tmem_ld32(tDP + lane_addr + ch * 32, b);
-        tmem_ld_wait();
-        if (ch == 3) {
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&bars->s_free);
+      uint32_t a0[32], a1[32], b0[32], b1[32];
+      tmem_ld32(tS + lane_addr + h * 64, a0);
+      tmem_ld32(tS + lane_addr + h * 64 + 32, a1);
+      tmem_ld32(tDP + lane_addr + h * 64, b0);
+      tmem_ld32(tDP + lane_addr + h * 64 + 32, b1);
+      tmem_ld_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars->s_free);
+      const float2 cc = make_float2(scale_log2, scale_log2), nl = make_float2(-lse2, -lse2);
+      const float2 nd = make_float2(-Dr, -Dr);
+      uint32_t pd[32];
+      auto pair = [&](int e, uint32_t s0, uint32_t s1, uint32_t g0, uint32_t g1, bool diag) {
+        const float2 x = ffma2(make_float2(__uint_as_float(s0), __uint_as_float(s1)), cc, nl);
+        float2 p = make_float2(ex2(x.x), ex2(x.y));
+        if (diag) {  // keys past the query: masked
+          if (h * 64 + e > r) p.x = 0.0f;
+          if (h * 64 + e + 1 > r) p.y = 0.0f;
         }
-        uint32_t pd[16];
+        const float2 ds = fmul2(p, fadd2(make_float2(__uint_as_float(g0), __uint_as_float(g1)), nd));
+        pd[e >> 1] = h2_sat(ds.x, ds.y);
+      };
+      if (j == qt) {
 #pragma unroll
         for (int e = 0; e < 32; e += 2) {
-          const int k = ch * 32 + e;
-          float p0 = ex2(fmaf(__uint_as_float(a[e]), scale_log2, -lse2));
-          float p1 = ex2(fmaf(__uint_as_float(a[e + 1]), scale_log2, -lse2));
-          if (diag && k > r) p0 = 0.0f;
-          if (diag && k + 1 > r) p1 = 0.0f;
-          pd[e >> 1] = pack_h2_sat(p0 * (__uint_as_float(b[e]) - Dr),
-                                   p1 * (__uint_as_float(b[e + 1]) - Dr));
+          pair(e, a0[e], a0[e + 1], b0[e], b0[e + 1], true);
+          pair(e + 32, a1[e], a1[e + 1], b1[e], b1[e + 1], true);
         }
-        if (ch == 0 && j > 0 && !(ok = warp_wait(&bars->dsdone, (j - 1) & 1, abort, kStatus))) break;
+      } else {
 #pragma unroll
-        for (int qd = 0; qd < 4; ++qd) {
-          const int c = ch * 4 + qd;
-          const uint32_t off = (c >> 3) * 16384 + swz(r, c & 7);
-          *reinterpret_cast<uint4*>(sDS + off) =
-              make_uint4(pd[4 * qd], pd[4 * qd + 1], pd[4 * qd + 2], pd[4 * qd + 3]);
+        for (int e = 0; e < 32; e += 2) {
+          pair(e, a0[e], a0[e + 1], b0[e], b0[e + 1], false);
+          pair(e + 32, a1[e], a1[e + 1], b1[e], b1[e + 1], false);
         }
       }
-      if (!ok) break;
+      const int b = j & 1;
+      if (j >= 2 && !(ok = warp_wait(&bars->dsdone[b], ((j - 2) >> 1) & 1, abort, kStatus))) break;
+      store_row_half(sDS + b * 32768 + h * 16384, r, pd);
       fence_async_smem();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&bars->ds_full);
+      if (lane == 0) mbar_arrive(&bars->ds_full[b]);
     }
-    if (ok) ok = warp_wait(&bars->dsdone, (n - 1) & 1, abort, kStatus);
-    if (ok) {  // whole warps load TMEM; only rows inside the sequence are stored
+    if (ok) ok = warp_wait(&bars->dsdone[(n - 1) & 1], ((n - 1) >> 1) & 1, abort, kStatus);
+    if (ok) {
       tc_fence_after();
-      float* gq = dqs + ((int64_t)u * S + row) * D;
+      constexpr int DH = D / 2;
+      float* gq = dqs + ((int64_t)u * S + row) * D + h * DH;
 #pragma unroll
-      for (int h = 0; h < D / 32; ++h) {
+      for (int c = 0; c < DH / 32; ++c) {
         uint32_t v[32];
-        tmem_ld32(tDQ + lane_addr + h * 32, v);
+        tmem_ld32(tDQ + lane_addr + h * DH + c * 32, v);
         tmem_ld_wait();
         if (in) {
 #pragma unroll
-          for (int c = 0; c < 8; ++c)
-            *reinterpret_cast<float4*>(gq + h * 32 + 4 * c) =
-                make_float4(__uint_as_float(v[4 * c]) * scale, __uint_as_float(v[4 * c + 1]) * scale,
-                            __uint_as_float(v[4 * c + 2]) * scale, __uint_as_float(v[4 * c + 3]) * scale);
+          for (int x = 0; x < 8; ++x)
+            *reinterpret_cast<float4*>(gq + c * 32 + 4 * x) =
+                make_float4(__uint_as_float(v[4 * x]) * scale, __uint_as_float(v[4 * x + 1]) * scale,
+                            __uint_as_float(v[4 * x + 2]) * scale, __uint_as_float(v[4 * x + 3]) * scale);
         }
       }
     }
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 5) {
+  if (warp == 9) {
     tc_fence_after();
-    tmem_dealloc(tmem, 512);
+    tmem_dealloc(tmem, kTmemCols);
   }
 }
 
@@ -828,10 +867,11 @@ cudaError_t fwd_d(const Geom& g, const __half* qs, const __half* ks, const __hal
       cudaFuncSetAttribute(k_attn_fwd_tc<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   const int ntiles = (int)((g.S + 127) / 128);
-  for (int64_t u0 = 0; u0 < g.U; u0 += 65535) {
-    const int64_t nu = g.U - u0 < 65535 ? g.U - u0 : 65535;
-    k_attn_fwd_tc<D><<<dim3(ntiles, (unsigned)nu), kFwdThreads, smem, st>>>(
-        mq, mk, mv, os, lse, (int)g.S, (int)u0, scale * kLog2e, ntiles);
+  const int64_t per = 0x7fffffff / ntiles;  // units per launch (grid.x limit)
+  for (int64_t u0 = 0; u0 < g.U; u0 += per) {
+    const int64_t nu = g.U - u0 < per ? g.U - u0 : per;
+    k_attn_fwd_tc<D><<<(unsigned)(nu * ntiles), kThreads, smem, st>>>(
+        mq, mk, mv, os, lse, (int)g.S, (int)u0, (int)nu, scale * kLog2e, ntiles);
   }
   return cudaGetLastError();
 }
@@ -851,12 +891,14 @@ cudaError_t bwd_d(const Geom& g, const __half* qs, const __half* ks, const __hal
   e = cudaFuncSetAttribute(k_attn_bwd_dq_tc<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_b);
   if (e != cudaSuccess) return e;
   const int ntiles = (int)((g.S + 127) / 128);
-  for (int64_t u0 = 0; u0 < g.U; u0 += 65535) {
-    const int64_t nu = g.U - u0 < 65535 ? g.U - u0 : 65535;
-    k_attn_bwd_dkdv_tc<D><<<dim3(ntiles, (unsigned)nu), kFwdThreads, smem_a, st>>>(
-        mq, mk, mv, mdo, lse, Dv, dks, dvs, (int)g.S, (int)u0, scale, scale * kLog2e, ntiles);
-    k_attn_bwd_dq_tc<D><<<dim3(ntiles, (unsigned)nu), kFwdThreads, smem_b, st>>>(
-        mq, mk, mv, mdo, lse, Dv, dqs, (int)g.S, (int)u0, scale, scale * kLog2e, ntiles);
+  const int64_t per = 0x7fffffff / ntiles;
+  for (int64_t u0 = 0; u0 < g.U; u0 += per) {
+    const int64_t nu = g.U - u0 < per ? g.U - u0 : per;
+    k_attn_bwd_dkdv_tc<D><<<(unsigned)(nu * ntiles), kThreads, smem_a, st>>>(
+        mq, mk, mv, mdo, lse, Dv, dks, dvs, (int)g.S, (int)u0, (int)nu, scale, scale * kLog2e,
+        ntiles);
+    k_attn_bwd_dq_tc<D><<<(unsigned)(nu * ntiles), kThreads, smem_b, st>>>(
+        mq, mk, mv, mdo, lse, Dv, dqs, (int)g.S, (int)u0, (int)nu, scale, scale * kLog2e, ntiles);
   }
   return cudaGetLastError();
 }
@@ -873,8 +915,11 @@ bool attn_tc_available() {
   return major == 10 && minor == 0 && tc::encode_fn() != nullptr;
 }
 bool attn_tc_bwd_available() { return attn_tc_available(); }
-int attn_tc_fwd_launches(const Geom& g) { return (int)((g.U + 65534) / 65535); }
-int attn_tc_bwd_launches(const Geom& g) { return 2 * (int)((g.U + 65534) / 65535); }
+int attn_tc_fwd_launches(const Geom& g) {
+  const int64_t ntiles = (g.S + 127) / 128, per = 0x7fffffff / ntiles;
+  return (int)((g.U + per - 1) / per);
+}
+int attn_tc_bwd_launches(const Geom& g) { return 2 * attn_tc_fwd_launches(g); }
 
 cudaError_t launch_attn_fwd_tc(const Geom& g, const __half* qs, const __half* ks,
                                const __half* vs, float scale, __half* os, float* lse,
