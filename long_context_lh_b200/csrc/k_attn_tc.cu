@@ -20,6 +20,8 @@
 // the roles drain, loads and MMAs in flight are waited for, TMEM is freed.
 // Rows past S are zero-filled by TMA (3-D tensor maps) and never stored; the
 // TMEM loads, being warp-collective, are always executed by whole warps.
+#include <type_traits>
+
 #include "tc_common.cuh"
 
 namespace lh {
@@ -63,11 +65,10 @@ struct FwdBars {
   uint64_t q_full;
   uint64_t kv_full[3], kv_empty[3];
   uint64_t s_full[2], s_free[2];
-  uint64_t p_full, pv_done, mma_done;
+  uint64_t p_full[2], pv_done[2], mma_done;  // [column half]
   uint32_t tmem;
   int abort;
-  float xmax[2][2][128];  // [tile parity][half][row]
-  float xsum[2][128];
+  float xm[2][128], xl[2][128];  // [half][row] final max and sum
 };
 
 template <int D>
@@ -119,8 +120,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&bars->s_full[b], 1);
       mbar_init(&bars->s_free[b], 8);
     }
-    mbar_init(&bars->p_full, 8);
-    mbar_init(&bars->pv_done, 1);
+    for (int h = 0; h < 2; ++h) {
+      mbar_init(&bars->p_full[h], 4);
+      mbar_init(&bars->pv_done[h], 1);
+    }
     mbar_init(&bars->mma_done, 1);
     bars->abort = 0;
     mbar_init_fence();
@@ -130,7 +133,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = bars->tmem;
-  const uint32_t tO = tmem + 256;  // O accumulates here over all key tiles
+  // O_h (h = key half of every tile) accumulates at tmem + 256 + h * D
+  const uint32_t tO = tmem + 256;
 
   if (warp == 8) {
     // ------------------------------------------------------------ TMA producer
@@ -159,14 +163,23 @@ __global__ void __launch_bounds__(kThreads, 1)
       constexpr uint32_t idS = idesc_f16(128, 128, false);
       constexpr uint32_t idPV = idesc_f16(128, D, true);
       const uint32_t aQ = smem_u32(sQ), aK = smem_u32(sK), aV = smem_u32(sV), aP = smem_u32(sP);
+      // O_h += P[:, keys of half h] V[keys of half h, :], once the row work
+      // of half h has stored its P
       auto issue_pv = [&](int i) {
         const int st = i % KS;
+        for (int h = 0; h < 2; ++h) {
+          if (!mbar_wait(&bars->p_full[h], i & 1, abort, kStatus)) return false;
+          tc_fence_after();
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          umma_f16(tO, desc_kmajor(aP + (kk >> 2) * 16384 + (kk & 3) * 32),
-                   desc_mnmajor(aV + st * Lt::kTile + kk * 2048, 16384), idPV, (i > 0 || kk > 0));
-        umma_commit(&bars->pv_done);
+          for (int k4 = 0; k4 < 4; ++k4) {
+            const int kk = h * 4 + k4;
+            umma_f16(tO + h * D, desc_kmajor(aP + h * 16384 + k4 * 32),
+                     desc_mnmajor(aV + st * Lt::kTile + kk * 2048, 16384), idPV, (i > 0 || k4 > 0));
+          }
+          umma_commit(&bars->pv_done[h]);
+        }
         umma_commit(&bars->kv_empty[st]);
+        return true;
       };
       bool ok = mbar_wait(&bars->q_full, 0, abort, kStatus);
       for (int j = 0; ok && j < n; ++j) {
@@ -182,146 +195,145 @@ __global__ void __launch_bounds__(kThreads, 1)
                    idS, kk > 0);
         }
         umma_commit(&bars->s_full[b]);
-        if (j >= 1) {
-          ok = mbar_wait(&bars->p_full, (j - 1) & 1, abort, kStatus);
-          if (!ok) break;
-          tc_fence_after();
-          issue_pv(j - 1);
-        }
+        if (j >= 1 && !(ok = issue_pv(j - 1))) break;
       }
-      if (ok && mbar_wait(&bars->p_full, (n - 1) & 1, abort, kStatus)) {
-        tc_fence_after();
-        issue_pv(n - 1);
-      }
+      if (ok) issue_pv(n - 1);
       umma_commit(&bars->mma_done);
       mbar_wait(&bars->mma_done, 0, abort, kStatus, false);
     }
   } else {
     // ------------------------------------------- row work: two threads per row
-    // O accumulates in TMEM.  P is formed against a running reference max
-    // m_ref and O is rescaled (in TMEM) only when a tile's max exceeds m_ref
-    // by more than kRescale in the exp2 domain, so P <= 2^kRescale fits fp16;
-    // softmax is invariant to the reference, so the result is the same.
+    // Thread (row r, half h) owns the 64 keys of half h in every tile and the
+    // partial softmax over them: its own running reference max m_ref, sum l
+    // and accumulator O_h in TMEM.  No exchange is needed until the end, where
+    // the two partials of a row are combined (the usual split-softmax merge).
+    // P is formed against m_ref, and O_h is rescaled in TMEM only when a tile's
+    // max exceeds m_ref by more than kRescale (exp2 domain), so P <= 2^kRescale
+    // fits fp16; softmax is invariant to the reference, so the result is the same.
     constexpr float kRescale = 8.0f;
     const int qd = warp & 3, h = warp >> 2;
     const int r = qd * 32 + lane;
     const uint32_t lane_addr = (uint32_t)(qd * 32) << 16;
-    constexpr int DH = D / 2;  // O columns of this thread
+    const uint32_t tOh = tO + h * D + lane_addr;
     float m_ref = -INFINITY, l = 0.0f;
     bool ok = true;
-    for (int j = 0; j < n; ++j) {
+    // one key tile; kDiag: the last (diagonal) tile, keys past the row masked
+    auto step = [&](int j, auto diag_tag) {
+      constexpr bool kDiag = decltype(diag_tag)::value;
       const int b = j & 1;
+      ok = warp_wait(&bars->s_full[b], (j >> 1) & 1, abort, kStatus);
+      if (!ok) return;
+      tc_fence_after();
       uint32_t v0[32], v1[32];
+      tmem_ld64(tmem + b * 128 + lane_addr + h * 64, v0, v1);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars->s_free[b]);  // S is in registers now
+      const int lim = r - h * 64;                     // keys i <= lim are visible
       float mx = -INFINITY;
-      if (ok) ok = warp_wait(&bars->s_full[b], (j >> 1) & 1, abort, kStatus);
-      if (ok) {
-        tc_fence_after();
-        tmem_ld64(tmem + b * 128 + lane_addr + h * 64, v0, v1);
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&bars->s_free[b]);  // S is in registers now
-        if (j == qt) {  // diagonal tile: keys past the query are masked
 #pragma unroll
-          for (int i = 0; i < 32; ++i)
-            mx = max3(mx, h * 64 + i <= r ? __uint_as_float(v0[i]) : -INFINITY,
-                      h * 64 + 32 + i <= r ? __uint_as_float(v1[i]) : -INFINITY);
+      for (int i = 0; i < 32; ++i) {
+        if (kDiag) {
+          mx = max3(mx, i <= lim ? __uint_as_float(v0[i]) : -INFINITY,
+                    i + 32 <= lim ? __uint_as_float(v1[i]) : -INFINITY);
         } else {
-#pragma unroll
-          for (int i = 0; i < 32; ++i) mx = max3(mx, __uint_as_float(v0[i]), __uint_as_float(v1[i]));
+          mx = max3(mx, __uint_as_float(v0[i]), __uint_as_float(v1[i]));
         }
       }
-      bars->xmax[b][h][r] = mx;
-      rows_bar();  // every row-work warp passes here once per tile, aborted or not
-      mx = fmaxf(mx, bars->xmax[b][h ^ 1][r]) * scale_log2;
-      // both threads of a row see the same mx and m_ref: same decision
+      mx *= scale_log2;
       const bool grow = mx > m_ref + kRescale;
       const float m_new = grow ? mx : m_ref;
-      if (ok && j > 0) {
-        // P of the previous tile must be consumed before this tile's P is stored,
-        // and O must be complete before it is rescaled
-        ok = warp_wait(&bars->pv_done, (j - 1) & 1, abort, kStatus);
-        if (ok && __any_sync(0xffffffffu, grow)) {
+      if (j > 0) {
+        // P_h of the previous tile must be consumed before this one is stored,
+        // and O_h must be complete before it is rescaled
+        ok = warp_wait(&bars->pv_done[h], (j - 1) & 1, abort, kStatus);
+        if (!ok) return;
+        if (__any_sync(0xffffffffu, grow)) {
           tc_fence_after();
           const float alpha = ex2(m_ref - m_new);  // 1 for rows that do not grow
 #pragma unroll
-          for (int c = 0; c < DH / 32; ++c) {
+          for (int c = 0; c < D / 32; ++c) {
             uint32_t ov[32];
-            tmem_ld32(tO + lane_addr + h * DH + c * 32, ov);
+            tmem_ld32(tOh + c * 32, ov);
             tmem_ld_wait();
 #pragma unroll
             for (int i = 0; i < 32; ++i) ov[i] = __float_as_uint(__uint_as_float(ov[i]) * alpha);
-            tmem_st32(tO + lane_addr + h * DH + c * 32, ov);
+            tmem_st32(tOh + c * 32, ov);
           }
           tmem_st_wait();
           l *= alpha;
         }
       }
       m_ref = m_new;
-      if (ok) {
-        uint32_t pk[32];
-        const float2 cc = make_float2(scale_log2, scale_log2), nm = make_float2(-m_ref, -m_ref);
-        float2 sa = make_float2(0.0f, 0.0f), sb = make_float2(0.0f, 0.0f);
-        if (j == qt) {  // diagonal tile
+      // a fully masked half (only in the diagonal tile) has m_ref = -inf: its
+      // exponent is NaN but every one of its elements is replaced by 0 below
+      uint32_t pk[32];
+      const float2 cc = make_float2(scale_log2, scale_log2), nm = make_float2(-m_ref, -m_ref);
+      float2 sa = make_float2(0.0f, 0.0f), sb = make_float2(0.0f, 0.0f);
 #pragma unroll
-          for (int i = 0; i < 32; i += 2) {
-            const float2 x = ffma2(make_float2(__uint_as_float(v0[i]), __uint_as_float(v0[i + 1])), cc, nm);
-            const float2 y = ffma2(make_float2(__uint_as_float(v1[i]), __uint_as_float(v1[i + 1])), cc, nm);
-            const float2 p = make_float2(h * 64 + i <= r ? ex2(x.x) : 0.0f, h * 64 + i + 1 <= r ? ex2(x.y) : 0.0f);
-            const float2 q = make_float2(h * 64 + 32 + i <= r ? ex2(y.x) : 0.0f,
-                                         h * 64 + 33 + i <= r ? ex2(y.y) : 0.0f);
-            sa = fadd2(sa, p);
-            sb = fadd2(sb, q);
-            pk[i >> 1] = h2(p.x, p.y);
-            pk[16 + (i >> 1)] = h2(q.x, q.y);
-          }
-        } else {
-#pragma unroll
-          for (int i = 0; i < 32; i += 2) {
-            const float2 x = ffma2(make_float2(__uint_as_float(v0[i]), __uint_as_float(v0[i + 1])), cc, nm);
-            const float2 y = ffma2(make_float2(__uint_as_float(v1[i]), __uint_as_float(v1[i + 1])), cc, nm);
-            const float2 p = make_float2(ex2(x.x), ex2(x.y));
-            const float2 q = make_float2(ex2(y.x), ex2(y.y));
-            sa = fadd2(sa, p);
-            sb = fadd2(sb, q);
-            pk[i >> 1] = h2(p.x, p.y);
-            pk[16 + (i >> 1)] = h2(q.x, q.y);
-          }
+      for (int i = 0; i < 32; i += 2) {
+        const float2 x = ffma2(make_float2(__uint_as_float(v0[i]), __uint_as_float(v0[i + 1])), cc, nm);
+        const float2 y = ffma2(make_float2(__uint_as_float(v1[i]), __uint_as_float(v1[i + 1])), cc, nm);
+        float2 p = make_float2(ex2(x.x), ex2(x.y));
+        float2 q = make_float2(ex2(y.x), ex2(y.y));
+        if (kDiag) {
+          p.x = i <= lim ? p.x : 0.0f;
+          p.y = i + 1 <= lim ? p.y : 0.0f;
+          q.x = i + 32 <= lim ? q.x : 0.0f;
+          q.y = i + 33 <= lim ? q.y : 0.0f;
         }
-        store_row_half(sP + h * 16384, r, pk);
-        tc_fence_before();  // orders the O rescale (TMEM stores) before the next product
-        fence_async_smem();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&bars->p_full);
-        l += (sa.x + sa.y) + (sb.x + sb.y);
+        sa = fadd2(sa, p);
+        sb = fadd2(sb, q);
+        pk[i >> 1] = h2(p.x, p.y);
+        pk[16 + (i >> 1)] = h2(q.x, q.y);
       }
-    }
-    if (ok) ok = warp_wait(&bars->pv_done, (n - 1) & 1, abort, kStatus);
-    bars->xsum[h][r] = l;
+      store_row_half(sP + h * 16384, r, pk);
+      tc_fence_before();  // orders the O_h rescale (TMEM stores) before the next product
+      fence_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars->p_full[h]);
+      l += (sa.x + sa.y) + (sb.x + sb.y);
+    };
+    for (int j = 0; j < n - 1 && ok; ++j) step(j, std::false_type{});
+    if (ok) step(n - 1, std::true_type{});
+    if (ok) ok = warp_wait(&bars->pv_done[h], (n - 1) & 1, abort, kStatus);
+    // merge the two halves of each row: O = sum_h 2^(m_h - m) O_h / sum_h 2^(m_h - m) l_h
+    bars->xm[h][r] = m_ref;
+    bars->xl[h][r] = l;
     rows_bar();
-    const float lt = l + bars->xsum[h ^ 1][r];
+    const float m0 = bars->xm[0][r], m1 = bars->xm[1][r];
+    const float m = fmaxf(m0, m1);  // finite: key 0 of half 0 is visible to every row
+    const float w0 = ex2(m0 - m), w1 = ex2(m1 - m);
+    const float lt = w0 * bars->xl[0][r] + w1 * bars->xl[1][r];
     const int row = qt * 128 + r;
     if (ok) {  // whole warps load TMEM; only rows inside the sequence are stored
       tc_fence_after();
+      constexpr int DH = D / 2;  // output columns of this thread
       const float inv = 1.0f / lt;
+      const float2 c0 = make_float2(w0 * inv, w0 * inv), c1 = make_float2(w1 * inv, w1 * inv);
       __half* dst = os + ((int64_t)u * S + row) * D + h * DH;
 #pragma unroll
       for (int c = 0; c < DH / 32; ++c) {
-        uint32_t ov[32];
-        tmem_ld32(tO + lane_addr + h * DH + c * 32, ov);
+        uint32_t o0[32], o1[32];
+        tmem_ld32(tO + lane_addr + h * DH + c * 32, o0);
+        tmem_ld32(tO + D + lane_addr + h * DH + c * 32, o1);
         tmem_ld_wait();
         if (row < S) {
 #pragma unroll
           for (int x = 0; x < 4; ++x) {
-            uint4 w;
-            w.x = h2_sat(__uint_as_float(ov[8 * x + 0]) * inv, __uint_as_float(ov[8 * x + 1]) * inv);
-            w.y = h2_sat(__uint_as_float(ov[8 * x + 2]) * inv, __uint_as_float(ov[8 * x + 3]) * inv);
-            w.z = h2_sat(__uint_as_float(ov[8 * x + 4]) * inv, __uint_as_float(ov[8 * x + 5]) * inv);
-            w.w = h2_sat(__uint_as_float(ov[8 * x + 6]) * inv, __uint_as_float(ov[8 * x + 7]) * inv);
-            *reinterpret_cast<uint4*>(dst + c * 32 + 8 * x) = w;
+            uint32_t w[4];
+#pragma unroll
+            for (int y = 0; y < 4; ++y) {
+              const int e = 8 * x + 2 * y;
+              const float2 f = ffma2(make_float2(__uint_as_float(o1[e]), __uint_as_float(o1[e + 1])), c1,
+                                     fmul2(make_float2(__uint_as_float(o0[e]), __uint_as_float(o0[e + 1])), c0));
+              w[y] = h2_sat(f.x, f.y);
+            }
+            *reinterpret_cast<uint4*>(dst + c * 32 + 8 * x) = make_uint4(w[0], w[1], w[2], w[3]);
           }
         }
       }
-      if (h == 0 && row < S) lse[(int64_t)u * S + row] = (m_ref + __log2f(lt)) * kLn2;
+      if (h == 0 && row < S) lse[(int64_t)u * S + row] = (m + __log2f(lt)) * kLn2;
     }
   }
   tc_fence_before();
@@ -508,11 +520,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int r = qd * 32 + lane;
     const uint32_t lane_addr = (uint32_t)(qd * 32) << 16;
     bool ok = true;
-    for (int t = 0; t < n && ok; ++t) {
+    // one query tile; kDiag: the first (diagonal) tile, queries before the key masked
+    auto step = [&](int t, auto diag_tag) {
+      constexpr bool kDiag = decltype(diag_tag)::value;
       const int st = t % STG;
       ok = warp_wait(&bars->q_full[st], (t / STG) & 1, abort, kStatus) &&
            warp_wait(&bars->s_full, t & 1, abort, kStatus);
-      if (!ok) break;
+      if (!ok) return;
       tc_fence_after();
       uint32_t a0[32], a1[32], b0[32], b1[32];
       tmem_ld32(tST + lane_addr + h * 64, a0);
@@ -523,43 +537,48 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars->st_free);  // S^T, dP^T are in registers now
-      const float* cl = sLse + st * 128 + h * 64;  // -lse2 of the 64 query columns
-      const float* cd = sDv + st * 128 + h * 64;   // -D
+      const float4* cl = reinterpret_cast<const float4*>(sLse + st * 128 + h * 64);  // -lse2
+      const float4* cd = reinterpret_cast<const float4*>(sDv + st * 128 + h * 64);   // -D
+      const int lim = r - h * 64;  // query columns e < lim precede the key
       const float2 cc = make_float2(scale_log2, scale_log2);
       uint32_t pp[32], pd[32];
-      auto pair = [&](int e, uint32_t s0, uint32_t s1, uint32_t g0, uint32_t g1, bool diag) {
-        const float2 nl = *reinterpret_cast<const float2*>(cl + e);
-        const float2 nd = *reinterpret_cast<const float2*>(cd + e);
-        const float2 x = ffma2(make_float2(__uint_as_float(s0), __uint_as_float(s1)), cc, nl);
-        float2 p = make_float2(ex2(x.x), ex2(x.y));
-        if (diag) {  // the query (column) precedes the key (row): masked
-          if (h * 64 + e < r) p.x = 0.0f;
-          if (h * 64 + e + 1 < r) p.y = 0.0f;
+      auto quad = [&](int e, const uint32_t* sv, const uint32_t* gv) {
+        const float4 nl = cl[e >> 2], nd = cd[e >> 2];
+        const int k = e & 31;
+        const float2 x0 = ffma2(make_float2(__uint_as_float(sv[k]), __uint_as_float(sv[k + 1])), cc,
+                                make_float2(nl.x, nl.y));
+        const float2 x1 = ffma2(make_float2(__uint_as_float(sv[k + 2]), __uint_as_float(sv[k + 3])), cc,
+                                make_float2(nl.z, nl.w));
+        float2 p0 = make_float2(ex2(x0.x), ex2(x0.y)), p1 = make_float2(ex2(x1.x), ex2(x1.y));
+        if (kDiag) {
+          p0.x = e < lim ? 0.0f : p0.x;
+          p0.y = e + 1 < lim ? 0.0f : p0.y;
+          p1.x = e + 2 < lim ? 0.0f : p1.x;
+          p1.y = e + 3 < lim ? 0.0f : p1.y;
         }
-        const float2 ds = fmul2(p, fadd2(make_float2(__uint_as_float(g0), __uint_as_float(g1)), nd));
-        pp[e >> 1] = h2(p.x, p.y);
-        pd[e >> 1] = h2_sat(ds.x, ds.y);
+        const float2 d0 = fmul2(p0, fadd2(make_float2(__uint_as_float(gv[k]), __uint_as_float(gv[k + 1])),
+                                          make_float2(nd.x, nd.y)));
+        const float2 d1 = fmul2(p1, fadd2(make_float2(__uint_as_float(gv[k + 2]), __uint_as_float(gv[k + 3])),
+                                          make_float2(nd.z, nd.w)));
+        pp[e >> 1] = h2(p0.x, p0.y);
+        pp[(e >> 1) + 1] = h2(p1.x, p1.y);
+        pd[e >> 1] = h2_sat(d0.x, d0.y);
+        pd[(e >> 1) + 1] = h2_sat(d1.x, d1.y);
       };
-      if (t == 0) {
 #pragma unroll
-        for (int e = 0; e < 32; e += 2) {
-          pair(e, a0[e], a0[e + 1], b0[e], b0[e + 1], true);
-          pair(e + 32, a1[e], a1[e + 1], b1[e], b1[e + 1], true);
-        }
-      } else {
-#pragma unroll
-        for (int e = 0; e < 32; e += 2) {
-          pair(e, a0[e], a0[e + 1], b0[e], b0[e + 1], false);
-          pair(e + 32, a1[e], a1[e + 1], b1[e], b1[e + 1], false);
-        }
+      for (int e = 0; e < 32; e += 4) {
+        quad(e, a0, b0);
+        quad(e + 32, a1, b1);
       }
-      if (t > 0 && !(ok = warp_wait(&bars->pdone, (t - 1) & 1, abort, kStatus))) break;
+      if (t > 0 && !(ok = warp_wait(&bars->pdone, (t - 1) & 1, abort, kStatus))) return;
       store_row_half(sPT + h * 16384, r, pp);
       store_row_half(sDST + h * 16384, r, pd);
       fence_async_smem();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars->p_full);
-    }
+    };
+    step(0, std::true_type{});
+    for (int t = 1; t < n && ok; ++t) step(t, std::false_type{});
     if (ok) ok = warp_wait(&bars->pdone, (n - 1) & 1, abort, kStatus);
     const int row = kt * 128 + r;
     if (ok) {
@@ -748,9 +767,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     const float lse2 = in ? __ldg(lse + (int64_t)u * S + row) * kLog2e : 0.0f;
     const float Dr = in ? __ldg(Dv + (int64_t)u * S + row) : 0.0f;
     bool ok = true;
-    for (int j = 0; j < n && ok; ++j) {
+    // one key tile; kDiag: the last (diagonal) tile, keys past the query masked
+    auto step = [&](int j, auto diag_tag) {
+      constexpr bool kDiag = decltype(diag_tag)::value;
       ok = warp_wait(&bars->s_full, j & 1, abort, kStatus);
-      if (!ok) break;
+      if (!ok) return;
       tc_fence_after();
       uint32_t a0[32], a1[32], b0[32], b1[32];
       tmem_ld32(tS + lane_addr + h * 64, a0);
@@ -763,37 +784,32 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (lane == 0) mbar_arrive(&bars->s_free);
       const float2 cc = make_float2(scale_log2, scale_log2), nl = make_float2(-lse2, -lse2);
       const float2 nd = make_float2(-Dr, -Dr);
+      const int lim = r - h * 64;  // key columns e > lim follow the query
       uint32_t pd[32];
-      auto pair = [&](int e, uint32_t s0, uint32_t s1, uint32_t g0, uint32_t g1, bool diag) {
+      auto pair = [&](int e, uint32_t s0, uint32_t s1, uint32_t g0, uint32_t g1) {
         const float2 x = ffma2(make_float2(__uint_as_float(s0), __uint_as_float(s1)), cc, nl);
         float2 p = make_float2(ex2(x.x), ex2(x.y));
-        if (diag) {  // keys past the query: masked
-          if (h * 64 + e > r) p.x = 0.0f;
-          if (h * 64 + e + 1 > r) p.y = 0.0f;
+        if (kDiag) {
+          p.x = e > lim ? 0.0f : p.x;
+          p.y = e + 1 > lim ? 0.0f : p.y;
         }
         const float2 ds = fmul2(p, fadd2(make_float2(__uint_as_float(g0), __uint_as_float(g1)), nd));
         pd[e >> 1] = h2_sat(ds.x, ds.y);
       };
-      if (j == qt) {
 #pragma unroll
-        for (int e = 0; e < 32; e += 2) {
-          pair(e, a0[e], a0[e + 1], b0[e], b0[e + 1], true);
-          pair(e + 32, a1[e], a1[e + 1], b1[e], b1[e + 1], true);
-        }
-      } else {
-#pragma unroll
-        for (int e = 0; e < 32; e += 2) {
-          pair(e, a0[e], a0[e + 1], b0[e], b0[e + 1], false);
-          pair(e + 32, a1[e], a1[e + 1], b1[e], b1[e + 1], false);
-        }
+      for (int e = 0; e < 32; e += 2) {
+        pair(e, a0[e], a0[e + 1], b0[e], b0[e + 1]);
+        pair(e + 32, a1[e], a1[e + 1], b1[e], b1[e + 1]);
       }
       const int b = j & 1;
-      if (j >= 2 && !(ok = warp_wait(&bars->dsdone[b], ((j - 2) >> 1) & 1, abort, kStatus))) break;
+      if (j >= 2 && !(ok = warp_wait(&bars->dsdone[b], ((j - 2) >> 1) & 1, abort, kStatus))) return;
       store_row_half(sDS + b * 32768 + h * 16384, r, pd);
       fence_async_smem();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars->ds_full[b]);
-    }
+    };
+    for (int j = 0; j < n - 1 && ok; ++j) step(j, std::false_type{});
+    if (ok) step(n - 1, std::true_type{});
     if (ok) ok = warp_wait(&bars->dsdone[(n - 1) & 1], ((n - 1) >> 1) & 1, abort, kStatus);
     if (ok) {
       tc_fence_after();
