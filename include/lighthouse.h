@@ -178,11 +178,12 @@ lh_status lh_subseq_attn_bwd(const lh_shape* shape, const void* qs, const void* 
  * under a memory planner which has already reserved every byte of the GPU, or
  * a runtime where calling cudaMalloc mid-step is not allowed because it can
  * synchronise the device.  The paper has no counterpart: this is a library
- * convenience, not part of the method.  It allocates nothing: its scratch (one
- * fp32 per row, the D vector) is a fixed 4 MiB array inside the library that
- * every GPU loading the library holds until the process exits.
- *   - At most 1,048,576 rows (B * H * S); larger shapes return
- *     LH_ERR_WORKSPACE before anything is enqueued.
+ * convenience, not part of the method.  It allocates nothing: its scratch (two
+ * fp32 per row, the softmax statistics, rows padded to whole 128-row tiles) is
+ * a fixed 8 MiB array inside the library that every GPU loading the library
+ * holds until the process exits.
+ *   - At most 1,048,576 padded rows (B * H * ceil(S / 128) * 128); larger
+ *     shapes return LH_ERR_WORKSPACE before anything is enqueued.
  *   - All calls on one device share that array: calls whose kernels overlap on
  *     the GPU (unordered streams) race; calls ordered on one stream are safe.
  *   - The first call on each device looks up the array's device address and

@@ -253,7 +253,7 @@ template <int D>
 __global__ void __launch_bounds__(128) k_attn_bwd_dkdv_mma(
     const __half* __restrict__ qs, const __half* __restrict__ ks,
     const __half* __restrict__ vs, const __half* __restrict__ dos,
-    const float* __restrict__ lse, const float* __restrict__ Dv, float* __restrict__ dks,
+    const float* __restrict__ stats, float* __restrict__ dks,
     float* __restrict__ dvs, int64_t S, float scale, float scale_log2, int ntiles) {
   constexpr int BK = 64, BQ = 64, ST = Tile<D>::kStride;
   extern __shared__ __align__(16) unsigned char smem_raw[];
@@ -270,16 +270,17 @@ __global__ void __launch_bounds__(128) k_attn_bwd_dkdv_mma(
   const int64_t k0 = (int64_t)kt * BK;
   const __half* Qg = qs + u * S * D;
   const __half* dOg = dos + u * S * D;
-  const float* Lg = lse + u * S;
-  const float* Dg = Dv + u * S;
+  // tile-padded statistics of this unit: -lse2 and -D per 128-row tile
+  const float* Stu = stats + u * ((S + 127) / 128) * 256;
 
   auto load_q = [&](int i, int stage) {
     load_tile<D, BQ>(sQ + stage * BQ * ST, Qg, (int64_t)i * BQ, S);
     load_tile<D, BQ>(sdO + stage * BQ * ST, dOg, (int64_t)i * BQ, S);
     if (threadIdx.x < BQ) {
       const int64_t r = (int64_t)i * BQ + threadIdx.x;
-      sL[stage * BQ + threadIdx.x] = r < S ? Lg[r] * kLog2e : 0.0f;
-      sD[stage * BQ + threadIdx.x] = r < S ? Dg[r] : 0.0f;
+      // padded rows read lse2 = +inf (P = 0) and D = 0
+      sL[stage * BQ + threadIdx.x] = -Stu[(r >> 7) * 256 + (r & 127)];
+      sD[stage * BQ + threadIdx.x] = -Stu[(r >> 7) * 256 + 128 + (r & 127)];
     }
   };
   load_tile<D, BK>(sK, ks + u * S * D, k0, S);
@@ -384,7 +385,7 @@ template <int D>
 __global__ void __launch_bounds__(128) k_attn_bwd_dq_mma(
     const __half* __restrict__ qs, const __half* __restrict__ ks,
     const __half* __restrict__ vs, const __half* __restrict__ dos,
-    const float* __restrict__ lse, const float* __restrict__ Dv, float* __restrict__ dqs,
+    const float* __restrict__ stats, float* __restrict__ dqs,
     int64_t S, float scale, float scale_log2, int ntiles) {
   constexpr int BM = 64, BN = 64, ST = Tile<D>::kStride;
   extern __shared__ __align__(16) unsigned char smem_raw[];
@@ -406,10 +407,11 @@ __global__ void __launch_bounds__(128) k_attn_bwd_dq_mma(
   cp_async_commit();
 
   const int64_t row_a = q0 + warp * 16 + (l >> 2), row_b = row_a + 8;
-  const float l2a = row_a < S ? lse[u * S + row_a] * kLog2e : 0.0f;
-  const float l2b = row_b < S ? lse[u * S + row_b] * kLog2e : 0.0f;
-  const float Da = row_a < S ? Dv[u * S + row_a] : 0.0f;
-  const float Db = row_b < S ? Dv[u * S + row_b] : 0.0f;
+  const float* Stu = stats + u * ((S + 127) / 128) * 256;
+  const float l2a = -Stu[(row_a >> 7) * 256 + (row_a & 127)];
+  const float l2b = -Stu[(row_b >> 7) * 256 + (row_b & 127)];
+  const float Da = -Stu[(row_a >> 7) * 256 + 128 + (row_a & 127)];
+  const float Db = -Stu[(row_b >> 7) * 256 + 128 + (row_b & 127)];
 
   float dq[D / 8][4];
 #pragma unroll
@@ -520,10 +522,10 @@ cudaError_t fwd_d(const Geom& g, const __half* qs, const __half* ks,
 
 template <int D>
 cudaError_t bwd_d(const Geom& g, const __half* qs, const __half* ks,
-                  const __half* vs, const __half* dos, const float* lse,
-                  const float* Dv, float scale, float* dqs, float* dks, float* dvs,
-                  cudaStream_t st) {
+                  const __half* vs, const __half* dos, const float* stats, float scale,
+                  float* dqs, float* dks, float* dvs, cudaStream_t st) {
   const int ntiles = (int)((g.S + 63) / 64);
+  const int64_t T = (g.S + 127) / 128;  // 128-row tiles of the statistics
   cudaError_t e = cudaFuncSetAttribute(k_attn_bwd_dkdv_mma<D>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)dkdv_smem<D>());
@@ -535,10 +537,10 @@ cudaError_t bwd_d(const Geom& g, const __half* qs, const __half* ks,
     const int64_t nu = g.U - u0 < 65535 ? g.U - u0 : 65535;
     const int64_t o = u0 * g.S * D;
     k_attn_bwd_dkdv_mma<D><<<dim3(ntiles, (unsigned)nu), 128, dkdv_smem<D>(), st>>>(
-        qs + o, ks + o, vs + o, dos + o, lse + u0 * g.S, Dv + u0 * g.S, dks + o, dvs + o, g.S,
-        scale, scale * kLog2e, ntiles);
+        qs + o, ks + o, vs + o, dos + o, stats + u0 * T * 256, dks + o, dvs + o, g.S, scale,
+        scale * kLog2e, ntiles);
     k_attn_bwd_dq_mma<D><<<dim3(ntiles, (unsigned)nu), 128, dq_smem<D>(), st>>>(
-        qs + o, ks + o, vs + o, dos + o, lse + u0 * g.S, Dv + u0 * g.S, dqs + o, g.S, scale,
+        qs + o, ks + o, vs + o, dos + o, stats + u0 * T * 256, dqs + o, g.S, scale,
         scale * kLog2e, ntiles);
   }
   return cudaGetLastError();
@@ -554,11 +556,10 @@ cudaError_t launch_attn_fwd_mma(const Geom& g, const __half* qs, const __half* k
 }
 
 cudaError_t launch_attn_bwd_mma(const Geom& g, const __half* qs, const __half* ks,
-                                const __half* vs, const __half* dos,
-                                const float* lse, const float* D, float scale, float* dqs,
-                                float* dks, float* dvs, cudaStream_t st) {
-  return g.d == 64 ? bwd_d<64>(g, qs, ks, vs, dos, lse, D, scale, dqs, dks, dvs, st)
-                   : bwd_d<128>(g, qs, ks, vs, dos, lse, D, scale, dqs, dks, dvs, st);
+                                const __half* vs, const __half* dos, const float* stats,
+                                float scale, float* dqs, float* dks, float* dvs, cudaStream_t st) {
+  return g.d == 64 ? bwd_d<64>(g, qs, ks, vs, dos, stats, scale, dqs, dks, dvs, st)
+                   : bwd_d<128>(g, qs, ks, vs, dos, stats, scale, dqs, dks, dvs, st);
 }
 
 }  // namespace lh

@@ -91,6 +91,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                   int ntiles) {
   using Lt = FwdLayout<D>;
   constexpr int KS = Lt::kKS;
+  static_assert(KS >= 2 && KS <= 3, "FwdBars holds at most 3 stages; the protocol needs 2");
   extern __shared__ __align__(1024) uint8_t smem[];
   if (smem_u32(smem) & 1023u) {
     if (threadIdx.x == 0) report_status(kStatusAttnFwdTimeout | 1u);
@@ -352,7 +353,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 // accumulate in TMEM over all query tiles (fixed order, no atomics).
 struct DkvBars {
   uint64_t kv_full;
-  uint64_t q_full[2], q_empty[2];
+  uint64_t q_full[3], q_empty[3];  // [stage], at most 3 stages
   uint64_t s_full, st_free, p_full, pdone, mma_done;
   uint32_t tmem;
   int abort;
@@ -360,7 +361,7 @@ struct DkvBars {
 
 template <int D>
 struct DkvLayout {
-  static constexpr int kStages = (D == 64) ? 2 : 1;
+  static constexpr int kStages = (D == 64) ? 3 : 1;  // DkvBars holds up to 3
   static constexpr int kTile = 128 * D * 2;
   static constexpr int kK = 0;
   static constexpr int kV = kK + kTile;
@@ -368,9 +369,8 @@ struct DkvLayout {
   static constexpr int kDO = kQ + kStages * kTile;
   static constexpr int kPT = kDO + kStages * kTile;
   static constexpr int kDST = kPT + 32768;
-  static constexpr int kLse = kDST + 32768;
-  static constexpr int kDv = kLse + kStages * 512;
-  static constexpr int kBar = kDv + kStages * 512;
+  static constexpr int kStat = kDST + 32768;  // per stage: -lse2[128], -D[128]
+  static constexpr int kBar = kStat + kStages * 1024;
   static constexpr int kBytes = kBar + (int)sizeof(DkvBars);
 };
 
@@ -378,11 +378,12 @@ template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
     k_attn_bwd_dkdv_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
                        const __grid_constant__ CUtensorMap tv, const __grid_constant__ CUtensorMap tdo,
-                       const float* __restrict__ lse, const float* __restrict__ Dv,
-                       float* __restrict__ dks, float* __restrict__ dvs, int S, int unit0,
+                       const float* __restrict__ stats, float* __restrict__ dks,
+                       float* __restrict__ dvs, int S, int unit0,
                        int nunits, float scale, float scale_log2, int ntiles) {
   using Lt = DkvLayout<D>;
   constexpr int STG = Lt::kStages;
+  static_assert(STG >= 1 && STG <= 3, "DkvBars holds at most 3 stages");
   extern __shared__ __align__(1024) uint8_t smem[];
   if (smem_u32(smem) & 1023u) {
     if (threadIdx.x == 0) report_status(kStatusAttnBwdTimeout | 1u);
@@ -395,8 +396,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* sDO = smem + Lt::kDO;
   uint8_t* sPT = smem + Lt::kPT;
   uint8_t* sDST = smem + Lt::kDST;
-  float* sLse = reinterpret_cast<float*>(smem + Lt::kLse);
-  float* sDv = reinterpret_cast<float*>(smem + Lt::kDv);
+  float* sStat = reinterpret_cast<float*>(smem + Lt::kStat);
   volatile int* abort = &bars->abort;
   constexpr uint32_t kStatus = kStatusAttnBwdTimeout;
 
@@ -408,8 +408,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (threadIdx.x == 0) {
     mbar_init(&bars->kv_full, 1);
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(&bars->q_full[i], 33);
+    for (int i = 0; i < STG; ++i) {
+      mbar_init(&bars->q_full[i], 1);
       mbar_init(&bars->q_empty[i], 1);
     }
     mbar_init(&bars->s_full, 1);
@@ -428,36 +428,25 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tST = tmem, tDPT = tmem + 128, tDV = tmem + 256, tDK = tmem + 256 + D;
 
   if (warp == 8) {
+    // TMA producer: K, V once; per query tile Q, dO and the tile's statistics
     if (lane == 0) {
       mbar_expect_tx(&bars->kv_full, 2 * Lt::kTile);
       for (int h = 0; h < D / 64; ++h) {
         tma_load_3d(sK + h * 16384, &tk, &bars->kv_full, h * 64, kt * 128, u);
         tma_load_3d(sV + h * 16384, &tv, &bars->kv_full, h * 64, kt * 128, u);
       }
-    }
-    int issued = 0;
-    for (int t = 0; t < n; ++t) {
-      const int st = t % STG, i = kt + t;
-      if (t >= STG && !warp_wait(&bars->q_empty[st], ((t - STG) / STG) & 1, abort, kStatus)) break;
-      if (lane == 0) {
-        mbar_expect_tx(&bars->q_full[st], 2 * Lt::kTile);
+      int issued = 0;
+      for (int t = 0; t < n; ++t) {
+        const int st = t % STG, i = kt + t;
+        if (t >= STG && !mbar_wait(&bars->q_empty[st], ((t - STG) / STG) & 1, abort, kStatus)) break;
+        mbar_expect_tx(&bars->q_full[st], 2 * Lt::kTile + 1024);
         for (int h = 0; h < D / 64; ++h) {
           tma_load_3d(sQ + st * Lt::kTile + h * 16384, &tq, &bars->q_full[st], h * 64, i * 128, u);
           tma_load_3d(sDO + st * Lt::kTile + h * 16384, &tdo, &bars->q_full[st], h * 64, i * 128, u);
         }
+        bulk_load(sStat + st * 256, stats + ((int64_t)u * ntiles + i) * 256, 1024, &bars->q_full[st]);
+        issued = t + 1;
       }
-      for (int c = lane; c < 128; c += 32) {
-        const int q = i * 128 + c;
-        const bool in = q < S;
-        // stored negated: -lse*log2(e) and -D; padded queries get -inf, which
-        // makes their P^T (and dS^T) exactly zero
-        sLse[st * 128 + c] = in ? -__ldg(lse + (int64_t)u * S + q) * kLog2e : -INFINITY;
-        sDv[st * 128 + c] = in ? -__ldg(Dv + (int64_t)u * S + q) : 0.0f;
-      }
-      mbar_arrive(&bars->q_full[st]);
-      issued = t + 1;
-    }
-    if (lane == 0) {
       mbar_wait(&bars->kv_full, 0, abort, kStatus, false);
       for (int t = (issued > STG ? issued - STG : 0); t < issued; ++t)
         mbar_wait(&bars->q_full[t % STG], (t / STG) & 1, abort, kStatus, false);
@@ -537,8 +526,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars->st_free);  // S^T, dP^T are in registers now
-      const float4* cl = reinterpret_cast<const float4*>(sLse + st * 128 + h * 64);  // -lse2
-      const float4* cd = reinterpret_cast<const float4*>(sDv + st * 128 + h * 64);   // -D
+      const float4* cl = reinterpret_cast<const float4*>(sStat + st * 256 + h * 64);        // -lse2
+      const float4* cd = reinterpret_cast<const float4*>(sStat + st * 256 + 128 + h * 64);  // -D
       const int lim = r - h * 64;  // query columns e < lim precede the key
       const float2 cc = make_float2(scale_log2, scale_log2);
       uint32_t pp[32], pd[32];
@@ -649,11 +638,12 @@ template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
     k_attn_bwd_dq_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
                      const __grid_constant__ CUtensorMap tv, const __grid_constant__ CUtensorMap tdo,
-                     const float* __restrict__ lse, const float* __restrict__ Dv,
-                     float* __restrict__ dqs, int S, int unit0, int nunits, float scale,
+                     const float* __restrict__ stats, float* __restrict__ dqs, int S,
+                     int unit0, int nunits, float scale,
                      float scale_log2, int ntiles) {
   using Lt = DqLayout<D>;
   constexpr int STG = Lt::kStages;
+  static_assert(STG >= 1 && STG <= 2, "DqBars holds at most 2 stages");
   extern __shared__ __align__(1024) uint8_t smem[];
   if (smem_u32(smem) & 1023u) {
     if (threadIdx.x == 0) report_status(kStatusAttnBwdTimeout | 2u);
@@ -764,8 +754,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t lane_addr = (uint32_t)(qd * 32) << 16;
     const int row = qt * 128 + r;
     const bool in = row < S;
-    const float lse2 = in ? __ldg(lse + (int64_t)u * S + row) * kLog2e : 0.0f;
-    const float Dr = in ? __ldg(Dv + (int64_t)u * S + row) : 0.0f;
+    // -lse*log2(e) and -D of this row (padded rows: -inf and 0, so P = 0)
+    const float* srow = stats + ((int64_t)u * ntiles + qt) * 256 + r;
+    const float nlse2 = __ldg(srow), nD = __ldg(srow + 128);
     bool ok = true;
     // one key tile; kDiag: the last (diagonal) tile, keys past the query masked
     auto step = [&](int j, auto diag_tag) {
@@ -782,8 +773,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars->s_free);
-      const float2 cc = make_float2(scale_log2, scale_log2), nl = make_float2(-lse2, -lse2);
-      const float2 nd = make_float2(-Dr, -Dr);
+      const float2 cc = make_float2(scale_log2, scale_log2), nl = make_float2(nlse2, nlse2);
+      const float2 nd = make_float2(nD, nD);
       const int lim = r - h * 64;  // key columns e > lim follow the query
       uint32_t pd[32];
       auto pair = [&](int e, uint32_t s0, uint32_t s1, uint32_t g0, uint32_t g1) {
@@ -894,8 +885,8 @@ cudaError_t fwd_d(const Geom& g, const __half* qs, const __half* ks, const __hal
 
 template <int D>
 cudaError_t bwd_d(const Geom& g, const __half* qs, const __half* ks, const __half* vs,
-                  const __half* dos, const float* lse, const float* Dv, float scale, float* dqs,
-                  float* dks, float* dvs, cudaStream_t st) {
+                  const __half* dos, const float* stats, float scale, float* dqs, float* dks,
+                  float* dvs, cudaStream_t st) {
   CUtensorMap mq, mk, mv, mdo;
   if (!make_map(&mq, qs, D, g.S, g.U) || !make_map(&mk, ks, D, g.S, g.U) ||
       !make_map(&mv, vs, D, g.S, g.U) || !make_map(&mdo, dos, D, g.S, g.U))
@@ -911,10 +902,10 @@ cudaError_t bwd_d(const Geom& g, const __half* qs, const __half* ks, const __hal
   for (int64_t u0 = 0; u0 < g.U; u0 += per) {
     const int64_t nu = g.U - u0 < per ? g.U - u0 : per;
     k_attn_bwd_dkdv_tc<D><<<(unsigned)(nu * ntiles), kThreads, smem_a, st>>>(
-        mq, mk, mv, mdo, lse, Dv, dks, dvs, (int)g.S, (int)u0, (int)nu, scale, scale * kLog2e,
+        mq, mk, mv, mdo, stats, dks, dvs, (int)g.S, (int)u0, (int)nu, scale, scale * kLog2e,
         ntiles);
     k_attn_bwd_dq_tc<D><<<(unsigned)(nu * ntiles), kThreads, smem_b, st>>>(
-        mq, mk, mv, mdo, lse, Dv, dqs, (int)g.S, (int)u0, (int)nu, scale, scale * kLog2e, ntiles);
+        mq, mk, mv, mdo, stats, dqs, (int)g.S, (int)u0, (int)nu, scale, scale * kLog2e, ntiles);
   }
   return cudaGetLastError();
 }
@@ -946,12 +937,11 @@ cudaError_t launch_attn_fwd_tc(const Geom& g, const __half* qs, const __half* ks
 }
 
 cudaError_t launch_attn_bwd_tc(const Geom& g, const __half* qs, const __half* ks,
-                               const __half* vs, const __half* dos, const float* lse,
-                               const float* Dv, float scale, float* dqs, float* dks, float* dvs,
-                               cudaStream_t st) {
+                               const __half* vs, const __half* dos, const float* stats,
+                               float scale, float* dqs, float* dks, float* dvs, cudaStream_t st) {
   if (g.S > 0x7fffffff || g.U > 0x7fffffff) return cudaErrorInvalidValue;
-  return g.d == 64 ? tc::bwd_d<64>(g, qs, ks, vs, dos, lse, Dv, scale, dqs, dks, dvs, st)
-                   : tc::bwd_d<128>(g, qs, ks, vs, dos, lse, Dv, scale, dqs, dks, dvs, st);
+  return g.d == 64 ? tc::bwd_d<64>(g, qs, ks, vs, dos, stats, scale, dqs, dks, dvs, st)
+                   : tc::bwd_d<128>(g, qs, ks, vs, dos, stats, scale, dqs, dks, dvs, st);
 }
 
 }  // namespace lh

@@ -337,18 +337,36 @@ __global__ void __launch_bounds__(256) k_gather_bwd(
   store8_stream(dv + o, av);
 }
 
-// ---------------------------------------------------------- D = rowsum(dO*O)
+// ------------------------------------------- backward softmax statistics
+// Tile-padded so that one bulk copy brings a 128-row tile's statistics: for
+// unit u and tile t (T tiles per unit), row r = 128 t + c of the sub-sequence,
+//   stats[(u T + t) 256 + c]       = -lse[r] log2(e)
+//   stats[(u T + t) 256 + 128 + c] = -D[r],  D[r] = rowsum(dos[r] * os[r]);
+// rows past S hold -inf and 0, which make every term they enter exactly zero.
 template <int D>
-__global__ void __launch_bounds__(256) k_rowdot(const __half* __restrict__ os,
-                                                const __half* __restrict__ dos,
-                                                float* __restrict__ Dout, int64_t rows) {
-  constexpr int G = D / 8;
+__global__ void __launch_bounds__(256) k_attn_stats(const __half* __restrict__ os,
+                                                    const __half* __restrict__ dos,
+                                                    const float* __restrict__ lse,
+                                                    float* __restrict__ stats, int S, int T,
+                                                    int64_t prows) {
+  constexpr int G = D / 8;  // threads per row, 8 columns each
   const int64_t gt = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-  const int64_t row = gt / G;
-  if (row >= rows) return;
+  const int64_t prow = gt / G;  // padded row over all units
+  if (prow >= prows) return;    // whole groups leave together
   const int c = (int)(gt % G);
+  const int64_t u = prow / ((int64_t)T * 128);
+  const int rr = (int)(prow - u * T * 128);
+  float* dst = stats + (u * T + (rr >> 7)) * 256 + (rr & 127);
+  if (rr >= S) {
+    if (c == 0) {
+      dst[0] = -INFINITY;
+      dst[128] = 0.0f;
+    }
+    return;
+  }
   const int lane = threadIdx.x & 31;
   const unsigned gmask = ((G == 32) ? 0xffffffffu : ((1u << G) - 1u)) << (lane & ~(G - 1));
+  const int64_t row = u * S + rr;
   float a[8], b[8];
   load8(os + row * D + 8 * c, a);
   load8(dos + row * D + 8 * c, b);
@@ -357,7 +375,10 @@ __global__ void __launch_bounds__(256) k_rowdot(const __half* __restrict__ os,
   for (int i = 0; i < 8; ++i) s = __fmaf_rn(a[i], b[i], s);
 #pragma unroll
   for (int off = 1; off < G; off <<= 1) s = __fadd_rn(s, __shfl_xor_sync(gmask, s, off));
-  if (c == 0) Dout[row] = s;
+  if (c == 0) {
+    dst[0] = -lse[row] * 1.4426950408889634f;
+    dst[128] = -s;
+  }
 }
 
 }  // namespace
@@ -508,14 +529,15 @@ cudaError_t launch_gather_bwd(const Geom& g, lh_dtype dt, const float* dqs, cons
   return cudaGetLastError();
 }
 
-cudaError_t launch_attn_rowdot(const Geom& g, const __half* os, const __half* dos,
-                               float* D, cudaStream_t st) {
-  const int64_t rows = g.U * g.S;
-  const unsigned nb = blocks_for(rows * (g.d / 8), 256);
+cudaError_t launch_attn_stats(const Geom& g, const __half* os, const __half* dos,
+                              const float* lse, float* stats, cudaStream_t st) {
+  const int T = (int)((g.S + 127) / 128);
+  const int64_t prows = g.U * T * 128;
+  const unsigned nb = blocks_for(prows * (g.d / 8), 256);
   if (g.d == 64)
-    k_rowdot<64><<<nb, 256, 0, st>>>(os, dos, D, rows);
+    k_attn_stats<64><<<nb, 256, 0, st>>>(os, dos, lse, stats, (int)g.S, T, prows);
   else
-    k_rowdot<128><<<nb, 256, 0, st>>>(os, dos, D, rows);
+    k_attn_stats<128><<<nb, 256, 0, st>>>(os, dos, lse, stats, (int)g.S, T, prows);
   return cudaGetLastError();
 }
 

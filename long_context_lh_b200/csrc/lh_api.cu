@@ -72,12 +72,12 @@ Layout fwd_ws_layout(const Geom& g) {
   return L;
 }
 
-enum BwdRegion { kDos = 0, kDvec, kDqs, kDks, kDvs };
+enum BwdRegion { kDos = 0, kStats, kDqs, kDks, kDvs };
 Layout bwd_ws_layout(const Geom& g) {
   Layout L;
   const size_t US = (size_t)g.U * g.S;
-  L.add(US * g.d * 2);  // dos
-  L.add(US * 4);        // D = rowsum(dos * os)
+  L.add(US * g.d * 2);                // dos
+  L.add(attn_stats_floats(g) * 4);   // softmax statistics, tile-padded
   for (int i = 0; i < 3; ++i) L.add(US * g.d * 4);
   return L;
 }
@@ -141,11 +141,11 @@ lh_status attn_fwd(const Geom& g, const __half* qs, const __half* ks,
 lh_status attn_bwd(const Geom& g, const __half* qs, const __half* ks,
                    const __half* vs, const __half* os, const float* lse,
                    const __half* dos, float scale, float* dqs, float* dks, float* dvs,
-                   float* Dvec, cudaStream_t st) {
-  LH_TRY(launch_attn_rowdot(g, os, dos, Dvec, st));
+                   float* stats, cudaStream_t st) {
+  LH_TRY(launch_attn_stats(g, os, dos, lse, stats, st));
   if (attn_bwd_uses_tc())
-    return cuda_status(launch_attn_bwd_tc(g, qs, ks, vs, dos, lse, Dvec, scale, dqs, dks, dvs, st));
-  return cuda_status(launch_attn_bwd_mma(g, qs, ks, vs, dos, lse, Dvec, scale, dqs, dks, dvs, st));
+    return cuda_status(launch_attn_bwd_tc(g, qs, ks, vs, dos, stats, scale, dqs, dks, dvs, st));
+  return cuda_status(launch_attn_bwd_mma(g, qs, ks, vs, dos, stats, scale, dqs, dks, dvs, st));
 }
 
 }  // namespace
@@ -205,7 +205,7 @@ size_t lh_topk_workspace_bytes(const lh_shape* shape) {
 size_t lh_attn_bwd_workspace_bytes(const lh_shape* shape) {
   if (check_shape(shape) != LH_OK) return 0;
   const Geom g = make_geom(*shape);
-  return align_up((size_t)g.U * g.S * 4);
+  return align_up(attn_stats_floats(g) * 4);
 }
 
 lh_status lh_build_pyramid(const lh_shape* shape, lh_dtype dtype, const void* q, const void* k,
@@ -405,13 +405,13 @@ lh_status lh_backward(const lh_shape* shape, lh_dtype dtype, const void* saved, 
   const float* lse = reinterpret_cast<const float*>(sv + sl.off[kLse]);
   const float* ic = reinterpret_cast<const float*>(sv + sl.off[kInvCnt]);
   auto* dos = reinterpret_cast<__half*>(w + wl.off[kDos]);
-  float* Dvec = reinterpret_cast<float*>(w + wl.off[kDvec]);
+  float* stats = reinterpret_cast<float*>(w + wl.off[kStats]);
   float* dqs = reinterpret_cast<float*>(w + wl.off[kDqs]);
   float* dks = reinterpret_cast<float*>(w + wl.off[kDks]);
   float* dvs = reinterpret_cast<float*>(w + wl.off[kDvs]);
 
   LH_TRY(launch_scatter_bwd(g, dtype, dO, slot, ic, dos, stream));
-  s = attn_bwd(g, qs, ks, vs, os, lse, dos, resolve_scale(g, scale), dqs, dks, dvs, Dvec, stream);
+  s = attn_bwd(g, qs, ks, vs, os, lse, dos, resolve_scale(g, scale), dqs, dks, dvs, stats, stream);
   if (s != LH_OK) return s;
   LH_TRY(launch_gather_bwd(g, dtype, dqs, dks, dvs, slot, ic, dq, dk, dv, stream));
   return LH_OK;

@@ -154,24 +154,26 @@ cudaError_t launch_gather_bwd(const Geom& g, lh_dtype dt, const float* dqs, cons
 cudaError_t launch_gather_pooled(const Geom& g, lh_dtype dt, const void* q, const void* k,
                                  const void* v, const int32_t* idx, __half* qs, __half* ks,
                                  __half* vs, cudaStream_t st);
-cudaError_t launch_attn_rowdot(const Geom& g, const __half* os, const __half* dos,
-                               float* D, cudaStream_t st);
+// Backward softmax statistics in the tile-padded layout both backward
+// implementations read: per unit and 128-row tile, 128 values of -lse*log2(e)
+// then 128 of -rowsum(dos*os); padded rows -inf and 0.
+inline size_t attn_stats_floats(const Geom& g) { return (size_t)g.U * ((g.S + 127) / 128) * 256; }
+cudaError_t launch_attn_stats(const Geom& g, const __half* os, const __half* dos,
+                              const float* lse, float* stats, cudaStream_t st);
 
 // Attention: two implementations with the same contract.
 cudaError_t launch_attn_fwd_mma(const Geom& g, const __half* qs, const __half* ks,
                                 const __half* vs, float scale, __half* os,
                                 float* lse, cudaStream_t st);
 cudaError_t launch_attn_bwd_mma(const Geom& g, const __half* qs, const __half* ks,
-                                const __half* vs, const __half* dos,
-                                const float* lse, const float* D, float scale, float* dqs,
-                                float* dks, float* dvs, cudaStream_t st);
+                                const __half* vs, const __half* dos, const float* stats,
+                                float scale, float* dqs, float* dks, float* dvs, cudaStream_t st);
 cudaError_t launch_attn_fwd_tc(const Geom& g, const __half* qs, const __half* ks,
                                const __half* vs, float scale, __half* os,
                                float* lse, cudaStream_t st);
 cudaError_t launch_attn_bwd_tc(const Geom& g, const __half* qs, const __half* ks,
-                               const __half* vs, const __half* dos,
-                               const float* lse, const float* D, float scale, float* dqs,
-                               float* dks, float* dvs, cudaStream_t st);
+                               const __half* vs, const __half* dos, const float* stats,
+                               float scale, float* dqs, float* dks, float* dvs, cudaStream_t st);
 bool attn_tc_available();      // tcgen05 forward can run on this device
 bool attn_tc_bwd_available();  // tcgen05 backward can run on this device
 bool attn_fwd_uses_tc();       // dispatch decisions (lh_set_attention_impl + availability)

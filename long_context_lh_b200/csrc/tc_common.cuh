@@ -50,17 +50,17 @@ __device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
 __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];\n" ::"r"(smem_u32(bar)) : "memory");
 }
-// Test for completion of phase `parity`; a waiting thread is suspended by the
-// hardware for up to kSuspendNs (woken early when the phase completes), so
-// waiting warps do not spin through issue slots.
-constexpr uint32_t kSuspendNs = 200000;
+// Test for completion of phase `parity` (the hardware may hold the thread for
+// a short, implementation-defined time before answering false).  No suspend
+// hint: the hinted form sleeps in steps and wakes late on the handoffs that
+// sit on the critical path.
 __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
-      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n"
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
       " selp.u32 %0, 1, 0, p;\n}\n"
       : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity), "r"(kSuspendNs)
+      : "r"(smem_u32(bar)), "r"(parity)
       : "memory");
   return ok != 0;
 }
@@ -98,6 +98,16 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volati
 }
 
 // --------------------------------------------------------------------- TMA
+// Untiled bulk copy of `bytes` from global to shared memory, completing on
+// `bar`.  Both addresses 16-byte aligned, bytes a multiple of 16.
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes,
+                                          uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];\n" ::"r"(
+          smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
 // 3-D tiled load (x = column, y = row within a unit, z = unit) into shared
 // memory, completing on `bar` with the bytes it delivers.  x * 2 bytes must be
 // a multiple of 16 (here x is 0 or 64).
