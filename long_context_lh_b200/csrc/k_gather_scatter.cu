@@ -12,6 +12,8 @@
 // coarsest span) and lane c columns [8c, 8c+8): all HBM traffic is 128-bit and
 // coalesced, and every output element is written by exactly one thread in a
 // fixed order of additions (no atomics), so results are bitwise reproducible.
+#include <type_traits>
+
 #include "lh_internal.cuh"
 
 namespace lh {
@@ -174,40 +176,76 @@ __global__ void __launch_bounds__(256) k_gather_pooled(
 
 // ------------------------------------------------------------- scatter-back
 // O[t] = (sum over selected entries covering t, ascending level, of os[slot]) / c_t.
-template <typename Tout, int D>
+// Grid: x = blocks of kRows tokens of one unit, y = unit (offset u0).
+__device__ __forceinline__ float div_count(float x, int cnt) {
+  // dividing by a power of two is exact as a product with its reciprocal;
+  // other counts take the correctly rounded division
+  return (cnt & (cnt - 1)) == 0 ? x * (1.0f / (float)cnt) : __fdiv_rn(x, (float)cnt);
+}
+
+// One thread: column chunk c of R consecutive tokens t0..t0+R-1 (R divides p,
+// t0 a multiple of R), which share every entry of level >= 1; so each thread
+// issues R + L - 1 slot loads and at most as many row loads, all independent.
+__device__ __forceinline__ void unpack8(const uint4& w, float (&x)[8]) {
+  x[0] = h_lo(w.x); x[1] = h_hi(w.x);
+  x[2] = h_lo(w.y); x[3] = h_hi(w.y);
+  x[4] = h_lo(w.z); x[5] = h_hi(w.z);
+  x[6] = h_lo(w.w); x[7] = h_hi(w.w);
+}
+
+template <typename Tout, int D, int L, int R>
 __global__ void __launch_bounds__(256) k_scatter(const __half* __restrict__ os,
                                                  const int32_t* __restrict__ slot,
                                                  Tout* __restrict__ o, float* __restrict__ inv_count,
-                                                 const Lv lv, int64_t rows) {
-  constexpr int G = D / 8;
-  const int64_t gt = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-  const int64_t row = gt / G;  // u * N + t
-  if (row >= rows) return;
-  const int c = (int)(gt % G);
-  const int64_t u = row / lv.N;
-  const int32_t t = (int32_t)(row - u * lv.N);
+                                                 const Lv lv, int64_t u0) {
+  constexpr int G = D / 8, kGroups = 256 / G;
+  constexpr int LC = (L > 1) ? L - 1 : 1;  // coarse levels (array size)
+  const int32_t t0 = ((int32_t)blockIdx.x * kGroups + (int32_t)(threadIdx.x / G)) * R;
+  if (t0 >= lv.N) return;
+  const int c = (int)(threadIdx.x % G);
+  const int64_t u = u0 + blockIdx.y;
   const int32_t* sl = slot + u * lv.M;
-  float acc[8];
+  const __half* src = os + u * lv.S * D + 8 * c;
+  int32_t s0[R], sc[LC];
 #pragma unroll
-  for (int i = 0; i < 8; ++i) acc[i] = 0.0f;
-  int cnt = 0;
-  for (int l = 0; l < lv.L; ++l) {
-    const int32_t s = __ldg(sl + lv.off[l] + lvl_index(lv, t, l));
-    if (s >= 0) {
-      float x[8];
-      load8(os + (u * lv.S + s) * D + 8 * c, x);
+  for (int r = 0; r < R; ++r) s0[r] = __ldg(sl + t0 + r);
 #pragma unroll
-      for (int i = 0; i < 8; ++i) acc[i] = __fadd_rn(acc[i], x[i]);
-      ++cnt;
+  for (int l = 1; l < L; ++l) sc[l - 1] = __ldg(sl + lv.off[l] + lvl_index(lv, t0, l));
+  uint4 w0[R], wc[LC];
+#pragma unroll
+  for (int r = 0; r < R; ++r)
+    if (s0[r] >= 0) w0[r] = __ldg(reinterpret_cast<const uint4*>(src + (int64_t)s0[r] * D));
+#pragma unroll
+  for (int l = 1; l < L; ++l)
+    if (sc[l - 1] >= 0) wc[l - 1] = __ldg(reinterpret_cast<const uint4*>(src + (int64_t)sc[l - 1] * D));
+#pragma unroll
+  for (int r = 0; r < R; ++r) {
+    float acc[8], x[8];
+    int cnt = 0;
+    if (s0[r] >= 0) {
+      unpack8(w0[r], acc);
+      cnt = 1;
+    } else {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) acc[i] = 0.0f;
     }
-  }
-  if (cnt > 0) {
-    const float fc = (float)cnt;
 #pragma unroll
-    for (int i = 0; i < 8; ++i) acc[i] = __fdiv_rn(acc[i], fc);
+    for (int l = 1; l < L; ++l) {  // ascending level, as defined
+      if (sc[l - 1] >= 0) {
+        unpack8(wc[l - 1], x);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) acc[i] = __fadd_rn(acc[i], x[i]);
+        ++cnt;
+      }
+    }
+    if (cnt > 0) {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) acc[i] = div_count(acc[i], cnt);
+    }
+    const int64_t row = u * lv.N + t0 + r;
+    store8_stream(o + row * D + 8 * c, acc);
+    if (inv_count && c == 0) inv_count[row] = cnt > 0 ? __frcp_rn((float)cnt) : 0.0f;
   }
-  store8_stream(o + row * D + 8 * c, acc);
-  if (inv_count && c == 0) inv_count[row] = cnt > 0 ? __frcp_rn((float)cnt) : 0.0f;
 }
 
 // ---------------------------------------------------------- scatter-back bwd
@@ -295,46 +333,57 @@ __global__ void __launch_bounds__(256) k_scatter_bwd(const Tin* __restrict__ dO,
 
 // --------------------------------------------------------------- gather bwd
 // dX[t] = sum_{l ascending, selected} dxs[slot_l(t)] / p^l, X in {Q, K, V}.
-template <typename Tout, int D>
+// Grid: x = blocks of kRows tokens of one unit, y = unit (offset u0).
+// One thread: column chunk c of R consecutive tokens sharing every entry of
+// level >= 1 (as in the scatter); the slots are looked up once and the three
+// arrays are done one after the other, each as one batch of independent loads.
+template <typename Tout, int D, int L, int R>
 __global__ void __launch_bounds__(256) k_gather_bwd(
     const float* __restrict__ dqs, const float* __restrict__ dks, const float* __restrict__ dvs,
-    const int32_t* __restrict__ slot, const float* __restrict__ inv_count, Tout* __restrict__ dq,
-    Tout* __restrict__ dk, Tout* __restrict__ dv, const Lv lv, int64_t rows) {
-  constexpr int G = D / 8;
-  const int64_t gt = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-  const int64_t row = gt / G;  // u * N + t
-  if (row >= rows) return;
-  const int c = (int)(gt % G);
-  const int64_t u = row / lv.N;
-  const int32_t t = (int32_t)(row - u * lv.N);
+    const int32_t* __restrict__ slot, Tout* __restrict__ dq, Tout* __restrict__ dk,
+    Tout* __restrict__ dv, const Lv lv, int64_t u0) {
+  constexpr int G = D / 8, kGroups = 256 / G;
+  constexpr int LC = (L > 1) ? L - 1 : 1;
+  const int32_t t0 = ((int32_t)blockIdx.x * kGroups + (int32_t)(threadIdx.x / G)) * R;
+  if (t0 >= lv.N) return;
+  const int c = (int)(threadIdx.x % G);
+  const int64_t u = u0 + blockIdx.y;
   const int32_t* sl = slot + u * lv.M;
-  float aq[8], ak[8], av[8];
+  const int64_t base = u * lv.S * D + 8 * c;
+  int32_t s0[R], sc[LC];
 #pragma unroll
-  for (int i = 0; i < 8; ++i) aq[i] = ak[i] = av[i] = 0.0f;
-  // a token with no selected entry covering it (known from the forward's counts)
-  // gets zero gradients without any slot lookups
-  const int nl = (inv_count && __ldg(inv_count + row) == 0.0f) ? 0 : lv.L;
-  for (int l = 0; l < nl; ++l) {
-    const int32_t s = __ldg(sl + lv.off[l] + lvl_index(lv, t, l));
-    if (s >= 0) {
-      const float inv = __frcp_rn((float)lv.pw[l]);
-      const int64_t o = (u * lv.S + s) * D + 8 * c;
-      float x[8];
-      load8(dqs + o, x);
+  for (int r = 0; r < R; ++r) s0[r] = __ldg(sl + t0 + r);
 #pragma unroll
-      for (int i = 0; i < 8; ++i) aq[i] = __fmaf_rn(x[i], inv, aq[i]);
-      load8(dks + o, x);
+  for (int l = 1; l < L; ++l) sc[l - 1] = __ldg(sl + lv.off[l] + lvl_index(lv, t0, l));
+  float inv[LC];
 #pragma unroll
-      for (int i = 0; i < 8; ++i) ak[i] = __fmaf_rn(x[i], inv, ak[i]);
-      load8(dvs + o, x);
+  for (int l = 1; l < L; ++l) inv[l - 1] = __frcp_rn((float)lv.pw[l]);
 #pragma unroll
-      for (int i = 0; i < 8; ++i) av[i] = __fmaf_rn(x[i], inv, av[i]);
+  for (int a = 0; a < 3; ++a) {
+    const float* src = (a == 0 ? dqs : a == 1 ? dks : dvs) + base;
+    Tout* dst = (a == 0 ? dq : a == 1 ? dk : dv) + (u * lv.N + t0) * D + 8 * c;
+    float x0[R][8], xc[LC][8];
+#pragma unroll
+    for (int r = 0; r < R; ++r)
+      if (s0[r] >= 0) load8(src + (int64_t)s0[r] * D, x0[r]);
+#pragma unroll
+    for (int l = 1; l < L; ++l)
+      if (sc[l - 1] >= 0) load8(src + (int64_t)sc[l - 1] * D, xc[l - 1]);
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+      float acc[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) acc[i] = s0[r] >= 0 ? x0[r][i] : 0.0f;  // level 0: weight 1
+#pragma unroll
+      for (int l = 1; l < L; ++l) {  // ascending level
+        if (sc[l - 1] >= 0) {
+#pragma unroll
+          for (int i = 0; i < 8; ++i) acc[i] = __fmaf_rn(xc[l - 1][i], inv[l - 1], acc[i]);
+        }
+      }
+      store8_stream(dst + (int64_t)r * D, acc);
     }
   }
-  const int64_t o = row * D + 8 * c;
-  store8_stream(dq + o, aq);
-  store8_stream(dk + o, ak);
-  store8_stream(dv + o, av);
 }
 
 // ------------------------------------------- backward softmax statistics
@@ -448,25 +497,87 @@ cudaError_t launch_gather_pooled(const Geom& g, lh_dtype dt, const void* q, cons
                    : gather_pooled_d<float, 128>(g, a, b, c, idx, qs, ks, vs, st);
 }
 
-cudaError_t launch_scatter(const Geom& g, lh_dtype dt, const __half* os,
-                           const int32_t* slot, void* o, float* inv_count, cudaStream_t st) {
-  const Lv lv = make_lv(g);
-  const int64_t rows = g.U * g.N;
-  const unsigned nb = blocks_for(rows * (g.d / 8), 256);
-  if (dt == LH_BF16) {
-    auto* out = static_cast<__nv_bfloat16*>(o);
-    if (g.d == 64)
-      k_scatter<__nv_bfloat16, 64><<<nb, 256, 0, st>>>(os, slot, out, inv_count, lv, rows);
-    else
-      k_scatter<__nv_bfloat16, 128><<<nb, 256, 0, st>>>(os, slot, out, inv_count, lv, rows);
-  } else {
-    auto* out = static_cast<float*>(o);
-    if (g.d == 64)
-      k_scatter<float, 64><<<nb, 256, 0, st>>>(os, slot, out, inv_count, lv, rows);
-    else
-      k_scatter<float, 128><<<nb, 256, 0, st>>>(os, slot, out, inv_count, lv, rows);
+namespace {
+// Runs f(std::integral_constant<int, L>) for the shape's level count.
+template <typename F>
+cudaError_t with_levels(int L, F&& f) {
+  switch (L) {
+    case 1: f(std::integral_constant<int, 1>{}); break;
+    case 2: f(std::integral_constant<int, 2>{}); break;
+    case 3: f(std::integral_constant<int, 3>{}); break;
+    case 4: f(std::integral_constant<int, 4>{}); break;
+    case 5: f(std::integral_constant<int, 5>{}); break;
+    case 6: f(std::integral_constant<int, 6>{}); break;
+    case 7: f(std::integral_constant<int, 7>{}); break;
+    case 8: f(std::integral_constant<int, 8>{}); break;
+    default: return cudaErrorInvalidValue;
   }
   return cudaGetLastError();
+}
+
+// 2-D grid over (token blocks of one unit, units), units in chunks of 65535.
+template <typename F>
+void per_unit_chunks(int64_t U, F&& f) {
+  for (int64_t u0 = 0; u0 < U; u0 += 65535) f(u0, (unsigned)(U - u0 < 65535 ? U - u0 : 65535));
+}
+
+// Tokens per thread for the scatter and the gather adjoint: R consecutive
+// tokens share all coarser entries when R divides p (and L > 1).
+inline int tokens_per_thread(const Geom& g) {
+  if (g.L < 2) return 1;
+  return g.p % 4 == 0 ? 4 : (g.p % 2 == 0 ? 2 : 1);
+}
+
+template <typename F>
+cudaError_t with_tokens(int R, F&& f) {
+  if (R == 4) return f(std::integral_constant<int, 4>{});
+  if (R == 2) return f(std::integral_constant<int, 2>{});
+  return f(std::integral_constant<int, 1>{});
+}
+
+template <typename Tout, int D>
+cudaError_t scatter_t(const Geom& g, const __half* os, const int32_t* slot, Tout* o,
+                      float* inv_count, cudaStream_t st) {
+  const Lv lv = make_lv(g);
+  const int R = tokens_per_thread(g);
+  const unsigned bx = blocks_for(g.N / R, 256 / (D / 8));
+  return with_tokens(R, [&](auto rc) {
+    return with_levels(g.L, [&](auto lc) {
+      per_unit_chunks(g.U, [&](int64_t u0, unsigned nu) {
+        k_scatter<Tout, D, decltype(lc)::value, decltype(rc)::value>
+            <<<dim3(bx, nu), 256, 0, st>>>(os, slot, o, inv_count, lv, u0);
+      });
+    });
+  });
+}
+
+template <typename Tout, int D>
+cudaError_t gather_bwd_t(const Geom& g, const float* dqs, const float* dks, const float* dvs,
+                         const int32_t* slot, Tout* dq, Tout* dk, Tout* dv, cudaStream_t st) {
+  const Lv lv = make_lv(g);
+  const int R = tokens_per_thread(g);
+  const unsigned bx = blocks_for(g.N / R, 256 / (D / 8));
+  return with_tokens(R, [&](auto rc) {
+    return with_levels(g.L, [&](auto lc) {
+      per_unit_chunks(g.U, [&](int64_t u0, unsigned nu) {
+        k_gather_bwd<Tout, D, decltype(lc)::value, decltype(rc)::value>
+            <<<dim3(bx, nu), 256, 0, st>>>(dqs, dks, dvs, slot, dq, dk, dv, lv, u0);
+      });
+    });
+  });
+}
+}  // namespace
+
+cudaError_t launch_scatter(const Geom& g, lh_dtype dt, const __half* os,
+                           const int32_t* slot, void* o, float* inv_count, cudaStream_t st) {
+  if (dt == LH_BF16) {
+    auto* out = static_cast<__nv_bfloat16*>(o);
+    return g.d == 64 ? scatter_t<__nv_bfloat16, 64>(g, os, slot, out, inv_count, st)
+                     : scatter_t<__nv_bfloat16, 128>(g, os, slot, out, inv_count, st);
+  }
+  auto* out = static_cast<float*>(o);
+  return g.d == 64 ? scatter_t<float, 64>(g, os, slot, out, inv_count, st)
+                   : scatter_t<float, 128>(g, os, slot, out, inv_count, st);
 }
 
 namespace {
@@ -504,29 +615,20 @@ cudaError_t launch_scatter_bwd(const Geom& g, lh_dtype dt, const void* dO, const
 }
 
 cudaError_t launch_gather_bwd(const Geom& g, lh_dtype dt, const float* dqs, const float* dks,
-                              const float* dvs, const int32_t* slot, const float* inv_count,
-                              void* dq, void* dk, void* dv, cudaStream_t st) {
-  const Lv lv = make_lv(g);
-  const int64_t rows = g.U * g.N;
-  const unsigned nb = blocks_for(rows * (g.d / 8), 256);
+                              const float* dvs, const int32_t* slot, void* dq, void* dk, void* dv,
+                              cudaStream_t st) {
   if (dt == LH_BF16) {
     auto* a = static_cast<__nv_bfloat16*>(dq);
     auto* b = static_cast<__nv_bfloat16*>(dk);
     auto* c = static_cast<__nv_bfloat16*>(dv);
-    if (g.d == 64)
-      k_gather_bwd<__nv_bfloat16, 64><<<nb, 256, 0, st>>>(dqs, dks, dvs, slot, inv_count, a, b, c, lv, rows);
-    else
-      k_gather_bwd<__nv_bfloat16, 128><<<nb, 256, 0, st>>>(dqs, dks, dvs, slot, inv_count, a, b, c, lv, rows);
-  } else {
-    auto* a = static_cast<float*>(dq);
-    auto* b = static_cast<float*>(dk);
-    auto* c = static_cast<float*>(dv);
-    if (g.d == 64)
-      k_gather_bwd<float, 64><<<nb, 256, 0, st>>>(dqs, dks, dvs, slot, inv_count, a, b, c, lv, rows);
-    else
-      k_gather_bwd<float, 128><<<nb, 256, 0, st>>>(dqs, dks, dvs, slot, inv_count, a, b, c, lv, rows);
+    return g.d == 64 ? gather_bwd_t<__nv_bfloat16, 64>(g, dqs, dks, dvs, slot, a, b, c, st)
+                     : gather_bwd_t<__nv_bfloat16, 128>(g, dqs, dks, dvs, slot, a, b, c, st);
   }
-  return cudaGetLastError();
+  auto* a = static_cast<float*>(dq);
+  auto* b = static_cast<float*>(dk);
+  auto* c = static_cast<float*>(dv);
+  return g.d == 64 ? gather_bwd_t<float, 64>(g, dqs, dks, dvs, slot, a, b, c, st)
+                   : gather_bwd_t<float, 128>(g, dqs, dks, dvs, slot, a, b, c, st);
 }
 
 cudaError_t launch_attn_stats(const Geom& g, const __half* os, const __half* dos,

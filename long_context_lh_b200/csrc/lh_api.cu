@@ -345,7 +345,7 @@ lh_status lh_gather_bwd(const lh_shape* shape, lh_dtype dtype, const float* dqs,
       !aligned16(dq) || !aligned16(dk) || !aligned16(dv))
     return LH_ERR_INVALID_ARG;
   return cuda_status(
-      launch_gather_bwd(make_geom(*shape), dtype, dqs, dks, dvs, slot, nullptr, dq, dk, dv, stream));
+      launch_gather_bwd(make_geom(*shape), dtype, dqs, dks, dvs, slot, dq, dk, dv, stream));
 }
 
 lh_status lh_forward(const lh_shape* shape, lh_dtype dtype, const void* q, const void* k,
@@ -413,7 +413,7 @@ lh_status lh_backward(const lh_shape* shape, lh_dtype dtype, const void* saved, 
   LH_TRY(launch_scatter_bwd(g, dtype, dO, slot, ic, dos, stream));
   s = attn_bwd(g, qs, ks, vs, os, lse, dos, resolve_scale(g, scale), dqs, dks, dvs, stats, stream);
   if (s != LH_OK) return s;
-  LH_TRY(launch_gather_bwd(g, dtype, dqs, dks, dvs, slot, ic, dq, dk, dv, stream));
+  LH_TRY(launch_gather_bwd(g, dtype, dqs, dks, dvs, slot, dq, dk, dv, stream));
   return LH_OK;
 }
 

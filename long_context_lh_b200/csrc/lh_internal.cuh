@@ -149,8 +149,8 @@ cudaError_t launch_scatter(const Geom& g, lh_dtype dt, const __half* os,
 cudaError_t launch_scatter_bwd(const Geom& g, lh_dtype dt, const void* dO, const int32_t* slot,
                                const float* inv_count, __half* dos, cudaStream_t st);
 cudaError_t launch_gather_bwd(const Geom& g, lh_dtype dt, const float* dqs, const float* dks,
-                              const float* dvs, const int32_t* slot, const float* inv_count,
-                              void* dq, void* dk, void* dv, cudaStream_t st);
+                              const float* dvs, const int32_t* slot, void* dq, void* dk, void* dv,
+                              cudaStream_t st);
 cudaError_t launch_gather_pooled(const Geom& g, lh_dtype dt, const void* q, const void* k,
                                  const void* v, const int32_t* idx, __half* qs, __half* ks,
                                  __half* vs, cudaStream_t st);
