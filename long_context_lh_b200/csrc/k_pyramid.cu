@@ -6,57 +6,74 @@
 // per entry, coarse levels inherit the max of their children); the averaging is
 // phase 1 ("Pyramid Pool") of bitsgeniais.com.br "Adeus Custo Quadrático! ...".
 //
-// Work decomposition: a group of G = d/8 consecutive lanes owns one coarsest
-// span (p^(L-1) tokens) of one unit; lane c owns columns [8c, 8c+8).  The group
-// walks its span row by row with 128-bit loads, so every element of Q, K and V
-// is read from HBM exactly once, and keeps one running sum per level in
-// registers: when p children of level l are complete their mean is written and
-// added to level l+1.  The level-0 score needs the whole row, so the G lanes
-// combine their partial sums of squares with an xor-shuffle tree that yields
-// the same bits in every lane.
+// Work decomposition.  A block owns a chunk of CR consecutive tokens of one
+// unit (CR = m p^J <= 64, J the highest level whose entries fit in a chunk).
+// It copies the chunk's rows of Q, K (and V) into shared memory with 16-byte
+// asynchronous copies -- every element is read from HBM once, and the several
+// blocks resident per SM keep enough copies in flight to cover the latency --
+// then computes, from shared memory:
+//   level 0   the scores, G = d/8 lanes per row, lane c owning columns [8c, 8c+8);
+//   level l   (1 <= l <= J) one thread per (entry, 8-column chunk, tensor): the
+//             sum of the p children in order, then the mean; the max of the
+//             children's scores.  Level l is kept in shared memory (fp32) for l+1.
+// Levels above J (entries wider than a chunk) are built by a small kernel per
+// level from the level below in HBM; for p^(L-1) <= 64 there are none.
 //
-// Score arithmetic (fixed, so the selection is reproducible bit for bit):
-//   a_c = fmaf chain over x[8c+0..7]^2 from 0;  tree over c with offsets
-//   1, 2, 4(, 8);  score = sqrt_rn(ss(Q)) + sqrt_rn(ss(K)).
+// Arithmetic (fixed, so the selection is reproducible bit for bit):
+//   score:  a_c = fmaf chain over x[8c+0..7]^2 from 0; tree over c with offsets
+//           1, 2, 4(, 8); score = sqrt_rn(ss(Q)) + sqrt_rn(ss(K));
+//           coarse score = max(0, children in order) (scores are >= 0);
+//   mean:   ((0 + c_0) + c_1) + ... + c_{p-1}, then / p (round to nearest; for
+//           p a power of two the product with 1/p, which is the same number).
+#include <type_traits>
+
 #include "lh_internal.cuh"
 
 namespace lh {
 namespace {
 
-struct PyrParams {
-  int64_t N, M, spans, groups, Ptop;
-  int p;
-  int64_t off[kMaxLevels + 1];
-  int64_t pw[kMaxLevels + 1];
+constexpr int kChunkRows = 64;  // upper bound on CR
+
+struct PyrPrm {
+  int32_t N, M, CR, p, J, L;
+  int32_t pow2;  // p is a power of two: mean = sum * inv_p exactly
+  float inv_p;
+  int32_t off[kMaxLevels + 1];
+  int32_t pw[kMaxLevels + 1];
 };
 
-template <typename T>
-struct Raw;
-template <>
-struct Raw<__nv_bfloat16> {
-  uint4 w;
-  __device__ __forceinline__ void load(const __nv_bfloat16* p) {
-    w = __ldcs(reinterpret_cast<const uint4*>(p));
-  }
-  __device__ __forceinline__ void unpack(float (&x)[8]) const {
-    x[0] = bf16_lo(w.x); x[1] = bf16_hi(w.x);
-    x[2] = bf16_lo(w.y); x[3] = bf16_hi(w.y);
-    x[4] = bf16_lo(w.z); x[5] = bf16_hi(w.z);
-    x[6] = bf16_lo(w.w); x[7] = bf16_hi(w.w);
-  }
-};
-template <>
-struct Raw<float> {
-  float4 a, b;
-  __device__ __forceinline__ void load(const float* p) {
-    a = __ldcs(reinterpret_cast<const float4*>(p));
-    b = __ldcs(reinterpret_cast<const float4*>(p) + 1);
-  }
-  __device__ __forceinline__ void unpack(float (&x)[8]) const {
-    x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w;
-    x[4] = b.x; x[5] = b.y; x[6] = b.z; x[7] = b.w;
-  }
-};
+__device__ __forceinline__ float mean_of(float sum, const PyrPrm& prm) {
+  return prm.pow2 ? sum * prm.inv_p : __fdiv_rn(sum, (float)prm.p);
+}
+
+__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(
+                   (uint32_t)__cvta_generic_to_shared(dst)),
+               "l"(src)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() {
+  asm volatile("cp.async.commit_group;\ncp.async.wait_group 0;\n" ::: "memory");
+}
+
+// 8 consecutive elements of a shared-memory row as float
+__device__ __forceinline__ void smem8(const __nv_bfloat16* p, float (&x)[8]) {
+  const uint4 w = *reinterpret_cast<const uint4*>(p);
+  x[0] = bf16_lo(w.x); x[1] = bf16_hi(w.x);
+  x[2] = bf16_lo(w.y); x[3] = bf16_hi(w.y);
+  x[4] = bf16_lo(w.z); x[5] = bf16_hi(w.z);
+  x[6] = bf16_lo(w.w); x[7] = bf16_hi(w.w);
+}
+__device__ __forceinline__ void smem8(const float* p, float (&x)[8]) {
+  const float4 a = *reinterpret_cast<const float4*>(p);
+  const float4 b = *reinterpret_cast<const float4*>(p + 4);
+  x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w;
+  x[4] = b.x; x[5] = b.y; x[6] = b.z; x[7] = b.w;
+}
+__device__ __forceinline__ void put8(float* p, const float (&x)[8]) {
+  *reinterpret_cast<float4*>(p) = make_float4(x[0], x[1], x[2], x[3]);
+  *reinterpret_cast<float4*>(p + 4) = make_float4(x[4], x[5], x[6], x[7]);
+}
 
 __device__ __forceinline__ float sumsq8(const float (&x)[8]) {
   float a = 0.0f;
@@ -65,173 +82,236 @@ __device__ __forceinline__ float sumsq8(const float (&x)[8]) {
   return a;
 }
 
-// Rows of the coarsest span processed per batch of loads (loads issued first).
-constexpr int kRowBatch = 4;
+// Shared memory of the chunk kernel, in bytes.
+template <typename Tin, int D, bool kPyr>
+struct ChunkSmem {
+  static constexpr int NT = kPyr ? 3 : 2;
+  static constexpr size_t in_bytes(int CR) { return (size_t)NT * CR * D * sizeof(Tin); }
+  // two score rows of CR floats, padded so the fp32 level buffers stay 16-byte aligned
+  static constexpr int score_floats(int CR) { return (2 * CR + 3) & ~3; }
+  static constexpr size_t score_bytes(int CR) { return (size_t)score_floats(CR) * sizeof(float); }
+  // ping-pong fp32 level buffers: A holds CR/p rows per tensor, B CR/p^2 (>= 1)
+  static size_t lev_rows_a(int CR, int p) { return (size_t)(CR / p); }
+  static size_t lev_rows_b(int CR, int p) { return (size_t)(CR / p / p > 0 ? CR / p / p : 1); }
+  static size_t bytes(int CR, int p) {
+    size_t b = in_bytes(CR) + score_bytes(CR);
+    if (kPyr) b += (size_t)3 * (lev_rows_a(CR, p) + lev_rows_b(CR, p)) * D * sizeof(float);
+    return b;
+  }
+};
 
-template <typename Tin, int D, int L, bool kPyr, bool kScore>
-__global__ void __launch_bounds__(256) k_pyramid_score(
+template <typename Tin, int D, bool kPyr, bool kScore>
+__global__ void __launch_bounds__(256) k_pyr_chunk(
     const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin* __restrict__ v,
     float* __restrict__ pq, float* __restrict__ pk, float* __restrict__ pv,
-    float* __restrict__ score, const PyrParams prm) {
+    float* __restrict__ score, const PyrPrm prm, int64_t u0) {
+  using Sm = ChunkSmem<Tin, D, kPyr>;
   constexpr int G = D / 8;
-  constexpr int NL = (L > 1) ? (L - 1) : 1;  // accumulators for levels 1..L-1
-  const int64_t gtid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-  const int64_t group = gtid / G;
-  const int c = (int)(gtid % G);
-  if (group >= prm.groups) return;  // whole groups leave together (G | 32)
-  const int lane = threadIdx.x & 31;
-  const unsigned gmask = ((G == 32) ? 0xffffffffu : ((1u << G) - 1u)) << (lane & ~(G - 1));
+  constexpr int NT = Sm::NT;
+  extern __shared__ __align__(16) uint8_t smem[];
+  const int CR = prm.CR;
+  Tin* sIn = reinterpret_cast<Tin*>(smem);  // [NT][CR][D]
+  float* sSc = reinterpret_cast<float*>(smem + Sm::in_bytes(CR));  // [2][CR] ping-pong
+  float* sLa = sSc + Sm::score_floats(CR);                           // [3][CR/p][D]
+  float* sLb = sLa + (size_t)3 * (CR / prm.p) * D;                   // [3][CR/p^2][D]
+  const int ra = CR / prm.p, rb = (CR / prm.p / prm.p > 0) ? CR / prm.p / prm.p : 1;
 
-  const int64_t u = group / prm.spans;
-  const int64_t t0 = (group % prm.spans) * prm.Ptop;
-  const int64_t row0 = (u * prm.N + t0) * D + 8 * c;
-  const Tin* qp = q + row0;
-  const Tin* kp = k + row0;
-  const Tin* vp = v + row0;
+  const int tid = threadIdx.x;
+  const int32_t t0 = (int32_t)blockIdx.x * CR;
+  const int64_t u = u0 + blockIdx.y;
+  const int rows = (prm.N - t0 < CR) ? prm.N - t0 : CR;  // a multiple of p^J
+
+  // ---- the chunk's rows into shared memory
+  {
+    const int64_t g0 = (u * prm.N + t0) * D;
+    const int n16 = rows * D * (int)sizeof(Tin) / 16;  // 16-byte pieces per tensor
+#pragma unroll
+    for (int t = 0; t < NT; ++t) {
+      const uint8_t* src = reinterpret_cast<const uint8_t*>((t == 0 ? q : t == 1 ? k : v) + g0);
+      uint8_t* dst = reinterpret_cast<uint8_t*>(sIn + (size_t)t * CR * D);
+      for (int i = tid; i < n16; i += 256) cp_async16(dst + 16 * i, src + 16 * i);
+    }
+    cp_async_wait_all();
+    __syncthreads();
+  }
   float* sc = score + u * prm.M;
-  const int64_t pyr_unit = u * (prm.M - prm.N);
 
-  float aq[NL][8], ak[NL][8], av[NL][8];
-  float smax[NL];
-  int cnt[NL];
+  // ---- level 0: scores
+  if (kScore) {
+    const int c = tid % G;
+    const int lane = tid & 31;
+    const unsigned gmask = ((G == 32) ? 0xffffffffu : ((1u << G) - 1u)) << (lane & ~(G - 1));
+    for (int r = tid / G; r < rows; r += 256 / G) {  // whole groups iterate together
+      float xq[8], xk[8];
+      smem8(sIn + (size_t)r * D + 8 * c, xq);
+      smem8(sIn + (size_t)(CR + r) * D + 8 * c, xk);
+      float ssq = sumsq8(xq), ssk = sumsq8(xk);
 #pragma unroll
-  for (int l = 0; l < NL; ++l) {
-    smax[l] = 0.0f;
-    cnt[l] = 0;
-#pragma unroll
-    for (int i = 0; i < 8; ++i) aq[l][i] = ak[l][i] = av[l][i] = 0.0f;
+      for (int off = 1; off < G; off <<= 1) {
+        ssq = __fadd_rn(ssq, __shfl_xor_sync(gmask, ssq, off));
+        ssk = __fadd_rn(ssk, __shfl_xor_sync(gmask, ssk, off));
+      }
+      if (c == 0) sSc[r] = __fadd_rn(__fsqrt_rn(ssq), __fsqrt_rn(ssk));
+    }
+    __syncthreads();
+    for (int r = tid; r < rows; r += 256) sc[t0 + r] = sSc[r];
   }
 
-  for (int64_t r0 = 0; r0 < prm.Ptop; r0 += kRowBatch) {
-    Raw<Tin> rq[kRowBatch], rk[kRowBatch], rv[kRowBatch];
+  // ---- levels 1..J
+  int nprev = rows;
+  for (int l = 1; l <= prm.J; ++l) {
+    const int n = nprev / prm.p;
+    const int32_t j0 = t0 / prm.pw[l];  // first entry of this chunk at level l
+    const float* prevS = sSc + ((l - 1) & 1) * CR;
+    float* curS = sSc + (l & 1) * CR;
+    if (kPyr) {
+      const float* prevL = (l & 1) ? sLb : sLa;  // level l-1 (l >= 2)
+      float* curL = (l & 1) ? sLa : sLb;
+      const int prow = (l & 1) ? rb : ra;        // rows per tensor of prevL
+      const int crow = (l & 1) ? ra : rb;        // rows per tensor of curL
+      const int items = 3 * n * G;
+      for (int it = tid; it < items; it += 256) {
+        const int t = it / (n * G);
+        const int rem = it - t * n * G;
+        const int e = rem / G, c = rem - (rem / G) * G;
+        float acc[8], x[8];
 #pragma unroll
-    for (int b = 0; b < kRowBatch; ++b) {
-      if (r0 + b < prm.Ptop) {
-        const int64_t o = (r0 + b) * D;
-        rq[b].load(qp + o);
-        rk[b].load(kp + o);
-        if (kPyr) rv[b].load(vp + o);
+        for (int i = 0; i < 8; ++i) acc[i] = 0.0f;
+        for (int i = 0; i < prm.p; ++i) {
+          const int ch = e * prm.p + i;
+          if (l == 1)
+            smem8(sIn + ((size_t)t * CR + ch) * D + 8 * c, x);
+          else
+            smem8(prevL + ((size_t)t * prow + ch) * D + 8 * c, x);
+#pragma unroll
+          for (int z = 0; z < 8; ++z) acc[z] = __fadd_rn(acc[z], x[z]);
+        }
+#pragma unroll
+        for (int z = 0; z < 8; ++z) acc[z] = mean_of(acc[z], prm);
+        float* dst = (t == 0 ? pq : t == 1 ? pk : pv);
+        put8(dst + ((u * (prm.M - prm.N) + prm.off[l] - prm.N + j0 + e) * D + 8 * c), acc);
+        if (l < prm.J) put8(curL + ((size_t)t * crow + e) * D + 8 * c, acc);
       }
     }
-#pragma unroll
-    for (int b = 0; b < kRowBatch; ++b) {
-      const int64_t r = r0 + b;
-      if (r >= prm.Ptop) break;
-      float xq[8], xk[8], xv[8];
-      rq[b].unpack(xq);
-      rk[b].unpack(xk);
-      if (kPyr) rv[b].unpack(xv);
-      // level-0 score (all lanes of the group end with identical bits)
-      float s0 = 0.0f;
-      if (kScore) {
-        float ssq = sumsq8(xq), ssk = sumsq8(xk);
-#pragma unroll
-        for (int off = 1; off < G; off <<= 1) {
-          ssq = __fadd_rn(ssq, __shfl_xor_sync(gmask, ssq, off));
-          ssk = __fadd_rn(ssk, __shfl_xor_sync(gmask, ssk, off));
-        }
-        s0 = __fadd_rn(__fsqrt_rn(ssq), __fsqrt_rn(ssk));
-        if (c == (int)(r % G)) sc[t0 + r] = s0;
-      }
-      if constexpr (L == 1) continue;
-      // feed level 1
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        if (kPyr) {
-          aq[0][i] = __fadd_rn(aq[0][i], xq[i]);
-          ak[0][i] = __fadd_rn(ak[0][i], xk[i]);
-          av[0][i] = __fadd_rn(av[0][i], xv[i]);
-        }
-      }
-      smax[0] = fmaxf(smax[0], s0);
-      cnt[0] += 1;
-      // cascade completed levels upward
-#pragma unroll
-      for (int l = 0; l < NL; ++l) {
-        if (cnt[l] == prm.p) {
-          const int lev = l + 1;
-          const int64_t j = (t0 + r + 1) / prm.pw[lev] - 1;
-          const float fp = (float)prm.p;
-          float mq[8], mk[8], mv[8];
-#pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            mq[i] = __fdiv_rn(aq[l][i], fp);
-            mk[i] = __fdiv_rn(ak[l][i], fp);
-            mv[i] = __fdiv_rn(av[l][i], fp);
-          }
-          if (kPyr) {
-            const int64_t prow = (pyr_unit + prm.off[lev] - prm.N + j) * D + 8 * c;
-            store8(pq + prow, mq);
-            store8(pk + prow, mk);
-            store8(pv + prow, mv);
-          }
-          if (kScore && c == 0) sc[prm.off[lev] + j] = smax[l];
-          if (l + 1 < NL) {
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-              aq[l + 1][i] = __fadd_rn(aq[l + 1][i], mq[i]);
-              ak[l + 1][i] = __fadd_rn(ak[l + 1][i], mk[i]);
-              av[l + 1][i] = __fadd_rn(av[l + 1][i], mv[i]);
-            }
-            smax[l + 1] = fmaxf(smax[l + 1], smax[l]);
-            cnt[l + 1] += 1;
-          }
-#pragma unroll
-          for (int i = 0; i < 8; ++i) aq[l][i] = ak[l][i] = av[l][i] = 0.0f;
-          smax[l] = 0.0f;
-          cnt[l] = 0;
-        }
+    if (kScore) {
+      for (int e = tid; e < n; e += 256) {
+        float m = 0.0f;
+        for (int i = 0; i < prm.p; ++i) m = fmaxf(m, prevS[e * prm.p + i]);
+        curS[e] = m;
+        sc[prm.off[l] + j0 + e] = m;
       }
     }
+    __syncthreads();
+    nprev = n;
   }
 }
 
-template <typename Tin, int D, int L>
-cudaError_t launch_tl(const Geom& g, const void* q, const void* k, const void* v, float* pq,
-                      float* pk, float* pv, float* score, cudaStream_t st) {
-  PyrParams prm;
-  prm.N = g.N;
-  prm.M = g.M;
-  prm.p = g.p;
-  prm.Ptop = g.pw[g.L - 1];
-  prm.spans = g.N / prm.Ptop;
-  prm.groups = g.U * prm.spans;
-  for (int l = 0; l <= kMaxLevels; ++l) {
-    prm.off[l] = g.off[l];
-    prm.pw[l] = g.pw[l];
+// Level l > J from level l-1 in HBM (level 0 being the input): one thread per
+// (entry, 8-column chunk, tensor) for the means, one per entry for the score.
+template <typename Tin, int D, bool kPyr, bool kScore>
+__global__ void __launch_bounds__(256) k_pyr_upper(
+    const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin* __restrict__ v,
+    float* __restrict__ pq, float* __restrict__ pk, float* __restrict__ pv,
+    float* __restrict__ score, const PyrPrm prm, int l, int64_t u0) {
+  constexpr int G = D / 8;
+  const int n = prm.N / prm.pw[l];  // entries of level l per unit
+  const int it = (int)blockIdx.x * 256 + (int)threadIdx.x;
+  const int64_t u = u0 + blockIdx.y;
+  if (kPyr && it < 3 * n * G) {
+    const int t = it / (n * G);
+    const int rem = it - t * n * G;
+    const int e = rem / G, c = rem - (rem / G) * G;
+    float acc[8], x[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) acc[i] = 0.0f;
+    for (int i = 0; i < prm.p; ++i) {
+      const int ch = e * prm.p + i;  // child index at level l-1
+      if (l == 1) {
+        const Tin* src = (t == 0 ? q : t == 1 ? k : v) + (u * prm.N + ch) * D + 8 * c;
+        load8(src, x);
+      } else {
+        const float* src = (t == 0 ? pq : t == 1 ? pk : pv) +
+                           (u * (prm.M - prm.N) + prm.off[l - 1] - prm.N + ch) * D + 8 * c;
+        load8(src, x);
+      }
+#pragma unroll
+      for (int z = 0; z < 8; ++z) acc[z] = __fadd_rn(acc[z], x[z]);
+    }
+#pragma unroll
+    for (int z = 0; z < 8; ++z) acc[z] = mean_of(acc[z], prm);
+    float* dst = (t == 0 ? pq : t == 1 ? pk : pv);
+    float* o = dst + (u * (prm.M - prm.N) + prm.off[l] - prm.N + e) * D + 8 * c;
+    *reinterpret_cast<float4*>(o) = make_float4(acc[0], acc[1], acc[2], acc[3]);
+    *reinterpret_cast<float4*>(o + 4) = make_float4(acc[4], acc[5], acc[6], acc[7]);
   }
-  const int64_t threads = prm.groups * (D / 8);
-  const int block = 256;
-  const int64_t grid = (threads + block - 1) / block;
-  const Tin* tq = static_cast<const Tin*>(q);
-  const Tin* tk = static_cast<const Tin*>(k);
-  const Tin* tv = static_cast<const Tin*>(v);
-  if (pq && score)
-    k_pyramid_score<Tin, D, L, true, true><<<grid, block, 0, st>>>(tq, tk, tv, pq, pk, pv, score, prm);
-  else if (pq)
-    k_pyramid_score<Tin, D, L, true, false><<<grid, block, 0, st>>>(tq, tk, tv, pq, pk, pv, score, prm);
-  else
-    k_pyramid_score<Tin, D, L, false, true><<<grid, block, 0, st>>>(tq, tk, tv, pq, pk, pv, score, prm);
+  if (kScore && it < n) {
+    float* sc = score + u * prm.M;
+    float m = 0.0f;
+    for (int i = 0; i < prm.p; ++i) m = fmaxf(m, sc[prm.off[l - 1] + it * prm.p + i]);
+    sc[prm.off[l] + it] = m;
+  }
+}
+
+PyrPrm make_prm(const Geom& g) {
+  PyrPrm prm;
+  prm.N = (int32_t)g.N;
+  prm.M = (int32_t)g.M;
+  prm.p = g.p;
+  prm.L = g.L;
+  prm.pow2 = (g.p & (g.p - 1)) == 0;
+  prm.inv_p = 1.0f / (float)g.p;  // exact when p is a power of two
+  for (int l = 0; l <= kMaxLevels; ++l) {
+    prm.off[l] = (int32_t)g.off[l];
+    prm.pw[l] = (int32_t)(g.pw[l] > 0x7fffffff ? 0x7fffffff : g.pw[l]);
+  }
+  int J = 0;
+  while (J + 1 <= g.L - 1 && g.pw[J + 1] <= kChunkRows) ++J;
+  prm.J = J;
+  prm.CR = (int32_t)(g.pw[J] * (kChunkRows / g.pw[J]));
+  return prm;
+}
+
+template <typename Tin, int D, bool kPyr, bool kScore>
+cudaError_t launch_flags(const Geom& g, const Tin* q, const Tin* k, const Tin* v, float* pq,
+                         float* pk, float* pv, float* score, cudaStream_t st) {
+  const PyrPrm prm = make_prm(g);
+  const size_t smem = ChunkSmem<Tin, D, kPyr>::bytes(prm.CR, prm.p);
+  auto* kc = k_pyr_chunk<Tin, D, kPyr, kScore>;
+  cudaError_t e = cudaFuncSetAttribute(kc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  const unsigned bx = (unsigned)((g.N + prm.CR - 1) / prm.CR);
+  for (int64_t u0 = 0; u0 < g.U; u0 += 65535) {
+    const unsigned nu = (unsigned)(g.U - u0 < 65535 ? g.U - u0 : 65535);
+    kc<<<dim3(bx, nu), 256, smem, st>>>(q, k, v, pq, pk, pv, score, prm, u0);
+    for (int l = prm.J + 1; l <= g.L - 1; ++l) {
+      const int64_t n = g.N / g.pw[l];
+      const int64_t items = kPyr ? 3 * n * (D / 8) : n;
+      const unsigned ub = (unsigned)((items + 255) / 256);
+      k_pyr_upper<Tin, D, kPyr, kScore><<<dim3(ub, nu), 256, 0, st>>>(q, k, v, pq, pk, pv, score,
+                                                                      prm, l, u0);
+    }
+  }
   return cudaGetLastError();
 }
 
 template <typename Tin, int D>
 cudaError_t launch_t(const Geom& g, const void* q, const void* k, const void* v, float* pq,
                      float* pk, float* pv, float* score, cudaStream_t st) {
-  switch (g.L) {
-    case 1: return launch_tl<Tin, D, 1>(g, q, k, v, pq, pk, pv, score, st);
-    case 2: return launch_tl<Tin, D, 2>(g, q, k, v, pq, pk, pv, score, st);
-    case 3: return launch_tl<Tin, D, 3>(g, q, k, v, pq, pk, pv, score, st);
-    case 4: return launch_tl<Tin, D, 4>(g, q, k, v, pq, pk, pv, score, st);
-    case 5: return launch_tl<Tin, D, 5>(g, q, k, v, pq, pk, pv, score, st);
-    case 6: return launch_tl<Tin, D, 6>(g, q, k, v, pq, pk, pv, score, st);
-    case 7: return launch_tl<Tin, D, 7>(g, q, k, v, pq, pk, pv, score, st);
-    case 8: return launch_tl<Tin, D, 8>(g, q, k, v, pq, pk, pv, score, st);
-  }
-  return cudaErrorInvalidValue;
+  const Tin* tq = static_cast<const Tin*>(q);
+  const Tin* tk = static_cast<const Tin*>(k);
+  const Tin* tv = static_cast<const Tin*>(v);
+  if (pq && score) return launch_flags<Tin, D, true, true>(g, tq, tk, tv, pq, pk, pv, score, st);
+  if (pq) return launch_flags<Tin, D, true, false>(g, tq, tk, tv, pq, pk, pv, score, st);
+  return launch_flags<Tin, D, false, true>(g, tq, tk, tv, pq, pk, pv, score, st);
 }
 
 }  // namespace
+
+int pyramid_launches(const Geom& g) {
+  const PyrPrm prm = make_prm(g);
+  const int64_t chunks = (g.U + 65534) / 65535;
+  return (int)(chunks * (1 + (g.L - 1 - prm.J)));
+}
 
 // pq/pk/pv == nullptr: scores only; score == nullptr: pyramid only.
 cudaError_t launch_pyramid_score(const Geom& g, lh_dtype dt, const void* q, const void* k,

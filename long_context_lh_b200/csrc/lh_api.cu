@@ -440,11 +440,12 @@ int lh_kernel_launches(const lh_shape* shape, int backward) {
   const Geom g = make_geom(*shape);
   const int chunks = (int)((g.U + 65534) / 65535);  // grid.y limit per launch
   if (!backward) {
-    // pyramid+score, top-k (per chunk), gather, attention (per chunk), scatter
-    return 1 + chunks + 1 + (attn_fwd_uses_tc() ? attn_tc_fwd_launches(g) : chunks) + 1;
+    // pyramid+score, top-k (per chunk), gather, attention (per chunk), scatter (per chunk)
+    return pyramid_launches(g) + chunks + 1 +
+           (attn_fwd_uses_tc() ? attn_tc_fwd_launches(g) : chunks) + chunks;
   }
-  // scatter-back bwd, row dot, attention bwd, gather bwd
-  return 1 + 1 + (attn_bwd_uses_tc() ? attn_tc_bwd_launches(g) : 2 * chunks) + 1;
+  // scatter-back bwd, softmax statistics, attention bwd, gather bwd (per chunk)
+  return 1 + 1 + (attn_bwd_uses_tc() ? attn_tc_bwd_launches(g) : 2 * chunks) + chunks;
 }
 
 }  // extern "C"

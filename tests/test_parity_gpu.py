@@ -81,6 +81,8 @@ STAGE_CASES = [
     dict(dtype="bf16", L=1, N=1000, S=333),
     dict(dtype="bf16", p=2, L=2, N=256, S=384),               # S = M: everything selected
     dict(dtype="bf16", N=512, S=1),
+    dict(dtype="bf16", p=4, L=5, N=2048, S=300),             # level 4 wider than a 64-row chunk
+    dict(p=5, L=4, N=1000, S=100),                            # p^3 = 125 > 64, last chunk ragged
 ]
 
 
