@@ -315,7 +315,8 @@ def run_ours(args, rank, world, local_rank):
 def launches_per_step(lh, w):
     """Kernels of this library launched per step (lh_forward + lh_backward)."""
     shp = lh.make_shape(w.B, w.H, w.N, w.d, w.p, w.L, w.S)
-    return lh.lh_kernel_launches(shp, False) + lh.lh_kernel_launches(shp, True)
+    dt = lh.dtype_code(w.torch_dtype)
+    return lh.lh_kernel_launches(shp, dt, False) + lh.lh_kernel_launches(shp, dt, True)
 
 
 def dense_sdpa(w, q, k, v, dO, stream, args):

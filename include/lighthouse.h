@@ -245,9 +245,9 @@ int lh_set_attention_impl(int impl);
 int lh_attention_impl_in_use(void);
 
 /* Number of kernel launches lh_forward (backward = 0) or lh_backward
- * (backward = 1) enqueues for this shape with the current implementation;
- * -1 for an invalid shape. */
-int lh_kernel_launches(const lh_shape* shape, int backward);
+ * (backward = 1) enqueues for this shape and input dtype with the current
+ * implementation; -1 for an invalid shape or dtype. */
+int lh_kernel_launches(const lh_shape* shape, lh_dtype dtype, int backward);
 
 #ifdef __cplusplus
 }

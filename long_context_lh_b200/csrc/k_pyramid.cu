@@ -7,17 +7,22 @@
 // phase 1 ("Pyramid Pool") of bitsgeniais.com.br "Adeus Custo Quadrático! ...".
 //
 // Work decomposition.  A block owns a chunk of CR consecutive tokens of one
-// unit (CR = m p^J <= 64, J the highest level whose entries fit in a chunk).
+// unit (CR = m p^J <= 64 rows and <= 8 KB per tensor, J the highest level
+// whose entries fit in a chunk).
 // It copies the chunk's rows of Q, K (and V) into shared memory with 16-byte
 // asynchronous copies -- every element is read from HBM once, and the several
 // blocks resident per SM keep enough copies in flight to cover the latency --
 // then computes, from shared memory:
-//   level 0   the scores, G = d/8 lanes per row, lane c owning columns [8c, 8c+8);
-//   level l   (1 <= l <= J) one thread per (entry, 8-column chunk, tensor): the
-//             sum of the p children in order, then the mean; the max of the
-//             children's scores.  Level l is kept in shared memory (fp32) for l+1.
+//   level 1   one thread per (entry, 8-column chunk c, tensor): the sum of the
+//             p children in order, then the mean; for Q and K the same thread
+//             also forms each child row's partial sum of squares a_c;
+//   level 0   the scores, one thread per row, from the partials a_c;
+//   level l   (2 <= l <= J) as level 1 from level l-1; scores: max of the
+//             children.  Level l is kept in shared memory (fp32) for l+1.
+// (Without level 1 in the chunk -- L = 1, or scores only -- G = d/8 lanes per
+// row form the level-0 scores with a shuffle tree instead.)
 // Levels above J (entries wider than a chunk) are built by a small kernel per
-// level from the level below in HBM; for p^(L-1) <= 64 there are none.
+// level from the level below in HBM; when p^(L-1) fits a chunk there are none.
 //
 // Arithmetic (fixed, so the selection is reproducible bit for bit):
 //   score:  a_c = fmaf chain over x[8c+0..7]^2 from 0; tree over c with offsets
@@ -32,7 +37,12 @@
 namespace lh {
 namespace {
 
-constexpr int kChunkRows = 64;  // upper bound on CR
+// Upper bound on CR: 64 rows and 8 KB of each tensor per chunk (64 rows of
+// bf16 at d = 64).
+inline int chunk_rows_cap(int d, size_t elem) {
+  const int cap = (int)(8192 / ((size_t)d * elem));
+  return cap < 64 ? cap : 64;
+}
 
 struct PyrPrm {
   int32_t N, M, CR, p, J, L;
@@ -95,7 +105,10 @@ struct ChunkSmem {
   static size_t lev_rows_b(int CR, int p) { return (size_t)(CR / p / p > 0 ? CR / p / p : 1); }
   static size_t bytes(int CR, int p) {
     size_t b = in_bytes(CR) + score_bytes(CR);
-    if (kPyr) b += (size_t)3 * (lev_rows_a(CR, p) + lev_rows_b(CR, p)) * D * sizeof(float);
+    if (kPyr) {
+      b += (size_t)3 * (lev_rows_a(CR, p) + lev_rows_b(CR, p)) * D * sizeof(float);
+      b += (size_t)2 * CR * (D / 8) * sizeof(float);  // partial sums of squares
+    }
     return b;
   }
 };
@@ -135,9 +148,11 @@ __global__ void __launch_bounds__(256) k_pyr_chunk(
     __syncthreads();
   }
   float* sc = score + u * prm.M;
+  float* sPart = sLb + (size_t)3 * rb * D;  // [2][CR][G] partial sums of squares (kPyr)
+  const bool fused = kPyr && prm.J >= 1;    // scores from the level-1 pass
 
-  // ---- level 0: scores
-  if (kScore) {
+  // ---- level-0 scores without a level-1 pass: G lanes per row, shuffle tree
+  if (kScore && !fused) {
     const int c = tid % G;
     const int lane = tid & 31;
     const unsigned gmask = ((G == 32) ? 0xffffffffu : ((1u << G) - 1u)) << (lane & ~(G - 1));
@@ -169,20 +184,23 @@ __global__ void __launch_bounds__(256) k_pyr_chunk(
       float* curL = (l & 1) ? sLa : sLb;
       const int prow = (l & 1) ? rb : ra;        // rows per tensor of prevL
       const int crow = (l & 1) ? ra : rb;        // rows per tensor of curL
-      const int items = 3 * n * G;
-      for (int it = tid; it < items; it += 256) {
-        const int t = it / (n * G);
-        const int rem = it - t * n * G;
-        const int e = rem / G, c = rem - (rem / G) * G;
+      const int nG = n * G;
+      for (int it = tid; it < 3 * nG; it += 256) {
+        const int t = it >= 2 * nG ? 2 : (it >= nG ? 1 : 0);
+        const int rem = it - t * nG;
+        const int e = rem / G, c = rem % G;
         float acc[8], x[8];
 #pragma unroll
         for (int i = 0; i < 8; ++i) acc[i] = 0.0f;
         for (int i = 0; i < prm.p; ++i) {
           const int ch = e * prm.p + i;
-          if (l == 1)
+          if (l == 1) {
             smem8(sIn + ((size_t)t * CR + ch) * D + 8 * c, x);
-          else
+            // the child row's partial a_c of its score (Q and K)
+            if (kScore && t < 2) sPart[((size_t)t * CR + ch) * G + c] = sumsq8(x);
+          } else {
             smem8(prevL + ((size_t)t * prow + ch) * D + 8 * c, x);
+          }
 #pragma unroll
           for (int z = 0; z < 8; ++z) acc[z] = __fadd_rn(acc[z], x[z]);
         }
@@ -194,6 +212,32 @@ __global__ void __launch_bounds__(256) k_pyr_chunk(
       }
     }
     if (kScore) {
+      if (l == 1 && fused) {
+        __syncthreads();  // all partials written
+        // level-0 scores, one thread per row: the same pairwise tree over the
+        // partials a_0..a_{G-1} as the shuffle tree (offsets 1, 2, 4(, 8))
+        for (int r = tid; r < rows; r += 256) {
+          float a[G], b[G];
+#pragma unroll
+          for (int c = 0; c < G; c += 4) {  // 16-byte aligned: G is a multiple of 8
+            const float4 x = *reinterpret_cast<const float4*>(sPart + (size_t)r * G + c);
+            const float4 y = *reinterpret_cast<const float4*>(sPart + ((size_t)CR + r) * G + c);
+            a[c] = x.x; a[c + 1] = x.y; a[c + 2] = x.z; a[c + 3] = x.w;
+            b[c] = y.x; b[c + 1] = y.y; b[c + 2] = y.z; b[c + 3] = y.w;
+          }
+#pragma unroll
+          for (int off = 1; off < G; off <<= 1)
+#pragma unroll
+            for (int c = 0; c < G; c += 2 * off) {
+              a[c] = __fadd_rn(a[c], a[c + off]);
+              b[c] = __fadd_rn(b[c], b[c + off]);
+            }
+          const float s0 = __fadd_rn(__fsqrt_rn(a[0]), __fsqrt_rn(b[0]));
+          sSc[r] = s0;
+          sc[t0 + r] = s0;
+        }
+        __syncthreads();
+      }
       for (int e = tid; e < n; e += 256) {
         float m = 0.0f;
         for (int i = 0; i < prm.p; ++i) m = fmaxf(m, prevS[e * prm.p + i]);
@@ -252,7 +296,7 @@ __global__ void __launch_bounds__(256) k_pyr_upper(
   }
 }
 
-PyrPrm make_prm(const Geom& g) {
+PyrPrm make_prm(const Geom& g, int cap) {
   PyrPrm prm;
   prm.N = (int32_t)g.N;
   prm.M = (int32_t)g.M;
@@ -265,16 +309,16 @@ PyrPrm make_prm(const Geom& g) {
     prm.pw[l] = (int32_t)(g.pw[l] > 0x7fffffff ? 0x7fffffff : g.pw[l]);
   }
   int J = 0;
-  while (J + 1 <= g.L - 1 && g.pw[J + 1] <= kChunkRows) ++J;
+  while (J + 1 <= g.L - 1 && g.pw[J + 1] <= cap) ++J;
   prm.J = J;
-  prm.CR = (int32_t)(g.pw[J] * (kChunkRows / g.pw[J]));
+  prm.CR = (int32_t)(g.pw[J] * (cap / g.pw[J]));
   return prm;
 }
 
 template <typename Tin, int D, bool kPyr, bool kScore>
 cudaError_t launch_flags(const Geom& g, const Tin* q, const Tin* k, const Tin* v, float* pq,
                          float* pk, float* pv, float* score, cudaStream_t st) {
-  const PyrPrm prm = make_prm(g);
+  const PyrPrm prm = make_prm(g, chunk_rows_cap(D, sizeof(Tin)));
   const size_t smem = ChunkSmem<Tin, D, kPyr>::bytes(prm.CR, prm.p);
   auto* kc = k_pyr_chunk<Tin, D, kPyr, kScore>;
   cudaError_t e = cudaFuncSetAttribute(kc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
@@ -307,8 +351,8 @@ cudaError_t launch_t(const Geom& g, const void* q, const void* k, const void* v,
 
 }  // namespace
 
-int pyramid_launches(const Geom& g) {
-  const PyrPrm prm = make_prm(g);
+int pyramid_launches(const Geom& g, lh_dtype dt) {
+  const PyrPrm prm = make_prm(g, chunk_rows_cap(g.d, dt == LH_BF16 ? 2 : 4));
   const int64_t chunks = (g.U + 65534) / 65535;
   return (int)(chunks * (1 + (g.L - 1 - prm.J)));
 }

@@ -435,13 +435,14 @@ int lh_attention_impl_in_use(void) {
   return f && b ? 0 : (!f && !b ? 1 : 2);
 }
 
-int lh_kernel_launches(const lh_shape* shape, int backward) {
+int lh_kernel_launches(const lh_shape* shape, lh_dtype dtype, int backward) {
   if (check_shape(shape) != LH_OK) return -1;
+  if (dtype != LH_BF16 && dtype != LH_F32) return -1;
   const Geom g = make_geom(*shape);
   const int chunks = (int)((g.U + 65534) / 65535);  // grid.y limit per launch
   if (!backward) {
     // pyramid+score, top-k (per chunk), gather, attention (per chunk), scatter (per chunk)
-    return pyramid_launches(g) + chunks + 1 +
+    return pyramid_launches(g, dtype) + chunks + 1 +
            (attn_fwd_uses_tc() ? attn_tc_fwd_launches(g) : chunks) + chunks;
   }
   // scatter-back bwd, softmax statistics, attention bwd, gather bwd (per chunk)

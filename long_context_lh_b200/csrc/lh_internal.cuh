@@ -139,7 +139,7 @@ __device__ __forceinline__ void store8_stream(float* p, const float (&x)[8]) {
 cudaError_t launch_pyramid_score(const Geom& g, lh_dtype dt, const void* q, const void* k,
                                  const void* v, float* pq, float* pk, float* pv, float* score,
                                  cudaStream_t st);
-int pyramid_launches(const Geom& g);  // kernel launches of one launch_pyramid_score
+int pyramid_launches(const Geom& g, lh_dtype dt);  // kernel launches of one launch_pyramid_score
 cudaError_t launch_topk(const Geom& g, const float* score, int32_t* idx, int32_t* pos,
                         int32_t* slot, cudaStream_t st);
 cudaError_t launch_gather(const Geom& g, lh_dtype dt, const void* q, const void* k, const void* v,

@@ -79,7 +79,7 @@ _SIGS = {
     "lh_read_device_status": ([_VP, ctypes.POINTER(ctypes.c_uint32)], _I),
     "lh_set_attention_impl": ([_I], _I),
     "lh_attention_impl_in_use": ([], _I),
-    "lh_kernel_launches": ([_SP, _I], _I),
+    "lh_kernel_launches": ([_SP, _I, _I], _I),
 }
 EXPORTED = tuple(_SIGS)
 
@@ -174,8 +174,8 @@ def lh_attention_impl_in_use() -> int:
     return int(_lib().lh_attention_impl_in_use())
 
 
-def lh_kernel_launches(shape: Shape, backward: bool) -> int:
-    return int(_lib().lh_kernel_launches(ctypes.byref(shape), int(backward)))
+def lh_kernel_launches(shape: Shape, dtype: int, backward: bool) -> int:
+    return int(_lib().lh_kernel_launches(ctypes.byref(shape), int(dtype), int(backward)))
 
 
 def lh_read_device_status(stream=None) -> int:
