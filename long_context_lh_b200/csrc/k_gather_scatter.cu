@@ -177,11 +177,10 @@ __global__ void __launch_bounds__(256) k_gather_pooled(
 // ------------------------------------------------------------- scatter-back
 // O[t] = (sum over selected entries covering t, ascending level, of os[slot]) / c_t.
 // Grid: x = blocks of kRows tokens of one unit, y = unit (offset u0).
-__device__ __forceinline__ float div_count(float x, int cnt) {
-  // dividing by a power of two is exact as a product with its reciprocal;
-  // other counts take the correctly rounded division
-  return (cnt & (cnt - 1)) == 0 ? x * (1.0f / (float)cnt) : __fdiv_rn(x, (float)cnt);
-}
+// 1/c in fp64 for the contributor counts c = 0..kMaxLevels (entry 0 unused)
+__constant__ double kInvCount[kMaxLevels + 1] = {0.0,       1.0,       1.0 / 2.0,
+                                                 1.0 / 3.0, 1.0 / 4.0, 1.0 / 5.0,
+                                                 1.0 / 6.0, 1.0 / 7.0, 1.0 / 8.0};
 
 // One thread: column chunk c of R consecutive tokens t0..t0+R-1 (R divides p,
 // t0 a multiple of R), which share every entry of level >= 1; so each thread
@@ -213,34 +212,36 @@ __global__ void __launch_bounds__(256) k_scatter(const __half* __restrict__ os,
   for (int l = 1; l < L; ++l) sc[l - 1] = __ldg(sl + lv.off[l] + lvl_index(lv, t0, l));
   uint4 w0[R], wc[LC];
 #pragma unroll
-  for (int r = 0; r < R; ++r)
+  for (int r = 0; r < R; ++r) {
+    w0[r] = make_uint4(0u, 0u, 0u, 0u);
     if (s0[r] >= 0) w0[r] = __ldg(reinterpret_cast<const uint4*>(src + (int64_t)s0[r] * D));
+  }
 #pragma unroll
-  for (int l = 1; l < L; ++l)
+  for (int l = 1; l < L; ++l) {
+    wc[l - 1] = make_uint4(0u, 0u, 0u, 0u);
     if (sc[l - 1] >= 0) wc[l - 1] = __ldg(reinterpret_cast<const uint4*>(src + (int64_t)sc[l - 1] * D));
+  }
+  // branch-free: an unselected level adds +0 (exact; at most the sign of a zero differs)
+  float xc[LC][8];
+  int cc = 0;
+#pragma unroll
+  for (int l = 1; l < L; ++l) {
+    unpack8(wc[l - 1], xc[l - 1]);
+    cc += sc[l - 1] >= 0 ? 1 : 0;
+  }
 #pragma unroll
   for (int r = 0; r < R; ++r) {
-    float acc[8], x[8];
-    int cnt = 0;
-    if (s0[r] >= 0) {
-      unpack8(w0[r], acc);
-      cnt = 1;
-    } else {
+    float acc[8];
+    unpack8(w0[r], acc);  // zeros when not selected
 #pragma unroll
-      for (int i = 0; i < 8; ++i) acc[i] = 0.0f;
-    }
+    for (int l = 1; l < L; ++l)  // ascending level, as defined
 #pragma unroll
-    for (int l = 1; l < L; ++l) {  // ascending level, as defined
-      if (sc[l - 1] >= 0) {
-        unpack8(wc[l - 1], x);
-#pragma unroll
-        for (int i = 0; i < 8; ++i) acc[i] = __fadd_rn(acc[i], x[i]);
-        ++cnt;
-      }
-    }
+      for (int i = 0; i < 8; ++i) acc[i] = __fadd_rn(acc[i], xc[l - 1][i]);
+    const int cnt = cc + (s0[r] >= 0 ? 1 : 0);
     if (cnt > 0) {
+      const double inv = kInvCount[cnt];
 #pragma unroll
-      for (int i = 0; i < 8; ++i) acc[i] = div_count(acc[i], cnt);
+      for (int i = 0; i < 8; ++i) acc[i] = div_exact(acc[i], inv);
     }
     const int64_t row = u * lv.N + t0 + r;
     store8_stream(o + row * D + 8 * c, acc);

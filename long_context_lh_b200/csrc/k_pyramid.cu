@@ -48,13 +48,18 @@ struct PyrPrm {
   int32_t N, M, CR, p, J, L;
   int32_t pow2;  // p is a power of two: mean = sum * inv_p exactly
   float inv_p;
+  double inv_pd;  // 1/p in fp64 for the exact division (div_exact) otherwise
   int32_t off[kMaxLevels + 1];
   int32_t pw[kMaxLevels + 1];
 };
 
+template <int P>
 __device__ __forceinline__ float mean_of(float sum, const PyrPrm& prm) {
-  return prm.pow2 ? sum * prm.inv_p : __fdiv_rn(sum, (float)prm.p);
+  if constexpr (P > 0 && (P & (P - 1)) == 0) return sum * (1.0f / (float)P);
+  return prm.pow2 ? sum * prm.inv_p : div_exact(sum, prm.inv_pd);
 }
+
+constexpr int ipow(int b, int e) { return e == 0 ? 1 : b * ipow(b, e - 1); }
 
 __device__ __forceinline__ void cp_async16(void* dst, const void* src) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(
@@ -113,7 +118,9 @@ struct ChunkSmem {
   }
 };
 
-template <typename Tin, int D, bool kPyr, bool kScore>
+// P > 0: p == P known at compile time (child loops unrolled, level widths
+// constant); P == 0: any p.
+template <typename Tin, int D, int P, bool kPyr, bool kScore>
 __global__ void __launch_bounds__(256) k_pyr_chunk(
     const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin* __restrict__ v,
     float* __restrict__ pq, float* __restrict__ pk, float* __restrict__ pv,
@@ -123,11 +130,12 @@ __global__ void __launch_bounds__(256) k_pyr_chunk(
   constexpr int NT = Sm::NT;
   extern __shared__ __align__(16) uint8_t smem[];
   const int CR = prm.CR;
+  const int p = P > 0 ? P : prm.p;
   Tin* sIn = reinterpret_cast<Tin*>(smem);  // [NT][CR][D]
   float* sSc = reinterpret_cast<float*>(smem + Sm::in_bytes(CR));  // [2][CR] ping-pong
   float* sLa = sSc + Sm::score_floats(CR);                           // [3][CR/p][D]
-  float* sLb = sLa + (size_t)3 * (CR / prm.p) * D;                   // [3][CR/p^2][D]
-  const int ra = CR / prm.p, rb = (CR / prm.p / prm.p > 0) ? CR / prm.p / prm.p : 1;
+  float* sLb = sLa + (size_t)3 * (CR / p) * D;                       // [3][CR/p^2][D]
+  const int ra = CR / p, rb = (CR / p / p > 0) ? CR / p / p : 1;
 
   const int tid = threadIdx.x;
   const int32_t t0 = (int32_t)blockIdx.x * CR;
@@ -174,9 +182,12 @@ __global__ void __launch_bounds__(256) k_pyr_chunk(
 
   // ---- levels 1..J
   int nprev = rows;
-  for (int l = 1; l <= prm.J; ++l) {
-    const int n = nprev / prm.p;
-    const int32_t j0 = t0 / prm.pw[l];  // first entry of this chunk at level l
+#pragma unroll
+  for (int l = 1; l < kMaxLevels; ++l) {  // unrolled: off[l] and pw[l] are constant indices
+    if (l > prm.J) break;
+    const int n = nprev / p;
+    const int32_t pwl = P > 0 ? ipow(P > 0 ? P : 1, l) : prm.pw[l];
+    const int32_t j0 = t0 / pwl;  // first entry of this chunk at level l
     const float* prevS = sSc + ((l - 1) & 1) * CR;
     float* curS = sSc + (l & 1) * CR;
     if (kPyr) {
@@ -192,8 +203,9 @@ __global__ void __launch_bounds__(256) k_pyr_chunk(
         float acc[8], x[8];
 #pragma unroll
         for (int i = 0; i < 8; ++i) acc[i] = 0.0f;
-        for (int i = 0; i < prm.p; ++i) {
-          const int ch = e * prm.p + i;
+#pragma unroll
+        for (int i = 0; i < p; ++i) {
+          const int ch = e * p + i;
           if (l == 1) {
             smem8(sIn + ((size_t)t * CR + ch) * D + 8 * c, x);
             // the child row's partial a_c of its score (Q and K)
@@ -205,7 +217,7 @@ __global__ void __launch_bounds__(256) k_pyr_chunk(
           for (int z = 0; z < 8; ++z) acc[z] = __fadd_rn(acc[z], x[z]);
         }
 #pragma unroll
-        for (int z = 0; z < 8; ++z) acc[z] = mean_of(acc[z], prm);
+        for (int z = 0; z < 8; ++z) acc[z] = mean_of<P>(acc[z], prm);
         float* dst = (t == 0 ? pq : t == 1 ? pk : pv);
         put8(dst + ((u * (prm.M - prm.N) + prm.off[l] - prm.N + j0 + e) * D + 8 * c), acc);
         if (l < prm.J) put8(curL + ((size_t)t * crow + e) * D + 8 * c, acc);
@@ -240,7 +252,8 @@ __global__ void __launch_bounds__(256) k_pyr_chunk(
       }
       for (int e = tid; e < n; e += 256) {
         float m = 0.0f;
-        for (int i = 0; i < prm.p; ++i) m = fmaxf(m, prevS[e * prm.p + i]);
+#pragma unroll
+        for (int i = 0; i < p; ++i) m = fmaxf(m, prevS[e * p + i]);
         curS[e] = m;
         sc[prm.off[l] + j0 + e] = m;
       }
@@ -282,7 +295,7 @@ __global__ void __launch_bounds__(256) k_pyr_upper(
       for (int z = 0; z < 8; ++z) acc[z] = __fadd_rn(acc[z], x[z]);
     }
 #pragma unroll
-    for (int z = 0; z < 8; ++z) acc[z] = mean_of(acc[z], prm);
+    for (int z = 0; z < 8; ++z) acc[z] = mean_of<0>(acc[z], prm);
     float* dst = (t == 0 ? pq : t == 1 ? pk : pv);
     float* o = dst + (u * (prm.M - prm.N) + prm.off[l] - prm.N + e) * D + 8 * c;
     *reinterpret_cast<float4*>(o) = make_float4(acc[0], acc[1], acc[2], acc[3]);
@@ -304,6 +317,7 @@ PyrPrm make_prm(const Geom& g, int cap) {
   prm.L = g.L;
   prm.pow2 = (g.p & (g.p - 1)) == 0;
   prm.inv_p = 1.0f / (float)g.p;  // exact when p is a power of two
+  prm.inv_pd = 1.0 / (double)g.p;
   for (int l = 0; l <= kMaxLevels; ++l) {
     prm.off[l] = (int32_t)g.off[l];
     prm.pw[l] = (int32_t)(g.pw[l] > 0x7fffffff ? 0x7fffffff : g.pw[l]);
@@ -315,12 +329,12 @@ PyrPrm make_prm(const Geom& g, int cap) {
   return prm;
 }
 
-template <typename Tin, int D, bool kPyr, bool kScore>
+template <typename Tin, int D, int P, bool kPyr, bool kScore>
 cudaError_t launch_flags(const Geom& g, const Tin* q, const Tin* k, const Tin* v, float* pq,
                          float* pk, float* pv, float* score, cudaStream_t st) {
   const PyrPrm prm = make_prm(g, chunk_rows_cap(D, sizeof(Tin)));
   const size_t smem = ChunkSmem<Tin, D, kPyr>::bytes(prm.CR, prm.p);
-  auto* kc = k_pyr_chunk<Tin, D, kPyr, kScore>;
+  auto* kc = k_pyr_chunk<Tin, D, P, kPyr, kScore>;
   cudaError_t e = cudaFuncSetAttribute(kc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   const unsigned bx = (unsigned)((g.N + prm.CR - 1) / prm.CR);
@@ -344,9 +358,15 @@ cudaError_t launch_t(const Geom& g, const void* q, const void* k, const void* v,
   const Tin* tq = static_cast<const Tin*>(q);
   const Tin* tk = static_cast<const Tin*>(k);
   const Tin* tv = static_cast<const Tin*>(v);
-  if (pq && score) return launch_flags<Tin, D, true, true>(g, tq, tk, tv, pq, pk, pv, score, st);
-  if (pq) return launch_flags<Tin, D, true, false>(g, tq, tk, tv, pq, pk, pv, score, st);
-  return launch_flags<Tin, D, false, true>(g, tq, tk, tv, pq, pk, pv, score, st);
+  auto go = [&](auto pc) {
+    constexpr int P = decltype(pc)::value;
+    if (pq && score) return launch_flags<Tin, D, P, true, true>(g, tq, tk, tv, pq, pk, pv, score, st);
+    if (pq) return launch_flags<Tin, D, P, true, false>(g, tq, tk, tv, pq, pk, pv, score, st);
+    return launch_flags<Tin, D, P, false, true>(g, tq, tk, tv, pq, pk, pv, score, st);
+  };
+  if (g.p == 4) return go(std::integral_constant<int, 4>{});
+  if (g.p == 2) return go(std::integral_constant<int, 2>{});
+  return go(std::integral_constant<int, 0>{});
 }
 
 }  // namespace

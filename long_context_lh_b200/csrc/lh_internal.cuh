@@ -134,6 +134,16 @@ __device__ __forceinline__ void store8_stream(float* p, const float (&x)[8]) {
   __stcs(reinterpret_cast<float4*>(p) + 1, make_float4(x[4], x[5], x[6], x[7]));
 }
 
+// x / c rounded to nearest fp32, for an integer 1 <= c < 2^20, as one fp64
+// product with inv_c = 1/c (rounded to fp64) rounded once to fp32.  It is the
+// correctly rounded quotient: with c = 2^a c' (c' odd) and the quotient
+// measured in half-ulps, x / c' = N / c' for an even integer N, so it is never
+// a rounding midpoint and lies at least 1/c' > 2^-20 half-ulps from one, while
+// the fp64 product is within 2^-52 relative (< 2^-28 ulp) of the quotient.
+__device__ __forceinline__ float div_exact(float x, double inv_c) {
+  return __double2float_rn((double)x * inv_c);
+}
+
 // ---------------------------------------------------------------- launchers
 // Each returns cudaSuccess or the launch error; arguments are already checked.
 cudaError_t launch_pyramid_score(const Geom& g, lh_dtype dt, const void* q, const void* k,
