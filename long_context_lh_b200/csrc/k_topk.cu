@@ -28,6 +28,7 @@
 #include <cooperative_groups.h>
 
 #include <atomic>
+#include <type_traits>
 
 #include "lh_internal.cuh"
 
@@ -39,6 +40,8 @@ namespace {
 constexpr int kThreads = 1024;
 constexpr int kWarps = kThreads / 32;
 constexpr int kBins = 2048;
+// Shared memory for a CTA's cached keys (the static part holds the histograms).
+constexpr int64_t kKeyCacheBytes = 180 * 1024;
 
 struct TopkParams {
   int32_t N, M;  // within-unit sizes fit 32 bits (M < 2^31 is a checked limit)
@@ -103,9 +106,9 @@ struct Pick {
 
 // Cluster-summed histogram -> digit where the need-th candidate falls.
 // descending: rank digits from the largest value down (scores), else up (gids).
+template <int CL>  // a multiple of 8
 __device__ Pick pick_digit(cg::cluster_group& cluster, uint32_t* hist, int nbins, bool descending,
                            uint32_t need, uint32_t* warp_buf, uint32_t* sh) {
-  const int CL = (int)cluster.num_blocks();
   const int per = nbins / kThreads;  // 2 or 1 ordinals per thread
   uint32_t tot[2] = {0, 0};
   uint32_t local = 0;
@@ -113,7 +116,14 @@ __device__ Pick pick_digit(cg::cluster_group& cluster, uint32_t* hist, int nbins
     const int ord = threadIdx.x * per + i;
     const int bin = descending ? (nbins - 1 - ord) : ord;
     uint32_t s = 0;
-    for (int r = 0; r < CL; ++r) s += cluster.map_shared_rank(hist, r)[bin];
+#pragma unroll
+    for (int r0 = 0; r0 < CL; r0 += 8) {  // eight remote loads in flight at a time
+      uint32_t v[8];
+#pragma unroll
+      for (int r = 0; r < 8; ++r) v[r] = cluster.map_shared_rank(hist, r0 + r)[bin];
+#pragma unroll
+      for (int r = 0; r < 8; ++r) s += v[r];
+    }
     tot[i] = s;
     local += s;
   }
@@ -134,11 +144,16 @@ __device__ Pick pick_digit(cg::cluster_group& cluster, uint32_t* hist, int nbins
   return pk;
 }
 
+// CTA r of the cluster owns the tokens [t_b, t_e) (whole coarsest spans) and
+// every entry whose span lies in them: at level l the contiguous gids
+// off[l] + [t_b / p^l, t_e / p^l).  Its keys are copied to shared memory once
+// (cached != 0; else read from L2 in each pass); the histograms, the tie pass
+// and the compaction then only touch the CTA's own keys.
+template <int CL>
 __global__ void __launch_bounds__(kThreads, 1)
     k_topk(const float* __restrict__ score, int32_t* __restrict__ idx, int32_t* __restrict__ pos,
-           int32_t* __restrict__ slot, const TopkParams prm) {
+           int32_t* __restrict__ slot, const TopkParams prm, int cached) {
   cg::cluster_group cluster = cg::this_cluster();
-  const int CL = (int)cluster.num_blocks();
   const int rank = (int)cluster.block_rank();
   const int64_t u = prm.unit0 + blockIdx.y;
 
@@ -147,14 +162,38 @@ __global__ void __launch_bounds__(kThreads, 1)
   __shared__ uint32_t sh[4];
   __shared__ uint32_t warp_tot[kWarps];
   __shared__ uint32_t cta_total;
+  extern __shared__ uint32_t skey[];  // the CTA's keys, level by level (cached)
 
   const uint32_t* key = reinterpret_cast<const uint32_t*>(score + u * prm.M);
-  const int64_t M = prm.M;
-  const int64_t per = (M + CL - 1) / CL;
-  const int64_t g_begin = imin64(M, (int64_t)rank * per);
-  const int64_t g_end = imin64(M, g_begin + per);
+  const int32_t Ptop = prm.pw[prm.L - 1];
+  const int32_t spans = prm.N / Ptop;
+  const int32_t sper = (spans + CL - 1) / CL;
+  const int32_t t_b = (int32_t)imin64(prm.N, (int64_t)rank * sper * Ptop);
+  const int32_t t_e = (int32_t)imin64(prm.N, (int64_t)t_b + (int64_t)sper * Ptop);
+  // level l: entries jb[l] .. jb[l] + nl[l] - 1, cached at skey[kb[l] ..]
+  int32_t jb[kMaxLevels], nl[kMaxLevels], kb[kMaxLevels];
+  int32_t nk = 0;
+#pragma unroll
+  for (int l = 0; l < kMaxLevels; ++l) {
+    jb[l] = l < prm.L ? t_b / prm.pw[l] : 0;
+    nl[l] = l < prm.L ? (t_e - t_b) / prm.pw[l] : 0;
+    kb[l] = nk;
+    nk += nl[l];
+  }
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  if (cached) {
+#pragma unroll
+    for (int l = 0; l < kMaxLevels; ++l) {
+      const uint32_t* src = key + prm.off[l] + jb[l];
+#pragma unroll 4
+      for (int32_t j = threadIdx.x; j < nl[l]; j += kThreads) skey[kb[l] + j] = __ldg(src + j);
+    }
+  }
+  auto key_of = [&](int l, int32_t j) -> uint32_t {  // j: index within the CTA's level-l range
+    return cached ? skey[kb[l] + j] : __ldg(key + prm.off[l] + jb[l] + j);
+  };
 
-  cluster.sync();  // every CTA of the cluster is running before DSMEM use
+  cluster.sync();  // every CTA is running (DSMEM) and its keys are in place
 
   // ---- 1. threshold score by radix select on the key bits (descending)
   uint32_t prefix = 0, pmask = 0, need = (uint32_t)prm.S, ties = 0;
@@ -166,13 +205,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t dmask = (uint32_t)nb - 1u;
     for (int i = threadIdx.x; i < kBins; i += kThreads) hist[buf][i] = 0;
     __syncthreads();
-    for (int64_t g0 = g_begin + (threadIdx.x & ~31); g0 < g_end; g0 += kThreads) {
-      const int64_t g = g0 + (threadIdx.x & 31);
-      const uint32_t kv = g < g_end ? __ldg(key + g) : 0u;
-      hist_add(hist[buf], g < g_end && (kv & pmask) == prefix, (kv >> shift) & dmask);
+#pragma unroll
+    for (int l = 0; l < kMaxLevels; ++l) {
+      for (int32_t j0 = warp * 32; j0 < nl[l]; j0 += kThreads) {  // warp-uniform trip count
+        const int32_t j = j0 + lane;
+        const uint32_t kv = j < nl[l] ? key_of(l, j) : 0u;
+        hist_add(hist[buf], j < nl[l] && (kv & pmask) == prefix, (kv >> shift) & dmask);
+      }
     }
     cluster.sync();
-    Pick pk = pick_digit(cluster, hist[buf], nb, true, need, warp_buf, sh);
+    Pick pk = pick_digit<CL>(cluster, hist[buf], nb, true, need, warp_buf, sh);
     prefix |= pk.bin << shift;
     pmask |= dmask << shift;
     need -= pk.before;
@@ -185,7 +227,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   int64_t gid_thr = INT64_MAX;
   if (need < ties) {
     int nbits = 1;
-    while (nbits < 31 && ((int64_t)1 << nbits) < M) ++nbits;
+    while (nbits < 31 && ((int64_t)1 << nbits) < prm.M) ++nbits;
     uint32_t gprefix = 0, gmask = 0;
     for (int hi = nbits; hi > 0;) {
       const int w = hi >= 11 ? 11 : hi;
@@ -194,17 +236,20 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t dmask = (uint32_t)nb - 1u;
       for (int i = threadIdx.x; i < kBins; i += kThreads) hist[buf][i] = 0;
       __syncthreads();
-      for (int64_t g0 = g_begin + (threadIdx.x & ~31); g0 < g_end; g0 += kThreads) {
-        const int64_t g = g0 + (threadIdx.x & 31);
-        const bool in = g < g_end && __ldg(key + (g < g_end ? g : g0)) == T &&
-                        (((uint32_t)g) & gmask) == gprefix;
-        hist_add(hist[buf], in, ((uint32_t)g >> shift) & dmask);
+#pragma unroll
+      for (int l = 0; l < kMaxLevels; ++l) {
+        for (int32_t j0 = warp * 32; j0 < nl[l]; j0 += kThreads) {
+          const int32_t j = j0 + lane;
+          const uint32_t gid = (uint32_t)(prm.off[l] + jb[l] + j);
+          const bool in = j < nl[l] && key_of(l, j < nl[l] ? j : 0) == T && (gid & gmask) == gprefix;
+          hist_add(hist[buf], in, (gid >> shift) & dmask);
+        }
       }
       cluster.sync();
       // pick_digit needs nbins to be a multiple of the thread count or equal to
       // 1024/2048; smaller digit widths are padded with empty bins.
       const int nbp = nb < kThreads ? kThreads : nb;
-      Pick pk = pick_digit(cluster, hist[buf], nbp, false, need, warp_buf, sh);
+      Pick pk = pick_digit<CL>(cluster, hist[buf], nbp, false, need, warp_buf, sh);
       gprefix |= pk.bin << shift;
       gmask |= dmask << shift;
       need -= pk.before;
@@ -214,29 +259,27 @@ __global__ void __launch_bounds__(kThreads, 1)
     gid_thr = (int64_t)gprefix;
   }
 
-  // ---- 3. ordered compaction over (token, level)
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int64_t tper = (prm.N + CL - 1) / CL;
-  const int64_t t_begin = imin64(prm.N, (int64_t)rank * tper);
-  const int64_t t_end = imin64(prm.N, t_begin + tper);
-  const int64_t wper = ((t_end - t_begin + kWarps - 1) / kWarps + 31) / 32 * 32;
-  const int64_t w_begin = imin64(t_end, t_begin + warp * wper);
-  const int64_t w_end = imin64(t_end, w_begin + wper);
-
-  auto selected = [&](int64_t g) -> bool {
-    const uint32_t kv = __ldg(key + g);
-    return kv > T || (kv == T && g <= gid_thr);
+  // ---- 3. ordered compaction over (token, level) of the CTA's tokens
+  const int32_t wper = ((t_e - t_b + kWarps - 1) / kWarps + 31) / 32 * 32;
+  const int32_t w_begin = (int32_t)imin64(t_e, (int64_t)t_b + (int64_t)warp * wper);
+  const int32_t w_end = (int32_t)imin64(t_e, (int64_t)w_begin + wper);
+  // level-l entry whose span ends at token t (t1 = t + 1, requires ends_at)
+  auto selected = [&](int l, uint32_t t1) -> bool {
+    const int32_t g = gid_at(prm, t1, l);
+    const uint32_t kv = key_of(l, g - prm.off[l] - jb[l]);
+    return kv > T || (kv == T && (int64_t)g <= gid_thr);
   };
   // pass A: count per warp
   uint32_t wcount = 0;
-  for (int64_t tb = w_begin; tb < w_end; tb += 32) {
-    const int64_t t = tb + lane;
+  for (int32_t tb = w_begin; tb < w_end; tb += 32) {
+    const int32_t t = tb + lane;
     uint32_t c = 0;
     if (t < w_end) {
       const uint32_t t1 = (uint32_t)t + 1u;
-      for (int l = 0; l < prm.L; ++l) {
-        if (!ends_at(prm, t1, l)) break;  // spans end at t only up to some level
-        c += selected(gid_at(prm, t1, l)) ? 1u : 0u;
+#pragma unroll
+      for (int l = 0; l < kMaxLevels; ++l) {  // unrolled: jb[l], kb[l] stay in registers
+        if (l >= prm.L || !ends_at(prm, t1, l)) break;  // spans end at t up to some level
+        c += selected(l, t1) ? 1u : 0u;
       }
     }
     wcount += __reduce_add_sync(0xffffffffu, c);
@@ -257,15 +300,16 @@ __global__ void __launch_bounds__(kThreads, 1)
   int32_t* idx_u = idx + u * prm.S;
   int32_t* pos_u = pos + u * prm.S;
   int32_t* slot_u = slot + u * prm.M;
-  for (int64_t tb = w_begin; tb < w_end; tb += 32) {
-    const int64_t t = tb + lane;
+  for (int32_t tb = w_begin; tb < w_end; tb += 32) {
+    const int32_t t = tb + lane;
     uint32_t c = 0;
     uint32_t selmask = 0;
     if (t < w_end) {
       const uint32_t t1 = (uint32_t)t + 1u;
-      for (int l = 0; l < prm.L; ++l) {
-        if (!ends_at(prm, t1, l)) break;
-        if (selected(gid_at(prm, t1, l))) {
+#pragma unroll
+      for (int l = 0; l < kMaxLevels; ++l) {
+        if (l >= prm.L || !ends_at(prm, t1, l)) break;
+        if (selected(l, t1)) {
           selmask |= 1u << l;
           ++c;
         }
@@ -275,8 +319,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint32_t k = base + incl - c;
     if (t < w_end) {
       const uint32_t t1 = (uint32_t)t + 1u;
-      for (int l = 0; l < prm.L; ++l) {
-        if (!ends_at(prm, t1, l)) break;
+#pragma unroll
+      for (int l = 0; l < kMaxLevels; ++l) {
+        if (l >= prm.L || !ends_at(prm, t1, l)) break;
         const int32_t g = gid_at(prm, t1, l);
         if (selmask & (1u << l)) {
           idx_u[k] = (int32_t)g;
@@ -319,7 +364,7 @@ cudaError_t launch_topk(const Geom& g, const float* score, int32_t* idx, int32_t
     int state = dev < 64 ? ok16[dev].load() : 2;
     if (state == 0) {
       state = 2;
-      if (cudaFuncSetAttribute(k_topk, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) ==
+      if (cudaFuncSetAttribute(k_topk<16>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) ==
           cudaSuccess) {
         cudaLaunchConfig_t q = {};
         q.gridDim = dim3(16, 1, 1);
@@ -332,7 +377,8 @@ cudaError_t launch_topk(const Geom& g, const float* score, int32_t* idx, int32_t
         q.attrs = a;
         q.numAttrs = 1;
         int nclusters = 0;
-        if (cudaOccupancyMaxActiveClusters(&nclusters, k_topk, &q) == cudaSuccess && nclusters > 0)
+        if (cudaOccupancyMaxActiveClusters(&nclusters, k_topk<16>, &q) == cudaSuccess &&
+            nclusters > 0)
           state = 1;
       }
       (void)cudaGetLastError();
@@ -340,25 +386,44 @@ cudaError_t launch_topk(const Geom& g, const float* score, int32_t* idx, int32_t
     }
     if (state == 1) CL = 16;
   }
-  for (int64_t u0 = 0; u0 < g.U; u0 += 65535) {
-    prm.unit0 = u0;
-    const int64_t nu = g.U - u0 < 65535 ? g.U - u0 : 65535;
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)CL, (unsigned)nu, 1);
-    cfg.blockDim = dim3(kThreads, 1, 1);
-    cfg.dynamicSmemBytes = 0;
-    cfg.stream = st;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = (unsigned)CL;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    cudaError_t e = cudaLaunchKernelEx(&cfg, k_topk, score, idx, pos, slot, prm);
+  // keys of one CTA: whole coarsest spans, every level
+  const int64_t Ptop = g.pw[g.L - 1];
+  const int64_t spans = g.N / Ptop;
+  const int64_t sper = (spans + CL - 1) / CL;
+  int64_t per_span = 0;
+  for (int l = 0; l < g.L; ++l) per_span += Ptop / g.pw[l];
+  const int64_t key_bytes = sper * per_span * 4;
+  const int cached = key_bytes <= kKeyCacheBytes ? 1 : 0;
+  const size_t dyn = cached ? (size_t)key_bytes : 0;
+  auto launch = [&](auto clc) -> cudaError_t {
+    constexpr int C = decltype(clc)::value;
+    auto* kf = k_topk<C>;
+    cudaError_t e = cudaFuncSetAttribute(kf, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dyn);
     if (e != cudaSuccess) return e;
-  }
-  return cudaSuccess;
+    if (C > 8 && (e = cudaFuncSetAttribute(kf, cudaFuncAttributeNonPortableClusterSizeAllowed, 1)) !=
+                     cudaSuccess)
+      return e;
+    for (int64_t u0 = 0; u0 < g.U; u0 += 65535) {
+      prm.unit0 = u0;
+      const int64_t nu = g.U - u0 < 65535 ? g.U - u0 : 65535;
+      cudaLaunchConfig_t cfg = {};
+      cfg.gridDim = dim3((unsigned)C, (unsigned)nu, 1);
+      cfg.blockDim = dim3(kThreads, 1, 1);
+      cfg.dynamicSmemBytes = dyn;
+      cfg.stream = st;
+      cudaLaunchAttribute attr[1];
+      attr[0].id = cudaLaunchAttributeClusterDimension;
+      attr[0].val.clusterDim.x = (unsigned)C;
+      attr[0].val.clusterDim.y = 1;
+      attr[0].val.clusterDim.z = 1;
+      cfg.attrs = attr;
+      cfg.numAttrs = 1;
+      e = cudaLaunchKernelEx(&cfg, kf, score, idx, pos, slot, prm, cached);
+      if (e != cudaSuccess) return e;
+    }
+    return cudaSuccess;
+  };
+  return CL == 16 ? launch(std::integral_constant<int, 16>{}) : launch(std::integral_constant<int, 8>{});
 }
 
 }  // namespace lh

@@ -124,6 +124,32 @@ def test_front_stages_match_oracle(case):
             check_pyramid(t.cpu().numpy(), ref, "pyramid")
 
 
+@pytest.mark.parametrize("case", [dict(N=524288, L=2, S=3000), dict(N=262144, p=2, L=3, S=100000)],
+                         ids=str)
+def test_topk_on_large_units_matches_oracle(case):
+    """The first case (more than 2^19 entries per unit) takes the 16-CTA cluster
+    where the device allows it, with the keys cached in shared memory; the second
+    has too many keys per CTA for the cache and reads them from L2 in each pass.
+    The selection must be exact either way."""
+    w = workload(dtype="bf16", dist="outliers", H=2, **case)
+    xc = make_inputs(w, "cpu", with_dO=False)
+    x = to_dev(xc)
+    shp, dt = lshape(w), lh.dtype_code(x["q"].dtype)
+    M = lh.lh_num_entries(shp)
+    score = torch.zeros((w.B, w.H, M), dtype=torch.float32, device=DEV)
+    lh.lh_score(shp, dt, x["q"], x["k"], score)
+    idx = torch.full((w.B, w.H, w.S), -7, dtype=torch.int32, device=DEV)
+    pos = torch.full_like(idx, -7)
+    slot = torch.full((w.B, w.H, M), -7, dtype=torch.int32, device=DEV)
+    lh.lh_topk_select(shp, score, idx, pos, slot)
+    torch.cuda.synchronize()
+    s = oshape(w)
+    i_ref, p_ref, s_ref = oracle.select(s, score.cpu().numpy())  # scores are pinned elsewhere
+    assert np.array_equal(idx.cpu().numpy(), i_ref)
+    assert np.array_equal(pos.cpu().numpy(), p_ref)
+    assert np.array_equal(slot.cpu().numpy(), s_ref)
+
+
 def test_ties_beyond_inheritance_are_broken_by_gid():
     """Quantised inputs make many equal scores; the radix select on gids must agree."""
     w = workload(dtype="bf16", N=2048, S=300, H=3)
