@@ -614,7 +614,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 // dS = P (dP - D) in fp16 shared memory (double-buffered); dQ += dS K_j in TMEM.
 struct DqBars {
   uint64_t q_full;
-  uint64_t kv_full[2], kv_empty[2];
+  uint64_t kv_full[3], kv_empty[3];  // [stage], at most 3 stages
   uint64_t s_full, s_free, mma_done;
   uint64_t ds_full[2], dsdone[2];
   uint32_t tmem;
@@ -623,7 +623,7 @@ struct DqBars {
 
 template <int D>
 struct DqLayout {
-  static constexpr int kStages = (D == 64) ? 2 : 1;
+  static constexpr int kStages = (D == 64) ? 3 : 1;  // DqBars holds up to 3
   static constexpr int kTile = 128 * D * 2;
   static constexpr int kQ = 0;
   static constexpr int kDO = kQ + kTile;
@@ -643,7 +643,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                      float scale_log2, int ntiles) {
   using Lt = DqLayout<D>;
   constexpr int STG = Lt::kStages;
-  static_assert(STG >= 1 && STG <= 2, "DqBars holds at most 2 stages");
+  static_assert(STG >= 1 && STG <= 3, "DqBars holds at most 3 stages");
   extern __shared__ __align__(1024) uint8_t smem[];
   if (smem_u32(smem) & 1023u) {
     if (threadIdx.x == 0) report_status(kStatusAttnBwdTimeout | 2u);
@@ -665,9 +665,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (threadIdx.x == 0) {
     mbar_init(&bars->q_full, 1);
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < STG; ++i) {
       mbar_init(&bars->kv_full[i], 1);
       mbar_init(&bars->kv_empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
       mbar_init(&bars->ds_full[i], 8);
       mbar_init(&bars->dsdone[i], 1);
     }
