@@ -32,6 +32,7 @@ sys.path.insert(0, ROOT)
 
 import torch  # noqa: E402
 
+from long_context_lh_b200 import replicas  # noqa: E402
 from long_context_lh_b200.synth import WORKLOADS, make_inputs  # noqa: E402
 
 METRIC = "Lighthouse layer tokens/s fwd & fwd+bwd at N=98K/512K; % of HBM/TC roofline"
@@ -130,10 +131,11 @@ class ClockSampler:
 
 
 # ------------------------------------------------------------------ our arm
-def run_ours(args, rank, world, local_rank):
+def run_ours(args, rk):
     import numpy as np  # noqa: F401
     from long_context_lh_b200 import lighthouse as lh
 
+    rank, world, local_rank = rk.rank, rk.world, rk.local_rank
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
     w = WORKLOADS[args.workload]
@@ -146,7 +148,7 @@ def run_ours(args, rank, world, local_rank):
     peaks, peaks_src = load_peaks()
     shp = lh.make_shape(w.B, w.H, w.N, w.d, w.p, w.L, w.S)
     dt = lh.dtype_code(w.torch_dtype)
-    x = make_inputs(w, dev)
+    x = make_inputs(w, dev, batch=rank)  # each rank: its own independent batch
     q, k, v, dO = x["q"], x["k"], x["v"], x["dO"]
     o = torch.empty_like(q)
     dq, dk, dv = (torch.empty_like(q) for _ in range(3))
@@ -208,14 +210,9 @@ def run_ours(args, rank, world, local_rank):
         lh.lh_gather_bwd(shp, dt, dqs, dks, dvs, slot, dq, dk, dv, sp)
         evs[8].record(stream)
 
-    dist = world > 1
-
-    def barrier():
-        if dist:
-            torch.distributed.barrier()
-
     def timed(fn, K):
-        barrier()
+        """Device time of K calls on this rank; the max over ranks is returned."""
+        replicas.barrier(rk)
         torch.cuda.synchronize()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
@@ -224,12 +221,8 @@ def run_ours(args, rank, world, local_rank):
         e1.record(stream)
         torch.cuda.synchronize()
         ms = e0.elapsed_time(e1)
-        barrier()
-        if dist:
-            t = torch.tensor([ms], device=dev)
-            torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-            ms = float(t.item())
-        return ms
+        replicas.barrier(rk)
+        return replicas.max_over_ranks(rk, ms, dev)
 
     with torch.cuda.stream(stream):
         for _ in range(args.warmup):
@@ -253,7 +246,7 @@ def run_ours(args, rank, world, local_rank):
         status |= lh.lh_read_device_status(stream)
 
     tokens = w.B * w.N
-    value = world * tokens / (ms_step / 1e3)
+    value = replicas.job_rate(tokens, world, ms_step / 1e3)
     # rows the pooled gather must read: p^level for every selected entry
     gids = idx.view(U, w.S).long()
     offs = torch.tensor([sum(w.level_len(m) for m in range(l)) for l in range(w.L + 1)], device=dev)
@@ -288,7 +281,7 @@ def run_ours(args, rank, world, local_rank):
         dense = dense_sdpa(w, q, k, v, dO, stream, args)
 
     # end to end through the public API with pinned host buffers
-    e2e = None if args.no_e2e else e2e_run(lh, w, shp, dt, x, dev, stream, args, dist)
+    e2e = None if args.no_e2e else e2e_run(lh, w, shp, dt, x, dev, stream, args, rk)
     launches = launches_per_step(lh, w)
     out = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
@@ -300,7 +293,7 @@ def run_ours(args, rank, world, local_rank):
                    "l2": "inputs larger than L2 (3 x %.0f MB + dO), no flush" % (w.B * w.H * w.N * w.d * 2 / 1e6),
                    "attention": {0: "tcgen05", 1: "mma_sync", 2: "tcgen05 fwd, mma_sync bwd"}[lh.lh_attention_impl_in_use()],
                    "parallelism": f"replicas x{world} (heads independent)"},
-        "fwd_tokens_per_s": world * tokens / (ms_fwd / 1e3), "ms_fwd": ms_fwd,
+        "fwd_tokens_per_s": replicas.job_rate(tokens, world, ms_fwd / 1e3), "ms_fwd": ms_fwd,
         "roofline": roof, "stages": stage_report, "dense_sdpa": dense, "e2e": e2e,
         "gpu_launches": launches * args.steps, "gpu_launches_per_step": launches,
         "device_status": status, "peaks": peaks, "peaks_source": peaks_src,
@@ -355,7 +348,7 @@ def dense_sdpa(w, q, k, v, dO, stream, args):
         return {"error": str(ex)[:200]}
 
 
-def e2e_run(lh, w, shp, dt, x, dev, stream, args, dist):
+def e2e_run(lh, w, shp, dt, x, dev, stream, args, rk):
     """Same step through lh_forward/lh_backward with host<->device copies inside."""
     host = {n: t.cpu().pin_memory() for n, t in x.items()}
     dev_in = {n: torch.empty_like(t) for n, t in x.items()}
@@ -381,21 +374,16 @@ def e2e_run(lh, w, shp, dt, x, dev, stream, args, dist):
     with torch.cuda.stream(stream):
         step()
         torch.cuda.synchronize()
-        if dist:
-            torch.distributed.barrier()
+        replicas.barrier(rk)
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
         for _ in range(K):
             step()
         e1.record(stream)
         torch.cuda.synchronize()
-    ms = e0.elapsed_time(e1) / K
-    if dist:
-        t = torch.tensor([ms], device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms = float(t.item())
-    world = torch.distributed.get_world_size() if dist else 1
-    return {"value": world * w.B * w.N / (ms / 1e3), "unit": "tokens/s", "ms_per_step": ms,
+    ms = replicas.max_over_ranks(rk, e0.elapsed_time(e1) / K, dev)
+    return {"value": replicas.job_rate(w.B * w.N, rk.world, ms / 1e3), "unit": "tokens/s",
+            "ms_per_step": ms,
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
 
 
@@ -437,9 +425,10 @@ def cpu_baseline(w, budget_s=20.0, steps=None, warmup=0):
             "per_head_s": times}
 
 
-def run_reference(args, rank, world):
-    if rank != 0:
+def run_reference(args, rk):
+    if rk.rank != 0:  # the CPU oracle runs once, on rank 0; the other ranks exit
         return
+    world = rk.world
     w = WORKLOADS[args.workload]
     cb = cpu_baseline(w, steps=args.steps, warmup=args.warmup)
     out = {"impl": "reference", "metric": METRIC, "value": cb["value"], "unit": "tokens/s",
@@ -469,22 +458,17 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3) if args.impl == "ours" else args.warmup
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    rk = replicas.from_env()
     if args.impl == "reference":
-        run_reference(args, rank, world)
+        run_reference(args, rk)
         return
-    if world > 1:
-        import datetime
-        torch.cuda.set_device(local_rank)
-        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
-                                             device_id=torch.device("cuda", local_rank))
+    if rk.multi:
+        torch.cuda.set_device(rk.local_rank)
+    replicas.init(rk, "nccl", 300.0, torch.device("cuda", rk.local_rank) if rk.multi else None)
     try:
-        run_ours(args, rank, world, local_rank)
+        run_ours(args, rk)
     finally:
-        if world > 1:
-            torch.distributed.destroy_process_group()
+        replicas.finish(rk)
 
 
 if __name__ == "__main__":

@@ -89,10 +89,13 @@ def _gen(device, seed: int) -> torch.Generator:
     return g
 
 
-def make_inputs(w: Workload, device="cpu", with_dO: bool = True):
-    """Draw q, k, v (and dO) of shape [B, H, N, d] in the workload's dtype."""
+def make_inputs(w: Workload, device="cpu", with_dO: bool = True, batch: int = 0):
+    """Draw q, k, v (and dO) of shape [B, H, N, d] in the workload's dtype.
+
+    batch selects an independent draw of the same workload (the replica a rank
+    of a multi-GPU run processes); batch 0 is the draw every test uses."""
     device = torch.device(device)
-    salt = 0x1F1F * w.wid
+    salt = 0x1F1F * w.wid + 0x9E3779B1 * batch
     shape = (w.B, w.H, w.N, w.d)
     out = {}
     scale_tok = None
