@@ -41,10 +41,6 @@ constexpr float kLog2e = 1.4426950408889634f;
 constexpr int kThreads = 320;
 constexpr uint32_t kTmemCols = 512;
 
-__device__ __forceinline__ void rows_bar() {  // the 8 row-work warps only
-  asm volatile("bar.sync 1, 256;\n" ::: "memory");
-}
-
 // Two tcgen05.ld of 32 columns each, then one wait.
 __device__ __forceinline__ void tmem_ld64(uint32_t taddr, uint32_t (&a)[32], uint32_t (&b)[32]) {
   tmem_ld32(taddr, a);
@@ -61,47 +57,71 @@ __device__ __forceinline__ void store_row_half(uint8_t* tile_half, int r, const 
 }
 
 // ================================================================= forward
+// Column groups: every 128-key tile is split into NG groups of CW = 128/NG
+// keys; the 4 warps of group g (one per TMEM lane quarter) own the keys of
+// group g in every tile, with their own running reference max, sum and TMEM
+// accumulator O_g (D columns).  NG = 2: eight row-work warps, two per SM
+// sub-partition (four groups, 16 warps, measured slower at d = 64: the
+// per-thread register cap of 18 warps and four P handoffs per tile).
+template <int D>
+struct FwdCfg {
+  static constexpr int NG = 2;
+  static constexpr int CW = 128 / NG;        // keys per group and tile
+  static constexpr int kRowWarps = 4 * NG;
+  static constexpr int kTmaWarp = kRowWarps, kMmaWarp = kRowWarps + 1;
+  static constexpr int kThreads = 32 * (kRowWarps + 2);
+  static constexpr int OC = D / NG;          // output columns per thread
+  static_assert(256 + NG * D <= (int)kTmemCols, "TMEM: two S buffers and NG accumulators");
+  static_assert(CW % 64 == 0, "P of a group is stored as whole 32-column TMEM stores");
+};
+
+template <int NG>
 struct FwdBars {
   uint64_t q_full;
-  uint64_t kv_full[3], kv_empty[3];
+  uint64_t kv_full[4], kv_empty[4];
   uint64_t s_full[2], s_free[2];
-  uint64_t p_full[2], pv_done[2], mma_done;  // [column half]
+  uint64_t p_full[NG], pv_done[NG], mma_done;  // [column group]
   uint32_t tmem;
   int abort;
-  float xm[2][128], xl[2][128];  // [half][row] final max and sum
+  float xm[NG][128], xl[NG][128];  // [group][row] final reference max and sum
 };
 
 template <int D>
 struct FwdLayout {
-  static constexpr int kKS = (D == 64) ? 3 : 2;  // K/V stages
+  static constexpr int kKS = (D == 64) ? 4 : 2;  // K/V stages
   static constexpr int kTile = 128 * D * 2;
   static constexpr int kQ = 0;
   static constexpr int kK = kQ + kTile;
   static constexpr int kV = kK + kKS * kTile;
-  static constexpr int kP = kV + kKS * kTile;  // 128 x 128 fp16
-  static constexpr int kBar = kP + 32768;
-  static constexpr int kBytes = kBar + (int)sizeof(FwdBars);
+  static constexpr int kBar = kV + kKS * kTile;  // (P lives in TMEM, over S)
+  static constexpr int kBytes = kBar + (int)sizeof(FwdBars<FwdCfg<D>::NG>);
 };
 
+template <int NT>
+__device__ __forceinline__ void named_bar() {  // the NT row-work threads only
+  asm volatile("bar.sync 1, %0;\n" ::"n"(NT) : "memory");
+}
+
 template <int D>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(FwdCfg<D>::kThreads, 1)
     k_attn_fwd_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
                   const __grid_constant__ CUtensorMap tv, __half* __restrict__ os,
                   float* __restrict__ lse, int S, int unit0, int nunits, float scale_log2,
                   int ntiles) {
   using Lt = FwdLayout<D>;
+  using Cf = FwdCfg<D>;
+  constexpr int NG = Cf::NG, CW = Cf::CW;
   constexpr int KS = Lt::kKS;
-  static_assert(KS >= 2 && KS <= 3, "FwdBars holds at most 3 stages; the protocol needs 2");
+  static_assert(KS >= 2 && KS <= 4, "FwdBars holds at most 4 stages; the protocol needs 2");
   extern __shared__ __align__(1024) uint8_t smem[];
   if (smem_u32(smem) & 1023u) {
     if (threadIdx.x == 0) report_status(kStatusAttnFwdTimeout | 1u);
     return;
   }
-  FwdBars* bars = reinterpret_cast<FwdBars*>(smem + Lt::kBar);
+  auto* bars = reinterpret_cast<FwdBars<NG>*>(smem + Lt::kBar);
   uint8_t* sQ = smem + Lt::kQ;
   uint8_t* sK = smem + Lt::kK;
   uint8_t* sV = smem + Lt::kV;
-  uint8_t* sP = smem + Lt::kP;
   volatile int* abort = &bars->abort;
   constexpr uint32_t kStatus = kStatusAttnFwdTimeout;
 
@@ -119,25 +139,26 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&bars->s_full[b], 1);
-      mbar_init(&bars->s_free[b], 8);
+      mbar_init(&bars->s_free[b], Cf::kRowWarps);
     }
-    for (int h = 0; h < 2; ++h) {
-      mbar_init(&bars->p_full[h], 4);
-      mbar_init(&bars->pv_done[h], 1);
+    for (int g = 0; g < NG; ++g) {
+      mbar_init(&bars->p_full[g], 4);
+      mbar_init(&bars->pv_done[g], 1);
     }
     mbar_init(&bars->mma_done, 1);
     bars->abort = 0;
     mbar_init_fence();
   }
-  if (warp == 9) tmem_alloc(&bars->tmem, kTmemCols);
+  if (warp == Cf::kMmaWarp) tmem_alloc(&bars->tmem, kTmemCols);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = bars->tmem;
-  // O_h (h = key half of every tile) accumulates at tmem + 256 + h * D
+  // S double buffer at tmem + 0 / + 128 (P_g of a tile is written over the first
+  // CW/2 of its group's S columns); O_g at tmem + 256 + g * D
   const uint32_t tO = tmem + 256;
 
-  if (warp == 8) {
+  if (warp == Cf::kTmaWarp) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
       mbar_expect_tx(&bars->q_full, Lt::kTile);
@@ -158,26 +179,28 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int j = (issued > KS ? issued - KS : 0); j < issued; ++j)
         mbar_wait(&bars->kv_full[j % KS], (j / KS) & 1, abort, kStatus, false);
     }
-  } else if (warp == 9) {
+  } else if (warp == Cf::kMmaWarp) {
     // -------------------------------------------------------------- MMA issuer
     if (lane == 0) {
       constexpr uint32_t idS = idesc_f16(128, 128, false);
       constexpr uint32_t idPV = idesc_f16(128, D, true);
-      const uint32_t aQ = smem_u32(sQ), aK = smem_u32(sK), aV = smem_u32(sV), aP = smem_u32(sP);
-      // O_h += P[:, keys of half h] V[keys of half h, :], once the row work
-      // of half h has stored its P
+      const uint32_t aQ = smem_u32(sQ), aK = smem_u32(sK), aV = smem_u32(sV);
+      // O_g += P[:, keys of group g] V[keys of group g, :], once group g has
+      // written its P (TMEM, over S of tile i) -- issued before S of tile i + 2
+      // overwrites that buffer
       auto issue_pv = [&](int i) {
         const int st = i % KS;
-        for (int h = 0; h < 2; ++h) {
-          if (!mbar_wait(&bars->p_full[h], i & 1, abort, kStatus)) return false;
+        const uint32_t tP = tmem + (i & 1) * 128;
+        for (int g = 0; g < NG; ++g) {
+          if (!mbar_wait(&bars->p_full[g], i & 1, abort, kStatus)) return false;
           tc_fence_after();
 #pragma unroll
-          for (int k4 = 0; k4 < 4; ++k4) {
-            const int kk = h * 4 + k4;
-            umma_f16(tO + h * D, desc_kmajor(aP + h * 16384 + k4 * 32),
-                     desc_mnmajor(aV + st * Lt::kTile + kk * 2048, 16384), idPV, (i > 0 || k4 > 0));
+          for (int k = 0; k < CW / 16; ++k) {
+            const int kk = g * (CW / 16) + k;  // 16-key step within the tile
+            umma_f16_ta(tO + g * D, tP + g * CW + 8 * k,
+                        desc_mnmajor(aV + st * Lt::kTile + kk * 2048, 16384), idPV, (i > 0 || k > 0));
           }
-          umma_commit(&bars->pv_done[h]);
+          umma_commit(&bars->pv_done[g]);
         }
         umma_commit(&bars->kv_empty[st]);
         return true;
@@ -203,19 +226,19 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_wait(&bars->mma_done, 0, abort, kStatus, false);
     }
   } else {
-    // ------------------------------------------- row work: two threads per row
-    // Thread (row r, half h) owns the 64 keys of half h in every tile and the
-    // partial softmax over them: its own running reference max m_ref, sum l
-    // and accumulator O_h in TMEM.  No exchange is needed until the end, where
-    // the two partials of a row are combined (the usual split-softmax merge).
-    // P is formed against m_ref, and O_h is rescaled in TMEM only when a tile's
-    // max exceeds m_ref by more than kRescale (exp2 domain), so P <= 2^kRescale
-    // fits fp16; softmax is invariant to the reference, so the result is the same.
+    // ------------------------------------ row work: NG threads per row (one per group)
+    // Thread (row r, group g) owns the CW keys of group g in every tile and the
+    // partial softmax over them: its own running reference max m_ref, sum l and
+    // accumulator O_g in TMEM.  Nothing is exchanged until the end, where the NG
+    // partials of a row are merged (the usual split-softmax merge).  P is formed
+    // against m_ref, and O_g is rescaled in TMEM only when a tile's max exceeds
+    // m_ref by more than kRescale (exp2 domain), so P <= 2^kRescale fits fp16;
+    // softmax is invariant to the reference, so the result is the same.
     constexpr float kRescale = 8.0f;
-    const int qd = warp & 3, h = warp >> 2;
+    const int qd = warp & 3, g = warp >> 2;
     const int r = qd * 32 + lane;
     const uint32_t lane_addr = (uint32_t)(qd * 32) << 16;
-    const uint32_t tOh = tO + h * D + lane_addr;
+    const uint32_t tOg = tO + g * D + lane_addr;
     float m_ref = -INFINITY, l = 0.0f;
     bool ok = true;
     // one key tile; kDiag: the last (diagonal) tile, keys past the row masked
@@ -225,121 +248,146 @@ __global__ void __launch_bounds__(kThreads, 1)
       ok = warp_wait(&bars->s_full[b], (j >> 1) & 1, abort, kStatus);
       if (!ok) return;
       tc_fence_after();
-      uint32_t v0[32], v1[32];
-      tmem_ld64(tmem + b * 128 + lane_addr + h * 64, v0, v1);
+      uint32_t v[CW];
+#pragma unroll
+      for (int c = 0; c < CW / 32; ++c)
+        tmem_ld32(tmem + b * 128 + lane_addr + g * CW + 32 * c,
+                  reinterpret_cast<uint32_t(&)[32]>(v[32 * c]));
+      tmem_ld_wait();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars->s_free[b]);  // S is in registers now
-      const int lim = r - h * 64;                     // keys i <= lim are visible
-      float mx = -INFINITY;
+      const int lim = r - g * CW;                     // keys i <= lim are visible
+      // row max: four independent chains (max is exact in any order)
+      float mc[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-      for (int i = 0; i < 32; ++i) {
+      for (int i = 0; i < CW; i += 2) {
+        const int c = (i >> 1) & 3;
         if (kDiag) {
-          mx = max3(mx, i <= lim ? __uint_as_float(v0[i]) : -INFINITY,
-                    i + 32 <= lim ? __uint_as_float(v1[i]) : -INFINITY);
+          mc[c] = max3(mc[c], i <= lim ? __uint_as_float(v[i]) : -INFINITY,
+                       i + 1 <= lim ? __uint_as_float(v[i + 1]) : -INFINITY);
         } else {
-          mx = max3(mx, __uint_as_float(v0[i]), __uint_as_float(v1[i]));
+          mc[c] = max3(mc[c], __uint_as_float(v[i]), __uint_as_float(v[i + 1]));
         }
       }
+      float mx = fmaxf(max3(mc[0], mc[1], mc[2]), mc[3]);
       mx *= scale_log2;
       const bool grow = mx > m_ref + kRescale;
       const float m_new = grow ? mx : m_ref;
-      if (j > 0) {
-        // P_h of the previous tile must be consumed before this one is stored,
-        // and O_h must be complete before it is rescaled
-        ok = warp_wait(&bars->pv_done[h], (j - 1) & 1, abort, kStatus);
-        if (!ok) return;
-        if (__any_sync(0xffffffffu, grow)) {
-          tc_fence_after();
-          const float alpha = ex2(m_ref - m_new);  // 1 for rows that do not grow
-#pragma unroll
-          for (int c = 0; c < D / 32; ++c) {
-            uint32_t ov[32];
-            tmem_ld32(tOh + c * 32, ov);
-            tmem_ld_wait();
-#pragma unroll
-            for (int i = 0; i < 32; ++i) ov[i] = __float_as_uint(__uint_as_float(ov[i]) * alpha);
-            tmem_st32(tOh + c * 32, ov);
-          }
-          tmem_st_wait();
-          l *= alpha;
-        }
-      }
-      m_ref = m_new;
-      // a fully masked half (only in the diagonal tile) has m_ref = -inf: its
+      // P first (against the new reference), so S is dead before O is touched;
+      // a fully masked group (only in the diagonal tile) has m_new = -inf: its
       // exponent is NaN but every one of its elements is replaced by 0 below
-      uint32_t pk[32];
-      const float2 cc = make_float2(scale_log2, scale_log2), nm = make_float2(-m_ref, -m_ref);
-      float2 sa = make_float2(0.0f, 0.0f), sb = make_float2(0.0f, 0.0f);
+      uint32_t pk[CW / 2];
+      const float2 cc = make_float2(scale_log2, scale_log2), nm = make_float2(-m_new, -m_new);
+      // row sum: four independent paired accumulators
+      float2 sacc[4] = {make_float2(0.0f, 0.0f), make_float2(0.0f, 0.0f), make_float2(0.0f, 0.0f),
+                        make_float2(0.0f, 0.0f)};
 #pragma unroll
-      for (int i = 0; i < 32; i += 2) {
-        const float2 x = ffma2(make_float2(__uint_as_float(v0[i]), __uint_as_float(v0[i + 1])), cc, nm);
-        const float2 y = ffma2(make_float2(__uint_as_float(v1[i]), __uint_as_float(v1[i + 1])), cc, nm);
+      for (int i = 0; i < CW; i += 4) {
+        const float2 x = ffma2(make_float2(__uint_as_float(v[i]), __uint_as_float(v[i + 1])), cc, nm);
+        const float2 y = ffma2(make_float2(__uint_as_float(v[i + 2]), __uint_as_float(v[i + 3])), cc, nm);
         float2 p = make_float2(ex2(x.x), ex2(x.y));
         float2 q = make_float2(ex2(y.x), ex2(y.y));
         if (kDiag) {
           p.x = i <= lim ? p.x : 0.0f;
           p.y = i + 1 <= lim ? p.y : 0.0f;
-          q.x = i + 32 <= lim ? q.x : 0.0f;
-          q.y = i + 33 <= lim ? q.y : 0.0f;
+          q.x = i + 2 <= lim ? q.x : 0.0f;
+          q.y = i + 3 <= lim ? q.y : 0.0f;
         }
-        sa = fadd2(sa, p);
-        sb = fadd2(sb, q);
+        const int c = (i >> 2) & 1;
+        sacc[2 * c] = fadd2(sacc[2 * c], p);
+        sacc[2 * c + 1] = fadd2(sacc[2 * c + 1], q);
         pk[i >> 1] = h2(p.x, p.y);
-        pk[16 + (i >> 1)] = h2(q.x, q.y);
+        pk[(i >> 1) + 1] = h2(q.x, q.y);
       }
-      store_row_half(sP + h * 16384, r, pk);
-      tc_fence_before();  // orders the O_h rescale (TMEM stores) before the next product
-      fence_async_smem();
+      // every phase of pv_done[g] is waited for, in order (a parity wait must
+      // never run two phases ahead of the barrier); the previous tile's product
+      // is normally complete by now.  O_g must be complete before a rescale.
+      if (j > 0) {
+        ok = warp_wait(&bars->pv_done[g], (j - 1) & 1, abort, kStatus);
+        if (!ok) return;
+      }
+      if (j > 0 && __any_sync(0xffffffffu, grow)) {
+        tc_fence_after();
+        const float alpha = ex2(m_ref - m_new);  // 1 for rows that do not grow
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t ov[32];
+          tmem_ld32(tOg + c * 32, ov);
+          tmem_ld_wait();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) ov[i] = __float_as_uint(__uint_as_float(ov[i]) * alpha);
+          tmem_st32(tOg + c * 32, ov);
+        }
+        l *= alpha;
+      }
+      m_ref = m_new;
+      // P (CW keys = CW/2 packed columns) over this group's S columns of buffer b
+#pragma unroll
+      for (int c = 0; c < CW / 64; ++c)
+        tmem_st32(tmem + b * 128 + lane_addr + g * CW + 32 * c,
+                  reinterpret_cast<const uint32_t(&)[32]>(pk[32 * c]));
+      tmem_st_wait();
+      tc_fence_before();  // orders P and the O_g rescale (TMEM stores) before the product
       __syncwarp();
-      if (lane == 0) mbar_arrive(&bars->p_full[h]);
-      l += (sa.x + sa.y) + (sb.x + sb.y);
+      if (lane == 0) mbar_arrive(&bars->p_full[g]);
+      const float2 s01 = fadd2(sacc[0], sacc[1]), s23 = fadd2(sacc[2], sacc[3]);
+      l += (s01.x + s01.y) + (s23.x + s23.y);
     };
     for (int j = 0; j < n - 1 && ok; ++j) step(j, std::false_type{});
     if (ok) step(n - 1, std::true_type{});
-    if (ok) ok = warp_wait(&bars->pv_done[h], (n - 1) & 1, abort, kStatus);
-    // merge the two halves of each row: O = sum_h 2^(m_h - m) O_h / sum_h 2^(m_h - m) l_h
-    bars->xm[h][r] = m_ref;
-    bars->xl[h][r] = l;
-    rows_bar();
-    const float m0 = bars->xm[0][r], m1 = bars->xm[1][r];
-    const float m = fmaxf(m0, m1);  // finite: key 0 of half 0 is visible to every row
-    const float w0 = ex2(m0 - m), w1 = ex2(m1 - m);
-    const float lt = w0 * bars->xl[0][r] + w1 * bars->xl[1][r];
+    if (ok) ok = warp_wait(&bars->pv_done[g], (n - 1) & 1, abort, kStatus);
+    // merge the NG partials of each row:
+    //   O = sum_q 2^(m_q - m) O_q / sum_q 2^(m_q - m) l_q,  m = max_q m_q
+    bars->xm[g][r] = m_ref;
+    bars->xl[g][r] = l;
+    named_bar<32 * Cf::kRowWarps>();
+    float m = bars->xm[0][r];  // finite: key 0 of group 0 is visible to every row
+#pragma unroll
+    for (int q = 1; q < NG; ++q) m = fmaxf(m, bars->xm[q][r]);
+    float wq[NG];
+    float lt = 0.0f;
+#pragma unroll
+    for (int q = 0; q < NG; ++q) {
+      wq[q] = ex2(bars->xm[q][r] - m);
+      lt = __fmaf_rn(wq[q], bars->xl[q][r], lt);
+    }
     const int row = qt * 128 + r;
     if (ok) {  // whole warps load TMEM; only rows inside the sequence are stored
       tc_fence_after();
-      constexpr int DH = D / 2;  // output columns of this thread
+      constexpr int OC = Cf::OC;  // output columns of this thread: [g*OC, (g+1)*OC)
       const float inv = 1.0f / lt;
-      const float2 c0 = make_float2(w0 * inv, w0 * inv), c1 = make_float2(w1 * inv, w1 * inv);
-      __half* dst = os + ((int64_t)u * S + row) * D + h * DH;
 #pragma unroll
-      for (int c = 0; c < DH / 32; ++c) {
-        uint32_t o0[32], o1[32];
-        tmem_ld32(tO + lane_addr + h * DH + c * 32, o0);
-        tmem_ld32(tO + D + lane_addr + h * DH + c * 32, o1);
-        tmem_ld_wait();
+      for (int q = 0; q < NG; ++q) wq[q] *= inv;
+      __half* dst = os + ((int64_t)u * S + row) * D + g * OC;
+#pragma unroll
+      for (int c = 0; c < OC / 16; ++c) {
+        float f[16];
+#pragma unroll
+        for (int q = 0; q < NG; ++q) {
+          uint32_t ov[16];
+          tmem_ld16(tO + q * D + lane_addr + g * OC + 16 * c, ov);
+          tmem_ld_wait();
+#pragma unroll
+          for (int i = 0; i < 16; ++i)
+            f[i] = q == 0 ? __uint_as_float(ov[i]) * wq[0] : __fmaf_rn(__uint_as_float(ov[i]), wq[q], f[i]);
+        }
         if (row < S) {
-#pragma unroll
-          for (int x = 0; x < 4; ++x) {
-            uint32_t w[4];
-#pragma unroll
-            for (int y = 0; y < 4; ++y) {
-              const int e = 8 * x + 2 * y;
-              const float2 f = ffma2(make_float2(__uint_as_float(o1[e]), __uint_as_float(o1[e + 1])), c1,
-                                     fmul2(make_float2(__uint_as_float(o0[e]), __uint_as_float(o0[e + 1])), c0));
-              w[y] = h2_sat(f.x, f.y);
-            }
-            *reinterpret_cast<uint4*>(dst + c * 32 + 8 * x) = make_uint4(w[0], w[1], w[2], w[3]);
-          }
+          uint4 w0, w1;
+          w0.x = h2_sat(f[0], f[1]);   w0.y = h2_sat(f[2], f[3]);
+          w0.z = h2_sat(f[4], f[5]);   w0.w = h2_sat(f[6], f[7]);
+          w1.x = h2_sat(f[8], f[9]);   w1.y = h2_sat(f[10], f[11]);
+          w1.z = h2_sat(f[12], f[13]); w1.w = h2_sat(f[14], f[15]);
+          *reinterpret_cast<uint4*>(dst + 16 * c) = w0;
+          *reinterpret_cast<uint4*>(dst + 16 * c + 8) = w1;
         }
       }
-      if (h == 0 && row < S) lse[(int64_t)u * S + row] = (m + __log2f(lt)) * kLn2;
+      if (g == 0 && row < S) lse[(int64_t)u * S + row] = (m + __log2f(lt)) * kLn2;
     }
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 9) {
+  if (warp == Cf::kMmaWarp) {
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);
   }
@@ -879,7 +927,7 @@ cudaError_t fwd_d(const Geom& g, const __half* qs, const __half* ks, const __hal
   const int64_t per = 0x7fffffff / ntiles;  // units per launch (grid.x limit)
   for (int64_t u0 = 0; u0 < g.U; u0 += per) {
     const int64_t nu = g.U - u0 < per ? g.U - u0 : per;
-    k_attn_fwd_tc<D><<<(unsigned)(nu * ntiles), kThreads, smem, st>>>(
+    k_attn_fwd_tc<D><<<(unsigned)(nu * ntiles), FwdCfg<D>::kThreads, smem, st>>>(
         mq, mk, mv, os, lse, (int)g.S, (int)u0, (int)nu, scale * kLog2e, ntiles);
   }
   return cudaGetLastError();
