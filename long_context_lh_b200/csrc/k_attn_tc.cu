@@ -397,11 +397,12 @@ __global__ void __launch_bounds__(FwdCfg<D>::kThreads, 1)
 // One CTA per (unit, 128-key tile kt), walking the query tiles i >= kt:
 // S^T = K Q_i^T and dP^T = V dO_i^T in TMEM; two threads per key row form
 // P^T = 2^(S^T c - lse2) (zero where the query precedes the key) and
-// dS^T = P^T (dP^T - D) in fp16 shared memory; dV += P^T dO_i and dK += dS^T Q_i
-// accumulate in TMEM over all query tiles (fixed order, no atomics).
+// dS^T = P^T (dP^T - D) in fp16 -- in TMEM at d = 64 (columns 384..511, read
+// as the A operand), in shared memory at d = 128 (TMEM full); dV += P^T dO_i and
+// dK += dS^T Q_i accumulate in TMEM over all query tiles (fixed order, no atomics).
 struct DkvBars {
   uint64_t kv_full;
-  uint64_t q_full[3], q_empty[3];  // [stage], at most 3 stages
+  uint64_t q_full[4], q_empty[4];  // [stage], at most 4 stages
   uint64_t s_full, st_free, p_full, pdone, mma_done;
   uint32_t tmem;
   int abort;
@@ -409,15 +410,16 @@ struct DkvBars {
 
 template <int D>
 struct DkvLayout {
-  static constexpr int kStages = (D == 64) ? 3 : 1;  // DkvBars holds up to 3
+  static constexpr bool kTmemP = (D == 64);  // P^T, dS^T in TMEM (else shared memory)
+  static constexpr int kStages = (D == 64) ? 4 : 1;  // DkvBars holds up to 4
   static constexpr int kTile = 128 * D * 2;
   static constexpr int kK = 0;
   static constexpr int kV = kK + kTile;
   static constexpr int kQ = kV + kTile;
   static constexpr int kDO = kQ + kStages * kTile;
   static constexpr int kPT = kDO + kStages * kTile;
-  static constexpr int kDST = kPT + 32768;
-  static constexpr int kStat = kDST + 32768;  // per stage: -lse2[128], -D[128]
+  static constexpr int kDST = kPT + (kTmemP ? 0 : 32768);
+  static constexpr int kStat = kDST + (kTmemP ? 0 : 32768);  // per stage: -lse2[128], -D[128]
   static constexpr int kBar = kStat + kStages * 1024;
   static constexpr int kBytes = kBar + (int)sizeof(DkvBars);
 };
@@ -431,7 +433,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                        int nunits, float scale, float scale_log2, int ntiles) {
   using Lt = DkvLayout<D>;
   constexpr int STG = Lt::kStages;
-  static_assert(STG >= 1 && STG <= 3, "DkvBars holds at most 3 stages");
+  static_assert(STG >= 1 && STG <= 4, "DkvBars holds at most 4 stages");
+  constexpr bool kTmemP = Lt::kTmemP;
   extern __shared__ __align__(1024) uint8_t smem[];
   if (smem_u32(smem) & 1023u) {
     if (threadIdx.x == 0) report_status(kStatusAttnBwdTimeout | 1u);
@@ -474,6 +477,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = bars->tmem;
   const uint32_t tST = tmem, tDPT = tmem + 128, tDV = tmem + 256, tDK = tmem + 256 + D;
+  const uint32_t tPT = tmem + 384, tDST = tmem + 448;  // P^T, dS^T packed fp16 (kTmemP)
 
   if (warp == 8) {
     // TMA producer: K, V once; per query tile Q, dO and the tile's statistics
@@ -511,8 +515,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int kk = 0; kk < 8; ++kk) {
           const uint32_t a = (kk >> 2) * 16384 + (kk & 3) * 32;
           const uint32_t b = st * Lt::kTile + kk * 2048;
-          umma_f16(tDV, desc_kmajor(aPT + a), desc_mnmajor(aDO + b, 16384), idAcc, (t > 0 || kk > 0));
-          umma_f16(tDK, desc_kmajor(aDST + a), desc_mnmajor(aQ + b, 16384), idAcc, (t > 0 || kk > 0));
+          if constexpr (kTmemP) {
+            umma_f16_ta(tDV, tPT + 8 * kk, desc_mnmajor(aDO + b, 16384), idAcc, (t > 0 || kk > 0));
+            umma_f16_ta(tDK, tDST + 8 * kk, desc_mnmajor(aQ + b, 16384), idAcc, (t > 0 || kk > 0));
+          } else {
+            umma_f16(tDV, desc_kmajor(aPT + a), desc_mnmajor(aDO + b, 16384), idAcc, (t > 0 || kk > 0));
+            umma_f16(tDK, desc_kmajor(aDST + a), desc_mnmajor(aQ + b, 16384), idAcc, (t > 0 || kk > 0));
+          }
         }
         umma_commit(&bars->pdone);
         umma_commit(&bars->q_empty[st]);
@@ -608,9 +617,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         quad(e + 32, a1, b1);
       }
       if (t > 0 && !(ok = warp_wait(&bars->pdone, (t - 1) & 1, abort, kStatus))) return;
-      store_row_half(sPT + h * 16384, r, pp);
-      store_row_half(sDST + h * 16384, r, pd);
-      fence_async_smem();
+      if constexpr (kTmemP) {  // this row's 64 query columns = 32 packed columns
+        tmem_st32(tPT + lane_addr + h * 32, pp);
+        tmem_st32(tDST + lane_addr + h * 32, pd);
+        tmem_st_wait();
+        tc_fence_before();
+      } else {
+        store_row_half(sPT + h * 16384, r, pp);
+        store_row_half(sDST + h * 16384, r, pd);
+        fence_async_smem();
+      }
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars->p_full);
     };
@@ -659,10 +675,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 // ============================================================= backward: dQ
 // One CTA per (unit, 128-query tile qt), walking the key tiles j <= qt:
 // S = Q K_j^T, dP = dO V_j^T in TMEM; two threads per query row form
-// dS = P (dP - D) in fp16 shared memory (double-buffered); dQ += dS K_j in TMEM.
+// dS = P (dP - D) in fp16, double-buffered in TMEM (read as the A operand);
+// dQ += dS K_j in TMEM.
 struct DqBars {
   uint64_t q_full;
-  uint64_t kv_full[3], kv_empty[3];  // [stage], at most 3 stages
+  uint64_t kv_full[4], kv_empty[4];  // [stage], at most 4 stages
   uint64_t s_full, s_free, mma_done;
   uint64_t ds_full[2], dsdone[2];
   uint32_t tmem;
@@ -671,14 +688,13 @@ struct DqBars {
 
 template <int D>
 struct DqLayout {
-  static constexpr int kStages = (D == 64) ? 3 : 1;  // DqBars holds up to 3
+  static constexpr int kStages = (D == 64) ? 4 : 2;  // DqBars holds up to 4
   static constexpr int kTile = 128 * D * 2;
   static constexpr int kQ = 0;
   static constexpr int kDO = kQ + kTile;
   static constexpr int kK = kDO + kTile;
   static constexpr int kV = kK + kStages * kTile;
-  static constexpr int kDS = kV + kStages * kTile;  // 2 buffers of 128 x 128 fp16
-  static constexpr int kBar = kDS + 2 * 32768;
+  static constexpr int kBar = kV + kStages * kTile;  // (dS lives in TMEM)
   static constexpr int kBytes = kBar + (int)sizeof(DqBars);
 };
 
@@ -691,7 +707,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                      float scale_log2, int ntiles) {
   using Lt = DqLayout<D>;
   constexpr int STG = Lt::kStages;
-  static_assert(STG >= 1 && STG <= 3, "DqBars holds at most 3 stages");
+  static_assert(STG >= 1 && STG <= 4, "DqBars holds at most 4 stages");
   extern __shared__ __align__(1024) uint8_t smem[];
   if (smem_u32(smem) & 1023u) {
     if (threadIdx.x == 0) report_status(kStatusAttnBwdTimeout | 2u);
@@ -702,7 +718,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* sDO = smem + Lt::kDO;
   uint8_t* sK = smem + Lt::kK;
   uint8_t* sV = smem + Lt::kV;
-  uint8_t* sDS = smem + Lt::kDS;
   volatile int* abort = &bars->abort;
   constexpr uint32_t kStatus = kStatusAttnBwdTimeout;
 
@@ -733,6 +748,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = bars->tmem;
   const uint32_t tS = tmem, tDP = tmem + 128, tDQ = tmem + 256;
+  const uint32_t tDS = tmem + 256 + D;  // 2 buffers of 64 packed fp16 columns (dS of a tile)
 
   if (warp == 8) {
     if (lane == 0) {
@@ -761,17 +777,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       constexpr uint32_t idS = idesc_f16(128, 128, false);
       constexpr uint32_t idAcc = idesc_f16(128, D, true);
       const uint32_t aQ = smem_u32(sQ), aDO = smem_u32(sDO), aK = smem_u32(sK), aV = smem_u32(sV);
-      const uint32_t aDS = smem_u32(sDS);
-      auto issue_dq = [&](int j) {  // dQ += dS_j K_j
+      auto issue_dq = [&](int j) {  // dQ += dS_j K_j, dS_j from TMEM
         const int st = j % STG, b = j & 1;
         if (!mbar_wait(&bars->ds_full[b], (j >> 1) & 1, abort, kStatus)) return false;
         tc_fence_after();
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint32_t a = aDS + b * 32768 + (kk >> 2) * 16384 + (kk & 3) * 32;
-          umma_f16(tDQ, desc_kmajor(a), desc_mnmajor(aK + st * Lt::kTile + kk * 2048, 16384), idAcc,
-                   (j > 0 || kk > 0));
-        }
+        for (int kk = 0; kk < 8; ++kk)
+          umma_f16_ta(tDQ, tDS + b * 64 + 8 * kk,
+                      desc_mnmajor(aK + st * Lt::kTile + kk * 2048, 16384), idAcc, (j > 0 || kk > 0));
         umma_commit(&bars->dsdone[b]);
         umma_commit(&bars->kv_empty[st]);
         return true;
@@ -844,8 +857,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       const int b = j & 1;
       if (j >= 2 && !(ok = warp_wait(&bars->dsdone[b], ((j - 2) >> 1) & 1, abort, kStatus))) return;
-      store_row_half(sDS + b * 32768 + h * 16384, r, pd);
-      fence_async_smem();
+      tmem_st32(tDS + b * 64 + lane_addr + h * 32, pd);  // 64 key columns, packed
+      tmem_st_wait();
+      tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars->ds_full[b]);
     };
