@@ -287,7 +287,8 @@ __global__ void __launch_bounds__(FwdCfg<D>::kThreads, 1)
         const float2 x = ffma2(make_float2(__uint_as_float(v[i]), __uint_as_float(v[i + 1])), cc, nm);
         const float2 y = ffma2(make_float2(__uint_as_float(v[i + 2]), __uint_as_float(v[i + 3])), cc, nm);
         float2 p = make_float2(ex2(x.x), ex2(x.y));
-        float2 q = make_float2(ex2(y.x), ex2(y.y));
+        // a quarter of the exponentials on the FMA pipe, the rest on MUFU
+        float2 q = (i & 7) == 4 ? ex2_fma2(y) : make_float2(ex2(y.x), ex2(y.y));
         if (kDiag) {
           p.x = i <= lim ? p.x : 0.0f;
           p.y = i + 1 <= lim ? p.y : 0.0f;
