@@ -288,11 +288,9 @@ def run_ours(args, rk):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded N(0,1) Q/K/V/dO, 1% tokens x4; no corpus or weights)",
-        "config": {"workload": f"{w.name}: B={w.B} H={w.H} N={w.N} d={w.d} p={w.p} L={w.L} S={w.S} {w.dtype}",
-                   "B": w.B, "H": w.H, "N": w.N, "d": w.d, "p": w.p, "L": w.L, "S": w.S,
-                   "l2": "inputs larger than L2 (3 x %.0f MB + dO), no flush" % (w.B * w.H * w.N * w.d * 2 / 1e6),
-                   "attention": {0: "tcgen05", 1: "mma_sync", 2: "tcgen05 fwd, mma_sync bwd"}[lh.lh_attention_impl_in_use()],
-                   "parallelism": f"replicas x{world} (heads independent)"},
+        "config": workload_config(w, world,
+                                  {0: "tcgen05", 1: "mma_sync", 2: "tcgen05 fwd, mma_sync bwd"}[
+                                      lh.lh_attention_impl_in_use()]),
         "fwd_tokens_per_s": replicas.job_rate(tokens, world, ms_fwd / 1e3), "ms_fwd": ms_fwd,
         "roofline": roof, "stages": stage_report, "dense_sdpa": dense, "e2e": e2e,
         "gpu_launches": launches * args.steps, "gpu_launches_per_step": launches,
@@ -303,6 +301,15 @@ def run_ours(args, rk):
         if not args.no_cpu:
             out["cpu_baseline"] = cpu_baseline(w, budget_s=args.cpu_budget)
         print(json.dumps(out), flush=True)
+
+
+def workload_config(w, world, attention):
+    """The config object both arms print (same workload, same keys)."""
+    return {"workload": f"{w.name}: B={w.B} H={w.H} N={w.N} d={w.d} p={w.p} L={w.L} S={w.S} {w.dtype}",
+            "B": w.B, "H": w.H, "N": w.N, "d": w.d, "p": w.p, "L": w.L, "S": w.S,
+            "l2": "inputs larger than L2 (3 x %.0f MB + dO), no flush" % (w.B * w.H * w.N * w.d * 2 / 1e6),
+            "attention": attention,
+            "parallelism": f"replicas x{world} (heads independent)"}
 
 
 def launches_per_step(lh, w):
@@ -435,7 +442,8 @@ def run_reference(args, rk):
            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
            "ms_per_step": 1e3 * sum(cb["per_head_s"]) / max(len(cb["per_head_s"]), 1),
            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-           "data": "synthetic", "config": {"workload": f"{w.name} (one head per step)"},
+           "data": "synthetic (seeded N(0,1) Q/K/V/dO, 1% tokens x4; no corpus or weights)",
+           "config": workload_config(w, world, "CPU oracle (fp64), one head per step"),
            "cpu_baseline": {k: cb[k] for k in ("value", "unit", "cores", "kind", "sample")},
            "e2e": {"value": cb["value"], "unit": "tokens/s", "h2d_bytes_per_step": 0,
                    "d2h_bytes_per_step": 0}}
