@@ -39,6 +39,42 @@ METRIC = "Lighthouse layer tokens/s fwd & fwd+bwd at N=98K/512K; % of HBM/TC roo
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
+# DRAM bytes (read + written) per launch of each stage, from one ncu capture of
+# the pretraining workload with 4 heads (profiles/memory_kernels_pretrain_h4.md,
+# profiles/attn_tc_pretrain_h4.md), scaled by the units to the 16-head launch.
+# Each entry carries a hash of the sources its kernels are built from; when they
+# no longer match, the kernel has changed since the counters were taken and the
+# traffic is reported as null.  (At 4 heads part of each stage's writes is still
+# in L2 when it ends, so these undercount writes.)
+MEASURED_TRAFFIC = {  # workload: {stage: (bytes per full launch, sources, sha1[:16])}
+    "pretrain": {
+        "pyramid_score": (8.602e+08, ("k_pyramid.cu", "lh_internal.cuh"), "64fedac8a3e613a7"),
+        "topk": (8.649e+06, ("k_topk.cu", "lh_internal.cuh"), "c32ba6e137685eea"),
+        "gather": (8.584e+07, ("k_gather_scatter.cu", "lh_internal.cuh"), "06de88f37c7464d1"),
+        "scatter": (3.217e+07, ("k_gather_scatter.cu", "lh_internal.cuh"), "06de88f37c7464d1"),
+        "scatter_bwd": (2.167e+08, ("k_gather_scatter.cu", "lh_internal.cuh"), "06de88f37c7464d1"),
+        "gather_bwd": (4.798e+08, ("k_gather_scatter.cu", "lh_internal.cuh"), "06de88f37c7464d1"),
+        "attn_fwd": (5.051e+07, ("k_attn_tc.cu", "tc_common.cuh"), "bd8b1f0925e92946"),
+        "attn_bwd": (1.708e+08, ("k_attn_tc.cu", "tc_common.cuh", "k_gather_scatter.cu",
+                                 "lh_internal.cuh"), "70788de6cb32b83f"),
+    },
+}
+
+
+def measured_traffic(workload: str, stage: str):
+    """DRAM bytes per launch of the stage, or None when unmeasured or stale."""
+    import hashlib
+    ent = MEASURED_TRAFFIC.get(workload, {}).get(stage)
+    if ent is None:
+        return None
+    nbytes, srcs, sha = ent
+    d = hashlib.sha1()
+    for f in srcs:
+        with open(os.path.join(ROOT, "long_context_lh_b200", "csrc", f), "rb") as fh:
+            d.update(fh.read())
+    return nbytes if d.hexdigest()[:16] == sha else None
+
+
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -264,16 +300,20 @@ def run_ours(args, rk):
         else:
             b = alg[s]
             stage_report[s] = {"ms": stage_ms[s], "gbs": b / t / 1e9, "frac_hbm": b / t / 1e9 / hbm}
+        stage_report[s]["traffic"] = measured_traffic(w.name if not args.heads else "", s)
     dominant = max(stages, key=lambda s: stage_ms[s])
     if dominant.startswith("attn"):
         ach = stage_report[dominant]["tflops"]
         roof = {"kernel": dominant, "bound": "tensor", "achieved": ach, "peak": tc,
-                "unit": "TFLOP/s", "frac": ach / tc, "traffic": None,
+                "unit": "TFLOP/s", "frac": ach / tc,
+                "traffic": measured_traffic(w.name if not args.heads else "", dominant),
                 "peak_source": f"{peaks_src} bf16_tflops (burst)"}
     else:
         ach = stage_report[dominant]["gbs"]
         roof = {"kernel": dominant, "bound": "hbm", "achieved": ach, "peak": hbm, "unit": "GB/s",
-                "frac": ach / hbm, "traffic": None, "peak_source": f"{peaks_src} hbm_gbs"}
+                "frac": ach / hbm,
+                "traffic": measured_traffic(w.name if not args.heads else "", dominant),
+                "peak_source": f"{peaks_src} hbm_gbs"}
 
     # dense causal attention (torch SDPA, flash/cuDNN backend) on the same shapes
     dense = None
