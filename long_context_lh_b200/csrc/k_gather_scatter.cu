@@ -252,7 +252,11 @@ __global__ void __launch_bounds__(256) k_scatter(const __half* __restrict__ os,
 // ---------------------------------------------------------- scatter-back bwd
 // dos[k] = sum_{t in span(k)} dO[t] / c_t, as a sum-pyramid of w[t] = dO[t]/c_t
 // over each coarsest span: dO is read once, each selected row written once.
-template <typename Tin, int D, int L>
+// RG row-groups of d/8 lanes share a span (RG = p, or 1): row-group r walks the
+// r-th level-(L-2) entry of the span, and the span's top-level sum is formed
+// from the RG partial sums in order with shuffles -- the same additions, in the
+// same order, as one group walking the whole span (0 + s_0 = s_0 exactly).
+template <typename Tin, int D, int L, int RG>
 __global__ void __launch_bounds__(256) k_scatter_bwd(const Tin* __restrict__ dO,
                                                      const int32_t* __restrict__ slot,
                                                      const float* __restrict__ inv_count,
@@ -261,13 +265,15 @@ __global__ void __launch_bounds__(256) k_scatter_bwd(const Tin* __restrict__ dO,
   constexpr int G = D / 8;
   constexpr int NL = (L > 1) ? (L - 1) : 1;
   constexpr int RB = 4;  // rows of dO whose loads are in flight together
+  static_assert(RG == 1 || (L > 1 && G * RG <= 32), "row-groups of a span share one warp");
   const int64_t gt = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-  const int64_t group = gt / G;
-  if (group >= groups) return;
+  const int64_t group = gt / (G * RG);  // span
+  if (group >= groups) return;          // whole spans leave together (G * RG divides 32)
   const int c = (int)(gt % G);
-  const int32_t Ptop = lv.pw[L - 1];
+  const int rg = (int)((gt / G) % RG);
+  const int32_t Ptop = lv.pw[L - 1] / RG;  // rows this row-group walks
   const int64_t u = group / spans;
-  const int32_t t0 = (int32_t)(group - u * spans) * Ptop;
+  const int32_t t0 = (int32_t)(group - u * spans) * lv.pw[L - 1] + rg * Ptop;
   const int32_t* sl = slot + u * lv.M;
   const Tin* src = dO + (u * lv.N + t0) * D + 8 * c;
   __half* dst = dos + u * lv.S * D + 8 * c;
@@ -328,6 +334,26 @@ __global__ void __launch_bounds__(256) k_scatter_bwd(const Tin* __restrict__ dO,
           cnt[l] = 0;
         }
       }
+    }
+  }
+  if constexpr (RG > 1) {
+    // the span's level-(L-1) entry: its RG partial sums (each row-group's
+    // acc[L-2] holds exactly one level-(L-2) sum) added in row-group order
+    const int lane = threadIdx.x & 31;
+    const int base = lane - rg * G;  // lane of row-group 0 with this chunk
+    const unsigned mask = (G * RG == 32) ? 0xffffffffu
+                                         : (((1u << (G * RG)) - 1u) << (lane & ~(G * RG - 1)));
+    float tot[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) tot[i] = __shfl_sync(mask, acc[NL - 1][i], base);
+#pragma unroll
+    for (int r = 1; r < RG; ++r)
+#pragma unroll
+      for (int i = 0; i < 8; ++i) tot[i] = __fadd_rn(tot[i], __shfl_sync(mask, acc[NL - 1][i], base + r * G));
+    if (rg == 0) {
+      const int32_t j = (t0 + lv.pw[L - 1]) / lv.pw[L - 1] - 1;  // the span's entry at level L-1
+      const int32_t s = __ldg(sl + lv.off[L - 1] + j);
+      if (s >= 0) store8(dst + (int64_t)s * D, tot);
     }
   }
 }
@@ -588,18 +614,25 @@ cudaError_t scatter_bwd_d(const Geom& g, const Tin* dO, const int32_t* slot, con
   const Lv lv = make_lv(g);
   const int64_t spans = g.N / g.pw[g.L - 1];
   const int64_t groups = g.U * spans;
-  const unsigned nb = blocks_for(groups * (D / 8), 256);
-  switch (g.L) {
-#define LH_CASE(LL)                                                                      \
-  case LL:                                                                               \
-    k_scatter_bwd<Tin, D, LL><<<nb, 256, 0, st>>>(dO, slot, ic, dos, lv, spans, groups); \
-    break;
-    LH_CASE(1) LH_CASE(2) LH_CASE(3) LH_CASE(4) LH_CASE(5) LH_CASE(6) LH_CASE(7) LH_CASE(8)
-#undef LH_CASE
-    default:
-      return cudaErrorInvalidValue;
-  }
-  return cudaGetLastError();
+  // row-groups per span: p when p in {2, 4} and the span's lanes fit one warp
+  const int RG = (g.L > 1 && (g.p == 2 || g.p == 4) && (D / 8) * g.p <= 32) ? g.p : 1;
+  const unsigned nb = blocks_for(groups * (D / 8) * RG, 256);
+  return with_levels(g.L, [&](auto lc) {
+    constexpr int LL = decltype(lc)::value;
+    if constexpr (LL > 1) {
+      if (RG == 4) {
+        if constexpr ((D / 8) * 4 <= 32) {
+          k_scatter_bwd<Tin, D, LL, 4><<<nb, 256, 0, st>>>(dO, slot, ic, dos, lv, spans, groups);
+          return;
+        }
+      }
+      if (RG == 2) {
+        k_scatter_bwd<Tin, D, LL, 2><<<nb, 256, 0, st>>>(dO, slot, ic, dos, lv, spans, groups);
+        return;
+      }
+    }
+    k_scatter_bwd<Tin, D, LL, 1><<<nb, 256, 0, st>>>(dO, slot, ic, dos, lv, spans, groups);
+  });
 }
 }  // namespace
 
