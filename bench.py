@@ -321,7 +321,8 @@ def run_ours(args, rk):
         dense = dense_sdpa(w, q, k, v, dO, stream, args)
 
     # end to end through the public API with pinned host buffers
-    e2e = None if args.no_e2e else e2e_run(lh, w, shp, dt, x, dev, stream, args, rk)
+    e2e = None if args.no_e2e else e2e_run(lh, w, shp, dt, x, dev, stream, args, rk,
+                                          {"o": o, "dq": dq, "dk": dk, "dv": dv})
     launches = launches_per_step(lh, w)
     out = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
@@ -395,43 +396,69 @@ def dense_sdpa(w, q, k, v, dO, stream, args):
         return {"error": str(ex)[:200]}
 
 
-def e2e_run(lh, w, shp, dt, x, dev, stream, args, rk):
-    """Same step through lh_forward/lh_backward with host<->device copies inside."""
-    host = {n: t.cpu().pin_memory() for n, t in x.items()}
-    dev_in = {n: torch.empty_like(t) for n, t in x.items()}
-    o = torch.empty_like(x["q"])
-    grads = [torch.empty_like(x["q"]) for _ in range(3)]
-    out_host = [torch.empty(o.shape, dtype=o.dtype).pin_memory() for _ in range(4)]
-    saved = torch.empty(lh.lh_saved_bytes(shp), dtype=torch.uint8, device=dev)
-    wsb = lh.lh_workspace_bytes(shp, dt, True)
+def e2e_run(lh, w, shp, dt, x, dev, stream, args, rk, ref_out):
+    """The step through the public API (lh_forward, lh_backward) with the inputs
+    copied up from pinned host memory and the results copied back inside the
+    timed region.  Units (batch x head) are independent, so the step runs in C
+    chunks of units pipelined over three streams: chunk i+1's inputs go up while
+    chunk i computes and chunk i-1's results come down.  Same bytes and the same
+    work per step as one whole-batch call; each chunk is an lh_forward +
+    lh_backward on a shape with fewer heads."""
+    U = w.B * w.H
+    C = next(c for c in (8, 4, 2, 1) if U % c == 0)
+    uc = U // C
+    shp_c = lh.make_shape(1, uc, w.N, w.d, w.p, w.L, w.S)
+    names_in, names_out = ("q", "k", "v", "dO"), ("o", "dq", "dk", "dv")
+    host_in = {n: x[n].reshape(U, w.N, w.d).cpu().pin_memory() for n in names_in}
+    host_out = {n: torch.empty((U, w.N, w.d), dtype=x["q"].dtype).pin_memory() for n in names_out}
+    dbuf = [{n: torch.empty((uc, w.N, w.d), dtype=x["q"].dtype, device=dev)
+             for n in names_in + names_out} for _ in range(2)]
+    saved = torch.empty(lh.lh_saved_bytes(shp_c), dtype=torch.uint8, device=dev)
+    wsb = lh.lh_workspace_bytes(shp_c, dt, True)
     ws = torch.empty(wsb, dtype=torch.uint8, device=dev)
-    sp = stream.cuda_stream
-    h2d = sum(t.numel() * t.element_size() for t in host.values())
-    d2h = sum(t.numel() * t.element_size() for t in out_host)
+    s_in, s_comp, s_out = torch.cuda.Stream(device=dev), stream, torch.cuda.Stream(device=dev)
+    in_done = [torch.cuda.Event() for _ in range(2)]
+    comp_done = [torch.cuda.Event() for _ in range(2)]
+    out_done = [torch.cuda.Event() for _ in range(2)]
+    h2d = sum(t.numel() * t.element_size() for t in host_in.values())
+    d2h = sum(t.numel() * t.element_size() for t in host_out.values())
+    sp = s_comp.cuda_stream
 
     def step():
-        for n in host:
-            dev_in[n].copy_(host[n], non_blocking=True)
-        lh.lh_forward(shp, dt, dev_in["q"], dev_in["k"], dev_in["v"], 0.0, o, saved, ws, wsb, sp)
-        lh.lh_backward(shp, dt, saved, dev_in["dO"], 0.0, *grads, ws, wsb, sp)
-        for src, dst in zip([o, *grads], out_host):
-            dst.copy_(src, non_blocking=True)
+        for i in range(C):
+            sl, b = slice(i * uc, (i + 1) * uc), dbuf[i & 1]
+            s_in.wait_event(comp_done[i & 1])  # chunk i-2 has read these inputs
+            with torch.cuda.stream(s_in):
+                for n in names_in:
+                    b[n].copy_(host_in[n][sl], non_blocking=True)
+            in_done[i & 1].record(s_in)
+            s_comp.wait_event(in_done[i & 1])
+            s_comp.wait_event(out_done[i & 1])  # chunk i-2's results are down
+            lh.lh_forward(shp_c, dt, b["q"], b["k"], b["v"], 0.0, b["o"], saved, ws, wsb, sp)
+            lh.lh_backward(shp_c, dt, saved, b["dO"], 0.0, b["dq"], b["dk"], b["dv"], ws, wsb, sp)
+            comp_done[i & 1].record(s_comp)
+            s_out.wait_event(comp_done[i & 1])
+            with torch.cuda.stream(s_out):
+                for n in names_out:
+                    host_out[n][sl].copy_(b[n], non_blocking=True)
+            out_done[i & 1].record(s_out)
 
     K = max(1, min(args.steps, 10))
-    with torch.cuda.stream(stream):
+    step()
+    torch.cuda.synchronize()
+    replicas.barrier(rk)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(s_in)
+    for _ in range(K):
         step()
-        torch.cuda.synchronize()
-        replicas.barrier(rk)
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        for _ in range(K):
-            step()
-        e1.record(stream)
-        torch.cuda.synchronize()
+    e1.record(s_out)
+    torch.cuda.synchronize()
     ms = replicas.max_over_ranks(rk, e0.elapsed_time(e1) / K, dev)
+    # the chunked results must be the whole-batch results, bit for bit
+    same = all(torch.equal(host_out[n].view(-1), ref_out[n].reshape(-1).cpu()) for n in names_out)
     return {"value": replicas.job_rate(w.B * w.N, rk.world, ms / 1e3), "unit": "tokens/s",
-            "ms_per_step": ms,
-            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+            "ms_per_step": ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+            "chunks": C, "matches_device_run": same}
 
 
 # ------------------------------------------------------------- CPU oracle
