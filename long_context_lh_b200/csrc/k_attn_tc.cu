@@ -57,68 +57,55 @@ __device__ __forceinline__ void store_row_half(uint8_t* tile_half, int r, const 
 }
 
 // ================================================================= forward
-// Column groups: every 128-key tile is split into NG groups of CW = 128/NG
-// keys; the 4 warps of group g (one per TMEM lane quarter) own the keys of
-// group g in every tile, with their own running reference max, sum and TMEM
-// accumulator O_g (D columns).  NG = 2: eight row-work warps, two per SM
-// sub-partition (four groups, 16 warps, measured slower at d = 64: the
-// per-thread register cap of 18 warps and four P handoffs per tile).
-template <int D>
-struct FwdCfg {
-  static constexpr int NG = 2;
-  static constexpr int CW = 128 / NG;        // keys per group and tile
-  static constexpr int kRowWarps = 4 * NG;
-  static constexpr int kTmaWarp = kRowWarps, kMmaWarp = kRowWarps + 1;
-  static constexpr int kThreads = 32 * (kRowWarps + 2);
-  static constexpr int OC = D / NG;          // output columns per thread
-  static_assert(256 + NG * D <= (int)kTmemCols, "TMEM: two S buffers and NG accumulators");
-  static_assert(CW % 64 == 0, "P of a group is stored as whole 32-column TMEM stores");
-};
-
-template <int NG>
-struct FwdBars {
-  uint64_t q_full;
-  uint64_t kv_full[4], kv_empty[4];
-  uint64_t s_full[2], s_free[2];
-  uint64_t p_full[NG], pv_done[NG], mma_done;  // [column group]
-  uint32_t tmem;
-  int abort;
-  float xm[NG][128], xl[NG][128];  // [group][row] final reference max and sum
-};
-
+// Ping-pong: one CTA per (unit, pair of query tiles) -- tiles A = 2i+1 and
+// B = 2i (A alone when it is the last, odd one).  Both walk the same key tiles
+// (B one fewer), so each K/V tile is loaded once for both.  Row-work warps 0-3
+// own tile A, warps 4-7 tile B, one thread per row and all 128 keys of a tile:
+// every SM sub-partition holds one warp of each tile, and the two alternate
+// (while one computes its exponentials, the tensor core serves the other).
+// TMEM: S_A, S_B (128 columns each; P is written as packed fp16 over the S
+// columns already consumed), O_A, O_B (D columns each).  The MMA warp issues
+// S_T(j+1) right after O_T += P_T(j) V(j), so tile T's next scores are ready
+// while the other tile computes.
 template <int D>
 struct FwdLayout {
   static constexpr int kKS = (D == 64) ? 4 : 2;  // K/V stages
   static constexpr int kTile = 128 * D * 2;
-  static constexpr int kQ = 0;
-  static constexpr int kK = kQ + kTile;
+  static constexpr int kQ = 0;                   // Q_A, Q_B
+  static constexpr int kK = kQ + 2 * kTile;
   static constexpr int kV = kK + kKS * kTile;
-  static constexpr int kBar = kV + kKS * kTile;  // (P lives in TMEM, over S)
-  static constexpr int kBytes = kBar + (int)sizeof(FwdBars<FwdCfg<D>::NG>);
+  static constexpr int kBar = kV + kKS * kTile;
 };
 
-template <int NT>
-__device__ __forceinline__ void named_bar() {  // the NT row-work threads only
-  asm volatile("bar.sync 1, %0;\n" ::"n"(NT) : "memory");
+struct FwdBars {
+  uint64_t q_full;
+  uint64_t kv_full[4], kv_empty[4];
+  uint64_t s_full[2], p_full[2], pv_done[2], mma_done;  // [tile A, B]
+  uint32_t tmem;
+  int abort;
+};
+
+template <int D>
+constexpr int fwd_smem_bytes() {
+  return FwdLayout<D>::kBar + (int)sizeof(FwdBars);
 }
 
 template <int D>
-__global__ void __launch_bounds__(FwdCfg<D>::kThreads, 1)
+__global__ void __launch_bounds__(kThreads, 1)
     k_attn_fwd_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
                   const __grid_constant__ CUtensorMap tv, __half* __restrict__ os,
                   float* __restrict__ lse, int S, int unit0, int nunits, float scale_log2,
                   int ntiles) {
   using Lt = FwdLayout<D>;
-  using Cf = FwdCfg<D>;
-  constexpr int NG = Cf::NG, CW = Cf::CW;
   constexpr int KS = Lt::kKS;
-  static_assert(KS >= 2 && KS <= 4, "FwdBars holds at most 4 stages; the protocol needs 2");
+  static_assert(KS >= 1 && KS <= 4, "FwdBars holds at most 4 stages");
+  static_assert(256 + 2 * D <= (int)kTmemCols, "TMEM: S_A, S_B, O_A, O_B");
   extern __shared__ __align__(1024) uint8_t smem[];
   if (smem_u32(smem) & 1023u) {
     if (threadIdx.x == 0) report_status(kStatusAttnFwdTimeout | 1u);
     return;
   }
-  auto* bars = reinterpret_cast<FwdBars<NG>*>(smem + Lt::kBar);
+  FwdBars* bars = reinterpret_cast<FwdBars*>(smem + Lt::kBar);
   uint8_t* sQ = smem + Lt::kQ;
   uint8_t* sK = smem + Lt::kK;
   uint8_t* sV = smem + Lt::kV;
@@ -126,10 +113,14 @@ __global__ void __launch_bounds__(FwdCfg<D>::kThreads, 1)
   constexpr uint32_t kStatus = kStatusAttnFwdTimeout;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  // 1-D grid ordered by work: all units' last (longest) query tiles first
-  const int qt = ntiles - 1 - (int)(blockIdx.x / nunits);
+  // 1-D grid ordered by work: all units' last (longest) pairs first
+  const int npairs = (ntiles + 1) / 2;
+  const int pi = npairs - 1 - (int)(blockIdx.x / nunits);
   const int u = unit0 + (int)(blockIdx.x % nunits);
-  const int n = qt + 1;
+  const bool hasB = 2 * pi + 1 < ntiles;
+  const int qtA = hasB ? 2 * pi + 1 : 2 * pi;  // the longer tile
+  const int qtB = hasB ? 2 * pi : -1;
+  const int nA = qtA + 1, nB = qtB + 1;         // key tiles of each (nB = 0: no tile B)
 
   if (threadIdx.x == 0) {
     mbar_init(&bars->q_full, 1);
@@ -137,35 +128,32 @@ __global__ void __launch_bounds__(FwdCfg<D>::kThreads, 1)
       mbar_init(&bars->kv_full[i], 1);
       mbar_init(&bars->kv_empty[i], 1);
     }
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(&bars->s_full[b], 1);
-      mbar_init(&bars->s_free[b], Cf::kRowWarps);
-    }
-    for (int g = 0; g < NG; ++g) {
-      mbar_init(&bars->p_full[g], 4);
-      mbar_init(&bars->pv_done[g], 1);
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(&bars->s_full[t], 1);
+      mbar_init(&bars->p_full[t], 4);
+      mbar_init(&bars->pv_done[t], 1);
     }
     mbar_init(&bars->mma_done, 1);
     bars->abort = 0;
     mbar_init_fence();
   }
-  if (warp == Cf::kMmaWarp) tmem_alloc(&bars->tmem, kTmemCols);
+  if (warp == 9) tmem_alloc(&bars->tmem, kTmemCols);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = bars->tmem;
-  // S double buffer at tmem + 0 / + 128 (P_g of a tile is written over the first
-  // CW/2 of its group's S columns); O_g at tmem + 256 + g * D
-  const uint32_t tO = tmem + 256;
+  const uint32_t tO = tmem + 256;  // O_A at +256, O_B at +256+D; S_T at +128*T
 
-  if (warp == Cf::kTmaWarp) {
+  if (warp == 8) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
-      mbar_expect_tx(&bars->q_full, Lt::kTile);
-      for (int h = 0; h < D / 64; ++h)
-        tma_load_3d(sQ + h * 16384, &tq, &bars->q_full, h * 64, qt * 128, u);
+      mbar_expect_tx(&bars->q_full, (hasB ? 2 : 1) * Lt::kTile);
+      for (int h = 0; h < D / 64; ++h) {
+        tma_load_3d(sQ + h * 16384, &tq, &bars->q_full, h * 64, qtA * 128, u);
+        if (hasB) tma_load_3d(sQ + Lt::kTile + h * 16384, &tq, &bars->q_full, h * 64, qtB * 128, u);
+      }
       int issued = 0;
-      for (int j = 0; j < n; ++j) {
+      for (int j = 0; j < nA; ++j) {
         const int st = j % KS;
         if (j >= KS && !mbar_wait(&bars->kv_empty[st], ((j - KS) / KS) & 1, abort, kStatus)) break;
         mbar_expect_tx(&bars->kv_full[st], 2 * Lt::kTile);
@@ -179,133 +167,109 @@ __global__ void __launch_bounds__(FwdCfg<D>::kThreads, 1)
       for (int j = (issued > KS ? issued - KS : 0); j < issued; ++j)
         mbar_wait(&bars->kv_full[j % KS], (j / KS) & 1, abort, kStatus, false);
     }
-  } else if (warp == Cf::kMmaWarp) {
+  } else if (warp == 9) {
     // -------------------------------------------------------------- MMA issuer
     if (lane == 0) {
       constexpr uint32_t idS = idesc_f16(128, 128, false);
       constexpr uint32_t idPV = idesc_f16(128, D, true);
       const uint32_t aQ = smem_u32(sQ), aK = smem_u32(sK), aV = smem_u32(sV);
-      // O_g += P[:, keys of group g] V[keys of group g, :], once group g has
-      // written its P (TMEM, over S of tile i) -- issued before S of tile i + 2
-      // overwrites that buffer
-      auto issue_pv = [&](int i) {
-        const int st = i % KS;
-        const uint32_t tP = tmem + (i & 1) * 128;
-        for (int g = 0; g < NG; ++g) {
-          if (!mbar_wait(&bars->p_full[g], i & 1, abort, kStatus)) return false;
-          tc_fence_after();
-#pragma unroll
-          for (int k = 0; k < CW / 16; ++k) {
-            const int kk = g * (CW / 16) + k;  // 16-key step within the tile
-            umma_f16_ta(tO + g * D, tP + g * CW + 8 * k,
-                        desc_mnmajor(aV + st * Lt::kTile + kk * 2048, 16384), idPV, (i > 0 || k > 0));
-          }
-          umma_commit(&bars->pv_done[g]);
-        }
-        umma_commit(&bars->kv_empty[st]);
-        return true;
-      };
-      bool ok = mbar_wait(&bars->q_full, 0, abort, kStatus);
-      for (int j = 0; ok && j < n; ++j) {
-        const int st = j % KS, b = j & 1;
-        ok = mbar_wait(&bars->kv_full[st], (j / KS) & 1, abort, kStatus) &&
-             (j < 2 || mbar_wait(&bars->s_free[b], ((j - 2) >> 1) & 1, abort, kStatus));
-        if (!ok) break;
-        tc_fence_after();
+      auto issue_s = [&](int t, int j) {  // S_t = Q_t K_j^T
+        const int st = j % KS;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-          umma_f16(tmem + b * 128, desc_kmajor(aQ + off), desc_kmajor(aK + st * Lt::kTile + off),
-                   idS, kk > 0);
+          umma_f16(tmem + t * 128, desc_kmajor(aQ + t * Lt::kTile + off),
+                   desc_kmajor(aK + st * Lt::kTile + off), idS, kk > 0);
         }
-        umma_commit(&bars->s_full[b]);
-        if (j >= 1 && !(ok = issue_pv(j - 1))) break;
+        umma_commit(&bars->s_full[t]);
+      };
+      auto issue_pv = [&](int t, int j) {  // O_t += P_t(j) V_j, P_t from TMEM
+        const int st = j % KS;
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          umma_f16_ta(tO + t * D, tmem + t * 128 + 8 * kk,
+                      desc_mnmajor(aV + st * Lt::kTile + kk * 2048, 16384), idPV, (j > 0 || kk > 0));
+        umma_commit(&bars->pv_done[t]);
+      };
+      bool ok = mbar_wait(&bars->q_full, 0, abort, kStatus) &&
+                mbar_wait(&bars->kv_full[0], 0, abort, kStatus);
+      if (ok) {
+        tc_fence_after();
+        issue_s(0, 0);
+        if (nB > 0) issue_s(1, 0);
       }
-      if (ok) issue_pv(n - 1);
+      for (int j = 0; ok && j < nA; ++j) {
+        const int st = j % KS;
+        const bool next = j + 1 < nA;
+        // tile A: its product with V_j, then (S_A buffer free again) its next scores
+        if (!(ok = mbar_wait(&bars->p_full[0], j & 1, abort, kStatus))) break;
+        tc_fence_after();
+        issue_pv(0, j);
+        if (next) {
+          if (!(ok = mbar_wait(&bars->kv_full[(j + 1) % KS], ((j + 1) / KS) & 1, abort, kStatus))) break;
+          tc_fence_after();
+          issue_s(0, j + 1);
+        }
+        // tile B likewise
+        if (j < nB) {
+          if (!(ok = mbar_wait(&bars->p_full[1], j & 1, abort, kStatus))) break;
+          tc_fence_after();
+          issue_pv(1, j);
+          if (j + 1 < nB) issue_s(1, j + 1);
+        }
+        umma_commit(&bars->kv_empty[st]);  // K_j, V_j no longer needed
+      }
       umma_commit(&bars->mma_done);
       mbar_wait(&bars->mma_done, 0, abort, kStatus, false);
     }
   } else {
-    // ------------------------------------ row work: NG threads per row (one per group)
-    // Thread (row r, group g) owns the CW keys of group g in every tile and the
-    // partial softmax over them: its own running reference max m_ref, sum l and
-    // accumulator O_g in TMEM.  Nothing is exchanged until the end, where the NG
-    // partials of a row are merged (the usual split-softmax merge).  P is formed
-    // against m_ref, and O_g is rescaled in TMEM only when a tile's max exceeds
-    // m_ref by more than kRescale (exp2 domain), so P <= 2^kRescale fits fp16;
-    // softmax is invariant to the reference, so the result is the same.
+    // -------------------- row work: one thread per row of its tile, all 128 keys
+    // P is formed against a running reference max m_ref, and O_t is rescaled in
+    // TMEM only when a tile's max exceeds m_ref by more than kRescale (exp2
+    // domain), so P <= 2^kRescale fits fp16; softmax is invariant to the
+    // reference, so the result is the same.
     constexpr float kRescale = 8.0f;
-    const int qd = warp & 3, g = warp >> 2;
+    const int t = warp >> 2;  // 0: tile A, 1: tile B
+    const int qd = warp & 3;
     const int r = qd * 32 + lane;
+    const int n = t == 0 ? nA : nB;
+    const int qt = t == 0 ? qtA : qtB;
     const uint32_t lane_addr = (uint32_t)(qd * 32) << 16;
-    const uint32_t tOg = tO + g * D + lane_addr;
+    const uint32_t tS = tmem + t * 128 + lane_addr;
+    const uint32_t tOt = tO + t * D + lane_addr;
     float m_ref = -INFINITY, l = 0.0f;
     bool ok = true;
     // one key tile; kDiag: the last (diagonal) tile, keys past the row masked
     auto step = [&](int j, auto diag_tag) {
       constexpr bool kDiag = decltype(diag_tag)::value;
-      const int b = j & 1;
-      ok = warp_wait(&bars->s_full[b], (j >> 1) & 1, abort, kStatus);
+      ok = warp_wait(&bars->s_full[t], j & 1, abort, kStatus);
       if (!ok) return;
       tc_fence_after();
-      uint32_t v[CW];
-#pragma unroll
-      for (int c = 0; c < CW / 32; ++c)
-        tmem_ld32(tmem + b * 128 + lane_addr + g * CW + 32 * c,
-                  reinterpret_cast<uint32_t(&)[32]>(v[32 * c]));
-      tmem_ld_wait();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bars->s_free[b]);  // S is in registers now
-      const int lim = r - g * CW;                     // keys i <= lim are visible
-      // row max: four independent chains (max is exact in any order)
+      // pass 1: the row max, 32 columns at a time (four independent chains)
       float mc[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-      for (int i = 0; i < CW; i += 2) {
-        const int c = (i >> 1) & 3;
-        if (kDiag) {
-          mc[c] = max3(mc[c], i <= lim ? __uint_as_float(v[i]) : -INFINITY,
-                       i + 1 <= lim ? __uint_as_float(v[i + 1]) : -INFINITY);
-        } else {
-          mc[c] = max3(mc[c], __uint_as_float(v[i]), __uint_as_float(v[i + 1]));
+      for (int c = 0; c < 4; ++c) {
+        uint32_t v[32];
+        tmem_ld32(tS + 32 * c, v);
+        tmem_ld_wait();
+#pragma unroll
+        for (int i = 0; i < 32; i += 2) {
+          const int k = (i >> 1) & 3;
+          if (kDiag) {
+            mc[k] = max3(mc[k], 32 * c + i <= r ? __uint_as_float(v[i]) : -INFINITY,
+                         32 * c + i + 1 <= r ? __uint_as_float(v[i + 1]) : -INFINITY);
+          } else {
+            mc[k] = max3(mc[k], __uint_as_float(v[i]), __uint_as_float(v[i + 1]));
+          }
         }
       }
-      float mx = fmaxf(max3(mc[0], mc[1], mc[2]), mc[3]);
-      mx *= scale_log2;
+      const float mx = fmaxf(max3(mc[0], mc[1], mc[2]), mc[3]) * scale_log2;  // finite: key 0
       const bool grow = mx > m_ref + kRescale;
       const float m_new = grow ? mx : m_ref;
-      // P first (against the new reference), so S is dead before O is touched;
-      // a fully masked group (only in the diagonal tile) has m_new = -inf: its
-      // exponent is NaN but every one of its elements is replaced by 0 below
-      uint32_t pk[CW / 2];
-      const float2 cc = make_float2(scale_log2, scale_log2), nm = make_float2(-m_new, -m_new);
-      // row sum: four independent paired accumulators
-      float2 sacc[4] = {make_float2(0.0f, 0.0f), make_float2(0.0f, 0.0f), make_float2(0.0f, 0.0f),
-                        make_float2(0.0f, 0.0f)};
-#pragma unroll
-      for (int i = 0; i < CW; i += 4) {
-        const float2 x = ffma2(make_float2(__uint_as_float(v[i]), __uint_as_float(v[i + 1])), cc, nm);
-        const float2 y = ffma2(make_float2(__uint_as_float(v[i + 2]), __uint_as_float(v[i + 3])), cc, nm);
-        float2 p = make_float2(ex2(x.x), ex2(x.y));
-        // a quarter of the exponentials on the FMA pipe, the rest on MUFU
-        float2 q = (i & 7) == 4 ? ex2_fma2(y) : make_float2(ex2(y.x), ex2(y.y));
-        if (kDiag) {
-          p.x = i <= lim ? p.x : 0.0f;
-          p.y = i + 1 <= lim ? p.y : 0.0f;
-          q.x = i + 2 <= lim ? q.x : 0.0f;
-          q.y = i + 3 <= lim ? q.y : 0.0f;
-        }
-        const int c = (i >> 2) & 1;
-        sacc[2 * c] = fadd2(sacc[2 * c], p);
-        sacc[2 * c + 1] = fadd2(sacc[2 * c + 1], q);
-        pk[i >> 1] = h2(p.x, p.y);
-        pk[(i >> 1) + 1] = h2(q.x, q.y);
-      }
-      // every phase of pv_done[g] is waited for, in order (a parity wait must
-      // never run two phases ahead of the barrier); the previous tile's product
-      // is normally complete by now.  O_g must be complete before a rescale.
+      // every phase of pv_done[t] is waited for, in order; O_t (and the P of the
+      // previous tile) must be done with before O_t is rescaled or P rewritten
       if (j > 0) {
-        ok = warp_wait(&bars->pv_done[g], (j - 1) & 1, abort, kStatus);
+        ok = warp_wait(&bars->pv_done[t], (j - 1) & 1, abort, kStatus);
         if (!ok) return;
       }
       if (j > 0 && __any_sync(0xffffffffu, grow)) {
@@ -314,81 +278,88 @@ __global__ void __launch_bounds__(FwdCfg<D>::kThreads, 1)
 #pragma unroll
         for (int c = 0; c < D / 32; ++c) {
           uint32_t ov[32];
-          tmem_ld32(tOg + c * 32, ov);
+          tmem_ld32(tOt + c * 32, ov);
           tmem_ld_wait();
 #pragma unroll
           for (int i = 0; i < 32; ++i) ov[i] = __float_as_uint(__uint_as_float(ov[i]) * alpha);
-          tmem_st32(tOg + c * 32, ov);
+          tmem_st32(tOt + c * 32, ov);
         }
         l *= alpha;
       }
       m_ref = m_new;
-      // P (CW keys = CW/2 packed columns) over this group's S columns of buffer b
+      // pass 2: P = 2^(S c - m_ref), 32 columns at a time, packed fp16 written
+      // over S columns already read (chunk c writes columns 16c..16c+15)
+      const float2 cc = make_float2(scale_log2, scale_log2), nm = make_float2(-m_ref, -m_ref);
+      float2 sacc[4] = {make_float2(0.0f, 0.0f), make_float2(0.0f, 0.0f), make_float2(0.0f, 0.0f),
+                        make_float2(0.0f, 0.0f)};
 #pragma unroll
-      for (int c = 0; c < CW / 64; ++c)
-        tmem_st32(tmem + b * 128 + lane_addr + g * CW + 32 * c,
-                  reinterpret_cast<const uint32_t(&)[32]>(pk[32 * c]));
+      for (int c = 0; c < 4; ++c) {
+        uint32_t v[32];
+        tmem_ld32(tS + 32 * c, v);
+        tmem_ld_wait();
+        uint32_t pk[16];
+#pragma unroll
+        for (int i = 0; i < 32; i += 4) {
+          const float2 x = ffma2(make_float2(__uint_as_float(v[i]), __uint_as_float(v[i + 1])), cc, nm);
+          const float2 y = ffma2(make_float2(__uint_as_float(v[i + 2]), __uint_as_float(v[i + 3])), cc, nm);
+          float2 p = make_float2(ex2(x.x), ex2(x.y));
+          // a quarter of the exponentials on the FMA pipe, the rest on MUFU
+          float2 q = (i & 7) == 4 ? ex2_fma2(y) : make_float2(ex2(y.x), ex2(y.y));
+          if (kDiag) {
+            const int k0 = 32 * c + i;
+            p.x = k0 <= r ? p.x : 0.0f;
+            p.y = k0 + 1 <= r ? p.y : 0.0f;
+            q.x = k0 + 2 <= r ? q.x : 0.0f;
+            q.y = k0 + 3 <= r ? q.y : 0.0f;
+          }
+          const int k = (i >> 2) & 1;
+          sacc[2 * k] = fadd2(sacc[2 * k], p);
+          sacc[2 * k + 1] = fadd2(sacc[2 * k + 1], q);
+          pk[i >> 1] = h2(p.x, p.y);
+          pk[(i >> 1) + 1] = h2(q.x, q.y);
+        }
+        tmem_st16(tS + 16 * c, pk);
+      }
       tmem_st_wait();
-      tc_fence_before();  // orders P and the O_g rescale (TMEM stores) before the product
+      tc_fence_before();  // orders P and the O_t rescale (TMEM stores) before the product
       __syncwarp();
-      if (lane == 0) mbar_arrive(&bars->p_full[g]);
+      if (lane == 0) mbar_arrive(&bars->p_full[t]);
       const float2 s01 = fadd2(sacc[0], sacc[1]), s23 = fadd2(sacc[2], sacc[3]);
       l += (s01.x + s01.y) + (s23.x + s23.y);
     };
-    for (int j = 0; j < n - 1 && ok; ++j) step(j, std::false_type{});
-    if (ok) step(n - 1, std::true_type{});
-    if (ok) ok = warp_wait(&bars->pv_done[g], (n - 1) & 1, abort, kStatus);
-    // merge the NG partials of each row:
-    //   O = sum_q 2^(m_q - m) O_q / sum_q 2^(m_q - m) l_q,  m = max_q m_q
-    bars->xm[g][r] = m_ref;
-    bars->xl[g][r] = l;
-    named_bar<32 * Cf::kRowWarps>();
-    float m = bars->xm[0][r];  // finite: key 0 of group 0 is visible to every row
+    if (n > 0) {
+      for (int j = 0; j < n - 1 && ok; ++j) step(j, std::false_type{});
+      if (ok) step(n - 1, std::true_type{});
+      if (ok) ok = warp_wait(&bars->pv_done[t], (n - 1) & 1, abort, kStatus);
+      const int row = qt * 128 + r;
+      if (ok) {  // whole warps load TMEM; only rows inside the sequence are stored
+        tc_fence_after();
+        const float inv = 1.0f / l;
+        __half* dst = os + ((int64_t)u * S + row) * D;
 #pragma unroll
-    for (int q = 1; q < NG; ++q) m = fmaxf(m, bars->xm[q][r]);
-    float wq[NG];
-    float lt = 0.0f;
-#pragma unroll
-    for (int q = 0; q < NG; ++q) {
-      wq[q] = ex2(bars->xm[q][r] - m);
-      lt = __fmaf_rn(wq[q], bars->xl[q][r], lt);
-    }
-    const int row = qt * 128 + r;
-    if (ok) {  // whole warps load TMEM; only rows inside the sequence are stored
-      tc_fence_after();
-      constexpr int OC = Cf::OC;  // output columns of this thread: [g*OC, (g+1)*OC)
-      const float inv = 1.0f / lt;
-#pragma unroll
-      for (int q = 0; q < NG; ++q) wq[q] *= inv;
-      __half* dst = os + ((int64_t)u * S + row) * D + g * OC;
-#pragma unroll
-      for (int c = 0; c < OC / 16; ++c) {
-        float f[16];
-#pragma unroll
-        for (int q = 0; q < NG; ++q) {
-          uint32_t ov[16];
-          tmem_ld16(tO + q * D + lane_addr + g * OC + 16 * c, ov);
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t ov[32];
+          tmem_ld32(tOt + c * 32, ov);
           tmem_ld_wait();
+          if (row < S) {
 #pragma unroll
-          for (int i = 0; i < 16; ++i)
-            f[i] = q == 0 ? __uint_as_float(ov[i]) * wq[0] : __fmaf_rn(__uint_as_float(ov[i]), wq[q], f[i]);
+            for (int x = 0; x < 4; ++x) {
+              uint4 w;
+              w.x = h2_sat(__uint_as_float(ov[8 * x + 0]) * inv, __uint_as_float(ov[8 * x + 1]) * inv);
+              w.y = h2_sat(__uint_as_float(ov[8 * x + 2]) * inv, __uint_as_float(ov[8 * x + 3]) * inv);
+              w.z = h2_sat(__uint_as_float(ov[8 * x + 4]) * inv, __uint_as_float(ov[8 * x + 5]) * inv);
+              w.w = h2_sat(__uint_as_float(ov[8 * x + 6]) * inv, __uint_as_float(ov[8 * x + 7]) * inv);
+              *reinterpret_cast<uint4*>(dst + c * 32 + 8 * x) = w;
+            }
+          }
         }
-        if (row < S) {
-          uint4 w0, w1;
-          w0.x = h2_sat(f[0], f[1]);   w0.y = h2_sat(f[2], f[3]);
-          w0.z = h2_sat(f[4], f[5]);   w0.w = h2_sat(f[6], f[7]);
-          w1.x = h2_sat(f[8], f[9]);   w1.y = h2_sat(f[10], f[11]);
-          w1.z = h2_sat(f[12], f[13]); w1.w = h2_sat(f[14], f[15]);
-          *reinterpret_cast<uint4*>(dst + 16 * c) = w0;
-          *reinterpret_cast<uint4*>(dst + 16 * c + 8) = w1;
-        }
+        if (row < S) lse[(int64_t)u * S + row] = (m_ref + __log2f(l)) * kLn2;
       }
-      if (g == 0 && row < S) lse[(int64_t)u * S + row] = (m + __log2f(lt)) * kLn2;
     }
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == Cf::kMmaWarp) {
+  if (warp == 9) {
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);
   }
@@ -934,15 +905,16 @@ cudaError_t fwd_d(const Geom& g, const __half* qs, const __half* ks, const __hal
   if (!make_map(&mq, qs, D, g.S, g.U) || !make_map(&mk, ks, D, g.S, g.U) ||
       !make_map(&mv, vs, D, g.S, g.U))
     return cudaErrorNotSupported;
-  constexpr int smem = FwdLayout<D>::kBytes;
+  constexpr int smem = fwd_smem_bytes<D>();
   cudaError_t e =
       cudaFuncSetAttribute(k_attn_fwd_tc<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   const int ntiles = (int)((g.S + 127) / 128);
-  const int64_t per = 0x7fffffff / ntiles;  // units per launch (grid.x limit)
+  const int npairs = (ntiles + 1) / 2;
+  const int64_t per = 0x7fffffff / npairs;  // units per launch (grid.x limit)
   for (int64_t u0 = 0; u0 < g.U; u0 += per) {
     const int64_t nu = g.U - u0 < per ? g.U - u0 : per;
-    k_attn_fwd_tc<D><<<(unsigned)(nu * ntiles), FwdCfg<D>::kThreads, smem, st>>>(
+    k_attn_fwd_tc<D><<<(unsigned)(nu * npairs), kThreads, smem, st>>>(
         mq, mk, mv, os, lse, (int)g.S, (int)u0, (int)nu, scale * kLog2e, ntiles);
   }
   return cudaGetLastError();
@@ -988,10 +960,13 @@ bool attn_tc_available() {
 }
 bool attn_tc_bwd_available() { return attn_tc_available(); }
 int attn_tc_fwd_launches(const Geom& g) {
-  const int64_t ntiles = (g.S + 127) / 128, per = 0x7fffffff / ntiles;
+  const int64_t npairs = ((g.S + 127) / 128 + 1) / 2, per = 0x7fffffff / npairs;
   return (int)((g.U + per - 1) / per);
 }
-int attn_tc_bwd_launches(const Geom& g) { return 2 * attn_tc_fwd_launches(g); }
+int attn_tc_bwd_launches(const Geom& g) {
+  const int64_t ntiles = (g.S + 127) / 128, per = 0x7fffffff / ntiles;
+  return 2 * (int)((g.U + per - 1) / per);
+}
 
 cudaError_t launch_attn_fwd_tc(const Geom& g, const __half* qs, const __half* ks,
                                const __half* vs, float scale, __half* os, float* lse,
