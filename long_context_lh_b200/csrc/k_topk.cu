@@ -61,7 +61,11 @@ __device__ __forceinline__ int32_t gid_at(const TopkParams& prm, uint32_t t1, in
   return prm.off[l] + (int32_t)j1 - 1;
 }
 
-// Histogram increment with warp aggregation: lanes with the same bin add once.
+// Histogram increment.  Warp-aggregated (lanes with the same bin add once) when
+// the keys crowd a few bins (the first digit); plain otherwise.
+__device__ __forceinline__ void hist_add_plain(uint32_t* hist, bool active, uint32_t bin) {
+  if (active) atomicAdd(&hist[bin], 1u);
+}
 __device__ __forceinline__ void hist_add(uint32_t* hist, bool active, uint32_t bin) {
   const unsigned act = __ballot_sync(0xffffffffu, active);
   if (!active) return;
@@ -111,22 +115,30 @@ __device__ Pick pick_digit(cg::cluster_group& cluster, uint32_t* hist, int nbins
                            uint32_t need, uint32_t* warp_buf, uint32_t* sh) {
   const int per = nbins / kThreads;  // 2 or 1 ordinals per thread
   uint32_t tot[2] = {0, 0};
-  uint32_t local = 0;
-  for (int i = 0; i < per; ++i) {
-    const int ord = threadIdx.x * per + i;
-    const int bin = descending ? (nbins - 1 - ord) : ord;
-    uint32_t s = 0;
+  if (per == 2) {
+    // the thread's two ordinals are adjacent bins: one 8-byte load per rank,
+    // every rank's load in flight at once
+    const int lo = descending ? nbins - 2 - 2 * (int)threadIdx.x : 2 * (int)threadIdx.x;
+    uint2 v[CL];
 #pragma unroll
-    for (int r0 = 0; r0 < CL; r0 += 8) {  // eight remote loads in flight at a time
-      uint32_t v[8];
+    for (int r = 0; r < CL; ++r) v[r] = *reinterpret_cast<const uint2*>(cluster.map_shared_rank(hist, r) + lo);
+    uint32_t a = 0, b = 0;
 #pragma unroll
-      for (int r = 0; r < 8; ++r) v[r] = cluster.map_shared_rank(hist, r0 + r)[bin];
-#pragma unroll
-      for (int r = 0; r < 8; ++r) s += v[r];
+    for (int r = 0; r < CL; ++r) {
+      a += v[r].x;
+      b += v[r].y;
     }
-    tot[i] = s;
-    local += s;
+    tot[0] = descending ? b : a;  // ordinal 2t first
+    tot[1] = descending ? a : b;
+  } else {
+    const int bin = descending ? (nbins - 1 - (int)threadIdx.x) : (int)threadIdx.x;
+    uint32_t v[CL];
+#pragma unroll
+    for (int r = 0; r < CL; ++r) v[r] = cluster.map_shared_rank(hist, r)[bin];
+#pragma unroll
+    for (int r = 0; r < CL; ++r) tot[0] += v[r];
   }
+  const uint32_t local = tot[0] + tot[1];
   uint32_t all;
   uint32_t before = block_excl_scan(local, warp_buf, &all);
   for (int i = 0; i < per; ++i) {
@@ -210,7 +222,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int32_t j0 = warp * 32; j0 < nl[l]; j0 += kThreads) {  // warp-uniform trip count
         const int32_t j = j0 + lane;
         const uint32_t kv = j < nl[l] ? key_of(l, j) : 0u;
-        hist_add(hist[buf], j < nl[l] && (kv & pmask) == prefix, (kv >> shift) & dmask);
+        const bool act = j < nl[l] && (kv & pmask) == prefix;
+        if (pass == 0)
+          hist_add(hist[buf], act, (kv >> shift) & dmask);
+        else
+          hist_add_plain(hist[buf], act, (kv >> shift) & dmask);
       }
     }
     cluster.sync();
@@ -242,7 +258,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int32_t j = j0 + lane;
           const uint32_t gid = (uint32_t)(prm.off[l] + jb[l] + j);
           const bool in = j < nl[l] && key_of(l, j < nl[l] ? j : 0) == T && (gid & gmask) == gprefix;
-          hist_add(hist[buf], in, (gid >> shift) & dmask);
+          hist_add_plain(hist[buf], in, (gid >> shift) & dmask);
         }
       }
       cluster.sync();
