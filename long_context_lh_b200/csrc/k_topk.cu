@@ -164,7 +164,7 @@ __device__ Pick pick_digit(cg::cluster_group& cluster, uint32_t* hist, int nbins
 template <int CL>
 __global__ void __launch_bounds__(kThreads, 1)
     k_topk(const float* __restrict__ score, int32_t* __restrict__ idx, int32_t* __restrict__ pos,
-           int32_t* __restrict__ slot, const TopkParams prm, int cached) {
+           int32_t* __restrict__ slot, const TopkParams prm, int cached, int kcap, int masks) {
   cg::cluster_group cluster = cg::this_cluster();
   const int rank = (int)cluster.block_rank();
   const int64_t u = prm.unit0 + blockIdx.y;
@@ -174,7 +174,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   __shared__ uint32_t sh[4];
   __shared__ uint32_t warp_tot[kWarps];
   __shared__ uint32_t cta_total;
-  extern __shared__ uint32_t skey[];  // the CTA's keys, level by level (cached)
+  extern __shared__ uint32_t skey[];  // the CTA's keys, level by level (cached), kcap words
+  // then per token of the CTA: bits 0-7 the selected levels ending at it,
+  // bits 8-15 all levels ending at it (written by the counting pass)
+  uint16_t* smask = reinterpret_cast<uint16_t*>(skey + kcap);
 
   const uint32_t* key = reinterpret_cast<const uint32_t*>(score + u * prm.M);
   const int32_t Ptop = prm.pw[prm.L - 1];
@@ -285,18 +288,22 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t kv = key_of(l, g - prm.off[l] - jb[l]);
     return kv > T || (kv == T && (int64_t)g <= gid_thr);
   };
-  // pass A: count per warp
+  // pass A: per token, which levels end at it and which of those are selected
+  // (kept for pass B); counts per warp
   uint32_t wcount = 0;
   for (int32_t tb = w_begin; tb < w_end; tb += 32) {
     const int32_t t = tb + lane;
     uint32_t c = 0;
     if (t < w_end) {
       const uint32_t t1 = (uint32_t)t + 1u;
+      uint32_t mask = 0;
 #pragma unroll
       for (int l = 0; l < kMaxLevels; ++l) {  // unrolled: jb[l], kb[l] stay in registers
         if (l >= prm.L || !ends_at(prm, t1, l)) break;  // spans end at t up to some level
-        c += selected(l, t1) ? 1u : 0u;
+        mask |= (selected(l, t1) ? 1u : 0u) << l | 1u << (8 + l);
       }
+      if (masks) smask[t - t_b] = (uint16_t)mask;
+      c = __popc(mask & 0xffu);
     }
     wcount += __reduce_add_sync(0xffffffffu, c);
   }
@@ -312,41 +319,40 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint32_t base = 0;
   for (int r = 0; r < rank; ++r) base += *cluster.map_shared_rank(&cta_total, r);
   base += warp_tot[warp];
-  // pass B: write
+  // pass B: write idx, pos and the slot map from the masks
   int32_t* idx_u = idx + u * prm.S;
   int32_t* pos_u = pos + u * prm.S;
   int32_t* slot_u = slot + u * prm.M;
   for (int32_t tb = w_begin; tb < w_end; tb += 32) {
     const int32_t t = tb + lane;
-    uint32_t c = 0;
-    uint32_t selmask = 0;
+    uint32_t mask = 0;
     if (t < w_end) {
-      const uint32_t t1 = (uint32_t)t + 1u;
+      if (masks) {
+        mask = smask[t - t_b];
+      } else {  // masks did not fit in shared memory: recompute them
+        const uint32_t t1 = (uint32_t)t + 1u;
 #pragma unroll
-      for (int l = 0; l < kMaxLevels; ++l) {
-        if (l >= prm.L || !ends_at(prm, t1, l)) break;
-        if (selected(l, t1)) {
-          selmask |= 1u << l;
-          ++c;
+        for (int l = 0; l < kMaxLevels; ++l) {
+          if (l >= prm.L || !ends_at(prm, t1, l)) break;
+          mask |= (selected(l, t1) ? 1u : 0u) << l | 1u << (8 + l);
         }
       }
     }
+    const uint32_t c = __popc(mask & 0xffu);
     const uint32_t incl = warp_incl_scan(c);
     uint32_t k = base + incl - c;
-    if (t < w_end) {
-      const uint32_t t1 = (uint32_t)t + 1u;
+    const uint32_t t1 = (uint32_t)t + 1u;
 #pragma unroll
-      for (int l = 0; l < kMaxLevels; ++l) {
-        if (l >= prm.L || !ends_at(prm, t1, l)) break;
-        const int32_t g = gid_at(prm, t1, l);
-        if (selmask & (1u << l)) {
-          idx_u[k] = (int32_t)g;
-          pos_u[k] = (int32_t)t;
-          slot_u[g] = (int32_t)k;
-          ++k;
-        } else {
-          slot_u[g] = -1;
-        }
+    for (int l = 0; l < kMaxLevels; ++l) {
+      if (!((mask >> (8 + l)) & 1u)) break;
+      const int32_t g = gid_at(prm, t1, l);
+      if ((mask >> l) & 1u) {
+        idx_u[k] = (int32_t)g;
+        pos_u[k] = (int32_t)t;
+        slot_u[g] = (int32_t)k;
+        ++k;
+      } else {
+        slot_u[g] = -1;
       }
     }
     base += __shfl_sync(0xffffffffu, incl, 31);
@@ -409,8 +415,12 @@ cudaError_t launch_topk(const Geom& g, const float* score, int32_t* idx, int32_t
   int64_t per_span = 0;
   for (int l = 0; l < g.L; ++l) per_span += Ptop / g.pw[l];
   const int64_t key_bytes = sper * per_span * 4;
-  const int cached = key_bytes <= kKeyCacheBytes ? 1 : 0;
-  const size_t dyn = cached ? (size_t)key_bytes : 0;
+  int64_t mask_bytes = (sper * Ptop * 2 + 15) / 16 * 16;  // 16 bits per token
+  const int masks = mask_bytes <= kKeyCacheBytes ? 1 : 0;   // else pass B recomputes them
+  if (!masks) mask_bytes = 0;
+  const int cached = key_bytes + mask_bytes <= kKeyCacheBytes ? 1 : 0;
+  const int kcap = cached ? (int)(key_bytes / 4) : 0;
+  const size_t dyn = (size_t)kcap * 4 + (size_t)mask_bytes;
   auto launch = [&](auto clc) -> cudaError_t {
     constexpr int C = decltype(clc)::value;
     auto* kf = k_topk<C>;
@@ -434,7 +444,7 @@ cudaError_t launch_topk(const Geom& g, const float* score, int32_t* idx, int32_t
       attr[0].val.clusterDim.z = 1;
       cfg.attrs = attr;
       cfg.numAttrs = 1;
-      e = cudaLaunchKernelEx(&cfg, kf, score, idx, pos, slot, prm, cached);
+      e = cudaLaunchKernelEx(&cfg, kf, score, idx, pos, slot, prm, cached, kcap, masks);
       if (e != cudaSuccess) return e;
     }
     return cudaSuccess;
