@@ -177,10 +177,10 @@ __global__ void __launch_bounds__(256) k_gather_pooled(
 // ------------------------------------------------------------- scatter-back
 // O[t] = (sum over selected entries covering t, ascending level, of os[slot]) / c_t.
 // Grid: x = blocks of kRows tokens of one unit, y = unit (offset u0).
-// 1/c in fp64 for the contributor counts c = 0..kMaxLevels (entry 0 unused)
-__constant__ double kInvCount[kMaxLevels + 1] = {0.0,       1.0,       1.0 / 2.0,
-                                                 1.0 / 3.0, 1.0 / 4.0, 1.0 / 5.0,
-                                                 1.0 / 6.0, 1.0 / 7.0, 1.0 / 8.0};
+// 1/c rounded to fp32 for the contributor counts c = 0..kMaxLevels (entry 0 unused)
+__constant__ float kRcpCount[kMaxLevels + 1] = {0.0f,        1.0f,        1.0f / 2.0f,
+                                                1.0f / 3.0f, 1.0f / 4.0f, 1.0f / 5.0f,
+                                                1.0f / 6.0f, 1.0f / 7.0f, 1.0f / 8.0f};
 
 // One thread: column chunk c of R consecutive tokens t0..t0+R-1 (R divides p,
 // t0 a multiple of R), which share every entry of level >= 1; so each thread
@@ -238,14 +238,14 @@ __global__ void __launch_bounds__(256) k_scatter(const __half* __restrict__ os,
 #pragma unroll
       for (int i = 0; i < 8; ++i) acc[i] = __fadd_rn(acc[i], xc[l - 1][i]);
     const int cnt = cc + (s0[r] >= 0 ? 1 : 0);
-    if (cnt > 0) {
-      const double inv = kInvCount[cnt];
+    if (cnt > 0) {  // sums of fp16 values: 0 or |acc| >= 2^-24, inside div_small's range
+      const float y = kRcpCount[cnt], cf = (float)cnt;
 #pragma unroll
-      for (int i = 0; i < 8; ++i) acc[i] = div_exact(acc[i], inv);
+      for (int i = 0; i < 8; ++i) acc[i] = div_small(acc[i], cf, y);
     }
     const int64_t row = u * lv.N + t0 + r;
     store8_stream(o + row * D + 8 * c, acc);
-    if (inv_count && c == 0) inv_count[row] = cnt > 0 ? __frcp_rn((float)cnt) : 0.0f;
+    if (inv_count && c == 0) inv_count[row] = kRcpCount[cnt];  // 1/c rounded; 0 when c = 0
   }
 }
 
@@ -302,7 +302,7 @@ __global__ void __launch_bounds__(256) k_scatter_bwd(const Tin* __restrict__ dO,
           int n = 0;
 #pragma unroll
           for (int l = 0; l < L; ++l) n += (__ldg(sl + lv.off[l] + lvl_index(lv, t, l)) >= 0) ? 1 : 0;
-          ic[b] = n > 0 ? __frcp_rn((float)n) : 0.0f;
+          ic[b] = kRcpCount[n];
         }
       }
     }

@@ -144,6 +144,21 @@ __device__ __forceinline__ float div_exact(float x, double inv_c) {
   return __double2float_rn((double)x * inv_c);
 }
 
+// x / c rounded to nearest fp32 for a small integer c, in fp32 FMAs only (no
+// fp64 conversions, which run on the narrow conversion pipe): q = x*y with
+// y = 1/c rounded to fp32, the residual r = q*c - x is exact under FMA, and
+// q - r*y is the correctly rounded quotient -- Markstein's correction step
+// (P. W. Markstein, "Computation of elementary functions on the IBM RISC
+// System/6000 processor", IBM J. Res. Develop. 34(1), 1990).  Checked
+// exhaustively against IEEE division for c = 1..8 and every finite fp32 x
+// with |x| >= 2^-123 (below that, c = 6 can miss by an ulp of a subnormal);
+// a zero quotient may differ in its sign.
+__device__ __forceinline__ float div_small(float x, float c, float y) {
+  const float q = x * y;
+  const float r = fmaf(q, c, -x);
+  return fmaf(-r, y, q);
+}
+
 // ---------------------------------------------------------------- launchers
 // Each returns cudaSuccess or the launch error; arguments are already checked.
 cudaError_t launch_pyramid_score(const Geom& g, lh_dtype dt, const void* q, const void* k,

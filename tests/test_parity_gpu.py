@@ -174,7 +174,29 @@ def gpu_gather(w, x, pyr, idx):
     return out
 
 
-@pytest.mark.parametrize("case", STAGE_CASES[:4], ids=str)
+def scatter_f32(s, os_, slot):
+    """Scatter-back restated in fp32, the kernel's precision: per token, the rows
+    of its selected entries summed in ascending level order, then one IEEE
+    division by their count (zero when none).  The fp32 output must equal it
+    value for value."""
+    os_ = np.asarray(os_, np.float32)
+    t = np.arange(s.N)
+    acc = np.zeros((s.B, s.H, s.N, s.d), np.float32)
+    cnt = np.zeros((s.B, s.H, s.N), np.int64)
+    for l in range(s.L):
+        sl = slot[:, :, s.level_off(l) + t // s.p ** l]
+        sel = sl >= 0
+        rows = np.take_along_axis(os_, np.maximum(sl, 0)[..., None], axis=2)
+        acc = acc + np.where(sel[..., None], rows, np.float32(0))
+        cnt += sel
+    div = np.maximum(cnt, 1).astype(np.float32)[..., None]
+    return np.where(cnt[..., None] > 0, acc / div, np.float32(0)), cnt
+
+
+GS_CASES = STAGE_CASES[:4] + [STAGE_CASES[8], dict(p=2, L=8, N=1024, S=600)]
+
+
+@pytest.mark.parametrize("case", GS_CASES, ids=str)
 def test_gather_and_scatter_match_oracle(case):
     w = workload(**case)
     xc = make_inputs(w, "cpu")
@@ -196,6 +218,14 @@ def test_gather_and_scatter_match_oracle(case):
     ref = oracle.scatter(s, f64(os_), slot.cpu().numpy())
     tol = 2.0 ** -8 if w.dtype == "bf16" else 1e-6
     assert np.all(np.abs(f64(o) - ref) <= tol * np.abs(ref) + 1e-6)  # output-dtype rounding
+    if w.dtype == "f32":  # the correctly rounded fp32 quotient, for every count that occurs
+        exact, cnt = scatter_f32(s, f64(os_), slot.cpu().numpy())
+        got = o.cpu().numpy()
+        assert np.all(got == exact), f"scatter: {np.count_nonzero(got != exact)} values differ"
+        if w.L == 8:  # counts 2..8 all occur in this draw
+            assert set(np.unique(cnt)) >= set(range(2, 9))
+        icg = ic.cpu().numpy()
+        assert np.array_equal(icg, np.where(cnt > 0, np.float32(1) / np.maximum(cnt, 1).astype(np.float32), 0))
     # scatter-back adjoint, with and without the saved counts
     dO = x["dO"]
     for use_ic in (True, False):
