@@ -249,6 +249,155 @@ __global__ void __launch_bounds__(256) k_scatter(const __half* __restrict__ os,
   }
 }
 
+constexpr int ipow(int b, int e) { return e == 0 ? 1 : b * ipow(b, e - 1); }
+
+// 8 output elements packed once and stored any number of times (streaming).
+template <typename T>
+struct Packed8;
+template <>
+struct Packed8<__nv_bfloat16> {
+  uint4 w;
+  __device__ __forceinline__ void pack(const float (&x)[8]) {
+    w = make_uint4(pack_bf16(x[0], x[1]), pack_bf16(x[2], x[3]), pack_bf16(x[4], x[5]),
+                   pack_bf16(x[6], x[7]));
+  }
+  __device__ __forceinline__ void store(__nv_bfloat16* p) const { __stcs(reinterpret_cast<uint4*>(p), w); }
+};
+template <>
+struct Packed8<float> {
+  float4 a, b;
+  __device__ __forceinline__ void pack(const float (&x)[8]) {
+    a = make_float4(x[0], x[1], x[2], x[3]);
+    b = make_float4(x[4], x[5], x[6], x[7]);
+  }
+  __device__ __forceinline__ void store(float* p) const {
+    __stcs(reinterpret_cast<float4*>(p), a);
+    __stcs(reinterpret_cast<float4*>(p) + 1, b);
+  }
+};
+
+// Same result as k_scatter (the same additions in the same order), for p = P in
+// {2, 4} known at compile time.  A thread owns NE consecutive level-1 entries
+// (P tokens each) and walks them with the next entry's slot loads in flight while
+// the current entry's rows load, so each entry costs one memory round trip.
+// A token not selected at level 0 sums 0 + x_1 + x_2 + ... = x_1 + x_2 + ...,
+// the same value for all P tokens of its level-1 entry, so that sum, its
+// division and its packing are done once per entry and stored P times; only the
+// (few) tokens selected at level 0 form their own chain.  Grid: x = blocks of
+// level-1 entries of one unit, y = unit (offset u0).
+constexpr int kScatterEntries = 4;  // level-1 entries per thread
+
+template <typename Tout, int D, int L, int P>
+__global__ void __launch_bounds__(128) k_scatter_pp(const __half* __restrict__ os,
+                                                    const int32_t* __restrict__ slot,
+                                                    Tout* __restrict__ o, float* __restrict__ inv_count,
+                                                    const Lv lv, int64_t u0) {
+  static_assert(L >= 2 && (P == 2 || P == 4), "specialised on p in {2, 4}, L >= 2");
+  constexpr int G = D / 8, kGroups = 128 / G, NE = kScatterEntries;
+  constexpr int NU = (L > 2) ? L - 2 : 1;  // levels >= 2: one entry each
+  const int32_t n1 = lv.N / P;            // level-1 entries (N is a multiple of P)
+  const int32_t e0 = ((int32_t)blockIdx.x * kGroups + (int32_t)(threadIdx.x / G)) * NE;
+  if (e0 >= n1) return;
+  const int c = (int)(threadIdx.x % G);
+  const int64_t u = u0 + blockIdx.y;
+  const int32_t* sl = slot + u * lv.M;
+  const __half* src = os + u * lv.S * D + 8 * c;
+
+  struct Slots {
+    int32_t s0[P], s1, su[NU];
+  };
+  auto load_slots = [&](int32_t e, Slots& sv) {  // entry e < n1
+    const int32_t t = e * P;
+#pragma unroll
+    for (int r = 0; r < P; ++r) sv.s0[r] = __ldg(sl + t + r);
+    sv.s1 = __ldg(sl + lv.off[1] + e);
+    static_for<2, L>([&](auto lc) {
+      constexpr int l = decltype(lc)::value;
+      sv.su[l - 2] = __ldg(sl + lv.off[l] + (int32_t)((uint32_t)e / (uint32_t)ipow(P, l - 1)));
+    });
+  };
+  auto row = [&](int32_t sidx) {
+    uint4 w = make_uint4(0u, 0u, 0u, 0u);
+    if (sidx >= 0) w = __ldg(reinterpret_cast<const uint4*>(src + (int64_t)sidx * D));
+    return w;
+  };
+  Slots cur;
+  load_slots(e0, cur);
+#pragma unroll
+  for (int k = 0; k < NE; ++k) {
+    const int32_t e = e0 + k;
+    if (e >= n1) break;  // warp-uniform except in the last block of a unit
+    uint4 w0[P], w1, wu[NU];
+#pragma unroll
+    for (int r = 0; r < P; ++r) w0[r] = row(cur.s0[r]);
+    w1 = row(cur.s1);
+#pragma unroll
+    for (int l = 2; l < L; ++l) wu[l - 2] = row(cur.su[l - 2]);
+    Slots nxt;
+    if (k + 1 < NE && e + 1 < n1) load_slots(e + 1, nxt);  // in flight with this entry's rows
+
+    // the chain of a token unselected at level 0: x_1 + x_2 + ... (0 + x_1 = x_1
+    // exactly, up to the sign of a zero), ascending level
+    float x1[8], base[8];
+    unpack8(w1, x1);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) base[i] = x1[i];
+    int cb = cur.s1 >= 0 ? 1 : 0;
+#pragma unroll
+    for (int l = 2; l < L; ++l) {
+      float xu[8];
+      unpack8(wu[l - 2], xu);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) base[i] = __fadd_rn(base[i], xu[i]);
+      cb += cur.su[l - 2] >= 0 ? 1 : 0;
+    }
+    if (cb > 0) {  // sums of fp16 values: 0 or |sum| >= 2^-24, inside div_small's range
+      const float y = kRcpCount[cb], cf = (float)cb;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) base[i] = div_small(base[i], cf, y);
+    }
+    Packed8<Tout> ob;
+    ob.pack(base);
+    Tout* out = o + (u * lv.N + (int64_t)e * P) * D + 8 * c;
+    float icv[P];
+#pragma unroll
+    for (int r = 0; r < P; ++r) {
+      if (cur.s0[r] >= 0) {  // selected at level 0: its own chain x_0 + x_1 + x_2 + ...
+        float acc[8];
+        unpack8(w0[r], acc);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) acc[i] = __fadd_rn(acc[i], x1[i]);
+#pragma unroll
+        for (int l = 2; l < L; ++l) {
+          float xu[8];
+          unpack8(wu[l - 2], xu);
+#pragma unroll
+          for (int i = 0; i < 8; ++i) acc[i] = __fadd_rn(acc[i], xu[i]);
+        }
+        const int cnt = cb + 1;
+        const float y = kRcpCount[cnt], cf = (float)cnt;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) acc[i] = div_small(acc[i], cf, y);
+        Packed8<Tout> pr;
+        pr.pack(acc);
+        pr.store(out + r * D);
+        icv[r] = y;
+      } else {
+        ob.store(out + r * D);
+        icv[r] = kRcpCount[cb];
+      }
+    }
+    if (inv_count && c == 0) {  // the entry's P counts, one aligned vector store
+      float* ip = inv_count + u * lv.N + (int64_t)e * P;
+      if constexpr (P == 4)
+        *reinterpret_cast<float4*>(ip) = make_float4(icv[0], icv[1], icv[2], icv[3]);
+      else
+        *reinterpret_cast<float2*>(ip) = make_float2(icv[0], icv[1]);
+    }
+    if (k + 1 < NE) cur = nxt;
+  }
+}
+
 // ---------------------------------------------------------- scatter-back bwd
 // dos[k] = sum_{t in span(k)} dO[t] / c_t, as a sum-pyramid of w[t] = dO[t]/c_t
 // over each coarsest span: dO is read once, each selected row written once.
@@ -353,6 +502,208 @@ __global__ void __launch_bounds__(256) k_scatter_bwd(const Tin* __restrict__ dO,
     if (rg == 0) {
       const int32_t j = (t0 + lv.pw[L - 1]) / lv.pw[L - 1] - 1;  // the span's entry at level L-1
       const int32_t s = __ldg(sl + lv.off[L - 1] + j);
+      if (s >= 0) store8(dst + (int64_t)s * D, tot);
+    }
+  }
+}
+
+__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(
+                   (uint32_t)__cvta_generic_to_shared(dst)),
+               "l"(src)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;\n" ::"n"(N) : "memory");
+}
+
+// 8 consecutive elements staged in shared memory (16 bytes of bf16, 32 of fp32) as fp32
+__device__ __forceinline__ void staged8(const uint4* p, int stride, __nv_bfloat16*, float (&x)[8]) {
+  const uint4 w = p[0];
+  (void)stride;
+  x[0] = bf16_lo(w.x); x[1] = bf16_hi(w.x);
+  x[2] = bf16_lo(w.y); x[3] = bf16_hi(w.y);
+  x[4] = bf16_lo(w.z); x[5] = bf16_hi(w.z);
+  x[6] = bf16_lo(w.w); x[7] = bf16_hi(w.w);
+}
+__device__ __forceinline__ void staged8(const uint4* p, int stride, float*, float (&x)[8]) {
+  const float4 a = *reinterpret_cast<const float4*>(p);
+  const float4 b = *reinterpret_cast<const float4*>(p + stride);
+  x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w;
+  x[4] = b.x; x[5] = b.y; x[6] = b.z; x[7] = b.w;
+}
+
+constexpr int kScatterBwdThreads = 128;
+
+// Same sums as k_scatter_bwd (the same additions in the same order), for p = P
+// in {2, 4} known at compile time and the saved 1/c_t.  A row-group walks its
+// rows in batches of RB, two batches in flight: the rows of dO are copied by
+// 16-byte cp.async into this thread's own slots of shared memory (consecutive
+// threads take consecutive 16 bytes, so reads back are conflict-free), and each
+// batch's slots, 1/c_t and the slots of the coarse entries that complete inside it
+// are loaded into registers one batch ahead -- the stores of completed entries
+// never wait on a slot load, and a thread keeps 2 * RB rows in flight without
+// holding them in registers.
+template <typename Tin, int D, int L, int P, int RG>
+struct ScatterBwdCfg {
+  static constexpr int G = D / 8;
+  static constexpr int LW = (RG == 1) ? L - 1 : L - 2;  // coarse levels completed inside the walk
+  static constexpr int Ptop = ipow(P, L - 1) / RG;        // rows one row-group walks
+  static constexpr int CPR = sizeof(Tin) / 2;             // 16-byte copies per lane per row
+  static constexpr int RBmax = 8 / CPR;
+  static constexpr int RB = Ptop < RBmax ? Ptop : RBmax;  // rows per batch
+  static constexpr int NB = Ptop / RB;                    // batches
+  // level-l entries whose slot a batch loads: those inside it, or the one it ends in
+  static constexpr int cnt(int l) { return ipow(P, l) <= RB ? RB / ipow(P, l) : 1; }
+  static constexpr int first(int l) { return l <= 1 ? 0 : first(l - 1) + cnt(l - 1); }
+  static constexpr int NCS = LW > 0 ? first(LW + 1) : 1;  // coarse slots per batch
+  static constexpr size_t smem_bytes = (size_t)2 * RB * CPR * kScatterBwdThreads * 16;
+};
+
+// Grid: x = blocks of spans of one unit, y = unit (offset u0).
+template <typename Tin, int D, int L, int P, int RG>
+__global__ void __launch_bounds__(kScatterBwdThreads) k_scatter_bwd_pp(
+    const Tin* __restrict__ dO, const int32_t* __restrict__ slot,
+    const float* __restrict__ inv_count, __half* __restrict__ dos, const Lv lv, int32_t spans,
+    int64_t u0) {
+  using C = ScatterBwdCfg<Tin, D, L, P, RG>;
+  constexpr int G = C::G, LW = C::LW, Ptop = C::Ptop, CPR = C::CPR, RB = C::RB, NB = C::NB;
+  constexpr int NCS = C::NCS, NA = LW > 0 ? LW : 1, NT = kScatterBwdThreads;
+  static_assert(L >= 2 && (P == 2 || P == 4), "specialised on p in {2, 4}, L >= 2");
+  static_assert(RG == 1 || (RG == P && G * RG <= 32), "row-groups of a span share one warp");
+  static_assert(Ptop % RB == 0, "batches tile the walk");
+  extern __shared__ uint4 sbuf[];  // [2 stages][RB][CPR][NT], this thread's column tid
+
+  const int tid = (int)threadIdx.x;
+  const int32_t gt = (int32_t)blockIdx.x * NT + tid;
+  const int32_t span = gt / (G * RG);
+  if (span >= spans) return;  // whole spans leave together (G * RG divides 32)
+  const int c = gt % G;
+  const int rg = (gt / G) % RG;
+  const int64_t u = u0 + blockIdx.y;
+  const int32_t t0 = span * ipow(P, L - 1) + rg * Ptop;
+  const int32_t* sl = slot + u * lv.M;
+  const float* icu = inv_count + u * lv.N;
+  const Tin* src = dO + (u * lv.N + t0) * D + 8 * c;
+  __half* dst = dos + u * lv.S * D + 8 * c;
+
+  auto issue = [&](int bi) {  // rows of batch bi into stage bi & 1
+    uint4* st = sbuf + (bi & 1) * (RB * CPR * NT) + tid;
+    const Tin* g = src + bi * (RB * D);
+    static_for<0, RB>([&](auto bc) {
+      constexpr int b = decltype(bc)::value;
+      static_for<0, CPR>([&](auto qc) {
+        constexpr int q = decltype(qc)::value;
+        cp_async16(st + (b * CPR + q) * NT, g + b * D + 4 * q);
+      });
+    });
+    cp_async_commit();
+  };
+  auto small_loads = [&](int bi, int32_t (&s0_)[RB], float (&ic_)[RB], int32_t (&cs_)[NCS]) {
+    const int32_t tb = t0 + bi * RB;  // first token of the batch
+    static_for<0, RB>([&](auto bc) {
+      constexpr int b = decltype(bc)::value;
+      s0_[b] = __ldg(sl + tb + b);
+      ic_[b] = __ldg(icu + tb + b);
+    });
+    static_for<1, LW + 1>([&](auto lc) {
+      constexpr int l = decltype(lc)::value;
+      constexpr uint32_t pl = (uint32_t)ipow(P, l);
+      constexpr int n = C::first(l), k = C::cnt(l);
+      const int32_t j0 = (int32_t)((uint32_t)(tb + (pl <= (uint32_t)RB ? 0 : RB - 1)) / pl);
+      static_for<0, k>([&](auto ic2) {
+        constexpr int i = decltype(ic2)::value;
+        cs_[n + i] = __ldg(sl + lv.off[l] + j0 + i);
+      });
+    });
+  };
+  int32_t s0[RB], cs[NCS];
+  float ic[RB];
+  issue(0);
+  if (NB > 1) issue(1);
+  small_loads(0, s0, ic, cs);
+
+  float acc[NA][8];  // acc[l-1]: running sum of the current level-l entry
+#pragma unroll
+  for (int l = 0; l < NA; ++l)
+#pragma unroll
+    for (int i = 0; i < 8; ++i) acc[l][i] = 0.0f;
+  float part[8];  // the walk's last completed entry (level LW; a row when LW = 0)
+
+  for (int bi = 0; bi < NB; ++bi) {
+    const int32_t r0 = bi * RB;
+    int32_t s0n[RB], csn[NCS];
+    float icn[RB];
+    if (bi + 1 < NB) small_loads(bi + 1, s0n, icn, csn);
+    if (bi + 1 < NB) cp_async_wait<1>(); else cp_async_wait<0>();
+    const uint4* stg = sbuf + (bi & 1) * (RB * CPR * NT) + tid;
+    static_for<0, RB>([&](auto bc) {
+      constexpr int b = decltype(bc)::value;
+      float w[8];
+      staged8(stg + b * CPR * NT, NT, (Tin*)nullptr, w);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) w[i] = __fmul_rn(w[i], ic[b]);
+      if (s0[b] >= 0) store8(dst + (int64_t)s0[b] * D, w);
+      if constexpr (LW == 0) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) part[i] = w[i];
+      } else {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) acc[0][i] = __fadd_rn(acc[0][i], w[i]);
+        // entries completed by row r0 + b, finest first (each adds into the next level)
+        static_for<1, LW + 1>([&](auto lc) {
+          constexpr int l = decltype(lc)::value;
+          constexpr int pl = ipow(P, l);
+          constexpr bool inside = pl <= RB;  // the level's entries lie inside a batch
+          constexpr int k = C::first(l) + (inside ? (b + 1) / pl - 1 : 0);
+          bool done;
+          if constexpr (inside)
+            done = ((b + 1) % pl) == 0;
+          else
+            done = (b == RB - 1) && ((r0 + RB) % pl) == 0;
+          if (done) {
+            if (cs[k] >= 0) store8(dst + (int64_t)cs[k] * D, acc[l - 1]);
+            if constexpr (l < LW) {
+#pragma unroll
+              for (int i = 0; i < 8; ++i) acc[l][i] = __fadd_rn(acc[l][i], acc[l - 1][i]);
+            } else {
+#pragma unroll
+              for (int i = 0; i < 8; ++i) part[i] = acc[l - 1][i];
+            }
+#pragma unroll
+            for (int i = 0; i < 8; ++i) acc[l - 1][i] = 0.0f;
+          }
+        });
+      }
+    });
+    if (bi + 2 < NB) issue(bi + 2);  // into the stage this thread just read
+    if (bi + 1 < NB) {
+#pragma unroll
+      for (int b = 0; b < RB; ++b) {
+        s0[b] = s0n[b];
+        ic[b] = icn[b];
+      }
+#pragma unroll
+      for (int i = 0; i < NCS; ++i) cs[i] = csn[i];
+    }
+  }
+  if constexpr (RG > 1) {
+    // the span's level-(L-1) entry: the RG partial sums, added in row-group order
+    const int lane = threadIdx.x & 31;
+    const int base = lane - rg * G;  // lane of row-group 0 with this chunk
+    const unsigned mask = (G * RG == 32) ? 0xffffffffu
+                                         : (((1u << (G * RG)) - 1u) << (lane & ~(G * RG - 1)));
+    float tot[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) tot[i] = __shfl_sync(mask, part[i], base);
+#pragma unroll
+    for (int r = 1; r < RG; ++r)
+#pragma unroll
+      for (int i = 0; i < 8; ++i) tot[i] = __fadd_rn(tot[i], __shfl_sync(mask, part[i], base + r * G));
+    if (rg == 0) {
+      const int32_t s = __ldg(sl + lv.off[L - 1] + span);
       if (s >= 0) store8(dst + (int64_t)s * D, tot);
     }
   }
@@ -566,6 +917,20 @@ template <typename Tout, int D>
 cudaError_t scatter_t(const Geom& g, const __half* os, const int32_t* slot, Tout* o,
                       float* inv_count, cudaStream_t st) {
   const Lv lv = make_lv(g);
+  if (g.L >= 2 && (g.p == 2 || g.p == 4)) {  // p known at compile time: p tokens a thread
+    const unsigned bxp = blocks_for(g.N / g.p, (128 / (D / 8)) * kScatterEntries);
+    return with_levels(g.L, [&](auto lc) {
+      constexpr int LL = decltype(lc)::value;
+      if constexpr (LL >= 2) {
+        per_unit_chunks(g.U, [&](int64_t u0, unsigned nu) {
+          if (g.p == 4)
+            k_scatter_pp<Tout, D, LL, 4><<<dim3(bxp, nu), 128, 0, st>>>(os, slot, o, inv_count, lv, u0);
+          else
+            k_scatter_pp<Tout, D, LL, 2><<<dim3(bxp, nu), 128, 0, st>>>(os, slot, o, inv_count, lv, u0);
+        });
+      }
+    });
+  }
   const int R = tokens_per_thread(g);
   const unsigned bx = blocks_for(g.N / R, 256 / (D / 8));
   return with_tokens(R, [&](auto rc) {
@@ -620,6 +985,28 @@ cudaError_t scatter_bwd_d(const Geom& g, const Tin* dO, const int32_t* slot, con
   return with_levels(g.L, [&](auto lc) {
     constexpr int LL = decltype(lc)::value;
     if constexpr (LL > 1) {
+      if (ic != nullptr && (g.p == 2 || g.p == 4)) {  // staged loads, p known at compile time
+        auto go = [&](auto pc, auto rgc) {
+          constexpr int PP = decltype(pc)::value, RR = decltype(rgc)::value;
+          using C = ScatterBwdCfg<Tin, D, LL, PP, RR>;
+          const unsigned bx = blocks_for(spans * (D / 8) * RR, kScatterBwdThreads);
+          per_unit_chunks(g.U, [&](int64_t u0, unsigned nu) {
+            k_scatter_bwd_pp<Tin, D, LL, PP, RR><<<dim3(bx, nu), kScatterBwdThreads, C::smem_bytes, st>>>(
+                dO, slot, ic, dos, lv, (int32_t)spans, u0);
+          });
+        };
+        if (g.p == 4) {
+          if (RG == 4) {
+            if constexpr ((D / 8) * 4 <= 32)
+              go(std::integral_constant<int, 4>{}, std::integral_constant<int, 4>{});
+          } else {
+            go(std::integral_constant<int, 4>{}, std::integral_constant<int, 1>{});
+          }
+        } else {
+          go(std::integral_constant<int, 2>{}, std::integral_constant<int, 2>{});
+        }
+        return;
+      }
       if (RG == 4) {
         if constexpr ((D / 8) * 4 <= 32) {
           k_scatter_bwd<Tin, D, LL, 4><<<nb, 256, 0, st>>>(dO, slot, ic, dos, lv, spans, groups);

@@ -1,6 +1,8 @@
 // lh_internal.cuh -- shared definitions of the CUDA library (not part of the ABI).
 #pragma once
 
+#include <type_traits>
+
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
@@ -36,6 +38,17 @@ enum : uint32_t {
 };
 
 __device__ __forceinline__ int64_t imin64(int64_t a, int64_t b) { return a < b ? a : b; }
+
+// f(std::integral_constant<int, i>) for i = I .. N-1: a loop whose index is a
+// compile-time constant in the body (register arrays stay in registers, powers
+// and divisions by them fold), whether or not the compiler would unroll it.
+template <int I, int N, typename F>
+__device__ __forceinline__ void static_for(F&& f) {
+  if constexpr (I < N) {
+    f(std::integral_constant<int, I>{});
+    static_for<I + 1, N>(f);
+  }
+}
 
 // ---------------------------------------------------------------- small helpers
 __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }

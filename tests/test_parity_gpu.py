@@ -193,7 +193,14 @@ def scatter_f32(s, os_, slot):
     return np.where(cnt[..., None] > 0, acc / div, np.float32(0)), cnt
 
 
-GS_CASES = STAGE_CASES[:4] + [STAGE_CASES[8], dict(p=2, L=8, N=1024, S=600)]
+GS_CASES = STAGE_CASES[:4] + [
+    STAGE_CASES[8],
+    dict(p=2, L=8, N=1024, S=600),
+    dict(dtype="bf16", p=4, L=2, N=1000, S=256),   # N not a multiple of p^2: ragged last thread
+    dict(dtype="bf16", p=2, L=2, N=1002, S=384),
+    dict(dtype="bf16", d=128, p=4, L=4, N=4096, S=512),
+    dict(p=4, L=5, N=2048, S=384),                 # fp32 input, several batches per span walk
+]
 
 
 @pytest.mark.parametrize("case", GS_CASES, ids=str)
