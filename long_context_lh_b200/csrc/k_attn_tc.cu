@@ -78,7 +78,7 @@ struct FwdLayout {
 };
 
 struct FwdBars {
-  uint64_t q_full;
+  uint64_t q_full, q_tmem;  // Q tiles in shared memory; (d = 64) copied on into TMEM
   uint64_t kv_full[4], kv_empty[4];
   uint64_t s_full[2], p_full[2], pv_done[2], mma_done;  // [tile A, B]
   uint32_t tmem;
@@ -134,6 +134,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&bars->pv_done[t], 1);
     }
     mbar_init(&bars->mma_done, 1);
+    mbar_init(&bars->q_tmem, 8);
     bars->abort = 0;
     mbar_init_fence();
   }
@@ -143,6 +144,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = bars->tmem;
   const uint32_t tO = tmem + 256;  // O_A at +256, O_B at +256+D; S_T at +128*T
+  // d = 64: Q_A, Q_B also live in TMEM (32 columns each, at +384 and +416) and
+  // are the A operand of S = Q K^T, so those products read only K from shared
+  // memory (both operands from shared memory halve their rate)
+  constexpr bool kQT = (D == 64);
+  static_assert(!kQT || 256 + 2 * D + 64 <= (int)kTmemCols, "TMEM: S_A, S_B, O_A, O_B, Q_A, Q_B");
+  const uint32_t tQ = tmem + 256 + 2 * D;
 
   if (warp == 8) {
     // ------------------------------------------------------------ TMA producer
@@ -184,7 +191,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint64_t off = (uint64_t)((((kk >> 2) * 16384) + ((kk & 3) * 32)) >> 4);
-          umma_f16(tmem + t * 128, q + off, k + off, idS, kk > 0);
+          if constexpr (kQT)
+            umma_f16_ta(tmem + t * 128, tQ + t * 32 + 8 * kk, k + off, idS, kk > 0);
+          else
+            umma_f16(tmem + t * 128, q + off, k + off, idS, kk > 0);
         }
         umma_commit(&bars->s_full[t]);
       }
@@ -201,7 +211,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       __syncwarp();
     };
-    bool ok = warp_wait(&bars->q_full, 0, abort, kStatus) &&
+    bool ok = warp_wait(kQT ? &bars->q_tmem : &bars->q_full, 0, abort, kStatus) &&
               warp_wait(&bars->kv_full[0], 0, abort, kStatus);
     if (ok) {
       tc_fence_after();
@@ -257,19 +267,22 @@ __global__ void __launch_bounds__(kThreads, 1)
       ok = warp_wait(&bars->s_full[t], j & 1, abort, kStatus);
       if (!ok) return;
       tc_fence_after();
-      // pass 1: the row max, 32 columns at a time (four independent chains)
+      // the row max over the whole row of S (128 columns): four loads, one wait,
+      // four independent chains
       float mc[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        uint32_t v[32];
-        tmem_ld32(tS + 32 * c, v);
+      {
+        uint32_t v[128];
+        tmem_ld32_at<0>(tS, v);
+        tmem_ld32_at<32>(tS + 32, v);
+        tmem_ld32_at<64>(tS + 64, v);
+        tmem_ld32_at<96>(tS + 96, v);
         tmem_ld_wait();
 #pragma unroll
-        for (int i = 0; i < 32; i += 2) {
+        for (int i = 0; i < 128; i += 2) {
           const int k = (i >> 1) & 3;
           if (kDiag) {
-            mc[k] = max3(mc[k], 32 * c + i <= r ? __uint_as_float(v[i]) : -INFINITY,
-                         32 * c + i + 1 <= r ? __uint_as_float(v[i + 1]) : -INFINITY);
+            mc[k] = max3(mc[k], i <= r ? __uint_as_float(v[i]) : -INFINITY,
+                         i + 1 <= r ? __uint_as_float(v[i + 1]) : -INFINITY);
           } else {
             mc[k] = max3(mc[k], __uint_as_float(v[i]), __uint_as_float(v[i + 1]));
           }
@@ -299,23 +312,29 @@ __global__ void __launch_bounds__(kThreads, 1)
         l *= alpha;
       }
       m_ref = m_new;
-      // pass 2: P = 2^(S c - m_ref), 32 columns at a time, packed fp16 written
-      // over S columns already read (chunk c writes columns 16c..16c+15)
+      // P = 2^(S c - m_ref): S read again in two 64-column halves (two loads, one
+      // wait each), packed fp16 written over S columns already read (chunk c of
+      // 32 columns writes columns 16c..16c+15)
       const float2 cc = make_float2(scale_log2, scale_log2), nm = make_float2(-m_ref, -m_ref);
       float2 sacc[4] = {make_float2(0.0f, 0.0f), make_float2(0.0f, 0.0f), make_float2(0.0f, 0.0f),
                         make_float2(0.0f, 0.0f)};
+      uint32_t v[64];
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
-        uint32_t v[32];
-        tmem_ld32(tS + 32 * c, v);
-        tmem_ld_wait();
+        if ((c & 1) == 0) {
+          tmem_ld32_at<0>(tS + 32 * c, v);
+          tmem_ld32_at<32>(tS + 32 * c + 32, v);
+          tmem_ld_wait();
+        }
         uint32_t pk[16];
 #pragma unroll
         for (int i = 0; i < 32; i += 4) {
-          const float2 x = ffma2(make_float2(__uint_as_float(v[i]), __uint_as_float(v[i + 1])), cc, nm);
-          const float2 y = ffma2(make_float2(__uint_as_float(v[i + 2]), __uint_as_float(v[i + 3])), cc, nm);
+          const int a = 32 * (c & 1) + i;
+          const float2 x = ffma2(make_float2(__uint_as_float(v[a]), __uint_as_float(v[a + 1])), cc, nm);
+          const float2 y = ffma2(make_float2(__uint_as_float(v[a + 2]), __uint_as_float(v[a + 3])), cc, nm);
           float2 p = make_float2(ex2(x.x), ex2(x.y));
-          // a quarter of the exponentials on the FMA pipe, the rest on MUFU
+          // a quarter of the exponentials on the FMA pipe, the rest on MUFU (half
+          // on the FMA pipe measured slower: the row work is then issue-bound)
           float2 q = (i & 7) == 4 ? ex2_fma2(y) : make_float2(ex2(y.x), ex2(y.y));
           if (kDiag) {
             const int k0 = 32 * c + i;
@@ -339,7 +358,30 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float2 s01 = fadd2(sacc[0], sacc[1]), s23 = fadd2(sacc[2], sacc[3]);
       l += (s01.x + s01.y) + (s23.x + s23.y);
     };
-    if (n > 0) {
+    if constexpr (kQT) {
+      // this thread's row of its Q tile: shared memory (128-byte swizzled) -> TMEM
+      // columns of Q_t, two fp16 along K per column (lower index in the low half).
+      // Every row-work warp arrives (a tile B that does not exist copies zeros).
+      ok = warp_wait(&bars->q_full, 0, abort, kStatus);
+      if (ok) {
+        const uint8_t* qrow = sQ + t * Lt::kTile;
+        uint32_t w[32];
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          const uint4 x = *reinterpret_cast<const uint4*>(qrow + swz(r, c));
+          w[4 * c] = x.x;
+          w[4 * c + 1] = x.y;
+          w[4 * c + 2] = x.z;
+          w[4 * c + 3] = x.w;
+        }
+        tmem_st32(tQ + t * 32 + lane_addr, w);
+        tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars->q_tmem);
+      }
+    }
+    if (n > 0 && ok) {
       for (int j = 0; j < n - 1 && ok; ++j) step(j, std::false_type{});
       if (ok) step(n - 1, std::true_type{});
       if (ok) ok = warp_wait(&bars->pv_done[t], (n - 1) & 1, abort, kStatus);
