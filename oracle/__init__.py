@@ -201,6 +201,52 @@ def attn_bwd(s: Shape, qs, ks, vs, dos, scale, nthreads=None):
     return dq.reshape(shp), dk.reshape(shp), dv.reshape(shp)
 
 
+def attn_bwd_sampled(qs, ks, vs, dos, scale, rows, chunk=1024):
+    """Gradients of causal softmax attention (one unit, fp64 numpy) at sampled
+    positions, for sub-sequences too long for the full O(S^2 d) loops above.
+
+    The softmax adjoint is separable: with P = softmax over k' <= k of
+    scale * q_k . k_k', O = P V, D_k = dO_k . O_k and dS = P * (dO V^T - D),
+      dQ[k]  = scale * sum_k' dS[k, k'] K[k']        (row k of dS),
+      dK[k'] = scale * sum_k  dS[k, k'] Q[k]         (column k' of dS),
+      dV[k'] = sum_k P[k, k'] dO[k]                  (column k' of P),
+    ([ES] gist.science/es "Resumen Técnico: Pre-entrenamiento con Contexto
+    Largo mediante Atención Lighthouse", §2.B: the backward through the dense
+    sub-sequence attention is the stock one).  Row k needs every key; column
+    k' needs every query's LSE and D, which one blocked pass over all rows of
+    P gives.  Inputs [S, d]; returns dq[rows], dk[rows], dv[rows], [len(rows), d].
+    """
+    q, k, v, do = (np.asarray(t, np.float64) for t in (qs, ks, vs, dos))
+    S = q.shape[0]
+    rows = np.asarray(rows, np.int64)
+    lse = np.empty(S)
+    o = np.empty_like(q)
+    for a in range(0, S, chunk):  # LSE and O of every row, blocked over rows
+        b = min(S, a + chunk)
+        z = scale * (q[a:b] @ k.T)
+        z[np.arange(S)[None, :] > np.arange(a, b)[:, None]] = -np.inf  # key after the query
+        m = z.max(axis=1, keepdims=True)
+        e = np.exp(z - m)
+        ssum = e.sum(axis=1, keepdims=True)
+        lse[a:b] = (m + np.log(ssum))[:, 0]
+        o[a:b] = (e / ssum) @ v
+    dsum = np.einsum("kd,kd->k", do, o)  # D_k
+    # rows of dS -> dQ
+    zr = scale * (q[rows] @ k.T)
+    keep = np.arange(S)[None, :] <= rows[:, None]
+    pr = np.where(keep, np.exp(zr - lse[rows, None]), 0.0)
+    dsr = pr * ((do[rows] @ v.T) - dsum[rows, None])
+    dq = scale * (dsr @ k)
+    # columns of P and dS -> dV, dK
+    zc = scale * (q @ k[rows].T)  # [S, len(rows)]
+    keepc = np.arange(S)[:, None] >= rows[None, :]
+    pc = np.where(keepc, np.exp(zc - lse[:, None]), 0.0)
+    dv = pc.T @ do
+    dsc = pc * ((do @ v[rows].T) - dsum[:, None])
+    dk = scale * (dsc.T @ q)
+    return dq, dk, dv
+
+
 def scatter(s: Shape, os_, slot) -> np.ndarray:
     os_ = _f64(os_).reshape(s.U, s.S, s.d)
     slot = _i32(slot).reshape(s.U, s.M)

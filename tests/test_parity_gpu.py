@@ -344,63 +344,84 @@ def test_bitwise_deterministic():
         assert torch.equal(a, b)
 
 
-def test_pretraining_shape_full_size():
-    """The benchmark's workload (H=16, N=98,304, S=8192) in the launch the bench times.
+def check_full_size(name, device_draw=False, n_tokens=24, full_backward_head0=False):
+    """A benchmark workload at full size, through lh_forward / lh_backward as the
+    bench launches them.
 
-    Every head: scores and the selection bit-exact.  Heads 0 and H-1: pyramid,
-    gathered rows, 64 sampled attention rows and the tokens they scatter to;
-    head 0: the full attention backward."""
-    w = WORKLOADS["pretrain"]
-    xc = make_inputs(w, "cpu")
-    x = to_dev(xc)
+    Every head: scores and the selection (idx, slot) bit-exact.  Heads 0 and
+    H-1: gathered rows; the contributor slots R of n_tokens random tokens (plus
+    tokens without contributors): attention rows os[R] from the oracle, and the
+    layer's outputs O, dQ, dK, dV at those tokens, each built by the oracle's own
+    scatter-back / gather adjoint from the oracle's rows R (oracle.scatter_bwd
+    for dos, oracle.attn_bwd_sampled for the gradient rows and columns).  No
+    oracle input comes from the GPU: the selection it uses is its own (checked
+    equal first)."""
+    w = WORKLOADS[name]
+    xg = make_inputs(w, "cuda" if device_draw else "cpu")
+    x = to_dev(xg)
     o, saved = lh.forward(x["q"], x["k"], x["v"], w.p, w.L, w.S)
     dq, dk, dv = lh.backward(saved, x["dO"])
     torch.cuda.synchronize()
-    s = oshape(w)
-    qf, kf = xc["q"].float().numpy(), xc["k"].float().numpy()
-    sc_ref = oracle.score(s, qf, kf)
-    i_ref, p_ref, s_ref = oracle.select(s, sc_ref)
     sv = lambda which: lh.saved_view(saved.shape, saved.buf, which)
-    assert np.array_equal(sv(lh.SAVED_IDX).cpu().numpy(), i_ref)
-    assert np.array_equal(sv(lh.SAVED_SLOT).cpu().numpy(), s_ref)
+    idx_g, slot_g = sv(lh.SAVED_IDX).cpu().numpy(), sv(lh.SAVED_SLOT).cpu().numpy()
+    s1 = oshape(w).unit()
+    head = lambda t, h: t[:, h:h + 1].float().cpu().numpy()
+    refs = {}
+    for h in range(w.H):
+        sc = oracle.score(s1, head(xg["q"], h), head(xg["k"], h))
+        i_ref, _, s_ref = oracle.select(s1, sc)
+        assert np.array_equal(idx_g[:, h:h + 1], i_ref), f"idx head {h}"
+        assert np.array_equal(slot_g[:, h:h + 1], s_ref), f"slot head {h}"
+        refs[h] = (i_ref, s_ref)
     rng = np.random.default_rng(7)
+    scale = 1.0 / np.sqrt(w.d)
     for h in (0, w.H - 1):
-        s1 = s.unit()
+        i_ref, s_ref = refs[h]
         xs = []
         for n in ("q", "k", "v"):
-            a = xc[n][:, h:h + 1].float().numpy()
-            xs.append(oracle.gather(s1, a, oracle.pyramid(s1, a), i_ref[:, h:h + 1]))
+            a = head(xg[n], h)
+            xs.append(oracle.gather(s1, a, oracle.pyramid(s1, a), i_ref))
         for ref, which in zip(xs, (lh.SAVED_QS, lh.SAVED_KS, lh.SAVED_VS)):
             check_gathered(f64(sv(which)[:, h:h + 1]), ref)
-        rows = np.sort(rng.choice(w.S, 64, replace=False)).astype(np.int32)
-        os_ref, lse_ref = oracle.attn_fwd(s1, *xs, 1.0 / np.sqrt(w.d), rows=rows)
-        check_attn(f64(sv(lh.SAVED_OS)[:, h:h + 1, rows]), os_ref, f"os head {h}")
-        # tokens whose contributors are all among the sampled rows
-        slot_h = s_ref[0, h]
-        os_full = np.full((w.S, w.d), np.nan)
-        os_full[rows] = os_ref[0, 0]
-        toks = rng.choice(w.N, 4096, replace=False)
-        got_o = f64(o[0, h])
-        checked = 0
-        for t in toks:
-            sl = [slot_h[s.level_off(l) + t // w.p ** l] for l in range(w.L)]
-            sl = [z for z in sl if z >= 0]
-            if not sl or not all(z in set(rows.tolist()) for z in sl):
-                continue
-            ref_t = np.mean([os_full[z] for z in sl], axis=0)
-            check_attn(got_o[t][None], ref_t[None], f"o token {t}")
-            checked += 1
-        assert checked > 0
-    # full attention backward of head 0 on the GPU's own bf16 operands
-    s1 = s.unit()
-    dos_gpu = torch.empty((1, 1, w.S, w.d), dtype=torch.float16, device=DEV)
-    lh.lh_scatter_back_bwd(lh.make_shape(1, 1, w.N, w.d, w.p, w.L, w.S), lh.LH_BF16,
-                           x["dO"][:, :1].contiguous(), sv(lh.SAVED_SLOT)[:, :1].contiguous(),
-                           sv(lh.SAVED_INV_COUNT)[:, :1].contiguous(), dos_gpu)
-    ops = [f64(sv(which)[:, :1]) for which in (lh.SAVED_QS, lh.SAVED_KS, lh.SAVED_VS)]
-    dos_ref = oracle.scatter_bwd(s1, xc["dO"][:, :1].float().numpy(), i_ref[:, :1], s_ref[:, :1])
-    check_attn(f64(dos_gpu), dos_ref, "dos head 0")
-    refs = oracle.attn_bwd(s1, *ops, f64(dos_gpu), 1.0 / np.sqrt(w.d))
-    dref = [oracle.gather_bwd(s1, r, s_ref[:, :1]) for r in refs]
-    for name, t, r in zip(("dq", "dk", "dv"), (dq, dk, dv), dref):
-        check_attn(f64(t[:, :1]), r, f"{name} head 0")
+        slot_h = s_ref[0, 0]
+        contrib = lambda t: [int(slot_h[s1.level_off(l) + t // w.p ** l]) for l in range(w.L)]
+        toks, uncovered = [], []
+        while len(toks) < n_tokens:
+            t = int(rng.integers(w.N))
+            (toks if any(z >= 0 for z in contrib(t)) else uncovered).append(t)
+        rows = np.unique([z for t in toks for z in contrib(t) if z >= 0]).astype(np.int32)
+        toks = np.array(toks + uncovered[:8], dtype=np.int64)
+        os_r, _ = oracle.attn_fwd(s1, *xs, scale, rows=rows)
+        check_attn(f64(sv(lh.SAVED_OS)[:, h:h + 1, rows]), os_r, f"os head {h}")
+        os_part = np.zeros((1, 1, w.S, w.d))
+        os_part[0, 0, rows] = os_r[0, 0]
+        o_ref = oracle.scatter(s1, os_part, s_ref)[0, 0, toks]
+        check_attn(f64(o[0, h, toks]), o_ref, f"o head {h}")
+        dos_ref = oracle.scatter_bwd(s1, head(xg["dO"], h), i_ref, s_ref)
+        g_r = oracle.attn_bwd_sampled(*(t[0, 0] for t in xs), dos_ref[0, 0], scale, rows)
+        for gname, g_rows, got in zip(("dq", "dk", "dv"), g_r, (dq, dk, dv)):
+            part = np.zeros((1, 1, w.S, w.d))
+            part[0, 0, rows] = g_rows
+            g_ref = oracle.gather_bwd(s1, part, s_ref)[0, 0, toks]
+            check_attn(f64(got[0, h, toks]), g_ref, f"{gname} head {h}")
+        if full_backward_head0 and h == 0:  # every token of head 0, from the full oracle backward
+            full = oracle.attn_bwd(s1, *xs, dos_ref, scale)
+            for gname, g_s, got in zip(("dq", "dk", "dv"), full, (dq, dk, dv)):
+                check_attn(f64(got[:, :1]), oracle.gather_bwd(s1, g_s, s_ref), f"{gname} head 0 (all tokens)")
+
+
+def test_pretraining_shape_full_size():
+    """The pretraining workload (H=16, N=98,304, S=8192), as the bench runs it; head 0's
+    gradients at every token from the oracle's full attention backward."""
+    check_full_size("pretrain", full_backward_head0=True)
+
+
+def test_long_context_full_size():
+    """The long-context workload (H=16, N=524,288, L=5, S=16,384), as the bench runs it."""
+    check_full_size("long", device_draw=True)
+
+
+def test_extreme_context_full_size():
+    """The one-GPU extreme workload (H=8, N=1,048,576, d=128, L=6, S=16,384, log-normal
+    token norms), as the bench runs it."""
+    check_full_size("extreme", device_draw=True)
