@@ -167,84 +167,39 @@ class ClockSampler:
 
 
 # ------------------------------------------------------------------ our arm
-def run_ours(args, rk):
-    import numpy as np  # noqa: F401
-    from long_context_lh_b200 import lighthouse as lh
+STAGES_FWD = ["pyramid_score", "topk", "gather", "attn_fwd", "scatter"]
+STAGES_BWD = ["scatter_bwd", "attn_bwd", "gather_bwd"]
 
-    rank, world, local_rank = rk.rank, rk.world, rk.local_rank
-    torch.cuda.set_device(local_rank)
-    dev = torch.device("cuda", local_rank)
-    w = WORKLOADS[args.workload]
-    if args.heads:
-        w = w.with_(H=args.heads)
-    if args.attn == "mma":
-        lh.lh_set_attention_impl(1)
-    elif args.attn == "tc":
-        lh.lh_set_attention_impl(0)
-    peaks, peaks_src = load_peaks()
+
+def measure(lh, w, args, rk, dev, peaks, steps, warmup, backward=True, batch=0, clocks=False):
+    """Time one workload through lh_forward (+ lh_backward) on this rank's GPU, then
+    replay the same launches stage by stage with events between stages.  Returns
+    the timings, the per-stage roofline report, the tensors of the fused run and
+    the peak device memory the fused path held (inputs, outputs, saved state and
+    workspace)."""
+    torch.cuda.synchronize()
+    torch.cuda.reset_peak_memory_stats(dev)
+    mem0 = torch.cuda.memory_allocated(dev)
     shp = lh.make_shape(w.B, w.H, w.N, w.d, w.p, w.L, w.S)
     dt = lh.dtype_code(w.torch_dtype)
-    x = make_inputs(w, dev, batch=rank)  # each rank: its own independent batch
-    q, k, v, dO = x["q"], x["k"], x["v"], x["dO"]
+    x = make_inputs(w, dev, with_dO=backward, batch=batch)  # each rank: its own batch
+    q, k, v = x["q"], x["k"], x["v"]
+    dO = x.get("dO")
     o = torch.empty_like(q)
-    dq, dk, dv = (torch.empty_like(q) for _ in range(3))
+    dq, dk, dv = ((torch.empty_like(q) for _ in range(3)) if backward else (None, None, None))
     saved = torch.empty(lh.lh_saved_bytes(shp), dtype=torch.uint8, device=dev)
-    wsb = lh.lh_workspace_bytes(shp, dt, True)
+    wsb = lh.lh_workspace_bytes(shp, dt, backward)
     ws = torch.empty(wsb, dtype=torch.uint8, device=dev)
     stream = torch.cuda.Stream(device=dev)
     sp = stream.cuda_stream
 
-    def step():
-        lh.lh_forward(shp, dt, q, k, v, 0.0, o, saved, ws, wsb, sp)
-        lh.lh_backward(shp, dt, saved, dO, 0.0, dq, dk, dv, ws, wsb, sp)
-
     def fwd_only():
         lh.lh_forward(shp, dt, q, k, v, 0.0, o, saved, ws, wsb, sp)
 
-    # stage-by-stage replica of the same launches, for per-kernel durations
-    M = w.M
-    U = w.B * w.H
-    base = saved
-
-    def view(which, dtype, n):
-        off = lh.lh_saved_offset(shp, which)
-        return base[off:off + n * torch.tensor([], dtype=dtype).element_size()].view(dtype)
-
-    idx = view(lh.SAVED_IDX, torch.int32, U * w.S)
-    pos = view(lh.SAVED_POS, torch.int32, U * w.S)
-    slot = view(lh.SAVED_SLOT, torch.int32, U * M)
-    qs, ks, vs, os_ = (view(i, torch.float16, U * w.S * w.d)
-                       for i in (lh.SAVED_QS, lh.SAVED_KS, lh.SAVED_VS, lh.SAVED_OS))
-    lse = view(lh.SAVED_LSE, torch.float32, U * w.S)
-    ic = view(lh.SAVED_INV_COUNT, torch.float32, U * w.N)
-    npyr = max(U * (M - w.N) * w.d, 1)
-    pq, pk, pv = (torch.empty(npyr, dtype=torch.float32, device=dev) for _ in range(3))
-    score = torch.empty(U * M, dtype=torch.float32, device=dev)
-    dos = torch.empty(U * w.S * w.d, dtype=torch.float16, device=dev)
-    dqs, dks, dvs = (torch.empty(U * w.S * w.d, dtype=torch.float32, device=dev) for _ in range(3))
-    abw = lh.lh_attn_bwd_workspace_bytes(shp)
-    aws = torch.empty(abw, dtype=torch.uint8, device=dev)
-    stages = ["pyramid_score", "topk", "gather", "attn_fwd", "scatter", "scatter_bwd", "attn_bwd",
-              "gather_bwd"]
-    def staged(evs):
-        # identical launches to lh_forward + lh_backward, with events between stages
-        evs[0].record(stream)
-        lh.lh_build_pyramid_score(shp, dt, q, k, v, pq, pk, pv, score, sp)
-        evs[1].record(stream)
-        lh.lh_topk_select(shp, score, idx, pos, slot, None, 0, sp)
-        evs[2].record(stream)
-        lh.lh_gather(shp, dt, q, k, v, pq, pk, pv, idx, qs, ks, vs, sp)
-        evs[3].record(stream)
-        lh.lh_subseq_attn_fwd(shp, qs, ks, vs, 0.0, os_, lse, sp)
-        evs[4].record(stream)
-        lh.lh_scatter_back(shp, dt, os_, slot, o, ic, sp)
-        evs[5].record(stream)
-        lh.lh_scatter_back_bwd(shp, dt, dO, slot, ic, dos, sp)
-        evs[6].record(stream)
-        lh.lh_subseq_attn_bwd(shp, qs, ks, vs, os_, lse, dos, 0.0, dqs, dks, dvs, aws, abw, sp)
-        evs[7].record(stream)
-        lh.lh_gather_bwd(shp, dt, dqs, dks, dvs, slot, dq, dk, dv, sp)
-        evs[8].record(stream)
+    def step():
+        fwd_only()
+        if backward:
+            lh.lh_backward(shp, dt, saved, dO, 0.0, dq, dk, dv, ws, wsb, sp)
 
     def timed(fn, K):
         """Device time of K calls on this rank; the max over ranks is returned."""
@@ -260,70 +215,205 @@ def run_ours(args, rk):
         replicas.barrier(rk)
         return replicas.max_over_ranks(rk, ms, dev)
 
+    clk = ClockSampler(rk.local_rank) if clocks else None
     with torch.cuda.stream(stream):
-        for _ in range(args.warmup):
+        for _ in range(warmup):
             step()
         torch.cuda.synchronize()
         status = lh.lh_read_device_status(stream)
-        with ClockSampler(local_rank) as clk:
-            ms_total = timed(step, args.steps)
-        ms_step = ms_total / args.steps
-        ms_fwd = timed(fwd_only, args.steps) / args.steps
-        # per-stage durations over the same number of steps
+        if clk:
+            with clk:
+                ms_step = timed(step, steps) / steps
+        else:
+            ms_step = timed(step, steps) / steps
+        ms_fwd = timed(fwd_only, steps) / steps if backward else ms_step
+    torch.cuda.synchronize()
+    peak_bytes = torch.cuda.max_memory_allocated(dev) - mem0
+
+    # stage-by-stage replica of the same launches, for per-kernel durations
+    M, U = w.M, w.B * w.H
+    stages = STAGES_FWD + (STAGES_BWD if backward else [])
+
+    def view(which, dtype, n):
+        off = lh.lh_saved_offset(shp, which)
+        return saved[off:off + n * torch.tensor([], dtype=dtype).element_size()].view(dtype)
+
+    idx = view(lh.SAVED_IDX, torch.int32, U * w.S)
+    pos = view(lh.SAVED_POS, torch.int32, U * w.S)
+    slot = view(lh.SAVED_SLOT, torch.int32, U * M)
+    qs, ks, vs, os_ = (view(i, torch.float16, U * w.S * w.d)
+                       for i in (lh.SAVED_QS, lh.SAVED_KS, lh.SAVED_VS, lh.SAVED_OS))
+    lse = view(lh.SAVED_LSE, torch.float32, U * w.S)
+    ic = view(lh.SAVED_INV_COUNT, torch.float32, U * w.N)
+    npyr = max(U * (M - w.N) * w.d, 1)
+    pq, pk, pv = (torch.empty(npyr, dtype=torch.float32, device=dev) for _ in range(3))
+    score = torch.empty(U * M, dtype=torch.float32, device=dev)
+    if backward:
+        dos = torch.empty(U * w.S * w.d, dtype=torch.float16, device=dev)
+        dqs, dks, dvs = (torch.empty(U * w.S * w.d, dtype=torch.float32, device=dev) for _ in range(3))
+        abw = lh.lh_attn_bwd_workspace_bytes(shp)
+        aws = torch.empty(abw, dtype=torch.uint8, device=dev)
+
+    def staged(evs):
+        # identical launches to lh_forward (+ lh_backward), with events between stages
+        evs[0].record(stream)
+        lh.lh_build_pyramid_score(shp, dt, q, k, v, pq, pk, pv, score, sp)
+        evs[1].record(stream)
+        lh.lh_topk_select(shp, score, idx, pos, slot, None, 0, sp)
+        evs[2].record(stream)
+        lh.lh_gather(shp, dt, q, k, v, pq, pk, pv, idx, qs, ks, vs, sp)
+        evs[3].record(stream)
+        lh.lh_subseq_attn_fwd(shp, qs, ks, vs, 0.0, os_, lse, sp)
+        evs[4].record(stream)
+        lh.lh_scatter_back(shp, dt, os_, slot, o, ic, sp)
+        evs[5].record(stream)
+        if backward:
+            lh.lh_scatter_back_bwd(shp, dt, dO, slot, ic, dos, sp)
+            evs[6].record(stream)
+            lh.lh_subseq_attn_bwd(shp, qs, ks, vs, os_, lse, dos, 0.0, dqs, dks, dvs, aws, abw, sp)
+            evs[7].record(stream)
+            lh.lh_gather_bwd(shp, dt, dqs, dks, dvs, slot, dq, dk, dv, sp)
+            evs[8].record(stream)
+
+    with torch.cuda.stream(stream):
         evs_all = []
         torch.cuda.synchronize()
-        for _ in range(args.steps):
-            evs = [torch.cuda.Event(enable_timing=True) for _ in range(9)]
+        for _ in range(steps):
+            evs = [torch.cuda.Event(enable_timing=True) for _ in range(len(stages) + 1)]
             staged(evs)
             evs_all.append(evs)
         torch.cuda.synchronize()
-        stage_ms = {s: statistics.mean(e[i].elapsed_time(e[i + 1]) for e in evs_all)
-                    for i, s in enumerate(stages)}
+        stage_ms = {st: statistics.mean(e[i].elapsed_time(e[i + 1]) for e in evs_all)
+                    for i, st in enumerate(stages)}
         status |= lh.lh_read_device_status(stream)
 
-    tokens = w.B * w.N
-    value = replicas.job_rate(tokens, world, ms_step / 1e3)
     # rows the pooled gather must read: p^level for every selected entry
     gids = idx.view(U, w.S).long()
     offs = torch.tensor([sum(w.level_len(m) for m in range(l)) for l in range(w.L + 1)], device=dev)
     lev = torch.bucketize(gids, offs[1:], right=True)
     span_rows = int((torch.tensor(w.p, device=dev, dtype=torch.float64) ** lev).sum().item())
     alg = algorithmic(w, span_rows)
-    hbm = peaks["hbm_gbs"]
-    tc = peaks["bf16_tflops"]
-    stage_report = {}
-    for s in stages:
-        t = stage_ms[s] / 1e3
-        if s.startswith("attn"):
-            fl = alg[s + "_flop"]
-            stage_report[s] = {"ms": stage_ms[s], "tflops": fl / t / 1e12, "frac_tc": fl / t / 1e12 / tc}
+    hbm, tc = peaks["hbm_gbs"], peaks["bf16_tflops"]
+    traffic_key = w.name if w.H == WORKLOADS.get(w.name, w).H else ""
+    report = {}
+    for st in stages:
+        t = stage_ms[st] / 1e3
+        if st.startswith("attn"):
+            fl = alg[st + "_flop"]
+            report[st] = {"ms": stage_ms[st], "tflops": fl / t / 1e12, "frac_tc": fl / t / 1e12 / tc}
         else:
-            b = alg[s]
-            stage_report[s] = {"ms": stage_ms[s], "gbs": b / t / 1e9, "frac_hbm": b / t / 1e9 / hbm}
-        stage_report[s]["traffic"] = measured_traffic(w.name if not args.heads else "", s)
-    dominant = max(stages, key=lambda s: stage_ms[s])
+            bts = alg[st]
+            report[st] = {"ms": stage_ms[st], "gbs": bts / t / 1e9, "frac_hbm": bts / t / 1e9 / hbm}
+        report[st]["traffic"] = measured_traffic(traffic_key, st)
+    return {"ms_step": ms_step, "ms_fwd": ms_fwd, "stages": report, "status": status,
+            "peak_bytes": peak_bytes, "clk": clk, "traffic_key": traffic_key,
+            "tensors": {"x": x, "o": o, "dq": dq, "dk": dk, "dv": dv}, "shp": shp, "dt": dt,
+            "stream": stream}
+
+
+def roofline_of(report, peaks, peaks_src, traffic_key):
+    """The roofline object of the stage that takes the longest."""
+    dominant = max(report, key=lambda st: report[st]["ms"])
+    r = report[dominant]
     if dominant.startswith("attn"):
-        ach = stage_report[dominant]["tflops"]
-        roof = {"kernel": dominant, "bound": "tensor", "achieved": ach, "peak": tc,
-                "unit": "TFLOP/s", "frac": ach / tc,
-                "traffic": measured_traffic(w.name if not args.heads else "", dominant),
+        return {"kernel": dominant, "bound": "tensor", "achieved": r["tflops"],
+                "peak": peaks["bf16_tflops"], "unit": "TFLOP/s", "frac": r["frac_tc"],
+                "traffic": measured_traffic(traffic_key, dominant),
                 "peak_source": f"{peaks_src} bf16_tflops (burst)"}
-    else:
-        ach = stage_report[dominant]["gbs"]
-        roof = {"kernel": dominant, "bound": "hbm", "achieved": ach, "peak": hbm, "unit": "GB/s",
-                "frac": ach / hbm,
-                "traffic": measured_traffic(w.name if not args.heads else "", dominant),
-                "peak_source": f"{peaks_src} hbm_gbs"}
+    return {"kernel": dominant, "bound": "hbm", "achieved": r["gbs"], "peak": peaks["hbm_gbs"],
+            "unit": "GB/s", "frac": r["frac_hbm"], "traffic": measured_traffic(traffic_key, dominant),
+            "peak_source": f"{peaks_src} hbm_gbs"}
+
+
+def extra_leg(lh, name, args, rk, dev, peaks, peaks_src, dense=False):
+    """A further workload of the metric (the 512K and 1M contexts), measured the same
+    way with a few steps; reported beside the main line, not as its value."""
+    w = WORKLOADS[name]
+    m = measure(lh, w, args, rk, dev, peaks, steps=5, warmup=3)
+    tokens = w.B * w.N
+    leg = {"config": workload_config(w, rk.world, "tcgen05"),
+           "tokens_per_s": replicas.job_rate(tokens, rk.world, m["ms_step"] / 1e3),
+           "fwd_tokens_per_s": replicas.job_rate(tokens, rk.world, m["ms_fwd"] / 1e3),
+           "ms_per_step": m["ms_step"], "ms_fwd": m["ms_fwd"], "stages": m["stages"],
+           "roofline": roofline_of(m["stages"], peaks, peaks_src, m["traffic_key"]),
+           "peak_hbm_bytes": m["peak_bytes"], "device_status": m["status"]}
+    if dense:
+        t = m["tensors"]
+        leg["dense_sdpa"] = dense_sdpa(w, t["x"]["q"], t["x"]["k"], t["x"]["v"], t["x"]["dO"],
+                                       m["stream"], args, n=2)
+        if "fwd_ms" in leg["dense_sdpa"]:
+            leg["speedup_vs_dense"] = {"fwd": leg["dense_sdpa"]["fwd_ms"] / m["ms_fwd"],
+                                       "fwd_bwd": leg["dense_sdpa"]["fwd_bwd_ms"] / m["ms_step"]}
+    del m
+    torch.cuda.empty_cache()
+    return leg
+
+
+def run_sweep(args, rk):
+    """Forward-only per-stage times over the hyperparameter sweep (p, L, S) at the
+    pretraining shape; one JSON line."""
+    from long_context_lh_b200 import lighthouse as lh
+    from long_context_lh_b200.synth import sweep_workloads
+    dev = torch.device("cuda", rk.local_rank)
+    torch.cuda.set_device(dev)
+    peaks, peaks_src = load_peaks()
+    points = []
+    for w in sweep_workloads():
+        m = measure(lh, w, args, rk, dev, peaks, steps=max(1, min(args.steps, 10)),
+                    warmup=args.warmup, backward=False)
+        points.append({"p": w.p, "L": w.L, "S": w.S, "M": w.M, "ms_fwd": m["ms_fwd"],
+                       "fwd_tokens_per_s": w.B * w.N / (m["ms_fwd"] / 1e3),
+                       "stages_ms": {k: v["ms"] for k, v in m["stages"].items()},
+                       "attn_fwd_frac_tc": m["stages"]["attn_fwd"]["frac_tc"]})
+        del m
+        torch.cuda.empty_cache()
+    if rk.rank == 0:
+        print(json.dumps({"metric": METRIC, "sweep": points, "n_gpus": 1, "peaks_source": peaks_src,
+                          "config": {"workload": "sweep: B=1 H=16 N=98304 d=64 bf16, p x L x S"}}),
+              flush=True)
+
+
+def run_ours(args, rk):
+    from long_context_lh_b200 import lighthouse as lh
+
+    rank, world, local_rank = rk.rank, rk.world, rk.local_rank
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    w = WORKLOADS[args.workload]
+    if args.heads:
+        w = w.with_(H=args.heads)
+    if args.attn == "mma":
+        lh.lh_set_attention_impl(1)
+    elif args.attn == "tc":
+        lh.lh_set_attention_impl(0)
+    peaks, peaks_src = load_peaks()
+    m = measure(lh, w, args, rk, dev, peaks, steps=args.steps, warmup=args.warmup,
+                batch=rank, clocks=True)
+    ms_step, ms_fwd, stage_report, status = m["ms_step"], m["ms_fwd"], m["stages"], m["status"]
+    tokens = w.B * w.N
+    value = replicas.job_rate(tokens, world, ms_step / 1e3)
+    roof = roofline_of(stage_report, peaks, peaks_src, m["traffic_key"])
+    t = m["tensors"]
+    x = t["x"]
 
     # dense causal attention (torch SDPA, flash/cuDNN backend) on the same shapes
     dense = None
     if not args.no_dense and rank == 0:
-        dense = dense_sdpa(w, q, k, v, dO, stream, args)
+        dense = dense_sdpa(w, x["q"], x["k"], x["v"], x["dO"], m["stream"], args)
 
     # end to end through the public API with pinned host buffers
-    e2e = None if args.no_e2e else e2e_run(lh, w, shp, dt, x, dev, stream, args, rk,
-                                          {"o": o, "dq": dq, "dk": dk, "dv": dv})
+    e2e = None if args.no_e2e else e2e_run(lh, w, m["shp"], m["dt"], x, dev, m["stream"], args, rk,
+                                          {"o": t["o"], "dq": t["dq"], "dk": t["dk"], "dv": t["dv"]})
     launches = launches_per_step(lh, w)
+    clk = m["clk"]
+    del m, t, x
+    torch.cuda.empty_cache()
+    # the metric's other context lengths, on one GPU only (the scaling runs stay short)
+    extra = {}
+    if world == 1 and not args.heads and args.workload == "pretrain":
+        for name in [n for n in args.also.split(",") if n]:
+            extra[name] = extra_leg(lh, name, args, rk, dev, peaks, peaks_src,
+                                    dense=(name == "long" and not args.no_dense))
     out = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
@@ -337,6 +427,9 @@ def run_ours(args, rk):
         "gpu_launches": launches * args.steps, "gpu_launches_per_step": launches,
         "device_status": status, "peaks": peaks, "peaks_source": peaks_src,
     }
+    if dense and "fwd_ms" in dense:
+        out["speedup_vs_dense"] = {"fwd": dense["fwd_ms"] / ms_fwd, "fwd_bwd": dense["fwd_bwd_ms"] / ms_step}
+    out.update(extra)
     if rank == 0:
         out["clocks"] = clk.summary()
         if not args.no_cpu:
@@ -360,7 +453,7 @@ def launches_per_step(lh, w):
     return lh.lh_kernel_launches(shp, dt, False) + lh.lh_kernel_launches(shp, dt, True)
 
 
-def dense_sdpa(w, q, k, v, dO, stream, args):
+def dense_sdpa(w, q, k, v, dO, stream, args, n=None):
     import torch.nn.functional as F
     try:
         qd = q.detach().requires_grad_(True)
@@ -379,7 +472,7 @@ def dense_sdpa(w, q, k, v, dO, stream, args):
                     f()
                 fb()
             torch.cuda.synchronize()
-            n = max(1, min(args.steps, 5))
+            n = max(1, min(args.steps, 5)) if n is None else n
             e0, e1, e2 = (torch.cuda.Event(enable_timing=True) for _ in range(3))
             e0.record(stream)
             for _ in range(n):
@@ -531,6 +624,10 @@ def main():
     ap.add_argument("--heads", type=int, default=0,
                     help="override H (smaller cases for profiler captures; not a bench line)")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--also", default="long,extreme",
+                    help="further workloads measured beside the main line (1 GPU; '' for none)")
+    ap.add_argument("--sweep", action="store_true",
+                    help="forward-only per-stage times over the p x L x S sweep (one JSON line)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3) if args.impl == "ours" else args.warmup
     rk = replicas.from_env()
@@ -541,7 +638,10 @@ def main():
         torch.cuda.set_device(rk.local_rank)
     replicas.init(rk, "nccl", 300.0, torch.device("cuda", rk.local_rank) if rk.multi else None)
     try:
-        run_ours(args, rk)
+        if args.sweep:
+            run_sweep(args, rk)
+        else:
+            run_ours(args, rk)
     finally:
         replicas.finish(rk)
 
