@@ -40,23 +40,22 @@ PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 
 
 # DRAM bytes (read + written) per launch of each stage, from one ncu capture of
-# the pretraining workload with 4 heads (profiles/memory_kernels_pretrain_h4.md,
-# profiles/attn_tc_pretrain_h4.md), scaled by the units to the 16-head launch.
-# Each entry carries a hash of the sources its kernels are built from; when they
-# no longer match, the kernel has changed since the counters were taken and the
-# traffic is reported as null.  (At 4 heads part of each stage's writes is still
-# in L2 when it ends, so these undercount writes.)
-MEASURED_TRAFFIC = {  # workload: {stage: (bytes per full launch, sources, sha1[:16])}
+# the full-size pretraining workload (profiles/launches_pretrain.md: the launch
+# list with dram__bytes_read.sum and dram__bytes_write.sum, one pass).  Each entry
+# carries a hash of the sources its kernels are built from; when they no longer
+# match, the kernel has changed since the counters were taken and the traffic is
+# reported as null.  Writes still in L2 when a kernel ends are counted by the
+# kernel that evicts them, so a stage that writes more than L2 holds reads low.
+MEASURED_TRAFFIC = {  # workload: {stage: (bytes per launch, sources, sha1[:16])}
     "pretrain": {
-        "pyramid_score": (8.602e+08, ("k_pyramid.cu", "lh_internal.cuh"), "64fedac8a3e613a7"),
-        "topk": (8.649e+06, ("k_topk.cu", "lh_internal.cuh"), "c32ba6e137685eea"),
-        "gather": (8.584e+07, ("k_gather_scatter.cu", "lh_internal.cuh"), "06de88f37c7464d1"),
-        "scatter": (3.217e+07, ("k_gather_scatter.cu", "lh_internal.cuh"), "06de88f37c7464d1"),
-        "scatter_bwd": (2.167e+08, ("k_gather_scatter.cu", "lh_internal.cuh"), "06de88f37c7464d1"),
-        "gather_bwd": (4.798e+08, ("k_gather_scatter.cu", "lh_internal.cuh"), "06de88f37c7464d1"),
-        "attn_fwd": (5.051e+07, ("k_attn_tc.cu", "tc_common.cuh"), "bd8b1f0925e92946"),
-        "attn_bwd": (1.708e+08, ("k_attn_tc.cu", "tc_common.cuh", "k_gather_scatter.cu",
-                                 "lh_internal.cuh"), "70788de6cb32b83f"),
+        "pyramid_score": (9.6660e+08, ('k_pyramid.cu', 'lh_internal.cuh'), "0fe10c5f7c160b21"),
+        "topk": (8.4000e+06, ('k_topk.cu', 'lh_internal.cuh'), "956b5193a7a7a1b3"),
+        "gather": (9.6400e+07, ('k_gather_scatter.cu', 'lh_internal.cuh'), "a9918a7354a15cac"),
+        "scatter": (1.7010e+08, ('k_gather_scatter.cu', 'lh_internal.cuh'), "a9918a7354a15cac"),
+        "scatter_bwd": (2.2560e+08, ('k_gather_scatter.cu', 'lh_internal.cuh'), "a9918a7354a15cac"),
+        "gather_bwd": (6.5040e+08, ('k_gather_scatter.cu', 'lh_internal.cuh'), "a9918a7354a15cac"),
+        "attn_fwd": (5.0500e+07, ('k_attn_tc.cu', 'tc_common.cuh'), "aec417ec05129960"),
+        "attn_bwd": (1.9450e+08, ('k_attn_tc.cu', 'tc_common.cuh', 'k_gather_scatter.cu', 'lh_internal.cuh'), "c1ad5e42a553ab4f"),
     },
 }
 
