@@ -249,6 +249,52 @@ int lh_attention_impl_in_use(void);
  * implementation; -1 for an invalid shape or dtype. */
 int lh_kernel_launches(const lh_shape* shape, lh_dtype dtype, int backward);
 
+/* -------------------------------------------------------------- variants */
+
+/* How the two level-0 norms of an entry combine into its score.  The pages fix
+ * that each entry is scored, without parameters, by the l2 norms of its
+ * projected Q and K vectors ([ES] §2.B; [PT] phase 2: two scores per entry),
+ * not how the two combine: the sum is the default reading, the product and the
+ * norm of the concatenation are ablations of that reading.  All in fp32 from the
+ * two squared norms ss(q), ss(k) of lh_score:
+ *   SUM     sqrt(ss(q)) + sqrt(ss(k))
+ *   PRODUCT sqrt(ss(q)) * sqrt(ss(k))
+ *   CONCAT  sqrt(ss(q) + ss(k))        (IEEE sqrt, one rounding per operation) */
+typedef enum { LH_SCORE_SUM = 0, LH_SCORE_PRODUCT = 1, LH_SCORE_CONCAT = 2 } lh_score_mode;
+
+/* Variants of the layer.  A NULL pointer, or all fields 0, is the default layer
+ * the entry points above compute.
+ *   keep_coarsest: 1 = every entry of the coarsest level L-1 is selected, which
+ *     gives every original position at least one contributor ([PT] phase 1);
+ *     the coarsest entries rank above every score (key bits of +inf; among
+ *     themselves by gid), the other S - N/p^(L-1) slots go to the largest keys
+ *     as usual.  Needs N / p^(L-1) <= S, else LH_ERR_SHAPE.
+ *   score_mode: an lh_score_mode.
+ *   reserved: must be 0 (LH_ERR_INVALID_ARG otherwise).                      */
+typedef struct {
+  int32_t keep_coarsest;
+  int32_t score_mode;
+  int32_t reserved[2];
+} lh_options;
+
+/* Host-only check of a shape and options (NULL allowed); no CUDA call. */
+lh_status lh_validate_options(const lh_shape* shape, const lh_options* opt);
+
+/* The stage and fused calls that the options change, with the options; the
+ * calls without _ex above are these with opt = NULL.  The backward does not
+ * depend on them (it reads the selection that lh_forward_ex saved).          */
+lh_status lh_build_pyramid_score_ex(const lh_shape* shape, lh_dtype dtype, const void* q,
+                                    const void* k, const void* v, float* pq, float* pk, float* pv,
+                                    float* score, const lh_options* opt, lh_stream_t stream);
+lh_status lh_score_ex(const lh_shape* shape, lh_dtype dtype, const void* q, const void* k,
+                      float* score, const lh_options* opt, lh_stream_t stream);
+lh_status lh_topk_select_ex(const lh_shape* shape, const float* score, int32_t* idx,
+                            int32_t* pos, int32_t* slot, void* ws, size_t ws_bytes,
+                            const lh_options* opt, lh_stream_t stream);
+lh_status lh_forward_ex(const lh_shape* shape, lh_dtype dtype, const void* q, const void* k,
+                        const void* v, float scale, void* o, void* saved, void* ws,
+                        size_t ws_bytes, const lh_options* opt, lh_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -26,7 +26,8 @@
 //
 // Arithmetic (fixed, so the selection is reproducible bit for bit):
 //   score:  a_c = fmaf chain over x[8c+0..7]^2 from 0; tree over c with offsets
-//           1, 2, 4(, 8); score = sqrt_rn(ss(Q)) + sqrt_rn(ss(K));
+//           1, 2, 4(, 8); score = sqrt_rn(ss(Q)) + sqrt_rn(ss(K)) (the default;
+//           the ablations: their product, or sqrt_rn(ss(Q) + ss(K)));
 //           coarse score = max(0, children in order) (scores are >= 0);
 //   mean:   ((0 + c_0) + c_1) + ... + c_{p-1}, then / p (round to nearest; for
 //           p a power of two the product with 1/p, which is the same number).
@@ -46,12 +47,21 @@ inline int chunk_rows_cap(int d, size_t elem) {
 
 struct PyrPrm {
   int32_t N, M, CR, p, J, L;
+  int32_t score_mode;  // lh_score_mode
   int32_t pow2;  // p is a power of two: mean = sum * inv_p exactly
   float inv_p;
   double inv_pd;  // 1/p in fp64 for the exact division (div_exact) otherwise
   int32_t off[kMaxLevels + 1];
   int32_t pw[kMaxLevels + 1];
 };
+
+// Level-0 score from the squared norms of the token's q and k rows: their norms'
+// sum (default), product, or the norm of the concatenation [q; k].
+__device__ __forceinline__ float combine_norms(float ssq, float ssk, int mode) {
+  if (mode == LH_SCORE_PRODUCT) return __fmul_rn(__fsqrt_rn(ssq), __fsqrt_rn(ssk));
+  if (mode == LH_SCORE_CONCAT) return __fsqrt_rn(__fadd_rn(ssq, ssk));
+  return __fadd_rn(__fsqrt_rn(ssq), __fsqrt_rn(ssk));
+}
 
 template <int P>
 __device__ __forceinline__ float mean_of(float sum, const PyrPrm& prm) {
@@ -174,7 +184,7 @@ __global__ void __launch_bounds__(256) k_pyr_chunk(
         ssq = __fadd_rn(ssq, __shfl_xor_sync(gmask, ssq, off));
         ssk = __fadd_rn(ssk, __shfl_xor_sync(gmask, ssk, off));
       }
-      if (c == 0) sSc[r] = __fadd_rn(__fsqrt_rn(ssq), __fsqrt_rn(ssk));
+      if (c == 0) sSc[r] = combine_norms(ssq, ssk, prm.score_mode);
     }
     __syncthreads();
     for (int r = tid; r < rows; r += 256) sc[t0 + r] = sSc[r];
@@ -244,7 +254,7 @@ __global__ void __launch_bounds__(256) k_pyr_chunk(
               a[c] = __fadd_rn(a[c], a[c + off]);
               b[c] = __fadd_rn(b[c], b[c + off]);
             }
-          const float s0 = __fadd_rn(__fsqrt_rn(a[0]), __fsqrt_rn(b[0]));
+          const float s0 = combine_norms(a[0], b[0], prm.score_mode);
           sSc[r] = s0;
           sc[t0 + r] = s0;
         }
@@ -315,6 +325,7 @@ PyrPrm make_prm(const Geom& g, int cap) {
   prm.M = (int32_t)g.M;
   prm.p = g.p;
   prm.L = g.L;
+  prm.score_mode = g.score_mode;
   prm.pow2 = (g.p & (g.p - 1)) == 0;
   prm.inv_p = 1.0f / (float)g.p;  // exact when p is a power of two
   prm.inv_pd = 1.0 / (double)g.p;

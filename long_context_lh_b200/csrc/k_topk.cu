@@ -42,10 +42,14 @@ constexpr int kWarps = kThreads / 32;
 constexpr int kBins = 2048;
 // Shared memory for a CTA's cached keys (the static part holds the histograms).
 constexpr int64_t kKeyCacheBytes = 180 * 1024;
+// Key bits of a kept coarsest entry: +inf, above every finite score; ties among
+// kept entries go to the lower gid like any other tie.
+constexpr uint32_t kTopBits = 0x7F800000u;
 
 struct TopkParams {
   int32_t N, M;  // within-unit sizes fit 32 bits (M < 2^31 is a checked limit)
   int p, L, S, log2p;
+  int keep_top;  // level L-1 ranks as +inf (keep-coarsest-level variant)
   int64_t unit0;
   int32_t off[kMaxLevels + 1];
   int32_t pw[kMaxLevels + 1];
@@ -200,12 +204,15 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
     for (int l = 0; l < kMaxLevels; ++l) {
       const uint32_t* src = key + prm.off[l] + jb[l];
+      const bool top = prm.keep_top && l == prm.L - 1;
 #pragma unroll 4
-      for (int32_t j = threadIdx.x; j < nl[l]; j += kThreads) skey[kb[l] + j] = __ldg(src + j);
+      for (int32_t j = threadIdx.x; j < nl[l]; j += kThreads)
+        skey[kb[l] + j] = top ? kTopBits : __ldg(src + j);
     }
   }
   auto key_of = [&](int l, int32_t j) -> uint32_t {  // j: index within the CTA's level-l range
-    return cached ? skey[kb[l] + j] : __ldg(key + prm.off[l] + jb[l] + j);
+    if (cached) return skey[kb[l] + j];
+    return (prm.keep_top && l == prm.L - 1) ? kTopBits : __ldg(key + prm.off[l] + jb[l] + j);
   };
 
   cluster.sync();  // every CTA is running (DSMEM) and its keys are in place
@@ -371,6 +378,7 @@ cudaError_t launch_topk(const Geom& g, const float* score, int32_t* idx, int32_t
   prm.L = g.L;
   prm.S = g.S;
   prm.log2p = ((g.p & (g.p - 1)) == 0) ? __builtin_ctz((unsigned)g.p) : -1;
+  prm.keep_top = g.keep_top;
   for (int l = 0; l <= kMaxLevels; ++l) {
     prm.off[l] = (int32_t)g.off[l];
     prm.pw[l] = (int32_t)(g.pw[l] > 0x7fffffff ? 0x7fffffff : g.pw[l]);

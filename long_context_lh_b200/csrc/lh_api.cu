@@ -148,6 +148,16 @@ lh_status attn_bwd(const Geom& g, const __half* qs, const __half* ks,
   return cuda_status(launch_attn_bwd_mma(g, qs, ks, vs, dos, stats, scale, dqs, dks, dvs, st));
 }
 
+// The geometry of a shape with the variant options applied (options validated).
+Geom geom_with(const lh_shape& shape, const lh_options* opt) {
+  Geom g = make_geom(shape);
+  if (opt) {
+    g.score_mode = opt->score_mode;
+    g.keep_top = opt->keep_coarsest;
+  }
+  return g;
+}
+
 }  // namespace
 }  // namespace lh
 
@@ -208,6 +218,20 @@ size_t lh_attn_bwd_workspace_bytes(const lh_shape* shape) {
   return align_up(attn_stats_floats(g) * 4);
 }
 
+lh_status lh_validate_options(const lh_shape* shape, const lh_options* opt) {
+  lh_status s = check_shape(shape);
+  if (s != LH_OK) return s;
+  if (opt == nullptr) return LH_OK;
+  if (opt->reserved[0] != 0 || opt->reserved[1] != 0) return LH_ERR_INVALID_ARG;
+  if (opt->score_mode < LH_SCORE_SUM || opt->score_mode > LH_SCORE_CONCAT) return LH_ERR_INVALID_ARG;
+  if (opt->keep_coarsest != 0 && opt->keep_coarsest != 1) return LH_ERR_INVALID_ARG;
+  if (opt->keep_coarsest) {
+    const Geom g = make_geom(*shape);
+    if (g.N / g.pw[g.L - 1] > g.S) return LH_ERR_SHAPE;  // the coarsest level alone exceeds S
+  }
+  return LH_OK;
+}
+
 lh_status lh_build_pyramid(const lh_shape* shape, lh_dtype dtype, const void* q, const void* k,
                            const void* v, float* pq, float* pk, float* pv, lh_stream_t stream) {
   lh_status s = lh_validate(shape, dtype);
@@ -219,39 +243,59 @@ lh_status lh_build_pyramid(const lh_shape* shape, lh_dtype dtype, const void* q,
   return cuda_status(launch_pyramid_score(g, dtype, q, k, v, pq, pk, pv, nullptr, stream));
 }
 
-lh_status lh_build_pyramid_score(const lh_shape* shape, lh_dtype dtype, const void* q,
-                                 const void* k, const void* v, float* pq, float* pk, float* pv,
-                                 float* score, lh_stream_t stream) {
+lh_status lh_build_pyramid_score_ex(const lh_shape* shape, lh_dtype dtype, const void* q,
+                                    const void* k, const void* v, float* pq, float* pk, float* pv,
+                                    float* score, const lh_options* opt, lh_stream_t stream) {
   lh_status s = lh_validate(shape, dtype);
   if (s != LH_OK) return s;
+  if ((s = lh_validate_options(shape, opt)) != LH_OK) return s;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(score))
     return LH_ERR_INVALID_ARG;
   if (shape->L > 1 && (!aligned16(pq) || !aligned16(pk) || !aligned16(pv)))
     return LH_ERR_INVALID_ARG;
-  const Geom g = make_geom(*shape);
+  const Geom g = geom_with(*shape, opt);
   if (g.L == 1) pq = pk = pv = nullptr;
   return cuda_status(launch_pyramid_score(g, dtype, q, k, v, pq, pk, pv, score, stream));
 }
 
-lh_status lh_score(const lh_shape* shape, lh_dtype dtype, const void* q, const void* k,
-                   float* score, lh_stream_t stream) {
+lh_status lh_build_pyramid_score(const lh_shape* shape, lh_dtype dtype, const void* q,
+                                 const void* k, const void* v, float* pq, float* pk, float* pv,
+                                 float* score, lh_stream_t stream) {
+  return lh_build_pyramid_score_ex(shape, dtype, q, k, v, pq, pk, pv, score, nullptr, stream);
+}
+
+lh_status lh_score_ex(const lh_shape* shape, lh_dtype dtype, const void* q, const void* k,
+                      float* score, const lh_options* opt, lh_stream_t stream) {
   lh_status s = lh_validate(shape, dtype);
   if (s != LH_OK) return s;
+  if ((s = lh_validate_options(shape, opt)) != LH_OK) return s;
   if (!aligned16(q) || !aligned16(k) || !aligned16(score)) return LH_ERR_INVALID_ARG;
-  const Geom g = make_geom(*shape);
+  const Geom g = geom_with(*shape, opt);
   return cuda_status(
       launch_pyramid_score(g, dtype, q, k, nullptr, nullptr, nullptr, nullptr, score, stream));
 }
 
-lh_status lh_topk_select(const lh_shape* shape, const float* score, int32_t* idx, int32_t* pos,
-                         int32_t* slot, void* ws, size_t ws_bytes, lh_stream_t stream) {
+lh_status lh_score(const lh_shape* shape, lh_dtype dtype, const void* q, const void* k,
+                   float* score, lh_stream_t stream) {
+  return lh_score_ex(shape, dtype, q, k, score, nullptr, stream);
+}
+
+lh_status lh_topk_select_ex(const lh_shape* shape, const float* score, int32_t* idx,
+                            int32_t* pos, int32_t* slot, void* ws, size_t ws_bytes,
+                            const lh_options* opt, lh_stream_t stream) {
   (void)ws;
   (void)ws_bytes;
   lh_status s = check_shape(shape);
   if (s != LH_OK) return s;
+  if ((s = lh_validate_options(shape, opt)) != LH_OK) return s;
   if (!aligned16(score) || !aligned16(idx) || !aligned16(pos) || !aligned16(slot))
     return LH_ERR_INVALID_ARG;
-  return cuda_status(launch_topk(make_geom(*shape), score, idx, pos, slot, stream));
+  return cuda_status(launch_topk(geom_with(*shape, opt), score, idx, pos, slot, stream));
+}
+
+lh_status lh_topk_select(const lh_shape* shape, const float* score, int32_t* idx, int32_t* pos,
+                         int32_t* slot, void* ws, size_t ws_bytes, lh_stream_t stream) {
+  return lh_topk_select_ex(shape, score, idx, pos, slot, ws, ws_bytes, nullptr, stream);
 }
 
 lh_status lh_gather(const lh_shape* shape, lh_dtype dtype, const void* q, const void* k,
@@ -351,13 +395,20 @@ lh_status lh_gather_bwd(const lh_shape* shape, lh_dtype dtype, const float* dqs,
 lh_status lh_forward(const lh_shape* shape, lh_dtype dtype, const void* q, const void* k,
                      const void* v, float scale, void* o, void* saved, void* ws,
                      size_t ws_bytes, lh_stream_t stream) {
+  return lh_forward_ex(shape, dtype, q, k, v, scale, o, saved, ws, ws_bytes, nullptr, stream);
+}
+
+lh_status lh_forward_ex(const lh_shape* shape, lh_dtype dtype, const void* q, const void* k,
+                        const void* v, float scale, void* o, void* saved, void* ws,
+                        size_t ws_bytes, const lh_options* opt, lh_stream_t stream) {
   lh_status s = lh_validate(shape, dtype);
   if (s != LH_OK) return s;
+  if ((s = lh_validate_options(shape, opt)) != LH_OK) return s;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(saved) ||
       !aligned16(ws))
     return LH_ERR_INVALID_ARG;
   if (ws_bytes < lh_workspace_bytes(shape, dtype, 0)) return LH_ERR_WORKSPACE;
-  const Geom g = make_geom(*shape);
+  const Geom g = geom_with(*shape, opt);
   const Layout sl = saved_layout(g), wl = fwd_ws_layout(g);
   char* sv = static_cast<char*>(saved);
   char* w = static_cast<char*>(ws);

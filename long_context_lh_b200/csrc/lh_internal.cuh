@@ -22,6 +22,8 @@ struct Geom {
   int d, p, L, S;
   int64_t pw[kMaxLevels + 1];   // p^l
   int64_t off[kMaxLevels + 1];  // first gid of level l; off[L] = M
+  int score_mode = 0;           // lh_score_mode
+  int keep_top = 0;             // keep every level-(L-1) entry (lh_options.keep_coarsest)
 };
 
 Geom make_geom(const lh_shape& s);

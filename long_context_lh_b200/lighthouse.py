@@ -48,6 +48,26 @@ def make_shape(B, H, N, d, p, L, S) -> Shape:
     return Shape(int(B), int(H), int(N), int(d), int(p), int(L), int(S))
 
 
+LH_SCORE_SUM, LH_SCORE_PRODUCT, LH_SCORE_CONCAT = 0, 1, 2
+
+
+class Options(ctypes.Structure):
+    """lh_options: layer variants (keep-coarsest-level, score ablations)."""
+    _fields_ = [("keep_coarsest", ctypes.c_int32), ("score_mode", ctypes.c_int32),
+                ("reserved", ctypes.c_int32 * 2)]
+
+
+def make_options(keep_coarsest=False, score_mode=LH_SCORE_SUM) -> Options:
+    o = Options()
+    o.keep_coarsest = 1 if keep_coarsest else 0
+    o.score_mode = int(score_mode)
+    return o
+
+
+def _opt(options):
+    return None if options is None else ctypes.byref(options)
+
+
 _VP = ctypes.c_void_p
 _SP = ctypes.POINTER(Shape)
 _I, _F, _SZ, _I64 = ctypes.c_int, ctypes.c_float, ctypes.c_size_t, ctypes.c_int64
@@ -78,6 +98,11 @@ _SIGS = {
     "lh_backward": ([_SP, _I, _VP, _VP, _F, _VP, _VP, _VP, _VP, _SZ, _VP], _I),
     "lh_read_device_status": ([_VP, ctypes.POINTER(ctypes.c_uint32)], _I),
     "lh_set_attention_impl": ([_I], _I),
+    "lh_validate_options": ([_SP, _VP], _I),
+    "lh_build_pyramid_score_ex": ([_SP, _I, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP], _I),
+    "lh_score_ex": ([_SP, _I, _VP, _VP, _VP, _VP, _VP], _I),
+    "lh_topk_select_ex": ([_SP, _VP, _VP, _VP, _VP, _VP, _SZ, _VP, _VP], _I),
+    "lh_forward_ex": ([_SP, _I, _VP, _VP, _VP, _F, _VP, _VP, _VP, _SZ, _VP, _VP], _I),
     "lh_attention_impl_in_use": ([], _I),
     "lh_kernel_launches": ([_SP, _I, _I], _I),
 }
@@ -198,6 +223,33 @@ def lh_build_pyramid_score(shape, dtype, q, k, v, pq, pk, pv, score, stream=None
         _st(stream)))
 
 
+def lh_validate_options(shape, options):
+    return _lib().lh_validate_options(ctypes.byref(shape), _opt(options))
+
+
+def lh_build_pyramid_score_ex(shape, dtype, q, k, v, pq, pk, pv, score, options, stream=None):
+    _check("lh_build_pyramid_score_ex", _lib().lh_build_pyramid_score_ex(
+        ctypes.byref(shape), dtype, _p(q), _p(k), _p(v), _p(pq), _p(pk), _p(pv), _p(score),
+        _opt(options), _st(stream)))
+
+
+def lh_score_ex(shape, dtype, q, k, score, options, stream=None):
+    _check("lh_score_ex", _lib().lh_score_ex(ctypes.byref(shape), dtype, _p(q), _p(k), _p(score),
+                                             _opt(options), _st(stream)))
+
+
+def lh_topk_select_ex(shape, score, idx, pos, slot, options, ws=None, ws_bytes=0, stream=None):
+    _check("lh_topk_select_ex", _lib().lh_topk_select_ex(
+        ctypes.byref(shape), _p(score), _p(idx), _p(pos), _p(slot), _p(ws), ws_bytes,
+        _opt(options), _st(stream)))
+
+
+def lh_forward_ex(shape, dtype, q, k, v, scale, o, saved, ws, ws_bytes, options, stream=None):
+    _check("lh_forward_ex", _lib().lh_forward_ex(
+        ctypes.byref(shape), dtype, _p(q), _p(k), _p(v), float(scale), _p(o), _p(saved), _p(ws),
+        ws_bytes, _opt(options), _st(stream)))
+
+
 def lh_score(shape, dtype, q, k, score, stream=None):
     _check("lh_score", _lib().lh_score(ctypes.byref(shape), dtype, _p(q), _p(k), _p(score),
                                        _st(stream)))
@@ -300,17 +352,22 @@ class Saved:
     buf: torch.Tensor
 
 
-def forward(q, k, v, p: int, L: int, S: int, scale: float = 0.0, stream=None):
-    """o, Saved = forward(q, k, v, p, L, S): whole layer through lh_forward."""
+def forward(q, k, v, p: int, L: int, S: int, scale: float = 0.0, stream=None, options=None):
+    """o, Saved = forward(q, k, v, p, L, S): whole layer through lh_forward
+    (lh_forward_ex when `options`, an Options, is given)."""
     B, H, N, d = q.shape
     shp = make_shape(B, H, N, d, p, L, S)
     dt = dtype_code(q.dtype)
     _check("lh_validate", lh_validate(shp, dt))
+    _check("lh_validate_options", lh_validate_options(shp, options))
     o = torch.empty_like(q)
     saved = torch.empty(lh_saved_bytes(shp), dtype=torch.uint8, device=q.device)
     wsb = lh_workspace_bytes(shp, dt, False)
     ws = torch.empty(max(wsb, 256), dtype=torch.uint8, device=q.device)
-    lh_forward(shp, dt, q, k, v, scale, o, saved, ws, wsb, stream)
+    if options is None:
+        lh_forward(shp, dt, q, k, v, scale, o, saved, ws, wsb, stream)
+    else:
+        lh_forward_ex(shp, dt, q, k, v, scale, o, saved, ws, wsb, options, stream)
     return o, Saved(shp, dt, scale, saved)
 
 

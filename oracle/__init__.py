@@ -98,6 +98,8 @@ def _L():
             "lho_pyramid": ([sp, P, P, i], None),
             "lho_score": ([sp, P, P, P, i], None),
             "lho_select": ([sp, P, P, P, P, i], None),
+            "lho_score_mode": ([sp, P, P, P, i, i], None),
+            "lho_select_opt": ([sp, P, P, P, P, i, i], None),
             "lho_gather": ([sp, P, P, P, P], None),
             "lho_attn_fwd": ([sp, P, P, P, d, P, i64, P, P, i], None),
             "lho_attn_bwd": ([sp, P, P, P, P, d, P, P, P, i], None),
@@ -146,24 +148,30 @@ def pyramid(s: Shape, x, nthreads=None) -> np.ndarray:
     return out.reshape(s.B, s.H, s.M - s.N, s.d)
 
 
-def score(s: Shape, q, k, nthreads=None) -> np.ndarray:
-    """fp32 scores of all M entries [B,H,M] (norm sum at level 0, max-pool above)."""
+SCORE_SUM, SCORE_PRODUCT, SCORE_CONCAT = 0, 1, 2  # how the two level-0 norms combine
+
+
+def score(s: Shape, q, k, nthreads=None, mode=SCORE_SUM) -> np.ndarray:
+    """fp32 scores of all M entries [B,H,M] (at level 0 the norm sum, or the
+    ablations: norm product, norm of [q; k]; max-pool above)."""
     q = _f32(q).reshape(s.U, s.N, s.d)
     k = _f32(k).reshape(s.U, s.N, s.d)
     out = np.zeros((s.U, s.M), np.float32)
-    _L().lho_score(ctypes.byref(s.c()), _p(q), _p(k), _p(out), _threads(nthreads))
+    _L().lho_score_mode(ctypes.byref(s.c()), _p(q), _p(k), _p(out), int(mode), _threads(nthreads))
     return out.reshape(s.B, s.H, s.M)
 
 
-def select(s: Shape, sc, nthreads=None):
-    """Joint top-S by (score desc, gid asc), ordered by (pos asc, level asc).
+def select(s: Shape, sc, nthreads=None, keep_coarsest=False):
+    """Joint top-S by (score desc, gid asc), ordered by (pos asc, level asc);
+    keep_coarsest ranks every level-(L-1) entry above every score.
 
     Returns idx [B,H,S] (gid), pos [B,H,S], slot [B,H,M] (slot or -1)."""
     sc = _f32(sc).reshape(s.U, s.M)
     idx = np.zeros((s.U, s.S), np.int32)
     pos = np.zeros((s.U, s.S), np.int32)
     slot = np.zeros((s.U, s.M), np.int32)
-    _L().lho_select(ctypes.byref(s.c()), _p(sc), _p(idx), _p(pos), _p(slot), _threads(nthreads))
+    _L().lho_select_opt(ctypes.byref(s.c()), _p(sc), _p(idx), _p(pos), _p(slot),
+                        1 if keep_coarsest else 0, _threads(nthreads))
     return (idx.reshape(s.B, s.H, s.S), pos.reshape(s.B, s.H, s.S),
             slot.reshape(s.B, s.H, s.M))
 
@@ -277,12 +285,13 @@ def default_scale(s: Shape, scale=None) -> float:
     return 1.0 / float(np.sqrt(s.d)) if (scale is None or scale <= 0) else float(scale)
 
 
-def forward(s: Shape, q, k, v, scale=None, nthreads=None) -> dict:
+def forward(s: Shape, q, k, v, scale=None, nthreads=None, score_mode=SCORE_SUM,
+            keep_coarsest=False) -> dict:
     """The whole forward; returns every intermediate (fp64 except score)."""
     scale = default_scale(s, scale)
     pq, pk, pv = (pyramid(s, x, nthreads) for x in (q, k, v))
-    sc = score(s, q, k, nthreads)
-    idx, pos, slot = select(s, sc, nthreads)
+    sc = score(s, q, k, nthreads, mode=score_mode)
+    idx, pos, slot = select(s, sc, nthreads, keep_coarsest=keep_coarsest)
     qs, ks, vs = gather(s, q, pq, idx), gather(s, k, pk, idx), gather(s, v, pv, idx)
     os_, lse = attn_fwd(s, qs, ks, vs, scale, nthreads=nthreads)
     o = scatter(s, os_, slot)

@@ -180,6 +180,7 @@ typedef struct {
   const lho_shape* s;
   const float *q, *k;
   float* score;
+  int mode; /* 0 sum of the norms (default), 1 their product, 2 norm of [q; k] */
 } score_ctx;
 
 static void score_unit(void* vctx, int64_t u) {
@@ -191,9 +192,14 @@ static void score_unit(void* vctx, int64_t u) {
   const float* k = c->k + u * N * d;
   float* sc = c->score + u * M;
   for (int64_t t = 0; t < N; ++t) {
-    float nq = sqrtf(ss_canonical(q + t * d, d));
-    float nk = sqrtf(ss_canonical(k + t * d, d));
-    sc[t] = nq + nk;
+    float sq = ss_canonical(q + t * d, d);
+    float sk = ss_canonical(k + t * d, d);
+    if (c->mode == 1)
+      sc[t] = sqrtf(sq) * sqrtf(sk);
+    else if (c->mode == 2)
+      sc[t] = sqrtf(sq + sk);
+    else
+      sc[t] = sqrtf(sq) + sqrtf(sk);
   }
   for (int l = 1; l < s->L; ++l) {
     int64_t nl = level_len(s, l), o = level_off(s, l), oc = level_off(s, l - 1);
@@ -208,9 +214,17 @@ static void score_unit(void* vctx, int64_t u) {
   }
 }
 
-void lho_score(const lho_shape* s, const float* q, const float* k, float* score, int nthreads) {
-  score_ctx c = {s, q, k, score};
+/* Ablations of the reading above (how the two norms combine), same fp32 order
+ * for the squared norms: mode 1 = sqrtf(ss(q)) * sqrtf(ss(k)), mode 2 =
+ * sqrtf(ss(q) + ss(k)), the norm of the concatenated vector [q; k].          */
+void lho_score_mode(const lho_shape* s, const float* q, const float* k, float* score, int mode,
+                    int nthreads) {
+  score_ctx c = {s, q, k, score, mode};
   lho_parallel_for(s->B * s->H, nthreads, score_unit, &c);
+}
+
+void lho_score(const lho_shape* s, const float* q, const float* k, float* score, int nthreads) {
+  lho_score_mode(s, q, k, score, 0, nthreads);
 }
 
 /* ------------------------------------------- c.5/c.6 joint top-K + order
@@ -248,6 +262,7 @@ typedef struct {
   const lho_shape* s;
   const float* score;
   int32_t *idx, *pos, *slot;
+  int keep_coarsest;
 } sel_ctx;
 
 static void select_unit(void* vctx, int64_t u) {
@@ -260,7 +275,9 @@ static void select_unit(void* vctx, int64_t u) {
   for (int64_t g = 0; g < M; ++g) {
     int l = gid_level(s, g);
     int64_t j = g - level_off(s, l);
-    items[g].score = sc[g];
+    /* keep-coarsest-level variant ([PT] phase 1: the coarsest level keeps a
+     * contributor for every position): its entries rank above every score */
+    items[g].score = (c->keep_coarsest && l == s->L - 1) ? INFINITY : sc[g];
     items[g].gid = g;
     items[g].level = l;
     items[g].pos = (j + 1) * ipow(s->p, l) - 1;
@@ -277,10 +294,15 @@ static void select_unit(void* vctx, int64_t u) {
   free(items);
 }
 
+void lho_select_opt(const lho_shape* s, const float* score, int32_t* idx, int32_t* pos,
+                    int32_t* slot, int keep_coarsest, int nthreads) {
+  sel_ctx c = {s, score, idx, pos, slot, keep_coarsest};
+  lho_parallel_for(s->B * s->H, nthreads, select_unit, &c);
+}
+
 void lho_select(const lho_shape* s, const float* score, int32_t* idx, int32_t* pos, int32_t* slot,
                 int nthreads) {
-  sel_ctx c = {s, score, idx, pos, slot};
-  lho_parallel_for(s->B * s->H, nthreads, select_unit, &c);
+  lho_select_opt(s, score, idx, pos, slot, 0, nthreads);
 }
 
 /* ------------------------------------------------------------ c.7 gather

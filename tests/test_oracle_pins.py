@@ -354,3 +354,66 @@ def test_attention_bwd_sampled_matches_full_backward_and_autograd(S, chunk):
     out.backward(torch.tensor(do))
     for got, t in ((dq, tq), (dk, tk), (dv, tv)):
         np.testing.assert_allclose(got, t.grad.numpy()[rows], rtol=1e-10, atol=1e-12)
+
+
+# --------------------------------------------------- variants (ablations, keep-coarsest)
+@pytest.mark.parametrize("d", [64, 128, 8])
+def test_score_modes_close_to_fp64_closed_forms(d):
+    """The product of the two norms and the norm of [q; k] agree with exact fp64
+    values to a few ulp, and coarse levels still inherit the exact span max."""
+    s = Shape(1, 2, 256, d, 4, 3, 16)
+    q, k, _ = rand_qkv(s, 3.0, True)
+    nq = np.linalg.norm(q.astype(np.float64), axis=-1)
+    nk = np.linalg.norm(k.astype(np.float64), axis=-1)
+    for mode, exact in ((oracle.SCORE_PRODUCT, nq * nk), (oracle.SCORE_CONCAT, np.sqrt(nq ** 2 + nk ** 2))):
+        sc = oracle.score(s, q, k, mode=mode)
+        rel = np.abs(sc[:, :, :s.N] - exact) / exact
+        assert rel.max() < (d + 8) * 2.0 ** -24, mode
+        lvl0 = sc[:, :, :s.N]
+        for l in range(1, s.L):
+            w = s.p ** l
+            got = sc[:, :, s.level_off(l): s.level_off(l) + s.N // w]
+            assert np.array_equal(got, lvl0.reshape(s.B, s.H, s.N // w, w).max(axis=-1))
+
+
+def test_score_modes_special_cases():
+    """Zero K: the product is 0 and the concatenation's norm is ||q|| (as the sum's);
+    q = k: the product is ||q||^2 and the concatenation sqrt(2) ||q||."""
+    s = Shape(1, 1, 64, 64, 4, 2, 8)
+    q, _, _ = rand_qkv(s)
+    z = np.zeros_like(q)
+    n = np.linalg.norm(q.astype(np.float64), axis=-1)
+    assert np.all(oracle.score(s, q, z, mode=oracle.SCORE_PRODUCT)[..., :s.N] == 0)
+    np.testing.assert_allclose(oracle.score(s, q, z, mode=oracle.SCORE_CONCAT)[..., :s.N], n, rtol=1e-6)
+    np.testing.assert_allclose(oracle.score(s, q, q, mode=oracle.SCORE_PRODUCT)[..., :s.N], n ** 2, rtol=1e-5)
+    np.testing.assert_allclose(oracle.score(s, q, q, mode=oracle.SCORE_CONCAT)[..., :s.N], np.sqrt(2) * n, rtol=1e-6)
+
+
+@pytest.mark.parametrize("p,L,S", [(2, 3, 40), (4, 3, 30), (3, 2, 20), (4, 2, 12)])
+def test_select_keep_coarsest_brute_force(p, L, S):
+    """Keep-coarsest: every level-(L-1) entry is selected; the remaining
+    S - n_{L-1} slots hold the largest (score, -gid) keys of the other levels
+    (pure-Python sort); the order is (pos, level) as usual."""
+    N = p ** (L - 1) * 12
+    s = Shape(1, 2, N, 8, p, L, S)
+    q, k, _ = rand_qkv(s)
+    sc = oracle.score(s, q, k)
+    idx, pos, slot = oracle.select(s, sc, keep_coarsest=True)
+    top = s.level_off(L - 1)
+    ncoarse = s.M - top
+    assert ncoarse <= S
+    for h in range(s.H):
+        g = idx[0, h].tolist()
+        assert set(range(top, s.M)) <= set(g)
+        rest = sorted(range(top), key=lambda e: (-float(sc[0, h, e]), e))[: S - ncoarse]
+        assert set(g) == set(rest) | set(range(top, s.M))
+        items = []
+        for e in g:
+            l = max(l for l in range(s.L) if e >= s.level_off(l))
+            items.append(((e - s.level_off(l) + 1) * s.p ** l - 1, l))
+        assert items == sorted(items) and pos[0, h].tolist() == [it[0] for it in items]
+        for kk, e in enumerate(g):
+            assert slot[0, h, e] == kk
+    # every token then has a contributor: the scatter-back count is >= 1 everywhere
+    o = oracle.scatter(s, np.ones((1, 2, S, 8)), slot)
+    assert np.all(o == 1.0)

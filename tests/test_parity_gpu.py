@@ -320,6 +320,85 @@ def test_fused_forward_backward_match_oracle(case):
         check_attn(f64(t), bref[name], name)
 
 
+VARIANT_CASES = [
+    dict(score_mode=1, keep=False, w=dict(dtype="bf16", dist="outliers")),
+    dict(score_mode=2, keep=False, w=dict(dtype="bf16", d=128, p=2, L=5, N=2048, S=640)),
+    dict(score_mode=0, keep=True, w=dict(dtype="bf16", N=4096, L=4, S=300)),   # 64 coarsest of 300
+    dict(score_mode=2, keep=True, w=dict(p=3, L=3, N=1152, S=200)),            # fp32, generic p
+    dict(score_mode=1, keep=True, w=dict(dtype="bf16", p=4, L=2, N=1024, S=256)),  # S = n_{L-1}
+    dict(score_mode=0, keep=True, w=dict(dtype="bf16", dist="outliers", H=2, N=524288, L=5, S=4096)),
+]
+
+
+@pytest.mark.parametrize("case", VARIANT_CASES, ids=str)
+def test_variant_stages_match_oracle(case):
+    """Score ablations and keep-coarsest through the _ex stage calls: scores and
+    the selection bit-exact against the oracle with the same options."""
+    w = workload(**case["w"])
+    opt = lh.make_options(case["keep"], case["score_mode"])
+    xc = make_inputs(w, "cpu", with_dO=False)
+    x = to_dev(xc)
+    shp, dt = lshape(w), lh.dtype_code(x["q"].dtype)
+    M = lh.lh_num_entries(shp)
+    score = torch.zeros((w.B, w.H, M), dtype=torch.float32, device=DEV)
+    score2 = torch.zeros_like(score)
+    pyr = [torch.zeros((w.B, w.H, max(M - w.N, 1), w.d), dtype=torch.float32, device=DEV)
+           for _ in range(3)]
+    lh.lh_score_ex(shp, dt, x["q"], x["k"], score, opt)
+    lh.lh_build_pyramid_score_ex(shp, dt, x["q"], x["k"], x["v"], *pyr, score2, opt)
+    idx = torch.full((w.B, w.H, w.S), -7, dtype=torch.int32, device=DEV)
+    pos = torch.full_like(idx, -7)
+    slot = torch.full((w.B, w.H, M), -7, dtype=torch.int32, device=DEV)
+    lh.lh_topk_select_ex(shp, score, idx, pos, slot, opt)
+    torch.cuda.synchronize()
+    s = oshape(w)
+    sc_ref = oracle.score(s, xc["q"].float().numpy(), xc["k"].float().numpy(), mode=case["score_mode"])
+    assert np.array_equal(score.cpu().numpy(), sc_ref), "scores differ in some bit"
+    assert np.array_equal(score2.cpu().numpy(), sc_ref), "fused pass: scores differ"
+    i_ref, p_ref, s_ref = oracle.select(s, sc_ref, keep_coarsest=case["keep"])
+    assert np.array_equal(idx.cpu().numpy(), i_ref)
+    assert np.array_equal(pos.cpu().numpy(), p_ref)
+    assert np.array_equal(slot.cpu().numpy(), s_ref)
+
+
+@pytest.mark.parametrize("case", VARIANT_CASES[:4], ids=str)
+def test_variant_forward_backward_match_oracle(case):
+    """lh_forward_ex (+ lh_backward on its saved selection) against the oracle
+    pipeline with the same options."""
+    w = workload(**case["w"])
+    opt = lh.make_options(case["keep"], case["score_mode"])
+    xc = make_inputs(w, "cpu")
+    x = to_dev(xc)
+    o, saved = lh.forward(x["q"], x["k"], x["v"], w.p, w.L, w.S, options=opt)
+    dq, dk, dv = lh.backward(saved, x["dO"])
+    torch.cuda.synchronize()
+    s = oshape(w)
+    f = [xc[n].float().numpy() for n in ("q", "k", "v", "dO")]
+    ref = oracle.forward(s, *f[:3], score_mode=case["score_mode"], keep_coarsest=case["keep"])
+    sv = lambda which: lh.saved_view(saved.shape, saved.buf, which).cpu().numpy()
+    assert np.array_equal(sv(lh.SAVED_IDX), ref["idx"])
+    assert np.array_equal(sv(lh.SAVED_SLOT), ref["slot"])
+    check_attn(f64(o), ref["o"], "o")
+    bref = oracle.backward(s, ref, f[3])
+    for name, t in (("dq", dq), ("dk", dk), ("dv", dv)):
+        check_attn(f64(t), bref[name], name)
+    if case["keep"]:  # every token has a contributor, so no output row is left at zero
+        assert np.all(sv(lh.SAVED_INV_COUNT) > 0)
+
+
+def test_variant_options_rejected_on_the_host():
+    w = workload(dtype="bf16", N=4096, L=3, S=128)   # 256 coarsest entries > S
+    shp = lshape(w)
+    assert lh.lh_validate_options(shp, lh.make_options(True)) == lh.LH_ERR_SHAPE
+    assert lh.lh_validate_options(shp, lh.make_options(False, 7)) == lh.LH_ERR_INVALID_ARG
+    bad = lh.make_options(False)
+    bad.reserved[1] = 1
+    assert lh.lh_validate_options(shp, bad) == lh.LH_ERR_INVALID_ARG
+    x = to_dev(make_inputs(w, "cpu", with_dO=False))
+    with pytest.raises(lh.LighthouseError):
+        lh.forward(x["q"], x["k"], x["v"], w.p, w.L, w.S, options=lh.make_options(True))
+
+
 def test_degenerate_L1_full_selection_equals_causal_sdpa():
     w = workload(dtype="bf16", L=1, N=512, S=512, H=2)
     xc = make_inputs(w, "cpu")
