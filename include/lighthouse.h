@@ -262,6 +262,19 @@ int lh_kernel_launches(const lh_shape* shape, lh_dtype dtype, int backward);
  *   CONCAT  sqrt(ss(q) + ss(k))        (IEEE sqrt, one rounding per operation) */
 typedef enum { LH_SCORE_SUM = 0, LH_SCORE_PRODUCT = 1, LH_SCORE_CONCAT = 2 } lh_score_mode;
 
+/* How a selected entry's output spreads back over the original positions.  The
+ * pages fix a deterministic scatter-back to a fully dense output with "at least
+ * one contributor" per position ([ES] §2.C; [PT] phases 1 and 4), not the
+ * weights: the mean over the contributors covering a token is the default
+ * reading; the ablations are
+ *   SUM   the contributors' outputs added, no division;
+ *   LAST  an entry reaches only the last token of its span (its position), the
+ *         strictly causal reading of "the output does not see the future"; a
+ *         token takes the mean of what reaches it.
+ * inv_count (lh_scatter_back) then holds each token's weight in the adjoint:
+ * 1/c_t (MEAN, LAST), 1 (SUM), 0 where nothing reaches the token.             */
+typedef enum { LH_SCATTER_MEAN = 0, LH_SCATTER_SUM = 1, LH_SCATTER_LAST = 2 } lh_scatter_mode;
+
 /* Variants of the layer.  A NULL pointer, or all fields 0, is the default layer
  * the entry points above compute.
  *   keep_coarsest: 1 = every entry of the coarsest level L-1 is selected, which
@@ -270,19 +283,22 @@ typedef enum { LH_SCORE_SUM = 0, LH_SCORE_PRODUCT = 1, LH_SCORE_CONCAT = 2 } lh_
  *     themselves by gid), the other S - N/p^(L-1) slots go to the largest keys
  *     as usual.  Needs N / p^(L-1) <= S, else LH_ERR_SHAPE.
  *   score_mode: an lh_score_mode.
+ *   scatter_mode: an lh_scatter_mode (the backward must be given the same).
  *   reserved: must be 0 (LH_ERR_INVALID_ARG otherwise).                      */
 typedef struct {
   int32_t keep_coarsest;
   int32_t score_mode;
-  int32_t reserved[2];
+  int32_t scatter_mode;
+  int32_t reserved;
 } lh_options;
 
 /* Host-only check of a shape and options (NULL allowed); no CUDA call. */
 lh_status lh_validate_options(const lh_shape* shape, const lh_options* opt);
 
 /* The stage and fused calls that the options change, with the options; the
- * calls without _ex above are these with opt = NULL.  The backward does not
- * depend on them (it reads the selection that lh_forward_ex saved).          */
+ * calls without _ex above are these with opt = NULL.  The backward reads the
+ * selection that lh_forward_ex saved; of the options only scatter_mode changes
+ * it, so lh_backward_ex must get the options lh_forward_ex got.              */
 lh_status lh_build_pyramid_score_ex(const lh_shape* shape, lh_dtype dtype, const void* q,
                                     const void* k, const void* v, float* pq, float* pk, float* pv,
                                     float* score, const lh_options* opt, lh_stream_t stream);
@@ -294,6 +310,15 @@ lh_status lh_topk_select_ex(const lh_shape* shape, const float* score, int32_t* 
 lh_status lh_forward_ex(const lh_shape* shape, lh_dtype dtype, const void* q, const void* k,
                         const void* v, float scale, void* o, void* saved, void* ws,
                         size_t ws_bytes, const lh_options* opt, lh_stream_t stream);
+lh_status lh_scatter_back_ex(const lh_shape* shape, lh_dtype dtype, const void* os,
+                             const int32_t* slot, void* o, float* inv_count, const lh_options* opt,
+                             lh_stream_t stream);
+lh_status lh_scatter_back_bwd_ex(const lh_shape* shape, lh_dtype dtype, const void* dO,
+                                 const int32_t* slot, const float* inv_count, void* dos,
+                                 const lh_options* opt, lh_stream_t stream);
+lh_status lh_backward_ex(const lh_shape* shape, lh_dtype dtype, const void* saved, const void* dO,
+                         float scale, void* dq, void* dk, void* dv, void* ws, size_t ws_bytes,
+                         const lh_options* opt, lh_stream_t stream);
 
 #ifdef __cplusplus
 }

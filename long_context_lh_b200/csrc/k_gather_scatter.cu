@@ -25,6 +25,7 @@ namespace {
 struct Lv {
   int32_t N, M, S;
   int32_t L, p, log2p;
+  int32_t mode;  // lh_scatter_mode of the scatter-back (mean, sum, last token)
   int32_t off[kMaxLevels + 1];
   int32_t pw[kMaxLevels + 1];
 };
@@ -37,6 +38,7 @@ Lv make_lv(const Geom& g) {
   v.L = g.L;
   v.p = g.p;
   v.log2p = ((g.p & (g.p - 1)) == 0) ? __builtin_ctz((unsigned)g.p) : -1;
+  v.mode = g.scatter_mode;
   for (int l = 0; l <= kMaxLevels; ++l) {
     v.off[l] = (int32_t)g.off[l];
     v.pw[l] = (int32_t)(g.pw[l] > 0x7fffffff ? 0x7fffffff : g.pw[l]);
@@ -238,14 +240,15 @@ __global__ void __launch_bounds__(256) k_scatter(const __half* __restrict__ os,
 #pragma unroll
       for (int i = 0; i < 8; ++i) acc[i] = __fadd_rn(acc[i], xc[l - 1][i]);
     const int cnt = cc + (s0[r] >= 0 ? 1 : 0);
-    if (cnt > 0) {  // sums of fp16 values: 0 or |acc| >= 2^-24, inside div_small's range
+    if (cnt > 0 && lv.mode != LH_SCATTER_SUM) {  // sums of fp16 values: 0 or |acc| >= 2^-24, inside div_small's range
       const float y = kRcpCount[cnt], cf = (float)cnt;
 #pragma unroll
       for (int i = 0; i < 8; ++i) acc[i] = div_small(acc[i], cf, y);
     }
     const int64_t row = u * lv.N + t0 + r;
     store8_stream(o + row * D + 8 * c, acc);
-    if (inv_count && c == 0) inv_count[row] = kRcpCount[cnt];  // 1/c rounded; 0 when c = 0
+    // the weight of dO[t] in the adjoint: 1/c rounded (mean), 1 (sum); 0 when c = 0
+    if (inv_count && c == 0) inv_count[row] = lv.mode == LH_SCATTER_SUM ? (cnt > 0 ? 1.0f : 0.0f) : kRcpCount[cnt];
   }
 }
 
@@ -351,7 +354,8 @@ __global__ void __launch_bounds__(128) k_scatter_pp(const __half* __restrict__ o
       for (int i = 0; i < 8; ++i) base[i] = __fadd_rn(base[i], xu[i]);
       cb += cur.su[l - 2] >= 0 ? 1 : 0;
     }
-    if (cb > 0) {  // sums of fp16 values: 0 or |sum| >= 2^-24, inside div_small's range
+    const bool mean = lv.mode != LH_SCATTER_SUM;
+    if (cb > 0 && mean) {  // sums of fp16 values: 0 or |sum| >= 2^-24, inside div_small's range
       const float y = kRcpCount[cb], cf = (float)cb;
 #pragma unroll
       for (int i = 0; i < 8; ++i) base[i] = div_small(base[i], cf, y);
@@ -376,15 +380,17 @@ __global__ void __launch_bounds__(128) k_scatter_pp(const __half* __restrict__ o
         }
         const int cnt = cb + 1;
         const float y = kRcpCount[cnt], cf = (float)cnt;
+        if (mean) {
 #pragma unroll
-        for (int i = 0; i < 8; ++i) acc[i] = div_small(acc[i], cf, y);
+          for (int i = 0; i < 8; ++i) acc[i] = div_small(acc[i], cf, y);
+        }
         Packed8<Tout> pr;
         pr.pack(acc);
         pr.store(out + r * D);
-        icv[r] = y;
+        icv[r] = mean ? y : 1.0f;
       } else {
         ob.store(out + r * D);
-        icv[r] = kRcpCount[cb];
+        icv[r] = mean ? kRcpCount[cb] : (cb > 0 ? 1.0f : 0.0f);
       }
     }
     if (inv_count && c == 0) {  // the entry's P counts, one aligned vector store
@@ -451,7 +457,7 @@ __global__ void __launch_bounds__(256) k_scatter_bwd(const Tin* __restrict__ dO,
           int n = 0;
 #pragma unroll
           for (int l = 0; l < L; ++l) n += (__ldg(sl + lv.off[l] + lvl_index(lv, t, l)) >= 0) ? 1 : 0;
-          ic[b] = kRcpCount[n];
+          ic[b] = lv.mode == LH_SCATTER_SUM ? (n > 0 ? 1.0f : 0.0f) : kRcpCount[n];
         }
       }
     }
@@ -709,6 +715,81 @@ __global__ void __launch_bounds__(kScatterBwdThreads) k_scatter_bwd_pp(
   }
 }
 
+// ------------------------------------------- scatter-back, last-token variant
+// An entry delivers its output only to the last token of its span, pos(e); a
+// token takes the mean of what reaches it (levels ascending): the level-0 entry
+// at t and the entries of level l >= 1 whose span ends at t (p^l divides t + 1).
+// One d/8-lane group per token; generic in p and L (an ablation, not the hot path).
+__device__ __forceinline__ bool ends_at_t(const Lv& lv, int32_t t, int l) {
+  return l == 0 || ((uint32_t)(t + 1) % (uint32_t)lv.pw[l]) == 0u;
+}
+
+template <typename Tout, int D>
+__global__ void __launch_bounds__(256) k_scatter_last(const __half* __restrict__ os,
+                                                      const int32_t* __restrict__ slot,
+                                                      Tout* __restrict__ o, float* __restrict__ inv_count,
+                                                      const Lv lv, int64_t u0) {
+  constexpr int G = D / 8, kGroups = 256 / G;
+  const int32_t t = (int32_t)blockIdx.x * kGroups + (int32_t)(threadIdx.x / G);
+  if (t >= lv.N) return;
+  const int c = (int)(threadIdx.x % G);
+  const int64_t u = u0 + blockIdx.y;
+  const int32_t* sl = slot + u * lv.M;
+  const __half* src = os + u * lv.S * D + 8 * c;
+  float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+  int cnt = 0;
+  for (int l = 0; l < lv.L; ++l) {
+    if (!ends_at_t(lv, t, l)) continue;
+    const int32_t s = __ldg(sl + lv.off[l] + lvl_index(lv, t, l));
+    if (s < 0) continue;
+    float x[8];
+    unpack8(__ldg(reinterpret_cast<const uint4*>(src + (int64_t)s * D)), x);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) acc[i] = __fadd_rn(acc[i], x[i]);
+    ++cnt;
+  }
+  if (cnt > 0) {
+    const float y = kRcpCount[cnt], cf = (float)cnt;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) acc[i] = div_small(acc[i], cf, y);
+  }
+  const int64_t row = u * lv.N + t;
+  store8_stream(o + row * D + 8 * c, acc);
+  if (inv_count && c == 0) inv_count[row] = kRcpCount[cnt];
+}
+
+// Adjoint: every selected entry is reached by exactly one token (its pos), so
+// token t writes dO[t] / c_t to the slot of each entry that ends at it -- each
+// row of dos exactly once, no accumulation.
+template <typename Tin, int D>
+__global__ void __launch_bounds__(256) k_scatter_bwd_last(const Tin* __restrict__ dO,
+                                                          const int32_t* __restrict__ slot,
+                                                          const float* __restrict__ inv_count,
+                                                          __half* __restrict__ dos, const Lv lv,
+                                                          int64_t u0) {
+  constexpr int G = D / 8, kGroups = 256 / G;
+  const int32_t t = (int32_t)blockIdx.x * kGroups + (int32_t)(threadIdx.x / G);
+  if (t >= lv.N) return;
+  const int c = (int)(threadIdx.x % G);
+  const int64_t u = u0 + blockIdx.y;
+  const int32_t* sl = slot + u * lv.M;
+  int32_t ss[kMaxLevels];
+  int cnt = 0;
+  for (int l = 0; l < lv.L; ++l) {
+    ss[l] = ends_at_t(lv, t, l) ? __ldg(sl + lv.off[l] + lvl_index(lv, t, l)) : -1;
+    cnt += ss[l] >= 0 ? 1 : 0;
+  }
+  if (cnt == 0) return;
+  const float w = inv_count ? __ldg(inv_count + u * lv.N + t) : kRcpCount[cnt];
+  float x[8];
+  load8(dO + (u * lv.N + t) * D + 8 * c, x);
+#pragma unroll
+  for (int i = 0; i < 8; ++i) x[i] = __fmul_rn(x[i], w);
+  __half* dst = dos + u * lv.S * D + 8 * c;
+  for (int l = 0; l < lv.L; ++l)
+    if (ss[l] >= 0) store8(dst + (int64_t)ss[l] * D, x);
+}
+
 // --------------------------------------------------------------- gather bwd
 // dX[t] = sum_{l ascending, selected} dxs[slot_l(t)] / p^l, X in {Q, K, V}.
 // Grid: x = blocks of kRows tokens of one unit, y = unit (offset u0).
@@ -917,6 +998,13 @@ template <typename Tout, int D>
 cudaError_t scatter_t(const Geom& g, const __half* os, const int32_t* slot, Tout* o,
                       float* inv_count, cudaStream_t st) {
   const Lv lv = make_lv(g);
+  if (g.scatter_mode == LH_SCATTER_LAST) {
+    const unsigned bxl = blocks_for(g.N, 256 / (D / 8));
+    per_unit_chunks(g.U, [&](int64_t u0, unsigned nu) {
+      k_scatter_last<Tout, D><<<dim3(bxl, nu), 256, 0, st>>>(os, slot, o, inv_count, lv, u0);
+    });
+    return cudaGetLastError();
+  }
   if (g.L >= 2 && (g.p == 2 || g.p == 4)) {  // p known at compile time: p tokens a thread
     const unsigned bxp = blocks_for(g.N / g.p, (128 / (D / 8)) * kScatterEntries);
     return with_levels(g.L, [&](auto lc) {
@@ -977,6 +1065,13 @@ template <typename Tin, int D>
 cudaError_t scatter_bwd_d(const Geom& g, const Tin* dO, const int32_t* slot, const float* ic,
                           __half* dos, cudaStream_t st) {
   const Lv lv = make_lv(g);
+  if (g.scatter_mode == LH_SCATTER_LAST) {
+    const unsigned bxl = blocks_for(g.N, 256 / (D / 8));
+    per_unit_chunks(g.U, [&](int64_t u0, unsigned nu) {
+      k_scatter_bwd_last<Tin, D><<<dim3(bxl, nu), 256, 0, st>>>(dO, slot, ic, dos, lv, u0);
+    });
+    return cudaGetLastError();
+  }
   const int64_t spans = g.N / g.pw[g.L - 1];
   const int64_t groups = g.U * spans;
   // row-groups per span: p when p in {2, 4} and the span's lanes fit one warp

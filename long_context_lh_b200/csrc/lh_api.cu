@@ -154,6 +154,7 @@ Geom geom_with(const lh_shape& shape, const lh_options* opt) {
   if (opt) {
     g.score_mode = opt->score_mode;
     g.keep_top = opt->keep_coarsest;
+    g.scatter_mode = opt->scatter_mode;
   }
   return g;
 }
@@ -222,8 +223,10 @@ lh_status lh_validate_options(const lh_shape* shape, const lh_options* opt) {
   lh_status s = check_shape(shape);
   if (s != LH_OK) return s;
   if (opt == nullptr) return LH_OK;
-  if (opt->reserved[0] != 0 || opt->reserved[1] != 0) return LH_ERR_INVALID_ARG;
+  if (opt->reserved != 0) return LH_ERR_INVALID_ARG;
   if (opt->score_mode < LH_SCORE_SUM || opt->score_mode > LH_SCORE_CONCAT) return LH_ERR_INVALID_ARG;
+  if (opt->scatter_mode < LH_SCATTER_MEAN || opt->scatter_mode > LH_SCATTER_LAST)
+    return LH_ERR_INVALID_ARG;
   if (opt->keep_coarsest != 0 && opt->keep_coarsest != 1) return LH_ERR_INVALID_ARG;
   if (opt->keep_coarsest) {
     const Geom g = make_geom(*shape);
@@ -358,26 +361,40 @@ lh_status lh_subseq_attn_bwd(const lh_shape* shape, const void* qs, const void* 
                   dvs, static_cast<float*>(ws), stream);
 }
 
-lh_status lh_scatter_back(const lh_shape* shape, lh_dtype dtype, const void* os,
-                          const int32_t* slot, void* o, float* inv_count, lh_stream_t stream) {
+lh_status lh_scatter_back_ex(const lh_shape* shape, lh_dtype dtype, const void* os,
+                             const int32_t* slot, void* o, float* inv_count, const lh_options* opt,
+                             lh_stream_t stream) {
   lh_status s = lh_validate(shape, dtype);
   if (s != LH_OK) return s;
+  if ((s = lh_validate_options(shape, opt)) != LH_OK) return s;
   if (!aligned16(os) || !aligned16(slot) || !aligned16(o)) return LH_ERR_INVALID_ARG;
   if (inv_count && !aligned16(inv_count)) return LH_ERR_INVALID_ARG;
-  return cuda_status(launch_scatter(make_geom(*shape), dtype,
+  return cuda_status(launch_scatter(geom_with(*shape, opt), dtype,
                                     static_cast<const __half*>(os), slot, o, inv_count,
                                     stream));
+}
+
+lh_status lh_scatter_back(const lh_shape* shape, lh_dtype dtype, const void* os,
+                          const int32_t* slot, void* o, float* inv_count, lh_stream_t stream) {
+  return lh_scatter_back_ex(shape, dtype, os, slot, o, inv_count, nullptr, stream);
+}
+
+lh_status lh_scatter_back_bwd_ex(const lh_shape* shape, lh_dtype dtype, const void* dO,
+                                 const int32_t* slot, const float* inv_count, void* dos,
+                                 const lh_options* opt, lh_stream_t stream) {
+  lh_status s = lh_validate(shape, dtype);
+  if (s != LH_OK) return s;
+  if ((s = lh_validate_options(shape, opt)) != LH_OK) return s;
+  if (!aligned16(dO) || !aligned16(slot) || !aligned16(dos)) return LH_ERR_INVALID_ARG;
+  if (inv_count && !aligned16(inv_count)) return LH_ERR_INVALID_ARG;
+  return cuda_status(launch_scatter_bwd(geom_with(*shape, opt), dtype, dO, slot, inv_count,
+                                        static_cast<__half*>(dos), stream));
 }
 
 lh_status lh_scatter_back_bwd(const lh_shape* shape, lh_dtype dtype, const void* dO,
                               const int32_t* slot, const float* inv_count, void* dos,
                               lh_stream_t stream) {
-  lh_status s = lh_validate(shape, dtype);
-  if (s != LH_OK) return s;
-  if (!aligned16(dO) || !aligned16(slot) || !aligned16(dos)) return LH_ERR_INVALID_ARG;
-  if (inv_count && !aligned16(inv_count)) return LH_ERR_INVALID_ARG;
-  return cuda_status(launch_scatter_bwd(make_geom(*shape), dtype, dO, slot, inv_count,
-                                        static_cast<__half*>(dos), stream));
+  return lh_scatter_back_bwd_ex(shape, dtype, dO, slot, inv_count, dos, nullptr, stream);
 }
 
 lh_status lh_gather_bwd(const lh_shape* shape, lh_dtype dtype, const float* dqs,
@@ -438,13 +455,20 @@ lh_status lh_forward_ex(const lh_shape* shape, lh_dtype dtype, const void* q, co
 lh_status lh_backward(const lh_shape* shape, lh_dtype dtype, const void* saved, const void* dO,
                       float scale, void* dq, void* dk, void* dv, void* ws, size_t ws_bytes,
                       lh_stream_t stream) {
+  return lh_backward_ex(shape, dtype, saved, dO, scale, dq, dk, dv, ws, ws_bytes, nullptr, stream);
+}
+
+lh_status lh_backward_ex(const lh_shape* shape, lh_dtype dtype, const void* saved, const void* dO,
+                         float scale, void* dq, void* dk, void* dv, void* ws, size_t ws_bytes,
+                         const lh_options* opt, lh_stream_t stream) {
   lh_status s = lh_validate(shape, dtype);
   if (s != LH_OK) return s;
+  if ((s = lh_validate_options(shape, opt)) != LH_OK) return s;
   if (!aligned16(saved) || !aligned16(dO) || !aligned16(dq) || !aligned16(dk) ||
       !aligned16(dv) || !aligned16(ws))
     return LH_ERR_INVALID_ARG;
   if (ws_bytes < bwd_ws_layout(make_geom(*shape)).total) return LH_ERR_WORKSPACE;
-  const Geom g = make_geom(*shape);
+  const Geom g = geom_with(*shape, opt);
   const Layout sl = saved_layout(g), wl = bwd_ws_layout(g);
   const char* sv = static_cast<const char*>(saved);
   char* w = static_cast<char*>(ws);

@@ -24,6 +24,7 @@ struct Geom {
   int64_t off[kMaxLevels + 1];  // first gid of level l; off[L] = M
   int score_mode = 0;           // lh_score_mode
   int keep_top = 0;             // keep every level-(L-1) entry (lh_options.keep_coarsest)
+  int scatter_mode = 0;         // lh_scatter_mode
 };
 
 Geom make_geom(const lh_shape& s);

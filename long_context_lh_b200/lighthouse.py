@@ -49,18 +49,21 @@ def make_shape(B, H, N, d, p, L, S) -> Shape:
 
 
 LH_SCORE_SUM, LH_SCORE_PRODUCT, LH_SCORE_CONCAT = 0, 1, 2
+LH_SCATTER_MEAN, LH_SCATTER_SUM, LH_SCATTER_LAST = 0, 1, 2
 
 
 class Options(ctypes.Structure):
-    """lh_options: layer variants (keep-coarsest-level, score ablations)."""
+    """lh_options: layer variants (keep-coarsest-level, score and scatter ablations)."""
     _fields_ = [("keep_coarsest", ctypes.c_int32), ("score_mode", ctypes.c_int32),
-                ("reserved", ctypes.c_int32 * 2)]
+                ("scatter_mode", ctypes.c_int32), ("reserved", ctypes.c_int32)]
 
 
-def make_options(keep_coarsest=False, score_mode=LH_SCORE_SUM) -> Options:
+def make_options(keep_coarsest=False, score_mode=LH_SCORE_SUM,
+                 scatter_mode=LH_SCATTER_MEAN) -> Options:
     o = Options()
     o.keep_coarsest = 1 if keep_coarsest else 0
     o.score_mode = int(score_mode)
+    o.scatter_mode = int(scatter_mode)
     return o
 
 
@@ -103,6 +106,9 @@ _SIGS = {
     "lh_score_ex": ([_SP, _I, _VP, _VP, _VP, _VP, _VP], _I),
     "lh_topk_select_ex": ([_SP, _VP, _VP, _VP, _VP, _VP, _SZ, _VP, _VP], _I),
     "lh_forward_ex": ([_SP, _I, _VP, _VP, _VP, _F, _VP, _VP, _VP, _SZ, _VP, _VP], _I),
+    "lh_backward_ex": ([_SP, _I, _VP, _VP, _F, _VP, _VP, _VP, _VP, _SZ, _VP, _VP], _I),
+    "lh_scatter_back_ex": ([_SP, _I, _VP, _VP, _VP, _VP, _VP, _VP], _I),
+    "lh_scatter_back_bwd_ex": ([_SP, _I, _VP, _VP, _VP, _VP, _VP, _VP], _I),
     "lh_attention_impl_in_use": ([], _I),
     "lh_kernel_launches": ([_SP, _I, _I], _I),
 }
@@ -250,6 +256,24 @@ def lh_forward_ex(shape, dtype, q, k, v, scale, o, saved, ws, ws_bytes, options,
         ws_bytes, _opt(options), _st(stream)))
 
 
+def lh_backward_ex(shape, dtype, saved, dO, scale, dq, dk, dv, ws, ws_bytes, options, stream=None):
+    _check("lh_backward_ex", _lib().lh_backward_ex(
+        ctypes.byref(shape), dtype, _p(saved), _p(dO), float(scale), _p(dq), _p(dk), _p(dv),
+        _p(ws), ws_bytes, _opt(options), _st(stream)))
+
+
+def lh_scatter_back_ex(shape, dtype, os_, slot, o, inv_count, options, stream=None):
+    _check("lh_scatter_back_ex", _lib().lh_scatter_back_ex(
+        ctypes.byref(shape), dtype, _p(os_), _p(slot), _p(o), _p(inv_count), _opt(options),
+        _st(stream)))
+
+
+def lh_scatter_back_bwd_ex(shape, dtype, dO, slot, inv_count, dos, options, stream=None):
+    _check("lh_scatter_back_bwd_ex", _lib().lh_scatter_back_bwd_ex(
+        ctypes.byref(shape), dtype, _p(dO), _p(slot), _p(inv_count), _p(dos), _opt(options),
+        _st(stream)))
+
+
 def lh_score(shape, dtype, q, k, score, stream=None):
     _check("lh_score", _lib().lh_score(ctypes.byref(shape), dtype, _p(q), _p(k), _p(score),
                                        _st(stream)))
@@ -350,6 +374,7 @@ class Saved:
     dtype: int
     scale: float
     buf: torch.Tensor
+    options: object = None  # the Options lh_forward_ex got (the backward needs them too)
 
 
 def forward(q, k, v, p: int, L: int, S: int, scale: float = 0.0, stream=None, options=None):
@@ -368,7 +393,7 @@ def forward(q, k, v, p: int, L: int, S: int, scale: float = 0.0, stream=None, op
         lh_forward(shp, dt, q, k, v, scale, o, saved, ws, wsb, stream)
     else:
         lh_forward_ex(shp, dt, q, k, v, scale, o, saved, ws, wsb, options, stream)
-    return o, Saved(shp, dt, scale, saved)
+    return o, Saved(shp, dt, scale, saved, options)
 
 
 def backward(saved: Saved, dO, stream=None):
@@ -377,7 +402,11 @@ def backward(saved: Saved, dO, stream=None):
     dq, dk, dv = (torch.empty_like(dO) for _ in range(3))
     wsb = lh_workspace_bytes(shp, dt, True)
     ws = torch.empty(max(wsb, 256), dtype=torch.uint8, device=dO.device)
-    lh_backward(shp, dt, saved.buf, dO, saved.scale, dq, dk, dv, ws, wsb, stream)
+    if saved.options is None:
+        lh_backward(shp, dt, saved.buf, dO, saved.scale, dq, dk, dv, ws, wsb, stream)
+    else:
+        lh_backward_ex(shp, dt, saved.buf, dO, saved.scale, dq, dk, dv, ws, wsb, saved.options,
+                       stream)
     return dq, dk, dv
 
 

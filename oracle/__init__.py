@@ -105,6 +105,8 @@ def _L():
             "lho_attn_bwd": ([sp, P, P, P, P, d, P, P, P, i], None),
             "lho_scatter": ([sp, P, P, P], None),
             "lho_scatter_bwd": ([sp, P, P, P, P], None),
+            "lho_scatter_mode": ([sp, P, P, P, i], None),
+            "lho_scatter_bwd_mode": ([sp, P, P, P, P, i], None),
             "lho_gather_bwd": ([sp, P, P, P], None),
         }
         for name, (args, res) in sig.items():
@@ -255,20 +257,25 @@ def attn_bwd_sampled(qs, ks, vs, dos, scale, rows, chunk=1024):
     return dq, dk, dv
 
 
-def scatter(s: Shape, os_, slot) -> np.ndarray:
+SCATTER_MEAN, SCATTER_SUM, SCATTER_LAST = 0, 1, 2  # how a coarse output spreads over its span
+
+
+def scatter(s: Shape, os_, slot, mode=SCATTER_MEAN) -> np.ndarray:
+    """Scatter-back: the mean over a token's contributors (or the ablations: their
+    sum; last-token-only delivery)."""
     os_ = _f64(os_).reshape(s.U, s.S, s.d)
     slot = _i32(slot).reshape(s.U, s.M)
     out = np.zeros((s.U, s.N, s.d), np.float64)
-    _L().lho_scatter(ctypes.byref(s.c()), _p(os_), _p(slot), _p(out))
+    _L().lho_scatter_mode(ctypes.byref(s.c()), _p(os_), _p(slot), _p(out), int(mode))
     return out.reshape(s.B, s.H, s.N, s.d)
 
 
-def scatter_bwd(s: Shape, dO, idx, slot) -> np.ndarray:
+def scatter_bwd(s: Shape, dO, idx, slot, mode=SCATTER_MEAN) -> np.ndarray:
     dO = _f64(dO).reshape(s.U, s.N, s.d)
     idx = _i32(idx).reshape(s.U, s.S)
     slot = _i32(slot).reshape(s.U, s.M)
     out = np.zeros((s.U, s.S, s.d), np.float64)
-    _L().lho_scatter_bwd(ctypes.byref(s.c()), _p(dO), _p(idx), _p(slot), _p(out))
+    _L().lho_scatter_bwd_mode(ctypes.byref(s.c()), _p(dO), _p(idx), _p(slot), _p(out), int(mode))
     return out.reshape(s.B, s.H, s.S, s.d)
 
 
@@ -286,7 +293,7 @@ def default_scale(s: Shape, scale=None) -> float:
 
 
 def forward(s: Shape, q, k, v, scale=None, nthreads=None, score_mode=SCORE_SUM,
-            keep_coarsest=False) -> dict:
+            keep_coarsest=False, scatter_mode=SCATTER_MEAN) -> dict:
     """The whole forward; returns every intermediate (fp64 except score)."""
     scale = default_scale(s, scale)
     pq, pk, pv = (pyramid(s, x, nthreads) for x in (q, k, v))
@@ -294,14 +301,14 @@ def forward(s: Shape, q, k, v, scale=None, nthreads=None, score_mode=SCORE_SUM,
     idx, pos, slot = select(s, sc, nthreads, keep_coarsest=keep_coarsest)
     qs, ks, vs = gather(s, q, pq, idx), gather(s, k, pk, idx), gather(s, v, pv, idx)
     os_, lse = attn_fwd(s, qs, ks, vs, scale, nthreads=nthreads)
-    o = scatter(s, os_, slot)
+    o = scatter(s, os_, slot, scatter_mode)
     return dict(pq=pq, pk=pk, pv=pv, score=sc, idx=idx, pos=pos, slot=slot, qs=qs, ks=ks,
-                vs=vs, os=os_, lse=lse, o=o, scale=scale)
+                vs=vs, os=os_, lse=lse, o=o, scale=scale, scatter_mode=scatter_mode)
 
 
 def backward(s: Shape, fwd: dict, dO, nthreads=None) -> dict:
     """Backward through scatter-back, attention and gather with the saved selection."""
-    dos = scatter_bwd(s, dO, fwd["idx"], fwd["slot"])
+    dos = scatter_bwd(s, dO, fwd["idx"], fwd["slot"], fwd.get("scatter_mode", SCATTER_MEAN))
     dqs, dks, dvs = attn_bwd(s, fwd["qs"], fwd["ks"], fwd["vs"], dos, fwd["scale"], nthreads)
     return dict(dos=dos, dqs=dqs, dks=dks, dvs=dvs,
                 dq=gather_bwd(s, dqs, fwd["slot"]), dk=gather_bwd(s, dks, fwd["slot"]),

@@ -508,14 +508,34 @@ static int contributors(const lho_shape* s, const int32_t* slot_u, int64_t t, in
   return c;
 }
 
-void lho_scatter(const lho_shape* s, const double* os, const int32_t* slot, double* o) {
+/* Ablations of reading (i) above (how a coarse output spreads over its span):
+ *   mode 0 (default) mean over the contributors covering t;
+ *   mode 1 their sum (no division);
+ *   mode 2 last token only: an entry delivers its output only to pos(e), the
+ *          last token of its span (the strictly causal reading of [PT] phase 4,
+ *          "the output does not see the future"), and a token takes the mean of
+ *          what is delivered to it.
+ * delivered() gives the slots that reach token t under the mode (-1 = none). */
+static int delivered(const lho_shape* s, const int32_t* slot_u, int64_t t, int mode, int32_t* sl) {
+  int c = contributors(s, slot_u, t, sl);
+  if (mode != 2) return c;
+  c = 0;
+  for (int l = 0; l < s->L; ++l) {
+    if ((t + 1) % ipow(s->p, l) != 0) sl[l] = -1;  /* the entry's span ends later */
+    if (sl[l] >= 0) ++c;
+  }
+  return c;
+}
+
+void lho_scatter_mode(const lho_shape* s, const double* os, const int32_t* slot, double* o,
+                      int mode) {
   const int64_t U = s->B * s->H, N = s->N, M = lho_num_entries(s);
   const int d = s->d, S = s->S;
   int32_t sl[64];
   for (int64_t u = 0; u < U; ++u) {
     for (int64_t t = 0; t < N; ++t) {
       double* dst = o + (u * N + t) * d;
-      int cnt = contributors(s, slot + u * M, t, sl);
+      int cnt = delivered(s, slot + u * M, t, mode, sl);
       for (int i = 0; i < d; ++i) dst[i] = 0.0;
       if (cnt == 0) continue;
       for (int l = 0; l < s->L; ++l) {
@@ -523,14 +543,20 @@ void lho_scatter(const lho_shape* s, const double* os, const int32_t* slot, doub
         const double* src = os + (u * S + sl[l]) * d;
         for (int i = 0; i < d; ++i) dst[i] += src[i];
       }
-      for (int i = 0; i < d; ++i) dst[i] /= (double)cnt;
+      if (mode != 1)
+        for (int i = 0; i < d; ++i) dst[i] /= (double)cnt;
     }
   }
 }
 
-/* Adjoint of lho_scatter: dos[k] = sum_{t in span(e_k)} dO[t] / c_t, t ascending. */
-void lho_scatter_bwd(const lho_shape* s, const double* dO, const int32_t* idx,
-                     const int32_t* slot, double* dos) {
+void lho_scatter(const lho_shape* s, const double* os, const int32_t* slot, double* o) {
+  lho_scatter_mode(s, os, slot, o, 0);
+}
+
+/* Adjoint of lho_scatter_mode: dos[k] = sum over the tokens t of span(e_k) that
+ * e_k reaches of dO[t] / c_t (/ 1 for the sum), t ascending. */
+void lho_scatter_bwd_mode(const lho_shape* s, const double* dO, const int32_t* idx,
+                          const int32_t* slot, double* dos, int mode) {
   const int64_t U = s->B * s->H, N = s->N, M = lho_num_entries(s);
   const int d = s->d, S = s->S;
   int32_t sl[64];
@@ -542,12 +568,19 @@ void lho_scatter_bwd(const lho_shape* s, const double* dO, const int32_t* idx,
       double* dst = dos + (u * S + k) * d;
       for (int i = 0; i < d; ++i) dst[i] = 0.0;
       for (int64_t t = j * w; t < (j + 1) * w; ++t) {
-        int cnt = contributors(s, slot + u * M, t, sl);
+        int cnt = delivered(s, slot + u * M, t, mode, sl);
+        if (sl[l] != k) continue;  /* this entry does not reach t (last-token mode) */
         const double* g0 = dO + (u * N + t) * d;
-        for (int i = 0; i < d; ++i) dst[i] += g0[i] / (double)cnt;
+        const double c = (mode == 1) ? 1.0 : (double)cnt;
+        for (int i = 0; i < d; ++i) dst[i] += g0[i] / c;
       }
     }
   }
+}
+
+void lho_scatter_bwd(const lho_shape* s, const double* dO, const int32_t* idx,
+                     const int32_t* slot, double* dos) {
+  lho_scatter_bwd_mode(s, dO, idx, slot, dos, 0);
 }
 
 /* Adjoint of pyramid + gather (pooling is linear, the mean's adjoint is 1/p^l):

@@ -417,3 +417,54 @@ def test_select_keep_coarsest_brute_force(p, L, S):
     # every token then has a contributor: the scatter-back count is >= 1 everywhere
     o = oracle.scatter(s, np.ones((1, 2, S, 8)), slot)
     assert np.all(o == 1.0)
+
+
+def entry_centric_scatter(s: Shape, os_unit, idx_unit, mode):
+    """Scatter-back written from the entries' side: entry e (slot k) reaches every
+    token of its span (mean, sum) or only pos(e) (last); row t of the N x S
+    weight matrix is then normalised by its count (mean, last) or not (sum)."""
+    W = np.zeros((s.N, s.S))
+    for kk, g in enumerate(idx_unit):
+        l = max(l for l in range(s.L) if g >= s.level_off(l))
+        j = g - s.level_off(l)
+        w = s.p ** l
+        toks = [(j + 1) * w - 1] if mode == oracle.SCATTER_LAST else range(j * w, (j + 1) * w)
+        for t in toks:
+            W[t, kk] = 1.0
+    if mode != oracle.SCATTER_SUM:
+        c = W.sum(axis=1, keepdims=True)
+        W = np.divide(W, c, out=np.zeros_like(W), where=c > 0)
+    return W @ os_unit
+
+
+@pytest.mark.parametrize("mode", [0, 1, 2])
+@pytest.mark.parametrize("p,L,S", [(2, 4, 30), (4, 3, 40), (3, 3, 25)])
+def test_scatter_modes_entry_centric_and_adjoint(mode, p, L, S):
+    """Each scatter mode equals the entry-side construction above, and its
+    backward is its exact adjoint: <scatter(Y), Z> = <Y, scatter_bwd(Z)>."""
+    N = p ** (L - 1) * 6
+    s = Shape(1, 2, N, 8, p, L, S)
+    q, k, _ = rand_qkv(s)
+    idx, _, slot = oracle.select(s, oracle.score(s, q, k))
+    Y = rng.standard_normal((1, 2, S, 8))
+    Z = rng.standard_normal((1, 2, N, 8))
+    o = oracle.scatter(s, Y, slot, mode)
+    for h in range(2):
+        np.testing.assert_allclose(o[0, h], entry_centric_scatter(s, Y[0, h], idx[0, h], mode),
+                                   rtol=1e-12, atol=1e-12)
+    lhs = np.sum(o * Z)
+    rhs = np.sum(Y * oracle.scatter_bwd(s, Z, idx, slot, mode))
+    assert math.isclose(lhs, rhs, rel_tol=1e-12)
+    if mode == oracle.SCATTER_LAST:  # causal: a token receives nothing from entries ending later
+        for h in range(2):
+            for t in range(N):
+                for l in range(L):
+                    e = slot[0, h, s.level_off(l) + t // p ** l]
+                    if e >= 0 and (t + 1) % p ** l:
+                        Yp = Y.copy()
+                        Yp[0, h, e] += 1.0
+                        assert np.array_equal(oracle.scatter(s, Yp, slot, mode)[0, h, t], o[0, h, t])
+                        break
+                else:
+                    continue
+                break

@@ -327,6 +327,10 @@ VARIANT_CASES = [
     dict(score_mode=2, keep=True, w=dict(p=3, L=3, N=1152, S=200)),            # fp32, generic p
     dict(score_mode=1, keep=True, w=dict(dtype="bf16", p=4, L=2, N=1024, S=256)),  # S = n_{L-1}
     dict(score_mode=0, keep=True, w=dict(dtype="bf16", dist="outliers", H=2, N=524288, L=5, S=4096)),
+    dict(score_mode=0, keep=False, scatter=1, w=dict(dtype="bf16", dist="outliers")),      # sum
+    dict(score_mode=0, keep=False, scatter=2, w=dict(dtype="bf16", dist="outliers")),      # last token
+    dict(score_mode=2, keep=True, scatter=2, w=dict(p=3, L=3, N=1152, S=200)),
+    dict(score_mode=0, keep=False, scatter=1, w=dict(dtype="bf16", d=128, p=2, L=5, N=2048, S=640)),
 ]
 
 
@@ -361,12 +365,12 @@ def test_variant_stages_match_oracle(case):
     assert np.array_equal(slot.cpu().numpy(), s_ref)
 
 
-@pytest.mark.parametrize("case", VARIANT_CASES[:4], ids=str)
+@pytest.mark.parametrize("case", VARIANT_CASES[:4] + VARIANT_CASES[6:], ids=str)
 def test_variant_forward_backward_match_oracle(case):
-    """lh_forward_ex (+ lh_backward on its saved selection) against the oracle
+    """lh_forward_ex (+ lh_backward_ex on its saved selection) against the oracle
     pipeline with the same options."""
     w = workload(**case["w"])
-    opt = lh.make_options(case["keep"], case["score_mode"])
+    opt = lh.make_options(case["keep"], case["score_mode"], case.get("scatter", 0))
     xc = make_inputs(w, "cpu")
     x = to_dev(xc)
     o, saved = lh.forward(x["q"], x["k"], x["v"], w.p, w.L, w.S, options=opt)
@@ -374,7 +378,8 @@ def test_variant_forward_backward_match_oracle(case):
     torch.cuda.synchronize()
     s = oshape(w)
     f = [xc[n].float().numpy() for n in ("q", "k", "v", "dO")]
-    ref = oracle.forward(s, *f[:3], score_mode=case["score_mode"], keep_coarsest=case["keep"])
+    ref = oracle.forward(s, *f[:3], score_mode=case["score_mode"], keep_coarsest=case["keep"],
+                         scatter_mode=case.get("scatter", 0))
     sv = lambda which: lh.saved_view(saved.shape, saved.buf, which).cpu().numpy()
     assert np.array_equal(sv(lh.SAVED_IDX), ref["idx"])
     assert np.array_equal(sv(lh.SAVED_SLOT), ref["slot"])
@@ -382,8 +387,33 @@ def test_variant_forward_backward_match_oracle(case):
     bref = oracle.backward(s, ref, f[3])
     for name, t in (("dq", dq), ("dk", dk), ("dv", dv)):
         check_attn(f64(t), bref[name], name)
-    if case["keep"]:  # every token has a contributor, so no output row is left at zero
+    if case["keep"] and case.get("scatter", 0) != 2:  # every token has a contributor
         assert np.all(sv(lh.SAVED_INV_COUNT) > 0)
+
+
+@pytest.mark.parametrize("mode", [1, 2])
+@pytest.mark.parametrize("case", [GS_CASES[1], GS_CASES[3], GS_CASES[5]], ids=str)
+def test_scatter_modes_match_oracle(case, mode):
+    """The scatter ablations (sum, last token) and their adjoints through the
+    _ex stage calls, with and without the saved weights, against the oracle."""
+    w = workload(**case)
+    x = to_dev(make_inputs(w, "cpu"))
+    _, _, idx, _, slot = run_front(w, x)
+    opt = lh.make_options(False, 0, mode)
+    shp, dt = lshape(w), lh.dtype_code(x["q"].dtype)
+    s = oshape(w)
+    os_ = torch.randn((w.B, w.H, w.S, w.d), device=DEV).to(torch.float16)
+    o = torch.empty((w.B, w.H, w.N, w.d), dtype=x["q"].dtype, device=DEV)
+    ic = torch.empty((w.B, w.H, w.N), dtype=torch.float32, device=DEV)
+    lh.lh_scatter_back_ex(shp, dt, os_, slot, o, ic, opt)
+    ref = oracle.scatter(s, f64(os_), slot.cpu().numpy(), mode)
+    tol = 2.0 ** -8 if w.dtype == "bf16" else 1e-6
+    assert np.all(np.abs(f64(o) - ref) <= tol * np.abs(ref) + 1e-6)
+    for use_ic in (True, False):
+        dos = torch.empty((w.B, w.H, w.S, w.d), dtype=torch.float16, device=DEV)
+        lh.lh_scatter_back_bwd_ex(shp, dt, x["dO"], slot, ic if use_ic else None, dos, opt)
+        ref = oracle.scatter_bwd(s, f64(x["dO"]), idx.cpu().numpy(), slot.cpu().numpy(), mode)
+        assert np.all(np.abs(f64(dos) - ref) <= 2.0 ** -11 * np.abs(ref) + 1e-5 * (1 + np.abs(ref).max()))
 
 
 def test_variant_options_rejected_on_the_host():
@@ -392,8 +422,9 @@ def test_variant_options_rejected_on_the_host():
     assert lh.lh_validate_options(shp, lh.make_options(True)) == lh.LH_ERR_SHAPE
     assert lh.lh_validate_options(shp, lh.make_options(False, 7)) == lh.LH_ERR_INVALID_ARG
     bad = lh.make_options(False)
-    bad.reserved[1] = 1
+    bad.reserved = 1
     assert lh.lh_validate_options(shp, bad) == lh.LH_ERR_INVALID_ARG
+    assert lh.lh_validate_options(shp, lh.make_options(False, 0, 3)) == lh.LH_ERR_INVALID_ARG
     x = to_dev(make_inputs(w, "cpu", with_dO=False))
     with pytest.raises(lh.LighthouseError):
         lh.forward(x["q"], x["k"], x["v"], w.p, w.L, w.S, options=lh.make_options(True))
