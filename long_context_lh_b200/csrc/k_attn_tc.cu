@@ -63,10 +63,13 @@ __device__ __forceinline__ void store_row_half(uint8_t* tile_half, int r, const 
 // own tile A, warps 4-7 tile B, one thread per row and all 128 keys of a tile:
 // every SM sub-partition holds one warp of each tile, and the two alternate
 // (while one computes its exponentials, the tensor core serves the other).
-// TMEM: S_A, S_B (128 columns each; P is written as packed fp16 over the S
-// columns already consumed), O_A, O_B (D columns each).  The MMA warp issues
-// S_T(j+1) right after O_T += P_T(j) V(j), so tile T's next scores are ready
-// while the other tile computes.
+// TMEM: S_A, S_B (128 columns each), O_A, O_B (D columns each) and, at d = 64,
+// P_A, P_B (64 columns each, packed fp16).  At d = 64 a tile's row work releases
+// S_T as soon as it has read it (before its exponentials are done), and the MMA
+// warp issues S_T(j+1) then, so the next scores are computed under the current
+// tile's exponentials and O_T += P_T(j) V(j) runs under the next tile's row max.
+// At d = 128 TMEM is full: P is written over the S columns already read, and
+// S_T(j+1) follows O_T += P_T(j) V(j).
 template <int D>
 struct FwdLayout {
   static constexpr int kKS = (D == 64) ? 4 : 2;  // K/V stages
@@ -78,9 +81,9 @@ struct FwdLayout {
 };
 
 struct FwdBars {
-  uint64_t q_full, q_tmem;  // Q tiles in shared memory; (d = 64) copied on into TMEM
+  uint64_t q_full;
   uint64_t kv_full[4], kv_empty[4];
-  uint64_t s_full[2], p_full[2], pv_done[2], mma_done;  // [tile A, B]
+  uint64_t s_full[2], s_free[2], p_full[2], pv_done[2], mma_done;  // [tile A, B]
   uint32_t tmem;
   int abort;
 };
@@ -130,11 +133,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int t = 0; t < 2; ++t) {
       mbar_init(&bars->s_full[t], 1);
+      mbar_init(&bars->s_free[t], 4);
       mbar_init(&bars->p_full[t], 4);
       mbar_init(&bars->pv_done[t], 1);
     }
     mbar_init(&bars->mma_done, 1);
-    mbar_init(&bars->q_tmem, 8);
     bars->abort = 0;
     mbar_init_fence();
   }
@@ -144,12 +147,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = bars->tmem;
   const uint32_t tO = tmem + 256;  // O_A at +256, O_B at +256+D; S_T at +128*T
-  // d = 64: Q_A, Q_B also live in TMEM (32 columns each, at +384 and +416) and
-  // are the A operand of S = Q K^T, so those products read only K from shared
-  // memory (both operands from shared memory halve their rate)
-  constexpr bool kQT = (D == 64);
-  static_assert(!kQT || 256 + 2 * D + 64 <= (int)kTmemCols, "TMEM: S_A, S_B, O_A, O_B, Q_A, Q_B");
-  const uint32_t tQ = tmem + 256 + 2 * D;
+  // d = 64: P_A, P_B in their own columns (+384, +448), so S_T(j+1) need not
+  // wait for O_T += P_T(j) V_j
+  constexpr bool kSepP = (D == 64);
+  static_assert(!kSepP || 256 + 2 * D + 128 <= (int)kTmemCols, "TMEM: S_A, S_B, O_A, O_B, P_A, P_B");
+  const uint32_t tP = tmem + 256 + 2 * D;
 
   if (warp == 8) {
     // ------------------------------------------------------------ TMA producer
@@ -191,10 +193,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint64_t off = (uint64_t)((((kk >> 2) * 16384) + ((kk & 3) * 32)) >> 4);
-          if constexpr (kQT)
-            umma_f16_ta(tmem + t * 128, tQ + t * 32 + 8 * kk, k + off, idS, kk > 0);
-          else
-            umma_f16(tmem + t * 128, q + off, k + off, idS, kk > 0);
+          umma_f16(tmem + t * 128, q + off, k + off, idS, kk > 0);
         }
         umma_commit(&bars->s_full[t]);
       }
@@ -202,23 +201,53 @@ __global__ void __launch_bounds__(kThreads, 1)
     };
     auto issue_pv = [&](int t, int j) {  // O_t += P_t(j) V_j, P_t from TMEM
       const uint64_t v = dV + (uint64_t)(((j % KS) * Lt::kTile) >> 4);
+      const uint32_t pt = kSepP ? tP + t * 64 : tmem + t * 128;
       if (lane == 0) {
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
-          umma_f16_ta(tO + t * D, tmem + t * 128 + 8 * kk, v + (uint64_t)((kk * 2048) >> 4), idPV,
+          umma_f16_ta(tO + t * D, pt + 8 * kk, v + (uint64_t)((kk * 2048) >> 4), idPV,
                       (j > 0 || kk > 0));
         umma_commit(&bars->pv_done[t]);
       }
       __syncwarp();
     };
-    bool ok = warp_wait(kQT ? &bars->q_tmem : &bars->q_full, 0, abort, kStatus) &&
+    bool ok = warp_wait(&bars->q_full, 0, abort, kStatus) &&
               warp_wait(&bars->kv_full[0], 0, abort, kStatus);
     if (ok) {
       tc_fence_after();
       issue_s(0, 0);
       if (nB > 0) issue_s(1, 0);
     }
-    for (int j = 0; ok && j < nA; ++j) {
+    if constexpr (kSepP) {
+      // per key tile j: S_A(j+1) once S_A(j) is read, O_A += P_A(j) V_j once P_A(j)
+      // is written, then the same for tile B; the waits follow the order in which
+      // the row work produces these events
+      for (int j = 0; ok && j < nA; ++j) {
+        const int st = j % KS;
+        if (j + 1 < nA) {
+          if (!(ok = warp_wait(&bars->s_free[0], j & 1, abort, kStatus))) break;
+          if (!(ok = warp_wait(&bars->kv_full[(j + 1) % KS], ((j + 1) / KS) & 1, abort, kStatus))) break;
+          tc_fence_after();
+          issue_s(0, j + 1);
+        }
+        if (!(ok = warp_wait(&bars->p_full[0], j & 1, abort, kStatus))) break;
+        tc_fence_after();
+        issue_pv(0, j);
+        if (j < nB) {
+          if (j + 1 < nB) {  // K_{j+1} is in place (waited for above: j + 1 < nB <= nA)
+            if (!(ok = warp_wait(&bars->s_free[1], j & 1, abort, kStatus))) break;
+            tc_fence_after();
+            issue_s(1, j + 1);
+          }
+          if (!(ok = warp_wait(&bars->p_full[1], j & 1, abort, kStatus))) break;
+          tc_fence_after();
+          issue_pv(1, j);
+        }
+        if (lane == 0) umma_commit(&bars->kv_empty[st]);  // K_j, V_j no longer needed
+        __syncwarp();
+      }
+    }
+    for (int j = 0; !kSepP && ok && j < nA; ++j) {
       const int st = j % KS;
       const bool next = j + 1 < nA;
       // tile A: its product with V_j, then (S_A buffer free again) its next scores
@@ -293,29 +322,35 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float m_new = grow ? mx : m_ref;
       // every phase of pv_done[t] is waited for, in order; O_t (and the P of the
       // previous tile) must be done with before O_t is rescaled or P rewritten
-      if (j > 0) {
-        ok = warp_wait(&bars->pv_done[t], (j - 1) & 1, abort, kStatus);
+      auto pv_wait_rescale = [&]() -> bool {
+        if (j > 0 && !warp_wait(&bars->pv_done[t], (j - 1) & 1, abort, kStatus)) return false;
+        if (j > 0 && __any_sync(0xffffffffu, grow)) {
+          tc_fence_after();
+          const float alpha = ex2(m_ref - m_new);  // 1 for rows that do not grow
+#pragma unroll
+          for (int c = 0; c < D / 32; ++c) {
+            uint32_t ov[32];
+            tmem_ld32(tOt + c * 32, ov);
+            tmem_ld_wait();
+#pragma unroll
+            for (int i = 0; i < 32; ++i) ov[i] = __float_as_uint(__uint_as_float(ov[i]) * alpha);
+            tmem_st32(tOt + c * 32, ov);
+          }
+          l *= alpha;
+        }
+        m_ref = m_new;
+        return true;
+      };
+      // at d = 64 the wait is deferred to the first P store (after the first
+      // 32 exponentials), so the previous P V runs under the row max
+      if constexpr (!kSepP) {
+        ok = pv_wait_rescale();
         if (!ok) return;
       }
-      if (j > 0 && __any_sync(0xffffffffu, grow)) {
-        tc_fence_after();
-        const float alpha = ex2(m_ref - m_new);  // 1 for rows that do not grow
-#pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
-          uint32_t ov[32];
-          tmem_ld32(tOt + c * 32, ov);
-          tmem_ld_wait();
-#pragma unroll
-          for (int i = 0; i < 32; ++i) ov[i] = __float_as_uint(__uint_as_float(ov[i]) * alpha);
-          tmem_st32(tOt + c * 32, ov);
-        }
-        l *= alpha;
-      }
-      m_ref = m_new;
       // P = 2^(S c - m_ref): S read again in two 64-column halves (two loads, one
       // wait each), packed fp16 written over S columns already read (chunk c of
       // 32 columns writes columns 16c..16c+15)
-      const float2 cc = make_float2(scale_log2, scale_log2), nm = make_float2(-m_ref, -m_ref);
+      const float2 cc = make_float2(scale_log2, scale_log2), nm = make_float2(-m_new, -m_new);
       float2 sacc[4] = {make_float2(0.0f, 0.0f), make_float2(0.0f, 0.0f), make_float2(0.0f, 0.0f),
                         make_float2(0.0f, 0.0f)};
       uint32_t v[64];
@@ -325,6 +360,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           tmem_ld32_at<0>(tS + 32 * c, v);
           tmem_ld32_at<32>(tS + 32 * c + 32, v);
           tmem_ld_wait();
+          if (kSepP && c == 2) {  // S_t(j) fully read: the MMA warp may overwrite it
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bars->s_free[t]);
+          }
         }
         uint32_t pk[16];
 #pragma unroll
@@ -349,7 +389,15 @@ __global__ void __launch_bounds__(kThreads, 1)
           pk[i >> 1] = h2(p.x, p.y);
           pk[(i >> 1) + 1] = h2(q.x, q.y);
         }
-        tmem_st16(tS + 16 * c, pk);
+        if constexpr (kSepP) {
+          if (c == 0) {
+            ok = pv_wait_rescale();
+            if (!ok) return;
+          }
+          tmem_st16(tP + t * 64 + lane_addr + 16 * c, pk);
+        } else {
+          tmem_st16(tS + 16 * c, pk);
+        }
       }
       tmem_st_wait();
       tc_fence_before();  // orders P and the O_t rescale (TMEM stores) before the product
@@ -358,30 +406,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float2 s01 = fadd2(sacc[0], sacc[1]), s23 = fadd2(sacc[2], sacc[3]);
       l += (s01.x + s01.y) + (s23.x + s23.y);
     };
-    if constexpr (kQT) {
-      // this thread's row of its Q tile: shared memory (128-byte swizzled) -> TMEM
-      // columns of Q_t, two fp16 along K per column (lower index in the low half).
-      // Every row-work warp arrives (a tile B that does not exist copies zeros).
-      ok = warp_wait(&bars->q_full, 0, abort, kStatus);
-      if (ok) {
-        const uint8_t* qrow = sQ + t * Lt::kTile;
-        uint32_t w[32];
-#pragma unroll
-        for (int c = 0; c < 8; ++c) {
-          const uint4 x = *reinterpret_cast<const uint4*>(qrow + swz(r, c));
-          w[4 * c] = x.x;
-          w[4 * c + 1] = x.y;
-          w[4 * c + 2] = x.z;
-          w[4 * c + 3] = x.w;
-        }
-        tmem_st32(tQ + t * 32 + lane_addr, w);
-        tmem_st_wait();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&bars->q_tmem);
-      }
-    }
-    if (n > 0 && ok) {
+    if (n > 0) {
       for (int j = 0; j < n - 1 && ok; ++j) step(j, std::false_type{});
       if (ok) step(n - 1, std::true_type{});
       if (ok) ok = warp_wait(&bars->pv_done[t], (n - 1) & 1, abort, kStatus);
