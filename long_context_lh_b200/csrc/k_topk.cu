@@ -178,7 +178,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   __shared__ uint32_t sh[4];
   __shared__ uint32_t warp_tot[kWarps];
   __shared__ uint32_t cta_total;
-  extern __shared__ uint32_t skey[];  // the CTA's keys, level by level (cached), kcap words
+  extern __shared__ __align__(16) uint32_t skey[];  // the CTA's keys, level by level (cached), kcap words
   // then per token of the CTA: bits 0-7 the selected levels ending at it,
   // bits 8-15 all levels ending at it (written by the counting pass)
   uint16_t* smask = reinterpret_cast<uint16_t*>(skey + kcap);
@@ -227,16 +227,39 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t dmask = (uint32_t)nb - 1u;
     for (int i = threadIdx.x; i < kBins; i += kThreads) hist[buf][i] = 0;
     __syncthreads();
+    if (cached) {
+      // the level does not matter here: one flat pass over the CTA's keys, four
+      // per 16-byte shared-memory load (the tail, nk % 4 keys, one by one)
+      const int32_t nq = nk >> 2;
+      for (int32_t i0 = warp * 32; i0 < nq; i0 += kThreads) {  // warp-uniform trip count
+        const int32_t i = i0 + lane;
+        const uint4 k4 = i < nq ? reinterpret_cast<const uint4*>(skey)[i] : make_uint4(0u, 0u, 0u, 0u);
+        const uint32_t kk[4] = {k4.x, k4.y, k4.z, k4.w};
 #pragma unroll
-    for (int l = 0; l < kMaxLevels; ++l) {
-      for (int32_t j0 = warp * 32; j0 < nl[l]; j0 += kThreads) {  // warp-uniform trip count
-        const int32_t j = j0 + lane;
-        const uint32_t kv = j < nl[l] ? key_of(l, j) : 0u;
-        const bool act = j < nl[l] && (kv & pmask) == prefix;
-        if (pass == 0)
-          hist_add(hist[buf], act, (kv >> shift) & dmask);
-        else
-          hist_add_plain(hist[buf], act, (kv >> shift) & dmask);
+        for (int e = 0; e < 4; ++e) {
+          const bool act = i < nq && (kk[e] & pmask) == prefix;
+          if (pass == 0)
+            hist_add(hist[buf], act, (kk[e] >> shift) & dmask);
+          else
+            hist_add_plain(hist[buf], act, (kk[e] >> shift) & dmask);
+        }
+      }
+      for (int32_t i = 4 * nq + (int32_t)threadIdx.x; i < nk; i += kThreads) {
+        const uint32_t kv = skey[i];
+        if ((kv & pmask) == prefix) atomicAdd(&hist[buf][(kv >> shift) & dmask], 1u);
+      }
+    } else {
+#pragma unroll
+      for (int l = 0; l < kMaxLevels; ++l) {
+        for (int32_t j0 = warp * 32; j0 < nl[l]; j0 += kThreads) {  // warp-uniform trip count
+          const int32_t j = j0 + lane;
+          const uint32_t kv = j < nl[l] ? key_of(l, j) : 0u;
+          const bool act = j < nl[l] && (kv & pmask) == prefix;
+          if (pass == 0)
+            hist_add(hist[buf], act, (kv >> shift) & dmask);
+          else
+            hist_add_plain(hist[buf], act, (kv >> shift) & dmask);
+        }
       }
     }
     cluster.sync();
@@ -262,13 +285,27 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t dmask = (uint32_t)nb - 1u;
       for (int i = threadIdx.x; i < kBins; i += kThreads) hist[buf][i] = 0;
       __syncthreads();
+      if (cached) {
+        // flat over the cached keys; a key at position i of level l has gid
+        // off[l] + jb[l] + (i - kb[l]), the level found by comparing i with kb[]
+        for (int32_t i = (int32_t)threadIdx.x; i < nk; i += kThreads) {
+          if (skey[i] != T) continue;
+          int32_t gb = prm.off[0] + jb[0] - kb[0];
 #pragma unroll
-      for (int l = 0; l < kMaxLevels; ++l) {
-        for (int32_t j0 = warp * 32; j0 < nl[l]; j0 += kThreads) {
-          const int32_t j = j0 + lane;
-          const uint32_t gid = (uint32_t)(prm.off[l] + jb[l] + j);
-          const bool in = j < nl[l] && key_of(l, j < nl[l] ? j : 0) == T && (gid & gmask) == gprefix;
-          hist_add_plain(hist[buf], in, (gid >> shift) & dmask);
+          for (int l = 1; l < kMaxLevels; ++l)
+            if (l < prm.L && i >= kb[l]) gb = prm.off[l] + jb[l] - kb[l];
+          const uint32_t gid = (uint32_t)(gb + i);
+          if ((gid & gmask) == gprefix) atomicAdd(&hist[buf][(gid >> shift) & dmask], 1u);
+        }
+      } else {
+#pragma unroll
+        for (int l = 0; l < kMaxLevels; ++l) {
+          for (int32_t j0 = warp * 32; j0 < nl[l]; j0 += kThreads) {
+            const int32_t j = j0 + lane;
+            const uint32_t gid = (uint32_t)(prm.off[l] + jb[l] + j);
+            const bool in = j < nl[l] && key_of(l, j < nl[l] ? j : 0) == T && (gid & gmask) == gprefix;
+            hist_add_plain(hist[buf], in, (gid >> shift) & dmask);
+          }
         }
       }
       cluster.sync();
