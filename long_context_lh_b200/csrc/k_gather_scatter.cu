@@ -845,6 +845,117 @@ __global__ void __launch_bounds__(256) k_gather_bwd(
   }
 }
 
+// Same result as k_gather_bwd (the same fused multiply-adds in the same order),
+// for p = P in {2, 4} known at compile time.  One array per thread (grid z), and
+// a thread walks kGatherEntries consecutive level-1 entries (P tokens each) with
+// the next entry's slot loads in flight while the current entry's rows load, so
+// an entry costs one memory round trip.  A token not selected at level 0 starts
+// its chain from 0 (0 + x*w = x*w exactly in the first fused multiply-add), the
+// same chain for all P tokens of its level-1 entry: done once, stored P times.
+constexpr int kGatherEntries = 4;
+
+template <typename Tout, int D, int L, int P>
+__global__ void __launch_bounds__(128) k_gather_bwd_pp(
+    const float* __restrict__ dqs, const float* __restrict__ dks, const float* __restrict__ dvs,
+    const int32_t* __restrict__ slot, Tout* __restrict__ dq, Tout* __restrict__ dk,
+    Tout* __restrict__ dv, const Lv lv, int64_t u0) {
+  static_assert(L >= 2 && (P == 2 || P == 4), "specialised on p in {2, 4}, L >= 2");
+  constexpr int G = D / 8, kGroups = 128 / G, NE = kGatherEntries;
+  constexpr int NU = (L > 2) ? L - 2 : 1;  // levels >= 2: one entry each
+  const int32_t n1 = lv.N / P;
+  const int32_t e0 = ((int32_t)blockIdx.x * kGroups + (int32_t)(threadIdx.x / G)) * NE;
+  if (e0 >= n1) return;
+  const int c = (int)(threadIdx.x % G);
+  const int64_t u = u0 + blockIdx.y;
+  const int a = (int)blockIdx.z;
+  const int32_t* sl = slot + u * lv.M;
+  const float* src = (a == 0 ? dqs : a == 1 ? dks : dvs) + u * lv.S * D + 8 * c;
+  Tout* dst = (a == 0 ? dq : a == 1 ? dk : dv) + u * lv.N * D + 8 * c;
+
+  struct Slots {
+    int32_t s0[P], s1, su[NU];
+  };
+  auto load_slots = [&](int32_t e, Slots& sv) {
+    const int32_t t = e * P;
+#pragma unroll
+    for (int r = 0; r < P; ++r) sv.s0[r] = __ldg(sl + t + r);
+    sv.s1 = __ldg(sl + lv.off[1] + e);
+    static_for<2, L>([&](auto lc) {
+      constexpr int l = decltype(lc)::value;
+      sv.su[l - 2] = __ldg(sl + lv.off[l] + (int32_t)((uint32_t)e / (uint32_t)ipow(P, l - 1)));
+    });
+  };
+  auto row = [&](int32_t sidx, float (&x)[8]) {
+    if (sidx >= 0) {
+      load8(src + (int64_t)sidx * D, x);
+    } else {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) x[i] = 0.0f;
+    }
+  };
+  Slots cur;
+  load_slots(e0, cur);
+#pragma unroll 1
+  for (int k = 0; k < NE; ++k) {
+    const int32_t e = e0 + k;
+    if (e >= n1) break;
+    float x0[P][8], x1[8], xu[NU][8];
+#pragma unroll
+    for (int r = 0; r < P; ++r) row(cur.s0[r], x0[r]);
+    row(cur.s1, x1);
+#pragma unroll
+    for (int l = 2; l < L; ++l) row(cur.su[l - 2], xu[l - 2]);
+    Slots nxt;
+    if (k + 1 < NE && e + 1 < n1) load_slots(e + 1, nxt);  // in flight with this entry's rows
+    // chain of a token unselected at level 0: 0, then + x_l / p^l for the
+    // selected coarse levels, ascending (a level not selected adds nothing)
+    float base[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) base[i] = 0.0f;
+    if (cur.s1 >= 0) {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) base[i] = __fmaf_rn(x1[i], 1.0f / (float)P, base[i]);
+    }
+    static_for<2, L>([&](auto lc) {
+      constexpr int l = decltype(lc)::value;
+      if (cur.su[l - 2] >= 0) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+          base[i] = __fmaf_rn(xu[l - 2][i], 1.0f / (float)ipow(P, l), base[i]);
+      }
+    });
+    Packed8<Tout> ob;
+    ob.pack(base);
+    Tout* out = dst + (int64_t)e * P * D;
+#pragma unroll
+    for (int r = 0; r < P; ++r) {
+      if (cur.s0[r] >= 0) {  // selected at level 0: its own chain x_0 + x_1/p + ...
+        float acc[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) acc[i] = x0[r][i];
+        if (cur.s1 >= 0) {
+#pragma unroll
+          for (int i = 0; i < 8; ++i) acc[i] = __fmaf_rn(x1[i], 1.0f / (float)P, acc[i]);
+        }
+        static_for<2, L>([&](auto lc) {
+          constexpr int l = decltype(lc)::value;
+          if (cur.su[l - 2] >= 0) {
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+              acc[i] = __fmaf_rn(xu[l - 2][i], 1.0f / (float)ipow(P, l), acc[i]);
+          }
+        });
+        Packed8<Tout> pr;
+        pr.pack(acc);
+        pr.store(out + r * D);
+      } else {
+        ob.store(out + r * D);
+      }
+    }
+    if (k + 1 < NE) cur = nxt;
+  }
+}
+
 // ------------------------------------------- backward softmax statistics
 // Tile-padded so that one bulk copy brings a 128-row tile's statistics: for
 // unit u and tile t (T tiles per unit), row r = 128 t + c of the sub-sequence,
@@ -1035,6 +1146,20 @@ template <typename Tout, int D>
 cudaError_t gather_bwd_t(const Geom& g, const float* dqs, const float* dks, const float* dvs,
                          const int32_t* slot, Tout* dq, Tout* dk, Tout* dv, cudaStream_t st) {
   const Lv lv = make_lv(g);
+  if (g.L >= 2 && (g.p == 2 || g.p == 4)) {  // p known at compile time, one array per thread
+    const unsigned bxp = blocks_for(g.N / g.p, (128 / (D / 8)) * kGatherEntries);
+    return with_levels(g.L, [&](auto lc) {
+      constexpr int LL = decltype(lc)::value;
+      if constexpr (LL >= 2) {
+        per_unit_chunks(g.U, [&](int64_t u0, unsigned nu) {
+          if (g.p == 4)
+            k_gather_bwd_pp<Tout, D, LL, 4><<<dim3(bxp, nu, 3), 128, 0, st>>>(dqs, dks, dvs, slot, dq, dk, dv, lv, u0);
+          else
+            k_gather_bwd_pp<Tout, D, LL, 2><<<dim3(bxp, nu, 3), 128, 0, st>>>(dqs, dks, dvs, slot, dq, dk, dv, lv, u0);
+        });
+      }
+    });
+  }
   const int R = tokens_per_thread(g);
   const unsigned bx = blocks_for(g.N / R, 256 / (D / 8));
   return with_tokens(R, [&](auto rc) {
