@@ -48,14 +48,14 @@ PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # kernel that evicts them, so a stage that writes more than L2 holds reads low.
 MEASURED_TRAFFIC = {  # workload: {stage: (bytes per launch, sources, sha1[:16])}
     "pretrain": {
-        "pyramid_score": (9.6660e+08, ('k_pyramid.cu', 'lh_internal.cuh'), "0fe10c5f7c160b21"),
-        "topk": (8.4000e+06, ('k_topk.cu', 'lh_internal.cuh'), "956b5193a7a7a1b3"),
-        "gather": (9.6400e+07, ('k_gather_scatter.cu', 'lh_internal.cuh'), "a9918a7354a15cac"),
-        "scatter": (1.7010e+08, ('k_gather_scatter.cu', 'lh_internal.cuh'), "a9918a7354a15cac"),
-        "scatter_bwd": (2.2560e+08, ('k_gather_scatter.cu', 'lh_internal.cuh'), "a9918a7354a15cac"),
-        "gather_bwd": (6.5040e+08, ('k_gather_scatter.cu', 'lh_internal.cuh'), "a9918a7354a15cac"),
-        "attn_fwd": (5.0500e+07, ('k_attn_tc.cu', 'tc_common.cuh'), "aec417ec05129960"),
-        "attn_bwd": (1.9450e+08, ('k_attn_tc.cu', 'tc_common.cuh', 'k_gather_scatter.cu', 'lh_internal.cuh'), "c1ad5e42a553ab4f"),
+        "pyramid_score": (9.6650e+08, ('k_pyramid.cu', 'lh_internal.cuh'), "72509e86a0d1d4f2"),
+        "topk": (8.4000e+06, ('k_topk.cu', 'lh_internal.cuh'), "4bd7debfe01a2b3a"),
+        "gather": (9.6500e+07, ('k_gather_scatter.cu', 'lh_internal.cuh'), "74de98f31e4efd8e"),
+        "scatter": (1.7000e+08, ('k_gather_scatter.cu', 'lh_internal.cuh'), "74de98f31e4efd8e"),
+        "scatter_bwd": (2.2560e+08, ('k_gather_scatter.cu', 'lh_internal.cuh'), "74de98f31e4efd8e"),
+        "gather_bwd": (6.5830e+08, ('k_gather_scatter.cu', 'lh_internal.cuh'), "74de98f31e4efd8e"),
+        "attn_fwd": (5.0400e+07, ('k_attn_tc.cu', 'tc_common.cuh'), "205c351e0fdd8680"),
+        "attn_bwd": (1.9440e+08, ('k_attn_tc.cu', 'tc_common.cuh', 'k_gather_scatter.cu', 'lh_internal.cuh'), "d71b4fd6b65b99dc"),
     },
 }
 
