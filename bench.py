@@ -348,6 +348,44 @@ def extra_leg(lh, name, args, rk, dev, peaks, peaks_src, dense=False):
     return leg
 
 
+def block_leg(w, args, dev, steps=5, warmup=3):
+    """A causal self-attention block (fused Q/K/V projection, the layer, output
+    projection; long_context_lh_b200.block) on the workload's shape, d_model = H*d:
+    one training step = forward, backward of a mean-square loss and an SGD update,
+    timed with CUDA events; beside it the same block with dense causal SDPA."""
+    from long_context_lh_b200.block import DenseBlock, LighthouseBlock
+    torch.manual_seed(0)
+    dm = w.H * w.d
+    x = torch.randn((w.B, w.N, dm), device=dev).to(torch.bfloat16)
+    out = {"d_model": dm, "heads": w.H, "tokens": w.B * w.N}
+    for name, cls in (("lighthouse", LighthouseBlock), ("dense", DenseBlock)):
+        blk = cls(dm, w.H, w.p, w.L, w.S, device=dev)
+        opt = torch.optim.SGD(blk.parameters(), lr=1e-3)
+
+        def step():
+            opt.zero_grad(set_to_none=True)
+            y = blk(x)
+            (y.float() ** 2).mean().backward()
+            opt.step()
+
+        n = steps if name == "lighthouse" else max(1, min(steps, 2))
+        for _ in range(warmup if name == "lighthouse" else 1):
+            step()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(n):
+            step()
+        e1.record()
+        torch.cuda.synchronize()
+        ms = e0.elapsed_time(e1) / n
+        out[name] = {"ms_per_step": ms, "tokens_per_s": w.B * w.N / (ms / 1e3)}
+        del blk, opt
+        torch.cuda.empty_cache()
+    out["speedup_vs_dense"] = out["dense"]["ms_per_step"] / out["lighthouse"]["ms_per_step"]
+    return out
+
+
 def run_sweep(args, rk):
     """Forward-only per-stage times over the hyperparameter sweep (p, L, S) at the
     pretraining shape; one JSON line."""
@@ -429,6 +467,8 @@ def run_ours(args, rk):
     if dense and "fwd_ms" in dense:
         out["speedup_vs_dense"] = {"fwd": dense["fwd_ms"] / ms_fwd, "fwd_bwd": dense["fwd_bwd_ms"] / ms_step}
     out.update(extra)
+    if world == 1 and not args.heads and args.workload == "pretrain" and args.block:
+        out["attention_block"] = block_leg(w, args, dev)
     if rank == 0:
         out["clocks"] = clk.summary()
         if not args.no_cpu:
@@ -625,6 +665,8 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--also", default="long,extreme",
                     help="further workloads measured beside the main line (1 GPU; '' for none)")
+    ap.add_argument("--block", type=int, default=1,
+                    help="1: also time a training step of the attention block (1 GPU)")
     ap.add_argument("--sweep", action="store_true",
                     help="forward-only per-stage times over the p x L x S sweep (one JSON line)")
     args = ap.parse_args()

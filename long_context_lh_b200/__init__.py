@@ -6,7 +6,7 @@ inputs; `long_context_lh_b200.build` compiles the CUDA sources in-tree.
 The binding is imported lazily so that the input generator and the build step
 work on a host without the built library.
 """
-__all__ = ["lighthouse", "synth", "build"]
+__all__ = ["lighthouse", "synth", "build", "block"]
 
 
 def __getattr__(name):

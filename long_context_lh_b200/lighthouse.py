@@ -411,15 +411,16 @@ def backward(saved: Saved, dO, stream=None):
 
 
 class LighthouseAttention(torch.autograd.Function):
-    """autograd wrapper: y = LighthouseAttention.apply(q, k, v, p, L, S, scale)."""
+    """autograd wrapper: y = LighthouseAttention.apply(q, k, v, p, L, S, scale, options)."""
 
     @staticmethod
-    def forward(ctx, q, k, v, p, L, S, scale=0.0):
-        o, saved = forward(q.contiguous(), k.contiguous(), v.contiguous(), p, L, S, scale)
+    def forward(ctx, q, k, v, p, L, S, scale=0.0, options=None):
+        o, saved = forward(q.contiguous(), k.contiguous(), v.contiguous(), p, L, S, scale,
+                           options=options)
         ctx.saved_state = saved
         return o
 
     @staticmethod
     def backward(ctx, dO):
         dq, dk, dv = backward(ctx.saved_state, dO.contiguous())
-        return dq, dk, dv, None, None, None, None
+        return dq, dk, dv, None, None, None, None, None

@@ -535,3 +535,51 @@ def test_extreme_context_full_size():
     """The one-GPU extreme workload (H=8, N=1,048,576, d=128, L=6, S=16,384, log-normal
     token norms), as the bench runs it."""
     check_full_size("extreme", device_draw=True)
+
+
+def test_attention_block_matches_oracle_chain():
+    """The block (projections + Lighthouse + output projection, autograd) against
+    the same chain with the attention and its backward taken from the oracle in
+    fp64 and the projections applied by hand: the output and the gradients of the
+    input and of both weight matrices."""
+    from long_context_lh_b200.block import LighthouseBlock
+    torch.manual_seed(3)
+    B, N, H, d, p, L, S = 1, 2048, 2, 64, 4, 3, 384
+    blk = LighthouseBlock(H * d, H, p, L, S, device=DEV)
+    with torch.no_grad():
+        for w in (blk.wqkv.weight, blk.wo.weight):
+            w.copy_(torch.randn_like(w, dtype=torch.float32) / np.sqrt(H * d))
+    x = torch.randn((B, N, H * d), device=DEV).to(torch.bfloat16).requires_grad_(True)
+    g = torch.randn((B, N, H * d), device=DEV).to(torch.bfloat16)
+    y = blk(x)
+    y.backward(g)
+    torch.cuda.synchronize()
+    # the chain by hand, attention from the oracle (fp64); inputs to it from torch only
+    s = oracle.Shape(B, H, N, d, p, L, S)
+    with torch.no_grad():
+        q, k, v = (t.float().cpu().numpy() for t in blk.split_heads(x))
+        wo = f64(blk.wo.weight)
+        wqkv = f64(blk.wqkv.weight)
+    ref = oracle.forward(s, q, k, v)
+    o = ref["o"]                                            # [B, H, N, d]
+    o_flat = o.transpose(0, 2, 1, 3).reshape(B, N, H * d)
+    y_ref = o_flat @ wo.T
+    check_attn(f64(y), y_ref, "block output")
+    gg = f64(g)
+    dO = (gg @ wo).reshape(B, N, H, d).transpose(0, 2, 1, 3)
+    bref = oracle.backward(s, ref, dO)
+    dqkv = np.stack([bref["dq"], bref["dk"], bref["dv"]])   # [3, B, H, N, d]
+    dqkv_flat = dqkv.transpose(1, 3, 0, 2, 4).reshape(B, N, 3 * H * d)
+    x64 = f64(x)
+    check_attn(f64(x.grad), dqkv_flat @ wqkv, "dx")
+    # The weight gradients are sums over all N tokens of (attention output or gradient)
+    # x (input or upstream gradient): per-element attention errors within the bound
+    # above accumulate like sqrt(N) in each entry, so these are checked in norm --
+    # mean relative error <= 1e-2 (as every attention result) and the largest
+    # error within 2% of the largest entry.
+    for name, got, ref_w in (
+            ("dWqkv", blk.wqkv.weight.grad, dqkv_flat.reshape(-1, 3 * H * d).T @ x64.reshape(-1, H * d)),
+            ("dWo", blk.wo.weight.grad, gg.reshape(-1, H * d).T @ o_flat.reshape(-1, H * d))):
+        err = np.abs(f64(got) - ref_w)
+        assert err.mean() / np.abs(ref_w).mean() <= 1e-2, f"{name}: mean relative error"
+        assert err.max() <= 2e-2 * np.abs(ref_w).max(), f"{name}: max err {err.max():.3g}"
