@@ -459,11 +459,14 @@ cudaError_t launch_topk(const Geom& g, const float* score, int32_t* idx, int32_t
   const int64_t sper = (spans + CL - 1) / CL;
   int64_t per_span = 0;
   for (int l = 0; l < g.L; ++l) per_span += Ptop / g.pw[l];
+  // Shared memory holds the CTA's keys if they fit (every pass reads them), and
+  // the per-token masks of the compaction only if both fit (else pass B
+  // recomputes them, cheaply, from the cached keys).
   const int64_t key_bytes = sper * per_span * 4;
   int64_t mask_bytes = (sper * Ptop * 2 + 15) / 16 * 16;  // 16 bits per token
-  const int masks = mask_bytes <= kKeyCacheBytes ? 1 : 0;   // else pass B recomputes them
+  const int cached = key_bytes <= kKeyCacheBytes ? 1 : 0;
+  const int masks = (cached ? key_bytes : 0) + mask_bytes <= kKeyCacheBytes ? 1 : 0;
   if (!masks) mask_bytes = 0;
-  const int cached = key_bytes + mask_bytes <= kKeyCacheBytes ? 1 : 0;
   const int kcap = cached ? (int)(key_bytes / 4) : 0;
   const size_t dyn = (size_t)kcap * 4 + (size_t)mask_bytes;
   auto launch = [&](auto clc) -> cudaError_t {
