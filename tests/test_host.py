@@ -103,3 +103,38 @@ def test_status_strings():
 def test_attention_impl_switch_roundtrip():
     prev = lh.lh_set_attention_impl(1)
     assert lh.lh_set_attention_impl(prev) == 1
+
+
+def test_options_are_checked_on_the_host():
+    """lh_options: NULL or zero is the default; keep_coarsest needs N/p^(L-1) <= S;
+    modes and the reserved word are range-checked; the _ex calls reject bad
+    options before any launch (and the same argument errors as the plain calls)."""
+    lib = lh._lib()
+    shp = S(1, 2, 4096, 64, 4, 4, 512)             # 64 coarsest entries <= 512
+    assert lh.lh_validate_options(shp, None) == lh.LH_OK
+    assert lh.lh_validate_options(shp, lh.make_options()) == lh.LH_OK
+    for sm in (0, 1, 2):
+        for cm in (0, 1, 2):
+            assert lh.lh_validate_options(shp, lh.make_options(True, sm, cm)) == lh.LH_OK
+    tight = S(1, 2, 4096, 64, 4, 2, 512)           # 1024 coarsest entries > 512
+    assert lh.lh_validate_options(tight, lh.make_options(True)) == lh.LH_ERR_SHAPE
+    assert lh.lh_validate_options(tight, lh.make_options(False)) == lh.LH_OK
+    for bad in (lh.make_options(False, 3), lh.make_options(False, -1), lh.make_options(False, 0, 3)):
+        assert lh.lh_validate_options(shp, bad) == lh.LH_ERR_INVALID_ARG
+    o = lh.make_options()
+    o.keep_coarsest = 2
+    assert lh.lh_validate_options(shp, o) == lh.LH_ERR_INVALID_ARG
+    o = lh.make_options()
+    o.reserved = 1
+    assert lh.lh_validate_options(shp, o) == lh.LH_ERR_INVALID_ARG
+    assert lh.lh_validate_options(S(d=96), None) == lh.LH_ERR_SHAPE
+    p = 1 << 20
+    ob = ctypes.byref(lh.make_options(False, 5))
+    assert lib.lh_forward_ex(ctypes.byref(shp), lh.LH_BF16, p, p, p, 0.0, p, p, p, 1 << 40, ob,
+                             None) == lh.LH_ERR_INVALID_ARG
+    assert lib.lh_topk_select_ex(ctypes.byref(tight), p, p, p, p, None, 0,
+                                 ctypes.byref(lh.make_options(True)), None) == lh.LH_ERR_SHAPE
+    assert lib.lh_backward_ex(ctypes.byref(shp), lh.LH_BF16, p, p, 0.0, p, p, p, p, 16,
+                              None, None) == lh.LH_ERR_WORKSPACE
+    assert lib.lh_scatter_back_ex(ctypes.byref(shp), lh.LH_BF16, p, p, p + 4, None, None,
+                                  None) == lh.LH_ERR_INVALID_ARG
