@@ -45,6 +45,9 @@ constexpr int64_t kKeyCacheBytes = 180 * 1024;
 // Key bits of a kept coarsest entry: +inf, above every finite score; ties among
 // kept entries go to the lower gid like any other tie.
 constexpr uint32_t kTopBits = 0x7F800000u;
+// At most this many entries tied at the threshold are resolved from a list;
+// more take the radix passes over the gids.
+constexpr int kTieCap = 256;
 
 struct TopkParams {
   int32_t N, M;  // within-unit sizes fit 32 bits (M < 2^31 is a checked limit)
@@ -178,6 +181,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   __shared__ uint32_t sh[4];
   __shared__ uint32_t warp_tot[kWarps];
   __shared__ uint32_t cta_total;
+  __shared__ uint32_t tie_n;                 // this CTA's keys equal to the threshold T
+  __shared__ uint32_t tie_gid[kTieCap];      // ... their gids
+  __shared__ uint32_t all_tie[kTieCap];      // the cluster's, gathered
   extern __shared__ __align__(16) uint32_t skey[];  // the CTA's keys, level by level (cached), kcap words
   // then per token of the CTA: bits 0-7 the selected levels ending at it,
   // bits 8-15 all levels ending at it (written by the counting pass)
@@ -274,7 +280,54 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   // ---- 2. among entries scoring exactly T, the need smallest gids
   int64_t gid_thr = INT64_MAX;
-  if (need < ties) {
+  if (need < ties && ties <= (uint32_t)kTieCap) {
+    // Few ties (the usual case: one max-inheritance chain, at most L entries):
+    // each CTA lists the gids of its keys equal to T, every CTA reads the
+    // cluster's lists through DSMEM and takes the need-th smallest directly.
+    if (threadIdx.x == 0) tie_n = 0;
+    __syncthreads();
+    auto add_tie = [&](uint32_t gid) {
+      const uint32_t k = atomicAdd(&tie_n, 1u);
+      if (k < (uint32_t)kTieCap) tie_gid[k] = gid;
+    };
+    if (cached) {
+      for (int32_t i = (int32_t)threadIdx.x; i < nk; i += kThreads) {
+        if (skey[i] != T) continue;
+        int32_t gb = prm.off[0] + jb[0] - kb[0];
+#pragma unroll
+        for (int l = 1; l < kMaxLevels; ++l)
+          if (l < prm.L && i >= kb[l]) gb = prm.off[l] + jb[l] - kb[l];
+        add_tie((uint32_t)(gb + i));
+      }
+    } else {
+#pragma unroll
+      for (int l = 0; l < kMaxLevels; ++l)
+        for (int32_t j = (int32_t)threadIdx.x; j < nl[l]; j += kThreads)
+          if (key_of(l, j) == T) add_tie((uint32_t)(prm.off[l] + jb[l] + j));
+    }
+    cluster.sync();  // every CTA's list is complete
+    // the cluster's ties, CTA by CTA (their total is `ties`, at most kTieCap)
+    if (threadIdx.x < (unsigned)ties) {
+      uint32_t i = threadIdx.x;
+      int r = 0;
+      for (; r < CL; ++r) {
+        const uint32_t nr = *cluster.map_shared_rank(&tie_n, r);
+        if (i < nr) break;
+        i -= nr;
+      }
+      all_tie[threadIdx.x] = r < CL ? cluster.map_shared_rank(tie_gid, r)[i] : 0xffffffffu;
+    }
+    __syncthreads();
+    if (threadIdx.x < (unsigned)ties) {  // gids are distinct: exactly one has rank need - 1
+      const uint32_t gme = all_tie[threadIdx.x];
+      uint32_t rank = 0;
+      for (uint32_t j = 0; j < ties; ++j) rank += all_tie[j] < gme ? 1u : 0u;
+      if (rank == need - 1) sh[3] = gme;
+    }
+    __syncthreads();
+    gid_thr = (int64_t)sh[3];
+    need = 0;
+  } else if (need < ties) {
     int nbits = 1;
     while (nbits < 31 && ((int64_t)1 << nbits) < prm.M) ++nbits;
     uint32_t gprefix = 0, gmask = 0;
