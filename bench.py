@@ -49,13 +49,13 @@ PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 MEASURED_TRAFFIC = {  # workload: {stage: (bytes per launch, sources, sha1[:16])}
     "pretrain": {
         "pyramid_score": (9.6650e+08, ('k_pyramid.cu', 'lh_internal.cuh'), "72509e86a0d1d4f2"),
-        "topk": (8.4000e+06, ('k_topk.cu', 'lh_internal.cuh'), "4bd7debfe01a2b3a"),
-        "gather": (9.6500e+07, ('k_gather_scatter.cu', 'lh_internal.cuh'), "74de98f31e4efd8e"),
-        "scatter": (1.7000e+08, ('k_gather_scatter.cu', 'lh_internal.cuh'), "74de98f31e4efd8e"),
+        "topk": (8.4000e+06, ('k_topk.cu', 'lh_internal.cuh'), "56d3e32b77bf9427"),
+        "gather": (9.6800e+07, ('k_gather_scatter.cu', 'lh_internal.cuh'), "74de98f31e4efd8e"),
+        "scatter": (1.6990e+08, ('k_gather_scatter.cu', 'lh_internal.cuh'), "74de98f31e4efd8e"),
         "scatter_bwd": (2.2560e+08, ('k_gather_scatter.cu', 'lh_internal.cuh'), "74de98f31e4efd8e"),
-        "gather_bwd": (6.5830e+08, ('k_gather_scatter.cu', 'lh_internal.cuh'), "74de98f31e4efd8e"),
+        "gather_bwd": (6.5820e+08, ('k_gather_scatter.cu', 'lh_internal.cuh'), "74de98f31e4efd8e"),
         "attn_fwd": (5.0400e+07, ('k_attn_tc.cu', 'tc_common.cuh'), "205c351e0fdd8680"),
-        "attn_bwd": (1.9440e+08, ('k_attn_tc.cu', 'tc_common.cuh', 'k_gather_scatter.cu', 'lh_internal.cuh'), "d71b4fd6b65b99dc"),
+        "attn_bwd": (1.9430e+08, ('k_attn_tc.cu', 'tc_common.cuh', 'k_gather_scatter.cu', 'lh_internal.cuh'), "d71b4fd6b65b99dc"),
     },
 }
 
