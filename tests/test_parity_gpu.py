@@ -10,6 +10,8 @@ Tolerances (written here, used everywhere below):
     (2e-2 absolute plus half a bf16 ulp for tensors stored in bf16), and
     mean|err| / mean|ref| <= 1e-2.
 """
+import ctypes
+
 import numpy as np
 import pytest
 import torch
@@ -583,3 +585,32 @@ def test_attention_block_matches_oracle_chain():
         err = np.abs(f64(got) - ref_w)
         assert err.mean() / np.abs(ref_w).mean() <= 1e-2, f"{name}: mean relative error"
         assert err.max() <= 2e-2 * np.abs(ref_w).max(), f"{name}: max err {err.max():.3g}"
+
+
+def test_non_finite_inputs_complete_and_leave_the_context_usable():
+    """Non-finite inputs give unspecified values but never an error, a hang or a
+    device status: NaN and +-inf rows in q, k, v and dO (the selection works on
+    key bits, every index it produces is in range, every loop has a fixed trip
+    count).  A normal call afterwards still matches the oracle."""
+    w = workload(dtype="bf16", N=4096, S=512, L=3, H=2)
+    x = to_dev(make_inputs(w, "cpu"))
+    for name, val, rows in (("q", float("nan"), (5, 77)), ("k", float("inf"), (100,)),
+                            ("v", float("-inf"), (1000,)), ("dO", float("nan"), (3,))):
+        for r in rows:
+            x[name][0, 0, r, :8] = val
+    o, saved = lh.forward(x["q"], x["k"], x["v"], w.p, w.L, w.S)
+    dq, dk, dv = lh.backward(saved, x["dO"])
+    torch.cuda.synchronize()
+    code = ctypes.c_uint32(0)
+    assert lh._lib().lh_read_device_status(None, ctypes.byref(code)) == lh.LH_OK
+    assert code.value == 0
+    idx = lh.saved_view(saved.shape, saved.buf, lh.SAVED_IDX).cpu().numpy()
+    assert idx.min() >= 0 and idx.max() < lh.lh_num_entries(saved.shape)
+    # the context is healthy: a normal call still agrees with the oracle
+    w2 = workload(dtype="bf16", N=2048, S=256, L=3, H=1)
+    xc = make_inputs(w2, "cpu")
+    x2 = to_dev(xc)
+    o2, _ = lh.forward(x2["q"], x2["k"], x2["v"], w2.p, w2.L, w2.S)
+    torch.cuda.synchronize()
+    ref = oracle.forward(oshape(w2), *(xc[n].float().numpy() for n in ("q", "k", "v")))
+    check_attn(f64(o2), ref["o"], "o after non-finite inputs")
