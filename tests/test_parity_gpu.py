@@ -85,6 +85,7 @@ STAGE_CASES = [
     dict(dtype="bf16", N=512, S=1),
     dict(dtype="bf16", p=4, L=5, N=2048, S=300),             # level 4 wider than a 64-row chunk
     dict(p=5, L=4, N=1000, S=100),                            # p^3 = 125 > 64, last chunk ragged
+    dict(B=3, H=2, dtype="bf16", dist="outliers", N=2048, S=256),  # several batch rows
 ]
 
 
@@ -301,7 +302,11 @@ def test_attention_matches_oracle(U, S, d, impl):
 
 
 @pytest.mark.parametrize("case", [dict(), dict(dtype="bf16", dist="outliers", N=8192, S=1024, L=4),
-                                  dict(dtype="bf16", d=128, p=2, L=4, N=2048, S=500)], ids=str)
+                                  dict(dtype="bf16", d=128, p=2, L=4, N=2048, S=500),
+                                  # several batch rows: units are (batch, head) pairs
+                                  dict(B=2, H=3, dtype="bf16", dist="outliers", N=4096, S=512, L=3),
+                                  dict(B=2, H=1, dtype="bf16", dist="lognormal", d=128, N=4096, S=640,
+                                       L=4)], ids=str)
 def test_fused_forward_backward_match_oracle(case):
     w = workload(**case)
     xc = make_inputs(w, "cpu")
