@@ -178,101 +178,93 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp == 9) {
     // -------------------------------------------------------------- MMA issuer
-    // The whole warp runs the loop, so the descriptors are warp-uniform (kept in
-    // uniform registers, no per-MMA register moves); lane 0 issues every MMA and
-    // commit.  A descriptor for base + off is the base descriptor plus off / 16
-    // (the 14-bit address field never overflows inside shared memory).
-    constexpr uint32_t idS = idesc_f16(128, 128, false);
-    constexpr uint32_t idPV = idesc_f16(128, D, true);
-    const uint64_t dQ = desc_kmajor(smem_u32(sQ)), dK = desc_kmajor(smem_u32(sK));
-    const uint64_t dV = desc_mnmajor(smem_u32(sV), 16384);
-    auto issue_s = [&](int t, int j) {  // S_t = Q_t K_j^T
-      const uint64_t q = dQ + (uint64_t)((t * Lt::kTile) >> 4);
-      const uint64_t k = dK + (uint64_t)(((j % KS) * Lt::kTile) >> 4);
-      if (lane == 0) {
+    // Lane 0 alone waits, issues every MMA and commit.  A descriptor for
+    // base + off is the base descriptor plus off / 16 (the 14-bit address field
+    // never overflows inside shared memory).
+    if (lane == 0) {
+      constexpr uint32_t idS = idesc_f16(128, 128, false);
+      constexpr uint32_t idPV = idesc_f16(128, D, true);
+      const uint64_t dQ = desc_kmajor(smem_u32(sQ)), dK = desc_kmajor(smem_u32(sK));
+      const uint64_t dV = desc_mnmajor(smem_u32(sV), 16384);
+      auto issue_s = [&](int t, int j) {  // S_t = Q_t K_j^T
+        const uint64_t q = dQ + (uint64_t)((t * Lt::kTile) >> 4);
+        const uint64_t k = dK + (uint64_t)(((j % KS) * Lt::kTile) >> 4);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint64_t off = (uint64_t)((((kk >> 2) * 16384) + ((kk & 3) * 32)) >> 4);
           umma_f16(tmem + t * 128, q + off, k + off, idS, kk > 0);
         }
         umma_commit(&bars->s_full[t]);
-      }
-      __syncwarp();
-    };
-    auto issue_pv = [&](int t, int j) {  // O_t += P_t(j) V_j, P_t from TMEM
-      const uint64_t v = dV + (uint64_t)(((j % KS) * Lt::kTile) >> 4);
-      const uint32_t pt = kSepP ? tP + t * 64 : tmem + t * 128;
-      if (lane == 0) {
+      };
+      auto issue_pv = [&](int t, int j) {  // O_t += P_t(j) V_j, P_t from TMEM
+        const uint64_t v = dV + (uint64_t)(((j % KS) * Lt::kTile) >> 4);
+        const uint32_t pt = kSepP ? tP + t * 64 : tmem + t * 128;
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
           umma_f16_ta(tO + t * D, pt + 8 * kk, v + (uint64_t)((kk * 2048) >> 4), idPV,
                       (j > 0 || kk > 0));
         umma_commit(&bars->pv_done[t]);
+      };
+      bool ok = mbar_wait(&bars->q_full, 0, abort, kStatus) &&
+                mbar_wait(&bars->kv_full[0], 0, abort, kStatus);
+      if (ok) {
+        tc_fence_after();
+        issue_s(0, 0);
+        if (nB > 0) issue_s(1, 0);
       }
-      __syncwarp();
-    };
-    bool ok = warp_wait(&bars->q_full, 0, abort, kStatus) &&
-              warp_wait(&bars->kv_full[0], 0, abort, kStatus);
-    if (ok) {
-      tc_fence_after();
-      issue_s(0, 0);
-      if (nB > 0) issue_s(1, 0);
-    }
-    if constexpr (kSepP) {
-      // per key tile j: S_A(j+1) once S_A(j) is read, O_A += P_A(j) V_j once P_A(j)
-      // is written, then the same for tile B; the waits follow the order in which
-      // the row work produces these events
-      for (int j = 0; ok && j < nA; ++j) {
+      if constexpr (kSepP) {
+        // per key tile j: S_A(j+1) once S_A(j) is read, O_A += P_A(j) V_j once P_A(j)
+        // is written, then the same for tile B; the waits follow the order in which
+        // the row work produces these events
+        for (int j = 0; ok && j < nA; ++j) {
+          const int st = j % KS;
+          if (j + 1 < nA) {
+            if (!(ok = mbar_wait(&bars->s_free[0], j & 1, abort, kStatus))) break;
+            if (!(ok = mbar_wait(&bars->kv_full[(j + 1) % KS], ((j + 1) / KS) & 1, abort, kStatus))) break;
+            tc_fence_after();
+            issue_s(0, j + 1);
+          }
+          if (!(ok = mbar_wait(&bars->p_full[0], j & 1, abort, kStatus))) break;
+          tc_fence_after();
+          issue_pv(0, j);
+          if (j < nB) {
+            if (j + 1 < nB) {  // K_{j+1} is in place (waited for above: j + 1 < nB <= nA)
+              if (!(ok = mbar_wait(&bars->s_free[1], j & 1, abort, kStatus))) break;
+              tc_fence_after();
+              issue_s(1, j + 1);
+            }
+            if (!(ok = mbar_wait(&bars->p_full[1], j & 1, abort, kStatus))) break;
+            tc_fence_after();
+            issue_pv(1, j);
+          }
+          umma_commit(&bars->kv_empty[st]);  // K_j, V_j no longer needed
+        }
+      }
+      for (int j = 0; !kSepP && ok && j < nA; ++j) {
         const int st = j % KS;
-        if (j + 1 < nA) {
-          if (!(ok = warp_wait(&bars->s_free[0], j & 1, abort, kStatus))) break;
-          if (!(ok = warp_wait(&bars->kv_full[(j + 1) % KS], ((j + 1) / KS) & 1, abort, kStatus))) break;
+        const bool next = j + 1 < nA;
+        // tile A: its product with V_j, then (S_A buffer free again) its next scores
+        if (!(ok = mbar_wait(&bars->p_full[0], j & 1, abort, kStatus))) break;
+        tc_fence_after();
+        issue_pv(0, j);
+        if (next) {
+          if (!(ok = mbar_wait(&bars->kv_full[(j + 1) % KS], ((j + 1) / KS) & 1, abort, kStatus))) break;
           tc_fence_after();
           issue_s(0, j + 1);
         }
-        if (!(ok = warp_wait(&bars->p_full[0], j & 1, abort, kStatus))) break;
-        tc_fence_after();
-        issue_pv(0, j);
+        // tile B likewise
         if (j < nB) {
-          if (j + 1 < nB) {  // K_{j+1} is in place (waited for above: j + 1 < nB <= nA)
-            if (!(ok = warp_wait(&bars->s_free[1], j & 1, abort, kStatus))) break;
-            tc_fence_after();
-            issue_s(1, j + 1);
-          }
-          if (!(ok = warp_wait(&bars->p_full[1], j & 1, abort, kStatus))) break;
+          if (!(ok = mbar_wait(&bars->p_full[1], j & 1, abort, kStatus))) break;
           tc_fence_after();
           issue_pv(1, j);
+          if (j + 1 < nB) issue_s(1, j + 1);
         }
-        if (lane == 0) umma_commit(&bars->kv_empty[st]);  // K_j, V_j no longer needed
-        __syncwarp();
+        umma_commit(&bars->kv_empty[st]);  // K_j, V_j no longer needed
       }
+      umma_commit(&bars->mma_done);
+      // every MMA issued has completed before TMEM is freed, aborted or not
+      mbar_wait(&bars->mma_done, 0, abort, kStatus, false);
     }
-    for (int j = 0; !kSepP && ok && j < nA; ++j) {
-      const int st = j % KS;
-      const bool next = j + 1 < nA;
-      // tile A: its product with V_j, then (S_A buffer free again) its next scores
-      if (!(ok = warp_wait(&bars->p_full[0], j & 1, abort, kStatus))) break;
-      tc_fence_after();
-      issue_pv(0, j);
-      if (next) {
-        if (!(ok = warp_wait(&bars->kv_full[(j + 1) % KS], ((j + 1) / KS) & 1, abort, kStatus))) break;
-        tc_fence_after();
-        issue_s(0, j + 1);
-      }
-      // tile B likewise
-      if (j < nB) {
-        if (!(ok = warp_wait(&bars->p_full[1], j & 1, abort, kStatus))) break;
-        tc_fence_after();
-        issue_pv(1, j);
-        if (j + 1 < nB) issue_s(1, j + 1);
-      }
-      if (lane == 0) umma_commit(&bars->kv_empty[st]);  // K_j, V_j no longer needed
-      __syncwarp();
-    }
-    if (lane == 0) umma_commit(&bars->mma_done);
-    __syncwarp();
-    // every MMA issued has completed before TMEM is freed, aborted or not
-    (void)__all_sync(0xffffffffu, mbar_wait(&bars->mma_done, 0, abort, kStatus, false));
   } else {
     // -------------------- row work: one thread per row of its tile, all 128 keys
     // P is formed against a running reference max m_ref, and O_t is rescaled in
