@@ -41,13 +41,6 @@ constexpr float kLog2e = 1.4426950408889634f;
 constexpr int kThreads = 320;
 constexpr uint32_t kTmemCols = 512;
 
-// Two tcgen05.ld of 32 columns each, then one wait.
-__device__ __forceinline__ void tmem_ld64(uint32_t taddr, uint32_t (&a)[32], uint32_t (&b)[32]) {
-  tmem_ld32(taddr, a);
-  tmem_ld32(taddr + 32, b);
-  tmem_ld_wait();
-}
-
 __device__ __forceinline__ void store_row_half(uint8_t* tile_half, int r, const uint32_t (&pk)[32]) {
   // one 64-column half of a row of a 128-byte-swizzled fp16 tile: 8 chunks of 16 B
 #pragma unroll
@@ -550,20 +543,25 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       constexpr uint32_t idS = idesc_f16(128, 128, false);
       constexpr uint32_t idAcc = idesc_f16(128, D, true);
-      const uint32_t aK = smem_u32(sK), aV = smem_u32(sV), aQ = smem_u32(sQ), aDO = smem_u32(sDO);
-      const uint32_t aPT = smem_u32(sPT), aDST = smem_u32(sDST);
+      // a descriptor for base + off is the base descriptor plus off / 16 (the
+      // 14-bit address field never overflows inside shared memory)
+      const uint64_t dK = desc_kmajor(smem_u32(sK)), dV = desc_kmajor(smem_u32(sV));
+      const uint64_t dQk = desc_kmajor(smem_u32(sQ)), dDOk = desc_kmajor(smem_u32(sDO));
+      const uint64_t dQm = desc_mnmajor(smem_u32(sQ), 16384), dDOm = desc_mnmajor(smem_u32(sDO), 16384);
+      const uint64_t dPT = desc_kmajor(smem_u32(sPT)), dDST = desc_kmajor(smem_u32(sDST));
       auto issue_grads = [&](int t) {  // dV += P^T dO_t, dK += dS^T Q_t
         const int st = t % STG;
+        const uint64_t so = (uint64_t)((st * Lt::kTile) >> 4);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
-          const uint32_t a = (kk >> 2) * 16384 + (kk & 3) * 32;
-          const uint32_t b = st * Lt::kTile + kk * 2048;
+          const uint64_t a = (uint64_t)((((kk >> 2) * 16384) + ((kk & 3) * 32)) >> 4);
+          const uint64_t b = so + (uint64_t)((kk * 2048) >> 4);
           if constexpr (kTmemP) {
-            umma_f16_ta(tDV, tPT + 8 * kk, desc_mnmajor(aDO + b, 16384), idAcc, (t > 0 || kk > 0));
-            umma_f16_ta(tDK, tDST + 8 * kk, desc_mnmajor(aQ + b, 16384), idAcc, (t > 0 || kk > 0));
+            umma_f16_ta(tDV, tPT + 8 * kk, dDOm + b, idAcc, (t > 0 || kk > 0));
+            umma_f16_ta(tDK, tDST + 8 * kk, dQm + b, idAcc, (t > 0 || kk > 0));
           } else {
-            umma_f16(tDV, desc_kmajor(aPT + a), desc_mnmajor(aDO + b, 16384), idAcc, (t > 0 || kk > 0));
-            umma_f16(tDK, desc_kmajor(aDST + a), desc_mnmajor(aQ + b, 16384), idAcc, (t > 0 || kk > 0));
+            umma_f16(tDV, dPT + a, dDOm + b, idAcc, (t > 0 || kk > 0));
+            umma_f16(tDK, dDST + a, dQm + b, idAcc, (t > 0 || kk > 0));
           }
         }
         umma_commit(&bars->pdone);
@@ -582,11 +580,12 @@ __global__ void __launch_bounds__(kThreads, 1)
              (t == 0 || mbar_wait(&bars->st_free, (t - 1) & 1, abort, kStatus));
         if (!ok) break;
         tc_fence_after();
+        const uint64_t so = (uint64_t)((st * Lt::kTile) >> 4);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-          umma_f16(tST, desc_kmajor(aK + off), desc_kmajor(aQ + st * Lt::kTile + off), idS, kk > 0);
-          umma_f16(tDPT, desc_kmajor(aV + off), desc_kmajor(aDO + st * Lt::kTile + off), idS, kk > 0);
+          const uint64_t off = (uint64_t)((((kk >> 2) * 16384) + ((kk & 3) * 32)) >> 4);
+          umma_f16(tST, dK + off, dQk + so + off, idS, kk > 0);
+          umma_f16(tDPT, dV + off, dDOk + so + off, idS, kk > 0);
         }
         umma_commit(&bars->s_full);
         if (STG > 1 && t > 0) {
@@ -819,15 +818,19 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       constexpr uint32_t idS = idesc_f16(128, 128, false);
       constexpr uint32_t idAcc = idesc_f16(128, D, true);
-      const uint32_t aQ = smem_u32(sQ), aDO = smem_u32(sDO), aK = smem_u32(sK), aV = smem_u32(sV);
+      // base descriptors plus offset / 16, as in the dK/dV kernel
+      const uint64_t dQ = desc_kmajor(smem_u32(sQ)), dDO = desc_kmajor(smem_u32(sDO));
+      const uint64_t dK = desc_kmajor(smem_u32(sK)), dV = desc_kmajor(smem_u32(sV));
+      const uint64_t dKm = desc_mnmajor(smem_u32(sK), 16384);
       auto issue_dq = [&](int j) {  // dQ += dS_j K_j, dS_j from TMEM
         const int st = j % STG, b = j & 1;
         if (!mbar_wait(&bars->ds_full[b], (j >> 1) & 1, abort, kStatus)) return false;
         tc_fence_after();
+        const uint64_t so = (uint64_t)((st * Lt::kTile) >> 4);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
-          umma_f16_ta(tDQ, tDS + b * 64 + 8 * kk,
-                      desc_mnmajor(aK + st * Lt::kTile + kk * 2048, 16384), idAcc, (j > 0 || kk > 0));
+          umma_f16_ta(tDQ, tDS + b * 64 + 8 * kk, dKm + so + (uint64_t)((kk * 2048) >> 4), idAcc,
+                      (j > 0 || kk > 0));
         umma_commit(&bars->dsdone[b]);
         umma_commit(&bars->kv_empty[st]);
         return true;
@@ -840,11 +843,12 @@ __global__ void __launch_bounds__(kThreads, 1)
              (j == 0 || mbar_wait(&bars->s_free, (j - 1) & 1, abort, kStatus));
         if (!ok) break;
         tc_fence_after();
+        const uint64_t so = (uint64_t)((st * Lt::kTile) >> 4);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-          umma_f16(tS, desc_kmajor(aQ + off), desc_kmajor(aK + st * Lt::kTile + off), idS, kk > 0);
-          umma_f16(tDP, desc_kmajor(aDO + off), desc_kmajor(aV + st * Lt::kTile + off), idS, kk > 0);
+          const uint64_t off = (uint64_t)((((kk >> 2) * 16384) + ((kk & 3) * 32)) >> 4);
+          umma_f16(tS, dQ + off, dK + so + off, idS, kk > 0);
+          umma_f16(tDP, dDO + off, dV + so + off, idS, kk > 0);
         }
         umma_commit(&bars->s_full);
         if (STG > 1 && j > 0 && !(ok = issue_dq(j - 1))) break;
