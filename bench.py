@@ -54,8 +54,8 @@ MEASURED_TRAFFIC = {  # workload: {stage: (bytes per launch, sources, sha1[:16])
         "scatter": (1.6990e+08, ('k_gather_scatter.cu', 'lh_internal.cuh'), "74de98f31e4efd8e"),
         "scatter_bwd": (2.2560e+08, ('k_gather_scatter.cu', 'lh_internal.cuh'), "74de98f31e4efd8e"),
         "gather_bwd": (6.5820e+08, ('k_gather_scatter.cu', 'lh_internal.cuh'), "74de98f31e4efd8e"),
-        "attn_fwd": (5.0400e+07, ('k_attn_tc.cu', 'tc_common.cuh'), "205c351e0fdd8680"),
-        "attn_bwd": (1.9430e+08, ('k_attn_tc.cu', 'tc_common.cuh', 'k_gather_scatter.cu', 'lh_internal.cuh'), "d71b4fd6b65b99dc"),
+        "attn_fwd": (5.0426e+07, ('k_attn_tc.cu', 'tc_common.cuh'), "65342d0b26370f8f"),
+        "attn_bwd": (1.9414e+08, ('k_attn_tc.cu', 'tc_common.cuh', 'k_gather_scatter.cu', 'lh_internal.cuh'), "6d238bb3c391ff16"),
     },
 }
 
