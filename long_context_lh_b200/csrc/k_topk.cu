@@ -117,7 +117,7 @@ struct Pick {
 
 // Cluster-summed histogram -> digit where the need-th candidate falls.
 // descending: rank digits from the largest value down (scores), else up (gids).
-template <int CL>  // a multiple of 8
+template <int CL>
 __device__ Pick pick_digit(cg::cluster_group& cluster, uint32_t* hist, int nbins, bool descending,
                            uint32_t need, uint32_t* warp_buf, uint32_t* sh) {
   const int per = nbins / kThreads;  // 2 or 1 ordinals per thread
@@ -459,6 +459,37 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 }  // namespace
 
+struct SmemPlan {
+  int cached, masks, kcap;
+  size_t dyn;
+};
+
+// How many clusters of C CTAs (dyn bytes of dynamic shared memory each) this
+// device runs at once; 0 when the query fails.
+template <int C>
+int max_active_clusters(size_t dyn) {
+  auto* kf = k_topk<C>;
+  if (cudaFuncSetAttribute(kf, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dyn) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return 0;
+  }
+  cudaLaunchConfig_t q = {};
+  q.gridDim = dim3((unsigned)C, 1, 1);
+  q.blockDim = dim3(kThreads, 1, 1);
+  q.dynamicSmemBytes = dyn;
+  cudaLaunchAttribute a[1];
+  a[0].id = cudaLaunchAttributeClusterDimension;
+  a[0].val.clusterDim.x = (unsigned)C;
+  a[0].val.clusterDim.y = 1;
+  a[0].val.clusterDim.z = 1;
+  q.attrs = a;
+  q.numAttrs = 1;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, kf, &q) != cudaSuccess) n = 0;
+  (void)cudaGetLastError();
+  return n;
+}
+
 cudaError_t launch_topk(const Geom& g, const float* score, int32_t* idx, int32_t* pos,
                         int32_t* slot, cudaStream_t st) {
   TopkParams prm;
@@ -506,22 +537,55 @@ cudaError_t launch_topk(const Geom& g, const float* score, int32_t* idx, int32_t
     }
     if (state == 1) CL = 16;
   }
-  // keys of one CTA: whole coarsest spans, every level
+  // keys of one CTA: whole coarsest spans, every level.  Shared memory holds
+  // the CTA's keys if they fit (every pass reads them), and the per-token masks
+  // of the compaction only if both fit (else pass B recomputes them, cheaply,
+  // from the cached keys).
   const int64_t Ptop = g.pw[g.L - 1];
   const int64_t spans = g.N / Ptop;
-  const int64_t sper = (spans + CL - 1) / CL;
   int64_t per_span = 0;
   for (int l = 0; l < g.L; ++l) per_span += Ptop / g.pw[l];
-  // Shared memory holds the CTA's keys if they fit (every pass reads them), and
-  // the per-token masks of the compaction only if both fit (else pass B
-  // recomputes them, cheaply, from the cached keys).
-  const int64_t key_bytes = sper * per_span * 4;
-  int64_t mask_bytes = (sper * Ptop * 2 + 15) / 16 * 16;  // 16 bits per token
-  const int cached = key_bytes <= kKeyCacheBytes ? 1 : 0;
-  const int masks = (cached ? key_bytes : 0) + mask_bytes <= kKeyCacheBytes ? 1 : 0;
-  if (!masks) mask_bytes = 0;
-  const int kcap = cached ? (int)(key_bytes / 4) : 0;
-  const size_t dyn = (size_t)kcap * 4 + (size_t)mask_bytes;
+  const auto plan = [&](int cl) -> SmemPlan {
+    const int64_t sper = (spans + cl - 1) / cl;
+    const int64_t key_bytes = sper * per_span * 4;
+    int64_t mask_bytes = (sper * Ptop * 2 + 15) / 16 * 16;  // 16 bits per token
+    SmemPlan sp;
+    sp.cached = key_bytes <= kKeyCacheBytes ? 1 : 0;
+    sp.masks = (sp.cached ? key_bytes : 0) + mask_bytes <= kKeyCacheBytes ? 1 : 0;
+    if (!sp.masks) mask_bytes = 0;
+    sp.kcap = sp.cached ? (int)(key_bytes / 4) : 0;
+    sp.dyn = (size_t)sp.kcap * 4 + (size_t)mask_bytes;
+    return sp;
+  };
+  if (CL == 8) {
+    // A unit is one cluster, and a cluster runs on one GPC: when the device
+    // holds fewer clusters of 8 at once than there are units, a second wave of
+    // clusters doubles the time.  Smaller clusters fit more at once, each CTA
+    // with proportionally more keys: take the size with the fewest waves per
+    // CTA of work, ceil(units / clusters at once) / CL, among those that keep
+    // the keys in shared memory when 8 does (ties to the larger cluster).
+    const int64_t units = g.U < 65535 ? g.U : 65535;
+    const SmemPlan p8 = plan(8);
+    double best = -1.0;
+    int best_cl = 8;
+    const int cands[3] = {8, 6, 4};
+    for (int c : cands) {
+      const SmemPlan pc = plan(c);
+      if (p8.cached && !pc.cached) continue;
+      const int fit = c == 8 ? max_active_clusters<8>(pc.dyn)
+                             : (c == 6 ? max_active_clusters<6>(pc.dyn) : max_active_clusters<4>(pc.dyn));
+      if (fit <= 0) continue;
+      const double cost = (double)((units + fit - 1) / fit) / (double)c;
+      if (best < 0.0 || cost < best) {
+        best = cost;
+        best_cl = c;
+      }
+    }
+    CL = best_cl;
+  }
+  const SmemPlan sp = plan(CL);
+  const int cached = sp.cached, masks = sp.masks, kcap = sp.kcap;
+  const size_t dyn = sp.dyn;
   auto launch = [&](auto clc) -> cudaError_t {
     constexpr int C = decltype(clc)::value;
     auto* kf = k_topk<C>;
@@ -550,7 +614,12 @@ cudaError_t launch_topk(const Geom& g, const float* score, int32_t* idx, int32_t
     }
     return cudaSuccess;
   };
-  return CL == 16 ? launch(std::integral_constant<int, 16>{}) : launch(std::integral_constant<int, 8>{});
+  switch (CL) {
+    case 16: return launch(std::integral_constant<int, 16>{});
+    case 6: return launch(std::integral_constant<int, 6>{});
+    case 4: return launch(std::integral_constant<int, 4>{});
+    default: return launch(std::integral_constant<int, 8>{});
+  }
 }
 
 }  // namespace lh

@@ -86,6 +86,9 @@ STAGE_CASES = [
     dict(dtype="bf16", p=4, L=5, N=2048, S=300),             # level 4 wider than a 64-row chunk
     dict(p=5, L=4, N=1000, S=100),                            # p^3 = 125 > 64, last chunk ragged
     dict(B=3, H=2, dtype="bf16", dist="outliers", N=2048, S=256),  # several batch rows
+    # more units than clusters of 8 CTAs run at once: the selection takes smaller clusters
+    dict(B=2, H=8, dtype="bf16", dist="outliers", N=4096, S=512),
+    dict(B=2, H=12, dtype="bf16", N=4096, S=512),
 ]
 
 
