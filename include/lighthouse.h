@@ -40,8 +40,9 @@
  *   - Q, K, V, O, dO, dQ, dK, dV are [B, H, N, d] in the call's lh_dtype.
  *     The gathered sub-sequence (qs, ks, vs, os, dos) is fp16 (IEEE binary16)
  *     [B, H, S, d]: the tensor-core operands of the attention, 3 more mantissa
- *     bits than bf16; values beyond +-65504 saturate.  Pyramid levels are fp32;
- *     gradients of the sub-sequence are fp32.
+ *     bits than bf16.  Finite values beyond +-65504 are clipped to it and
+ *     reported (LH_STATUS_FP16_SATURATED, lh_read_device_status).  Pyramid
+ *     levels are fp32; gradients of the sub-sequence are fp32.
  *   - The caller allocates and frees every buffer; the library allocates no
  *     device memory and never synchronises the stream (except
  *     lh_read_device_status).  All work is enqueued on `stream` (NULL = the
@@ -74,7 +75,7 @@ typedef enum {
   LH_ERR_UNSUPPORTED = 3,   /* no kernel for this device or configuration */
   LH_ERR_WORKSPACE = 4,     /* workspace smaller than the *_bytes query */
   LH_ERR_CUDA = 5,          /* a CUDA runtime call or launch failed */
-  LH_ERR_DEVICE_STATUS = 6  /* a kernel reported a bounded wait that timed out */
+  LH_ERR_DEVICE_STATUS = 6  /* a kernel set a status bit (lh_read_device_status) */
 } lh_status;
 
 typedef enum { LH_F32 = 0, LH_BF16 = 1 } lh_dtype; /* dtype of Q,K,V,O,dO,dQ,dK,dV */
@@ -186,8 +187,12 @@ lh_status lh_subseq_attn_bwd(const lh_shape* shape, const void* qs, const void* 
  *     shapes return LH_ERR_WORKSPACE before anything is enqueued.
  *   - All calls on one device share that array: calls whose kernels overlap on
  *     the GPU (unordered streams) race; calls ordered on one stream are safe.
- *   - The first call on each device looks up the array's device address and
- *     caches it; make that first call before any stream capture.
+ *   - The first call in each CUDA context of a device (normally one per
+ *     device, and a new one after cudaDeviceReset) looks up the array's device
+ *     address and caches it under that context's id; make that first call
+ *     before any stream capture.
+ *   - It runs the same kernels as lh_subseq_attn_bwd: the results are bitwise
+ *     equal to that call's.
  * Arguments and results as for lh_subseq_attn_bwd, without ws / ws_bytes.  */
 lh_status lh_subseq_attn_bwd_noalloc(const lh_shape* shape, const void* qs, const void* ks,
                                      const void* vs, const void* os, const float* lse,
@@ -229,9 +234,20 @@ lh_status lh_backward(const lh_shape* shape, lh_dtype dtype, const void* saved, 
                       float scale, void* dq, void* dk, void* dv, void* ws, size_t ws_bytes,
                       lh_stream_t stream);
 
-/* Reads and clears the device status word that bounded waits in the kernels
- * set when they give up (synchronises `stream`).  LH_OK or LH_ERR_DEVICE_STATUS;
- * *code (may be NULL) receives the raw word (0 = none). */
+/* Reads and clears the device status words (synchronises `stream`).  LH_OK or
+ * LH_ERR_DEVICE_STATUS; *code (may be NULL) receives the OR of the words, 0
+ * for none, else LH_STATUS_* bits:
+ *   LH_STATUS_ATTN_FWD_TIMEOUT / LH_STATUS_ATTN_BWD_TIMEOUT: a bounded wait in
+ *     an attention kernel gave up (the low bits say which); that call's
+ *     outputs are incomplete;
+ *   LH_STATUS_FP16_SATURATED: a finite value written into the fp16 sub-sequence
+ *     (qs, ks, vs by the gather; dos by the scatter-back adjoint) lay beyond
+ *     +-65504 and was clipped to it.  The selection is unaffected (it is
+ *     computed in fp32 from the inputs); the attention then ran on the clipped
+ *     rows.  Inputs whose pooled rows stay within +-65504 never set it. */
+#define LH_STATUS_ATTN_FWD_TIMEOUT 0x100u
+#define LH_STATUS_ATTN_BWD_TIMEOUT 0x200u
+#define LH_STATUS_FP16_SATURATED 0x400u
 lh_status lh_read_device_status(lh_stream_t stream, uint32_t* code);
 
 /* Selects the attention implementation for subsequent calls on this process:

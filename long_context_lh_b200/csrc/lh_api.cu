@@ -138,16 +138,6 @@ lh_status attn_fwd(const Geom& g, const __half* qs, const __half* ks,
   return cuda_status(launch_attn_fwd_mma(g, qs, ks, vs, scale, os, lse, st));
 }
 
-lh_status attn_bwd(const Geom& g, const __half* qs, const __half* ks,
-                   const __half* vs, const __half* os, const float* lse,
-                   const __half* dos, float scale, float* dqs, float* dks, float* dvs,
-                   float* stats, cudaStream_t st) {
-  LH_TRY(launch_attn_stats(g, os, dos, lse, stats, st));
-  if (attn_bwd_uses_tc())
-    return cuda_status(launch_attn_bwd_tc(g, qs, ks, vs, dos, stats, scale, dqs, dks, dvs, st));
-  return cuda_status(launch_attn_bwd_mma(g, qs, ks, vs, dos, stats, scale, dqs, dks, dvs, st));
-}
-
 // The geometry of a shape with the variant options applied (options validated).
 Geom geom_with(const lh_shape& shape, const lh_options* opt) {
   Geom g = make_geom(shape);
@@ -160,6 +150,17 @@ Geom geom_with(const lh_shape& shape, const lh_options* opt) {
 }
 
 }  // namespace
+
+lh_status attn_bwd(const Geom& g, const __half* qs, const __half* ks,
+                   const __half* vs, const __half* os, const float* lse,
+                   const __half* dos, float scale, float* dqs, float* dks, float* dvs,
+                   float* stats, cudaStream_t st) {
+  LH_TRY(launch_attn_stats(g, os, dos, lse, stats, st));
+  if (attn_bwd_uses_tc())
+    return cuda_status(launch_attn_bwd_tc(g, qs, ks, vs, dos, stats, scale, dqs, dks, dvs, st));
+  return cuda_status(launch_attn_bwd_mma(g, qs, ks, vs, dos, stats, scale, dqs, dks, dvs, st));
+}
+
 }  // namespace lh
 
 using namespace lh;
@@ -174,7 +175,8 @@ const char* lh_status_string(lh_status s) {
     case LH_ERR_UNSUPPORTED: return "LH_ERR_UNSUPPORTED: no kernel for this device/configuration";
     case LH_ERR_WORKSPACE: return "LH_ERR_WORKSPACE: workspace smaller than required";
     case LH_ERR_CUDA: return "LH_ERR_CUDA: a CUDA call or kernel launch failed";
-    case LH_ERR_DEVICE_STATUS: return "LH_ERR_DEVICE_STATUS: a kernel's bounded wait timed out";
+    case LH_ERR_DEVICE_STATUS:
+      return "LH_ERR_DEVICE_STATUS: a kernel reported a timed-out wait or an fp16 saturation";
   }
   return "LH_ERR_UNKNOWN";
 }
@@ -493,9 +495,11 @@ lh_status lh_backward_ex(const lh_shape* shape, lh_dtype dtype, const void* save
 }
 
 lh_status lh_read_device_status(lh_stream_t stream, uint32_t* code) {
-  uint32_t v = 0;
+  uint32_t v = 0, w = 0;
   if (cudaStreamSynchronize(stream) != cudaSuccess) return LH_ERR_CUDA;
   if (device_status_read_clear(&v) != cudaSuccess) return LH_ERR_CUDA;
+  if (subseq_status_read_clear(&w) != cudaSuccess) return LH_ERR_CUDA;
+  v |= w;
   if (code) *code = v;
   return v ? LH_ERR_DEVICE_STATUS : LH_OK;
 }

@@ -34,10 +34,15 @@ Geom make_geom(const lh_shape& s);
 // cleared by lh_read_device_status.  It lives in the translation unit of the
 // kernels that wait (k_attn_tc.cu); this reads and clears it (synchronous).
 cudaError_t device_status_read_clear(uint32_t* value);
+// The word of the kernels that write the fp16 sub-sequence from caller data
+// (gather, scatter-back adjoint; k_gather_scatter.cu), read and cleared alike.
+cudaError_t subseq_status_read_clear(uint32_t* value);
 
+// Bits of the status words (LH_STATUS_* in lighthouse.h).
 enum : uint32_t {
   kStatusAttnFwdTimeout = 0x100,
   kStatusAttnBwdTimeout = 0x200,
+  kStatusFp16Saturated = 0x400,
 };
 
 __device__ __forceinline__ int64_t imin64(int64_t a, int64_t b) { return a < b ? a : b; }
@@ -115,14 +120,21 @@ __device__ __forceinline__ void load8(const __half* p, float (&x)[8]) {
   x[4] = h_lo(w.z); x[5] = h_hi(w.z);
   x[6] = h_lo(w.w); x[7] = h_hi(w.w);
 }
-// fp16 store that saturates at +-65504 (never writes inf)
-__device__ __forceinline__ void store8(__half* p, const float (&x)[8]) {
+// fp16 store that saturates at +-65504 (never writes inf).  `sat` gets 1 when
+// a finite value beyond that range was clipped (non-finite values are not
+// counted: results from non-finite inputs are unspecified anyway).
+__device__ __forceinline__ void store8_h(__half* p, const float (&x)[8], uint32_t& sat) {
   uint4 w;
   w.x = pack_h2_sat(x[0], x[1]);
   w.y = pack_h2_sat(x[2], x[3]);
   w.z = pack_h2_sat(x[4], x[5]);
   w.w = pack_h2_sat(x[6], x[7]);
   *reinterpret_cast<uint4*>(p) = w;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const float a = fabsf(x[i]);
+    sat |= (a > kHalfMax && a < INFINITY) ? 1u : 0u;
+  }
 }
 
 __device__ __forceinline__ void store8(__nv_bfloat16* p, const float (&x)[8]) {
@@ -222,5 +234,11 @@ bool attn_fwd_uses_tc();       // dispatch decisions (lh_set_attention_impl + av
 bool attn_bwd_uses_tc();
 int attn_tc_fwd_launches(const Geom& g);
 int attn_tc_bwd_launches(const Geom& g);
+
+// The whole sub-sequence attention backward (softmax statistics into `stats`,
+// attn_stats_floats(g) floats, then the gradient kernels); scale already resolved.
+lh_status attn_bwd(const Geom& g, const __half* qs, const __half* ks, const __half* vs,
+                   const __half* os, const float* lse, const __half* dos, float scale,
+                   float* dqs, float* dks, float* dvs, float* stats, cudaStream_t st);
 
 }  // namespace lh
