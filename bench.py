@@ -40,8 +40,8 @@ PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 
 
 # DRAM bytes (read + written) per launch of each stage, from one ncu capture of
-# the full-size pretraining workload (profiles/launches_pretrain.md: the launch
-# list with dram__bytes_read.sum and dram__bytes_write.sum, one pass).  Each entry
+# the full-size pretraining workload (the committed launch-list capture, with
+# dram__bytes_read.sum and dram__bytes_write.sum, one pass).  Each entry
 # carries a hash of the sources its kernels are built from; when they no longer
 # match, the kernel has changed since the counters were taken and the traffic is
 # reported as null.  Writes still in L2 when a kernel ends are counted by the
@@ -454,7 +454,8 @@ def run_ours(args, rk):
     out = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16 io, fp16 MMA operands / fp32 accumulate",
         "data": "synthetic (seeded N(0,1) Q/K/V/dO, 1% tokens x4; no corpus or weights)",
         "config": workload_config(w, world,
                                   {0: "tcgen05", 1: "mma_sync", 2: "tcgen05 fwd, mma_sync bwd"}[

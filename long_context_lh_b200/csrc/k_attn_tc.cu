@@ -8,14 +8,16 @@
 // only path from the layer output back to the selected Q, K and V.
 //
 // All three kernels use one CTA per SM (512 TMEM columns) and 10 warps:
-//   warps 0-7  the row work: two threads per row of the 128-row tile (TMEM lane
-//              = row; warp w reads lanes 32*(w%4).. and one half of the columns,
-//              w/4), so 8 warps share the exponentials and the fp16 packing;
-//   warp 8     TMA producer (one lane issues; in the dK/dV kernel all 32 lanes
-//              also stage the per-query softmax statistics);
+//   warps 0-7  the row work (TMEM lane = row; warp w reads lanes 32*(w%4)..):
+//              in the forward, one thread per row of one of two query tiles
+//              (warps 0-3 tile A, 4-7 tile B, ping-pong); in the two backward
+//              kernels, two threads per row of the one 128-row tile, warp w
+//              taking the column half w/4;
+//   warp 8     TMA producer (one lane issues);
 //   warp 9     MMA issuer (one lane) and owner of the TMEM allocation.
-// Score tiles are read from TMEM into registers in one go and the buffer is
-// released at once, so the next tile's products run while the row work goes on.
+// The backward kernels read a score tile from TMEM into registers in one go
+// and release the buffer at once, so the next tile's products run while the
+// row work goes on; the forward releases it after its second read.
 // Every mbarrier wait is bounded (two seconds); on expiry a status bit is set,
 // the roles drain, loads and MMAs in flight are waited for, TMEM is freed.
 // Rows past S are zero-filled by TMA (3-D tensor maps) and never stored; the

@@ -17,7 +17,24 @@
 #include "lh_internal.cuh"
 
 namespace lh {
+
+// Status word of the kernels in this file: kStatusFp16Saturated when a finite
+// value written into the fp16 sub-sequence (qs, ks, vs by the gather, dos by
+// the scatter-back adjoint) was beyond +-65504 and clipped.
+__device__ uint32_t g_subseq_status = 0;
+
+cudaError_t subseq_status_read_clear(uint32_t* value) {
+  cudaError_t e = cudaMemcpyFromSymbol(value, g_subseq_status, sizeof(uint32_t));
+  if (e != cudaSuccess) return e;
+  const uint32_t zero = 0;
+  return cudaMemcpyToSymbol(g_subseq_status, &zero, sizeof(zero));
+}
+
 namespace {
+
+__device__ __forceinline__ void report_saturation(uint32_t sat) {
+  if (sat) atomicOr(&g_subseq_status, kStatusFp16Saturated);
+}
 
 // Per-unit geometry with 32-bit indices (M < 2^31 is a checked limit); unit
 // offsets stay 64-bit.  log2p >= 0 when p is a power of two: then the level-l
@@ -83,9 +100,11 @@ __global__ void __launch_bounds__(256) k_gather(
     load8(pv + o, xv);
   }
   const int64_t d = row * D + 8 * c;
-  store8(qs + d, xq);
-  store8(ks + d, xk);
-  store8(vs + d, xv);
+  uint32_t sat = 0;
+  store8_h(qs + d, xq, sat);
+  store8_h(ks + d, xk, sat);
+  store8_h(vs + d, xv, sat);
+  report_saturation(sat);
 }
 
 // ------------------------------------------------------------ pooled gather
@@ -165,6 +184,7 @@ __global__ void __launch_bounds__(256) k_gather_pooled(
   const int64_t d = row * D + 8 * c;
   const Tin* srcs[3] = {q + first, k + first, v + first};
   __half* dsts[3] = {qs + d, ks + d, vs + d};
+  uint32_t sat = 0;
 #pragma unroll
   for (int x = 0; x < 3; ++x) {
     float val[8];
@@ -172,8 +192,9 @@ __global__ void __launch_bounds__(256) k_gather_pooled(
       load8(srcs[x], val);
     else
       pool_span<Tin, D, L>(srcs[x], lev, lv, val);
-    store8(dsts[x], val);
+    store8_h(dsts[x], val, sat);
   }
+  report_saturation(sat);
 }
 
 // ------------------------------------------------------------- scatter-back
@@ -432,6 +453,7 @@ __global__ void __launch_bounds__(256) k_scatter_bwd(const Tin* __restrict__ dO,
   const int32_t* sl = slot + u * lv.M;
   const Tin* src = dO + (u * lv.N + t0) * D + 8 * c;
   __half* dst = dos + u * lv.S * D + 8 * c;
+  uint32_t sat = 0;
 
   float acc[NL][8];
   int cnt[NL];
@@ -467,7 +489,7 @@ __global__ void __launch_bounds__(256) k_scatter_bwd(const Tin* __restrict__ dO,
       const int32_t t = t0 + r0 + b;
 #pragma unroll
       for (int i = 0; i < 8; ++i) w[b][i] = __fmul_rn(w[b][i], ic[b]);
-      if (s0[b] >= 0) store8(dst + (int64_t)s0[b] * D, w[b]);
+      if (s0[b] >= 0) store8_h(dst + (int64_t)s0[b] * D, w[b], sat);
       if constexpr (L == 1) continue;
 #pragma unroll
       for (int i = 0; i < 8; ++i) acc[0][i] = __fadd_rn(acc[0][i], w[b][i]);
@@ -478,7 +500,7 @@ __global__ void __launch_bounds__(256) k_scatter_bwd(const Tin* __restrict__ dO,
           const int lev = l + 1;
           const int32_t j = lvl_index(lv, t, lev);
           const int32_t s = __ldg(sl + lv.off[lev] + j);
-          if (s >= 0) store8(dst + (int64_t)s * D, acc[l]);
+          if (s >= 0) store8_h(dst + (int64_t)s * D, acc[l], sat);
           if (l + 1 < NL) {
 #pragma unroll
             for (int i = 0; i < 8; ++i) acc[l + 1][i] = __fadd_rn(acc[l + 1][i], acc[l][i]);
@@ -508,9 +530,10 @@ __global__ void __launch_bounds__(256) k_scatter_bwd(const Tin* __restrict__ dO,
     if (rg == 0) {
       const int32_t j = (t0 + lv.pw[L - 1]) / lv.pw[L - 1] - 1;  // the span's entry at level L-1
       const int32_t s = __ldg(sl + lv.off[L - 1] + j);
-      if (s >= 0) store8(dst + (int64_t)s * D, tot);
+      if (s >= 0) store8_h(dst + (int64_t)s * D, tot, sat);
     }
   }
+  report_saturation(sat);
 }
 
 __device__ __forceinline__ void cp_async16(void* dst, const void* src) {
@@ -594,6 +617,7 @@ __global__ void __launch_bounds__(kScatterBwdThreads) k_scatter_bwd_pp(
   const float* icu = inv_count + u * lv.N;
   const Tin* src = dO + (u * lv.N + t0) * D + 8 * c;
   __half* dst = dos + u * lv.S * D + 8 * c;
+  uint32_t sat = 0;
 
   auto issue = [&](int bi) {  // rows of batch bi into stage bi & 1
     uint4* st = sbuf + (bi & 1) * (RB * CPR * NT) + tid;
@@ -651,7 +675,7 @@ __global__ void __launch_bounds__(kScatterBwdThreads) k_scatter_bwd_pp(
       staged8(stg + b * CPR * NT, NT, (Tin*)nullptr, w);
 #pragma unroll
       for (int i = 0; i < 8; ++i) w[i] = __fmul_rn(w[i], ic[b]);
-      if (s0[b] >= 0) store8(dst + (int64_t)s0[b] * D, w);
+      if (s0[b] >= 0) store8_h(dst + (int64_t)s0[b] * D, w, sat);
       if constexpr (LW == 0) {
 #pragma unroll
         for (int i = 0; i < 8; ++i) part[i] = w[i];
@@ -670,7 +694,7 @@ __global__ void __launch_bounds__(kScatterBwdThreads) k_scatter_bwd_pp(
           else
             done = (b == RB - 1) && ((r0 + RB) % pl) == 0;
           if (done) {
-            if (cs[k] >= 0) store8(dst + (int64_t)cs[k] * D, acc[l - 1]);
+            if (cs[k] >= 0) store8_h(dst + (int64_t)cs[k] * D, acc[l - 1], sat);
             if constexpr (l < LW) {
 #pragma unroll
               for (int i = 0; i < 8; ++i) acc[l][i] = __fadd_rn(acc[l][i], acc[l - 1][i]);
@@ -710,9 +734,10 @@ __global__ void __launch_bounds__(kScatterBwdThreads) k_scatter_bwd_pp(
       for (int i = 0; i < 8; ++i) tot[i] = __fadd_rn(tot[i], __shfl_sync(mask, part[i], base + r * G));
     if (rg == 0) {
       const int32_t s = __ldg(sl + lv.off[L - 1] + span);
-      if (s >= 0) store8(dst + (int64_t)s * D, tot);
+      if (s >= 0) store8_h(dst + (int64_t)s * D, tot, sat);
     }
   }
+  report_saturation(sat);
 }
 
 // ------------------------------------------- scatter-back, last-token variant
@@ -786,8 +811,10 @@ __global__ void __launch_bounds__(256) k_scatter_bwd_last(const Tin* __restrict_
 #pragma unroll
   for (int i = 0; i < 8; ++i) x[i] = __fmul_rn(x[i], w);
   __half* dst = dos + u * lv.S * D + 8 * c;
+  uint32_t sat = 0;
   for (int l = 0; l < lv.L; ++l)
-    if (ss[l] >= 0) store8(dst + (int64_t)ss[l] * D, x);
+    if (ss[l] >= 0) store8_h(dst + (int64_t)ss[l] * D, x, sat);
+  report_saturation(sat);
 }
 
 // --------------------------------------------------------------- gather bwd

@@ -22,6 +22,8 @@ LIB_PATH = os.path.join(_PKG, "liblighthouse.so")
 LH_OK, LH_ERR_INVALID_ARG, LH_ERR_SHAPE, LH_ERR_UNSUPPORTED = 0, 1, 2, 3
 LH_ERR_WORKSPACE, LH_ERR_CUDA, LH_ERR_DEVICE_STATUS = 4, 5, 6
 LH_F32, LH_BF16 = 0, 1
+# bits of the device status word (lh_read_device_status)
+LH_STATUS_ATTN_FWD_TIMEOUT, LH_STATUS_ATTN_BWD_TIMEOUT, LH_STATUS_FP16_SATURATED = 0x100, 0x200, 0x400
 
 SAVED_IDX, SAVED_POS, SAVED_SLOT, SAVED_QS, SAVED_KS, SAVED_VS, SAVED_OS, SAVED_LSE, \
     SAVED_INV_COUNT = range(9)
