@@ -64,5 +64,27 @@ def build(verbose: bool = False, force: bool = False) -> str:
     return LIB
 
 
+SELFTEST_SRC = os.path.join(PKG, "selftest", "lh_selftest.cu")
+SELFTEST_LIB = os.path.join(PKG, "liblh_selftest.so")
+
+
+def build_selftest(verbose: bool = False) -> str:
+    """liblh_selftest.so: device-helper test hooks, loaded by the tests only."""
+    deps = [SELFTEST_SRC] + glob.glob(os.path.join(CSRC, "*.cuh"))
+    if os.path.exists(SELFTEST_LIB) and all(os.path.getmtime(SELFTEST_LIB) >= os.path.getmtime(d)
+                                            for d in deps):
+        return SELFTEST_LIB
+    cmd = [NVCC, *ARCH, *FLAGS, "-shared", "-cudart", "static", SELFTEST_SRC, "-o",
+           SELFTEST_LIB + ".tmp"]
+    if verbose:
+        print(" ".join(cmd), flush=True)
+    r = subprocess.run(cmd, capture_output=True, text=True)
+    if r.returncode != 0:
+        raise RuntimeError(f"nvcc failed on {SELFTEST_SRC}:\n{r.stdout}\n{r.stderr}")
+    os.replace(SELFTEST_LIB + ".tmp", SELFTEST_LIB)
+    return SELFTEST_LIB
+
+
 if __name__ == "__main__":
     print(build(verbose=True, force="--force" in sys.argv))
+    print(build_selftest(verbose=True))

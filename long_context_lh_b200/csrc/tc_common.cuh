@@ -321,12 +321,13 @@ __device__ __forceinline__ float max3(float a, float b, float c) {
 // 2^x for two fp32 values on the FMA/ALU pipes (x <= 127), to take part of
 // the exponentials off the MUFU unit.  Cody-Waite reduction x = n + f with
 // n = rint(x) (the 1.5 * 2^23 shift trick; f = x - n is exact), 2^f on
-// [-1/2, 1/2] by a degree-3 polynomial (coefficients fitted here to the
-// relative error at Chebyshev nodes; max relative error 7.5e-5 with fp32
-// Horner steps, below fp16's 4.9e-4 rounding of the P values it feeds), and
-// 2^n by adding n to the exponent field.  x is clamped at -125 so the result
-// stays normal; below that the true value is < 2^-125 and only enters sums
-// whose largest term is >= 1.
+// [-1/2, 1/2] by the degree-3 polynomial of least maximum relative error
+// (Remez exchange; fit_ex2_poly.py beside this file reproduces the four fp32
+// constants), max relative error 7.5e-5 with fp32 Horner steps, below fp16's
+// 4.9e-4 rounding of the P values it feeds, and 2^n by adding n to the
+// exponent field.  x is clamped at -125 so the result stays normal; below
+// that the true value is < 2^-125 and only enters sums whose largest term is
+// >= 1.
 __device__ __forceinline__ float2 ex2_fma2(float2 x) {
   x.x = fmaxf(x.x, -125.0f);
   x.y = fmaxf(x.y, -125.0f);
@@ -334,7 +335,7 @@ __device__ __forceinline__ float2 ex2_fma2(float2 x) {
   const float2 t = fadd2(x, sh);                                          // sh + rint(x)
   const float2 n = fadd2(t, make_float2(-12582912.0f, -12582912.0f));     // rint(x), exact
   const float2 f = ffma2(n, make_float2(-1.0f, -1.0f), x);                // x - n, exact
-  float2 p = ffma2(f, make_float2(0.055171650f, 0.055171650f), make_float2(0.24261113f, 0.24261113f));
+  float2 p = ffma2(f, make_float2(0.055171669f, 0.055171669f), make_float2(0.24261113f, 0.24261113f));
   p = ffma2(p, f, make_float2(0.69326097f, 0.69326097f));
   p = ffma2(p, f, make_float2(0.99992806f, 0.99992806f));
   return make_float2(__uint_as_float(__float_as_uint(p.x) + (__float_as_uint(t.x) << 23)),

@@ -641,8 +641,15 @@ def test_finite_inputs_beyond_fp16_are_clipped_and_reported():
     """bf16 inputs may exceed the fp16 range of the sub-sequence.  The documented
     outcome: the selection is still exact (scores are fp32 from the inputs), the
     gathered rows are the oracle's rows clipped to +-65504, the attention output
-    is the oracle's attention over those clipped rows, and lh_read_device_status
-    reports LH_STATUS_FP16_SATURATED (once: reading clears it)."""
+    is the attention over those clipped fp16 rows, and lh_read_device_status
+    reports LH_STATUS_FP16_SATURATED (once: reading clears it).
+
+    Here the oracle's attention takes the clipped rows rounded to fp16 (on the
+    CPU, from its own fp64 rows), i.e. exactly the operands the library defines
+    the sub-sequence to hold: a logit of a 65504-sized row with a normal one
+    moves by ~10 units when the normal row is rounded to fp16, which no
+    attention tolerance absorbs, so unrounded operands would compare two
+    different softmax distributions rather than two computations of one."""
     w = workload(dtype="bf16", N=4096, S=512, L=3, H=2)
     xc = make_inputs(w, "cpu")
     for name, tok, val in (("q", 1234, 1.0e5), ("k", 1234, -2.0e5), ("v", 1234, 3.0e5),
@@ -674,6 +681,7 @@ def test_finite_inputs_beyond_fp16_are_clipped_and_reported():
             xs.append(ref)
         if h == 1:
             assert np.abs(xs[2]).max() == 65504.0  # the clipped rows were selected
+        xs = [a.astype(np.float16).astype(np.float64) for a in xs]
         os_r, _ = oracle.attn_fwd(s1, *xs, scale)
         check_attn(f64(sv(lh.SAVED_OS)[:, h:h + 1]), os_r, f"os head {h}", torch.float16)
     # a call with inputs in range afterwards reports nothing
