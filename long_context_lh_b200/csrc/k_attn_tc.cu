@@ -173,10 +173,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp == 9) {
     // -------------------------------------------------------------- MMA issuer
-    // Lane 0 alone waits, issues every MMA and commit.  A descriptor for
-    // base + off is the base descriptor plus off / 16 (the 14-bit address field
-    // never overflows inside shared memory).
-    if (lane == 0) {
+    // The whole warp runs the loop (its waits are warp-uniform) and computes the
+    // descriptors, so they stay warp-uniform values; one elected lane issues
+    // each group of MMAs and its commit.  (Issuing from lane 0 inside a
+    // lane-0-only branch measured ~1.4x slower per MMA when row-work warps share
+    // the issuer's SM sub-partition.)  A descriptor for base + off is the base
+    // descriptor plus off / 16 (the 14-bit address field never overflows inside
+    // shared memory).
+    {
       constexpr uint32_t idS = idesc_f16(128, 128, false);
       constexpr uint32_t idPV = idesc_f16(128, D, true);
       const uint64_t dQ = desc_kmajor(smem_u32(sQ)), dK = desc_kmajor(smem_u32(sK));
@@ -184,24 +188,30 @@ __global__ void __launch_bounds__(kThreads, 1)
       auto issue_s = [&](int t, int j) {  // S_t = Q_t K_j^T
         const uint64_t q = dQ + (uint64_t)((t * Lt::kTile) >> 4);
         const uint64_t k = dK + (uint64_t)(((j % KS) * Lt::kTile) >> 4);
+        if (elect_one()) {
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint64_t off = (uint64_t)((((kk >> 2) * 16384) + ((kk & 3) * 32)) >> 4);
-          umma_f16(tmem + t * 128, q + off, k + off, idS, kk > 0);
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint64_t off = (uint64_t)((((kk >> 2) * 16384) + ((kk & 3) * 32)) >> 4);
+            umma_f16(tmem + t * 128, q + off, k + off, idS, kk > 0);
+          }
+          umma_commit(&bars->s_full[t]);
         }
-        umma_commit(&bars->s_full[t]);
+        __syncwarp();
       };
       auto issue_pv = [&](int t, int j) {  // O_t += P_t(j) V_j, P_t from TMEM
         const uint64_t v = dV + (uint64_t)(((j % KS) * Lt::kTile) >> 4);
         const uint32_t pt = kSepP ? tP + t * 64 : tmem + t * 128;
+        if (elect_one()) {
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          umma_f16_ta(tO + t * D, pt + 8 * kk, v + (uint64_t)((kk * 2048) >> 4), idPV,
-                      (j > 0 || kk > 0));
-        umma_commit(&bars->pv_done[t]);
+          for (int kk = 0; kk < 8; ++kk)
+            umma_f16_ta(tO + t * D, pt + 8 * kk, v + (uint64_t)((kk * 2048) >> 4), idPV,
+                        (j > 0 || kk > 0));
+          umma_commit(&bars->pv_done[t]);
+        }
+        __syncwarp();
       };
-      bool ok = mbar_wait(&bars->q_full, 0, abort, kStatus) &&
-                mbar_wait(&bars->kv_full[0], 0, abort, kStatus);
+      bool ok = warp_wait(&bars->q_full, 0, abort, kStatus) &&
+                warp_wait(&bars->kv_full[0], 0, abort, kStatus);
       if (ok) {
         tc_fence_after();
         issue_s(0, 0);
@@ -214,51 +224,54 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int j = 0; ok && j < nA; ++j) {
           const int st = j % KS;
           if (j + 1 < nA) {
-            if (!(ok = mbar_wait(&bars->s_free[0], j & 1, abort, kStatus))) break;
-            if (!(ok = mbar_wait(&bars->kv_full[(j + 1) % KS], ((j + 1) / KS) & 1, abort, kStatus))) break;
+            if (!(ok = warp_wait(&bars->s_free[0], j & 1, abort, kStatus))) break;
+            if (!(ok = warp_wait(&bars->kv_full[(j + 1) % KS], ((j + 1) / KS) & 1, abort, kStatus))) break;
             tc_fence_after();
             issue_s(0, j + 1);
           }
-          if (!(ok = mbar_wait(&bars->p_full[0], j & 1, abort, kStatus))) break;
+          if (!(ok = warp_wait(&bars->p_full[0], j & 1, abort, kStatus))) break;
           tc_fence_after();
           issue_pv(0, j);
           if (j < nB) {
             if (j + 1 < nB) {  // K_{j+1} is in place (waited for above: j + 1 < nB <= nA)
-              if (!(ok = mbar_wait(&bars->s_free[1], j & 1, abort, kStatus))) break;
+              if (!(ok = warp_wait(&bars->s_free[1], j & 1, abort, kStatus))) break;
               tc_fence_after();
               issue_s(1, j + 1);
             }
-            if (!(ok = mbar_wait(&bars->p_full[1], j & 1, abort, kStatus))) break;
+            if (!(ok = warp_wait(&bars->p_full[1], j & 1, abort, kStatus))) break;
             tc_fence_after();
             issue_pv(1, j);
           }
-          umma_commit(&bars->kv_empty[st]);  // K_j, V_j no longer needed
+          if (elect_one()) umma_commit(&bars->kv_empty[st]);  // K_j, V_j no longer needed
+          __syncwarp();
         }
       }
       for (int j = 0; !kSepP && ok && j < nA; ++j) {
         const int st = j % KS;
         const bool next = j + 1 < nA;
         // tile A: its product with V_j, then (S_A buffer free again) its next scores
-        if (!(ok = mbar_wait(&bars->p_full[0], j & 1, abort, kStatus))) break;
+        if (!(ok = warp_wait(&bars->p_full[0], j & 1, abort, kStatus))) break;
         tc_fence_after();
         issue_pv(0, j);
         if (next) {
-          if (!(ok = mbar_wait(&bars->kv_full[(j + 1) % KS], ((j + 1) / KS) & 1, abort, kStatus))) break;
+          if (!(ok = warp_wait(&bars->kv_full[(j + 1) % KS], ((j + 1) / KS) & 1, abort, kStatus))) break;
           tc_fence_after();
           issue_s(0, j + 1);
         }
         // tile B likewise
         if (j < nB) {
-          if (!(ok = mbar_wait(&bars->p_full[1], j & 1, abort, kStatus))) break;
+          if (!(ok = warp_wait(&bars->p_full[1], j & 1, abort, kStatus))) break;
           tc_fence_after();
           issue_pv(1, j);
           if (j + 1 < nB) issue_s(1, j + 1);
         }
-        umma_commit(&bars->kv_empty[st]);  // K_j, V_j no longer needed
+        if (elect_one()) umma_commit(&bars->kv_empty[st]);  // K_j, V_j no longer needed
+        __syncwarp();
       }
-      umma_commit(&bars->mma_done);
+      if (elect_one()) umma_commit(&bars->mma_done);
+      __syncwarp();
       // every MMA issued has completed before TMEM is freed, aborted or not
-      mbar_wait(&bars->mma_done, 0, abort, kStatus, false);
+      warp_wait(&bars->mma_done, 0, abort, kStatus, false);
     }
   } else {
     // -------------------- row work: one thread per row of its tile, all 128 keys
@@ -542,7 +555,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_wait(&bars->q_full[t % STG], (t / STG) & 1, abort, kStatus, false);
     }
   } else if (warp == 9) {
-    if (lane == 0) {
+    // MMA issuer: the whole warp waits and computes descriptors (warp-uniform),
+    // one elected lane issues each group of MMAs and its commits
+    {
       constexpr uint32_t idS = idesc_f16(128, 128, false);
       constexpr uint32_t idAcc = idesc_f16(128, D, true);
       // a descriptor for base + off is the base descriptor plus off / 16 (the
@@ -554,55 +569,62 @@ __global__ void __launch_bounds__(kThreads, 1)
       auto issue_grads = [&](int t) {  // dV += P^T dO_t, dK += dS^T Q_t
         const int st = t % STG;
         const uint64_t so = (uint64_t)((st * Lt::kTile) >> 4);
+        if (elect_one()) {
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint64_t a = (uint64_t)((((kk >> 2) * 16384) + ((kk & 3) * 32)) >> 4);
-          const uint64_t b = so + (uint64_t)((kk * 2048) >> 4);
-          if constexpr (kTmemP) {
-            umma_f16_ta(tDV, tPT + 8 * kk, dDOm + b, idAcc, (t > 0 || kk > 0));
-            umma_f16_ta(tDK, tDST + 8 * kk, dQm + b, idAcc, (t > 0 || kk > 0));
-          } else {
-            umma_f16(tDV, dPT + a, dDOm + b, idAcc, (t > 0 || kk > 0));
-            umma_f16(tDK, dDST + a, dQm + b, idAcc, (t > 0 || kk > 0));
+          for (int kk = 0; kk < 8; ++kk) {
+            const uint64_t a = (uint64_t)((((kk >> 2) * 16384) + ((kk & 3) * 32)) >> 4);
+            const uint64_t b = so + (uint64_t)((kk * 2048) >> 4);
+            if constexpr (kTmemP) {
+              umma_f16_ta(tDV, tPT + 8 * kk, dDOm + b, idAcc, (t > 0 || kk > 0));
+              umma_f16_ta(tDK, tDST + 8 * kk, dQm + b, idAcc, (t > 0 || kk > 0));
+            } else {
+              umma_f16(tDV, dPT + a, dDOm + b, idAcc, (t > 0 || kk > 0));
+              umma_f16(tDK, dDST + a, dQm + b, idAcc, (t > 0 || kk > 0));
+            }
           }
+          umma_commit(&bars->pdone);
+          umma_commit(&bars->q_empty[st]);
         }
-        umma_commit(&bars->pdone);
-        umma_commit(&bars->q_empty[st]);
+        __syncwarp();
       };
-      bool ok = mbar_wait(&bars->kv_full, 0, abort, kStatus);
+      bool ok = warp_wait(&bars->kv_full, 0, abort, kStatus);
       for (int t = 0; ok && t < n; ++t) {
         const int st = t % STG;
         if (STG == 1 && t > 0) {  // one stage: free it before the next tile is loaded
-          ok = mbar_wait(&bars->p_full, (t - 1) & 1, abort, kStatus);
+          ok = warp_wait(&bars->p_full, (t - 1) & 1, abort, kStatus);
           if (!ok) break;
           tc_fence_after();
           issue_grads(t - 1);
         }
-        ok = mbar_wait(&bars->q_full[st], (t / STG) & 1, abort, kStatus) &&
-             (t == 0 || mbar_wait(&bars->st_free, (t - 1) & 1, abort, kStatus));
+        ok = warp_wait(&bars->q_full[st], (t / STG) & 1, abort, kStatus) &&
+             (t == 0 || warp_wait(&bars->st_free, (t - 1) & 1, abort, kStatus));
         if (!ok) break;
         tc_fence_after();
         const uint64_t so = (uint64_t)((st * Lt::kTile) >> 4);
+        if (elect_one()) {
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint64_t off = (uint64_t)((((kk >> 2) * 16384) + ((kk & 3) * 32)) >> 4);
-          umma_f16(tST, dK + off, dQk + so + off, idS, kk > 0);
-          umma_f16(tDPT, dV + off, dDOk + so + off, idS, kk > 0);
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint64_t off = (uint64_t)((((kk >> 2) * 16384) + ((kk & 3) * 32)) >> 4);
+            umma_f16(tST, dK + off, dQk + so + off, idS, kk > 0);
+            umma_f16(tDPT, dV + off, dDOk + so + off, idS, kk > 0);
+          }
+          umma_commit(&bars->s_full);
         }
-        umma_commit(&bars->s_full);
+        __syncwarp();
         if (STG > 1 && t > 0) {
-          ok = mbar_wait(&bars->p_full, (t - 1) & 1, abort, kStatus);
+          ok = warp_wait(&bars->p_full, (t - 1) & 1, abort, kStatus);
           if (!ok) break;
           tc_fence_after();
           issue_grads(t - 1);
         }
       }
-      if (ok && mbar_wait(&bars->p_full, (n - 1) & 1, abort, kStatus)) {
+      if (ok && warp_wait(&bars->p_full, (n - 1) & 1, abort, kStatus)) {
         tc_fence_after();
         issue_grads(n - 1);
       }
-      umma_commit(&bars->mma_done);
-      mbar_wait(&bars->mma_done, 0, abort, kStatus, false);
+      if (elect_one()) umma_commit(&bars->mma_done);
+      __syncwarp();
+      warp_wait(&bars->mma_done, 0, abort, kStatus, false);
     }
   } else {
     // --------------------------------------- row work: two threads per key row
@@ -817,7 +839,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_wait(&bars->kv_full[j % STG], (j / STG) & 1, abort, kStatus, false);
     }
   } else if (warp == 9) {
-    if (lane == 0) {
+    // MMA issuer: the whole warp waits and computes descriptors (warp-uniform),
+    // one elected lane issues each group of MMAs and its commits
+    {
       constexpr uint32_t idS = idesc_f16(128, 128, false);
       constexpr uint32_t idAcc = idesc_f16(128, D, true);
       // base descriptors plus offset / 16, as in the dK/dV kernel
@@ -826,38 +850,45 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint64_t dKm = desc_mnmajor(smem_u32(sK), 16384);
       auto issue_dq = [&](int j) {  // dQ += dS_j K_j, dS_j from TMEM
         const int st = j % STG, b = j & 1;
-        if (!mbar_wait(&bars->ds_full[b], (j >> 1) & 1, abort, kStatus)) return false;
+        if (!warp_wait(&bars->ds_full[b], (j >> 1) & 1, abort, kStatus)) return false;
         tc_fence_after();
         const uint64_t so = (uint64_t)((st * Lt::kTile) >> 4);
+        if (elect_one()) {
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          umma_f16_ta(tDQ, tDS + b * 64 + 8 * kk, dKm + so + (uint64_t)((kk * 2048) >> 4), idAcc,
-                      (j > 0 || kk > 0));
-        umma_commit(&bars->dsdone[b]);
-        umma_commit(&bars->kv_empty[st]);
+          for (int kk = 0; kk < 8; ++kk)
+            umma_f16_ta(tDQ, tDS + b * 64 + 8 * kk, dKm + so + (uint64_t)((kk * 2048) >> 4), idAcc,
+                        (j > 0 || kk > 0));
+          umma_commit(&bars->dsdone[b]);
+          umma_commit(&bars->kv_empty[st]);
+        }
+        __syncwarp();
         return true;
       };
-      bool ok = mbar_wait(&bars->q_full, 0, abort, kStatus);
+      bool ok = warp_wait(&bars->q_full, 0, abort, kStatus);
       for (int j = 0; ok && j < n; ++j) {
         const int st = j % STG;
         if (STG == 1 && j > 0 && !(ok = issue_dq(j - 1))) break;
-        ok = mbar_wait(&bars->kv_full[st], (j / STG) & 1, abort, kStatus) &&
-             (j == 0 || mbar_wait(&bars->s_free, (j - 1) & 1, abort, kStatus));
+        ok = warp_wait(&bars->kv_full[st], (j / STG) & 1, abort, kStatus) &&
+             (j == 0 || warp_wait(&bars->s_free, (j - 1) & 1, abort, kStatus));
         if (!ok) break;
         tc_fence_after();
         const uint64_t so = (uint64_t)((st * Lt::kTile) >> 4);
+        if (elect_one()) {
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint64_t off = (uint64_t)((((kk >> 2) * 16384) + ((kk & 3) * 32)) >> 4);
-          umma_f16(tS, dQ + off, dK + so + off, idS, kk > 0);
-          umma_f16(tDP, dDO + off, dV + so + off, idS, kk > 0);
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint64_t off = (uint64_t)((((kk >> 2) * 16384) + ((kk & 3) * 32)) >> 4);
+            umma_f16(tS, dQ + off, dK + so + off, idS, kk > 0);
+            umma_f16(tDP, dDO + off, dV + so + off, idS, kk > 0);
+          }
+          umma_commit(&bars->s_full);
         }
-        umma_commit(&bars->s_full);
+        __syncwarp();
         if (STG > 1 && j > 0 && !(ok = issue_dq(j - 1))) break;
       }
       if (ok) issue_dq(n - 1);
-      umma_commit(&bars->mma_done);
-      mbar_wait(&bars->mma_done, 0, abort, kStatus, false);
+      if (elect_one()) umma_commit(&bars->mma_done);
+      __syncwarp();
+      warp_wait(&bars->mma_done, 0, abort, kStatus, false);
     }
   } else {
     // ------------------------------------- row work: two threads per query row

@@ -107,11 +107,20 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
   }
 }
 
+// True in exactly one lane of the (converged) warp: the lowest active lane.
+__device__ __forceinline__ bool elect_one() {
+  uint32_t pred;
+  asm volatile(
+      "{\n .reg .pred p;\n elect.sync _|p, 0xffffffff;\n selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(pred));
+  return pred != 0;
+}
+
 // mbar_wait for a whole warp: every lane gets the same answer, so a warp never
 // splits around the warp-collective (.sync.aligned) tcgen05 instructions.
 __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
-                                          uint32_t code) {
-  return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort, code));
+                                          uint32_t code, bool honor_abort = true) {
+  return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort, code, honor_abort));
 }
 
 // --------------------------------------------------------------------- TMA
