@@ -244,10 +244,17 @@ lh_status lh_backward(const lh_shape* shape, lh_dtype dtype, const void* saved, 
  *     (qs, ks, vs by the gather; dos by the scatter-back adjoint) lay beyond
  *     +-65504 and was clipped to it.  The selection is unaffected (it is
  *     computed in fp32 from the inputs); the attention then ran on the clipped
- *     rows.  Inputs whose pooled rows stay within +-65504 never set it. */
+ *     rows.  Inputs whose pooled rows stay within +-65504 never set it;
+ *   LH_STATUS_BOUNDS (liblighthouse_debug.so only, the same library built with
+ *     -DLH_DEBUG=1): an index computed in a kernel from data (idx, pos, slot)
+ *     or from unit, tile or level coordinates fell outside its array; the
+ *     access was skipped.  Bits 16-24 name the kernel: pyramid, selection,
+ *     gather, scatter-back, its adjoint, gather adjoint, attention forward,
+ *     attention backward, softmax statistics. */
 #define LH_STATUS_ATTN_FWD_TIMEOUT 0x100u
 #define LH_STATUS_ATTN_BWD_TIMEOUT 0x200u
 #define LH_STATUS_FP16_SATURATED 0x400u
+#define LH_STATUS_BOUNDS 0x800u
 lh_status lh_read_device_status(lh_stream_t stream, uint32_t* code);
 
 /* Selects the attention implementation for subsequent calls on this process:

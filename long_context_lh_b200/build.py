@@ -30,11 +30,11 @@ def _deps(src: str):
     return [src] + glob.glob(os.path.join(CSRC, "*.cuh")) + [os.path.join(INCLUDE, "lighthouse.h")]
 
 
-def _compile(src: str, verbose: bool) -> str:
-    obj = os.path.join(BUILD, os.path.basename(src) + ".o")
+def _compile(src: str, verbose: bool, build_dir: str = BUILD, extra=()) -> str:
+    obj = os.path.join(build_dir, os.path.basename(src) + ".o")
     if os.path.exists(obj) and all(os.path.getmtime(obj) >= os.path.getmtime(d) for d in _deps(src)):
         return obj
-    cmd = [NVCC, *ARCH, *FLAGS, "-c", src, "-o", obj + ".tmp"]
+    cmd = [NVCC, *ARCH, *FLAGS, *extra, "-c", src, "-o", obj + ".tmp"]
     if verbose:
         print(" ".join(cmd), flush=True)
     r = subprocess.run(cmd, capture_output=True, text=True)
@@ -44,24 +44,39 @@ def _compile(src: str, verbose: bool) -> str:
     return obj
 
 
-def build(verbose: bool = False, force: bool = False) -> str:
-    os.makedirs(BUILD, exist_ok=True)
+BUILD_DEBUG = os.path.join(PKG, "_build_debug")
+LIB_DEBUG = os.path.join(PKG, "liblighthouse_debug.so")
+
+
+def _build_lib(lib: str, build_dir: str, extra, verbose: bool, force: bool) -> str:
+    os.makedirs(build_dir, exist_ok=True)
     srcs = sorted(glob.glob(os.path.join(CSRC, "*.cu")))
     if force:
-        for f in glob.glob(os.path.join(BUILD, "*.o")):
+        for f in glob.glob(os.path.join(build_dir, "*.o")):
             os.remove(f)
     with ThreadPoolExecutor(max_workers=min(8, len(srcs))) as ex:
-        objs = list(ex.map(lambda s: _compile(s, verbose), srcs))
-    if os.path.exists(LIB) and all(os.path.getmtime(LIB) >= os.path.getmtime(o) for o in objs):
-        return LIB
-    cmd = [NVCC, *ARCH, "-shared", "-cudart", "static", "-o", LIB + ".tmp", *objs]
+        objs = list(ex.map(lambda s: _compile(s, verbose, build_dir, extra), srcs))
+    if os.path.exists(lib) and all(os.path.getmtime(lib) >= os.path.getmtime(o) for o in objs):
+        return lib
+    cmd = [NVCC, *ARCH, "-shared", "-cudart", "static", "-o", lib + ".tmp", *objs]
     if verbose:
         print(" ".join(cmd), flush=True)
     r = subprocess.run(cmd, capture_output=True, text=True)
     if r.returncode != 0:
         raise RuntimeError(f"link failed:\n{r.stdout}\n{r.stderr}")
-    os.replace(LIB + ".tmp", LIB)
-    return LIB
+    os.replace(lib + ".tmp", lib)
+    return lib
+
+
+def build(verbose: bool = False, force: bool = False) -> str:
+    """liblighthouse.so, the library."""
+    return _build_lib(LIB, BUILD, (), verbose, force)
+
+
+def build_debug(verbose: bool = False, force: bool = False) -> str:
+    """liblighthouse_debug.so: the same sources with -DLH_DEBUG=1 (bounds checks
+    in the kernels, reported through lh_read_device_status)."""
+    return _build_lib(LIB_DEBUG, BUILD_DEBUG, ("-DLH_DEBUG=1",), verbose, force)
 
 
 SELFTEST_SRC = os.path.join(PKG, "selftest", "lh_selftest.cu")
@@ -87,4 +102,5 @@ def build_selftest(verbose: bool = False) -> str:
 
 if __name__ == "__main__":
     print(build(verbose=True, force="--force" in sys.argv))
+    print(build_debug(verbose=True, force="--force" in sys.argv))
     print(build_selftest(verbose=True))

@@ -16,6 +16,18 @@
 #include "lh_internal.cuh"
 
 namespace lh {
+
+// Status word of the mma.sync attention kernels (bounds checks of the debug build).
+__device__ uint32_t g_mma_status = 0;
+#define LH_STATUS_WORD g_mma_status
+
+cudaError_t mma_status_read_clear(uint32_t* value) {
+  cudaError_t e = cudaMemcpyFromSymbol(value, g_mma_status, sizeof(uint32_t));
+  if (e != cudaSuccess) return e;
+  const uint32_t zero = 0;
+  return cudaMemcpyToSymbol(g_mma_status, &zero, sizeof(zero));
+}
+
 namespace {
 
 constexpr float kLog2e = 1.4426950408889634f;
@@ -119,6 +131,7 @@ __global__ void __launch_bounds__(128) k_attn_fwd_mma(const __half* __restrict__
   // heaviest (last) query tiles first
   const int qt = ntiles - 1 - blockIdx.x;
   const int64_t u = blockIdx.y;
+  if (!LH_CHECK(dbg::in_range((int64_t)qt * BM, S), kBoundsAttnFwd)) return;  // whole CTA
   const __half* Qg = qs + u * S * D;
   const __half* Kg = ks + u * S * D;
   const __half* Vg = vs + u * S * D;
@@ -266,6 +279,7 @@ __global__ void __launch_bounds__(128) k_attn_bwd_dkdv_mma(
 
   const int kt = ntiles - 1 - blockIdx.x;  // short loops last
   const int64_t u = blockIdx.y;
+  if (!LH_CHECK(dbg::in_range((int64_t)kt * BK, S), kBoundsAttnBwd)) return;  // whole CTA
   const int warp = threadIdx.x >> 5, l = threadIdx.x & 31;
   const int64_t k0 = (int64_t)kt * BK;
   const __half* Qg = qs + u * S * D;
@@ -396,6 +410,7 @@ __global__ void __launch_bounds__(128) k_attn_bwd_dq_mma(
 
   const int qt = ntiles - 1 - blockIdx.x;
   const int64_t u = blockIdx.y;
+  if (!LH_CHECK(dbg::in_range((int64_t)qt * BM, S), kBoundsAttnBwd)) return;  // whole CTA
   const int warp = threadIdx.x >> 5, l = threadIdx.x & 31;
   const int64_t q0 = (int64_t)qt * BM;
   const __half* Kg = ks + u * S * D;

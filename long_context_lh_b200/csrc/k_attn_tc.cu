@@ -26,6 +26,12 @@
 
 #include "tc_common.cuh"
 
+// Exponentials of the backward row work computed on the FMA pipe (ex2_fma2)
+// instead of MUFU: 0 none, 1 a quarter, 2 half.
+#ifndef LH_BWD_POLY
+#define LH_BWD_POLY 0
+#endif
+
 namespace lh {
 
 cudaError_t device_status_read_clear(uint32_t* value) {
@@ -119,6 +125,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int qtA = hasB ? 2 * pi + 1 : 2 * pi;  // the longer tile
   const int qtB = hasB ? 2 * pi : -1;
   const int nA = qtA + 1, nB = qtB + 1;         // key tiles of each (nB = 0: no tile B)
+  // debug build: the CTA's unit and query tiles lie inside the problem (checked
+  // before any barrier or TMEM is set up, so a bad CTA leaves as a whole)
+  if (!LH_CHECK(pi >= 0 && u < unit0 + nunits && (int64_t)qtA * 128 < S && qtB < qtA, kBoundsAttnFwd))
+    return;
 
   if (threadIdx.x == 0) {
     mbar_init(&bars->q_full, 1);
@@ -507,6 +517,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int kt = (int)(blockIdx.x / nunits);
   const int u = unit0 + (int)(blockIdx.x % nunits);
   const int n = ntiles - kt;
+  if (!LH_CHECK(kt < ntiles && (int64_t)kt * 128 < S, kBoundsAttnBwd)) return;  // whole CTA
 
   if (threadIdx.x == 0) {
     mbar_init(&bars->kv_full, 1);
@@ -661,7 +672,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                                 make_float2(nl.x, nl.y));
         const float2 x1 = ffma2(make_float2(__uint_as_float(sv[k + 2]), __uint_as_float(sv[k + 3])), cc,
                                 make_float2(nl.z, nl.w));
-        float2 p0 = make_float2(ex2(x0.x), ex2(x0.y)), p1 = make_float2(ex2(x1.x), ex2(x1.y));
+        float2 p0 = make_float2(ex2(x0.x), ex2(x0.y));
+        float2 p1 = (LH_BWD_POLY == 2 || (LH_BWD_POLY == 1 && (e & 4)))
+                        ? ex2_fma2(x1)
+                        : make_float2(ex2(x1.x), ex2(x1.y));
         if (kDiag) {
           p0.x = e < lim ? 0.0f : p0.x;
           p0.y = e + 1 < lim ? 0.0f : p0.y;
@@ -791,6 +805,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int qt = ntiles - 1 - (int)(blockIdx.x / nunits);  // most key tiles first
   const int u = unit0 + (int)(blockIdx.x % nunits);
   const int n = qt + 1;
+  if (!LH_CHECK(qt >= 0 && (int64_t)qt * 128 < S, kBoundsAttnBwd)) return;  // whole CTA
 
   if (threadIdx.x == 0) {
     mbar_init(&bars->q_full, 1);
@@ -922,7 +937,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t pd[32];
       auto pair = [&](int e, uint32_t s0, uint32_t s1, uint32_t g0, uint32_t g1) {
         const float2 x = ffma2(make_float2(__uint_as_float(s0), __uint_as_float(s1)), cc, nl);
-        float2 p = make_float2(ex2(x.x), ex2(x.y));
+        float2 p = (LH_BWD_POLY == 2 ? (e & 2) : (LH_BWD_POLY == 1 && (e & 6) == 6))
+                       ? ex2_fma2(x)
+                       : make_float2(ex2(x.x), ex2(x.y));
         if (kDiag) {
           p.x = e > lim ? 0.0f : p.x;
           p.y = e + 1 > lim ? 0.0f : p.y;

@@ -20,8 +20,10 @@ namespace lh {
 
 // Status word of the kernels in this file: kStatusFp16Saturated when a finite
 // value written into the fp16 sub-sequence (qs, ks, vs by the gather, dos by
-// the scatter-back adjoint) was beyond +-65504 and clipped.
+// the scatter-back adjoint) was beyond +-65504 and clipped; in the debug build
+// also the bounds checks (kStatusBounds).
 __device__ uint32_t g_subseq_status = 0;
+#define LH_STATUS_WORD g_subseq_status
 
 cudaError_t subseq_status_read_clear(uint32_t* value) {
   cudaError_t e = cudaMemcpyFromSymbol(value, g_subseq_status, sizeof(uint32_t));
@@ -63,6 +65,15 @@ Lv make_lv(const Geom& g) {
   return v;
 }
 
+// Slot-map entry X of a unit, sl = the unit's map.  The debug build checks that
+// X lies in [0, M) and the value in [-1, S) and reads a bad one as -1 (skipped).
+__device__ __forceinline__ int32_t ld_slot(const int32_t* __restrict__ sl, int32_t X, const Lv& lv,
+                                           uint32_t bits) {
+  if (!LH_CHECK(dbg::in_range(X, lv.M), bits)) return -1;
+  const int32_t s = __ldg(sl + X);
+  return LH_CHECK(dbg::slot_ok(s, lv.S), bits) ? s : -1;
+}
+
 // index at level l of the entry covering token t: floor(t / p^l)
 __device__ __forceinline__ int32_t lvl_index(const Lv& lv, int32_t t, int l) {
   return lv.log2p >= 0 ? (t >> (l * lv.log2p)) : (int32_t)((uint32_t)t / (uint32_t)lv.pw[l]);
@@ -87,6 +98,7 @@ __global__ void __launch_bounds__(256) k_gather(
   const int c = (int)(gt % G);
   const int64_t u = row / lv.S;
   const int32_t gid = __ldg(idx + row);
+  if (!LH_CHECK(dbg::in_range(gid, lv.M), kBoundsGather)) return;
   float xq[8], xk[8], xv[8];
   if (gid < lv.N) {
     const int64_t o = (u * lv.N + gid) * D + 8 * c;
@@ -177,6 +189,7 @@ __global__ void __launch_bounds__(256) k_gather_pooled(
   const int c = (int)(gt % G);
   const int64_t u = row / lv.S;
   const int32_t gid = __ldg(idx + row);
+  if (!LH_CHECK(dbg::in_range(gid, lv.M), kBoundsGather)) return;
   int lev = 0;
   while (lev + 1 < lv.L && gid >= lv.off[lev + 1]) ++lev;
   const int32_t j = gid - lv.off[lev];
@@ -230,9 +243,9 @@ __global__ void __launch_bounds__(256) k_scatter(const __half* __restrict__ os,
   const __half* src = os + u * lv.S * D + 8 * c;
   int32_t s0[R], sc[LC];
 #pragma unroll
-  for (int r = 0; r < R; ++r) s0[r] = __ldg(sl + t0 + r);
+  for (int r = 0; r < R; ++r) s0[r] = ld_slot(sl, t0 + r, lv, kBoundsScatter);
 #pragma unroll
-  for (int l = 1; l < L; ++l) sc[l - 1] = __ldg(sl + lv.off[l] + lvl_index(lv, t0, l));
+  for (int l = 1; l < L; ++l) sc[l - 1] = ld_slot(sl, lv.off[l] + lvl_index(lv, t0, l), lv, kBoundsScatter);
   uint4 w0[R], wc[LC];
 #pragma unroll
   for (int r = 0; r < R; ++r) {
@@ -333,11 +346,11 @@ __global__ void __launch_bounds__(128) k_scatter_pp(const __half* __restrict__ o
   auto load_slots = [&](int32_t e, Slots& sv) {  // entry e < n1
     const int32_t t = e * P;
 #pragma unroll
-    for (int r = 0; r < P; ++r) sv.s0[r] = __ldg(sl + t + r);
-    sv.s1 = __ldg(sl + lv.off[1] + e);
+    for (int r = 0; r < P; ++r) sv.s0[r] = ld_slot(sl, t + r, lv, kBoundsScatter);
+    sv.s1 = ld_slot(sl, lv.off[1] + e, lv, kBoundsScatter);
     static_for<2, L>([&](auto lc) {
       constexpr int l = decltype(lc)::value;
-      sv.su[l - 2] = __ldg(sl + lv.off[l] + (int32_t)((uint32_t)e / (uint32_t)ipow(P, l - 1)));
+      sv.su[l - 2] = ld_slot(sl, lv.off[l] + (int32_t)((uint32_t)e / (uint32_t)ipow(P, l - 1)), lv, kBoundsScatter);
     });
   };
   auto row = [&](int32_t sidx) {
@@ -472,13 +485,13 @@ __global__ void __launch_bounds__(256) k_scatter_bwd(const Tin* __restrict__ dO,
       if (r0 + b < Ptop) {
         const int32_t t = t0 + r0 + b;
         load8_stream(src + (int64_t)(r0 + b) * D, w[b]);
-        s0[b] = __ldg(sl + t);
+        s0[b] = ld_slot(sl, t, lv, kBoundsScatterBwd);
         if (inv_count) {
           ic[b] = __ldg(inv_count + u * lv.N + t);
         } else {
           int n = 0;
 #pragma unroll
-          for (int l = 0; l < L; ++l) n += (__ldg(sl + lv.off[l] + lvl_index(lv, t, l)) >= 0) ? 1 : 0;
+          for (int l = 0; l < L; ++l) n += (ld_slot(sl, lv.off[l] + lvl_index(lv, t, l), lv, kBoundsScatterBwd) >= 0) ? 1 : 0;
           ic[b] = lv.mode == LH_SCATTER_SUM ? (n > 0 ? 1.0f : 0.0f) : kRcpCount[n];
         }
       }
@@ -499,7 +512,7 @@ __global__ void __launch_bounds__(256) k_scatter_bwd(const Tin* __restrict__ dO,
         if (cnt[l] == lv.p) {
           const int lev = l + 1;
           const int32_t j = lvl_index(lv, t, lev);
-          const int32_t s = __ldg(sl + lv.off[lev] + j);
+          const int32_t s = ld_slot(sl, lv.off[lev] + j, lv, kBoundsScatterBwd);
           if (s >= 0) store8_h(dst + (int64_t)s * D, acc[l], sat);
           if (l + 1 < NL) {
 #pragma unroll
@@ -529,7 +542,7 @@ __global__ void __launch_bounds__(256) k_scatter_bwd(const Tin* __restrict__ dO,
       for (int i = 0; i < 8; ++i) tot[i] = __fadd_rn(tot[i], __shfl_sync(mask, acc[NL - 1][i], base + r * G));
     if (rg == 0) {
       const int32_t j = (t0 + lv.pw[L - 1]) / lv.pw[L - 1] - 1;  // the span's entry at level L-1
-      const int32_t s = __ldg(sl + lv.off[L - 1] + j);
+      const int32_t s = ld_slot(sl, lv.off[L - 1] + j, lv, kBoundsScatterBwd);
       if (s >= 0) store8_h(dst + (int64_t)s * D, tot, sat);
     }
   }
@@ -635,7 +648,7 @@ __global__ void __launch_bounds__(kScatterBwdThreads) k_scatter_bwd_pp(
     const int32_t tb = t0 + bi * RB;  // first token of the batch
     static_for<0, RB>([&](auto bc) {
       constexpr int b = decltype(bc)::value;
-      s0_[b] = __ldg(sl + tb + b);
+      s0_[b] = ld_slot(sl, tb + b, lv, kBoundsScatterBwd);
       ic_[b] = __ldg(icu + tb + b);
     });
     static_for<1, LW + 1>([&](auto lc) {
@@ -645,7 +658,7 @@ __global__ void __launch_bounds__(kScatterBwdThreads) k_scatter_bwd_pp(
       const int32_t j0 = (int32_t)((uint32_t)(tb + (pl <= (uint32_t)RB ? 0 : RB - 1)) / pl);
       static_for<0, k>([&](auto ic2) {
         constexpr int i = decltype(ic2)::value;
-        cs_[n + i] = __ldg(sl + lv.off[l] + j0 + i);
+        cs_[n + i] = ld_slot(sl, lv.off[l] + j0 + i, lv, kBoundsScatterBwd);
       });
     });
   };
@@ -733,7 +746,7 @@ __global__ void __launch_bounds__(kScatterBwdThreads) k_scatter_bwd_pp(
 #pragma unroll
       for (int i = 0; i < 8; ++i) tot[i] = __fadd_rn(tot[i], __shfl_sync(mask, part[i], base + r * G));
     if (rg == 0) {
-      const int32_t s = __ldg(sl + lv.off[L - 1] + span);
+      const int32_t s = ld_slot(sl, lv.off[L - 1] + span, lv, kBoundsScatterBwd);
       if (s >= 0) store8_h(dst + (int64_t)s * D, tot, sat);
     }
   }
@@ -765,7 +778,7 @@ __global__ void __launch_bounds__(256) k_scatter_last(const __half* __restrict__
   int cnt = 0;
   for (int l = 0; l < lv.L; ++l) {
     if (!ends_at_t(lv, t, l)) continue;
-    const int32_t s = __ldg(sl + lv.off[l] + lvl_index(lv, t, l));
+    const int32_t s = ld_slot(sl, lv.off[l] + lvl_index(lv, t, l), lv, kBoundsScatter);
     if (s < 0) continue;
     float x[8];
     unpack8(__ldg(reinterpret_cast<const uint4*>(src + (int64_t)s * D)), x);
@@ -801,7 +814,7 @@ __global__ void __launch_bounds__(256) k_scatter_bwd_last(const Tin* __restrict_
   int32_t ss[kMaxLevels];
   int cnt = 0;
   for (int l = 0; l < lv.L; ++l) {
-    ss[l] = ends_at_t(lv, t, l) ? __ldg(sl + lv.off[l] + lvl_index(lv, t, l)) : -1;
+    ss[l] = ends_at_t(lv, t, l) ? ld_slot(sl, lv.off[l] + lvl_index(lv, t, l), lv, kBoundsScatterBwd) : -1;
     cnt += ss[l] >= 0 ? 1 : 0;
   }
   if (cnt == 0) return;
@@ -838,9 +851,9 @@ __global__ void __launch_bounds__(256) k_gather_bwd(
   const int64_t base = u * lv.S * D + 8 * c;
   int32_t s0[R], sc[LC];
 #pragma unroll
-  for (int r = 0; r < R; ++r) s0[r] = __ldg(sl + t0 + r);
+  for (int r = 0; r < R; ++r) s0[r] = ld_slot(sl, t0 + r, lv, kBoundsGatherBwd);
 #pragma unroll
-  for (int l = 1; l < L; ++l) sc[l - 1] = __ldg(sl + lv.off[l] + lvl_index(lv, t0, l));
+  for (int l = 1; l < L; ++l) sc[l - 1] = ld_slot(sl, lv.off[l] + lvl_index(lv, t0, l), lv, kBoundsGatherBwd);
   float inv[LC];
 #pragma unroll
   for (int l = 1; l < L; ++l) inv[l - 1] = __frcp_rn((float)lv.pw[l]);
@@ -905,11 +918,11 @@ __global__ void __launch_bounds__(128) k_gather_bwd_pp(
   auto load_slots = [&](int32_t e, Slots& sv) {
     const int32_t t = e * P;
 #pragma unroll
-    for (int r = 0; r < P; ++r) sv.s0[r] = __ldg(sl + t + r);
-    sv.s1 = __ldg(sl + lv.off[1] + e);
+    for (int r = 0; r < P; ++r) sv.s0[r] = ld_slot(sl, t + r, lv, kBoundsGatherBwd);
+    sv.s1 = ld_slot(sl, lv.off[1] + e, lv, kBoundsGatherBwd);
     static_for<2, L>([&](auto lc) {
       constexpr int l = decltype(lc)::value;
-      sv.su[l - 2] = __ldg(sl + lv.off[l] + (int32_t)((uint32_t)e / (uint32_t)ipow(P, l - 1)));
+      sv.su[l - 2] = ld_slot(sl, lv.off[l] + (int32_t)((uint32_t)e / (uint32_t)ipow(P, l - 1)), lv, kBoundsGatherBwd);
     });
   };
   auto row = [&](int32_t sidx, float (&x)[8]) {

@@ -36,6 +36,18 @@
 #include "lh_internal.cuh"
 
 namespace lh {
+
+// Status word of the pyramid and score kernels (bounds checks of the debug build).
+__device__ uint32_t g_pyramid_status = 0;
+#define LH_STATUS_WORD g_pyramid_status
+
+cudaError_t pyramid_status_read_clear(uint32_t* value) {
+  cudaError_t e = cudaMemcpyFromSymbol(value, g_pyramid_status, sizeof(uint32_t));
+  if (e != cudaSuccess) return e;
+  const uint32_t zero = 0;
+  return cudaMemcpyToSymbol(g_pyramid_status, &zero, sizeof(zero));
+}
+
 namespace {
 
 // Upper bound on CR: 64 rows and 8 KB of each tensor per chunk (64 rows of
@@ -187,7 +199,8 @@ __global__ void __launch_bounds__(256) k_pyr_chunk(
       if (c == 0) sSc[r] = combine_norms(ssq, ssk, prm.score_mode);
     }
     __syncthreads();
-    for (int r = tid; r < rows; r += 256) sc[t0 + r] = sSc[r];
+    for (int r = tid; r < rows; r += 256)
+      if (LH_CHECK(dbg::in_range(t0 + r, prm.N), kBoundsPyramid)) sc[t0 + r] = sSc[r];
   }
 
   // ---- levels 1..J
@@ -229,8 +242,10 @@ __global__ void __launch_bounds__(256) k_pyr_chunk(
 #pragma unroll
         for (int z = 0; z < 8; ++z) acc[z] = mean_of<P>(acc[z], prm);
         float* dst = (t == 0 ? pq : t == 1 ? pk : pv);
-        put8(dst + ((u * (prm.M - prm.N) + prm.off[l] - prm.N + j0 + e) * D + 8 * c), acc);
-        if (l < prm.J) put8(curL + ((size_t)t * crow + e) * D + 8 * c, acc);
+        if (LH_CHECK(dbg::entry_ok(j0 + e, prm.off[l], prm.off[l + 1]), kBoundsPyramid))
+          put8(dst + ((u * (prm.M - prm.N) + prm.off[l] - prm.N + j0 + e) * D + 8 * c), acc);
+        if (l < prm.J && LH_CHECK(dbg::in_range(e, crow), kBoundsPyramid))
+          put8(curL + ((size_t)t * crow + e) * D + 8 * c, acc);
       }
     }
     if (kScore) {
@@ -256,7 +271,7 @@ __global__ void __launch_bounds__(256) k_pyr_chunk(
             }
           const float s0 = combine_norms(a[0], b[0], prm.score_mode);
           sSc[r] = s0;
-          sc[t0 + r] = s0;
+          if (LH_CHECK(dbg::in_range(t0 + r, prm.N), kBoundsPyramid)) sc[t0 + r] = s0;
         }
         __syncthreads();
       }
@@ -265,7 +280,8 @@ __global__ void __launch_bounds__(256) k_pyr_chunk(
 #pragma unroll
         for (int i = 0; i < p; ++i) m = fmaxf(m, prevS[e * p + i]);
         curS[e] = m;
-        sc[prm.off[l] + j0 + e] = m;
+        if (LH_CHECK(dbg::entry_ok(j0 + e, prm.off[l], prm.off[l + 1]), kBoundsPyramid))
+          sc[prm.off[l] + j0 + e] = m;
       }
     }
     __syncthreads();
@@ -308,14 +324,16 @@ __global__ void __launch_bounds__(256) k_pyr_upper(
     for (int z = 0; z < 8; ++z) acc[z] = mean_of<0>(acc[z], prm);
     float* dst = (t == 0 ? pq : t == 1 ? pk : pv);
     float* o = dst + (u * (prm.M - prm.N) + prm.off[l] - prm.N + e) * D + 8 * c;
-    *reinterpret_cast<float4*>(o) = make_float4(acc[0], acc[1], acc[2], acc[3]);
-    *reinterpret_cast<float4*>(o + 4) = make_float4(acc[4], acc[5], acc[6], acc[7]);
+    if (LH_CHECK(dbg::entry_ok(e, prm.off[l], prm.off[l + 1]), kBoundsPyramid)) {
+      *reinterpret_cast<float4*>(o) = make_float4(acc[0], acc[1], acc[2], acc[3]);
+      *reinterpret_cast<float4*>(o + 4) = make_float4(acc[4], acc[5], acc[6], acc[7]);
+    }
   }
   if (kScore && it < n) {
     float* sc = score + u * prm.M;
     float m = 0.0f;
     for (int i = 0; i < prm.p; ++i) m = fmaxf(m, sc[prm.off[l - 1] + it * prm.p + i]);
-    sc[prm.off[l] + it] = m;
+    if (LH_CHECK(dbg::entry_ok(it, prm.off[l], prm.off[l + 1]), kBoundsPyramid)) sc[prm.off[l] + it] = m;
   }
 }
 

@@ -35,6 +35,18 @@
 namespace cg = cooperative_groups;
 
 namespace lh {
+
+// Status word of the selection kernel (bounds checks of the debug build).
+__device__ uint32_t g_topk_status = 0;
+#define LH_STATUS_WORD g_topk_status
+
+cudaError_t topk_status_read_clear(uint32_t* value) {
+  cudaError_t e = cudaMemcpyFromSymbol(value, g_topk_status, sizeof(uint32_t));
+  if (e != cudaSuccess) return e;
+  const uint32_t zero = 0;
+  return cudaMemcpyToSymbol(g_topk_status, &zero, sizeof(zero));
+}
+
 namespace {
 
 constexpr int kThreads = 1024;
@@ -206,7 +218,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     nk += nl[l];
   }
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  if (cached) {
+  // the CTA's key range fits the cache it was sized for, and its entries lie in the unit
+  const bool range_ok = LH_CHECK(!cached || nk <= (int32_t)kcap, kBoundsTopk) &&
+                        LH_CHECK(dbg::rows_ok(prm.off[0] + jb[0], nl[0], prm.M), kBoundsTopk);
+  if (cached && range_ok) {
 #pragma unroll
     for (int l = 0; l < kMaxLevels; ++l) {
       const uint32_t* src = key + prm.off[l] + jb[l];
@@ -443,10 +458,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int l = 0; l < kMaxLevels; ++l) {
       if (!((mask >> (8 + l)) & 1u)) break;
       const int32_t g = gid_at(prm, t1, l);
+      if (!LH_CHECK(dbg::in_range(g, prm.M), kBoundsTopk)) break;
       if ((mask >> l) & 1u) {
-        idx_u[k] = (int32_t)g;
-        pos_u[k] = (int32_t)t;
-        slot_u[g] = (int32_t)k;
+        if (LH_CHECK(dbg::in_range(k, prm.S), kBoundsTopk)) {
+          idx_u[k] = (int32_t)g;
+          pos_u[k] = (int32_t)t;
+          slot_u[g] = (int32_t)k;
+        }
         ++k;
       } else {
         slot_u[g] = -1;

@@ -495,11 +495,16 @@ lh_status lh_backward_ex(const lh_shape* shape, lh_dtype dtype, const void* save
 }
 
 lh_status lh_read_device_status(lh_stream_t stream, uint32_t* code) {
-  uint32_t v = 0, w = 0;
+  uint32_t v = 0;
   if (cudaStreamSynchronize(stream) != cudaSuccess) return LH_ERR_CUDA;
-  if (device_status_read_clear(&v) != cudaSuccess) return LH_ERR_CUDA;
-  if (subseq_status_read_clear(&w) != cudaSuccess) return LH_ERR_CUDA;
-  v |= w;
+  cudaError_t (*const words[])(uint32_t*) = {device_status_read_clear, subseq_status_read_clear,
+                                             pyramid_status_read_clear, topk_status_read_clear,
+                                             mma_status_read_clear};
+  for (auto read_clear : words) {
+    uint32_t w = 0;
+    if (read_clear(&w) != cudaSuccess) return LH_ERR_CUDA;
+    v |= w;
+  }
   if (code) *code = v;
   return v ? LH_ERR_DEVICE_STATUS : LH_OK;
 }

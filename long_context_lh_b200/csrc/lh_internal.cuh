@@ -43,7 +43,59 @@ enum : uint32_t {
   kStatusAttnFwdTimeout = 0x100,
   kStatusAttnBwdTimeout = 0x200,
   kStatusFp16Saturated = 0x400,
+  kStatusBounds = 0x800,  // a bounds check of the debug build failed (kernel bit below)
+  kBoundsPyramid = 1u << 16,
+  kBoundsTopk = 1u << 17,
+  kBoundsGather = 1u << 18,
+  kBoundsScatter = 1u << 19,
+  kBoundsScatterBwd = 1u << 20,
+  kBoundsGatherBwd = 1u << 21,
+  kBoundsAttnFwd = 1u << 22,
+  kBoundsAttnBwd = 1u << 23,
+  kBoundsAttnStats = 1u << 24,
 };
+// Status words of the other kernel files (each file's kernels report into a
+// word of their own; lh_read_device_status reads and clears all of them).
+cudaError_t pyramid_status_read_clear(uint32_t* value);
+cudaError_t topk_status_read_clear(uint32_t* value);
+cudaError_t mma_status_read_clear(uint32_t* value);
+
+// ---------------------------------------------------------------- debug build
+// Compiled with -DLH_DEBUG=1 (liblighthouse_debug.so), every global or shared
+// memory access whose index comes from data (idx, pos, slot) or from unit, tile
+// and level coordinates is preceded by a check; a failed check ORs
+// kStatusBounds and the kernel's bit into the status word of its file and the
+// access is skipped (no trap, no assert).  In the normal build LH_CHECK is the
+// constant true and the checks compile to nothing.
+#ifndef LH_DEBUG
+#define LH_DEBUG 0
+#endif
+
+namespace dbg {
+// 0 <= v < n
+__host__ __device__ constexpr bool in_range(int64_t v, int64_t n) { return v >= 0 && v < n; }
+// a slot-map entry: -1 (not selected) or a row of the sub-sequence, 0 <= s < S
+__host__ __device__ constexpr bool slot_ok(int64_t s, int64_t S) { return s >= -1 && s < S; }
+// rows [first, first + count) inside [0, n)
+__host__ __device__ constexpr bool rows_ok(int64_t first, int64_t count, int64_t n) {
+  return first >= 0 && count >= 0 && first <= n && count <= n - first;
+}
+// entry j of level l of a unit: off[l] <= off[l] + j < off[l + 1]
+__host__ __device__ constexpr bool entry_ok(int64_t j, int64_t off_l, int64_t off_next) {
+  return j >= 0 && off_l + j < off_next;
+}
+}  // namespace dbg
+
+__device__ __forceinline__ bool dbg_report(bool ok, uint32_t bits, uint32_t* word) {
+  if (!ok) atomicOr(word, kStatusBounds | bits);
+  return ok;
+}
+// LH_CHECK(ok, bits) with LH_STATUS_WORD naming the file's status word.
+#if LH_DEBUG
+#define LH_CHECK(ok, bits) (::lh::dbg_report((ok), (bits), &LH_STATUS_WORD))
+#else
+#define LH_CHECK(ok, bits) true
+#endif
 
 __device__ __forceinline__ int64_t imin64(int64_t a, int64_t b) { return a < b ? a : b; }
 

@@ -26,6 +26,7 @@ namespace lh {
 // (k_attn_tc.cu, which holds every kernel with bounded waits), so the word is
 // defined here once.
 __device__ uint32_t g_device_status = 0;
+#define LH_STATUS_WORD g_device_status
 __device__ __forceinline__ void report_status(uint32_t code) { atomicOr(&g_device_status, code); }
 
 namespace tc {
@@ -359,6 +360,19 @@ __device__ __forceinline__ uint32_t h2(float lo, float hi) {
 __device__ __forceinline__ uint32_t h2_sat(float lo, float hi) {
   uint32_t d;
   asm("cvt.rn.satfinite.f16x2.f32 %0, %1, %2;\n" : "=r"(d) : "f"(hi), "f"(lo));
+  return d;
+}
+
+// 2^x for two fp16 values packed in one register (MUFU, one instruction for both).
+__device__ __forceinline__ uint32_t ex2_h2(uint32_t x) {
+  uint32_t y;
+  asm("ex2.approx.f16x2 %0, %1;\n" : "=r"(y) : "r"(x));
+  return y;
+}
+// Packed fp16 product, round to nearest.
+__device__ __forceinline__ uint32_t hmul2(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("mul.rn.f16x2 %0, %1, %2;\n" : "=r"(d) : "r"(a), "r"(b));
   return d;
 }
 

@@ -17,13 +17,18 @@ from dataclasses import dataclass
 import torch
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_PKG, "liblighthouse.so")
+# LH_LIBRARY=debug selects the bounds-checking build (liblighthouse_debug.so):
+# the same entry points, with every data-dependent index checked in the kernels
+# and failures reported through lh_read_device_status.
+LIB_PATH = os.path.join(
+    _PKG, "liblighthouse_debug.so" if os.environ.get("LH_LIBRARY") == "debug" else "liblighthouse.so")
 
 LH_OK, LH_ERR_INVALID_ARG, LH_ERR_SHAPE, LH_ERR_UNSUPPORTED = 0, 1, 2, 3
 LH_ERR_WORKSPACE, LH_ERR_CUDA, LH_ERR_DEVICE_STATUS = 4, 5, 6
 LH_F32, LH_BF16 = 0, 1
 # bits of the device status word (lh_read_device_status)
 LH_STATUS_ATTN_FWD_TIMEOUT, LH_STATUS_ATTN_BWD_TIMEOUT, LH_STATUS_FP16_SATURATED = 0x100, 0x200, 0x400
+LH_STATUS_BOUNDS = 0x800  # debug build only
 
 SAVED_IDX, SAVED_POS, SAVED_SLOT, SAVED_QS, SAVED_KS, SAVED_VS, SAVED_OS, SAVED_LSE, \
     SAVED_INV_COUNT = range(9)

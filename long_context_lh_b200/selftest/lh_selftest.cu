@@ -5,7 +5,10 @@
 //
 //   lh_selftest_ex2_fma2: evaluates ex2_fma2 (tc_common.cuh), the FMA-pipe 2^x
 //   that the forward attention uses for a quarter of its exponentials, on n
-//   values, so a test can hold it to its stated error bound.
+//   values, so a test can hold it to its stated error bound;
+//   lh_selftest_bounds: the debug build's bounds predicates (lh_internal.cuh),
+//   compiled for the host, so a CPU test can feed them out-of-range indices
+//   (no kernel ever gets a bad index on purpose).
 #include "../csrc/tc_common.cuh"
 
 namespace {
@@ -30,4 +33,16 @@ extern "C" int lh_selftest_ex2_fma2(const float* x, float* y, int64_t n, void* s
   if (grid > 0x7fffffff) return 1;
   k_ex2_fma2<<<(unsigned)grid, block, 0, static_cast<cudaStream_t>(stream)>>>(x, y, pairs);
   return (int)cudaGetLastError();
+}
+
+// which: 0 in_range(a, b), 1 slot_ok(a, b), 2 rows_ok(a, b, c), 3 entry_ok(a, b, c).
+// Returns 1 (true), 0 (false) or -1 (unknown predicate).
+extern "C" int lh_selftest_bounds(int which, int64_t a, int64_t b, int64_t c) {
+  switch (which) {
+    case 0: return lh::dbg::in_range(a, b) ? 1 : 0;
+    case 1: return lh::dbg::slot_ok(a, b) ? 1 : 0;
+    case 2: return lh::dbg::rows_ok(a, b, c) ? 1 : 0;
+    case 3: return lh::dbg::entry_ok(a, b, c) ? 1 : 0;
+  }
+  return -1;
 }
