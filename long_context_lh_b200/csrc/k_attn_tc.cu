@@ -26,11 +26,6 @@
 
 #include "tc_common.cuh"
 
-// Exponentials of the backward row work computed on the FMA pipe (ex2_fma2)
-// instead of MUFU: 0 none, 1 a quarter, 2 half.
-#ifndef LH_BWD_POLY
-#define LH_BWD_POLY 0
-#endif
 
 namespace lh {
 
@@ -384,7 +379,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           const float2 y = ffma2(make_float2(__uint_as_float(v[a + 2]), __uint_as_float(v[a + 3])), cc, nm);
           float2 p = make_float2(ex2(x.x), ex2(x.y));
           // a quarter of the exponentials on the FMA pipe, the rest on MUFU (half
-          // on the FMA pipe measured slower: the row work is then issue-bound)
+          // on the FMA pipe measured slower: the row work is then issue-bound;
+          // three eighths the same as a quarter)
           float2 q = (i & 7) == 4 ? ex2_fma2(y) : make_float2(ex2(y.x), ex2(y.y));
           if (kDiag) {
             const int k0 = 32 * c + i;
@@ -672,10 +668,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                                 make_float2(nl.x, nl.y));
         const float2 x1 = ffma2(make_float2(__uint_as_float(sv[k + 2]), __uint_as_float(sv[k + 3])), cc,
                                 make_float2(nl.z, nl.w));
-        float2 p0 = make_float2(ex2(x0.x), ex2(x0.y));
-        float2 p1 = (LH_BWD_POLY == 2 || (LH_BWD_POLY == 1 && (e & 4)))
-                        ? ex2_fma2(x1)
-                        : make_float2(ex2(x1.x), ex2(x1.y));
+        float2 p0 = make_float2(ex2(x0.x), ex2(x0.y)), p1 = make_float2(ex2(x1.x), ex2(x1.y));
         if (kDiag) {
           p0.x = e < lim ? 0.0f : p0.x;
           p0.y = e + 1 < lim ? 0.0f : p0.y;
@@ -937,9 +930,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t pd[32];
       auto pair = [&](int e, uint32_t s0, uint32_t s1, uint32_t g0, uint32_t g1) {
         const float2 x = ffma2(make_float2(__uint_as_float(s0), __uint_as_float(s1)), cc, nl);
-        float2 p = (LH_BWD_POLY == 2 ? (e & 2) : (LH_BWD_POLY == 1 && (e & 6) == 6))
-                       ? ex2_fma2(x)
-                       : make_float2(ex2(x.x), ex2(x.y));
+        // a quarter of the exponentials on the FMA pipe (this row work is MUFU-bound;
+        // measured: none 571 us, a quarter 530, half 546 for the whole backward)
+        float2 p = (e & 6) == 6 ? ex2_fma2(x) : make_float2(ex2(x.x), ex2(x.y));
         if (kDiag) {
           p.x = e > lim ? 0.0f : p.x;
           p.y = e + 1 > lim ? 0.0f : p.y;
