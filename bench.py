@@ -253,37 +253,49 @@ def measure(lh, w, args, rk, dev, peaks, steps, warmup, backward=True, batch=0, 
         abw = lh.lh_attn_bwd_workspace_bytes(shp)
         aws = torch.empty(abw, dtype=torch.uint8, device=dev)
 
-    def staged(evs):
-        # identical launches to lh_forward (+ lh_backward), with events between stages
-        evs[0].record(stream)
-        lh.lh_build_pyramid_score(shp, dt, q, k, v, pq, pk, pv, score, sp)
-        evs[1].record(stream)
-        lh.lh_topk_select(shp, score, idx, pos, slot, None, 0, sp)
-        evs[2].record(stream)
-        lh.lh_gather(shp, dt, q, k, v, pq, pk, pv, idx, qs, ks, vs, sp)
-        evs[3].record(stream)
-        lh.lh_subseq_attn_fwd(shp, qs, ks, vs, 0.0, os_, lse, sp)
-        evs[4].record(stream)
-        lh.lh_scatter_back(shp, dt, os_, slot, o, ic, sp)
-        evs[5].record(stream)
+    def staged(evs, flush=None):
+        # identical launches to lh_forward (+ lh_backward), with events between
+        # stages; with `flush`, L2 is overwritten before each stage (evs: start,
+        # end per stage)
+        launches = [
+            lambda: lh.lh_build_pyramid_score(shp, dt, q, k, v, pq, pk, pv, score, sp),
+            lambda: lh.lh_topk_select(shp, score, idx, pos, slot, None, 0, sp),
+            lambda: lh.lh_gather(shp, dt, q, k, v, pq, pk, pv, idx, qs, ks, vs, sp),
+            lambda: lh.lh_subseq_attn_fwd(shp, qs, ks, vs, 0.0, os_, lse, sp),
+            lambda: lh.lh_scatter_back(shp, dt, os_, slot, o, ic, sp),
+        ]
         if backward:
-            lh.lh_scatter_back_bwd(shp, dt, dO, slot, ic, dos, sp)
-            evs[6].record(stream)
-            lh.lh_subseq_attn_bwd(shp, qs, ks, vs, os_, lse, dos, 0.0, dqs, dks, dvs, aws, abw, sp)
-            evs[7].record(stream)
-            lh.lh_gather_bwd(shp, dt, dqs, dks, dvs, slot, dq, dk, dv, sp)
-            evs[8].record(stream)
+            launches += [
+                lambda: lh.lh_scatter_back_bwd(shp, dt, dO, slot, ic, dos, sp),
+                lambda: lh.lh_subseq_attn_bwd(shp, qs, ks, vs, os_, lse, dos, 0.0, dqs, dks, dvs,
+                                              aws, abw, sp),
+                lambda: lh.lh_gather_bwd(shp, dt, dqs, dks, dvs, slot, dq, dk, dv, sp),
+            ]
+        for i, launch in enumerate(launches):
+            if flush is not None:
+                flush()
+            evs[2 * i].record(stream)
+            launch()
+            evs[2 * i + 1].record(stream)
 
-    with torch.cuda.stream(stream):
+    def replay(flush=None, reps=steps):
         evs_all = []
         torch.cuda.synchronize()
-        for _ in range(steps):
-            evs = [torch.cuda.Event(enable_timing=True) for _ in range(len(stages) + 1)]
-            staged(evs)
+        for _ in range(reps):
+            evs = [torch.cuda.Event(enable_timing=True) for _ in range(2 * len(stages))]
+            staged(evs, flush)
             evs_all.append(evs)
         torch.cuda.synchronize()
-        stage_ms = {st: statistics.mean(e[i].elapsed_time(e[i + 1]) for e in evs_all)
-                    for i, st in enumerate(stages)}
+        return {st: statistics.mean(e[2 * i].elapsed_time(e[2 * i + 1]) for e in evs_all)
+                for i, st in enumerate(stages)}
+
+    with torch.cuda.stream(stream):
+        stage_ms = replay()
+        # the same launches with L2 overwritten (a 256 MB write, twice L2) before
+        # each stage: no stage reads what the one before left in L2
+        l2_junk = torch.empty(64 << 20, dtype=torch.float32, device=dev)
+        stage_ms_flushed = replay(lambda: l2_junk.fill_(1.0), reps=max(3, min(steps, 10)))
+        del l2_junk
         status |= lh.lh_read_device_status(stream)
 
     # rows the pooled gather must read: p^level for every selected entry
@@ -302,7 +314,10 @@ def measure(lh, w, args, rk, dev, peaks, steps, warmup, backward=True, batch=0, 
             report[st] = {"ms": stage_ms[st], "tflops": fl / t / 1e12, "frac_tc": fl / t / 1e12 / tc}
         else:
             bts = alg[st]
-            report[st] = {"ms": stage_ms[st], "gbs": bts / t / 1e9, "frac_hbm": bts / t / 1e9 / hbm}
+            tf = stage_ms_flushed[st] / 1e3
+            report[st] = {"ms": stage_ms[st], "gbs": bts / t / 1e9, "frac_hbm": bts / t / 1e9 / hbm,
+                          "ms_l2_flushed": stage_ms_flushed[st],
+                          "frac_hbm_l2_flushed": bts / tf / 1e9 / hbm}
         report[st]["traffic"] = measured_traffic(traffic_key, st)
     return {"ms_step": ms_step, "ms_fwd": ms_fwd, "stages": report, "status": status,
             "peak_bytes": peak_bytes, "clk": clk, "traffic_key": traffic_key,
@@ -474,6 +489,9 @@ def run_ours(args, rk):
         out["clocks"] = clk.summary()
         if not args.no_cpu:
             out["cpu_baseline"] = cpu_baseline(w, budget_s=args.cpu_budget)
+            # the same oracle on one core: one head, forward + backward
+            one = cpu_baseline(w, steps=1, nthreads=1)
+            out["cpu_baseline_1core"] = {k: one[k] for k in ("value", "unit", "cores", "kind", "sample")}
         print(json.dumps(out), flush=True)
 
 
@@ -595,29 +613,31 @@ def e2e_run(lh, w, shp, dt, x, dev, stream, args, rk, ref_out):
 
 
 # ------------------------------------------------------------- CPU oracle
-def oracle_step(w, h, x_np):
-    """Oracle forward + backward of head h (all of its tokens)."""
+def oracle_step(w, h, x_np, nthreads=None):
+    """Oracle forward + backward of head h (all of its tokens); nthreads: the
+    oracle's worker threads (None: one per host core)."""
     import oracle
     s1 = oracle.Shape(1, 1, w.N, w.d, w.p, w.L, w.S)
     q, k, v, dO = (x_np[n][:, h:h + 1] for n in ("q", "k", "v", "dO"))
-    f = oracle.forward(s1, q, k, v)
-    oracle.backward(s1, f, dO)
+    f = oracle.forward(s1, q, k, v, nthreads=nthreads)
+    oracle.backward(s1, f, dO, nthreads=nthreads)
 
 
-def cpu_baseline(w, budget_s=20.0, steps=None, warmup=0):
-    """Time the oracle on this host's cores: whole heads, until the budget is spent."""
+def cpu_baseline(w, budget_s=20.0, steps=None, warmup=0, nthreads=None):
+    """Time the oracle on this host's cores (or on `nthreads` of them): whole
+    heads, until the budget is spent."""
     import numpy as np  # noqa: F401
     xc = make_inputs(w, "cpu")
     x_np = {n: t.float().numpy() for n, t in xc.items()}
-    cores = os.cpu_count() or 1
+    cores = nthreads or os.cpu_count() or 1
     for h in range(warmup):
-        oracle_step(w, h % w.H, x_np)
+        oracle_step(w, h % w.H, x_np, nthreads)
     t0 = time.perf_counter()
     heads = 0
     times = []
     while heads < w.H:
         t1 = time.perf_counter()
-        oracle_step(w, heads % w.H, x_np)
+        oracle_step(w, heads % w.H, x_np, nthreads)
         times.append(time.perf_counter() - t1)
         heads += 1
         if steps is not None and heads >= steps:
