@@ -41,7 +41,7 @@ namespace {
 
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kLog2e = 1.4426950408889634f;
-constexpr int kThreads = 320;
+constexpr int kThreads = 352;  // 8 row-work warps, TMA warp 8, MMA warps 9 and 10
 constexpr uint32_t kTmemCols = 512;
 
 __device__ __forceinline__ void store_row_half(uint8_t* tile_half, int r, const uint32_t (&pk)[32]) {
@@ -104,6 +104,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (threadIdx.x == 0) report_status(kStatusAttnFwdTimeout | 1u);
     return;
   }
+  constexpr bool kSepP = (D == 64);
   FwdBars* bars = reinterpret_cast<FwdBars*>(smem + Lt::kBar);
   uint8_t* sQ = smem + Lt::kQ;
   uint8_t* sK = smem + Lt::kK;
@@ -137,7 +138,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&bars->p_full[t], 4);
       mbar_init(&bars->pv_done[t], 1);
     }
-    mbar_init(&bars->mma_done, 1);
+    mbar_init(&bars->mma_done, kSepP ? 2 : 1);  // one commit from each MMA issuer
     bars->abort = 0;
     mbar_init_fence();
   }
@@ -148,8 +149,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem = bars->tmem;
   const uint32_t tO = tmem + 256;  // O_A at +256, O_B at +256+D; S_T at +128*T
   // d = 64: P_A, P_B in their own columns (+384, +448), so S_T(j+1) need not
-  // wait for O_T += P_T(j) V_j
-  constexpr bool kSepP = (D == 64);
+  // wait for O_T += P_T(j) V_j (kSepP, defined above)
   static_assert(!kSepP || 256 + 2 * D + 128 <= (int)kTmemCols, "TMEM: S_A, S_B, O_A, O_B, P_A, P_B");
   const uint32_t tP = tmem + 256 + 2 * D;
 
@@ -176,15 +176,19 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int j = (issued > KS ? issued - KS : 0); j < issued; ++j)
         mbar_wait(&bars->kv_full[j % KS], (j / KS) & 1, abort, kStatus, false);
     }
-  } else if (warp == 9) {
-    // -------------------------------------------------------------- MMA issuer
+  } else if (warp == 9 || (kSepP && warp == 10)) {
+    // ------------------------------------------------------------- MMA issuers
     // The whole warp runs the loop (its waits are warp-uniform) and computes the
     // descriptors, so they stay warp-uniform values; one elected lane issues
     // each group of MMAs and its commit.  (Issuing from lane 0 inside a
     // lane-0-only branch measured ~1.4x slower per MMA when row-work warps share
-    // the issuer's SM sub-partition.)  A descriptor for base + off is the base
-    // descriptor plus off / 16 (the 14-bit address field never overflows inside
-    // shared memory).
+    // the issuer's SM sub-partition.)  At d = 64 two warps on two sub-partitions
+    // issue: warp 9 the S products, warp 10 the P V products (an issuing warp
+    // competes with the row-work warps of its sub-partition; splitting halves
+    // that load).  At d = 128 P lives over S, so S_T(j+1) must follow
+    // O_T += P_T(j) V_j in one in-order stream: warp 9 issues everything.
+    // A descriptor for base + off is the base descriptor plus off / 16 (the
+    // 14-bit address field never overflows inside shared memory).
     {
       constexpr uint32_t idS = idesc_f16(128, 128, false);
       constexpr uint32_t idPV = idesc_f16(128, D, true);
@@ -215,40 +219,46 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         __syncwarp();
       };
-      bool ok = warp_wait(&bars->q_full, 0, abort, kStatus) &&
-                warp_wait(&bars->kv_full[0], 0, abort, kStatus);
-      if (ok) {
-        tc_fence_after();
-        issue_s(0, 0);
-        if (nB > 0) issue_s(1, 0);
+      bool ok = true;
+      if (warp == 9) {
+        ok = warp_wait(&bars->q_full, 0, abort, kStatus) &&
+             warp_wait(&bars->kv_full[0], 0, abort, kStatus);
+        if (ok) {
+          tc_fence_after();
+          issue_s(0, 0);
+          if (nB > 0) issue_s(1, 0);
+        }
       }
       if constexpr (kSepP) {
-        // per key tile j: S_A(j+1) once S_A(j) is read, O_A += P_A(j) V_j once P_A(j)
-        // is written, then the same for tile B; the waits follow the order in which
-        // the row work produces these events
-        for (int j = 0; ok && j < nA; ++j) {
-          const int st = j % KS;
-          if (j + 1 < nA) {
+        if (warp == 9) {
+          // S_T(j+1) once S_T(j) is read (and K_{j+1} is in place), tile A then B
+          for (int j = 0; ok && j + 1 < nA; ++j) {
             if (!(ok = warp_wait(&bars->s_free[0], j & 1, abort, kStatus))) break;
             if (!(ok = warp_wait(&bars->kv_full[(j + 1) % KS], ((j + 1) / KS) & 1, abort, kStatus))) break;
             tc_fence_after();
             issue_s(0, j + 1);
-          }
-          if (!(ok = warp_wait(&bars->p_full[0], j & 1, abort, kStatus))) break;
-          tc_fence_after();
-          issue_pv(0, j);
-          if (j < nB) {
             if (j + 1 < nB) {  // K_{j+1} is in place (waited for above: j + 1 < nB <= nA)
               if (!(ok = warp_wait(&bars->s_free[1], j & 1, abort, kStatus))) break;
               tc_fence_after();
               issue_s(1, j + 1);
             }
-            if (!(ok = warp_wait(&bars->p_full[1], j & 1, abort, kStatus))) break;
-            tc_fence_after();
-            issue_pv(1, j);
           }
-          if (elect_one()) umma_commit(&bars->kv_empty[st]);  // K_j, V_j no longer needed
-          __syncwarp();
+        } else {
+          // O_T += P_T(j) V_j once P_T(j) is written, tile A then B; then K_j, V_j
+          // are free (S_A(j), S_B(j) completed before the row work wrote P)
+          for (int j = 0; ok && j < nA; ++j) {
+            const int st = j % KS;
+            if (!(ok = warp_wait(&bars->p_full[0], j & 1, abort, kStatus))) break;
+            tc_fence_after();
+            issue_pv(0, j);
+            if (j < nB) {
+              if (!(ok = warp_wait(&bars->p_full[1], j & 1, abort, kStatus))) break;
+              tc_fence_after();
+              issue_pv(1, j);
+            }
+            if (elect_one()) umma_commit(&bars->kv_empty[st]);
+            __syncwarp();
+          }
         }
       }
       for (int j = 0; !kSepP && ok && j < nA; ++j) {
@@ -273,12 +283,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (elect_one()) umma_commit(&bars->kv_empty[st]);  // K_j, V_j no longer needed
         __syncwarp();
       }
-      if (elect_one()) umma_commit(&bars->mma_done);
+      if (elect_one()) umma_commit(&bars->mma_done);  // from each issuer
       __syncwarp();
       // every MMA issued has completed before TMEM is freed, aborted or not
       warp_wait(&bars->mma_done, 0, abort, kStatus, false);
     }
-  } else {
+  } else if (warp < 8) {
     // -------------------- row work: one thread per row of its tile, all 128 keys
     // P is formed against a running reference max m_ref, and O_t is rescaled in
     // TMEM only when a tile's max exceeds m_ref by more than kRescale (exp2
@@ -525,7 +535,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(&bars->st_free, 8);
     mbar_init(&bars->p_full, 8);
     mbar_init(&bars->pdone, 1);
-    mbar_init(&bars->mma_done, 1);
+    mbar_init(&bars->mma_done, 2);  // one commit from each MMA issuer
     bars->abort = 0;
     mbar_init_fence();
   }
@@ -561,19 +571,48 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int t = (issued > STG ? issued - STG : 0); t < issued; ++t)
         mbar_wait(&bars->q_full[t % STG], (t / STG) & 1, abort, kStatus, false);
     }
-  } else if (warp == 9) {
-    // MMA issuer: the whole warp waits and computes descriptors (warp-uniform),
-    // one elected lane issues each group of MMAs and its commits
-    {
-      constexpr uint32_t idS = idesc_f16(128, 128, false);
-      constexpr uint32_t idAcc = idesc_f16(128, D, true);
-      // a descriptor for base + off is the base descriptor plus off / 16 (the
-      // 14-bit address field never overflows inside shared memory)
+  } else if (warp == 9 || warp == 10) {
+    // Two MMA issuers on two SM sub-partitions: warp 9 the S^T and dP^T products
+    // of every query tile, warp 10 the dV and dK products.  (An issuing warp
+    // competes for issue slots with the row-work warps of its sub-partition,
+    // and those set the pace of every handoff; splitting the products halves
+    // that load.)  Each whole warp waits and computes the descriptors, so they
+    // stay warp-uniform; one elected lane issues each group and its commits.
+    // A descriptor for base + off is the base descriptor plus off / 16 (the
+    // 14-bit address field never overflows inside shared memory).
+    constexpr uint32_t idS = idesc_f16(128, 128, false);
+    constexpr uint32_t idAcc = idesc_f16(128, D, true);
+    bool ok = true;
+    if (warp == 9) {
       const uint64_t dK = desc_kmajor(smem_u32(sK)), dV = desc_kmajor(smem_u32(sV));
       const uint64_t dQk = desc_kmajor(smem_u32(sQ)), dDOk = desc_kmajor(smem_u32(sDO));
+      ok = warp_wait(&bars->kv_full, 0, abort, kStatus);
+      for (int t = 0; ok && t < n; ++t) {
+        const int st = t % STG;
+        // Q_t, dO_t in place; S^T, dP^T of the previous tile read by the row work
+        ok = warp_wait(&bars->q_full[st], (t / STG) & 1, abort, kStatus) &&
+             (t == 0 || warp_wait(&bars->st_free, (t - 1) & 1, abort, kStatus));
+        if (!ok) break;
+        tc_fence_after();
+        const uint64_t so = (uint64_t)((st * Lt::kTile) >> 4);
+        if (elect_one()) {
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint64_t off = (uint64_t)((((kk >> 2) * 16384) + ((kk & 3) * 32)) >> 4);
+            umma_f16(tST, dK + off, dQk + so + off, idS, kk > 0);
+            umma_f16(tDPT, dV + off, dDOk + so + off, idS, kk > 0);
+          }
+          umma_commit(&bars->s_full);
+        }
+        __syncwarp();
+      }
+    } else {
       const uint64_t dQm = desc_mnmajor(smem_u32(sQ), 16384), dDOm = desc_mnmajor(smem_u32(sDO), 16384);
       const uint64_t dPT = desc_kmajor(smem_u32(sPT)), dDST = desc_kmajor(smem_u32(sDST));
-      auto issue_grads = [&](int t) {  // dV += P^T dO_t, dK += dS^T Q_t
+      for (int t = 0; ok && t < n; ++t) {  // dV += P^T dO_t, dK += dS^T Q_t
+        ok = warp_wait(&bars->p_full, t & 1, abort, kStatus);  // P^T, dS^T of tile t written
+        if (!ok) break;
+        tc_fence_after();
         const int st = t % STG;
         const uint64_t so = (uint64_t)((st * Lt::kTile) >> 4);
         if (elect_one()) {
@@ -590,49 +629,15 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
           }
           umma_commit(&bars->pdone);
-          umma_commit(&bars->q_empty[st]);
+          umma_commit(&bars->q_empty[st]);  // stage st free for tile t + STG
         }
         __syncwarp();
-      };
-      bool ok = warp_wait(&bars->kv_full, 0, abort, kStatus);
-      for (int t = 0; ok && t < n; ++t) {
-        const int st = t % STG;
-        if (STG == 1 && t > 0) {  // one stage: free it before the next tile is loaded
-          ok = warp_wait(&bars->p_full, (t - 1) & 1, abort, kStatus);
-          if (!ok) break;
-          tc_fence_after();
-          issue_grads(t - 1);
-        }
-        ok = warp_wait(&bars->q_full[st], (t / STG) & 1, abort, kStatus) &&
-             (t == 0 || warp_wait(&bars->st_free, (t - 1) & 1, abort, kStatus));
-        if (!ok) break;
-        tc_fence_after();
-        const uint64_t so = (uint64_t)((st * Lt::kTile) >> 4);
-        if (elect_one()) {
-#pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint64_t off = (uint64_t)((((kk >> 2) * 16384) + ((kk & 3) * 32)) >> 4);
-            umma_f16(tST, dK + off, dQk + so + off, idS, kk > 0);
-            umma_f16(tDPT, dV + off, dDOk + so + off, idS, kk > 0);
-          }
-          umma_commit(&bars->s_full);
-        }
-        __syncwarp();
-        if (STG > 1 && t > 0) {
-          ok = warp_wait(&bars->p_full, (t - 1) & 1, abort, kStatus);
-          if (!ok) break;
-          tc_fence_after();
-          issue_grads(t - 1);
-        }
       }
-      if (ok && warp_wait(&bars->p_full, (n - 1) & 1, abort, kStatus)) {
-        tc_fence_after();
-        issue_grads(n - 1);
-      }
-      if (elect_one()) umma_commit(&bars->mma_done);
-      __syncwarp();
-      warp_wait(&bars->mma_done, 0, abort, kStatus, false);
     }
+    // both issuers commit: every MMA issued has completed before TMEM is freed
+    if (elect_one()) umma_commit(&bars->mma_done);
+    __syncwarp();
+    warp_wait(&bars->mma_done, 0, abort, kStatus, false);
   } else {
     // --------------------------------------- row work: two threads per key row
     const int qd = warp & 3, h = warp >> 2;
@@ -812,7 +817,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     mbar_init(&bars->s_full, 1);
     mbar_init(&bars->s_free, 8);
-    mbar_init(&bars->mma_done, 1);
+    mbar_init(&bars->mma_done, 2);  // one commit from each MMA issuer
     bars->abort = 0;
     mbar_init_fence();
   }
@@ -846,36 +851,20 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int j = (issued > STG ? issued - STG : 0); j < issued; ++j)
         mbar_wait(&bars->kv_full[j % STG], (j / STG) & 1, abort, kStatus, false);
     }
-  } else if (warp == 9) {
-    // MMA issuer: the whole warp waits and computes descriptors (warp-uniform),
-    // one elected lane issues each group of MMAs and its commits
-    {
-      constexpr uint32_t idS = idesc_f16(128, 128, false);
-      constexpr uint32_t idAcc = idesc_f16(128, D, true);
-      // base descriptors plus offset / 16, as in the dK/dV kernel
+  } else if (warp == 9 || warp == 10) {
+    // Two MMA issuers, as in the dK/dV kernel: warp 9 the S and dP products of
+    // every key tile, warp 10 the dQ products; descriptors are base descriptors
+    // plus offset / 16
+    constexpr uint32_t idS = idesc_f16(128, 128, false);
+    constexpr uint32_t idAcc = idesc_f16(128, D, true);
+    bool ok = true;
+    if (warp == 9) {
       const uint64_t dQ = desc_kmajor(smem_u32(sQ)), dDO = desc_kmajor(smem_u32(sDO));
       const uint64_t dK = desc_kmajor(smem_u32(sK)), dV = desc_kmajor(smem_u32(sV));
-      const uint64_t dKm = desc_mnmajor(smem_u32(sK), 16384);
-      auto issue_dq = [&](int j) {  // dQ += dS_j K_j, dS_j from TMEM
-        const int st = j % STG, b = j & 1;
-        if (!warp_wait(&bars->ds_full[b], (j >> 1) & 1, abort, kStatus)) return false;
-        tc_fence_after();
-        const uint64_t so = (uint64_t)((st * Lt::kTile) >> 4);
-        if (elect_one()) {
-#pragma unroll
-          for (int kk = 0; kk < 8; ++kk)
-            umma_f16_ta(tDQ, tDS + b * 64 + 8 * kk, dKm + so + (uint64_t)((kk * 2048) >> 4), idAcc,
-                        (j > 0 || kk > 0));
-          umma_commit(&bars->dsdone[b]);
-          umma_commit(&bars->kv_empty[st]);
-        }
-        __syncwarp();
-        return true;
-      };
-      bool ok = warp_wait(&bars->q_full, 0, abort, kStatus);
+      ok = warp_wait(&bars->q_full, 0, abort, kStatus);
       for (int j = 0; ok && j < n; ++j) {
         const int st = j % STG;
-        if (STG == 1 && j > 0 && !(ok = issue_dq(j - 1))) break;
+        // K_j, V_j in place; S, dP of the previous key tile read by the row work
         ok = warp_wait(&bars->kv_full[st], (j / STG) & 1, abort, kStatus) &&
              (j == 0 || warp_wait(&bars->s_free, (j - 1) & 1, abort, kStatus));
         if (!ok) break;
@@ -891,13 +880,30 @@ __global__ void __launch_bounds__(kThreads, 1)
           umma_commit(&bars->s_full);
         }
         __syncwarp();
-        if (STG > 1 && j > 0 && !(ok = issue_dq(j - 1))) break;
       }
-      if (ok) issue_dq(n - 1);
-      if (elect_one()) umma_commit(&bars->mma_done);
-      __syncwarp();
-      warp_wait(&bars->mma_done, 0, abort, kStatus, false);
+    } else {
+      const uint64_t dKm = desc_mnmajor(smem_u32(sK), 16384);
+      for (int j = 0; ok && j < n; ++j) {  // dQ += dS_j K_j, dS_j from TMEM
+        const int st = j % STG, b = j & 1;
+        ok = warp_wait(&bars->ds_full[b], (j >> 1) & 1, abort, kStatus);
+        if (!ok) break;
+        tc_fence_after();
+        const uint64_t so = (uint64_t)((st * Lt::kTile) >> 4);
+        if (elect_one()) {
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk)
+            umma_f16_ta(tDQ, tDS + b * 64 + 8 * kk, dKm + so + (uint64_t)((kk * 2048) >> 4), idAcc,
+                        (j > 0 || kk > 0));
+          umma_commit(&bars->dsdone[b]);
+          umma_commit(&bars->kv_empty[st]);  // K_j, V_j no longer needed (S, dP done before dS)
+        }
+        __syncwarp();
+      }
     }
+    // both issuers commit: every MMA issued has completed before TMEM is freed
+    if (elect_one()) umma_commit(&bars->mma_done);
+    __syncwarp();
+    warp_wait(&bars->mma_done, 0, abort, kStatus, false);
   } else {
     // ------------------------------------- row work: two threads per query row
     const int qd = warp & 3, h = warp >> 2;
