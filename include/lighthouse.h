@@ -234,6 +234,53 @@ lh_status lh_backward(const lh_shape* shape, lh_dtype dtype, const void* saved, 
                       float scale, void* dq, void* dk, void* dv, void* ws, size_t ws_bytes,
                       lh_stream_t stream);
 
+/* ---------------------------------------------------- context parallelism
+ * [PT] bitsgeniais.com.br, section "Escalando para o Céu (ou 1 Milhão de
+ * Tokens!): Paralelismo de Contexto": the sequence is split into P contiguous
+ * shards, one per GPU.  Each GPU runs the pyramid, the scores, the selection,
+ * the gather and the scatter-back on its own shard with no communication (the
+ * stage calls above, with the shard's N and S/P); the dense sub-sequence -- the
+ * shards' sub-sequences in shard order, which is (pos, level) order again --
+ * is attended with standard ring attention.  The calls below are one GPU's
+ * steps of that ring (long_context_lh_b200/cp.py drives it over NCCL).  A
+ * block has shape->S rows; shape->N must equal shape->S (p and L are only
+ * validated: pass p = 2, L = 1).  Blocks are fp16 [B,H,S,d] like qs/ks/vs.  */
+
+/* Attention of a query block against one key block of the same length.
+ * causal = 1: the diagonal block (row k sees keys k' <= k, as
+ * lh_subseq_attn_fwd); causal = 0: an earlier block, every key (rows and keys
+ * past S excluded).  os: fp16 [B,H,S,d], the normalised block output; lse: fp32
+ * [B,H,S].  causal = 0 needs the tcgen05 kernels (LH_ERR_UNSUPPORTED otherwise). */
+lh_status lh_block_attn_fwd(const lh_shape* shape, int causal, const void* qs, const void* ks,
+                            const void* vs, float scale, void* os, float* lse, lh_stream_t stream);
+
+/* Online merge of a block result into the running one, `rows` rows of d in
+ * {64, 128}: first = 1 copies (o_part, lse_part) into (o_acc, lse_acc);
+ * otherwise both become the softmax-weighted combination, weights
+ * exp(lse - lse_new), lse_new = log(exp(lse_acc) + exp(lse_part)).  o_acc,
+ * lse_acc fp32; o_part fp16; lse_part fp32.  Merging the blocks in a fixed
+ * order makes the result deterministic. */
+lh_status lh_block_attn_merge(int64_t rows, int32_t d, float* o_acc, float* lse_acc,
+                              const void* o_part, const float* lse_part, int first,
+                              lh_stream_t stream);
+
+/* os (fp16) = o_acc (fp32) rounded to nearest, `rows` rows of d. */
+lh_status lh_block_attn_finish(int64_t rows, int32_t d, const float* o_acc, void* os,
+                               lh_stream_t stream);
+
+/* Backward of one (query block, key block) pair, given the query block's final
+ * os, lse (after every merge) and dos: the pair's gradients dqs (for the query
+ * rows) and dks, dvs (for the key rows), fp32 [B,H,S,d], overwritten.
+ * causal as in lh_block_attn_fwd.  ws: lh_attn_bwd_workspace_bytes(shape). */
+lh_status lh_block_attn_bwd(const lh_shape* shape, int causal, const void* qs, const void* ks,
+                            const void* vs, const void* os, const float* lse, const void* dos,
+                            float scale, float* dqs, float* dks, float* dvs, void* ws,
+                            size_t ws_bytes, lh_stream_t stream);
+
+/* acc[i] += x[i] for n fp32 values (n a multiple of 4): one fp32 add per
+ * element, so gradients summed in a fixed order of calls are deterministic. */
+lh_status lh_accumulate(int64_t n, float* acc, const float* x, lh_stream_t stream);
+
 /* Reads and clears the device status words (synchronises `stream`).  LH_OK or
  * LH_ERR_DEVICE_STATUS; *code (may be NULL) receives the OR of the words, 0
  * for none, else LH_STATUS_* bits:

@@ -94,7 +94,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     k_attn_fwd_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
                   const __grid_constant__ CUtensorMap tv, __half* __restrict__ os,
                   float* __restrict__ lse, int S, int unit0, int nunits, float scale_log2,
-                  int ntiles) {
+                  int ntiles, int full) {
   using Lt = FwdLayout<D>;
   constexpr int KS = Lt::kKS;
   static_assert(KS >= 1 && KS <= 4, "FwdBars holds at most 4 stages");
@@ -120,7 +120,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   const bool hasB = 2 * pi + 1 < ntiles;
   const int qtA = hasB ? 2 * pi + 1 : 2 * pi;  // the longer tile
   const int qtB = hasB ? 2 * pi : -1;
-  const int nA = qtA + 1, nB = qtB + 1;         // key tiles of each (nB = 0: no tile B)
+  // key tiles of each (nB = 0: no tile B): causal, the tiles up to the diagonal;
+  // full (a query block against an earlier key block), all of them
+  const int nA = full ? ntiles : qtA + 1, nB = qtB < 0 ? 0 : (full ? ntiles : qtB + 1);
   // debug build: the CTA's unit and query tiles lie inside the problem (checked
   // before any barrier or TMEM is set up, so a bad CTA leaves as a whole)
   if (!LH_CHECK(pi >= 0 && u < unit0 + nunits && (int64_t)qtA * 128 < S && qtB < qtA, kBoundsAttnFwd))
@@ -305,7 +307,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tOt = tO + t * D + lane_addr;
     float m_ref = -INFINITY, l = 0.0f;
     bool ok = true;
-    // one key tile; kDiag: the last (diagonal) tile, keys past the row masked
+    // the masked (last) key tile keeps keys 0..lim: causal, the keys up to the
+    // row (the diagonal tile); full, the keys inside the block (a ragged tail)
+    const int lim = full ? ((S - 1) & 127) : r;
+    const bool mask_last = !full || (S & 127) != 0;
+    // one key tile; kDiag: the last tile with the mask above
     auto step = [&](int j, auto diag_tag) {
       constexpr bool kDiag = decltype(diag_tag)::value;
       ok = warp_wait(&bars->s_full[t], j & 1, abort, kStatus);
@@ -325,8 +331,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int i = 0; i < 128; i += 2) {
           const int k = (i >> 1) & 3;
           if (kDiag) {
-            mc[k] = max3(mc[k], i <= r ? __uint_as_float(v[i]) : -INFINITY,
-                         i + 1 <= r ? __uint_as_float(v[i + 1]) : -INFINITY);
+            mc[k] = max3(mc[k], i <= lim ? __uint_as_float(v[i]) : -INFINITY,
+                         i + 1 <= lim ? __uint_as_float(v[i + 1]) : -INFINITY);
           } else {
             mc[k] = max3(mc[k], __uint_as_float(v[i]), __uint_as_float(v[i + 1]));
           }
@@ -394,10 +400,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           float2 q = (i & 7) == 4 ? ex2_fma2(y) : make_float2(ex2(y.x), ex2(y.y));
           if (kDiag) {
             const int k0 = 32 * c + i;
-            p.x = k0 <= r ? p.x : 0.0f;
-            p.y = k0 + 1 <= r ? p.y : 0.0f;
-            q.x = k0 + 2 <= r ? q.x : 0.0f;
-            q.y = k0 + 3 <= r ? q.y : 0.0f;
+            p.x = k0 <= lim ? p.x : 0.0f;
+            p.y = k0 + 1 <= lim ? p.y : 0.0f;
+            q.x = k0 + 2 <= lim ? q.x : 0.0f;
+            q.y = k0 + 3 <= lim ? q.y : 0.0f;
           }
           const int k = (i >> 2) & 1;
           sacc[2 * k] = fadd2(sacc[2 * k], p);
@@ -424,7 +430,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     };
     if (n > 0) {
       for (int j = 0; j < n - 1 && ok; ++j) step(j, std::false_type{});
-      if (ok) step(n - 1, std::true_type{});
+      if (ok) {
+        if (mask_last)
+          step(n - 1, std::true_type{});
+        else
+          step(n - 1, std::false_type{});
+      }
       if (ok) ok = warp_wait(&bars->pv_done[t], (n - 1) & 1, abort, kStatus);
       const int row = qt * 128 + r;
       if (ok) {  // whole warps load TMEM; only rows inside the sequence are stored
@@ -497,7 +508,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                        const __grid_constant__ CUtensorMap tv, const __grid_constant__ CUtensorMap tdo,
                        const float* __restrict__ stats, float* __restrict__ dks,
                        float* __restrict__ dvs, int S, int unit0,
-                       int nunits, float scale, float scale_log2, int ntiles) {
+                       int nunits, float scale, float scale_log2, int ntiles, int full) {
   using Lt = DkvLayout<D>;
   constexpr int STG = Lt::kStages;
   static_assert(STG >= 1 && STG <= 4, "DkvBars holds at most 4 stages");
@@ -522,7 +533,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   // 1-D grid ordered by work: key tile 0 (the most query tiles) of every unit first
   const int kt = (int)(blockIdx.x / nunits);
   const int u = unit0 + (int)(blockIdx.x % nunits);
-  const int n = ntiles - kt;
+  // query tiles i0.. of this key tile: causal, from the diagonal on; full (an
+  // earlier key block), all of them, none masked (padded query rows have P = 0)
+  const int i0 = full ? 0 : kt;
+  const int n = ntiles - i0;
   if (!LH_CHECK(kt < ntiles && (int64_t)kt * 128 < S, kBoundsAttnBwd)) return;  // whole CTA
 
   if (threadIdx.x == 0) {
@@ -557,7 +571,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       int issued = 0;
       for (int t = 0; t < n; ++t) {
-        const int st = t % STG, i = kt + t;
+        const int st = t % STG, i = i0 + t;
         if (t >= STG && !mbar_wait(&bars->q_empty[st], ((t - STG) / STG) & 1, abort, kStatus)) break;
         mbar_expect_tx(&bars->q_full[st], 2 * Lt::kTile + 1024);
         for (int h = 0; h < D / 64; ++h) {
@@ -708,7 +722,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars->p_full);
     };
-    step(0, std::true_type{});
+    if (full)
+      step(0, std::false_type{});
+    else
+      step(0, std::true_type{});
     for (int t = 1; t < n && ok; ++t) step(t, std::false_type{});
     if (ok) ok = warp_wait(&bars->pdone, (n - 1) & 1, abort, kStatus);
     const int row = kt * 128 + r;
@@ -782,7 +799,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                      const __grid_constant__ CUtensorMap tv, const __grid_constant__ CUtensorMap tdo,
                      const float* __restrict__ stats, float* __restrict__ dqs, int S,
                      int unit0, int nunits, float scale,
-                     float scale_log2, int ntiles) {
+                     float scale_log2, int ntiles, int full) {
   using Lt = DqLayout<D>;
   constexpr int STG = Lt::kStages;
   static_assert(STG >= 1 && STG <= 4, "DqBars holds at most 4 stages");
@@ -802,7 +819,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int qt = ntiles - 1 - (int)(blockIdx.x / nunits);  // most key tiles first
   const int u = unit0 + (int)(blockIdx.x % nunits);
-  const int n = qt + 1;
+  const int n = full ? ntiles : qt + 1;  // key tiles: up to the diagonal, or all of the block
   if (!LH_CHECK(qt >= 0 && (int64_t)qt * 128 < S, kBoundsAttnBwd)) return;  // whole CTA
 
   if (threadIdx.x == 0) {
@@ -932,7 +949,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (lane == 0) mbar_arrive(&bars->s_free);
       const float2 cc = make_float2(scale_log2, scale_log2), nl = make_float2(nlse2, nlse2);
       const float2 nd = make_float2(nD, nD);
-      const int lim = r - h * 64;  // key columns e > lim follow the query
+      // key columns e > lim are masked in the last tile: those after the query
+      // (causal), those past the block's end (full, ragged tail)
+      const int lim = (full ? ((S - 1) & 127) : r) - h * 64;
       uint32_t pd[32];
       auto pair = [&](int e, uint32_t s0, uint32_t s1, uint32_t g0, uint32_t g1) {
         const float2 x = ffma2(make_float2(__uint_as_float(s0), __uint_as_float(s1)), cc, nl);
@@ -960,7 +979,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (lane == 0) mbar_arrive(&bars->ds_full[b]);
     };
     for (int j = 0; j < n - 1 && ok; ++j) step(j, std::false_type{});
-    if (ok) step(n - 1, std::true_type{});
+    if (ok) {
+      if (!full || (S & 127) != 0)
+        step(n - 1, std::true_type{});
+      else
+        step(n - 1, std::false_type{});
+    }
     if (ok) ok = warp_wait(&bars->dsdone[(n - 1) & 1], ((n - 1) >> 1) & 1, abort, kStatus);
     if (ok) {
       tc_fence_after();
@@ -1024,7 +1048,7 @@ bool make_map(CUtensorMap* map, const void* base, int d, int64_t S, int64_t U) {
 
 template <int D>
 cudaError_t fwd_d(const Geom& g, const __half* qs, const __half* ks, const __half* vs,
-                  float scale, __half* os, float* lse, cudaStream_t st) {
+                  float scale, __half* os, float* lse, int full, cudaStream_t st) {
   CUtensorMap mq, mk, mv;
   if (!make_map(&mq, qs, D, g.S, g.U) || !make_map(&mk, ks, D, g.S, g.U) ||
       !make_map(&mv, vs, D, g.S, g.U))
@@ -1039,7 +1063,7 @@ cudaError_t fwd_d(const Geom& g, const __half* qs, const __half* ks, const __hal
   for (int64_t u0 = 0; u0 < g.U; u0 += per) {
     const int64_t nu = g.U - u0 < per ? g.U - u0 : per;
     k_attn_fwd_tc<D><<<(unsigned)(nu * npairs), kThreads, smem, st>>>(
-        mq, mk, mv, os, lse, (int)g.S, (int)u0, (int)nu, scale * kLog2e, ntiles);
+        mq, mk, mv, os, lse, (int)g.S, (int)u0, (int)nu, scale * kLog2e, ntiles, full);
   }
   return cudaGetLastError();
 }
@@ -1047,7 +1071,7 @@ cudaError_t fwd_d(const Geom& g, const __half* qs, const __half* ks, const __hal
 template <int D>
 cudaError_t bwd_d(const Geom& g, const __half* qs, const __half* ks, const __half* vs,
                   const __half* dos, const float* stats, float scale, float* dqs, float* dks,
-                  float* dvs, cudaStream_t st) {
+                  float* dvs, int full, cudaStream_t st) {
   CUtensorMap mq, mk, mv, mdo;
   if (!make_map(&mq, qs, D, g.S, g.U) || !make_map(&mk, ks, D, g.S, g.U) ||
       !make_map(&mv, vs, D, g.S, g.U) || !make_map(&mdo, dos, D, g.S, g.U))
@@ -1064,9 +1088,10 @@ cudaError_t bwd_d(const Geom& g, const __half* qs, const __half* ks, const __hal
     const int64_t nu = g.U - u0 < per ? g.U - u0 : per;
     k_attn_bwd_dkdv_tc<D><<<(unsigned)(nu * ntiles), kThreads, smem_a, st>>>(
         mq, mk, mv, mdo, stats, dks, dvs, (int)g.S, (int)u0, (int)nu, scale, scale * kLog2e,
-        ntiles);
+        ntiles, full);
     k_attn_bwd_dq_tc<D><<<(unsigned)(nu * ntiles), kThreads, smem_b, st>>>(
-        mq, mk, mv, mdo, stats, dqs, (int)g.S, (int)u0, (int)nu, scale, scale * kLog2e, ntiles);
+        mq, mk, mv, mdo, stats, dqs, (int)g.S, (int)u0, (int)nu, scale, scale * kLog2e, ntiles,
+        full);
   }
   return cudaGetLastError();
 }
@@ -1094,18 +1119,19 @@ int attn_tc_bwd_launches(const Geom& g) {
 
 cudaError_t launch_attn_fwd_tc(const Geom& g, const __half* qs, const __half* ks,
                                const __half* vs, float scale, __half* os, float* lse,
-                               cudaStream_t st) {
+                               cudaStream_t st, int full) {
   if (g.S > 0x7fffffff || g.U > 0x7fffffff) return cudaErrorInvalidValue;
-  return g.d == 64 ? tc::fwd_d<64>(g, qs, ks, vs, scale, os, lse, st)
-                   : tc::fwd_d<128>(g, qs, ks, vs, scale, os, lse, st);
+  return g.d == 64 ? tc::fwd_d<64>(g, qs, ks, vs, scale, os, lse, full, st)
+                   : tc::fwd_d<128>(g, qs, ks, vs, scale, os, lse, full, st);
 }
 
 cudaError_t launch_attn_bwd_tc(const Geom& g, const __half* qs, const __half* ks,
                                const __half* vs, const __half* dos, const float* stats,
-                               float scale, float* dqs, float* dks, float* dvs, cudaStream_t st) {
+                               float scale, float* dqs, float* dks, float* dvs, cudaStream_t st,
+                               int full) {
   if (g.S > 0x7fffffff || g.U > 0x7fffffff) return cudaErrorInvalidValue;
-  return g.d == 64 ? tc::bwd_d<64>(g, qs, ks, vs, dos, stats, scale, dqs, dks, dvs, st)
-                   : tc::bwd_d<128>(g, qs, ks, vs, dos, stats, scale, dqs, dks, dvs, st);
+  return g.d == 64 ? tc::bwd_d<64>(g, qs, ks, vs, dos, stats, scale, dqs, dks, dvs, full, st)
+                   : tc::bwd_d<128>(g, qs, ks, vs, dos, stats, scale, dqs, dks, dvs, full, st);
 }
 
 }  // namespace lh

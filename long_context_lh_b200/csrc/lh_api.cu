@@ -154,10 +154,11 @@ Geom geom_with(const lh_shape& shape, const lh_options* opt) {
 lh_status attn_bwd(const Geom& g, const __half* qs, const __half* ks,
                    const __half* vs, const __half* os, const float* lse,
                    const __half* dos, float scale, float* dqs, float* dks, float* dvs,
-                   float* stats, cudaStream_t st) {
+                   float* stats, cudaStream_t st, int full) {
+  if (full && !attn_bwd_uses_tc()) return LH_ERR_UNSUPPORTED;  // checked before any launch
   LH_TRY(launch_attn_stats(g, os, dos, lse, stats, st));
   if (attn_bwd_uses_tc())
-    return cuda_status(launch_attn_bwd_tc(g, qs, ks, vs, dos, stats, scale, dqs, dks, dvs, st));
+    return cuda_status(launch_attn_bwd_tc(g, qs, ks, vs, dos, stats, scale, dqs, dks, dvs, st, full));
   return cuda_status(launch_attn_bwd_mma(g, qs, ks, vs, dos, stats, scale, dqs, dks, dvs, st));
 }
 

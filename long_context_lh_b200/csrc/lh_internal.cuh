@@ -274,12 +274,16 @@ cudaError_t launch_attn_fwd_mma(const Geom& g, const __half* qs, const __half* k
 cudaError_t launch_attn_bwd_mma(const Geom& g, const __half* qs, const __half* ks,
                                 const __half* vs, const __half* dos, const float* stats,
                                 float scale, float* dqs, float* dks, float* dvs, cudaStream_t st);
+// full = 1: a query block against a whole earlier key block of the same length
+// (no causal mask; the keys past the block's end masked) -- the off-diagonal
+// steps of ring attention; full = 0: causal attention within one sequence.
 cudaError_t launch_attn_fwd_tc(const Geom& g, const __half* qs, const __half* ks,
                                const __half* vs, float scale, __half* os,
-                               float* lse, cudaStream_t st);
+                               float* lse, cudaStream_t st, int full = 0);
 cudaError_t launch_attn_bwd_tc(const Geom& g, const __half* qs, const __half* ks,
                                const __half* vs, const __half* dos, const float* stats,
-                               float scale, float* dqs, float* dks, float* dvs, cudaStream_t st);
+                               float scale, float* dqs, float* dks, float* dvs, cudaStream_t st,
+                               int full = 0);
 bool attn_tc_available();      // tcgen05 forward can run on this device
 bool attn_tc_bwd_available();  // tcgen05 backward can run on this device
 bool attn_fwd_uses_tc();       // dispatch decisions (lh_set_attention_impl + availability)
@@ -291,6 +295,7 @@ int attn_tc_bwd_launches(const Geom& g);
 // attn_stats_floats(g) floats, then the gradient kernels); scale already resolved.
 lh_status attn_bwd(const Geom& g, const __half* qs, const __half* ks, const __half* vs,
                    const __half* os, const float* lse, const __half* dos, float scale,
-                   float* dqs, float* dks, float* dvs, float* stats, cudaStream_t st);
+                   float* dqs, float* dks, float* dvs, float* stats, cudaStream_t st,
+                   int full = 0);
 
 }  // namespace lh

@@ -101,6 +101,12 @@ _SIGS = {
                             _VP], _I),
     "lh_subseq_attn_bwd_noalloc": ([_SP, _VP, _VP, _VP, _VP, _VP, _VP, _F, _VP, _VP, _VP,
                                     _VP], _I),
+    "lh_block_attn_fwd": ([_SP, _I, _VP, _VP, _VP, _F, _VP, _VP, _VP], _I),
+    "lh_block_attn_merge": ([_I64, _I, _VP, _VP, _VP, _VP, _I, _VP], _I),
+    "lh_block_attn_finish": ([_I64, _I, _VP, _VP, _VP], _I),
+    "lh_block_attn_bwd": ([_SP, _I, _VP, _VP, _VP, _VP, _VP, _VP, _F, _VP, _VP, _VP, _VP, _SZ,
+                           _VP], _I),
+    "lh_accumulate": ([_I64, _VP, _VP, _VP], _I),
     "lh_scatter_back": ([_SP, _I, _VP, _VP, _VP, _VP, _VP], _I),
     "lh_scatter_back_bwd": ([_SP, _I, _VP, _VP, _VP, _VP, _VP], _I),
     "lh_gather_bwd": ([_SP, _I, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP], _I),
@@ -322,6 +328,34 @@ def lh_subseq_attn_bwd_noalloc(shape, qs, ks, vs, os_, lse, dos, scale, dqs, dks
     _check("lh_subseq_attn_bwd_noalloc", _lib().lh_subseq_attn_bwd_noalloc(
         ctypes.byref(shape), _p(qs), _p(ks), _p(vs), _p(os_), _p(lse), _p(dos), float(scale),
         _p(dqs), _p(dks), _p(dvs), _st(stream)))
+
+
+# ------------------------------------------------ context parallelism (one GPU's ring steps)
+def lh_block_attn_fwd(shape, causal, qs, ks, vs, scale, os_, lse, stream=None):
+    _check("lh_block_attn_fwd", _lib().lh_block_attn_fwd(
+        ctypes.byref(shape), int(causal), _p(qs), _p(ks), _p(vs), float(scale), _p(os_), _p(lse),
+        _st(stream)))
+
+
+def lh_block_attn_merge(rows, d, o_acc, lse_acc, o_part, lse_part, first, stream=None):
+    _check("lh_block_attn_merge", _lib().lh_block_attn_merge(
+        int(rows), int(d), _p(o_acc), _p(lse_acc), _p(o_part), _p(lse_part), int(first), _st(stream)))
+
+
+def lh_block_attn_finish(rows, d, o_acc, os_, stream=None):
+    _check("lh_block_attn_finish", _lib().lh_block_attn_finish(int(rows), int(d), _p(o_acc), _p(os_),
+                                                               _st(stream)))
+
+
+def lh_block_attn_bwd(shape, causal, qs, ks, vs, os_, lse, dos, scale, dqs, dks, dvs, ws, ws_bytes,
+                      stream=None):
+    _check("lh_block_attn_bwd", _lib().lh_block_attn_bwd(
+        ctypes.byref(shape), int(causal), _p(qs), _p(ks), _p(vs), _p(os_), _p(lse), _p(dos),
+        float(scale), _p(dqs), _p(dks), _p(dvs), _p(ws), int(ws_bytes), _st(stream)))
+
+
+def lh_accumulate(n, acc, x, stream=None):
+    _check("lh_accumulate", _lib().lh_accumulate(int(n), _p(acc), _p(x), _st(stream)))
 
 
 def lh_scatter_back(shape, dtype, os_, slot, o, inv_count=None, stream=None):

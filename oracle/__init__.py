@@ -321,3 +321,62 @@ def forward_fixed(s: Shape, q, k, v, idx, slot, scale=None, nthreads=None) -> np
     xs = [gather(s, x, pyramid(s, x, nthreads), idx) for x in (q, k, v)]
     os_, _ = attn_fwd(s, *xs, scale, nthreads=nthreads)
     return scatter(s, os_, slot)
+
+
+# ------------------------------------------------------- context parallelism
+def cp_shards(s: Shape, P: int) -> Shape:
+    """The per-shard shape of P-way context parallelism: N/P tokens, S/P entries."""
+    if P < 1 or s.N % P or s.S % P:
+        raise ValueError("N and S must be multiples of the shard count")
+    return Shape(s.B, s.H, s.N // P, s.d, s.p, s.L, s.S // P)
+
+
+def cp_forward(s: Shape, q, k, v, P: int, scale=None) -> dict:
+    """The layer under P-way context parallelism ([PT] bitsgeniais.com.br, section
+    "Escalando para o Céu (ou 1 Milhão de Tokens!): Paralelismo de Contexto"):
+    the sequence is cut into P contiguous shards; each shard builds its own
+    pyramid, scores and selection with a budget of S/P entries and gathers them
+    (local pre-attention, no communication); the dense sub-sequence is the
+    shards' sub-sequences in shard order -- (position, level) order again,
+    since the shards are contiguous -- and it is attended causally on the slot
+    index as one sequence (what ring attention computes); each shard's tokens
+    take their outputs back from their own entries.  Returns the per-shard
+    intermediates (lists) and the concatenated sub-sequence arrays."""
+    sh = cp_shards(s, P)
+    scale = default_scale(s, scale)
+    q, k, v = (_f64(t).reshape(s.B, s.H, s.N, s.d) for t in (q, k, v))
+    n = sh.N
+    parts = []
+    for r in range(P):
+        qr, kr, vr = (t[:, :, r * n:(r + 1) * n] for t in (q, k, v))
+        pq, pk, pv = (pyramid(sh, x) for x in (qr, kr, vr))
+        sc = score(sh, qr, kr)
+        idx, pos, slot = select(sh, sc)
+        parts.append(dict(idx=idx, pos=pos + r * n, slot=slot,
+                          qs=gather(sh, qr, pq, idx), ks=gather(sh, kr, pk, idx),
+                          vs=gather(sh, vr, pv, idx)))
+    cat = lambda key: np.concatenate([pt[key] for pt in parts], axis=2)
+    qs, ks, vs = cat("qs"), cat("ks"), cat("vs")
+    sfull = Shape(s.B, s.H, s.S, s.d, 2, 1, s.S)  # one sequence of S rows
+    os_, lse = attn_fwd(sfull, qs, ks, vs, scale)
+    o = np.concatenate([scatter(sh, os_[:, :, r * sh.S:(r + 1) * sh.S], parts[r]["slot"])
+                        for r in range(P)], axis=2)
+    return dict(parts=parts, qs=qs, ks=ks, vs=vs, os=os_, lse=lse, o=o, pos=cat("pos"),
+                scale=scale, P=P, shard=sh)
+
+
+def cp_backward(s: Shape, fwd: dict, dO) -> dict:
+    """Backward of cp_forward: each shard's scatter-back adjoint, the attention
+    backward over the concatenated sub-sequence, each shard's gather adjoint."""
+    sh, P = fwd["shard"], fwd["P"]
+    dO = _f64(dO).reshape(s.B, s.H, s.N, s.d)
+    n = sh.N
+    dos = np.concatenate([scatter_bwd(sh, dO[:, :, r * n:(r + 1) * n], fwd["parts"][r]["idx"],
+                                      fwd["parts"][r]["slot"]) for r in range(P)], axis=2)
+    sfull = Shape(s.B, s.H, s.S, s.d, 2, 1, s.S)
+    dqs, dks, dvs = attn_bwd(sfull, fwd["qs"], fwd["ks"], fwd["vs"], dos, fwd["scale"])
+    out = dict(dos=dos, dqs=dqs, dks=dks, dvs=dvs)
+    for name, g in (("dq", dqs), ("dk", dks), ("dv", dvs)):
+        out[name] = np.concatenate([gather_bwd(sh, g[:, :, r * sh.S:(r + 1) * sh.S],
+                                               fwd["parts"][r]["slot"]) for r in range(P)], axis=2)
+    return out

@@ -468,3 +468,59 @@ def test_scatter_modes_entry_centric_and_adjoint(mode, p, L, S):
                 else:
                     continue
                 break
+
+
+# ------------------------------------------------------- context parallelism
+def test_cp_one_shard_is_the_layer():
+    """One shard: the context-parallel layer is the single-GPU layer, bit for bit."""
+    s = Shape(1, 2, 512, 8, 4, 3, 96)
+    rng = np.random.default_rng(21)
+    q, k, v, dO = (rng.standard_normal((1, 2, 512, 8)) for _ in range(4))
+    a, b = oracle.forward(s, q, k, v), oracle.cp_forward(s, q, k, v, 1)
+    assert np.array_equal(a["o"], b["o"])
+    ga, gb = oracle.backward(s, a, dO), oracle.cp_backward(s, b, dO)
+    for n in ("dq", "dk", "dv"):
+        assert np.array_equal(ga[n], gb[n])
+
+
+@pytest.mark.parametrize("P", [2, 4])
+def test_cp_full_selection_is_causal_sdpa_over_the_whole_sequence(P):
+    """L = 1 and S = N: every shard selects all of its tokens, the concatenated
+    sub-sequence is the whole sequence in order, and the layer is causal SDPA over
+    all N tokens (forward and gradients, torch fp64 autograd) whatever the shard
+    count -- the shards only split the work."""
+    N, d = 256, 8
+    s = Shape(1, 2, N, d, 2, 1, N)
+    rng = np.random.default_rng(5 + P)
+    q, k, v, dO = (rng.standard_normal((1, 2, N, d)) for _ in range(4))
+    f = oracle.cp_forward(s, q, k, v, P)
+    g = oracle.cp_backward(s, f, dO)
+    tq, tk, tv = (torch.tensor(x, requires_grad=True) for x in (q, k, v))
+    ref = torch.nn.functional.scaled_dot_product_attention(tq, tk, tv, is_causal=True)
+    ref.backward(torch.tensor(dO))
+    assert np.allclose(f["o"], ref.detach().numpy(), atol=1e-12)
+    for name, t in (("dq", tq), ("dk", tk), ("dv", tv)):
+        assert np.allclose(g[name], t.grad.numpy(), atol=1e-11), name
+
+
+def test_cp_selection_is_per_shard_and_ordered():
+    """Each shard spends exactly S/P entries on its own tokens (a shard's high
+    scores cannot take another shard's budget), and the concatenated
+    sub-sequence is in (position, level) order over the whole sequence."""
+    P = 4
+    s = Shape(1, 1, 1024, 8, 4, 3, 128)
+    rng = np.random.default_rng(8)
+    q, k, v = (rng.standard_normal((1, 1, 1024, 8)) for _ in range(3))
+    q[:, :, :256] *= 10.0  # shard 0 has all the high norms; it still gets S/P entries only
+    k[:, :, :256] *= 10.0
+    f = oracle.cp_forward(s, q, k, v, P)
+    n, sp = 1024 // P, 128 // P
+    for r, part in enumerate(f["parts"]):
+        assert part["idx"].shape[-1] == sp
+        assert np.all((part["pos"] >= r * n) & (part["pos"] < (r + 1) * n))
+    pos = f["pos"][0, 0]
+    sh = f["shard"]
+    offs = np.array([sh.level_off(l) for l in range(1, sh.L)])
+    lev = np.concatenate([np.searchsorted(offs, part["idx"][0, 0], side="right") for part in f["parts"]])
+    keys = pos.astype(np.int64) * 16 + lev
+    assert np.all(np.diff(keys) > 0)
