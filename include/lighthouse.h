@@ -228,6 +228,14 @@ lh_status lh_forward(const lh_shape* shape, lh_dtype dtype, const void* q, const
                      const void* v, float scale, void* o, void* saved, void* ws,
                      size_t ws_bytes, lh_stream_t stream);
 
+/* How lh_forward gathers the sub-sequence for this shape: 0 through the fp32
+ * pyramid levels (lh_build_pyramid_score + lh_gather), 1 pooled from the input
+ * rows of each selected span (lh_score + lh_gather_pooled, no level written:
+ * chosen when even S entries all at the coarsest level read fewer bytes, with a
+ * margin of 4, than the levels take to write); -1 for an invalid shape or
+ * dtype.  Both give the same bits.  Host-only. */
+int lh_forward_gather_path(const lh_shape* shape, lh_dtype dtype);
+
 /* Whole backward with the saved selection: (f'), (e'), (d').  dO: [B,H,N,d]
  * dtype; dq, dk, dv: [B,H,N,d] dtype.  ws: lh_workspace_bytes(shape, dtype, 1). */
 lh_status lh_backward(const lh_shape* shape, lh_dtype dtype, const void* saved, const void* dO,

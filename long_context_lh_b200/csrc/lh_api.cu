@@ -138,6 +138,24 @@ lh_status attn_fwd(const Geom& g, const __half* qs, const __half* ks,
   return cuda_status(launch_attn_fwd_mma(g, qs, ks, vs, scale, os, lse, st));
 }
 
+// How lh_forward gathers the sub-sequence.  The pyramid path writes every fp32
+// level (12 (M - N) d bytes per unit) and reads S rows back; the pooled path
+// writes no level and reads, for each selected entry of level l, its p^l input
+// rows.  The selection is unknown when the path is chosen (no host sync), so the
+// rule takes the worst case, all S entries at the coarsest level: the pooled
+// path when S p^(L-1) rows of Q, K, V, with a margin of 4 for the pooled
+// kernel's per-span reads, cost less than the level writes.  For the
+// benchmark workloads the selections cover 1.27-1.38 N rows of spans and the
+// pyramid path is the faster one (measured: 0.29 vs 1.21 ms at the pretraining
+// shape), which the rule picks; small budgets over long inputs take the pooled path.
+bool use_pooled_gather(const Geom& g, lh_dtype dt) {
+  if (g.L == 1) return false;
+  const double s = dt == LH_BF16 ? 2.0 : 4.0;
+  const double worst = 4.0 * (double)g.S * (double)g.pw[g.L - 1] * 3.0 * g.d * s;
+  const double levels = 12.0 * (double)(g.M - g.N) * g.d;
+  return worst < levels;
+}
+
 // The geometry of a shape with the variant options applied (options validated).
 Geom geom_with(const lh_shape& shape, const lh_options* opt) {
   Geom g = make_geom(shape);
@@ -446,9 +464,17 @@ lh_status lh_forward_ex(const lh_shape* shape, lh_dtype dtype, const void* q, co
   float* pv = g.L > 1 ? reinterpret_cast<float*>(w + wl.off[kPv]) : nullptr;
   float* score = reinterpret_cast<float*>(w + wl.off[kScore]);
 
-  LH_TRY(launch_pyramid_score(g, dtype, q, k, v, pq, pk, pv, score, stream));
-  LH_TRY(launch_topk(g, score, idx, pos, slot, stream));
-  LH_TRY(launch_gather(g, dtype, q, k, v, pq, pk, pv, idx, qs, ks, vs, stream));
+  if (use_pooled_gather(g, dtype)) {
+    // scores only (no pyramid level written), then each selected coarse entry
+    // pooled from its span of input rows: the same bits as the pyramid gather
+    LH_TRY(launch_pyramid_score(g, dtype, q, k, nullptr, nullptr, nullptr, nullptr, score, stream));
+    LH_TRY(launch_topk(g, score, idx, pos, slot, stream));
+    LH_TRY(launch_gather_pooled(g, dtype, q, k, v, idx, qs, ks, vs, stream));
+  } else {
+    LH_TRY(launch_pyramid_score(g, dtype, q, k, v, pq, pk, pv, score, stream));
+    LH_TRY(launch_topk(g, score, idx, pos, slot, stream));
+    LH_TRY(launch_gather(g, dtype, q, k, v, pq, pk, pv, idx, qs, ks, vs, stream));
+  }
   s = attn_fwd(g, qs, ks, vs, resolve_scale(g, scale), os, lse, stream);
   if (s != LH_OK) return s;
   LH_TRY(launch_scatter(g, dtype, os, slot, o, ic, stream));
@@ -508,6 +534,11 @@ lh_status lh_read_device_status(lh_stream_t stream, uint32_t* code) {
   }
   if (code) *code = v;
   return v ? LH_ERR_DEVICE_STATUS : LH_OK;
+}
+
+int lh_forward_gather_path(const lh_shape* shape, lh_dtype dtype) {
+  if (lh_validate(shape, dtype) != LH_OK) return -1;
+  return use_pooled_gather(make_geom(*shape), dtype) ? 1 : 0;
 }
 
 int lh_set_attention_impl(int impl) {

@@ -107,6 +107,7 @@ _SIGS = {
     "lh_block_attn_bwd": ([_SP, _I, _VP, _VP, _VP, _VP, _VP, _VP, _F, _VP, _VP, _VP, _VP, _SZ,
                            _VP], _I),
     "lh_accumulate": ([_I64, _VP, _VP, _VP], _I),
+    "lh_forward_gather_path": ([_SP, _I], _I),
     "lh_scatter_back": ([_SP, _I, _VP, _VP, _VP, _VP, _VP], _I),
     "lh_scatter_back_bwd": ([_SP, _I, _VP, _VP, _VP, _VP, _VP], _I),
     "lh_gather_bwd": ([_SP, _I, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP], _I),
@@ -216,6 +217,10 @@ def lh_set_attention_impl(impl: int) -> int:
 
 def lh_attention_impl_in_use() -> int:
     return int(_lib().lh_attention_impl_in_use())
+
+
+def lh_forward_gather_path(shape: Shape, dtype: int) -> int:
+    return int(_lib().lh_forward_gather_path(ctypes.byref(shape), int(dtype)))
 
 
 def lh_kernel_launches(shape: Shape, dtype: int, backward: bool) -> int:

@@ -138,3 +138,15 @@ def test_options_are_checked_on_the_host():
                               None, None) == lh.LH_ERR_WORKSPACE
     assert lib.lh_scatter_back_ex(ctypes.byref(shp), lh.LH_BF16, p, p, p + 4, None, None,
                                   None) == lh.LH_ERR_INVALID_ARG
+
+
+def test_forward_gather_path_rule():
+    """lh_forward gathers through the pyramid for the benchmark workloads (their
+    worst-case spans are far more rows than the levels) and pooled from the input
+    for a small budget over a long input; invalid shapes give -1."""
+    for shp in (S(1, 16, 98304, 64, 4, 4, 8192), S(1, 16, 524288, 64, 4, 5, 16384),
+                S(1, 8, 1048576, 128, 4, 6, 16384), S()):
+        assert lh.lh_forward_gather_path(shp, lh.LH_BF16) == 0
+    assert lh.lh_forward_gather_path(S(1, 2, 65536, 64, 4, 3, 256), lh.LH_BF16) == 1
+    assert lh.lh_forward_gather_path(S(1, 1, 100, 64, 2, 1, 100), lh.LH_BF16) == 0  # L = 1: no level
+    assert lh.lh_forward_gather_path(S(d=96), lh.LH_BF16) == -1

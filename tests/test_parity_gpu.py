@@ -688,3 +688,35 @@ def test_finite_inputs_beyond_fp16_are_clipped_and_reported():
     x2 = to_dev(make_inputs(w, "cpu"))
     lh.forward(x2["q"], x2["k"], x2["v"], w.p, w.L, w.S)
     assert lh.lh_read_device_status() == 0
+
+
+def test_forward_pooled_path_matches_oracle_and_pyramid_stages():
+    """A small budget over a long input makes lh_forward gather pooled rows (no
+    pyramid level written).  Its selection and output must match the oracle, and
+    its gathered rows must be bitwise those of the pyramid stage path."""
+    w = workload(dtype="bf16", dist="outliers", N=65536, S=256, L=3, H=2)
+    shp = lshape(w)
+    assert lh.lh_forward_gather_path(shp, lh.LH_BF16) == 1
+    xc = make_inputs(w, "cpu")
+    x = to_dev(xc)
+    o, saved = lh.forward(x["q"], x["k"], x["v"], w.p, w.L, w.S)
+    dq, dk, dv = lh.backward(saved, x["dO"])
+    torch.cuda.synchronize()
+    sv = lambda which: lh.saved_view(saved.shape, saved.buf, which)
+    s = oshape(w)
+    f = [xc[n].float().numpy() for n in ("q", "k", "v", "dO")]
+    ref = oracle.forward(s, *f[:3])
+    assert np.array_equal(sv(lh.SAVED_IDX).cpu().numpy(), ref["idx"])
+    check_attn(f64(o), ref["o"], "o", o.dtype)
+    bref = oracle.backward(s, ref, f[3])
+    for name, t in (("dq", dq), ("dk", dk), ("dv", dv)):
+        check_attn(f64(t), bref[name], name, t.dtype)
+    # the pyramid stage path on the same selection gives the same rows, bit for bit
+    M = lh.lh_num_entries(shp)
+    pyr = [torch.empty((w.B, w.H, M - w.N, w.d), dtype=torch.float32, device=DEV) for _ in range(3)]
+    lh.lh_build_pyramid(shp, lh.LH_BF16, x["q"], x["k"], x["v"], *pyr)
+    rows = [torch.empty((w.B, w.H, w.S, w.d), dtype=torch.float16, device=DEV) for _ in range(3)]
+    lh.lh_gather(shp, lh.LH_BF16, x["q"], x["k"], x["v"], *pyr, sv(lh.SAVED_IDX), *rows)
+    torch.cuda.synchronize()
+    for got, which in zip(rows, (lh.SAVED_QS, lh.SAVED_KS, lh.SAVED_VS)):
+        assert torch.equal(got, sv(which))
