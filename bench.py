@@ -48,14 +48,14 @@ PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # kernel that evicts them, so a stage that writes more than L2 holds reads low.
 MEASURED_TRAFFIC = {  # workload: {stage: (bytes per launch, sources, sha1[:16])}
     "pretrain": {
-        "pyramid_score": (9.6650e+08, ('k_pyramid.cu', 'lh_internal.cuh'), "72509e86a0d1d4f2"),
-        "topk": (8.4000e+06, ('k_topk.cu', 'lh_internal.cuh'), "56d3e32b77bf9427"),
-        "gather": (9.6800e+07, ('k_gather_scatter.cu', 'lh_internal.cuh'), "74de98f31e4efd8e"),
-        "scatter": (1.6990e+08, ('k_gather_scatter.cu', 'lh_internal.cuh'), "74de98f31e4efd8e"),
-        "scatter_bwd": (2.2560e+08, ('k_gather_scatter.cu', 'lh_internal.cuh'), "74de98f31e4efd8e"),
-        "gather_bwd": (6.5820e+08, ('k_gather_scatter.cu', 'lh_internal.cuh'), "74de98f31e4efd8e"),
-        "attn_fwd": (5.0426e+07, ('k_attn_tc.cu', 'tc_common.cuh'), "65342d0b26370f8f"),
-        "attn_bwd": (1.9414e+08, ('k_attn_tc.cu', 'tc_common.cuh', 'k_gather_scatter.cu', 'lh_internal.cuh'), "6d238bb3c391ff16"),
+        "pyramid_score": (9.6650e+08, ('k_pyramid.cu', 'lh_internal.cuh'), "ac25a7b7b8340a38"),
+        "topk": (8.4000e+06, ('k_topk.cu', 'lh_internal.cuh'), "95620aa77e463653"),
+        "gather": (9.9000e+07, ('k_gather_scatter.cu', 'lh_internal.cuh'), "17fe79fe62f5a233"),
+        "scatter": (1.7010e+08, ('k_gather_scatter.cu', 'lh_internal.cuh'), "17fe79fe62f5a233"),
+        "scatter_bwd": (2.2550e+08, ('k_gather_scatter.cu', 'lh_internal.cuh'), "17fe79fe62f5a233"),
+        "gather_bwd": (6.5820e+08, ('k_gather_scatter.cu', 'lh_internal.cuh'), "17fe79fe62f5a233"),
+        "attn_fwd": (5.0500e+07, ('k_attn_tc.cu', 'tc_common.cuh', 'lh_internal.cuh'), "efccb5d61cea44c3"),
+        "attn_bwd": (1.9390e+08, ('k_attn_tc.cu', 'tc_common.cuh', 'k_gather_scatter.cu', 'lh_internal.cuh'), "d8362c7daed41782"),
     },
 }
 
