@@ -112,6 +112,69 @@ def algorithmic(w, span_rows=None):
 
 
 # --------------------------------------------------------------------- clocks
+class NvmlClockSampler:
+    """SM clock and throttle reasons of this process's GPU every ~2 ms through NVML
+    (read only), so that a timed region of a few tens of milliseconds has samples;
+    `window` marks the timed region (host clock) and the summary keeps the
+    samples inside it."""
+    HW_SLOWDOWN, SW_POWER_CAP, SW_THERMAL, HW_THERMAL = 0x8, 0x4, 0x20, 0x40
+
+    def __init__(self, device: torch.device):
+        import pynvml
+        self.nv = pynvml
+        pynvml.nvmlInit()
+        p = torch.cuda.get_device_properties(device)
+        bus = f"{p.pci_domain_id:08x}:{p.pci_bus_id:02x}:{p.pci_device_id:02x}.0"
+        self.h = pynvml.nvmlDeviceGetHandleByPciBusId(bus.encode())
+        self.max = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+        self.reasons_fn = getattr(pynvml, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+            pynvml.nvmlDeviceGetCurrentClocksThrottleReasons
+        self.samples, self.windows, self.stop = [], [], False
+
+    def __enter__(self):
+        self.thread = threading.Thread(target=self._run, daemon=True)
+        self.thread.start()
+        return self
+
+    def _run(self):
+        nv = self.nv
+        while not self.stop:
+            try:
+                sm = nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM)
+                rs = self.reasons_fn(self.h)
+                self.samples.append((time.perf_counter(), sm, rs))
+            except Exception:
+                pass
+            time.sleep(0.002)
+
+    def window(self, t0, t1):
+        self.windows.append((t0, t1))
+
+    def __exit__(self, *a):
+        self.stop = True
+        self.thread.join(timeout=1)
+
+    def summary(self):
+        inside = [smp for smp in self.samples if any(a <= smp[0] <= b for a, b in self.windows)]
+        reasons = set()
+        for _, _, rs in inside:
+            for bit, name in ((self.HW_SLOWDOWN, "hw_slowdown"), (self.HW_THERMAL, "hw_thermal_slowdown"),
+                              (self.SW_THERMAL, "sw_thermal_slowdown"), (self.SW_POWER_CAP, "sw_power_cap")):
+                if rs & bit:
+                    reasons.add(name)
+        sm = [smp[1] for smp in inside]
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": float(self.max),
+                "reasons": sorted(reasons), "samples": len(sm), "source": "nvml, every 2 ms"}
+
+
+def clock_sampler(local_rank: int, device: torch.device):
+    """The NVML sampler, or nvidia-smi's 50 ms loop where NVML is unavailable."""
+    try:
+        return NvmlClockSampler(device)
+    except Exception:
+        return ClockSampler(local_rank)
+
+
 class ClockSampler:
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
@@ -137,6 +200,9 @@ class ClockSampler:
     def _read(self):
         for line in self.proc.stdout:
             self.lines.append(line.strip())
+
+    def window(self, t0, t1):
+        pass
 
     def __exit__(self, *a):
         if self.proc:
@@ -200,29 +266,36 @@ def measure(lh, w, args, rk, dev, peaks, steps, warmup, backward=True, batch=0, 
         if backward:
             lh.lh_backward(shp, dt, saved, dO, 0.0, dq, dk, dv, ws, wsb, sp)
 
-    def timed(fn, K):
+    def timed(fn, K, clk=None):
         """Device time of K calls on this rank; the max over ranks is returned."""
         replicas.barrier(rk)
         torch.cuda.synchronize()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        h0 = time.perf_counter()
         e0.record(stream)
         for _ in range(K):
             fn()
         e1.record(stream)
         torch.cuda.synchronize()
+        if clk is not None:
+            clk.window(h0, time.perf_counter())
         ms = e0.elapsed_time(e1)
         replicas.barrier(rk)
         return replicas.max_over_ranks(rk, ms, dev)
 
-    clk = ClockSampler(rk.local_rank) if clocks else None
+    clk = clock_sampler(rk.local_rank, dev) if clocks else None
     with torch.cuda.stream(stream):
+        if clk:
+            clk.__enter__()  # sampling from the warm-up on; the summary keeps the timed region
         for _ in range(warmup):
             step()
         torch.cuda.synchronize()
         status = lh.lh_read_device_status(stream)
         if clk:
-            with clk:
-                ms_step = timed(step, steps) / steps
+            try:
+                ms_step = timed(step, steps, clk) / steps
+            finally:
+                clk.__exit__(None, None, None)
         else:
             ms_step = timed(step, steps) / steps
         ms_fwd = timed(fwd_only, steps) / steps if backward else ms_step

@@ -666,15 +666,13 @@ __global__ void __launch_bounds__(kThreads, 1)
            warp_wait(&bars->s_full, t & 1, abort, kStatus);
       if (!ok) return;
       tc_fence_after();
-      uint32_t a0[32], a1[32], b0[32], b1[32];
-      tmem_ld32(tST + lane_addr + h * 64, a0);
-      tmem_ld32(tST + lane_addr + h * 64 + 32, a1);
-      tmem_ld32(tDPT + lane_addr + h * 64, b0);
-      tmem_ld32(tDPT + lane_addr + h * 64 + 32, b1);
+      // this row's 64 query columns of S^T and dP^T in two 32-column halves (the
+      // second loaded once the first is consumed: the registers they free let a
+      // quarter of the exponentials run on the FMA pipe without spilling)
+      uint32_t a[32], b[32];
+      tmem_ld32(tST + lane_addr + h * 64, a);
+      tmem_ld32(tDPT + lane_addr + h * 64, b);
       tmem_ld_wait();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bars->st_free);  // S^T, dP^T are in registers now
       const float4* cl = reinterpret_cast<const float4*>(sStat + st * 256 + h * 64);        // -lse2
       const float4* cd = reinterpret_cast<const float4*>(sStat + st * 256 + 128 + h * 64);  // -D
       const int lim = r - h * 64;  // query columns e < lim precede the key
@@ -687,7 +685,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                                 make_float2(nl.x, nl.y));
         const float2 x1 = ffma2(make_float2(__uint_as_float(sv[k + 2]), __uint_as_float(sv[k + 3])), cc,
                                 make_float2(nl.z, nl.w));
-        float2 p0 = make_float2(ex2(x0.x), ex2(x0.y)), p1 = make_float2(ex2(x1.x), ex2(x1.y));
+        // a quarter of the exponentials on the FMA pipe (this row work is MUFU-bound)
+        float2 p0 = make_float2(ex2(x0.x), ex2(x0.y));
+        float2 p1 = (e & 4) ? ex2_fma2(x1) : make_float2(ex2(x1.x), ex2(x1.y));
         if (kDiag) {
           p0.x = e < lim ? 0.0f : p0.x;
           p0.y = e + 1 < lim ? 0.0f : p0.y;
@@ -704,10 +704,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         pd[(e >> 1) + 1] = h2_sat(d1.x, d1.y);
       };
 #pragma unroll
-      for (int e = 0; e < 32; e += 4) {
-        quad(e, a0, b0);
-        quad(e + 32, a1, b1);
-      }
+      for (int e = 0; e < 32; e += 4) quad(e, a, b);
+      tmem_ld32(tST + lane_addr + h * 64 + 32, a);
+      tmem_ld32(tDPT + lane_addr + h * 64 + 32, b);
+      tmem_ld_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars->st_free);  // S^T, dP^T are in registers now
+#pragma unroll
+      for (int e = 32; e < 64; e += 4) quad(e, a, b);
       if (t > 0 && !(ok = warp_wait(&bars->pdone, (t - 1) & 1, abort, kStatus))) return;
       if constexpr (kTmemP) {  // this row's 64 query columns = 32 packed columns
         tmem_st32(tPT + lane_addr + h * 32, pp);
