@@ -7,14 +7,19 @@
 // sub-sequence (row k sees k' <= k), scale 1/sqrt(d); §2.B: its backward is the
 // only path from the layer output back to the selected Q, K and V.
 //
-// All three kernels use one CTA per SM (512 TMEM columns) and 10 warps:
+// All three kernels use one CTA per SM (512 TMEM columns) and 11 warps:
 //   warps 0-7  the row work (TMEM lane = row; warp w reads lanes 32*(w%4)..):
 //              in the forward, one thread per row of one of two query tiles
 //              (warps 0-3 tile A, 4-7 tile B, ping-pong); in the two backward
 //              kernels, two threads per row of the one 128-row tile, warp w
 //              taking the column half w/4;
 //   warp 8     TMA producer (one lane issues);
-//   warp 9     MMA issuer (one lane) and owner of the TMEM allocation.
+//   warps 9-10 MMA issuers, on two SM sub-partitions: each waits as a whole
+//              converged warp and one elected lane issues.  Warp 9 issues the
+//              score products (S, or S^T and dP^T, or S and dP), warp 10 the
+//              products that consume them (P V, or dV and dK, or dQ); at d = 128
+//              the forward issues from warp 9 alone.  Warp 9 owns the TMEM
+//              allocation.
 // The backward kernels read a score tile from TMEM into registers in one go
 // and release the buffer at once, so the next tile's products run while the
 // row work goes on; the forward releases it after its second read.
