@@ -195,7 +195,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     // that load).  At d = 128 P lives over S, so S_T(j+1) must follow
     // O_T += P_T(j) V_j in one in-order stream: warp 9 issues everything.
     // A descriptor for base + off is the base descriptor plus off / 16 (the
-    // 14-bit address field never overflows inside shared memory).
+    // 14-bit address field never overflows inside shared memory).  At d = 64
+    // the two issuers sleep 16 ns between polls of a barrier (spinning, each
+    // slowed the row-work warps of its sub-partition: forward 190 -> 184 us at
+    // the pretraining shape with the sleep); the backward's issuers sit on the
+    // critical handoffs and poll without sleeping (the same sleep there: 509 ->
+    // 541 us).
+    constexpr uint32_t kIssuerSleepNs = 16;
     {
       constexpr uint32_t idS = idesc_f16(128, 128, false);
       constexpr uint32_t idPV = idesc_f16(128, D, true);
@@ -240,12 +246,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (warp == 9) {
           // S_T(j+1) once S_T(j) is read (and K_{j+1} is in place), tile A then B
           for (int j = 0; ok && j + 1 < nA; ++j) {
-            if (!(ok = warp_wait(&bars->s_free[0], j & 1, abort, kStatus))) break;
-            if (!(ok = warp_wait(&bars->kv_full[(j + 1) % KS], ((j + 1) / KS) & 1, abort, kStatus))) break;
+            if (!(ok = warp_wait_sleep(&bars->s_free[0], j & 1, abort, kStatus, kIssuerSleepNs))) break;
+            if (!(ok = warp_wait_sleep(&bars->kv_full[(j + 1) % KS], ((j + 1) / KS) & 1, abort, kStatus, kIssuerSleepNs))) break;
             tc_fence_after();
             issue_s(0, j + 1);
             if (j + 1 < nB) {  // K_{j+1} is in place (waited for above: j + 1 < nB <= nA)
-              if (!(ok = warp_wait(&bars->s_free[1], j & 1, abort, kStatus))) break;
+              if (!(ok = warp_wait_sleep(&bars->s_free[1], j & 1, abort, kStatus, kIssuerSleepNs))) break;
               tc_fence_after();
               issue_s(1, j + 1);
             }
@@ -255,11 +261,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           // are free (S_A(j), S_B(j) completed before the row work wrote P)
           for (int j = 0; ok && j < nA; ++j) {
             const int st = j % KS;
-            if (!(ok = warp_wait(&bars->p_full[0], j & 1, abort, kStatus))) break;
+            if (!(ok = warp_wait_sleep(&bars->p_full[0], j & 1, abort, kStatus, kIssuerSleepNs))) break;
             tc_fence_after();
             issue_pv(0, j);
             if (j < nB) {
-              if (!(ok = warp_wait(&bars->p_full[1], j & 1, abort, kStatus))) break;
+              if (!(ok = warp_wait_sleep(&bars->p_full[1], j & 1, abort, kStatus, kIssuerSleepNs))) break;
               tc_fence_after();
               issue_pv(1, j);
             }

@@ -124,6 +124,25 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volati
   return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort, code, honor_abort));
 }
 
+// warp_wait for a warp that only issues MMAs: between polls it sleeps `ns`
+// nanoseconds, leaving the issue slots of its SM sub-partition to the row-work
+// warps there (a spinning issuer measurably slows them).  Bounded like mbar_wait.
+__device__ __forceinline__ bool warp_wait_sleep(uint64_t* bar, uint32_t parity, volatile int* abort,
+                                                uint32_t code, uint32_t ns) {
+  if (__all_sync(0xffffffffu, mbar_test_wait(bar, parity))) return true;
+  const uint64_t t0 = global_ns();
+  for (;;) {
+    __nanosleep(ns);
+    if (__all_sync(0xffffffffu, mbar_test_wait(bar, parity))) return true;
+    if (__any_sync(0xffffffffu, global_ns() - t0 > kWaitLimitNs)) {
+      if ((threadIdx.x & 31) == 0) report_status(code);
+      *abort = 1;
+      return false;
+    }
+    if (__any_sync(0xffffffffu, *abort != 0)) return false;
+  }
+}
+
 // --------------------------------------------------------------------- TMA
 // Untiled bulk copy of `bytes` from global to shared memory, completing on
 // `bar`.  Both addresses 16-byte aligned, bytes a multiple of 16.
