@@ -54,8 +54,8 @@ MEASURED_TRAFFIC = {  # workload: {stage: (bytes per launch, sources, sha1[:16])
         "scatter": (1.7010e+08, ('k_gather_scatter.cu', 'lh_internal.cuh'), "17fe79fe62f5a233"),
         "scatter_bwd": (2.2550e+08, ('k_gather_scatter.cu', 'lh_internal.cuh'), "17fe79fe62f5a233"),
         "gather_bwd": (6.5820e+08, ('k_gather_scatter.cu', 'lh_internal.cuh'), "17fe79fe62f5a233"),
-        "attn_fwd": (5.0500e+07, ('k_attn_tc.cu', 'tc_common.cuh', 'lh_internal.cuh'), "16ea4ffa2f846348"),
-        "attn_bwd": (1.9390e+08, ('k_attn_tc.cu', 'tc_common.cuh', 'k_gather_scatter.cu', 'lh_internal.cuh'), "7ab453ece30671a5"),
+        "attn_fwd": (5.0400e+07, ('k_attn_tc.cu', 'tc_common.cuh', 'lh_internal.cuh'), "202d9cf1e39f0aac"),
+        "attn_bwd": (1.9370e+08, ('k_attn_tc.cu', 'tc_common.cuh', 'k_gather_scatter.cu', 'lh_internal.cuh'), "7aab4813c8a3ea67"),
     },
 }
 
