@@ -320,6 +320,10 @@ def measure(lh, w, args, rk, dev, peaks, steps, warmup, backward=True, batch=0, 
     npyr = max(U * (M - w.N) * w.d, 1)
     pq, pk, pv = (torch.empty(npyr, dtype=torch.float32, device=dev) for _ in range(3))
     score = torch.empty(U * M, dtype=torch.float32, device=dev)
+    # the selection as lh_forward runs it: device-wide passes (with a workspace) or
+    # one cluster per unit (without)
+    tbw = lh.lh_topk_workspace_bytes(shp) if lh.lh_forward_topk_path(shp) == 1 else 0
+    tws = torch.empty(tbw, dtype=torch.uint8, device=dev) if tbw else None
     if backward:
         dos = torch.empty(U * w.S * w.d, dtype=torch.float16, device=dev)
         dqs, dks, dvs = (torch.empty(U * w.S * w.d, dtype=torch.float32, device=dev) for _ in range(3))
@@ -332,7 +336,7 @@ def measure(lh, w, args, rk, dev, peaks, steps, warmup, backward=True, batch=0, 
         # end per stage)
         launches = [
             lambda: lh.lh_build_pyramid_score(shp, dt, q, k, v, pq, pk, pv, score, sp),
-            lambda: lh.lh_topk_select(shp, score, idx, pos, slot, None, 0, sp),
+            lambda: lh.lh_topk_select(shp, score, idx, pos, slot, tws, tbw, sp),
             lambda: lh.lh_gather(shp, dt, q, k, v, pq, pk, pv, idx, qs, ks, vs, sp),
             lambda: lh.lh_subseq_attn_fwd(shp, qs, ks, vs, 0.0, os_, lse, sp),
             lambda: lh.lh_scatter_back(shp, dt, os_, slot, o, ic, sp),

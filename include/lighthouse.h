@@ -133,7 +133,11 @@ lh_status lh_score(const lh_shape* shape, lh_dtype dtype, const void* q, const v
  * (score, -gid), then ordered by (pos, level), [ES] §2.C.
  * idx, pos: int32 [B,H,S] (gid and position of slot k); slot: int32 [B,H,M]
  * (slot of each entry, -1 if not selected).  Scores must be >= 0 (they are
- * sums of norms).  ws may be NULL when lh_topk_workspace_bytes() is 0.       */
+ * sums of norms).  Two implementations, the same bits: with ws = NULL one
+ * thread-block cluster per unit keeps all its state in distributed shared
+ * memory; with a workspace of lh_topk_workspace_bytes() (16-byte aligned,
+ * owned by the caller, overwritten) the selection runs as device-wide passes
+ * over every SM (what lh_forward uses); a smaller one is LH_ERR_WORKSPACE.   */
 size_t lh_topk_workspace_bytes(const lh_shape* shape);
 lh_status lh_topk_select(const lh_shape* shape, const float* score, int32_t* idx, int32_t* pos,
                          int32_t* slot, void* ws, size_t ws_bytes, lh_stream_t stream);
@@ -235,6 +239,12 @@ lh_status lh_forward(const lh_shape* shape, lh_dtype dtype, const void* q, const
  * margin of 4, than the levels take to write); -1 for an invalid shape or
  * dtype.  Both give the same bits.  Host-only. */
 int lh_forward_gather_path(const lh_shape* shape, lh_dtype dtype);
+
+/* How lh_forward runs the selection for this shape: 0 one thread-block cluster
+ * per unit (lh_topk_select without a workspace), 1 device-wide passes (with
+ * one: units of more than 2^19 entries); -1 for an invalid shape.  Both give
+ * the same bits.  Host-only. */
+int lh_forward_topk_path(const lh_shape* shape);
 
 /* Whole backward with the saved selection: (f'), (e'), (d').  dO: [B,H,N,d]
  * dtype; dq, dk, dv: [B,H,N,d] dtype.  ws: lh_workspace_bytes(shape, dtype, 1). */

@@ -640,4 +640,378 @@ cudaError_t launch_topk(const Geom& g, const float* score, int32_t* idx, int32_t
   }
 }
 
+
+// ================================================== device-wide pass selection
+// The same selection and slots as k_topk, as a sequence of short kernels over
+// all SMs instead of one thread-block cluster per unit (a unit's passes then run
+// on every SM, not on one GPC's; large units need no second wave of clusters).
+// State between the kernels lives in a per-unit workspace (zeroed first):
+//   hist[3][2048]  the three digit histograms of the key bits (high to low),
+//   st[16]         the radix state after each digit and the threshold (kSt*),
+//   tie_n, tie[kSelTies]  gids of the keys equal to the threshold, if needed,
+//   cnt[nbt]       selected entries per token block (for the slot offsets).
+// Every kernel takes a warp-uniform view of the same integers, so the result is
+// the cluster kernel's, bit for bit.
+namespace {
+
+constexpr int kSelThreads = 1024;
+constexpr int kSelKeys = 16384;    // keys per CTA of a histogram pass
+constexpr int kSelTokens = 8192;   // tokens per CTA of the count / write passes
+constexpr int kSelTies = 4096;     // ties at the threshold resolved from a list
+// state words: after digit 0 (written by pass 1), after digit 1 (pass 2), the
+// threshold (tie pass) and the largest tie gid that fits (resolve)
+enum : int {
+  kSt1Prefix = 0, kSt1Mask, kSt1Need, kSt2Prefix, kSt2Mask, kSt2Need, kStT, kStNeed, kStTies, kStGid,
+  kStCount = 16
+};
+constexpr int kWsHist = 0, kWsSt = 3 * kBins, kWsTieN = kWsSt + kStCount, kWsTie = kWsTieN + 8,
+              kWsCnt = kWsTie + kSelTies;
+
+struct SelPrm {
+  TopkParams t;
+  int32_t stride;  // workspace words per unit
+  int32_t nbk;     // CTAs per unit of a histogram pass
+  int32_t nbt;     // CTAs per unit of the count / write passes
+  int32_t top;     // first gid of the coarsest level (ranked +inf when kept)
+};
+
+__device__ __forceinline__ uint32_t sel_key(const SelPrm& sp, const uint32_t* key, int32_t g) {
+  return (sp.t.keep_top && g >= sp.top) ? kTopBits : __ldg(key + g);
+}
+
+// Block-wide exclusive scan (kSelThreads threads) of one value per thread.
+__device__ uint32_t sel_excl_scan(uint32_t v, uint32_t* warp_buf, uint32_t* total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const uint32_t incl = warp_incl_scan(v);
+  if (lane == 31) warp_buf[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    const uint32_t w = warp_buf[lane];
+    const uint32_t wi = warp_incl_scan(w);
+    warp_buf[lane] = wi - w;
+    if (lane == 31) *total = wi;
+  }
+  __syncthreads();
+  const uint32_t r = warp_buf[warp] + incl - v;
+  __syncthreads();
+  return r;
+}
+
+// The digit of a (global) histogram of nb bins where the need-th key falls,
+// counting from the largest digit (descending) or the smallest.
+__device__ Pick sel_pick(const uint32_t* hist, int nb, bool descending, uint32_t need,
+                         uint32_t* warp_buf, uint32_t* sh) {
+  const int per = nb / kSelThreads;  // 2 or 1
+  uint32_t c[2] = {0, 0};
+  for (int i = 0; i < per; ++i) {
+    const int ord = (int)threadIdx.x * per + i;
+    c[i] = __ldcg(hist + (descending ? nb - 1 - ord : ord));
+  }
+  uint32_t all;
+  uint32_t before = sel_excl_scan(c[0] + c[1], warp_buf, &all);
+  for (int i = 0; i < per; ++i) {
+    const int ord = (int)threadIdx.x * per + i;
+    if (before < need && need <= before + c[i]) {
+      sh[0] = (uint32_t)(descending ? nb - 1 - ord : ord);
+      sh[1] = before;
+      sh[2] = c[i];
+    }
+    before += c[i];
+  }
+  __syncthreads();
+  const Pick pk{sh[0], sh[1], sh[2]};
+  __syncthreads();
+  return pk;
+}
+
+// Histogram pass PASS (0, 1, 2: key bits [21,32), [10,21), [0,10)) over keys
+// [b kSelKeys, (b+1) kSelKeys) of unit u, among the keys matching the digits
+// chosen so far.  PASS 1 picks digit 0 from hist[0] (CTA 0 records the state);
+// PASS 2 reads that state and picks digit 1 from hist[1].
+template <int PASS>
+__global__ void __launch_bounds__(kSelThreads) k_sel_hist(const float* __restrict__ score,
+                                                          uint32_t* __restrict__ ws, const SelPrm sp) {
+  __shared__ uint32_t h[kBins];
+  __shared__ uint32_t warp_buf[32], sh[4];
+  const int64_t u = sp.t.unit0 + blockIdx.y;
+  uint32_t* w = ws + (int64_t)blockIdx.y * sp.stride;
+  const uint32_t* key = reinterpret_cast<const uint32_t*>(score + u * sp.t.M);
+  constexpr int shift = PASS == 0 ? 21 : (PASS == 1 ? 10 : 0);
+  constexpr uint32_t dmask = PASS == 2 ? 1023u : 2047u;
+  uint32_t prefix = 0, pmask = 0, need = (uint32_t)sp.t.S;
+  if (PASS == 1) {
+    const Pick pk = sel_pick(w + kWsHist, 2048, true, need, warp_buf, sh);
+    prefix = pk.bin << 21;
+    pmask = 2047u << 21;
+    need -= pk.before;
+    if (blockIdx.x == 0 && threadIdx.x == 0) {
+      w[kWsSt + kSt1Prefix] = prefix;
+      w[kWsSt + kSt1Mask] = pmask;
+      w[kWsSt + kSt1Need] = need;
+    }
+  } else if (PASS == 2) {
+    prefix = __ldcg(w + kWsSt + kSt1Prefix);
+    pmask = __ldcg(w + kWsSt + kSt1Mask);
+    need = __ldcg(w + kWsSt + kSt1Need);
+    const Pick pk = sel_pick(w + kWsHist + kBins, 2048, true, need, warp_buf, sh);
+    prefix |= pk.bin << 10;
+    pmask |= 2047u << 10;
+    need -= pk.before;
+    if (blockIdx.x == 0 && threadIdx.x == 0) {  // the state after two digits (read by the tie pass)
+      w[kWsSt + kSt2Prefix] = prefix;
+      w[kWsSt + kSt2Mask] = pmask;
+      w[kWsSt + kSt2Need] = need;
+    }
+  }
+  for (int i = threadIdx.x; i < kBins; i += kSelThreads) h[i] = 0;
+  __syncthreads();
+  const int32_t i0 = (int32_t)blockIdx.x * kSelKeys;
+  const int32_t i1 = (int32_t)imin64(sp.t.M, (int64_t)i0 + kSelKeys);
+  for (int32_t j0 = i0 + (int32_t)(threadIdx.x & ~31u); j0 < i1; j0 += kSelThreads) {  // warp-uniform
+    const int32_t j = j0 + (int32_t)(threadIdx.x & 31);
+    const uint32_t kv = j < i1 ? sel_key(sp, key, j) : 0u;
+    const bool act = j < i1 && (kv & pmask) == prefix;
+    if (PASS == 0)
+      hist_add(h, act, (kv >> shift) & dmask);
+    else
+      hist_add_plain(h, act, (kv >> shift) & dmask);
+  }
+  __syncthreads();
+  uint32_t* gh = w + kWsHist + PASS * kBins;
+  for (int i = threadIdx.x; i < kBins; i += kSelThreads)
+    if (h[i]) atomicAdd(gh + i, h[i]);
+}
+
+// The threshold T (digit 2 from hist[2]), how many keys equal to T are still
+// needed and how many there are; CTA 0 records them.  When only some of the ties
+// fit, every CTA lists the gids of its keys equal to T (up to kSelTies).
+__global__ void __launch_bounds__(kSelThreads) k_sel_ties(const float* __restrict__ score,
+                                                          uint32_t* __restrict__ ws, const SelPrm sp) {
+  __shared__ uint32_t warp_buf[32], sh[4];
+  const int64_t u = sp.t.unit0 + blockIdx.y;
+  uint32_t* w = ws + (int64_t)blockIdx.y * sp.stride;
+  const uint32_t* key = reinterpret_cast<const uint32_t*>(score + u * sp.t.M);
+  const uint32_t prefix = __ldcg(w + kWsSt + kSt2Prefix);
+  uint32_t need = __ldcg(w + kWsSt + kSt2Need);
+  const Pick pk = sel_pick(w + kWsHist + 2 * kBins, 1024, true, need, warp_buf, sh);
+  const uint32_t T = prefix | pk.bin;
+  need -= pk.before;
+  const uint32_t ties = pk.inbin;
+  if (blockIdx.x == 0 && threadIdx.x == 0) {
+    w[kWsSt + kStT] = T;
+    w[kWsSt + kStNeed] = need;
+    w[kWsSt + kStTies] = ties;
+  }
+  if (!(need < ties)) return;
+  const int32_t i0 = (int32_t)blockIdx.x * kSelKeys;
+  const int32_t i1 = (int32_t)imin64(sp.t.M, (int64_t)i0 + kSelKeys);
+  for (int32_t j = i0 + (int32_t)threadIdx.x; j < i1; j += kSelThreads) {
+    if (sel_key(sp, key, j) != T) continue;
+    const uint32_t k = atomicAdd(w + kWsTieN, 1u);
+    if (k < (uint32_t)kSelTies) w[kWsTie + k] = (uint32_t)j;
+  }
+}
+
+// One CTA per unit: the largest gid among the ties that still fit (the need-th
+// smallest gid equal to T), or all of them.  From the list when it holds every
+// tie; else radix passes on the gids over all the unit's keys (only when more
+// than kSelTies entries share the threshold score).
+__global__ void __launch_bounds__(kSelThreads) k_sel_resolve(const float* __restrict__ score,
+                                                             uint32_t* __restrict__ ws, const SelPrm sp) {
+  __shared__ uint32_t h[kBins];
+  __shared__ uint32_t warp_buf[32], sh[4];
+  __shared__ uint32_t list[kSelTies];
+  const int64_t u = sp.t.unit0 + blockIdx.x;
+  uint32_t* w = ws + (int64_t)blockIdx.x * sp.stride;
+  const uint32_t* key = reinterpret_cast<const uint32_t*>(score + u * sp.t.M);
+  const uint32_t T = __ldcg(w + kWsSt + kStT);
+  uint32_t need = __ldcg(w + kWsSt + kStNeed);
+  const uint32_t ties = __ldcg(w + kWsSt + kStTies);
+  if (!(need < ties)) {
+    if (threadIdx.x == 0) w[kWsSt + kStGid] = 0x7fffffffu;  // every key equal to T fits
+    return;
+  }
+  const bool listed = ties <= (uint32_t)kSelTies;
+  if (listed)
+    for (uint32_t i = threadIdx.x; i < ties; i += kSelThreads) list[i] = __ldcg(w + kWsTie + i);
+  int nbits = 1;
+  while (nbits < 31 && ((int64_t)1 << nbits) < sp.t.M) ++nbits;
+  uint32_t gprefix = 0, gmask = 0;
+  for (int hi = nbits; hi > 0;) {
+    const int wd = hi >= 11 ? 11 : hi;
+    const int shift = hi - wd;
+    const uint32_t dmask = (1u << wd) - 1u;
+    for (int i = threadIdx.x; i < kBins; i += kSelThreads) h[i] = 0;
+    __syncthreads();
+    if (listed) {
+      for (uint32_t i = threadIdx.x; i < ties; i += kSelThreads) {
+        const uint32_t gid = list[i];
+        if ((gid & gmask) == gprefix) atomicAdd(&h[(gid >> shift) & dmask], 1u);
+      }
+    } else {
+      for (int32_t j = (int32_t)threadIdx.x; j < sp.t.M; j += kSelThreads)
+        if (sel_key(sp, key, j) == T && ((uint32_t)j & gmask) == gprefix)
+          atomicAdd(&h[((uint32_t)j >> shift) & dmask], 1u);
+    }
+    __syncthreads();
+    // ascending over the 2048 shared bins (digits of fewer bits leave the top empty)
+    uint32_t c[2] = {h[2 * threadIdx.x], h[2 * threadIdx.x + 1]};
+    uint32_t all;
+    uint32_t before = sel_excl_scan(c[0] + c[1], warp_buf, &all);
+    for (int i = 0; i < 2; ++i) {
+      if (before < need && need <= before + c[i]) {
+        sh[0] = 2 * threadIdx.x + i;
+        sh[1] = before;
+      }
+      before += c[i];
+    }
+    __syncthreads();
+    gprefix |= sh[0] << shift;
+    gmask |= dmask << shift;
+    need -= sh[1];
+    __syncthreads();
+    hi = shift;
+  }
+  if (threadIdx.x == 0) w[kWsSt + kStGid] = gprefix;
+}
+
+// Is the level-l entry g (span ending at token t) selected?
+__device__ __forceinline__ bool sel_in(const SelPrm& sp, const uint32_t* key, int32_t g, uint32_t T,
+                                       uint32_t gthr) {
+  const uint32_t kv = sel_key(sp, key, g);
+  return kv > T || (kv == T && (uint32_t)g <= gthr);
+}
+
+// Selected entries per block of kSelTokens tokens (enumerated at their span's end).
+__global__ void __launch_bounds__(kSelThreads) k_sel_count(const float* __restrict__ score,
+                                                           uint32_t* __restrict__ ws, const SelPrm sp) {
+  __shared__ uint32_t warp_buf[32], tot;
+  const int64_t u = sp.t.unit0 + blockIdx.y;
+  uint32_t* w = ws + (int64_t)blockIdx.y * sp.stride;
+  const uint32_t* key = reinterpret_cast<const uint32_t*>(score + u * sp.t.M);
+  const uint32_t T = __ldcg(w + kWsSt + kStT), gthr = __ldcg(w + kWsSt + kStGid);
+  const int32_t t0 = (int32_t)blockIdx.x * kSelTokens;
+  const int32_t t1 = (int32_t)imin64(sp.t.N, (int64_t)t0 + kSelTokens);
+  uint32_t c = 0;
+  for (int32_t t = t0 + (int32_t)threadIdx.x; t < t1; t += kSelThreads) {
+    const uint32_t tt = (uint32_t)t + 1u;
+#pragma unroll
+    for (int l = 0; l < kMaxLevels; ++l) {
+      if (l >= sp.t.L || !ends_at(sp.t, tt, l)) break;
+      c += sel_in(sp, key, gid_at(sp.t, tt, l), T, gthr) ? 1u : 0u;
+    }
+  }
+  sel_excl_scan(c, warp_buf, &tot);
+  if (threadIdx.x == 0) w[kWsCnt + blockIdx.x] = tot;
+}
+
+// idx, pos and the slot map: block b's entries take slots from the count of
+// blocks 0..b-1 on, in (token, level) order.
+__global__ void __launch_bounds__(kSelThreads) k_sel_write(const float* __restrict__ score,
+                                                           uint32_t* __restrict__ ws, int32_t* __restrict__ idx,
+                                                           int32_t* __restrict__ pos, int32_t* __restrict__ slot,
+                                                           const SelPrm sp) {
+  __shared__ uint32_t warp_buf[32], tot;
+  const int64_t u = sp.t.unit0 + blockIdx.y;
+  const uint32_t* w = ws + (int64_t)blockIdx.y * sp.stride;
+  const uint32_t* key = reinterpret_cast<const uint32_t*>(score + u * sp.t.M);
+  const uint32_t T = __ldcg(w + kWsSt + kStT), gthr = __ldcg(w + kWsSt + kStGid);
+  uint32_t base;
+  {  // entries of the blocks before this one
+    uint32_t part = 0;
+    for (int i = threadIdx.x; i < (int)blockIdx.x; i += kSelThreads) part += __ldcg(w + kWsCnt + i);
+    sel_excl_scan(part, warp_buf, &tot);
+    base = tot;
+  }
+  int32_t* idx_u = idx + u * sp.t.S;
+  int32_t* pos_u = pos + u * sp.t.S;
+  int32_t* slot_u = slot + u * sp.t.M;
+  const int32_t t0 = (int32_t)blockIdx.x * kSelTokens;
+  const int32_t t1 = (int32_t)imin64(sp.t.N, (int64_t)t0 + kSelTokens);
+  for (int32_t tb = t0; tb < t1; tb += kSelThreads) {  // block-uniform trip count
+    const int32_t t = tb + (int32_t)threadIdx.x;
+    const uint32_t tt = (uint32_t)t + 1u;
+    uint32_t mask = 0;
+    if (t < t1) {
+#pragma unroll
+      for (int l = 0; l < kMaxLevels; ++l) {
+        if (l >= sp.t.L || !ends_at(sp.t, tt, l)) break;
+        mask |= (sel_in(sp, key, gid_at(sp.t, tt, l), T, gthr) ? 1u : 0u) << l | 1u << (8 + l);
+      }
+    }
+    const uint32_t c = __popc(mask & 0xffu);
+    uint32_t k = base + sel_excl_scan(c, warp_buf, &tot);
+#pragma unroll
+    for (int l = 0; l < kMaxLevels; ++l) {
+      if (!((mask >> (8 + l)) & 1u)) break;
+      const int32_t g = gid_at(sp.t, tt, l);
+      if (!LH_CHECK(dbg::in_range(g, sp.t.M), kBoundsTopk)) break;
+      if ((mask >> l) & 1u) {
+        // exactly S entries are selected, so k < S; the test is kept in every build
+        if (LH_CHECK(dbg::in_range(k, sp.t.S), kBoundsTopk) && k < (uint32_t)sp.t.S) {
+          idx_u[k] = g;
+          pos_u[k] = t;
+          slot_u[g] = (int32_t)k;
+        }
+        ++k;
+      } else {
+        slot_u[g] = -1;
+      }
+    }
+    base += tot;
+  }
+}
+
+SelPrm sel_prm(const Geom& g) {
+  SelPrm sp;
+  TopkParams& prm = sp.t;
+  prm.N = (int32_t)g.N;
+  prm.M = (int32_t)g.M;
+  prm.p = g.p;
+  prm.L = g.L;
+  prm.S = g.S;
+  prm.log2p = ((g.p & (g.p - 1)) == 0) ? __builtin_ctz((unsigned)g.p) : -1;
+  prm.keep_top = g.keep_top;
+  prm.unit0 = 0;
+  for (int l = 0; l <= kMaxLevels; ++l) {
+    prm.off[l] = (int32_t)g.off[l];
+    prm.pw[l] = (int32_t)(g.pw[l] > 0x7fffffff ? 0x7fffffff : g.pw[l]);
+  }
+  sp.top = (int32_t)g.off[g.L - 1];
+  sp.nbk = (int32_t)((g.M + kSelKeys - 1) / kSelKeys);
+  sp.nbt = (int32_t)((g.N + kSelTokens - 1) / kSelTokens);
+  sp.stride = (kWsCnt + sp.nbt + 63) / 64 * 64;
+  return sp;
+}
+
+}  // namespace
+
+size_t topk_passes_workspace_bytes(const Geom& g) {
+  return (size_t)g.U * sel_prm(g).stride * sizeof(uint32_t);
+}
+
+cudaError_t launch_topk_passes(const Geom& g, const float* score, int32_t* idx, int32_t* pos,
+                               int32_t* slot, void* ws, cudaStream_t st) {
+  SelPrm sp = sel_prm(g);
+  uint32_t* w = static_cast<uint32_t*>(ws);
+  cudaError_t e = cudaMemsetAsync(w, 0, topk_passes_workspace_bytes(g), st);
+  if (e != cudaSuccess) return e;
+  for (int64_t u0 = 0; u0 < g.U; u0 += 65535) {
+    const unsigned nu = (unsigned)(g.U - u0 < 65535 ? g.U - u0 : 65535);
+    sp.t.unit0 = u0;
+    uint32_t* wu = w + u0 * sp.stride;
+    const dim3 gk((unsigned)sp.nbk, nu), gt((unsigned)sp.nbt, nu);
+    k_sel_hist<0><<<gk, kSelThreads, 0, st>>>(score, wu, sp);
+    k_sel_hist<1><<<gk, kSelThreads, 0, st>>>(score, wu, sp);
+    k_sel_hist<2><<<gk, kSelThreads, 0, st>>>(score, wu, sp);
+    k_sel_ties<<<gk, kSelThreads, 0, st>>>(score, wu, sp);
+    k_sel_resolve<<<nu, kSelThreads, 0, st>>>(score, wu, sp);
+    k_sel_count<<<gt, kSelThreads, 0, st>>>(score, wu, sp);
+    k_sel_write<<<gt, kSelThreads, 0, st>>>(score, wu, idx, pos, slot, sp);
+  }
+  return cudaGetLastError();
+}
+
+int topk_passes_launches(const Geom& g) { return 7 * (int)((g.U + 65534) / 65535); }
+
 }  // namespace lh

@@ -61,7 +61,7 @@ Layout saved_layout(const Geom& g) {
   return L;
 }
 
-enum FwdRegion { kPq = 0, kPk, kPv, kScore };
+enum FwdRegion { kPq = 0, kPk, kPv, kScore, kTopk };
 Layout fwd_ws_layout(const Geom& g) {
   Layout L;
   const size_t pyr = (size_t)g.U * (g.M - g.N) * g.d * 4;
@@ -69,6 +69,7 @@ Layout fwd_ws_layout(const Geom& g) {
   L.add(pyr);
   L.add(pyr);
   L.add((size_t)g.U * g.M * 4);
+  L.add(topk_passes_workspace_bytes(g));  // the selection's device-wide passes
   return L;
 }
 
@@ -156,6 +157,14 @@ bool use_pooled_gather(const Geom& g, lh_dtype dt) {
   return worst < levels;
 }
 
+// How lh_forward selects: device-wide passes (launch_topk_passes) for units of
+// more than 2^19 entries, where the cluster kernel needs 16-CTA clusters, of
+// which a B200 runs only 7 at once (a third wave at 16 units); one cluster per
+// unit below that, where its single launch beats the passes' seven.  Measured:
+// 524,288 tokens 423 -> 241 us, 1,048,576 tokens 521 -> 256 us; 98,304 tokens
+// 67 (cluster) vs 95 us (passes).
+bool use_topk_passes(const Geom& g) { return g.M > ((int64_t)1 << 19); }
+
 // The geometry of a shape with the variant options applied (options validated).
 Geom geom_with(const lh_shape& shape, const lh_options* opt) {
   Geom g = make_geom(shape);
@@ -230,8 +239,8 @@ size_t lh_workspace_bytes(const lh_shape* shape, lh_dtype dtype, int with_backwa
 }
 
 size_t lh_topk_workspace_bytes(const lh_shape* shape) {
-  (void)shape;
-  return 0;  // the selection keeps all its state in (distributed) shared memory
+  if (check_shape(shape) != LH_OK) return 0;
+  return topk_passes_workspace_bytes(make_geom(*shape));
 }
 
 size_t lh_attn_bwd_workspace_bytes(const lh_shape* shape) {
@@ -307,14 +316,17 @@ lh_status lh_score(const lh_shape* shape, lh_dtype dtype, const void* q, const v
 lh_status lh_topk_select_ex(const lh_shape* shape, const float* score, int32_t* idx,
                             int32_t* pos, int32_t* slot, void* ws, size_t ws_bytes,
                             const lh_options* opt, lh_stream_t stream) {
-  (void)ws;
-  (void)ws_bytes;
   lh_status s = check_shape(shape);
   if (s != LH_OK) return s;
   if ((s = lh_validate_options(shape, opt)) != LH_OK) return s;
-  if (!aligned16(score) || !aligned16(idx) || !aligned16(pos) || !aligned16(slot))
+  if (!aligned16(score) || !aligned16(idx) || !aligned16(pos) || !aligned16(slot) ||
+      (ws != nullptr && !aligned16(ws)))
     return LH_ERR_INVALID_ARG;
-  return cuda_status(launch_topk(geom_with(*shape, opt), score, idx, pos, slot, stream));
+  const Geom g = geom_with(*shape, opt);
+  if (ws == nullptr)  // no workspace: one thread-block cluster per unit
+    return cuda_status(launch_topk(g, score, idx, pos, slot, stream));
+  if (ws_bytes < topk_passes_workspace_bytes(g)) return LH_ERR_WORKSPACE;
+  return cuda_status(launch_topk_passes(g, score, idx, pos, slot, ws, stream));
 }
 
 lh_status lh_topk_select(const lh_shape* shape, const float* score, int32_t* idx, int32_t* pos,
@@ -463,16 +475,19 @@ lh_status lh_forward_ex(const lh_shape* shape, lh_dtype dtype, const void* q, co
   float* pk = g.L > 1 ? reinterpret_cast<float*>(w + wl.off[kPk]) : nullptr;
   float* pv = g.L > 1 ? reinterpret_cast<float*>(w + wl.off[kPv]) : nullptr;
   float* score = reinterpret_cast<float*>(w + wl.off[kScore]);
+  void* tws = w + wl.off[kTopk];
 
   if (use_pooled_gather(g, dtype)) {
     // scores only (no pyramid level written), then each selected coarse entry
     // pooled from its span of input rows: the same bits as the pyramid gather
     LH_TRY(launch_pyramid_score(g, dtype, q, k, nullptr, nullptr, nullptr, nullptr, score, stream));
-    LH_TRY(launch_topk(g, score, idx, pos, slot, stream));
+    LH_TRY(use_topk_passes(g) ? launch_topk_passes(g, score, idx, pos, slot, tws, stream)
+                              : launch_topk(g, score, idx, pos, slot, stream));
     LH_TRY(launch_gather_pooled(g, dtype, q, k, v, idx, qs, ks, vs, stream));
   } else {
     LH_TRY(launch_pyramid_score(g, dtype, q, k, v, pq, pk, pv, score, stream));
-    LH_TRY(launch_topk(g, score, idx, pos, slot, stream));
+    LH_TRY(use_topk_passes(g) ? launch_topk_passes(g, score, idx, pos, slot, tws, stream)
+                              : launch_topk(g, score, idx, pos, slot, stream));
     LH_TRY(launch_gather(g, dtype, q, k, v, pq, pk, pv, idx, qs, ks, vs, stream));
   }
   s = attn_fwd(g, qs, ks, vs, resolve_scale(g, scale), os, lse, stream);
@@ -536,6 +551,11 @@ lh_status lh_read_device_status(lh_stream_t stream, uint32_t* code) {
   return v ? LH_ERR_DEVICE_STATUS : LH_OK;
 }
 
+int lh_forward_topk_path(const lh_shape* shape) {
+  if (check_shape(shape) != LH_OK) return -1;
+  return use_topk_passes(make_geom(*shape)) ? 1 : 0;
+}
+
 int lh_forward_gather_path(const lh_shape* shape, lh_dtype dtype) {
   if (lh_validate(shape, dtype) != LH_OK) return -1;
   return use_pooled_gather(make_geom(*shape), dtype) ? 1 : 0;
@@ -558,7 +578,7 @@ int lh_kernel_launches(const lh_shape* shape, lh_dtype dtype, int backward) {
   const int chunks = (int)((g.U + 65534) / 65535);  // grid.y limit per launch
   if (!backward) {
     // pyramid+score, top-k (per chunk), gather, attention (per chunk), scatter (per chunk)
-    return pyramid_launches(g, dtype) + chunks + 1 +
+    return pyramid_launches(g, dtype) + (use_topk_passes(g) ? topk_passes_launches(g) : chunks) + 1 +
            (attn_fwd_uses_tc() ? attn_tc_fwd_launches(g) : chunks) + chunks;
   }
   // scatter-back bwd, softmax statistics, attention bwd, gather bwd (per chunk)

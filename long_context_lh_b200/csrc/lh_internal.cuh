@@ -247,6 +247,12 @@ cudaError_t launch_pyramid_score(const Geom& g, lh_dtype dt, const void* q, cons
 int pyramid_launches(const Geom& g, lh_dtype dt);  // kernel launches of one launch_pyramid_score
 cudaError_t launch_topk(const Geom& g, const float* score, int32_t* idx, int32_t* pos,
                         int32_t* slot, cudaStream_t st);
+// The same selection as device-wide passes over a workspace of
+// topk_passes_workspace_bytes(g) (zeroed here, on the stream).
+size_t topk_passes_workspace_bytes(const Geom& g);
+cudaError_t launch_topk_passes(const Geom& g, const float* score, int32_t* idx, int32_t* pos,
+                               int32_t* slot, void* ws, cudaStream_t st);
+int topk_passes_launches(const Geom& g);
 cudaError_t launch_gather(const Geom& g, lh_dtype dt, const void* q, const void* k, const void* v,
                           const float* pq, const float* pk, const float* pv, const int32_t* idx,
                           __half* qs, __half* ks, __half* vs, cudaStream_t st);

@@ -92,6 +92,7 @@ _SIGS = {
     "lh_build_pyramid_score": ([_SP, _I, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP], _I),
     "lh_score": ([_SP, _I, _VP, _VP, _VP, _VP], _I),
     "lh_topk_workspace_bytes": ([_SP], _SZ),
+    "lh_forward_topk_path": ([_SP], _I),
     "lh_topk_select": ([_SP, _VP, _VP, _VP, _VP, _VP, _SZ, _VP], _I),
     "lh_gather": ([_SP, _I, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP], _I),
     "lh_gather_pooled": ([_SP, _I, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP], _I),
@@ -201,6 +202,10 @@ def lh_saved_offset(shape: Shape, which: int) -> int:
 
 def lh_topk_workspace_bytes(shape: Shape) -> int:
     return int(_lib().lh_topk_workspace_bytes(ctypes.byref(shape)))
+
+
+def lh_forward_topk_path(shape: Shape) -> int:
+    return int(_lib().lh_forward_topk_path(ctypes.byref(shape)))
 
 
 def lh_attn_bwd_workspace_bytes(shape: Shape) -> int:

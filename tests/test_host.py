@@ -72,7 +72,7 @@ def test_num_entries_and_sizes():
     assert ws_f >= U * (3 * (M - 98304) * 64 * 4 + M * 4)
     assert ws_b >= ws_f and ws_b >= U * 8192 * (64 * 2 + 4 + 3 * 64 * 4)
     assert lh.lh_workspace_bytes(S(d=96), lh.LH_BF16, True) == 0
-    assert lh.lh_topk_workspace_bytes(shp) == 0
+    assert lh.lh_topk_workspace_bytes(shp) > 0  # the device-wide passes
     assert lh.lh_attn_bwd_workspace_bytes(shp) >= U * 8192 * 4
 
 
@@ -138,6 +138,15 @@ def test_options_are_checked_on_the_host():
                               None, None) == lh.LH_ERR_WORKSPACE
     assert lib.lh_scatter_back_ex(ctypes.byref(shp), lh.LH_BF16, p, p, p + 4, None, None,
                                   None) == lh.LH_ERR_INVALID_ARG
+
+
+def test_forward_topk_path_rule():
+    """lh_forward selects with one cluster per unit up to 2^19 entries per unit,
+    with device-wide passes above (the 512K and 1M workloads)."""
+    assert lh.lh_forward_topk_path(S(1, 16, 98304, 64, 4, 4, 8192)) == 0
+    assert lh.lh_forward_topk_path(S(1, 16, 524288, 64, 4, 5, 16384)) == 1
+    assert lh.lh_forward_topk_path(S(1, 8, 1048576, 128, 4, 6, 16384)) == 1
+    assert lh.lh_forward_topk_path(S(d=96)) == -1
 
 
 def test_forward_gather_path_rule():

@@ -102,6 +102,32 @@ STAGE_CASES = [
 ]
 
 
+def topk_both(shp, score, opt=None):
+    """Both selection implementations (a thread-block cluster per unit without a
+    workspace, device-wide passes with one) on the same scores: they must agree
+    bit for bit; returns idx, pos, slot."""
+    B, H, M = score.shape
+    S_ = shp.S
+    outs = []
+    for with_ws in (False, True):
+        idx = torch.full((B, H, S_), -7, dtype=torch.int32, device=DEV)
+        pos = torch.full_like(idx, -7)
+        slot = torch.full((B, H, M), -7, dtype=torch.int32, device=DEV)
+        ws, wsb = None, 0
+        if with_ws:
+            wsb = lh.lh_topk_workspace_bytes(shp)
+            ws = torch.full((wsb,), 0x5A, dtype=torch.uint8, device=DEV)  # garbage: zeroed by the call
+        if opt is None:
+            lh.lh_topk_select(shp, score, idx, pos, slot, ws, wsb)
+        else:
+            lh.lh_topk_select_ex(shp, score, idx, pos, slot, opt, ws, wsb)
+        outs.append((idx, pos, slot))
+    torch.cuda.synchronize()
+    for a, b in zip(*outs):
+        assert torch.equal(a, b), "cluster and pass selections differ"
+    return outs[1]
+
+
 def run_front(w, x):
     """GPU pyramid, score and selection for inputs x (device tensors)."""
     shp, dt = lshape(w), lh.dtype_code(x["q"].dtype)
@@ -112,11 +138,7 @@ def run_front(w, x):
     score = torch.zeros((w.B, w.H, M), dtype=torch.float32, device=DEV)
     lh.lh_build_pyramid(shp, dt, x["q"], x["k"], x["v"], *pyr)
     lh.lh_score(shp, dt, x["q"], x["k"], score)
-    idx = torch.full((w.B, w.H, w.S), -7, dtype=torch.int32, device=DEV)
-    pos = torch.full_like(idx, -7)
-    slot = torch.full((w.B, w.H, M), -7, dtype=torch.int32, device=DEV)
-    lh.lh_topk_select(shp, score, idx, pos, slot)
-    torch.cuda.synchronize()
+    idx, pos, slot = topk_both(shp, score)
     del U
     return pyr, score, idx, pos, slot
 
@@ -154,11 +176,7 @@ def test_topk_on_large_units_matches_oracle(case):
     M = lh.lh_num_entries(shp)
     score = torch.zeros((w.B, w.H, M), dtype=torch.float32, device=DEV)
     lh.lh_score(shp, dt, x["q"], x["k"], score)
-    idx = torch.full((w.B, w.H, w.S), -7, dtype=torch.int32, device=DEV)
-    pos = torch.full_like(idx, -7)
-    slot = torch.full((w.B, w.H, M), -7, dtype=torch.int32, device=DEV)
-    lh.lh_topk_select(shp, score, idx, pos, slot)
-    torch.cuda.synchronize()
+    idx, pos, slot = topk_both(shp, score)
     s = oshape(w)
     sc_ref = oracle.score(s, xc["q"].float().numpy(), xc["k"].float().numpy())
     assert np.array_equal(score.cpu().numpy(), sc_ref), "scores differ in some bit"
@@ -168,9 +186,12 @@ def test_topk_on_large_units_matches_oracle(case):
     assert np.array_equal(slot.cpu().numpy(), s_ref)
 
 
-def test_ties_beyond_inheritance_are_broken_by_gid():
-    """Quantised inputs make many equal scores; the radix select on gids must agree."""
-    w = workload(dtype="bf16", N=2048, S=300, H=3)
+@pytest.mark.parametrize("N,S,L", [(2048, 300, 3), (32768, 3000, 2)], ids=["list", "beyond-list"])
+def test_ties_beyond_inheritance_are_broken_by_gid(N, S, L):
+    """Quantised inputs make many equal scores; the radix select on gids must agree.
+    The second case has thousands of entries tied at the threshold, more than the
+    pass selection resolves from a list (it then runs radix passes over the gids)."""
+    w = workload(dtype="bf16", N=N, S=S, L=L, H=3)
     xc = make_inputs(w, "cpu", with_dO=False)
     for n in ("q", "k"):
         xc[n] = (xc[n].float() * 0).to(torch.bfloat16)
@@ -372,10 +393,7 @@ def test_variant_stages_match_oracle(case):
            for _ in range(3)]
     lh.lh_score_ex(shp, dt, x["q"], x["k"], score, opt)
     lh.lh_build_pyramid_score_ex(shp, dt, x["q"], x["k"], x["v"], *pyr, score2, opt)
-    idx = torch.full((w.B, w.H, w.S), -7, dtype=torch.int32, device=DEV)
-    pos = torch.full_like(idx, -7)
-    slot = torch.full((w.B, w.H, M), -7, dtype=torch.int32, device=DEV)
-    lh.lh_topk_select_ex(shp, score, idx, pos, slot, opt)
+    idx, pos, slot = topk_both(shp, score, opt)
     torch.cuda.synchronize()
     s = oshape(w)
     sc_ref = oracle.score(s, xc["q"].float().numpy(), xc["k"].float().numpy(), mode=case["score_mode"])
