@@ -767,14 +767,33 @@ __global__ void __launch_bounds__(kSelThreads) k_sel_hist(const float* __restric
   __syncthreads();
   const int32_t i0 = (int32_t)blockIdx.x * kSelKeys;
   const int32_t i1 = (int32_t)imin64(sp.t.M, (int64_t)i0 + kSelKeys);
-  for (int32_t j0 = i0 + (int32_t)(threadIdx.x & ~31u); j0 < i1; j0 += kSelThreads) {  // warp-uniform
-    const int32_t j = j0 + (int32_t)(threadIdx.x & 31);
-    const uint32_t kv = j < i1 ? sel_key(sp, key, j) : 0u;
-    const bool act = j < i1 && (kv & pmask) == prefix;
-    if (PASS == 0)
-      hist_add(h, act, (kv >> shift) & dmask);
-    else
-      hist_add_plain(h, act, (kv >> shift) & dmask);
+  // keys up to the first 16-byte boundary one by one, then four per load (all of
+  // a thread's loads in flight at once), then the tail
+  const int32_t head = (int32_t)((4 - ((u * sp.t.M + i0) & 3)) & 3);
+  const int32_t q0 = (int32_t)imin64(i1, (int64_t)i0 + head);
+  const int32_t nq = (i1 - q0) >> 2;
+  auto one = [&](int32_t j) {
+    const uint32_t kv = sel_key(sp, key, j);
+    if ((kv & pmask) == prefix) atomicAdd(&h[(kv >> shift) & dmask], 1u);
+  };
+  for (int32_t j = i0 + (int32_t)threadIdx.x; j < q0; j += kSelThreads) one(j);
+  for (int32_t j = q0 + 4 * nq + (int32_t)threadIdx.x; j < i1; j += kSelThreads) one(j);
+  const uint4* kq = reinterpret_cast<const uint4*>(key + q0);
+#pragma unroll 4
+  for (int32_t b0 = (int32_t)(threadIdx.x & ~31u); b0 < nq; b0 += kSelThreads) {  // warp-uniform
+    const int32_t qi = b0 + (int32_t)(threadIdx.x & 31);
+    const uint4 v4 = qi < nq ? __ldg(kq + qi) : make_uint4(0u, 0u, 0u, 0u);
+    const uint32_t kk[4] = {v4.x, v4.y, v4.z, v4.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int32_t g = q0 + 4 * qi + e;
+      const uint32_t kv = (sp.t.keep_top && g >= sp.top) ? kTopBits : kk[e];
+      const bool act = qi < nq && (kv & pmask) == prefix;
+      if (PASS == 0)
+        hist_add(h, act, (kv >> shift) & dmask);
+      else
+        hist_add_plain(h, act, (kv >> shift) & dmask);
+    }
   }
   __syncthreads();
   uint32_t* gh = w + kWsHist + PASS * kBins;
@@ -882,7 +901,17 @@ __device__ __forceinline__ bool sel_in(const SelPrm& sp, const uint32_t* key, in
   return kv > T || (kv == T && (uint32_t)g <= gthr);
 }
 
-// Selected entries per block of kSelTokens tokens (enumerated at their span's end).
+// Entries of level l whose span ends inside tokens [t0, t1): the level-l entry j
+// spans tokens [j p^l, (j+1) p^l) and is enumerated at its last token.
+__device__ __forceinline__ void level_range(const SelPrm& sp, int l, int32_t t0, int32_t t1,
+                                            int32_t& j0, int32_t& j1) {
+  const int32_t pw = sp.t.pw[l];
+  j0 = (t0 + pw) / pw - 1;  // ceil((t0 + 1) / pw) - 1
+  j1 = t1 / pw;
+}
+
+// Selected entries per block of kSelTokens tokens, level by level (every load
+// independent of the others, so many are in flight at once).
 __global__ void __launch_bounds__(kSelThreads) k_sel_count(const float* __restrict__ score,
                                                            uint32_t* __restrict__ ws, const SelPrm sp) {
   __shared__ uint32_t warp_buf[32], tot;
@@ -893,72 +922,103 @@ __global__ void __launch_bounds__(kSelThreads) k_sel_count(const float* __restri
   const int32_t t0 = (int32_t)blockIdx.x * kSelTokens;
   const int32_t t1 = (int32_t)imin64(sp.t.N, (int64_t)t0 + kSelTokens);
   uint32_t c = 0;
-  for (int32_t t = t0 + (int32_t)threadIdx.x; t < t1; t += kSelThreads) {
-    const uint32_t tt = (uint32_t)t + 1u;
 #pragma unroll
-    for (int l = 0; l < kMaxLevels; ++l) {
-      if (l >= sp.t.L || !ends_at(sp.t, tt, l)) break;
-      c += sel_in(sp, key, gid_at(sp.t, tt, l), T, gthr) ? 1u : 0u;
-    }
+  for (int l = 0; l < kMaxLevels; ++l) {
+    if (l >= sp.t.L) break;
+    int32_t j0, j1;
+    level_range(sp, l, t0, t1, j0, j1);
+    const int32_t gb = sp.t.off[l];
+#pragma unroll 4
+    for (int32_t j = j0 + (int32_t)threadIdx.x; j < j1; j += kSelThreads)
+      c += sel_in(sp, key, gb + j, T, gthr) ? 1u : 0u;
   }
   sel_excl_scan(c, warp_buf, &tot);
   if (threadIdx.x == 0) w[kWsCnt + blockIdx.x] = tot;
 }
 
-// idx, pos and the slot map: block b's entries take slots from the count of
-// blocks 0..b-1 on, in (token, level) order.
+// idx, pos and the slot map of a block of tokens: per token a mask of its
+// selected levels (level by level into shared memory), a block scan of the
+// per-token counts from the blocks before it on, then slots level by level:
+// entry (t, l) takes tok_off[t] + the selected levels of t below l.
 __global__ void __launch_bounds__(kSelThreads) k_sel_write(const float* __restrict__ score,
                                                            uint32_t* __restrict__ ws, int32_t* __restrict__ idx,
                                                            int32_t* __restrict__ pos, int32_t* __restrict__ slot,
                                                            const SelPrm sp) {
   __shared__ uint32_t warp_buf[32], tot;
+  __shared__ uint8_t mask[kSelTokens];
+  __shared__ uint32_t tok_off[kSelTokens];
+  constexpr int kPer = kSelTokens / kSelThreads;  // consecutive tokens per thread in the scan
   const int64_t u = sp.t.unit0 + blockIdx.y;
   const uint32_t* w = ws + (int64_t)blockIdx.y * sp.stride;
   const uint32_t* key = reinterpret_cast<const uint32_t*>(score + u * sp.t.M);
   const uint32_t T = __ldcg(w + kWsSt + kStT), gthr = __ldcg(w + kWsSt + kStGid);
-  uint32_t base;
-  {  // entries of the blocks before this one
-    uint32_t part = 0;
-    for (int i = threadIdx.x; i < (int)blockIdx.x; i += kSelThreads) part += __ldcg(w + kWsCnt + i);
-    sel_excl_scan(part, warp_buf, &tot);
-    base = tot;
+  const int32_t t0 = (int32_t)blockIdx.x * kSelTokens;
+  const int32_t t1 = (int32_t)imin64(sp.t.N, (int64_t)t0 + kSelTokens);
+  // slots before this block: the counts of blocks 0..b-1
+  uint32_t part = 0;
+  for (int i = threadIdx.x; i < (int)blockIdx.x; i += kSelThreads) part += __ldcg(w + kWsCnt + i);
+  sel_excl_scan(part, warp_buf, &tot);
+  const uint32_t base = tot;
+  // per-token masks, one level at a time (level l + 1 ORs into bytes level l wrote)
+#pragma unroll
+  for (int l = 0; l < kMaxLevels; ++l) {
+    if (l >= sp.t.L) break;
+    int32_t j0, j1;
+    level_range(sp, l, t0, t1, j0, j1);
+    const int32_t gb = sp.t.off[l], pw = sp.t.pw[l];
+#pragma unroll 4
+    for (int32_t j = j0 + (int32_t)threadIdx.x; j < j1; j += kSelThreads) {
+      const int32_t t = (j + 1) * pw - 1 - t0;
+      const uint8_t bit = sel_in(sp, key, gb + j, T, gthr) ? (uint8_t)(1u << l) : (uint8_t)0;
+      if (l == 0)
+        mask[t] = bit;
+      else
+        mask[t] |= bit;
+    }
+    __syncthreads();
   }
+  // token offsets: kPer consecutive tokens per thread, then a block scan
+  const int32_t nt = t1 - t0;
+  uint32_t loc[kPer], sum = 0;
+#pragma unroll
+  for (int i = 0; i < kPer; ++i) {
+    const int32_t t = (int32_t)threadIdx.x * kPer + i;
+    loc[i] = sum;
+    sum += t < nt ? (uint32_t)__popc(mask[t]) : 0u;
+  }
+  const uint32_t toff = base + sel_excl_scan(sum, warp_buf, &tot);
+#pragma unroll
+  for (int i = 0; i < kPer; ++i) {
+    const int32_t t = (int32_t)threadIdx.x * kPer + i;
+    if (t < nt) tok_off[t] = toff + loc[i];
+  }
+  __syncthreads();
   int32_t* idx_u = idx + u * sp.t.S;
   int32_t* pos_u = pos + u * sp.t.S;
   int32_t* slot_u = slot + u * sp.t.M;
-  const int32_t t0 = (int32_t)blockIdx.x * kSelTokens;
-  const int32_t t1 = (int32_t)imin64(sp.t.N, (int64_t)t0 + kSelTokens);
-  for (int32_t tb = t0; tb < t1; tb += kSelThreads) {  // block-uniform trip count
-    const int32_t t = tb + (int32_t)threadIdx.x;
-    const uint32_t tt = (uint32_t)t + 1u;
-    uint32_t mask = 0;
-    if (t < t1) {
 #pragma unroll
-      for (int l = 0; l < kMaxLevels; ++l) {
-        if (l >= sp.t.L || !ends_at(sp.t, tt, l)) break;
-        mask |= (sel_in(sp, key, gid_at(sp.t, tt, l), T, gthr) ? 1u : 0u) << l | 1u << (8 + l);
-      }
-    }
-    const uint32_t c = __popc(mask & 0xffu);
-    uint32_t k = base + sel_excl_scan(c, warp_buf, &tot);
-#pragma unroll
-    for (int l = 0; l < kMaxLevels; ++l) {
-      if (!((mask >> (8 + l)) & 1u)) break;
-      const int32_t g = gid_at(sp.t, tt, l);
-      if (!LH_CHECK(dbg::in_range(g, sp.t.M), kBoundsTopk)) break;
-      if ((mask >> l) & 1u) {
+  for (int l = 0; l < kMaxLevels; ++l) {
+    if (l >= sp.t.L) break;
+    int32_t j0, j1;
+    level_range(sp, l, t0, t1, j0, j1);
+    const int32_t gb = sp.t.off[l], pw = sp.t.pw[l];
+    for (int32_t j = j0 + (int32_t)threadIdx.x; j < j1; j += kSelThreads) {
+      const int32_t t = (j + 1) * pw - 1 - t0;
+      const uint32_t m = mask[t];
+      const int32_t g = gb + j;
+      if (!LH_CHECK(dbg::in_range(g, sp.t.M), kBoundsTopk)) continue;
+      if ((m >> l) & 1u) {
+        const uint32_t k = tok_off[t] + (uint32_t)__popc(m & ((1u << l) - 1u));
         // exactly S entries are selected, so k < S; the test is kept in every build
         if (LH_CHECK(dbg::in_range(k, sp.t.S), kBoundsTopk) && k < (uint32_t)sp.t.S) {
           idx_u[k] = g;
-          pos_u[k] = t;
+          pos_u[k] = t0 + t;
           slot_u[g] = (int32_t)k;
         }
-        ++k;
       } else {
         slot_u[g] = -1;
       }
     }
-    base += tot;
   }
 }
 

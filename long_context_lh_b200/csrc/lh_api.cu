@@ -161,8 +161,7 @@ bool use_pooled_gather(const Geom& g, lh_dtype dt) {
 // more than 2^19 entries, where the cluster kernel needs 16-CTA clusters, of
 // which a B200 runs only 7 at once (a third wave at 16 units); one cluster per
 // unit below that, where its single launch beats the passes' seven.  Measured:
-// 524,288 tokens 423 -> 241 us, 1,048,576 tokens 521 -> 256 us; 98,304 tokens
-// 67 (cluster) vs 95 us (passes).
+// 524,288 tokens 411 -> 171 us; 98,304 tokens 71 (cluster) vs 75 us (passes).
 bool use_topk_passes(const Geom& g) { return g.M > ((int64_t)1 << 19); }
 
 // The geometry of a shape with the variant options applied (options validated).
