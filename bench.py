@@ -48,14 +48,14 @@ PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # kernel that evicts them, so a stage that writes more than L2 holds reads low.
 MEASURED_TRAFFIC = {  # workload: {stage: (bytes per launch, sources, sha1[:16])}
     "pretrain": {
-        "pyramid_score": (9.6650e+08, ('k_pyramid.cu', 'lh_internal.cuh'), "ac25a7b7b8340a38"),
-        "topk": (8.4000e+06, ('k_topk.cu', 'lh_internal.cuh'), "95620aa77e463653"),
-        "gather": (9.9000e+07, ('k_gather_scatter.cu', 'lh_internal.cuh'), "17fe79fe62f5a233"),
-        "scatter": (1.7010e+08, ('k_gather_scatter.cu', 'lh_internal.cuh'), "17fe79fe62f5a233"),
-        "scatter_bwd": (2.2550e+08, ('k_gather_scatter.cu', 'lh_internal.cuh'), "17fe79fe62f5a233"),
-        "gather_bwd": (6.5820e+08, ('k_gather_scatter.cu', 'lh_internal.cuh'), "17fe79fe62f5a233"),
-        "attn_fwd": (5.0400e+07, ('k_attn_tc.cu', 'tc_common.cuh', 'lh_internal.cuh'), "202d9cf1e39f0aac"),
-        "attn_bwd": (1.9370e+08, ('k_attn_tc.cu', 'tc_common.cuh', 'k_gather_scatter.cu', 'lh_internal.cuh'), "7aab4813c8a3ea67"),
+        "pyramid_score": (9.6640e+08, ('k_pyramid.cu', 'lh_internal.cuh'), "3a592d4c26ded79a"),
+        "topk": (8.4000e+06, ('k_topk.cu', 'lh_internal.cuh'), "33182a3cc3170ec8"),
+        "gather": (9.8900e+07, ('k_gather_scatter.cu', 'lh_internal.cuh'), "561cc6c760bc762a"),
+        "scatter": (1.7000e+08, ('k_gather_scatter.cu', 'lh_internal.cuh'), "561cc6c760bc762a"),
+        "scatter_bwd": (2.2590e+08, ('k_gather_scatter.cu', 'lh_internal.cuh'), "561cc6c760bc762a"),
+        "gather_bwd": (6.5820e+08, ('k_gather_scatter.cu', 'lh_internal.cuh'), "561cc6c760bc762a"),
+        "attn_fwd": (5.0400e+07, ('k_attn_tc.cu', 'tc_common.cuh', 'lh_internal.cuh'), "fddb1b46e4c21830"),
+        "attn_bwd": (1.9430e+08, ('k_attn_tc.cu', 'tc_common.cuh', 'k_gather_scatter.cu', 'lh_internal.cuh'), "a482e947f0cf6f7c"),
     },
 }
 
@@ -478,6 +478,52 @@ def block_leg(w, args, dev, steps=5, warmup=3):
     return out
 
 
+def run_topk_compare(args, rk):
+    """Both top-K implementations (one cluster per unit, device-wide passes) on the
+    same scores at the pretraining and 512K-token shapes: CUDA-event medians and
+    whether the selections are equal bit for bit; one JSON line."""
+    from long_context_lh_b200 import lighthouse as lh
+    from long_context_lh_b200.synth import WORKLOADS, make_inputs
+    dev = torch.device("cuda", rk.local_rank)
+    torch.cuda.set_device(dev)
+    points = []
+    for name in ("pretrain", "long"):
+        w = WORKLOADS[name]
+        x = make_inputs(w, dev, with_dO=False)
+        shp = lh.make_shape(w.B, w.H, w.N, w.d, w.p, w.L, w.S)
+        U, M = w.B * w.H, lh.lh_num_entries(shp)
+        score = torch.empty(U * M, dtype=torch.float32, device=dev)
+        lh.lh_score(shp, lh.dtype_code(x["q"].dtype), x["q"], x["k"], score)
+        res, outs = {}, {}
+        for impl in ("cluster", "passes"):
+            idx = torch.empty(U * w.S, dtype=torch.int32, device=dev)
+            pos = torch.empty_like(idx)
+            slot = torch.empty(U * M, dtype=torch.int32, device=dev)
+            wsb = lh.lh_topk_workspace_bytes(shp) if impl == "passes" else 0
+            ws = torch.empty(wsb, dtype=torch.uint8, device=dev) if wsb else None
+            run = lambda: lh.lh_topk_select(shp, score, idx, pos, slot, ws, wsb)  # noqa: E731
+            for _ in range(args.warmup):
+                run()
+            ts = []
+            for _ in range(max(args.steps, 5)):
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record()
+                run()
+                e1.record()
+                torch.cuda.synchronize()
+                ts.append(e0.elapsed_time(e1))
+            res[impl] = statistics.median(ts) * 1e3
+            outs[impl] = (idx, pos, slot)
+        equal = all(torch.equal(a, b) for a, b in zip(outs["cluster"], outs["passes"]))
+        points.append({"workload": name, "entries_per_unit": M, "us_cluster": res["cluster"],
+                       "us_passes": res["passes"], "equal": equal,
+                       "lh_forward_uses": ["cluster", "passes"][lh.lh_forward_topk_path(shp)]})
+        del x, score
+        torch.cuda.empty_cache()
+    if rk.rank == 0:
+        print(json.dumps({"topk_compare": points, "device_status": lh.lh_read_device_status()}))
+
+
 def run_sweep(args, rk):
     """Forward-only per-stage times over the hyperparameter sweep (p, L, S) at the
     pretraining shape; one JSON line."""
@@ -767,6 +813,8 @@ def main():
                     help="1: also time a training step of the attention block (1 GPU)")
     ap.add_argument("--sweep", action="store_true",
                     help="forward-only per-stage times over the p x L x S sweep (one JSON line)")
+    ap.add_argument("--topk-compare", action="store_true",
+                    help="both top-K implementations at the pretraining and 512K shapes (one JSON line)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3) if args.impl == "ours" else args.warmup
     rk = replicas.from_env()
@@ -779,6 +827,8 @@ def main():
     try:
         if args.sweep:
             run_sweep(args, rk)
+        elif args.topk_compare:
+            run_topk_compare(args, rk)
         else:
             run_ours(args, rk)
     finally:
