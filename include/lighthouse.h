@@ -242,8 +242,8 @@ int lh_forward_gather_path(const lh_shape* shape, lh_dtype dtype);
 
 /* How lh_forward runs the selection for this shape: 0 one thread-block cluster
  * per unit (lh_topk_select without a workspace), 1 device-wide passes (with
- * one: units of more than 2^19 entries); -1 for an invalid shape.  Both give
- * the same bits.  Host-only. */
+ * one; every valid shape at present); -1 for an invalid shape.  Both give the
+ * same bits.  Host-only. */
 int lh_forward_topk_path(const lh_shape* shape);
 
 /* Whole backward with the saved selection: (f'), (e'), (d').  dO: [B,H,N,d]

@@ -675,6 +675,14 @@ struct SelPrm {
   int32_t top;     // first gid of the coarsest level (ranked +inf when kept)
 };
 
+// Programmatic dependent launch: each pass is launched while the one before it
+// drains; it waits here until that pass has completed (its writes visible), then
+// lets the next pass be launched.  Both are no-ops for an ordinary launch.
+__device__ __forceinline__ void pdl_wait_then_release() {
+  asm volatile("griddepcontrol.wait;\n" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
+}
+
 __device__ __forceinline__ uint32_t sel_key(const SelPrm& sp, const uint32_t* key, int32_t g) {
   return (sp.t.keep_top && g >= sp.top) ? kTopBits : __ldg(key + g);
 }
@@ -731,6 +739,7 @@ __device__ Pick sel_pick(const uint32_t* hist, int nb, bool descending, uint32_t
 template <int PASS>
 __global__ void __launch_bounds__(kSelThreads) k_sel_hist(const float* __restrict__ score,
                                                           uint32_t* __restrict__ ws, const SelPrm sp) {
+  pdl_wait_then_release();
   __shared__ uint32_t h[kBins];
   __shared__ uint32_t warp_buf[32], sh[4];
   const int64_t u = sp.t.unit0 + blockIdx.y;
@@ -806,6 +815,7 @@ __global__ void __launch_bounds__(kSelThreads) k_sel_hist(const float* __restric
 // fit, every CTA lists the gids of its keys equal to T (up to kSelTies).
 __global__ void __launch_bounds__(kSelThreads) k_sel_ties(const float* __restrict__ score,
                                                           uint32_t* __restrict__ ws, const SelPrm sp) {
+  pdl_wait_then_release();
   __shared__ uint32_t warp_buf[32], sh[4];
   const int64_t u = sp.t.unit0 + blockIdx.y;
   uint32_t* w = ws + (int64_t)blockIdx.y * sp.stride;
@@ -837,6 +847,7 @@ __global__ void __launch_bounds__(kSelThreads) k_sel_ties(const float* __restric
 // than kSelTies entries share the threshold score).
 __global__ void __launch_bounds__(kSelThreads) k_sel_resolve(const float* __restrict__ score,
                                                              uint32_t* __restrict__ ws, const SelPrm sp) {
+  pdl_wait_then_release();
   __shared__ uint32_t h[kBins];
   __shared__ uint32_t warp_buf[32], sh[4];
   __shared__ uint32_t list[kSelTies];
@@ -914,6 +925,7 @@ __device__ __forceinline__ void level_range(const SelPrm& sp, int l, int32_t t0,
 // independent of the others, so many are in flight at once).
 __global__ void __launch_bounds__(kSelThreads) k_sel_count(const float* __restrict__ score,
                                                            uint32_t* __restrict__ ws, const SelPrm sp) {
+  pdl_wait_then_release();
   __shared__ uint32_t warp_buf[32], tot;
   const int64_t u = sp.t.unit0 + blockIdx.y;
   uint32_t* w = ws + (int64_t)blockIdx.y * sp.stride;
@@ -944,6 +956,7 @@ __global__ void __launch_bounds__(kSelThreads) k_sel_write(const float* __restri
                                                            uint32_t* __restrict__ ws, int32_t* __restrict__ idx,
                                                            int32_t* __restrict__ pos, int32_t* __restrict__ slot,
                                                            const SelPrm sp) {
+  pdl_wait_then_release();
   __shared__ uint32_t warp_buf[32], tot;
   __shared__ uint8_t mask[kSelTokens];
   __shared__ uint32_t tok_off[kSelTokens];
@@ -1061,13 +1074,26 @@ cudaError_t launch_topk_passes(const Geom& g, const float* score, int32_t* idx, 
     sp.t.unit0 = u0;
     uint32_t* wu = w + u0 * sp.stride;
     const dim3 gk((unsigned)sp.nbk, nu), gt((unsigned)sp.nbt, nu);
-    k_sel_hist<0><<<gk, kSelThreads, 0, st>>>(score, wu, sp);
-    k_sel_hist<1><<<gk, kSelThreads, 0, st>>>(score, wu, sp);
-    k_sel_hist<2><<<gk, kSelThreads, 0, st>>>(score, wu, sp);
-    k_sel_ties<<<gk, kSelThreads, 0, st>>>(score, wu, sp);
-    k_sel_resolve<<<nu, kSelThreads, 0, st>>>(score, wu, sp);
-    k_sel_count<<<gt, kSelThreads, 0, st>>>(score, wu, sp);
-    k_sel_write<<<gt, kSelThreads, 0, st>>>(score, wu, idx, pos, slot, sp);
+    k_sel_hist<0><<<gk, kSelThreads, 0, st>>>(score, wu, sp);  // after the memset: ordinary launch
+    // the later passes: programmatic dependent launches (see pdl_wait_then_release)
+    auto pdl = [&](dim3 grid, auto kern, auto... a) -> cudaError_t {
+      cudaLaunchConfig_t cfg = {};
+      cfg.gridDim = grid;
+      cfg.blockDim = dim3(kSelThreads, 1, 1);
+      cfg.stream = st;
+      cudaLaunchAttribute attr[1];
+      attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+      attr[0].val.programmaticStreamSerializationAllowed = 1;
+      cfg.attrs = attr;
+      cfg.numAttrs = 1;
+      return cudaLaunchKernelEx(&cfg, kern, a...);
+    };
+    if ((e = pdl(gk, k_sel_hist<1>, score, wu, sp)) != cudaSuccess) return e;
+    if ((e = pdl(gk, k_sel_hist<2>, score, wu, sp)) != cudaSuccess) return e;
+    if ((e = pdl(gk, k_sel_ties, score, wu, sp)) != cudaSuccess) return e;
+    if ((e = pdl(dim3(nu, 1, 1), k_sel_resolve, score, wu, sp)) != cudaSuccess) return e;
+    if ((e = pdl(gt, k_sel_count, score, wu, sp)) != cudaSuccess) return e;
+    if ((e = pdl(gt, k_sel_write, score, wu, idx, pos, slot, sp)) != cudaSuccess) return e;
   }
   return cudaGetLastError();
 }

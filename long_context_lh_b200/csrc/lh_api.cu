@@ -157,12 +157,14 @@ bool use_pooled_gather(const Geom& g, lh_dtype dt) {
   return worst < levels;
 }
 
-// How lh_forward selects: device-wide passes (launch_topk_passes) for units of
-// more than 2^19 entries, where the cluster kernel needs 16-CTA clusters, of
-// which a B200 runs only 7 at once (a third wave at 16 units); one cluster per
-// unit below that, where its single launch beats the passes' seven.  Measured:
-// 524,288 tokens 411 -> 171 us; 98,304 tokens 71 (cluster) vs 75 us (passes).
-bool use_topk_passes(const Geom& g) { return g.M > ((int64_t)1 << 19); }
+// How lh_forward selects: device-wide passes (launch_topk_passes, its later
+// passes dependent launches).  Measured against one cluster per unit (launch_topk):
+// 98,304 tokens 69 -> 62 us, 524,288 tokens 410 -> 160 us, where the cluster
+// kernel needs 16-CTA clusters, of which a B200 runs only 7 at once.
+bool use_topk_passes(const Geom& g) {
+  (void)g;
+  return true;
+}
 
 // The geometry of a shape with the variant options applied (options validated).
 Geom geom_with(const lh_shape& shape, const lh_options* opt) {

@@ -141,9 +141,9 @@ def test_options_are_checked_on_the_host():
 
 
 def test_forward_topk_path_rule():
-    """lh_forward selects with one cluster per unit up to 2^19 entries per unit,
-    with device-wide passes above (the 512K and 1M workloads)."""
-    assert lh.lh_forward_topk_path(S(1, 16, 98304, 64, 4, 4, 8192)) == 0
+    """lh_forward selects with the device-wide passes (faster than one cluster per
+    unit at every benchmark shape once the passes are dependent launches)."""
+    assert lh.lh_forward_topk_path(S(1, 16, 98304, 64, 4, 4, 8192)) == 1
     assert lh.lh_forward_topk_path(S(1, 16, 524288, 64, 4, 5, 16384)) == 1
     assert lh.lh_forward_topk_path(S(1, 8, 1048576, 128, 4, 6, 16384)) == 1
     assert lh.lh_forward_topk_path(S(d=96)) == -1
