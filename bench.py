@@ -49,7 +49,7 @@ PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 MEASURED_TRAFFIC = {  # workload: {stage: (bytes per launch, sources, sha1[:16])}
     "pretrain": {
         "pyramid_score": (9.6640e+08, ('k_pyramid.cu', 'lh_internal.cuh'), "3a592d4c26ded79a"),
-        "topk": (8.4000e+06, ('k_topk.cu', 'lh_internal.cuh'), "33182a3cc3170ec8"),
+        "topk": (4.7600e+07, ('k_topk.cu', 'lh_internal.cuh'), "d537cf8c45dc9c26"),
         "gather": (9.8900e+07, ('k_gather_scatter.cu', 'lh_internal.cuh'), "561cc6c760bc762a"),
         "scatter": (1.7000e+08, ('k_gather_scatter.cu', 'lh_internal.cuh'), "561cc6c760bc762a"),
         "scatter_bwd": (2.2590e+08, ('k_gather_scatter.cu', 'lh_internal.cuh'), "561cc6c760bc762a"),
