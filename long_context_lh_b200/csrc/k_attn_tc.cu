@@ -49,6 +49,16 @@ constexpr float kLog2e = 1.4426950408889634f;
 constexpr int kThreads = 352;  // 8 row-work warps, TMA warp 8, MMA warps 9 and 10
 constexpr uint32_t kTmemCols = 512;
 
+// The dQ kernel reads nothing the dK/dV kernel writes, so it is launched as a
+// programmatic dependent of it: the dK/dV kernel releases it once all its CTAs
+// run (pdl_release), and dQ CTAs fill the SMs its last wave frees.  Each dQ CTA
+// waits, before it exits, for the dK/dV kernel to have completed (pdl_join), so
+// that whatever follows the dQ kernel in the stream sees both kernels' results.
+__device__ __forceinline__ void pdl_release() {
+  asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
+}
+__device__ __forceinline__ void pdl_join() { asm volatile("griddepcontrol.wait;\n" ::: "memory"); }
+
 __device__ __forceinline__ void store_row_half(uint8_t* tile_half, int r, const uint32_t (&pk)[32]) {
   // one 64-column half of a row of a 128-byte-swizzled fp16 tile: 8 chunks of 16 B
 #pragma unroll
@@ -520,6 +530,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                        const float* __restrict__ stats, float* __restrict__ dks,
                        float* __restrict__ dvs, int S, int unit0,
                        int nunits, float scale, float scale_log2, int ntiles, int full) {
+  pdl_release();
   using Lt = DkvLayout<D>;
   constexpr int STG = Lt::kStages;
   static_assert(STG >= 1 && STG <= 4, "DkvBars holds at most 4 stages");
@@ -822,6 +833,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   extern __shared__ __align__(1024) uint8_t smem[];
   if (smem_u32(smem) & 1023u) {
     if (threadIdx.x == 0) report_status(kStatusAttnBwdTimeout | 2u);
+    pdl_join();
     return;
   }
   DqBars* bars = reinterpret_cast<DqBars*>(smem + Lt::kBar);
@@ -836,7 +848,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int qt = ntiles - 1 - (int)(blockIdx.x / nunits);  // most key tiles first
   const int u = unit0 + (int)(blockIdx.x % nunits);
   const int n = full ? ntiles : qt + 1;  // key tiles: up to the diagonal, or all of the block
-  if (!LH_CHECK(qt >= 0 && (int64_t)qt * 128 < S, kBoundsAttnBwd)) return;  // whole CTA
+  if (!LH_CHECK(qt >= 0 && (int64_t)qt * 128 < S, kBoundsAttnBwd)) {  // whole CTA
+    pdl_join();
+    return;
+  }
 
   if (threadIdx.x == 0) {
     mbar_init(&bars->q_full, 1);
@@ -1027,6 +1042,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);
   }
+  pdl_join();
 }
 
 // ------------------------------------------------------------------ host side
@@ -1105,9 +1121,20 @@ cudaError_t bwd_d(const Geom& g, const __half* qs, const __half* ks, const __hal
     k_attn_bwd_dkdv_tc<D><<<(unsigned)(nu * ntiles), kThreads, smem_a, st>>>(
         mq, mk, mv, mdo, stats, dks, dvs, (int)g.S, (int)u0, (int)nu, scale, scale * kLog2e,
         ntiles, full);
-    k_attn_bwd_dq_tc<D><<<(unsigned)(nu * ntiles), kThreads, smem_b, st>>>(
-        mq, mk, mv, mdo, stats, dqs, (int)g.S, (int)u0, (int)nu, scale, scale * kLog2e, ntiles,
-        full);
+    // a programmatic dependent of the dK/dV kernel (see pdl_release / pdl_join)
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(nu * ntiles), 1, 1);
+    cfg.blockDim = dim3(kThreads, 1, 1);
+    cfg.dynamicSmemBytes = smem_b;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, k_attn_bwd_dq_tc<D>, mq, mk, mv, mdo, stats, dqs, (int)g.S, (int)u0,
+                           (int)nu, scale, scale * kLog2e, ntiles, full);
+    if (e != cudaSuccess) return e;
   }
   return cudaGetLastError();
 }
