@@ -110,6 +110,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                   const __grid_constant__ CUtensorMap tv, __half* __restrict__ os,
                   float* __restrict__ lse, int S, int unit0, int nunits, float scale_log2,
                   int ntiles, int full) {
+  pdl_enter();
   using Lt = FwdLayout<D>;
   constexpr int KS = Lt::kKS;
   static_assert(KS >= 1 && KS <= 4, "FwdBars holds at most 4 stages");
@@ -530,7 +531,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                        const float* __restrict__ stats, float* __restrict__ dks,
                        float* __restrict__ dvs, int S, int unit0,
                        int nunits, float scale, float scale_log2, int ntiles, int full) {
-  pdl_release();
+  pdl_enter();
   using Lt = DkvLayout<D>;
   constexpr int STG = Lt::kStages;
   static_assert(STG >= 1 && STG <= 4, "DkvBars holds at most 4 stages");
@@ -1094,7 +1095,7 @@ cudaError_t fwd_d(const Geom& g, const __half* qs, const __half* ks, const __hal
   const int64_t per = 0x7fffffff / npairs;  // units per launch (grid.x limit)
   for (int64_t u0 = 0; u0 < g.U; u0 += per) {
     const int64_t nu = g.U - u0 < per ? g.U - u0 : per;
-    k_attn_fwd_tc<D><<<(unsigned)(nu * npairs), kThreads, smem, st>>>(
+    (void)launch_pdl(k_attn_fwd_tc<D>, (unsigned)(nu * npairs), kThreads, smem, st, 
         mq, mk, mv, os, lse, (int)g.S, (int)u0, (int)nu, scale * kLog2e, ntiles, full);
   }
   return cudaGetLastError();
@@ -1118,7 +1119,7 @@ cudaError_t bwd_d(const Geom& g, const __half* qs, const __half* ks, const __hal
   const int64_t per = 0x7fffffff / ntiles;
   for (int64_t u0 = 0; u0 < g.U; u0 += per) {
     const int64_t nu = g.U - u0 < per ? g.U - u0 : per;
-    k_attn_bwd_dkdv_tc<D><<<(unsigned)(nu * ntiles), kThreads, smem_a, st>>>(
+    (void)launch_pdl(k_attn_bwd_dkdv_tc<D>, (unsigned)(nu * ntiles), kThreads, smem_a, st, 
         mq, mk, mv, mdo, stats, dks, dvs, (int)g.S, (int)u0, (int)nu, scale, scale * kLog2e,
         ntiles, full);
     // a programmatic dependent of the dK/dV kernel (see pdl_release / pdl_join)

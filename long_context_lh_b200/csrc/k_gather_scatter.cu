@@ -91,6 +91,7 @@ __global__ void __launch_bounds__(256) k_gather(
     const float* __restrict__ pq, const float* __restrict__ pk, const float* __restrict__ pv,
     const int32_t* __restrict__ idx, __half* __restrict__ qs, __half* __restrict__ ks,
     __half* __restrict__ vs, const Lv lv, int64_t rows) {
+  pdl_enter();
   constexpr int G = D / 8;
   const int64_t gt = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   const int64_t row = gt / G;  // u * S + slot
@@ -182,6 +183,7 @@ __global__ void __launch_bounds__(256) k_gather_pooled(
     const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin* __restrict__ v,
     const int32_t* __restrict__ idx, __half* __restrict__ qs, __half* __restrict__ ks,
     __half* __restrict__ vs, const Lv lv, int64_t rows) {
+  pdl_enter();
   constexpr int G = D / 8;
   const int64_t gt = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   const int64_t row = gt / G;  // u * S + slot
@@ -233,6 +235,7 @@ __global__ void __launch_bounds__(256) k_scatter(const __half* __restrict__ os,
                                                  const int32_t* __restrict__ slot,
                                                  Tout* __restrict__ o, float* __restrict__ inv_count,
                                                  const Lv lv, int64_t u0) {
+  pdl_enter();
   constexpr int G = D / 8, kGroups = 256 / G;
   constexpr int LC = (L > 1) ? L - 1 : 1;  // coarse levels (array size)
   const int32_t t0 = ((int32_t)blockIdx.x * kGroups + (int32_t)(threadIdx.x / G)) * R;
@@ -329,6 +332,7 @@ __global__ void __launch_bounds__(128) k_scatter_pp(const __half* __restrict__ o
                                                     const int32_t* __restrict__ slot,
                                                     Tout* __restrict__ o, float* __restrict__ inv_count,
                                                     const Lv lv, int64_t u0) {
+  pdl_enter();
   static_assert(L >= 2 && (P == 2 || P == 4), "specialised on p in {2, 4}, L >= 2");
   constexpr int G = D / 8, kGroups = 128 / G, NE = kScatterEntries;
   constexpr int NU = (L > 2) ? L - 2 : 1;  // levels >= 2: one entry each
@@ -451,6 +455,7 @@ __global__ void __launch_bounds__(256) k_scatter_bwd(const Tin* __restrict__ dO,
                                                      const float* __restrict__ inv_count,
                                                      __half* __restrict__ dos, const Lv lv,
                                                      int64_t spans, int64_t groups) {
+  pdl_enter();
   constexpr int G = D / 8;
   constexpr int NL = (L > 1) ? (L - 1) : 1;
   constexpr int RB = 4;  // rows of dO whose loads are in flight together
@@ -610,6 +615,7 @@ __global__ void __launch_bounds__(kScatterBwdThreads) k_scatter_bwd_pp(
     const Tin* __restrict__ dO, const int32_t* __restrict__ slot,
     const float* __restrict__ inv_count, __half* __restrict__ dos, const Lv lv, int32_t spans,
     int64_t u0) {
+  pdl_enter();
   using C = ScatterBwdCfg<Tin, D, L, P, RG>;
   constexpr int G = C::G, LW = C::LW, Ptop = C::Ptop, CPR = C::CPR, RB = C::RB, NB = C::NB;
   constexpr int NCS = C::NCS, NA = LW > 0 ? LW : 1, NT = kScatterBwdThreads;
@@ -767,6 +773,7 @@ __global__ void __launch_bounds__(256) k_scatter_last(const __half* __restrict__
                                                       const int32_t* __restrict__ slot,
                                                       Tout* __restrict__ o, float* __restrict__ inv_count,
                                                       const Lv lv, int64_t u0) {
+  pdl_enter();
   constexpr int G = D / 8, kGroups = 256 / G;
   const int32_t t = (int32_t)blockIdx.x * kGroups + (int32_t)(threadIdx.x / G);
   if (t >= lv.N) return;
@@ -805,6 +812,7 @@ __global__ void __launch_bounds__(256) k_scatter_bwd_last(const Tin* __restrict_
                                                           const float* __restrict__ inv_count,
                                                           __half* __restrict__ dos, const Lv lv,
                                                           int64_t u0) {
+  pdl_enter();
   constexpr int G = D / 8, kGroups = 256 / G;
   const int32_t t = (int32_t)blockIdx.x * kGroups + (int32_t)(threadIdx.x / G);
   if (t >= lv.N) return;
@@ -841,6 +849,7 @@ __global__ void __launch_bounds__(256) k_gather_bwd(
     const float* __restrict__ dqs, const float* __restrict__ dks, const float* __restrict__ dvs,
     const int32_t* __restrict__ slot, Tout* __restrict__ dq, Tout* __restrict__ dk,
     Tout* __restrict__ dv, const Lv lv, int64_t u0) {
+  pdl_enter();
   constexpr int G = D / 8, kGroups = 256 / G;
   constexpr int LC = (L > 1) ? L - 1 : 1;
   const int32_t t0 = ((int32_t)blockIdx.x * kGroups + (int32_t)(threadIdx.x / G)) * R;
@@ -899,6 +908,7 @@ __global__ void __launch_bounds__(128) k_gather_bwd_pp(
     const float* __restrict__ dqs, const float* __restrict__ dks, const float* __restrict__ dvs,
     const int32_t* __restrict__ slot, Tout* __restrict__ dq, Tout* __restrict__ dk,
     Tout* __restrict__ dv, const Lv lv, int64_t u0) {
+  pdl_enter();
   static_assert(L >= 2 && (P == 2 || P == 4), "specialised on p in {2, 4}, L >= 2");
   constexpr int G = D / 8, kGroups = 128 / G, NE = kGatherEntries;
   constexpr int NU = (L > 2) ? L - 2 : 1;  // levels >= 2: one entry each
@@ -1008,6 +1018,7 @@ __global__ void __launch_bounds__(256) k_attn_stats(const __half* __restrict__ o
                                                     const float* __restrict__ lse,
                                                     float* __restrict__ stats, int S, int T,
                                                     int64_t prows) {
+  pdl_enter();
   constexpr int G = D / 8;  // threads per row, 8 columns each
   const int64_t gt = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   const int64_t prow = gt / G;  // padded row over all units
@@ -1053,17 +1064,17 @@ cudaError_t launch_gather(const Geom& g, lh_dtype dt, const void* q, const void*
     auto* b = static_cast<const __nv_bfloat16*>(k);
     auto* c = static_cast<const __nv_bfloat16*>(v);
     if (g.d == 64)
-      k_gather<__nv_bfloat16, 64><<<nb, 256, 0, st>>>(a, b, c, pq, pk, pv, idx, qs, ks, vs, lv, rows);
+      (void)launch_pdl(k_gather<__nv_bfloat16, 64>, nb, 256, 0, st, a, b, c, pq, pk, pv, idx, qs, ks, vs, lv, rows);
     else
-      k_gather<__nv_bfloat16, 128><<<nb, 256, 0, st>>>(a, b, c, pq, pk, pv, idx, qs, ks, vs, lv, rows);
+      (void)launch_pdl(k_gather<__nv_bfloat16, 128>, nb, 256, 0, st, a, b, c, pq, pk, pv, idx, qs, ks, vs, lv, rows);
   } else {
     auto* a = static_cast<const float*>(q);
     auto* b = static_cast<const float*>(k);
     auto* c = static_cast<const float*>(v);
     if (g.d == 64)
-      k_gather<float, 64><<<nb, 256, 0, st>>>(a, b, c, pq, pk, pv, idx, qs, ks, vs, lv, rows);
+      (void)launch_pdl(k_gather<float, 64>, nb, 256, 0, st, a, b, c, pq, pk, pv, idx, qs, ks, vs, lv, rows);
     else
-      k_gather<float, 128><<<nb, 256, 0, st>>>(a, b, c, pq, pk, pv, idx, qs, ks, vs, lv, rows);
+      (void)launch_pdl(k_gather<float, 128>, nb, 256, 0, st, a, b, c, pq, pk, pv, idx, qs, ks, vs, lv, rows);
   }
   return cudaGetLastError();
 }
@@ -1079,7 +1090,7 @@ cudaError_t gather_pooled_d(const Geom& g, const Tin* q, const Tin* k, const Tin
   switch (g.L) {
 #define LH_CASE(LL)                                                                              \
   case LL:                                                                                       \
-    k_gather_pooled<Tin, D, LL><<<nb, 256, 0, st>>>(q, k, v, idx, qs, ks, vs, lv, rows);        \
+    (void)launch_pdl(k_gather_pooled<Tin, D, LL>, nb, 256, 0, st, q, k, v, idx, qs, ks, vs, lv, rows);        \
     break;
     LH_CASE(1) LH_CASE(2) LH_CASE(3) LH_CASE(4) LH_CASE(5) LH_CASE(6) LH_CASE(7) LH_CASE(8)
 #undef LH_CASE
@@ -1152,7 +1163,7 @@ cudaError_t scatter_t(const Geom& g, const __half* os, const int32_t* slot, Tout
   if (g.scatter_mode == LH_SCATTER_LAST) {
     const unsigned bxl = blocks_for(g.N, 256 / (D / 8));
     per_unit_chunks(g.U, [&](int64_t u0, unsigned nu) {
-      k_scatter_last<Tout, D><<<dim3(bxl, nu), 256, 0, st>>>(os, slot, o, inv_count, lv, u0);
+      (void)launch_pdl(k_scatter_last<Tout, D>, dim3(bxl, nu), 256, 0, st, os, slot, o, inv_count, lv, u0);
     });
     return cudaGetLastError();
   }
@@ -1163,9 +1174,9 @@ cudaError_t scatter_t(const Geom& g, const __half* os, const int32_t* slot, Tout
       if constexpr (LL >= 2) {
         per_unit_chunks(g.U, [&](int64_t u0, unsigned nu) {
           if (g.p == 4)
-            k_scatter_pp<Tout, D, LL, 4><<<dim3(bxp, nu), 128, 0, st>>>(os, slot, o, inv_count, lv, u0);
+            (void)launch_pdl(k_scatter_pp<Tout, D, LL, 4>, dim3(bxp, nu), 128, 0, st, os, slot, o, inv_count, lv, u0);
           else
-            k_scatter_pp<Tout, D, LL, 2><<<dim3(bxp, nu), 128, 0, st>>>(os, slot, o, inv_count, lv, u0);
+            (void)launch_pdl(k_scatter_pp<Tout, D, LL, 2>, dim3(bxp, nu), 128, 0, st, os, slot, o, inv_count, lv, u0);
         });
       }
     });
@@ -1175,8 +1186,7 @@ cudaError_t scatter_t(const Geom& g, const __half* os, const int32_t* slot, Tout
   return with_tokens(R, [&](auto rc) {
     return with_levels(g.L, [&](auto lc) {
       per_unit_chunks(g.U, [&](int64_t u0, unsigned nu) {
-        k_scatter<Tout, D, decltype(lc)::value, decltype(rc)::value>
-            <<<dim3(bx, nu), 256, 0, st>>>(os, slot, o, inv_count, lv, u0);
+        (void)launch_pdl(k_scatter<Tout, D, decltype(lc)::value, decltype(rc)::value>, dim3(bx, nu), 256, 0, st, os, slot, o, inv_count, lv, u0);
       });
     });
   });
@@ -1193,9 +1203,9 @@ cudaError_t gather_bwd_t(const Geom& g, const float* dqs, const float* dks, cons
       if constexpr (LL >= 2) {
         per_unit_chunks(g.U, [&](int64_t u0, unsigned nu) {
           if (g.p == 4)
-            k_gather_bwd_pp<Tout, D, LL, 4><<<dim3(bxp, nu, 3), 128, 0, st>>>(dqs, dks, dvs, slot, dq, dk, dv, lv, u0);
+            (void)launch_pdl(k_gather_bwd_pp<Tout, D, LL, 4>, dim3(bxp, nu, 3), 128, 0, st, dqs, dks, dvs, slot, dq, dk, dv, lv, u0);
           else
-            k_gather_bwd_pp<Tout, D, LL, 2><<<dim3(bxp, nu, 3), 128, 0, st>>>(dqs, dks, dvs, slot, dq, dk, dv, lv, u0);
+            (void)launch_pdl(k_gather_bwd_pp<Tout, D, LL, 2>, dim3(bxp, nu, 3), 128, 0, st, dqs, dks, dvs, slot, dq, dk, dv, lv, u0);
         });
       }
     });
@@ -1205,8 +1215,7 @@ cudaError_t gather_bwd_t(const Geom& g, const float* dqs, const float* dks, cons
   return with_tokens(R, [&](auto rc) {
     return with_levels(g.L, [&](auto lc) {
       per_unit_chunks(g.U, [&](int64_t u0, unsigned nu) {
-        k_gather_bwd<Tout, D, decltype(lc)::value, decltype(rc)::value>
-            <<<dim3(bx, nu), 256, 0, st>>>(dqs, dks, dvs, slot, dq, dk, dv, lv, u0);
+        (void)launch_pdl(k_gather_bwd<Tout, D, decltype(lc)::value, decltype(rc)::value>, dim3(bx, nu), 256, 0, st, dqs, dks, dvs, slot, dq, dk, dv, lv, u0);
       });
     });
   });
@@ -1233,7 +1242,7 @@ cudaError_t scatter_bwd_d(const Geom& g, const Tin* dO, const int32_t* slot, con
   if (g.scatter_mode == LH_SCATTER_LAST) {
     const unsigned bxl = blocks_for(g.N, 256 / (D / 8));
     per_unit_chunks(g.U, [&](int64_t u0, unsigned nu) {
-      k_scatter_bwd_last<Tin, D><<<dim3(bxl, nu), 256, 0, st>>>(dO, slot, ic, dos, lv, u0);
+      (void)launch_pdl(k_scatter_bwd_last<Tin, D>, dim3(bxl, nu), 256, 0, st, dO, slot, ic, dos, lv, u0);
     });
     return cudaGetLastError();
   }
@@ -1251,7 +1260,7 @@ cudaError_t scatter_bwd_d(const Geom& g, const Tin* dO, const int32_t* slot, con
           using C = ScatterBwdCfg<Tin, D, LL, PP, RR>;
           const unsigned bx = blocks_for(spans * (D / 8) * RR, kScatterBwdThreads);
           per_unit_chunks(g.U, [&](int64_t u0, unsigned nu) {
-            k_scatter_bwd_pp<Tin, D, LL, PP, RR><<<dim3(bx, nu), kScatterBwdThreads, C::smem_bytes, st>>>(
+            (void)launch_pdl(k_scatter_bwd_pp<Tin, D, LL, PP, RR>, dim3(bx, nu), kScatterBwdThreads, C::smem_bytes, st, 
                 dO, slot, ic, dos, lv, (int32_t)spans, u0);
           });
         };
@@ -1269,16 +1278,16 @@ cudaError_t scatter_bwd_d(const Geom& g, const Tin* dO, const int32_t* slot, con
       }
       if (RG == 4) {
         if constexpr ((D / 8) * 4 <= 32) {
-          k_scatter_bwd<Tin, D, LL, 4><<<nb, 256, 0, st>>>(dO, slot, ic, dos, lv, spans, groups);
+          (void)launch_pdl(k_scatter_bwd<Tin, D, LL, 4>, nb, 256, 0, st, dO, slot, ic, dos, lv, spans, groups);
           return;
         }
       }
       if (RG == 2) {
-        k_scatter_bwd<Tin, D, LL, 2><<<nb, 256, 0, st>>>(dO, slot, ic, dos, lv, spans, groups);
+        (void)launch_pdl(k_scatter_bwd<Tin, D, LL, 2>, nb, 256, 0, st, dO, slot, ic, dos, lv, spans, groups);
         return;
       }
     }
-    k_scatter_bwd<Tin, D, LL, 1><<<nb, 256, 0, st>>>(dO, slot, ic, dos, lv, spans, groups);
+    (void)launch_pdl(k_scatter_bwd<Tin, D, LL, 1>, nb, 256, 0, st, dO, slot, ic, dos, lv, spans, groups);
   });
 }
 }  // namespace
@@ -1318,9 +1327,9 @@ cudaError_t launch_attn_stats(const Geom& g, const __half* os, const __half* dos
   const int64_t prows = g.U * T * 128;
   const unsigned nb = blocks_for(prows * (g.d / 8), 256);
   if (g.d == 64)
-    k_attn_stats<64><<<nb, 256, 0, st>>>(os, dos, lse, stats, (int)g.S, T, prows);
+    (void)launch_pdl(k_attn_stats<64>, nb, 256, 0, st, os, dos, lse, stats, (int)g.S, T, prows);
   else
-    k_attn_stats<128><<<nb, 256, 0, st>>>(os, dos, lse, stats, (int)g.S, T, prows);
+    (void)launch_pdl(k_attn_stats<128>, nb, 256, 0, st, os, dos, lse, stats, (int)g.S, T, prows);
   return cudaGetLastError();
 }
 

@@ -147,6 +147,7 @@ __global__ void __launch_bounds__(256) k_pyr_chunk(
     const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin* __restrict__ v,
     float* __restrict__ pq, float* __restrict__ pk, float* __restrict__ pv,
     float* __restrict__ score, const PyrPrm prm, int64_t u0) {
+  pdl_enter();
   using Sm = ChunkSmem<Tin, D, kPyr>;
   constexpr int G = D / 8;
   constexpr int NT = Sm::NT;
@@ -296,6 +297,7 @@ __global__ void __launch_bounds__(256) k_pyr_upper(
     const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin* __restrict__ v,
     float* __restrict__ pq, float* __restrict__ pk, float* __restrict__ pv,
     float* __restrict__ score, const PyrPrm prm, int l, int64_t u0) {
+  pdl_enter();
   constexpr int G = D / 8;
   const int n = prm.N / prm.pw[l];  // entries of level l per unit
   const int it = (int)blockIdx.x * 256 + (int)threadIdx.x;
@@ -369,12 +371,12 @@ cudaError_t launch_flags(const Geom& g, const Tin* q, const Tin* k, const Tin* v
   const unsigned bx = (unsigned)((g.N + prm.CR - 1) / prm.CR);
   for (int64_t u0 = 0; u0 < g.U; u0 += 65535) {
     const unsigned nu = (unsigned)(g.U - u0 < 65535 ? g.U - u0 : 65535);
-    kc<<<dim3(bx, nu), 256, smem, st>>>(q, k, v, pq, pk, pv, score, prm, u0);
+    (void)launch_pdl(kc, dim3(bx, nu), 256, smem, st, q, k, v, pq, pk, pv, score, prm, u0);
     for (int l = prm.J + 1; l <= g.L - 1; ++l) {
       const int64_t n = g.N / g.pw[l];
       const int64_t items = kPyr ? 3 * n * (D / 8) : n;
       const unsigned ub = (unsigned)((items + 255) / 256);
-      k_pyr_upper<Tin, D, kPyr, kScore><<<dim3(ub, nu), 256, 0, st>>>(q, k, v, pq, pk, pv, score,
+      (void)launch_pdl(k_pyr_upper<Tin, D, kPyr, kScore>, dim3(ub, nu), 256, 0, st, q, k, v, pq, pk, pv, score,
                                                                       prm, l, u0);
     }
   }

@@ -8,6 +8,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <utility>
+
 #include "../../include/lighthouse.h"
 
 namespace lh {
@@ -98,6 +100,32 @@ __device__ __forceinline__ bool dbg_report(bool ok, uint32_t bits, uint32_t* wor
 #endif
 
 __device__ __forceinline__ int64_t imin64(int64_t a, int64_t b) { return a < b ? a : b; }
+
+// Programmatic dependent launch.  The stage kernels are launched with
+// launch_pdl, which lets the GPU start a grid while the one before it in the
+// stream drains; each such kernel first waits (pdl_enter) until the grid before
+// it has completed and its writes are visible -- the order of an ordinary launch
+// -- and then releases the grid after it.  For an ordinary launch both
+// instructions are no-ops.
+__device__ __forceinline__ void pdl_enter() {
+  asm volatile("griddepcontrol.wait;\n" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
+}
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                              cudaStream_t st, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
 
 // f(std::integral_constant<int, i>) for i = I .. N-1: a loop whose index is a
 // compile-time constant in the body (register arrays stay in registers, powers
