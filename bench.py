@@ -48,14 +48,14 @@ PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # kernel that evicts them, so a stage that writes more than L2 holds reads low.
 MEASURED_TRAFFIC = {  # workload: {stage: (bytes per launch, sources, sha1[:16])}
     "pretrain": {
-        "pyramid_score": (9.6640e+08, ('k_pyramid.cu', 'lh_internal.cuh'), "3a592d4c26ded79a"),
-        "topk": (4.7600e+07, ('k_topk.cu', 'lh_internal.cuh'), "d537cf8c45dc9c26"),
-        "gather": (9.8900e+07, ('k_gather_scatter.cu', 'lh_internal.cuh'), "561cc6c760bc762a"),
-        "scatter": (1.7000e+08, ('k_gather_scatter.cu', 'lh_internal.cuh'), "561cc6c760bc762a"),
-        "scatter_bwd": (2.2590e+08, ('k_gather_scatter.cu', 'lh_internal.cuh'), "561cc6c760bc762a"),
-        "gather_bwd": (6.5820e+08, ('k_gather_scatter.cu', 'lh_internal.cuh'), "561cc6c760bc762a"),
-        "attn_fwd": (5.0400e+07, ('k_attn_tc.cu', 'tc_common.cuh', 'lh_internal.cuh'), "fddb1b46e4c21830"),
-        "attn_bwd": (1.9430e+08, ('k_attn_tc.cu', 'tc_common.cuh', 'k_gather_scatter.cu', 'lh_internal.cuh'), "a482e947f0cf6f7c"),
+        "pyramid_score": (9.6650e+08, ('k_pyramid.cu', 'lh_internal.cuh'), "faf8e790685b35eb"),
+        "topk": (4.7600e+07, ('k_topk.cu', 'lh_internal.cuh'), "61533dd39326a401"),
+        "gather": (9.8800e+07, ('k_gather_scatter.cu', 'lh_internal.cuh'), "3db08f39fc50e30c"),
+        "scatter": (1.6990e+08, ('k_gather_scatter.cu', 'lh_internal.cuh'), "3db08f39fc50e30c"),
+        "scatter_bwd": (2.2560e+08, ('k_gather_scatter.cu', 'lh_internal.cuh'), "3db08f39fc50e30c"),
+        "gather_bwd": (6.5840e+08, ('k_gather_scatter.cu', 'lh_internal.cuh'), "3db08f39fc50e30c"),
+        "attn_fwd": (5.0400e+07, ('k_attn_tc.cu', 'tc_common.cuh', 'lh_internal.cuh'), "c4abb2f38acc8eb9"),
+        "attn_bwd": (1.9460e+08, ('k_attn_tc.cu', 'tc_common.cuh', 'k_gather_scatter.cu', 'lh_internal.cuh'), "66ab60581431953c"),
     },
 }
 
