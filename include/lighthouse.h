@@ -46,7 +46,10 @@
  *   - The caller allocates and frees every buffer; the library allocates no
  *     device memory and never synchronises the stream (except
  *     lh_read_device_status).  All work is enqueued on `stream` (NULL = the
- *     legacy default stream).
+ *     legacy default stream), in stream order: the stage kernels are
+ *     programmatic dependent launches, each waiting at its start until the
+ *     work before it on the stream has completed, so the GPU can stage a
+ *     kernel while the previous one drains.
  *   - Arguments are checked on the host before any launch; a call that
  *     returns an error has enqueued nothing.  A launch failure returns
  *     LH_ERR_CUDA.  No call traps, asserts or exits.
